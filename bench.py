@@ -1,0 +1,425 @@
+"""Benchmark: radial block-sparse attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wan] [--impl ours|reference]
+
+One step = the whole hot path on one synthetic problem already resident in
+HBM: radial block-list build (count, scan, fill; asynchronous, into
+preallocated buffers), the longest-row-first work order, and the tcgen05
+attention kernel. Each GPU (one process per GPU under torchrun) runs its own
+independent problem, so per-GPU work is fixed as N grows (weak scaling) and
+no collective touches the data path; the only collectives are the timing
+barrier and the max over ranks.
+
+Prints one JSON line on rank 0. ``value`` is effective TFLOP/s on computed
+blocks over all ranks: 4 * D * sum over listed (query block, key block) of
+valid rows x valid cols, per head, divided by the slowest rank's time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "block-sparse attn fwd ms & effective TFLOP/s vs bf16 peak at 32k–120k tokens"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ("block_sparse_attention_radial_b200/csrc/attn_fwd_sm100.cuh",
+                  "block_sparse_attention_radial_b200/csrc/ptx_sm100.cuh")
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def load_traffic(workload: str):
+    """DRAM bytes per launch of the attention kernel from a committed ncu summary,
+    or None when the summary is missing or was taken on different kernel source."""
+    path = os.path.join(ROOT, "profiles", f"attn_fwd_sm100_{workload}_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks ---
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_uuid: str | None):
+        self.proc = None
+        self.path = os.path.join("/tmp", f"bsa_clocks_{os.getpid()}.csv")
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "200"]
+        if device_uuid:
+            cmd += ["-i", device_uuid]
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    rows.append((float(parts[0]), float(parts[1]), parts[3:]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        max_mhz = max(r[1] for r in rows)
+        loaded = [r for r in rows if r[0] > 0.5 * max_mhz] or rows
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[2][1:5])
+                          if v.strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max_mhz,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------- helpers ---
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    import datetime
+
+    import torch.distributed as dist
+
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+
+def max_over_ranks(value: float, device) -> float:
+    """Max of a per-rank float over all ranks (identity at world size 1)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+# ------------------------------------------------------------ CPU oracle ---
+
+def oracle_sample_rate(w, lists_host, q, k, v, budget_s: float, head: int = 0):
+    """Time the CPU oracle on query rows of one head; returns (TFLOP/s, seconds,
+    rows, flops). Rows are a contiguous run from the middle of the sequence,
+    sized by a short calibration run to take about ``budget_s``."""
+    import numpy as np
+
+    import oracle
+
+    rp, ci = lists_host
+    D = w.head_dim
+    qh, kh, vh = (t[:, head:head + 1].cpu() for t in (q, k, v))
+    valid = np.minimum(w.block, w.n - np.arange(w.nqb) * w.block)
+
+    def flops_of(rows):
+        f = 0
+        for r in rows:
+            qb = r // w.block
+            f += 4 * D * int(valid[ci[rp[qb]:rp[qb + 1]]].sum())
+        return f
+
+    start = (w.n // 2) // w.block * w.block
+    cal = np.arange(start, min(w.n, start + 64))
+    for _ in range(2):  # the first call pays one-time costs
+        t0 = time.perf_counter()
+        oracle.masked_attention_fp64(qh, kh, vh, rp, ci, 1, w.block, rows=cal)
+        t_cal = max(time.perf_counter() - t0, 1e-3)
+    nrows = int(min(w.n - start, max(64, cal.size * budget_s / t_cal)))
+    rows = np.arange(start, start + nrows)
+    t0 = time.perf_counter()
+    oracle.masked_attention_fp64(qh, kh, vh, rp, ci, 1, w.block, rows=rows)
+    dt = time.perf_counter() - t0
+    fl = flops_of(rows)
+    return fl / dt / 1e12, dt, rows, fl
+
+
+# ------------------------------------------------------------------ main ---
+
+def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle, as it stands, on the host cores."""
+    if rank != 0:
+        return 0
+    import numpy as np
+    import torch
+
+    import oracle
+    from workloads import WORKLOADS, make_qkv
+
+    w = WORKLOADS[args.workload]
+    q, k, v = make_qkv(w, "cpu", heads=1)
+    rp, ci = oracle.radial_block_lists(w.frames, w.tokens_per_frame, w.block)
+    per_step = max(0.2, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
+    rate, dt, rows, fl = oracle_sample_rate(w, (rp, ci), q, k, v, per_step)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        oracle.masked_attention_fp64(q, k, v, rp, ci, 1, w.block, rows=rows)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = fl * len(times) / total / 1e12
+    cores = blas_threads()
+    sample = (f"head 0, query rows {int(rows[0])}..{int(rows[-1])} ({rows.size} rows) of the "
+              f"{w.name} problem per step; fp64 NumPy oracle")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total / len(times) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, nnz=int(rp[-1])),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, nnz):
+    return {"workload": f"{w.name}: B={w.batch} H={w.heads} D={w.head_dim} "
+                        f"{w.frames}x{w.tokens_per_frame} tokens (n={w.n}), radial {w.block}x{w.block} blocks",
+            "global_batch": w.batch, "heads": w.heads, "head_dim": w.head_dim, "seq_len": w.n,
+            "frames": w.frames, "tokens_per_frame": w.tokens_per_frame, "block": w.block,
+            "nnz_blocks_per_head": nnz, "parallelism": "independent problem per GPU",
+            "l2": "inputs larger than L2 (Q, K, V per problem exceed 126 MB); no flush"}
+
+
+def run_ours(args, world, rank, local):
+    import numpy as np
+    import torch
+
+    import block_sparse_attention_radial_b200 as bsa
+    from workloads import WORKLOADS, make_qkv
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    w = WORKLOADS[args.workload]
+    assert w.radial, "the bench times the radial path"
+
+    q, k, v = make_qkv(w, dev)
+    lists = bsa.radial_block_lists(w.frames, w.tokens_per_frame, w.block, device=dev)
+    rp_h, ci_h = lists.row_ptr.cpu().numpy(), lists.col_idx.cpu().numpy()
+    flops = bsa.computed_flops(rp_h, ci_h, w.n, w.block, w.head_dim, w.batch, w.heads, 1)
+    dense_flops = 4 * w.head_dim * w.batch * w.heads * w.n * w.n
+    out = torch.empty_like(q)
+    lse = torch.empty((w.batch, w.heads, w.n), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(bsa.bsa_attn_fwd_workspace_bytes(w.batch, w.heads, lists), 16),
+                     dtype=torch.uint8, device=dev)
+    row_ptr, col_idx = lists.row_ptr, lists.col_idx
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 5  # mask count, scan, fill; work order; attention
+
+    def step(ev=None):
+        bsa.bsa_radial_mask_build(w.frames, w.tokens_per_frame, w.block, row_ptr, col_idx,
+                                  col_idx.numel(), want_nnz=False, stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        bsa.bsa_attn_fwd(q, k, v, lists, out, lse, ws, 0.0, stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    status = bsa.bsa_get_device_status()
+    if status != 0:
+        raise SystemExit(f"device status {status} after warm-up")
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid).replace("GPU-", "")
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid) if rank == 0 else None
+    if sampler is not None:
+        time.sleep(0.4)   # let the sampler start before the timed region
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(kev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    clocks = sampler.stop() if sampler is not None else None
+    ms_local = t_start.elapsed_time(t_end)
+    ms = max_over_ranks(ms_local, dev)
+    kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    status = bsa.bsa_get_device_status()
+    if status != 0:
+        raise SystemExit(f"device status {status} after the timed region")
+
+    # ---- end to end through the public API: pinned host inputs -> result on host
+    e2e_steps = max(3, min(args.steps, 10))
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        bsa.bsa_radial_mask_build(w.frames, w.tokens_per_frame, w.block, row_ptr, col_idx,
+                                  col_idx.numel(), want_nnz=False, stream=stream)
+        bsa.bsa_attn_fwd(qd, kd, vd, lists, out, lse, ws, 0.0, stream)
+        oh.copy_(out, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, dt, rows, fl = oracle_sample_rate(w, (rp_h, ci_h), q, k, v, args.cpu_seconds)
+        cpu_baseline = {"value": rate, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                        "sample": f"head 0, {rows.size} query rows ({int(rows[0])}..{int(rows[-1])}) "
+                                  f"of the {w.name} problem, {dt:.1f} s, fp64 NumPy"}
+
+    if rank == 0:
+        peaks, peak_kind = load_peaks()
+        peak = float(peaks["bf16_tflops"])
+        achieved = flops / (kernel_ms * 1e-3) / 1e12
+        traffic = load_traffic(w.name)
+        line = {
+            "metric": METRIC,
+            "value": flops * world * args.steps / (ms * 1e-3) / 1e12,
+            "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(w, nnz=int(rp_h[-1])),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_kind": f"{peak_kind} bf16 burst",
+                         "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
+                         "kernel": "attn_fwd_sm100_kernel<128,128> (+ work-order prepass)",
+                         "kernel_ms": kernel_ms, "flops_per_launch": flops},
+            "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": launches_per_step * args.steps,
+            "dense_equivalent_tflops": dense_flops * world * args.steps / (ms * 1e-3) / 1e12,
+            "clocks": clocks,
+            "cpu_baseline": cpu_baseline,
+        }
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="wan", choices=("wan", "hunyuan", "long4x", "tiny"))
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    return run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,223 @@
+"""Radial block-sparse softmax attention (forward) for NVIDIA B200 / sm_100a.
+
+A thin Python binding over libbsa's C ABI (include/bsa.h). The functions named
+``bsa_*`` mirror the C entry points one to one and only marshal arguments;
+PyTorch supplies device memory and the current CUDA stream. Every step of the
+computation runs in the library's CUDA kernels.
+
+Typical use::
+
+    import block_sparse_attention_radial_b200 as bsa
+    lists = bsa.radial_block_lists(frames=21, tokens_per_frame=1560, block=128)
+    out, lse = bsa.attention(q, k, v, lists)      # q, k, v: bf16 [B, H, n, D] on cuda
+"""
+
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import BlockListsC, STATUS_NAMES
+
+__all__ = [
+    "BsaError", "BlockLists", "bsa_radial_mask_build", "bsa_attn_fwd_workspace_bytes",
+    "bsa_attn_fwd", "bsa_attn_dense_masked_ref", "bsa_validate_lists", "bsa_get_device_status",
+    "bsa_get_timeout_detail", "bsa_status_string", "bsa_last_cuda_error", "bsa_set_test_hooks",
+    "radial_block_lists", "block_lists_from_csr", "attention", "dense_masked_reference",
+    "computed_flops",
+]
+
+
+class BsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        lib = _lib.load()
+        msg = lib.bsa_status_string(status).decode()
+        extra = lib.bsa_last_cuda_error().decode() if status == 3 else ""
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({msg}) {extra}".strip())
+        self.status = status
+
+
+def _check(status: int, where: str) -> int:
+    if status != 0:
+        raise BsaError(status, where)
+    return status
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+@dataclass
+class BlockLists:
+    """CSR key-block lists on the device (see ``bsa_block_lists`` in include/bsa.h)."""
+
+    row_ptr: torch.Tensor       # int32 [num_lists * num_q_blocks + 1]
+    col_idx: torch.Tensor       # int32 [nnz]
+    num_lists: int
+    num_q_blocks: int
+    block: int
+
+    @property
+    def num_k_blocks(self) -> int:
+        return self.num_q_blocks
+
+    @property
+    def nnz(self) -> int:
+        return int(self.col_idx.numel())
+
+    def c_struct(self) -> BlockListsC:
+        return BlockListsC(self.num_lists, self.num_q_blocks, self.num_k_blocks, self.block,
+                           self.nnz, self.row_ptr.data_ptr(),
+                           self.col_idx.data_ptr() if self.nnz else 0)
+
+
+# ------------------------------------------------------------- C entry points
+
+def bsa_radial_mask_build(frames: int, tokens_per_frame: int, block: int, row_ptr: torch.Tensor,
+                          col_idx: torch.Tensor | None = None, col_capacity: int = 0,
+                          want_nnz: bool = True, stream=None) -> int | None:
+    """Radial block lists into caller-owned int32 device tensors; returns nnz when asked
+    (that synchronises the stream)."""
+    lib = _lib.load()
+    nnz = ctypes.c_int64(-1)
+    st = lib.bsa_radial_mask_build(frames, tokens_per_frame, block, _ptr(row_ptr), _ptr(col_idx),
+                                   col_capacity if col_idx is not None else 0,
+                                   ctypes.byref(nnz) if want_nnz else None, _stream(stream))
+    _check(st, "bsa_radial_mask_build")
+    return int(nnz.value) if want_nnz else None
+
+
+def bsa_attn_fwd_workspace_bytes(batch: int, heads: int, lists: BlockLists) -> int:
+    return int(_lib.load().bsa_attn_fwd_workspace_bytes(batch, heads, ctypes.byref(lists.c_struct())))
+
+
+def bsa_attn_fwd(q, k, v, lists: BlockLists, out, lse=None, workspace=None,
+                 softmax_scale: float = 0.0, stream=None) -> None:
+    """Block-sparse attention forward on the tensor cores (asynchronous)."""
+    B, H, n, D = q.shape
+    lib = _lib.load()
+    ls = lists.c_struct()
+    if workspace is None:
+        workspace = torch.empty(max(lib.bsa_attn_fwd_workspace_bytes(B, H, ctypes.byref(ls)), 16),
+                                dtype=torch.uint8, device=q.device)
+    st = lib.bsa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), B, H, n, D, float(softmax_scale),
+                          ctypes.byref(ls), _ptr(out), _ptr(lse), _ptr(workspace),
+                          workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "bsa_attn_fwd")
+
+
+def bsa_attn_dense_masked_ref(q, k, v, lists: BlockLists, out, lse=None,
+                              softmax_scale: float = 0.0, stream=None) -> None:
+    """Same result from the plain fp32 CUDA-core reference kernel (asynchronous)."""
+    B, H, n, D = q.shape
+    st = _lib.load().bsa_attn_dense_masked_ref(_ptr(q), _ptr(k), _ptr(v), B, H, n, D,
+                                               float(softmax_scale), ctypes.byref(lists.c_struct()),
+                                               _ptr(out), _ptr(lse), _stream(stream))
+    _check(st, "bsa_attn_dense_masked_ref")
+
+
+def bsa_validate_lists(lists: BlockLists, stream=None) -> int:
+    """Returns the status (0 = well formed, 5 = BSA_ERR_BAD_LISTS); raises on other errors."""
+    st = _lib.load().bsa_validate_lists(ctypes.byref(lists.c_struct()), _stream(stream))
+    if st not in (0, 5):
+        _check(st, "bsa_validate_lists")
+    return st
+
+
+def bsa_get_device_status(stream=None) -> int:
+    st = _lib.load().bsa_get_device_status(_stream(stream))
+    if st == 3:
+        _check(st, "bsa_get_device_status")
+    return st
+
+
+def bsa_get_timeout_detail() -> list[int]:
+    out = (ctypes.c_int32 * 4)()
+    _check(_lib.load().bsa_get_timeout_detail(out), "bsa_get_timeout_detail")
+    return list(out)
+
+
+def bsa_status_string(status: int) -> str:
+    return _lib.load().bsa_status_string(status).decode()
+
+
+def bsa_last_cuda_error() -> str:
+    return _lib.load().bsa_last_cuda_error().decode()
+
+
+def bsa_set_test_hooks(wait_limit_ns: int = 0, fault_flags: int = 0) -> None:
+    _check(_lib.load().bsa_set_test_hooks(wait_limit_ns, fault_flags), "bsa_set_test_hooks")
+
+
+# ------------------------------------------------------------- conveniences
+
+def radial_block_lists(frames: int, tokens_per_frame: int, block: int = 128,
+                       device=None, stream=None) -> BlockLists:
+    """Build the radial lists on the GPU (two calls: count, then fill)."""
+    device = torch.device("cuda") if device is None else torch.device(device)
+    n = frames * tokens_per_frame
+    nqb = -(-n // block)
+    row_ptr = torch.empty(nqb + 1, dtype=torch.int32, device=device)
+    nnz = bsa_radial_mask_build(frames, tokens_per_frame, block, row_ptr, stream=stream)
+    col_idx = torch.empty(max(nnz, 1), dtype=torch.int32, device=device)
+    got = bsa_radial_mask_build(frames, tokens_per_frame, block, row_ptr, col_idx, col_idx.numel(),
+                                stream=stream)
+    assert got == nnz
+    return BlockLists(row_ptr, col_idx[:nnz], 1, nqb, block)
+
+
+def block_lists_from_csr(row_ptr, col_idx, num_lists: int, num_q_blocks: int, block: int,
+                         device=None) -> BlockLists:
+    """Wrap host or device CSR arrays (copied to ``device`` as int32)."""
+    device = torch.device("cuda") if device is None else torch.device(device)
+    rp = torch.as_tensor(row_ptr, dtype=torch.int32).to(device).contiguous()
+    ci = torch.as_tensor(col_idx, dtype=torch.int32).to(device).contiguous()
+    return BlockLists(rp, ci, num_lists, num_q_blocks, block)
+
+
+def attention(q, k, v, lists: BlockLists, softmax_scale: float = 0.0, want_lse: bool = True,
+              workspace=None, stream=None):
+    """Allocate outputs and run :func:`bsa_attn_fwd`; returns ``(out, lse)``."""
+    B, H, n, _ = q.shape
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device) if want_lse else None
+    bsa_attn_fwd(q, k, v, lists, out, lse, workspace, softmax_scale, stream)
+    return out, lse
+
+
+def dense_masked_reference(q, k, v, lists: BlockLists, softmax_scale: float = 0.0, stream=None):
+    B, H, n, _ = q.shape
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device)
+    bsa_attn_dense_masked_ref(q, k, v, lists, out, lse, softmax_scale, stream)
+    return out, lse
+
+
+def computed_flops(row_ptr, col_idx, n: int, block: int, head_dim: int, batch: int,
+                   heads: int, num_lists: int) -> int:
+    """FLOPs on computed blocks: 4 * D * sum over listed (qb, kb) of valid rows x valid cols,
+    over every batch item and head (host arrays)."""
+    import numpy as np
+
+    rp = np.asarray(row_ptr, dtype=np.int64)
+    ci = np.asarray(col_idx, dtype=np.int64)
+    nqb = -(-n // block)
+    valid = np.minimum(block, n - np.arange(nqb) * block)
+    total = 0
+    for lst in range(num_lists):
+        rows = np.arange(nqb) + lst * nqb
+        counts = np.diff(rp[lst * nqb: lst * nqb + nqb + 1])
+        qv = np.repeat(valid, counts)
+        kv = valid[ci[rp[rows[0]]:rp[rows[-1] + 1]]]
+        total += int((qv * kv).sum())
+    mult = heads if num_lists == 1 else 1
+    return 4 * head_dim * batch * mult * total

@@ -1,0 +1,481 @@
+// Block-sparse softmax attention forward for sm_100a: TMA-staged tiles,
+// tcgen05 MMAs accumulating in tensor memory, exp2 online softmax.
+//
+// One CTA per SM (persistent). Work items are (batch*head, query block); the
+// host-side prepass orders each list's query blocks longest row first and the
+// CTAs walk that order head-major in a static snake, so concurrently running
+// CTAs share the K/V of one or two heads in L2 and the cheapest rows finish
+// the job.
+//
+// Warp roles (192 threads):
+//   warps 0-3  softmax: thread t owns query row t of the 128-row tile
+//              (TMEM lane t); exp2 online softmax, P written back to TMEM as
+//              bf16, O rescaled in TMEM when the running max jumps, epilogue.
+//   warp 4     producer (one thread): TMA loads of Q and of the listed K and
+//              V tiles through an NS-stage ring, in the order the MMA warp
+//              consumes them.
+//   warp 5     MMA issuer (one thread): S = Q K^T into one of two TMEM S
+//              buffers, then O += P V with P read from TMEM.
+//
+// TMEM columns (512 allocated): S0 [0,128), S1 [128,256), O [256, 256+D).
+// Per block g (global counter) the MMA warp issues QK(g+1) before PV(g), so
+// the tensor core computes the next scores while the softmax warps work.
+//
+// Every wait is bounded (globaltimer). On expiry the thread records
+// BSA_ERR_DEVICE_TIMEOUT, raises a CTA-wide abort flag, and all roles leave
+// their loops; the producer waits (bounded) for its copies in flight, the MMA
+// thread waits for its MMAs, and TMEM is freed before the CTA exits.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "device_status.cuh"
+#include "ptx_sm100.cuh"
+
+namespace bsa {
+
+struct FwdParams {
+  const int32_t *row_ptr, *col_idx, *order;
+  __nv_bfloat16 *out;
+  float *lse;
+  int32_t heads, n, nqb, nkb, num_lists, nnz;
+  int32_t total_items;
+  float scale_log2;  // softmax_scale * log2(e)
+  unsigned long long wait_limit_ns;
+  int32_t fault_flags;
+};
+
+constexpr int kSmemLimit = 232448;  // 227 KB dynamic + static per CTA on sm_100
+
+template <int D, int BN>
+struct FwdCfg {
+  static constexpr int BM = 128;                 // tile rows (MMA M)
+  static constexpr int NCB = D / 64;             // 128-byte column blocks per row
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BN * D * 2;    // one K or V tile
+  static constexpr int NS_FIT = (kSmemLimit - 1024 - 512 - Q_BYTES) / KV_BYTES;
+  static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
+  // At least 120 KB so that a second CTA never fits on an SM: every CTA then
+  // owns its SM's tensor memory and the persistent grid covers all SMs.
+  static constexpr int DSMEM_USED = 1024 + Q_BYTES + NS * KV_BYTES;
+  static constexpr int DSMEM = DSMEM_USED > 122880 ? DSMEM_USED : 122880;
+  static constexpr uint32_t S_COL = 0;           // S buffer b at S_COL + 128 b
+  static constexpr uint32_t O_COL = 256;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int THREADS = 192;
+  static_assert(NS >= 2, "K/V ring needs at least two stages");
+  static_assert(D == 64 || D == 128, "head_dim");
+  static_assert(BN == 64 || BN == 128, "block");
+};
+
+enum : int { kRoleProducer = 1, kRoleMma = 2, kRoleSoftmax = 3 };
+enum : int {
+  kBarKvFull = 1, kBarKvEmpty, kBarQFull, kBarQEmpty, kBarSFull, kBarPFull, kBarODone,
+  kBarOEmpty, kBarFinal
+};
+
+struct WaitCtx {
+  volatile int *abort;
+  unsigned long long limit;
+  int role;
+};
+
+// Bounded parity wait. Returns false when the CTA is aborting or the limit ran
+// out (the first thread to run out records the timeout and raises the flag).
+__device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, const WaitCtx &w,
+                                          int bar_id, uint32_t counter) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*w.abort) return false;
+    if (global_timer_ns() - t0 > w.limit) {
+      if (atomicCAS(&g_status, 0u, 4u /* BSA_ERR_DEVICE_TIMEOUT */) == 0u) {
+        g_status_detail[0] = w.role;
+        g_status_detail[1] = bar_id;
+        g_status_detail[2] = counter;
+        g_status_detail[3] = blockIdx.x;
+      }
+      *w.abort = 1;
+      return false;
+    }
+  }
+}
+
+// Work item k of this CTA (static snake over the ordered item list); -1 when
+// the CTA has no item k.
+__device__ __forceinline__ int snake_item(int k, int total) {
+  const int G = gridDim.x;
+  const long long base = static_cast<long long>(k) * G;
+  if (base >= total) return -2;  // past the end for every CTA
+  const int idx = static_cast<int>(base) + ((k & 1) ? (G - 1 - static_cast<int>(blockIdx.x))
+                                                    : static_cast<int>(blockIdx.x));
+  return idx < total ? idx : -1;
+}
+
+struct Item {
+  int bh, qb, a, len;
+};
+
+__device__ __forceinline__ Item decode_item(int idx, const FwdParams &p) {
+  Item it;
+  it.bh = idx / p.nqb;
+  const int rank = idx - it.bh * p.nqb;
+  const int list = p.num_lists > 1 ? (it.bh % p.heads) : 0;
+  const long long lbase = static_cast<long long>(list) * p.nqb;
+  it.qb = min(max(p.order[lbase + rank], 0), p.nqb - 1);
+  const int a = min(max(p.row_ptr[lbase + it.qb], 0), p.nnz);
+  const int e = min(max(p.row_ptr[lbase + it.qb + 1], 0), p.nnz);
+  it.a = a;
+  it.len = max(e - a, 0);
+  return it;
+}
+
+__device__ __forceinline__ int key_block(const FwdParams &p, int e) {
+  return min(max(p.col_idx[e], 0), p.nkb - 1);
+}
+
+template <int D, int BN>
+__global__ void __launch_bounds__(192, 1)
+    attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using C = FwdCfg<D, BN>;
+  extern __shared__ uint8_t dsmem[];
+  __shared__ __align__(8) uint64_t bar_kv_full[C::NS];
+  __shared__ __align__(8) uint64_t bar_kv_empty[C::NS];
+  __shared__ __align__(8) uint64_t bar_q_full, bar_q_empty, bar_o_done, bar_o_empty, bar_final;
+  __shared__ __align__(8) uint64_t bar_s_full[2], bar_p_full[2];
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const uint32_t raw = smem_addr(dsmem);
+  uint8_t *base = dsmem + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t *sQ = base;
+  uint8_t *sKV = base + C::Q_BYTES;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(&bar_kv_full[s], 1);
+      mbar_init(&bar_kv_empty[s], 1);
+    }
+    mbar_init(&bar_q_full, 1);
+    mbar_init(&bar_q_empty, 1);
+    mbar_init(&bar_o_done, 1);
+    mbar_init(&bar_o_empty, 128);
+    mbar_init(&bar_final, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar_s_full[b], 1);
+      mbar_init(&bar_p_full[b], 128);
+    }
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  WaitCtx wc{&abort_flag, p.wait_limit_ns, 0};
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      wc.role = kRoleProducer;
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      uint32_t ring = 0, qcount = 0;
+      bool skip_next_k = (p.fault_flags & 1) && blockIdx.x == 0;
+      int skipped_ring = -1;
+      bool ok = true;
+      auto load_kv = [&](const CUtensorMap *map, int kb, int z, bool is_k) -> bool {
+        const uint32_t s = ring % C::NS;
+        if (!wait_bounded(&bar_kv_empty[s], ((ring / C::NS) & 1u) ^ 1u, wc, kBarKvEmpty, ring))
+          return false;
+        if (is_k && skip_next_k) {  // test hook: leave this stage's barrier without an arrival
+          skip_next_k = false;
+          skipped_ring = static_cast<int>(ring);
+          ++ring;
+          return true;
+        }
+        mbar_arrive_expect_tx(&bar_kv_full[s], C::KV_BYTES);
+        uint8_t *dst = sKV + s * C::KV_BYTES;
+#pragma unroll
+        for (int cb = 0; cb < C::NCB; ++cb)
+          tma_load_3d(dst + cb * BN * 128, map, &bar_kv_full[s], cb * 64, kb * BN, z);
+        ++ring;
+        return true;
+      };
+      for (int k = 0; ok; ++k) {
+        const int idx = snake_item(k, p.total_items);
+        if (idx == -2) break;
+        if (idx < 0) continue;
+        const Item it = decode_item(idx, p);
+        if (it.len == 0) continue;
+        if (!wait_bounded(&bar_q_empty, (qcount & 1u) ^ 1u, wc, kBarQEmpty, qcount)) break;
+        mbar_arrive_expect_tx(&bar_q_full, C::Q_BYTES);
+#pragma unroll
+        for (int cb = 0; cb < C::NCB; ++cb)
+          tma_load_3d(sQ + cb * C::BM * 128, &tm_q, &bar_q_full, cb * 64, it.qb * BN, it.bh);
+        ++qcount;
+        ok = load_kv(&tm_k, key_block(p, it.a), it.bh, true);
+        for (int j = 0; ok && j < it.len; ++j) {
+          if (j + 1 < it.len) ok = load_kv(&tm_k, key_block(p, it.a + j + 1), it.bh, true);
+          if (ok) ok = load_kv(&tm_v, key_block(p, it.a + j), it.bh, false);
+        }
+      }
+      // Copies still in flight must land before the CTA exits: wait for the
+      // latest use of every stage and for the last Q tile (bounded, even when
+      // aborting).
+      WaitCtx drain{&abort_flag, p.wait_limit_ns, kRoleProducer};
+      int zero = 0;
+      drain.abort = &zero;
+      const uint32_t first = ring > C::NS ? ring - C::NS : 0;
+      for (uint32_t r = first; r < ring; ++r) {
+        if (static_cast<int>(r) == skipped_ring) continue;
+        wait_bounded(&bar_kv_full[r % C::NS], (r / C::NS) & 1u, drain, kBarKvFull, r);
+      }
+      if (qcount > 0) wait_bounded(&bar_q_full, (qcount - 1) & 1u, drain, kBarQFull, qcount);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      wc.role = kRoleMma;
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+      const uint32_t q_addr = smem_addr(sQ);
+      const uint32_t kv_addr = smem_addr(sKV);
+      uint32_t ring = 0, qcount = 0, g = 0, items_done = 0;
+      bool ok = true;
+      auto issue_qk = [&](uint32_t gg) -> bool {
+        const uint32_t s = ring % C::NS;
+        if (!wait_bounded(&bar_kv_full[s], (ring / C::NS) & 1u, wc, kBarKvFull, ring)) return false;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + C::S_COL + (gg & 1u) * 128u;
+        const uint32_t k_base = kv_addr + s * C::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t cb = kk >> 2, within = (kk & 3) * 32;
+          const uint64_t a = smem_desc_sw128(q_addr + cb * (C::BM * 128) + within, 16, 1024);
+          const uint64_t b = smem_desc_sw128(k_base + cb * (BN * 128) + within, 16, 1024);
+          mma_ss(d_tmem, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bar_kv_empty[s]);
+        mma_commit(&bar_s_full[gg & 1u]);
+        ++ring;
+        return true;
+      };
+      for (int k = 0; ok; ++k) {
+        const int idx = snake_item(k, p.total_items);
+        if (idx == -2) break;
+        if (idx < 0) continue;
+        const Item it = decode_item(idx, p);
+        if (it.len == 0) continue;
+        if (!wait_bounded(&bar_q_full, qcount & 1u, wc, kBarQFull, qcount)) break;
+        tc_fence_after();
+        if (!(ok = issue_qk(g))) break;
+        if (it.len == 1) mma_commit(&bar_q_empty);
+        for (int j = 0; j < it.len; ++j) {
+          const uint32_t gg = g + j;
+          if (j + 1 < it.len) {
+            if (!(ok = issue_qk(gg + 1))) break;
+            if (j + 1 == it.len - 1) mma_commit(&bar_q_empty);
+          }
+          if (!(ok = wait_bounded(&bar_p_full[gg & 1u], (gg >> 1) & 1u, wc, kBarPFull, gg))) break;
+          tc_fence_after();
+          if (j == 0 && items_done > 0) {
+            if (!(ok = wait_bounded(&bar_o_empty, (items_done - 1) & 1u, wc, kBarOEmpty,
+                                    items_done)))
+              break;
+            tc_fence_after();
+          }
+          const uint32_t s = ring % C::NS;
+          if (!(ok = wait_bounded(&bar_kv_full[s], (ring / C::NS) & 1u, wc, kBarKvFull, ring)))
+            break;
+          tc_fence_after();
+          const uint32_t p_tmem = tmem + C::S_COL + (gg & 1u) * 128u;
+          const uint32_t v_base = kv_addr + s * C::KV_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            // V tile: key rows of 128 bytes (64 head-dim values), 64-wide
+            // head-dim chunks BN*128 bytes apart (MN-major operand).
+            const uint64_t b = smem_desc_sw128(v_base + kk * (16 * 128), BN * 128, 1024);
+            mma_ts(tmem + C::O_COL, p_tmem + kk * 8, b, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&bar_kv_empty[s]);
+          mma_commit(&bar_o_done);
+          ++ring;
+        }
+        g += it.len;
+        ++qcount;
+        ++items_done;
+      }
+      // Let every issued MMA finish before TMEM is released.
+      mma_commit(&bar_final);
+      WaitCtx drain{&abort_flag, p.wait_limit_ns, kRoleMma};
+      int zero = 0;
+      drain.abort = &zero;
+      wait_bounded(&bar_final, 0, drain, kBarFinal, g);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    wc.role = kRoleSoftmax;
+    const int row_in_tile = warp * 32 + lane;
+    const uint32_t lane_tmem = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const float sl2 = p.scale_log2;
+    uint32_t g = 0;
+    bool ok = true;
+    auto warp_wait = [&](uint64_t *bar, uint32_t parity, int bar_id, uint32_t counter) -> bool {
+      const bool r = wait_bounded(bar, parity, wc, bar_id, counter);
+      return __all_sync(0xffffffffu, r);
+    };
+    for (int k = 0; ok; ++k) {
+      const int idx = snake_item(k, p.total_items);
+      if (idx == -2) break;
+      if (idx < 0) continue;
+      const Item it = decode_item(idx, p);
+      const int row = it.qb * BN + row_in_tile;
+      const bool store = row_in_tile < BN && row < p.n;
+      const long long orow = static_cast<long long>(it.bh) * p.n + row;
+      if (it.len == 0) {
+        if (store) {
+          uint4 *dst = reinterpret_cast<uint4 *>(p.out + orow * D);
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+          if (p.lse) p.lse[orow] = -INFINITY;
+        }
+        continue;
+      }
+      float m_ref = 0.f, l = 0.f;
+      for (int j = 0; j < it.len; ++j) {
+        const uint32_t gg = g + j;
+        const uint32_t s_tmem = lane_tmem + C::S_COL + (gg & 1u) * 128u;
+        if (!(ok = warp_wait(&bar_s_full[gg & 1u], (gg >> 1) & 1u, kBarSFull, gg))) break;
+        tc_fence_after();
+        float s[BN];
+        {
+          uint32_t sr[BN / 32][32];
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c) tmem_ld32(s_tmem + c * 32, sr[c]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c) {
+            reg_fence32(sr[c]);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(sr[c][i]);
+          }
+        }
+        const int kb = key_block(p, it.a + j);
+        const int valid = p.n - kb * BN;
+        if (valid < BN) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (c >= valid) s[c] = -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+        const float mblk = mx * sl2;
+        float alpha = 1.f;
+        bool rescale = false;
+        if (j == 0) {
+          m_ref = mblk;
+        } else if (mblk > m_ref + 8.f) {
+          // lazy rescale: the reference max only moves when the block max
+          // exceeds it by more than 2^8; the final O / l is exact either way
+          alpha = ex2_approx(m_ref - mblk);
+          m_ref = mblk;
+          rescale = true;
+        }
+        const float neg = -m_ref;
+        float sum = 0.f;
+        uint32_t pk[BN / 2];
+#pragma unroll
+        for (int c = 0; c < BN / 2; ++c) {
+          const float p0 = ex2_approx(fmaf(s[2 * c], sl2, neg));
+          const float p1 = ex2_approx(fmaf(s[2 * c + 1], sl2, neg));
+          sum += p0 + p1;
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+        l = l * alpha + sum;
+        // P (bf16 pairs) overwrites the first BN/2 columns of this S buffer
+#pragma unroll
+        for (int c = 0; c < BN / 64; ++c) {
+          uint32_t r[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = pk[c * 32 + i];
+          tmem_st32(s_tmem + c * 32, r);
+        }
+        // PV(gg-1) must be complete before O is touched and before P(gg) is
+        // released; this also keeps the o_done phase tracking in lockstep.
+        if (gg >= 1 && !(ok = warp_wait(&bar_o_done, (gg - 1) & 1u, kBarODone, gg))) break;
+        if (__any_sync(0xffffffffu, rescale)) {
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(lane_tmem + C::O_COL + c * 32, r);
+            tmem_wait_ld();
+            reg_fence32(r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(lane_tmem + C::O_COL + c * 32, r);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar_p_full[gg & 1u]);
+      }
+      if (!ok) break;
+      const uint32_t gl = g + it.len - 1;
+      if (!(ok = warp_wait(&bar_o_done, gl & 1u, kBarODone, gl))) break;
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(lane_tmem + C::O_COL + c * 32, r);
+        tmem_wait_ld();
+        reg_fence32(r);
+        if (store) {
+          uint4 *dst = reinterpret_cast<uint4 *>(p.out + orow * D + c * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(r[8 * v4 + 0]) * inv_l, __uint_as_float(r[8 * v4 + 1]) * inv_l);
+            w.y = pack_bf16x2(__uint_as_float(r[8 * v4 + 2]) * inv_l, __uint_as_float(r[8 * v4 + 3]) * inv_l);
+            w.z = pack_bf16x2(__uint_as_float(r[8 * v4 + 4]) * inv_l, __uint_as_float(r[8 * v4 + 5]) * inv_l);
+            w.w = pack_bf16x2(__uint_as_float(r[8 * v4 + 6]) * inv_l, __uint_as_float(r[8 * v4 + 7]) * inv_l);
+            dst[v4] = w;
+          }
+        }
+      }
+      if (store && p.lse) p.lse[orow] = (m_ref + log2f(l)) * 0.69314718055994531f;
+      tc_fence_before();
+      mbar_arrive(&bar_o_empty);
+      g += it.len;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) {
+    __syncwarp();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace bsa

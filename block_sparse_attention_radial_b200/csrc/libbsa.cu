@@ -1,0 +1,414 @@
+// libbsa: host side of the C ABI declared in include/bsa.h.
+//
+// Argument checking, TMA descriptor encoding and kernel launches. The library
+// keeps no device allocations; per-device state is limited to the status word
+// (a __device__ variable) and a few cached device attributes.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "bsa.h"
+
+#include "attn_fwd_sm100.cuh"
+#include "dense_ref.cuh"
+#include "device_status.cuh"
+#include "lists.cuh"
+
+namespace bsa {
+namespace {
+
+thread_local char t_last_error[256] = "";
+
+int cuda_fail(cudaError_t e, const char *what) {
+  std::snprintf(t_last_error, sizeof(t_last_error), "%s: %s (%s)", what, cudaGetErrorName(e),
+                cudaGetErrorString(e));
+  return BSA_ERR_CUDA;
+}
+
+#define BSA_CUDA(call)                                  \
+  do {                                                  \
+    cudaError_t e_ = (call);                            \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
+  } while (0)
+
+// Test hooks (bsa_set_test_hooks).
+std::mutex g_hook_mu;
+unsigned long long g_wait_limit_ns = 2000000000ull;
+int g_fault_flags = 0;
+
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+  bool probed = false;
+  int cc_major = 0, cc_minor = 0, sms = 0;
+  bool attrs_set[4] = {false, false, false, false};
+  bool ref_attrs_set[4] = {false, false, false, false};
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int current_device(DeviceInfo **info) {
+  int dev = 0;
+  BSA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return BSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo &d = g_dev[dev];
+  if (!d.probed) {
+    BSA_CUDA(cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev));
+    BSA_CUDA(cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev));
+    BSA_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+    d.probed = true;
+  }
+  *info = &d;
+  return BSA_OK;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [batch*heads, n, D] bf16 viewed as a 3-D tensor; box of 64 x rows x 1 with
+// 128-byte swizzling (one 128-byte row segment per box row). Rows past n read
+// as zeros.
+int make_map(CUtensorMap *map, const void *ptr, int bh, int n, int D, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    std::snprintf(t_last_error, sizeof(t_last_error), "cuTensorMapEncodeTiled not available");
+    return BSA_ERR_CUDA;
+  }
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(n),
+                        static_cast<cuuint64_t>(bh)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                           static_cast<cuuint64_t>(n) * static_cast<cuuint64_t>(D) * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(t_last_error, sizeof(t_last_error), "cuTensorMapEncodeTiled failed (%d)",
+                  static_cast<int>(r));
+    return BSA_ERR_CUDA;
+  }
+  return BSA_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+// Shared argument checks of the two attention entry points.
+int check_attn_args(const void *q, const void *k, const void *v, int32_t batch, int32_t heads,
+                    int32_t n, int32_t head_dim, const bsa_block_lists *l, const void *out) {
+  if (!q || !k || !v || !out || !l || !l->row_ptr || (l->nnz > 0 && !l->col_idx))
+    return BSA_ERR_INVALID_ARG;
+  if (batch < 1 || heads < 1 || n < 1) return BSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
+  if (l->block != 64 && l->block != 128) return BSA_ERR_UNSUPPORTED;
+  const long long nb = (static_cast<long long>(n) + l->block - 1) / l->block;
+  if (l->num_q_blocks != nb || l->num_k_blocks != nb) return BSA_ERR_INVALID_ARG;
+  if (l->num_lists != 1 && l->num_lists != heads) return BSA_ERR_INVALID_ARG;
+  if (l->nnz < 0) return BSA_ERR_INVALID_ARG;
+  const long long bh = static_cast<long long>(batch) * heads;
+  if (bh * nb > 0x7fffffffLL || bh * n > 0x7fffffffLL) return BSA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return BSA_ERR_INVALID_ARG;
+  const size_t bytes = static_cast<size_t>(bh) * n * head_dim * 2;
+  if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes) ||
+      overlaps(out, bytes, v, bytes))
+    return BSA_ERR_INVALID_ARG;
+  return BSA_OK;
+}
+
+size_t order_bytes(const bsa_block_lists *l) {
+  return (static_cast<size_t>(l->num_lists) * l->num_q_blocks * sizeof(int32_t) + 255) & ~size_t(255);
+}
+
+constexpr int kLptMaxRows = 12288;  // rows whose costs fit in 48 KB of shared memory
+
+template <int D, int BN>
+int launch_fwd(const void *q, const void *k, const void *v, int32_t bh, int32_t n,
+               const FwdParams &p, DeviceInfo *dev, int slot, cudaStream_t stream) {
+  using C = FwdCfg<D, BN>;
+  CUtensorMap tq, tk, tv;
+  int st;
+  if ((st = make_map(&tq, q, bh, n, D, C::BM)) != BSA_OK) return st;
+  if ((st = make_map(&tk, k, bh, n, D, BN)) != BSA_OK) return st;
+  if ((st = make_map(&tv, v, bh, n, D, BN)) != BSA_OK) return st;
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!dev->attrs_set[slot]) {
+      BSA_CUDA(cudaFuncSetAttribute(attn_fwd_sm100_kernel<D, BN>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::DSMEM));
+      dev->attrs_set[slot] = true;
+    }
+  }
+  const int grid = p.total_items < dev->sms ? p.total_items : dev->sms;
+  attn_fwd_sm100_kernel<D, BN><<<grid, C::THREADS, C::DSMEM, stream>>>(tq, tk, tv, p);
+  BSA_CUDA(cudaGetLastError());
+  return BSA_OK;
+}
+
+template <int D, int BLK>
+int launch_ref(const RefParams &p, int batch, DeviceInfo *dev, int slot, cudaStream_t stream) {
+  const size_t smem = dense_ref_smem_bytes<D, BLK>(p.nkb);
+  if (smem > static_cast<size_t>(kSmemLimit) - 64) return BSA_ERR_UNSUPPORTED;
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!dev->ref_attrs_set[slot]) {
+      BSA_CUDA(cudaFuncSetAttribute(dense_masked_ref_kernel<D, BLK>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kSmemLimit - 64));
+      dev->ref_attrs_set[slot] = true;
+    }
+  }
+  dim3 grid(p.nqb, p.heads, batch);
+  dense_masked_ref_kernel<D, BLK><<<grid, 2 * BLK, smem, stream>>>(p);
+  BSA_CUDA(cudaGetLastError());
+  return BSA_OK;
+}
+
+int slot_of(int D, int BN) { return (D == 128 ? 2 : 0) + (BN == 128 ? 1 : 0); }
+
+}  // namespace
+}  // namespace bsa
+
+using namespace bsa;
+
+extern "C" {
+
+int bsa_radial_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t block,
+                          int32_t *row_ptr, int32_t *col_idx, int64_t col_capacity,
+                          int64_t *nnz_out, bsa_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (frames < 1 || tokens_per_frame < 1 || !row_ptr) return BSA_ERR_INVALID_ARG;
+  if (block != 64 && block != 128) return BSA_ERR_UNSUPPORTED;
+  const long long n = static_cast<long long>(frames) * tokens_per_frame;
+  if (n > 0x7fffffffLL) return BSA_ERR_INVALID_ARG;
+  const int nb = ceil_div(n, block);
+  if (nb > 262144) return BSA_ERR_UNSUPPORTED;
+  if (col_idx && col_capacity < 0) return BSA_ERR_INVALID_ARG;
+  RadialGeom g;
+  g.frames = frames;
+  g.tpf = tokens_per_frame;
+  g.block = block;
+  g.n = static_cast<int>(n);
+  g.nb = nb;
+  int rs = 0;
+  if (tokens_per_frame >= block)
+    while ((tokens_per_frame >> (rs + 1)) >= block) ++rs;
+  g.rstar = rs;
+  const size_t smem = static_cast<size_t>((nb + 31) / 32) * sizeof(uint32_t);
+  radial_count_kernel<<<nb, 128, smem, stream>>>(g, row_ptr);
+  BSA_CUDA(cudaGetLastError());
+  scan_rows_kernel<<<1, 1024, 0, stream>>>(row_ptr, nb);
+  BSA_CUDA(cudaGetLastError());
+  if (nnz_out) {
+    int32_t last = 0;
+    BSA_CUDA(cudaMemcpyAsync(&last, row_ptr + nb, sizeof(int32_t), cudaMemcpyDeviceToHost, stream));
+    BSA_CUDA(cudaStreamSynchronize(stream));
+    *nnz_out = last;
+    if (col_idx && last > col_capacity) return BSA_ERR_CAPACITY;
+  }
+  if (col_idx) {
+    radial_fill_kernel<<<nb, 128, smem, stream>>>(g, row_ptr, col_idx, col_capacity);
+    BSA_CUDA(cudaGetLastError());
+  }
+  return BSA_OK;
+}
+
+size_t bsa_attn_fwd_workspace_bytes(int32_t batch, int32_t heads, const bsa_block_lists *l) {
+  if (!l || batch < 1 || heads < 1 || l->num_q_blocks < 1) return 0;
+  if (l->num_lists != 1 && l->num_lists != heads) return 0;
+  return order_bytes(l);
+}
+
+int bsa_attn_fwd(const void *q, const void *k, const void *v, int32_t batch, int32_t heads,
+                 int32_t n, int32_t head_dim, float softmax_scale, const bsa_block_lists *l,
+                 void *out, float *lse, void *workspace, size_t workspace_bytes,
+                 bsa_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int st = check_attn_args(q, k, v, batch, heads, n, head_dim, l, out);
+  if (st != BSA_OK) return st;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < order_bytes(l))
+    return BSA_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return BSA_ERR_INVALID_ARG;
+  DeviceInfo *dev = nullptr;
+  if ((st = current_device(&dev)) != BSA_OK) return st;
+  if (dev->cc_major != 10) return BSA_ERR_UNSUPPORTED;
+
+  const int nqb = l->num_q_blocks;
+  int32_t *order = static_cast<int32_t *>(workspace);
+  const size_t lpt_smem = static_cast<size_t>(nqb <= kLptMaxRows ? nqb : 0) * sizeof(int);
+  lpt_order_kernel<<<l->num_lists, 1024, lpt_smem, stream>>>(l->row_ptr, nqb, l->nnz, order,
+                                                            kLptMaxRows);
+  BSA_CUDA(cudaGetLastError());
+
+  FwdParams p;
+  p.row_ptr = l->row_ptr;
+  p.col_idx = l->col_idx;
+  p.order = order;
+  p.out = static_cast<__nv_bfloat16 *>(out);
+  p.lse = lse;
+  p.heads = heads;
+  p.n = n;
+  p.nqb = nqb;
+  p.nkb = l->num_k_blocks;
+  p.num_lists = l->num_lists;
+  p.nnz = l->nnz;
+  p.total_items = batch * heads * nqb;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
+  p.scale_log2 = scale * 1.4426950408889634f;
+  {
+    std::lock_guard<std::mutex> lk(g_hook_mu);
+    p.wait_limit_ns = g_wait_limit_ns;
+    p.fault_flags = g_fault_flags;
+    g_fault_flags = 0;
+  }
+  const int bh = batch * heads;
+  const int slot = slot_of(head_dim, l->block);
+  if (head_dim == 128 && l->block == 128)
+    return launch_fwd<128, 128>(q, k, v, bh, n, p, dev, slot, stream);
+  if (head_dim == 128 && l->block == 64)
+    return launch_fwd<128, 64>(q, k, v, bh, n, p, dev, slot, stream);
+  if (head_dim == 64 && l->block == 128)
+    return launch_fwd<64, 128>(q, k, v, bh, n, p, dev, slot, stream);
+  return launch_fwd<64, 64>(q, k, v, bh, n, p, dev, slot, stream);
+}
+
+int bsa_attn_dense_masked_ref(const void *q, const void *k, const void *v, int32_t batch,
+                              int32_t heads, int32_t n, int32_t head_dim, float softmax_scale,
+                              const bsa_block_lists *l, void *out, float *lse,
+                              bsa_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int st = check_attn_args(q, k, v, batch, heads, n, head_dim, l, out);
+  if (st != BSA_OK) return st;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return BSA_ERR_INVALID_ARG;
+  if (batch > 65535 || heads > 65535) return BSA_ERR_UNSUPPORTED;
+  DeviceInfo *dev = nullptr;
+  if ((st = current_device(&dev)) != BSA_OK) return st;
+  RefParams p;
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.k = static_cast<const __nv_bfloat16 *>(k);
+  p.v = static_cast<const __nv_bfloat16 *>(v);
+  p.out = static_cast<__nv_bfloat16 *>(out);
+  p.lse = lse;
+  p.row_ptr = l->row_ptr;
+  p.col_idx = l->col_idx;
+  p.heads = heads;
+  p.n = n;
+  p.nqb = l->num_q_blocks;
+  p.nkb = l->num_k_blocks;
+  p.num_lists = l->num_lists;
+  p.nnz = l->nnz;
+  p.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
+  const int slot = slot_of(head_dim, l->block);
+  if (head_dim == 128 && l->block == 128) return launch_ref<128, 128>(p, batch, dev, slot, stream);
+  if (head_dim == 128 && l->block == 64) return launch_ref<128, 64>(p, batch, dev, slot, stream);
+  if (head_dim == 64 && l->block == 128) return launch_ref<64, 128>(p, batch, dev, slot, stream);
+  return launch_ref<64, 64>(p, batch, dev, slot, stream);
+}
+
+int bsa_validate_lists(const bsa_block_lists *l, bsa_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!l || !l->row_ptr || l->num_lists < 1 || l->num_q_blocks < 1 || l->num_k_blocks < 1 ||
+      l->nnz < 0 || (l->nnz > 0 && !l->col_idx))
+    return BSA_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(l->num_lists) * l->num_q_blocks;
+  if (rows > (1LL << 28)) return BSA_ERR_INVALID_ARG;
+  int32_t *host = static_cast<int32_t *>(std::malloc(static_cast<size_t>(rows + 1) * sizeof(int32_t)));
+  if (!host) return BSA_ERR_INVALID_ARG;
+  cudaError_t e = cudaMemcpyAsync(host, l->row_ptr, static_cast<size_t>(rows + 1) * sizeof(int32_t),
+                                  cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) {
+    std::free(host);
+    return cuda_fail(e, "bsa_validate_lists: read row_ptr");
+  }
+  bool bad = host[0] != 0 || host[rows] != l->nnz;
+  for (long long r = 0; r < rows && !bad; ++r) bad = host[r + 1] < host[r];
+  std::free(host);
+  if (bad) return BSA_ERR_BAD_LISTS;
+  // The device check reports through the status word; keep whatever another
+  // kernel recorded before and restore it afterwards.
+  unsigned int prior = 0, zero = 0, after = 0;
+  BSA_CUDA(cudaStreamSynchronize(stream));
+  BSA_CUDA(cudaMemcpyFromSymbol(&prior, g_status, sizeof(prior)));
+  BSA_CUDA(cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)));
+  const int threads = 256;
+  const long long blocks = (rows + threads - 1) / threads;
+  validate_cols_kernel<<<static_cast<int>(blocks < 4096 ? blocks : 4096), threads, 0, stream>>>(
+      l->row_ptr, l->col_idx, static_cast<int>(rows), l->num_k_blocks);
+  BSA_CUDA(cudaGetLastError());
+  BSA_CUDA(cudaStreamSynchronize(stream));
+  BSA_CUDA(cudaMemcpyFromSymbol(&after, g_status, sizeof(after)));
+  BSA_CUDA(cudaMemcpyToSymbol(g_status, &prior, sizeof(prior)));
+  return after == BSA_ERR_BAD_LISTS ? BSA_ERR_BAD_LISTS : BSA_OK;
+}
+
+int bsa_get_device_status(bsa_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  BSA_CUDA(cudaStreamSynchronize(stream));
+  unsigned int v = 0, zero = 0;
+  BSA_CUDA(cudaMemcpyFromSymbol(&v, g_status, sizeof(v)));
+  BSA_CUDA(cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)));
+  return static_cast<int>(v);
+}
+
+int bsa_get_timeout_detail(int32_t *out4) {
+  if (!out4) return BSA_ERR_INVALID_ARG;
+  unsigned int d[4];
+  BSA_CUDA(cudaMemcpyFromSymbol(d, g_status_detail, sizeof(d)));
+  for (int i = 0; i < 4; ++i) out4[i] = static_cast<int32_t>(d[i]);
+  return BSA_OK;
+}
+
+const char *bsa_status_string(int status) {
+  switch (status) {
+    case BSA_OK: return "ok";
+    case BSA_ERR_INVALID_ARG: return "invalid argument";
+    case BSA_ERR_UNSUPPORTED: return "unsupported head_dim, block or device";
+    case BSA_ERR_CUDA: return "CUDA runtime error";
+    case BSA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case BSA_ERR_BAD_LISTS: return "malformed block lists";
+    case BSA_ERR_CAPACITY: return "col_idx capacity too small";
+    default: return "unknown status";
+  }
+}
+
+const char *bsa_last_cuda_error(void) { return t_last_error; }
+
+int bsa_set_test_hooks(int64_t wait_limit_ns, int32_t fault_flags) {
+  if (wait_limit_ns < 0) return BSA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_hook_mu);
+  g_wait_limit_ns = wait_limit_ns == 0 ? 2000000000ull : static_cast<unsigned long long>(wait_limit_ns);
+  g_fault_flags = fault_flags;
+  return BSA_OK;
+}
+
+}  // extern "C"

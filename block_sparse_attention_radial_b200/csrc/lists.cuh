@@ -1,0 +1,204 @@
+// Block-list kernels: the radial mask builder, list validation and the
+// longest-row-first work order used by the attention kernel.
+#pragma once
+
+#include <cstdint>
+
+#include "device_status.cuh"
+
+namespace bsa {
+
+// ----------------------------------------------------------- block helpers --
+
+// Inclusive prefix sum over the CTA (blockDim.x a multiple of 32, <= 1024).
+// `scratch` holds 32 ints. Returns this thread's inclusive sum; `total` gets
+// the CTA total.
+template <typename T>
+__device__ T cta_inclusive_scan(T x, T *scratch, T &total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    T y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scratch[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    T w = lane < nwarps ? scratch[lane] : T(0);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      T y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    scratch[lane] = w;
+  }
+  __syncthreads();
+  if (warp > 0) x += scratch[warp - 1];
+  total = scratch[nwarps - 1];
+  __syncthreads();
+  return x;
+}
+
+// ------------------------------------------------------------ radial mask --
+
+struct RadialGeom {
+  int32_t frames, tpf, block, n, nb, rstar;
+};
+
+__device__ __forceinline__ int band_of(int d) { return 31 - __clz(d < 1 ? 1 : d); }
+
+// Sets, in the shared bitmap `bits`, every key block of query block `qb`.
+//
+// For one query frame f_i and one key frame f_j the admitted keys of query
+// in-frame position s form the window [st(s), st(s) + w) with
+// st(s) = clamp(s - w/2, 0, S - w). st is non-decreasing in s and moves by at
+// most one per step, so the union over the query block's positions
+// [s_lo, s_hi] in that frame is the single interval [st(s_lo), st(s_hi) + w).
+// Its key blocks are marked; the threads of the CTA share the (f_i, f_j) pairs.
+__device__ void radial_mark_row(const RadialGeom g, int qb, uint32_t *bits) {
+  const int t0 = qb * g.block;
+  const int t1 = min(g.n, t0 + g.block);  // query tokens [t0, t1)
+  const int fa = t0 / g.tpf, fb = (t1 - 1) / g.tpf;
+  const int pairs = (fb - fa + 1) * g.frames;
+  for (int p = threadIdx.x; p < pairs; p += blockDim.x) {
+    const int fi = fa + p / g.frames, fj = p % g.frames;
+    const int d = abs(fi - fj);
+    const int r = band_of(d);
+    if (r > g.rstar && (d & ((1 << (r - g.rstar)) - 1)) != 0) continue;  // thinned frame
+    const int w = max(1, g.tpf >> min(r, g.rstar));
+    const int s_lo = max(t0, fi * g.tpf) - fi * g.tpf;
+    const int s_hi = min(t1, (fi + 1) * g.tpf) - 1 - fi * g.tpf;
+    const int st_lo = min(max(s_lo - w / 2, 0), g.tpf - w);
+    const int st_hi = min(max(s_hi - w / 2, 0), g.tpf - w);
+    const int b0 = (fj * g.tpf + st_lo) / g.block;
+    const int b1 = (fj * g.tpf + st_hi + w - 1) / g.block;
+    for (int b = b0; b <= b1; ++b) atomicOr(&bits[b >> 5], 1u << (b & 31));
+  }
+}
+
+__device__ void radial_row_bitmap(const RadialGeom g, int qb, uint32_t *bits, int words) {
+  for (int i = threadIdx.x; i < words; i += blockDim.x) bits[i] = 0u;
+  __syncthreads();
+  radial_mark_row(g, qb, bits);
+  __syncthreads();
+}
+
+// One CTA per query block: row length into row_ptr[qb + 1].
+__global__ void radial_count_kernel(RadialGeom g, int32_t *row_ptr) {
+  extern __shared__ uint32_t bits[];
+  __shared__ int scratch[32];
+  const int words = (g.nb + 31) >> 5;
+  radial_row_bitmap(g, blockIdx.x, bits, words);
+  int c = 0;
+  for (int i = threadIdx.x; i < words; i += blockDim.x) c += __popc(bits[i]);
+  int total;
+  cta_inclusive_scan(c, scratch, total);
+  if (threadIdx.x == 0) {
+    row_ptr[blockIdx.x + 1] = total;
+    if (blockIdx.x == 0) row_ptr[0] = 0;
+  }
+}
+
+// Single CTA: in-place inclusive scan of row_ptr[1..rows]; row_ptr[0] = 0.
+__global__ void scan_rows_kernel(int32_t *row_ptr, int rows) {
+  __shared__ long long scratch[32];
+  long long carry = 0;
+  for (int base = 0; base < rows; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    long long x = i < rows ? row_ptr[i + 1] : 0;
+    long long total;
+    long long inc = cta_inclusive_scan(x, scratch, total);
+    const long long v = carry + inc;
+    if (i < rows) {
+      if (v > 0x7fffffffLL) record_status(6u /* BSA_ERR_CAPACITY */);
+      row_ptr[i + 1] = static_cast<int32_t>(v > 0x7fffffffLL ? 0x7fffffffLL : v);
+    }
+    carry += total;
+  }
+}
+
+// One CTA per query block: write the row's key blocks in ascending order.
+__global__ void radial_fill_kernel(RadialGeom g, const int32_t *row_ptr, int32_t *col_idx,
+                                   long long capacity) {
+  extern __shared__ uint32_t bits[];
+  __shared__ int scratch[32];
+  const int words = (g.nb + 31) >> 5;
+  radial_row_bitmap(g, blockIdx.x, bits, words);
+  // each thread owns a contiguous run of words, so ascending thread order is
+  // ascending block order
+  const int per = (words + blockDim.x - 1) / blockDim.x;
+  const int w0 = min(words, threadIdx.x * per), w1 = min(words, w0 + per);
+  int c = 0;
+  for (int i = w0; i < w1; ++i) c += __popc(bits[i]);
+  int total;
+  const int inc = cta_inclusive_scan(c, scratch, total);
+  long long pos = static_cast<long long>(row_ptr[blockIdx.x]) + (inc - c);
+  for (int i = w0; i < w1; ++i) {
+    uint32_t b = bits[i];
+    while (b) {
+      const int t = __ffs(b) - 1;
+      b &= b - 1;
+      if (pos < capacity) {
+        col_idx[pos] = i * 32 + t;
+      } else {
+        record_status(6u /* BSA_ERR_CAPACITY */);
+      }
+      ++pos;
+    }
+  }
+}
+
+// ------------------------------------------------------------- validation --
+
+// Grid-stride over rows; row_ptr has already been checked on the host to be
+// monotone and bounded by nnz, so every read here is in bounds.
+__global__ void validate_cols_kernel(const int32_t *row_ptr, const int32_t *col_idx, int rows,
+                                     int nkb) {
+  for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < rows; r += gridDim.x * blockDim.x) {
+    const int a = row_ptr[r], b = row_ptr[r + 1];
+    int prev = -1;
+    for (int e = a; e < b; ++e) {
+      const int c = col_idx[e];
+      if (c <= prev || c >= nkb) {
+        record_status(5u /* BSA_ERR_BAD_LISTS */);
+        break;
+      }
+      prev = c;
+    }
+  }
+}
+
+// ------------------------------------------------------------ work order --
+
+// One CTA per list. order[list * nqb + rank] = query block with the rank-th
+// longest row (ties: lower block first). Rows are ranked by counting, which
+// keeps the order deterministic. Lists with more rows than fit in shared
+// memory keep their natural order.
+__global__ void lpt_order_kernel(const int32_t *row_ptr, int nqb, int nnz, int32_t *order,
+                                 int max_smem_rows) {
+  extern __shared__ int cost[];
+  const int list = blockIdx.x;
+  const int32_t *rp = row_ptr + static_cast<long long>(list) * nqb;
+  int32_t *ord = order + static_cast<long long>(list) * nqb;
+  if (nqb > max_smem_rows) {
+    for (int r = threadIdx.x; r < nqb; r += blockDim.x) ord[r] = r;
+    return;
+  }
+  for (int r = threadIdx.x; r < nqb; r += blockDim.x) {
+    const int a = min(max(rp[r], 0), nnz), b = min(max(rp[r + 1], 0), nnz);
+    cost[r] = max(b - a, 0);
+  }
+  __syncthreads();
+  for (int r = threadIdx.x; r < nqb; r += blockDim.x) {
+    const int c = cost[r];
+    int rank = 0;
+    for (int o = 0; o < nqb; ++o) {
+      const int co = cost[o];
+      rank += (co > c) || (co == c && o < r);
+    }
+    ord[rank] = r;
+  }
+}
+
+}  // namespace bsa

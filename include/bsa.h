@@ -1,0 +1,195 @@
+/*
+ * bsa.h - C ABI of libbsa: radial block-sparse softmax attention, forward pass,
+ * for NVIDIA B200 (sm_100a).
+ *
+ * Sources of the operations (page title, section):
+ *  - "Radial Attention: O(nlog n) Sparse Attention with Energy Decay for Long
+ *    Video Generation" skill page (skillsmp.com, radial-attention-video),
+ *    Step 1 (radial mask: frame-major tokens, log2 temporal bands, decay) and
+ *    Step 2 (RadialAttention.forward: softmax(Q K^T * head_dim^-0.5 + mask) V,
+ *    layout [batch, heads, n, head_dim]).
+ *  - "Radial Attention: A Breakthrough in Efficient Long Video Generation"
+ *    (thismoment.ai), "How Radial Attention Works": density halves as temporal
+ *    distance doubles, a spatial window that shrinks for distant frames, and
+ *    128x128 block sparsity.
+ *  - Sparse-vDiT skill page (skillsmp.com), "Sparse attention patterns", and
+ *    the Compact Attention abstract (zhuanzhiai.com): per-head tile masks,
+ *    passed to bsa_attn_fwd as per-head block lists.
+ *
+ * Conventions for every entry point:
+ *  - Every function returns a bsa_status value (0 = BSA_OK).
+ *  - Device pointers are plain CUDA device addresses owned by the caller; the
+ *    library never frees or keeps them. The library allocates no device
+ *    memory; scratch memory is the caller's `workspace`.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream). All work
+ *    is stream-ordered and asynchronous unless a function says it
+ *    synchronises.
+ *  - Errors found on the host (bad argument, unsupported shape, launch
+ *    failure) are returned directly and nothing is launched. Errors found on
+ *    the device (a bounded wait that ran out, a list entry out of range, an
+ *    output buffer too small) are recorded in a per-device status word and
+ *    reported by bsa_get_device_status().
+ */
+#ifndef BSA_H
+#define BSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *bsa_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = 1,    /* null/misaligned pointer, inconsistent sizes, aliasing */
+  BSA_ERR_UNSUPPORTED = 2,    /* head_dim, block or device not supported */
+  BSA_ERR_CUDA = 3,           /* a CUDA runtime call failed; see bsa_last_cuda_error() */
+  BSA_ERR_DEVICE_TIMEOUT = 4, /* a bounded device-side wait ran out; results are invalid */
+  BSA_ERR_BAD_LISTS = 5,      /* block lists not monotone / sorted / in range */
+  BSA_ERR_CAPACITY = 6        /* col_idx capacity smaller than the list size */
+} bsa_status;
+
+/*
+ * Per-query-block key-block lists in CSR form (device memory).
+ *
+ * num_lists     1 (one list shared by every head) or `heads` (head h uses
+ *               list h, whose rows start at h * num_q_blocks).
+ * num_q_blocks  ceil(n / block); num_k_blocks is the same value.
+ * block         tile edge in tokens: 64 or 128.
+ * row_ptr       int32[num_lists * num_q_blocks + 1], row_ptr[0] = 0,
+ *               non-decreasing.
+ * col_idx       int32[nnz], each row strictly increasing, entries in
+ *               [0, num_k_blocks).
+ * nnz           entries in col_idx (= row_ptr[last]). Kernels clamp every row
+ *               bound into [0, nnz] and every entry into [0, num_k_blocks), so
+ *               malformed lists give wrong results, never an out-of-bounds
+ *               access; bsa_validate_lists() detects them.
+ *
+ * A query in query block qb attends to every key j < n of every key block the
+ * row lists (block granularity, thismoment.ai page: 128x128 block sparsity).
+ */
+typedef struct {
+  int32_t num_lists;
+  int32_t num_q_blocks;
+  int32_t num_k_blocks;
+  int32_t block;
+  int32_t nnz;
+  const int32_t *row_ptr;
+  const int32_t *col_idx;
+} bsa_block_lists;
+
+/*
+ * Build the radial block lists for `frames` x `tokens_per_frame` tokens
+ * (n = frames * tokens_per_frame, frame-major) at tile size `block`.
+ *
+ * Rule (skillsmp radial-attention-video Step 1; thismoment.ai "How Radial
+ * Attention Works"): temporal distance d = |f_i - f_j| has band
+ * r = floor(log2(max(d, 1))); band r keeps a window of S >> min(r, r*) keys
+ * (S = tokens_per_frame, r* = the last band whose window still holds `block`
+ * keys, 0 if S < block) centred on the query's in-frame index and clamped into
+ * the frame; bands beyond r* keep only frames with d % 2^(r - r*) == 0. A key
+ * block is listed for a query block when any admitted token pair falls in it.
+ *
+ * row_ptr      device int32[ceil(n/block) + 1], written.
+ * col_idx      device int32[col_capacity], or NULL to compute row_ptr only.
+ * col_capacity entries available in col_idx (ignored when col_idx is NULL).
+ * nnz_out      host int64*, or NULL. When given, the call synchronises
+ *              `stream`, writes the list size and returns BSA_ERR_CAPACITY if
+ *              col_idx was given and is too small (nothing beyond the capacity
+ *              is written). When NULL the call is asynchronous and an
+ *              overflow is reported by bsa_get_device_status().
+ * Limits: 1 <= frames, 1 <= tokens_per_frame, n < 2^31, block in {64, 128},
+ * ceil(n/block) <= 262144.
+ */
+int bsa_radial_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t block,
+                          int32_t *row_ptr, int32_t *col_idx, int64_t col_capacity,
+                          int64_t *nnz_out, bsa_stream_t stream);
+
+/*
+ * Bytes of device scratch memory bsa_attn_fwd needs for this problem (the
+ * longest-row-first work order of every list). Returns 0 for invalid lists.
+ */
+size_t bsa_attn_fwd_workspace_bytes(int32_t batch, int32_t heads, const bsa_block_lists *lists);
+
+/*
+ * Block-sparse softmax attention forward (skillsmp radial-attention-video
+ * Step 2, RadialAttention.forward, restricted to the listed blocks):
+ *   out[b,h,i,:] = sum_j softmax_j(scale * <q[b,h,i], k[b,h,j]>) v[b,h,j,:]
+ * over the keys j < n of the blocks listed for i's query block;
+ *   lse[b,h,i]   = natural log of sum_j exp(scale * <q[b,h,i], k[b,h,j]>).
+ * A row with an empty list gets out = 0 and lse = -inf.
+ *
+ * q, k, v       device bf16 [batch, heads, n, head_dim], contiguous, 16-byte
+ *               aligned. They may alias each other.
+ * head_dim      64 or 128.
+ * softmax_scale <= 0 selects head_dim^-0.5.
+ * lists         host pointer to the list descriptor (its arrays on device).
+ * out           device bf16 [batch, heads, n, head_dim]; must not overlap q/k/v.
+ * lse           device float [batch, heads, n], or NULL.
+ * workspace     device scratch of at least bsa_attn_fwd_workspace_bytes(),
+ *               16-byte aligned; overwritten.
+ * Runs on the tensor cores (tcgen05, TMEM accumulators, TMA-staged tiles) of
+ * an sm_100 device; returns BSA_ERR_UNSUPPORTED elsewhere. Asynchronous.
+ */
+int bsa_attn_fwd(const void *q, const void *k, const void *v,
+                 int32_t batch, int32_t heads, int32_t n, int32_t head_dim,
+                 float softmax_scale, const bsa_block_lists *lists,
+                 void *out, float *lse, void *workspace, size_t workspace_bytes,
+                 bsa_stream_t stream);
+
+/*
+ * Same operation, same arguments (no workspace), computed by a plain fp32
+ * CUDA-core kernel that scores every key of every listed block with scalar
+ * arithmetic. It is the full-tensor checker for sizes where the CPU oracle
+ * can only sample rows. Asynchronous.
+ */
+int bsa_attn_dense_masked_ref(const void *q, const void *k, const void *v,
+                              int32_t batch, int32_t heads, int32_t n, int32_t head_dim,
+                              float softmax_scale, const bsa_block_lists *lists,
+                              void *out, float *lse, bsa_stream_t stream);
+
+/*
+ * Check `lists`: row_ptr starts at 0, is non-decreasing and ends at nnz; each
+ * row is strictly increasing and in [0, num_k_blocks). Reads no col_idx entry
+ * at or beyond nnz. Synchronises `stream`. Returns BSA_OK, BSA_ERR_BAD_LISTS
+ * or BSA_ERR_INVALID_ARG (null pointers, sizes out of range).
+ */
+int bsa_validate_lists(const bsa_block_lists *lists, bsa_stream_t stream);
+
+/*
+ * Synchronise `stream`, then return and clear the current device's status
+ * word (BSA_OK, BSA_ERR_DEVICE_TIMEOUT, BSA_ERR_BAD_LISTS or BSA_ERR_CAPACITY).
+ */
+int bsa_get_device_status(bsa_stream_t stream);
+
+/*
+ * Where the first device-side wait that ran out gave up, for diagnosis:
+ * out4[0] role (1 producer, 2 MMA issuer, 3 softmax), out4[1] barrier id,
+ * out4[2] pipeline counter, out4[3] CTA index. Synchronous; not cleared by
+ * bsa_get_device_status().
+ */
+int bsa_get_timeout_detail(int32_t *out4);
+
+/* Static description of a status code. */
+const char *bsa_status_string(int status);
+
+/* Text of the last CUDA error seen by this thread in the library ("" if none). */
+const char *bsa_last_cuda_error(void);
+
+/*
+ * Test hooks. `wait_limit_ns` bounds every device-side wait of bsa_attn_fwd
+ * (0 restores the default of 2 s). `fault_flags` bit 0 makes the next
+ * bsa_attn_fwd launch skip its first K-tile load, so that the consumer's
+ * bounded wait runs out and the call reports BSA_ERR_DEVICE_TIMEOUT through
+ * bsa_get_device_status(); the flag clears itself after one launch.
+ */
+int bsa_set_test_hooks(int64_t wait_limit_ns, int32_t fault_flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H */

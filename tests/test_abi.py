@@ -1,0 +1,96 @@
+"""The C ABI library loads on a machine without a GPU, exports every entry point
+include/bsa.h declares, and rejects bad arguments on the host before any CUDA
+call (CPU only: nothing here launches a kernel)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bsa.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bsa_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_sparse_attention_radial_b200 import _lib
+
+    if not os.path.exists(_lib.LIB_PATH):
+        from block_sparse_attention_radial_b200.build import build
+
+        build()
+    return _lib.load()
+
+
+def test_header_declares_the_entry_points():
+    names = _declared()
+    for n in ("bsa_radial_mask_build", "bsa_attn_fwd", "bsa_attn_dense_masked_ref",
+              "bsa_attn_fwd_workspace_bytes", "bsa_get_device_status", "bsa_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from block_sparse_attention_radial_b200._lib import EXPORTS
+
+    names = _declared()
+    for name in names:
+        assert hasattr(lib, name), name
+    assert sorted(EXPORTS) == names
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        s = lib.bsa_status_string(code).decode()
+        assert s and s != "unknown status"
+    assert lib.bsa_status_string(99).decode() == "unknown status"
+
+
+def test_workspace_bytes(lib):
+    from block_sparse_attention_radial_b200._lib import BlockListsC
+
+    ls = BlockListsC(1, 256, 256, 128, 1000, 0, 0)
+    assert lib.bsa_attn_fwd_workspace_bytes(1, 40, ctypes.byref(ls)) == 1024
+    ls = BlockListsC(24, 256, 256, 128, 1000, 0, 0)
+    assert lib.bsa_attn_fwd_workspace_bytes(1, 24, ctypes.byref(ls)) == 24 * 256 * 4
+    ls = BlockListsC(3, 256, 256, 128, 1000, 0, 0)   # neither 1 nor heads
+    assert lib.bsa_attn_fwd_workspace_bytes(1, 24, ctypes.byref(ls)) == 0
+
+
+def test_host_side_argument_checks(lib):
+    from block_sparse_attention_radial_b200._lib import BlockListsC
+
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)   # never dereferenced: every call below fails its host checks
+    ls = BlockListsC(1, 8, 8, 128, 10, 1 << 22, 1 << 23)
+    call = lambda q, n, D, lst, out, ws=fake, wsb=1 << 12: lib.bsa_attn_fwd(
+        q, fake, fake, 1, 1, n, D, 0.0, ctypes.byref(lst), out, None, ws, wsb, None)
+    assert call(vp(0), 1024, 128, ls, vp(1 << 24)) == 1                       # null q
+    assert call(fake, 1024, 96, ls, vp(1 << 24)) == 2                         # head_dim
+    assert call(fake, 2000, 128, ls, vp(1 << 24)) == 1                        # n vs num_q_blocks
+    bad_block = BlockListsC(1, 8, 8, 32, 10, 1 << 22, 1 << 23)
+    assert call(fake, 256, 128, bad_block, vp(1 << 24)) == 2                  # block size
+    assert call(vp((1 << 20) + 8), 1024, 128, ls, vp(1 << 24)) == 1           # misaligned q
+    assert call(fake, 1024, 128, ls, vp(1 << 20)) == 1                        # out aliases q
+    assert call(fake, 1024, 128, ls, vp(1 << 24), ws=vp(0)) == 1              # no workspace
+    assert call(fake, 1024, 128, ls, vp(1 << 24), wsb=4) == 1                 # workspace too small
+    two = BlockListsC(2, 8, 8, 128, 10, 1 << 22, 1 << 23)
+    assert call(fake, 1024, 128, two, vp(1 << 24)) == 1                       # num_lists
+    assert lib.bsa_attn_dense_masked_ref(fake, fake, fake, 1, 1, 1024, 64, 0.0, ctypes.byref(ls),
+                                         vp(0), None, None) == 1              # null out
+
+
+def test_mask_build_argument_checks(lib):
+    vp = ctypes.c_void_p
+    assert lib.bsa_radial_mask_build(0, 256, 64, vp(1 << 20), None, 0, None, None) == 1
+    assert lib.bsa_radial_mask_build(4, 256, 64, vp(0), None, 0, None, None) == 1
+    assert lib.bsa_radial_mask_build(4, 256, 32, vp(1 << 20), None, 0, None, None) == 2
+    assert lib.bsa_radial_mask_build(1 << 16, 1 << 16, 128, vp(1 << 20), None, 0, None, None) == 1
+    assert lib.bsa_set_test_hooks(-1, 0) == 1
+    assert lib.bsa_set_test_hooks(0, 0) == 0
