@@ -27,8 +27,11 @@ __all__ = [
     "bsa_attn_fwd", "bsa_attn_dense_masked_ref", "bsa_validate_lists", "bsa_get_device_status",
     "bsa_get_timeout_detail", "bsa_status_string", "bsa_last_cuda_error", "bsa_set_test_hooks",
     "radial_block_lists", "block_lists_from_csr", "attention", "dense_masked_reference",
-    "computed_flops",
+    "computed_flops", "bsa_attn_fwd_noalloc", "NOALLOC_MAX_ORDER_ENTRIES",
 ]
+
+# Size of the fixed scratch array behind bsa_attn_fwd_noalloc (int32 entries).
+NOALLOC_MAX_ORDER_ENTRIES = 65536
 
 
 class BsaError(RuntimeError):
@@ -113,6 +116,21 @@ def bsa_attn_fwd(q, k, v, lists: BlockLists, out, lse=None, workspace=None,
                           ctypes.byref(ls), _ptr(out), _ptr(lse), _ptr(workspace),
                           workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "bsa_attn_fwd")
+
+
+def bsa_attn_fwd_noalloc(q, k, v, lists: BlockLists, out, lse=None,
+                         softmax_scale: float = 0.0, stream=None) -> None:
+    """bsa_attn_fwd without a workspace, for callers that cannot allocate device
+    memory (a plugin given only its input and output buffers, a runtime with a
+    memory plan fixed at start-up). Its scratch is a fixed array inside the
+    library, so it needs num_lists * num_q_blocks <= NOALLOC_MAX_ORDER_ENTRIES;
+    calls overlapping on the GPU race on that array. The first call on a device
+    resolves the array's address; make it before any stream capture."""
+    B, H, n, D = q.shape
+    st = _lib.load().bsa_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), B, H, n, D,
+                                          float(softmax_scale), ctypes.byref(lists.c_struct()),
+                                          _ptr(out), _ptr(lse), _stream(stream))
+    _check(st, "bsa_attn_fwd_noalloc")
 
 
 def bsa_attn_dense_masked_ref(q, k, v, lists: BlockLists, out, lse=None,

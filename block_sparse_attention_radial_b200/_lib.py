@@ -25,6 +25,7 @@ EXPORTS = (
     "bsa_status_string",
     "bsa_last_cuda_error",
     "bsa_set_test_hooks",
+    "bsa_attn_fwd_noalloc",
 )
 
 STATUS_NAMES = {
@@ -35,6 +36,7 @@ STATUS_NAMES = {
     4: "BSA_ERR_DEVICE_TIMEOUT",
     5: "BSA_ERR_BAD_LISTS",
     6: "BSA_ERR_CAPACITY",
+    7: "BSA_ERR_SCRATCH_LIMIT",
 }
 
 
@@ -80,6 +82,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "bsa_last_cuda_error": (ctypes.c_char_p, []),
         "bsa_set_test_hooks": (ctypes.c_int, [i64, i32]),
+        "bsa_attn_fwd_noalloc": (ctypes.c_int, [vp, vp, vp, i32, i32, i32, i32, ctypes.c_float,
+                                                lp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

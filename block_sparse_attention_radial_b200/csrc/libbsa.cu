@@ -397,6 +397,7 @@ const char *bsa_status_string(int status) {
     case BSA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
     case BSA_ERR_BAD_LISTS: return "malformed block lists";
     case BSA_ERR_CAPACITY: return "col_idx capacity too small";
+    case BSA_ERR_SCRATCH_LIMIT: return "problem exceeds the fixed scratch of bsa_attn_fwd_noalloc";
     default: return "unknown status";
   }
 }
@@ -412,3 +413,88 @@ int bsa_set_test_hooks(int64_t wait_limit_ns, int32_t fault_flags) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free entry point. Its scratch (the work order) is this fixed
+// array instead of a caller-provided workspace. In host code `g_noalloc_order`
+// names a host-side stand-in, not device memory, so the device address is
+// resolved once per device with cudaGetSymbolAddress and cached.
+// ---------------------------------------------------------------------------
+
+static __device__ __align__(256) int32_t g_noalloc_order[BSA_NOALLOC_MAX_ORDER_ENTRIES];
+
+namespace bsa {
+namespace {
+std::mutex g_noalloc_mu;
+int32_t *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_order on the current device (set up on first use).
+int noalloc_scratch(int32_t **out) {
+  int dev = 0;
+  BSA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return BSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *p = nullptr;
+    BSA_CUDA(cudaGetSymbolAddress(&p, g_noalloc_order));
+    g_noalloc_ptr[dev] = static_cast<int32_t *>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return BSA_OK;
+}
+}  // namespace
+}  // namespace bsa
+
+extern "C" int bsa_attn_fwd_noalloc(const void *q, const void *k, const void *v, int32_t batch,
+                                    int32_t heads, int32_t n, int32_t head_dim,
+                                    float softmax_scale, const bsa_block_lists *l, void *out,
+                                    float *lse, bsa_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int st = check_attn_args(q, k, v, batch, heads, n, head_dim, l, out);
+  if (st != BSA_OK) return st;
+  if (static_cast<long long>(l->num_lists) * l->num_q_blocks > BSA_NOALLOC_MAX_ORDER_ENTRIES)
+    return BSA_ERR_SCRATCH_LIMIT;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return BSA_ERR_INVALID_ARG;
+  DeviceInfo *dev = nullptr;
+  if ((st = current_device(&dev)) != BSA_OK) return st;
+  if (dev->cc_major != 10) return BSA_ERR_UNSUPPORTED;
+  int32_t *order = nullptr;
+  if ((st = noalloc_scratch(&order)) != BSA_OK) return st;
+
+  const int nqb = l->num_q_blocks;
+  const size_t lpt_smem = static_cast<size_t>(nqb <= kLptMaxRows ? nqb : 0) * sizeof(int);
+  lpt_order_kernel<<<l->num_lists, 1024, lpt_smem, stream>>>(l->row_ptr, nqb, l->nnz, order,
+                                                            kLptMaxRows);
+  BSA_CUDA(cudaGetLastError());
+
+  FwdParams p;
+  p.row_ptr = l->row_ptr;
+  p.col_idx = l->col_idx;
+  p.order = order;
+  p.out = static_cast<__nv_bfloat16 *>(out);
+  p.lse = lse;
+  p.heads = heads;
+  p.n = n;
+  p.nqb = nqb;
+  p.nkb = l->num_k_blocks;
+  p.num_lists = l->num_lists;
+  p.nnz = l->nnz;
+  p.total_items = batch * heads * nqb;
+  const float scale =
+      softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
+  p.scale_log2 = scale * 1.4426950408889634f;
+  {
+    std::lock_guard<std::mutex> lk(g_hook_mu);
+    p.wait_limit_ns = g_wait_limit_ns;
+    p.fault_flags = 0;
+  }
+  const int bh = batch * heads;
+  const int slot = slot_of(head_dim, l->block);
+  if (head_dim == 128 && l->block == 128)
+    return launch_fwd<128, 128>(q, k, v, bh, n, p, dev, slot, stream);
+  if (head_dim == 128 && l->block == 64)
+    return launch_fwd<128, 64>(q, k, v, bh, n, p, dev, slot, stream);
+  if (head_dim == 64 && l->block == 128)
+    return launch_fwd<64, 128>(q, k, v, bh, n, p, dev, slot, stream);
+  return launch_fwd<64, 64>(q, k, v, bh, n, p, dev, slot, stream);
+}

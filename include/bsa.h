@@ -49,7 +49,8 @@ typedef enum {
   BSA_ERR_CUDA = 3,           /* a CUDA runtime call failed; see bsa_last_cuda_error() */
   BSA_ERR_DEVICE_TIMEOUT = 4, /* a bounded device-side wait ran out; results are invalid */
   BSA_ERR_BAD_LISTS = 5,      /* block lists not monotone / sorted / in range */
-  BSA_ERR_CAPACITY = 6        /* col_idx capacity smaller than the list size */
+  BSA_ERR_CAPACITY = 6,       /* col_idx capacity smaller than the list size */
+  BSA_ERR_SCRATCH_LIMIT = 7   /* problem too large for bsa_attn_fwd_noalloc's fixed scratch */
 } bsa_status;
 
 /*
@@ -187,6 +188,35 @@ const char *bsa_last_cuda_error(void);
  * bsa_get_device_status(); the flag clears itself after one launch.
  */
 int bsa_set_test_hooks(int64_t wait_limit_ns, int32_t fault_flags);
+
+/*
+ * Allocation-free variant of bsa_attn_fwd. The pages have no counterpart: this
+ * entry point exists for callers that cannot allocate device memory, such as a
+ * plugin that its host framework hands only input and output buffers and no
+ * allocator, or a runtime whose memory plan is fixed at start-up and forbids
+ * later allocations. Those callers cannot provide bsa_attn_fwd's workspace.
+ *
+ * Same operation, arguments and results as bsa_attn_fwd, minus the workspace:
+ * the scratch it needs (the longest-row-first work order, one int32 per query
+ * block per list) lives in a fixed array compiled into the library, of
+ * BSA_NOALLOC_MAX_ORDER_ENTRIES int32 entries (256 KiB). Every GPU that loads
+ * the library holds that array until the process exits.
+ *
+ * - Returns BSA_ERR_SCRATCH_LIMIT, launching nothing, when
+ *   lists->num_lists * lists->num_q_blocks exceeds the maximum.
+ * - Calls no cudaMalloc, cudaFree or other allocating routine.
+ * - The first call on each device resolves the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ * - All calls share the one array and each call overwrites the entries it
+ *   uses (nothing in it has to start at zero). Calls whose kernels overlap on
+ *   the GPU (for example on two streams at once) race on it; serialise them.
+ */
+#define BSA_NOALLOC_MAX_ORDER_ENTRIES 65536
+int bsa_attn_fwd_noalloc(const void *q, const void *k, const void *v,
+                         int32_t batch, int32_t heads, int32_t n, int32_t head_dim,
+                         float softmax_scale, const bsa_block_lists *lists,
+                         void *out, float *lse, bsa_stream_t stream);
 
 #ifdef __cplusplus
 }
