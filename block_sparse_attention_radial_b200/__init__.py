@@ -27,7 +27,7 @@ __all__ = [
     "bsa_attn_fwd", "bsa_attn_dense_masked_ref", "bsa_validate_lists", "bsa_get_device_status",
     "bsa_get_timeout_detail", "bsa_status_string", "bsa_last_cuda_error", "bsa_set_test_hooks",
     "radial_block_lists", "block_lists_from_csr", "attention", "dense_masked_reference",
-    "computed_flops", "bsa_attn_fwd_noalloc", "NOALLOC_MAX_ORDER_ENTRIES",
+    "computed_flops", "bsa_attn_fwd_noalloc", "bsa_selftest_exp2", "NOALLOC_MAX_ORDER_ENTRIES",
 ]
 
 # Size of the fixed scratch array behind bsa_attn_fwd_noalloc (int32 entries).
@@ -170,6 +170,14 @@ def bsa_status_string(status: int) -> str:
 
 def bsa_last_cuda_error() -> str:
     return _lib.load().bsa_last_cuda_error().decode()
+
+
+def bsa_selftest_exp2(x: torch.Tensor):
+    """(poly, mufu, exp2f) results of the softmax's exponential paths on float32 ``x``."""
+    ys = [torch.empty_like(x) for _ in range(3)]
+    _check(_lib.load().bsa_selftest_exp2(_ptr(x), *(_ptr(y) for y in ys), x.numel(),
+                                         _stream(None)), "bsa_selftest_exp2")
+    return tuple(ys)
 
 
 def bsa_set_test_hooks(wait_limit_ns: int = 0, fault_flags: int = 0) -> None:

@@ -25,6 +25,7 @@ EXPORTS = (
     "bsa_status_string",
     "bsa_last_cuda_error",
     "bsa_set_test_hooks",
+    "bsa_selftest_exp2",
     "bsa_attn_fwd_noalloc",
 )
 
@@ -82,6 +83,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "bsa_last_cuda_error": (ctypes.c_char_p, []),
         "bsa_set_test_hooks": (ctypes.c_int, [i64, i32]),
+        "bsa_selftest_exp2": (ctypes.c_int, [vp, vp, vp, vp, i32, vp]),
         "bsa_attn_fwd_noalloc": (ctypes.c_int, [vp, vp, vp, i32, i32, i32, i32, ctypes.c_float,
                                                 lp, vp, vp, vp]),
     }

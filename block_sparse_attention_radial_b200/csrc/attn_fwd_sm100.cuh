@@ -106,6 +106,15 @@ __device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, const 
   }
 }
 
+// Whole-warp wait: a fast inline test, the bounded slow path only on a miss,
+// and a warp vote so every lane takes the same branch afterwards.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const WaitCtx &w,
+                                          int bar_id, uint32_t counter) {
+  bool r = mbar_try_wait(bar, parity);
+  if (!r) r = wait_bounded(bar, parity, w, bar_id, counter);
+  return __all_sync(0xffffffffu, r);
+}
+
 // Work item k of this CTA (static snake over the ordered item list); -1 when
 // the CTA has no item k.
 __device__ __forceinline__ int snake_item(int k, int total) {
@@ -137,6 +146,39 @@ __device__ __forceinline__ Item decode_item(int idx, const FwdParams &p) {
 
 __device__ __forceinline__ int key_block(const FwdParams &p, int e) {
   return min(max(p.col_idx[e], 0), p.nkb - 1);
+}
+
+#ifndef BSA_EMU_PAIRS
+#define BSA_EMU_PAIRS 0
+#endif
+// Of every 8 column pairs, this many take 2^x on the FMA pipe (exp2_poly2)
+// and the rest on the MUFU unit, so the two units share the softmax's
+// exponentials.
+constexpr int kEmuPairsPer8 = BSA_EMU_PAIRS;
+
+// p = 2^(s * sl2 + neg) for one row of BN scores: returns the fp32 row sum and
+// the values packed as bf16 pairs. EMU of every 8 pairs use the polynomial.
+template <int BN, int EMU>
+__device__ __forceinline__ float exp2_pack_row(const float (&s)[BN], float sl2, float neg,
+                                               uint32_t (&pk)[BN / 2]) {
+  const float2 neg2 = make_float2(neg, neg);
+  const float2 sl2v = make_float2(sl2, sl2);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int c = 0; c < BN / 2; ++c) {
+    const float2 x = ffma2(make_float2(s[2 * c], s[2 * c + 1]), sl2v, neg2);
+    float2 pp;
+    if ((c & 7) < EMU) {
+      pp = exp2_poly2(x);
+    } else {
+      pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+    }
+    acc[c & 3] = fadd2(acc[c & 3], pp);
+    pk[c] = pack_bf16x2(pp.x, pp.y);
+  }
+  const float2 a = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+  return a.x + a.y;
 }
 
 template <int D, int BN>
@@ -191,54 +233,67 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      wc.role = kRoleProducer;
+    // The whole warp walks the schedule; lane 0 issues the copies.
+    wc.role = kRoleProducer;
+    const bool leader = lane == 0;
+    if (leader) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      uint32_t ring = 0, qcount = 0;
-      bool skip_next_k = (p.fault_flags & 1) && blockIdx.x == 0;
-      int skipped_ring = -1;
-      bool ok = true;
-      auto load_kv = [&](const CUtensorMap *map, int kb, int z, bool is_k) -> bool {
-        const uint32_t s = ring % C::NS;
-        if (!wait_bounded(&bar_kv_empty[s], ((ring / C::NS) & 1u) ^ 1u, wc, kBarKvEmpty, ring))
-          return false;
-        if (is_k && skip_next_k) {  // test hook: leave this stage's barrier without an arrival
-          skip_next_k = false;
-          skipped_ring = static_cast<int>(ring);
-          ++ring;
-          return true;
-        }
-        mbar_arrive_expect_tx(&bar_kv_full[s], C::KV_BYTES);
-        uint8_t *dst = sKV + s * C::KV_BYTES;
-#pragma unroll
-        for (int cb = 0; cb < C::NCB; ++cb)
-          tma_load_3d(dst + cb * BN * 128, map, &bar_kv_full[s], cb * 64, kb * BN, z);
-        ++ring;
-        return true;
-      };
-      for (int k = 0; ok; ++k) {
-        const int idx = snake_item(k, p.total_items);
-        if (idx == -2) break;
-        if (idx < 0) continue;
-        const Item it = decode_item(idx, p);
-        if (it.len == 0) continue;
-        if (!wait_bounded(&bar_q_empty, (qcount & 1u) ^ 1u, wc, kBarQEmpty, qcount)) break;
+    }
+    uint32_t ring = 0, qcount = 0;
+    bool skip_next_k = (p.fault_flags & 1) && blockIdx.x == 0;
+    int skipped_ring = -1;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int idx = snake_item(k, p.total_items);
+      if (idx == -2) break;
+      if (idx < 0) continue;
+      const Item it = decode_item(idx, p);
+      if (it.len == 0) continue;
+      if (!(ok = warp_wait(&bar_q_empty, (qcount & 1u) ^ 1u, wc, kBarQEmpty, qcount))) break;
+      if (leader) {
         mbar_arrive_expect_tx(&bar_q_full, C::Q_BYTES);
 #pragma unroll
         for (int cb = 0; cb < C::NCB; ++cb)
           tma_load_3d(sQ + cb * C::BM * 128, &tm_q, &bar_q_full, cb * 64, it.qb * BN, it.bh);
-        ++qcount;
-        ok = load_kv(&tm_k, key_block(p, it.a), it.bh, true);
-        for (int j = 0; ok && j < it.len; ++j) {
-          if (j + 1 < it.len) ok = load_kv(&tm_k, key_block(p, it.a + j + 1), it.bh, true);
-          if (ok) ok = load_kv(&tm_v, key_block(p, it.a + j), it.bh, false);
-        }
       }
-      // Copies still in flight must land before the CTA exits: wait for the
-      // latest use of every stage and for the last Q tile (bounded, even when
-      // aborting).
+      ++qcount;
+      // K0, then (K(j+1), V(j)) for every j: the order the MMA warp consumes them
+      for (int t = 0; ok && t <= 2 * it.len; ++t) {
+        // t = 0: K0; then t = 2j+1: K(j+1), t = 2j+2: V(j)
+        bool is_k = true;
+        int j = 0;
+        if (t > 0) {
+          is_k = ((t - 1) & 1) == 0;
+          j = ((t - 1) >> 1) + (is_k ? 1 : 0);
+        }
+        if (is_k && j >= it.len) continue;  // no K beyond the row
+        const uint32_t s = ring % C::NS;
+        if (!(ok = warp_wait(&bar_kv_empty[s], ((ring / C::NS) & 1u) ^ 1u, wc, kBarKvEmpty, ring)))
+          break;
+        if (is_k && skip_next_k) {  // test hook: this stage's barrier never gets its arrival
+          skip_next_k = false;
+          skipped_ring = static_cast<int>(ring);
+          ++ring;
+          continue;
+        }
+        if (leader) {
+          const int kb = key_block(p, it.a + j);
+          mbar_arrive_expect_tx(&bar_kv_full[s], C::KV_BYTES);
+          uint8_t *dst = sKV + s * C::KV_BYTES;
+          const CUtensorMap *map = is_k ? &tm_k : &tm_v;
+#pragma unroll
+          for (int cb = 0; cb < C::NCB; ++cb)
+            tma_load_3d(dst + cb * BN * 128, map, &bar_kv_full[s], cb * 64, kb * BN, it.bh);
+        }
+        ++ring;
+      }
+    }
+    // Copies still in flight must land before the CTA exits: wait for the
+    // latest use of every stage and for the last Q tile (bounded, even when
+    // aborting).
+    if (leader) {
       WaitCtx drain{&abort_flag, p.wait_limit_ns, kRoleProducer};
       int zero = 0;
       drain.abort = &zero;
@@ -249,86 +304,99 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (qcount > 0) wait_bounded(&bar_q_full, (qcount - 1) & 1u, drain, kBarQFull, qcount);
     }
+    __syncwarp();
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      wc.role = kRoleMma;
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-      const uint32_t q_addr = smem_addr(sQ);
-      const uint32_t kv_addr = smem_addr(sKV);
-      uint32_t ring = 0, qcount = 0, g = 0, items_done = 0;
-      bool ok = true;
-      auto issue_qk = [&](uint32_t gg) -> bool {
-        const uint32_t s = ring % C::NS;
-        if (!wait_bounded(&bar_kv_full[s], (ring / C::NS) & 1u, wc, kBarKvFull, ring)) return false;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + C::S_COL + (gg & 1u) * 128u;
-        const uint32_t k_base = kv_addr + s * C::KV_BYTES;
+    // The whole warp walks the schedule and waits; lane 0 issues the MMAs.
+    // Descriptors are kept as 32-bit halves: the high half is the same for
+    // every operand (stride 1024 B, version 1, 128-byte swizzle) and the low
+    // half is the start address >> 4 plus the leading byte offset, so each
+    // k-step is one add on a precomputed base.
+    wc.role = kRoleMma;
+    const bool leader = lane == 0;
+    constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false);
+    constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+    constexpr uint32_t kHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+    constexpr uint32_t kLboK = 1u << 16;                          // 16 B (unused for K-major SW128)
+    constexpr uint32_t kLboV = static_cast<uint32_t>(BN * 128 / 16) << 16;  // 64-wide D chunks
+    const uint32_t q_lo = (smem_addr(sQ) >> 4) | kLboK;
+    const uint32_t kv_base = smem_addr(sKV) >> 4;
+    uint32_t ring = 0, qcount = 0, g = 0, items_done = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int idx = snake_item(k, p.total_items);
+      if (idx == -2) break;
+      if (idx < 0) continue;
+      const Item it = decode_item(idx, p);
+      if (it.len == 0) continue;
+      if (!(ok = warp_wait(&bar_q_full, qcount & 1u, wc, kBarQFull, qcount))) break;
+      tc_fence_after();
+      for (int t = 0; ok && t <= it.len; ++t) {
+        // step t: QK(t) if t < len, then PV(t-1) if t > 0
+        if (t < it.len) {
+          const uint32_t gg = g + t;
+          const uint32_t s = ring % C::NS;
+          if (!(ok = warp_wait(&bar_kv_full[s], (ring / C::NS) & 1u, wc, kBarKvFull, ring))) break;
+          tc_fence_after();
+          if (leader) {
+            const uint32_t d_tmem = tmem + C::S_COL + (gg & 1u) * 128u;
+            const uint32_t k_lo = (kv_base + s * (C::KV_BYTES >> 4)) | kLboK;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t cb = kk >> 2, within = (kk & 3) * 32;
-          const uint64_t a = smem_desc_sw128(q_addr + cb * (C::BM * 128) + within, 16, 1024);
-          const uint64_t b = smem_desc_sw128(k_base + cb * (BN * 128) + within, 16, 1024);
-          mma_ss(d_tmem, a, b, idesc_qk, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&bar_kv_empty[s]);
-        mma_commit(&bar_s_full[gg & 1u]);
-        ++ring;
-        return true;
-      };
-      for (int k = 0; ok; ++k) {
-        const int idx = snake_item(k, p.total_items);
-        if (idx == -2) break;
-        if (idx < 0) continue;
-        const Item it = decode_item(idx, p);
-        if (it.len == 0) continue;
-        if (!wait_bounded(&bar_q_full, qcount & 1u, wc, kBarQFull, qcount)) break;
-        tc_fence_after();
-        if (!(ok = issue_qk(g))) break;
-        if (it.len == 1) mma_commit(&bar_q_empty);
-        for (int j = 0; j < it.len; ++j) {
-          const uint32_t gg = g + j;
-          if (j + 1 < it.len) {
-            if (!(ok = issue_qk(gg + 1))) break;
-            if (j + 1 == it.len - 1) mma_commit(&bar_q_empty);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off_a = (kk >> 2) * (C::BM * 128 >> 4) + (kk & 3) * 2;
+              const uint32_t off_b = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
+              mma_ss_lh(d_tmem, q_lo + off_a, kHi, k_lo + off_b, kHi, idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&bar_kv_empty[s]);
+            mma_commit(&bar_s_full[gg & 1u]);
+            if (t == it.len - 1) mma_commit(&bar_q_empty);
           }
-          if (!(ok = wait_bounded(&bar_p_full[gg & 1u], (gg >> 1) & 1u, wc, kBarPFull, gg))) break;
+          __syncwarp();
+          ++ring;
+        }
+        if (t > 0) {
+          const int j = t - 1;
+          const uint32_t gg = g + j;
+          if (!(ok = warp_wait(&bar_p_full[gg & 1u], (gg >> 1) & 1u, wc, kBarPFull, gg))) break;
           tc_fence_after();
           if (j == 0 && items_done > 0) {
-            if (!(ok = wait_bounded(&bar_o_empty, (items_done - 1) & 1u, wc, kBarOEmpty,
-                                    items_done)))
+            if (!(ok = warp_wait(&bar_o_empty, (items_done - 1) & 1u, wc, kBarOEmpty, items_done)))
               break;
             tc_fence_after();
           }
           const uint32_t s = ring % C::NS;
-          if (!(ok = wait_bounded(&bar_kv_full[s], (ring / C::NS) & 1u, wc, kBarKvFull, ring)))
-            break;
+          if (!(ok = warp_wait(&bar_kv_full[s], (ring / C::NS) & 1u, wc, kBarKvFull, ring))) break;
           tc_fence_after();
-          const uint32_t p_tmem = tmem + C::S_COL + (gg & 1u) * 128u;
-          const uint32_t v_base = kv_addr + s * C::KV_BYTES;
+          if (leader) {
+            const uint32_t p_tmem = tmem + C::S_COL + (gg & 1u) * 128u;
+            const uint32_t v_lo = (kv_base + s * (C::KV_BYTES >> 4)) | kLboV;
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            // V tile: key rows of 128 bytes (64 head-dim values), 64-wide
-            // head-dim chunks BN*128 bytes apart (MN-major operand).
-            const uint64_t b = smem_desc_sw128(v_base + kk * (16 * 128), BN * 128, 1024);
-            mma_ts(tmem + C::O_COL, p_tmem + kk * 8, b, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BN / 16; ++kk) {
+              // V tile: key rows of 128 bytes (64 head-dim values), 64-wide
+              // head-dim chunks BN*128 bytes apart (MN-major operand)
+              mma_ts_lh(tmem + C::O_COL, p_tmem + kk * 8, v_lo + kk * (16 * 128 >> 4), kHi,
+                        idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&bar_kv_empty[s]);
+            mma_commit(&bar_o_done);
           }
-          mma_commit(&bar_kv_empty[s]);
-          mma_commit(&bar_o_done);
+          __syncwarp();
           ++ring;
         }
-        g += it.len;
-        ++qcount;
-        ++items_done;
       }
-      // Let every issued MMA finish before TMEM is released.
+      g += it.len;
+      ++qcount;
+      ++items_done;
+    }
+    // Let every issued MMA finish before TMEM is released.
+    if (leader) {
       mma_commit(&bar_final);
       WaitCtx drain{&abort_flag, p.wait_limit_ns, kRoleMma};
       int zero = 0;
       drain.abort = &zero;
       wait_bounded(&bar_final, 0, drain, kBarFinal, g);
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
     wc.role = kRoleSoftmax;
@@ -337,10 +405,6 @@ __global__ void __launch_bounds__(192, 1)
     const float sl2 = p.scale_log2;
     uint32_t g = 0;
     bool ok = true;
-    auto warp_wait = [&](uint64_t *bar, uint32_t parity, int bar_id, uint32_t counter) -> bool {
-      const bool r = wait_bounded(bar, parity, wc, bar_id, counter);
-      return __all_sync(0xffffffffu, r);
-    };
     for (int k = 0; ok; ++k) {
       const int idx = snake_item(k, p.total_items);
       if (idx == -2) break;
@@ -362,7 +426,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int j = 0; j < it.len; ++j) {
         const uint32_t gg = g + j;
         const uint32_t s_tmem = lane_tmem + C::S_COL + (gg & 1u) * 128u;
-        if (!(ok = warp_wait(&bar_s_full[gg & 1u], (gg >> 1) & 1u, kBarSFull, gg))) break;
+        if (!(ok = warp_wait(&bar_s_full[gg & 1u], (gg >> 1) & 1u, wc, kBarSFull, gg))) break;
         tc_fence_after();
         float s[BN];
         {
@@ -384,9 +448,17 @@ __global__ void __launch_bounds__(192, 1)
           for (int c = 0; c < BN; ++c)
             if (c >= valid) s[c] = -INFINITY;
         }
-        float mx = s[0];
+        // row max: eight independent chains of three-input max
+        float m8[8];
 #pragma unroll
-        for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+        for (int i = 0; i < 8; ++i) m8[i] = fmaxf(s[i], s[i + 8]);
+#pragma unroll
+        for (int c = 16; c < BN; c += 16) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m8[i] = fmax3(m8[i], s[c + i], s[c + 8 + i]);
+        }
+        const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                               fmaxf(m8[6], m8[7]));
         const float mblk = mx * sl2;
         float alpha = 1.f;
         bool rescale = false;
@@ -399,16 +471,9 @@ __global__ void __launch_bounds__(192, 1)
           m_ref = mblk;
           rescale = true;
         }
-        const float neg = -m_ref;
-        float sum = 0.f;
         uint32_t pk[BN / 2];
-#pragma unroll
-        for (int c = 0; c < BN / 2; ++c) {
-          const float p0 = ex2_approx(fmaf(s[2 * c], sl2, neg));
-          const float p1 = ex2_approx(fmaf(s[2 * c + 1], sl2, neg));
-          sum += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
-        }
+        const float sum = valid < BN ? exp2_pack_row<BN, 0>(s, sl2, -m_ref, pk)
+                                     : exp2_pack_row<BN, kEmuPairsPer8>(s, sl2, -m_ref, pk);
         l = l * alpha + sum;
         // P (bf16 pairs) overwrites the first BN/2 columns of this S buffer
 #pragma unroll
@@ -420,7 +485,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         // PV(gg-1) must be complete before O is touched and before P(gg) is
         // released; this also keeps the o_done phase tracking in lockstep.
-        if (gg >= 1 && !(ok = warp_wait(&bar_o_done, (gg - 1) & 1u, kBarODone, gg))) break;
+        if (gg >= 1 && !(ok = warp_wait(&bar_o_done, (gg - 1) & 1u, wc, kBarODone, gg))) break;
         if (__any_sync(0xffffffffu, rescale)) {
           tc_fence_after();
 #pragma unroll
@@ -440,7 +505,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (!ok) break;
       const uint32_t gl = g + it.len - 1;
-      if (!(ok = warp_wait(&bar_o_done, gl & 1u, kBarODone, gl))) break;
+      if (!(ok = warp_wait(&bar_o_done, gl & 1u, wc, kBarODone, gl))) break;
       tc_fence_after();
       const float inv_l = 1.f / l;
 #pragma unroll

@@ -195,6 +195,21 @@ int launch_ref(const RefParams &p, int batch, DeviceInfo *dev, int slot, cudaStr
 
 int slot_of(int D, int BN) { return (D == 128 ? 2 : 0) + (BN == 128 ? 1 : 0); }
 
+// Self-test of the two exp2 paths of the attention softmax against exp2f.
+__global__ void exp2_selftest_kernel(const float *x, float *y_poly, float *y_mufu,
+                                     float *y_ref, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (2 * i + 1 >= n) return;
+  const float2 v = make_float2(x[2 * i], x[2 * i + 1]);
+  const float2 p = exp2_poly2(v);
+  y_poly[2 * i] = p.x;
+  y_poly[2 * i + 1] = p.y;
+  y_mufu[2 * i] = ex2_approx(v.x);
+  y_mufu[2 * i + 1] = ex2_approx(v.y);
+  y_ref[2 * i] = exp2f(v.x);
+  y_ref[2 * i + 1] = exp2f(v.y);
+}
+
 }  // namespace
 }  // namespace bsa
 
@@ -403,6 +418,16 @@ const char *bsa_status_string(int status) {
 }
 
 const char *bsa_last_cuda_error(void) { return t_last_error; }
+
+int bsa_selftest_exp2(const float *x, float *y_poly, float *y_mufu, float *y_ref, int32_t n,
+                      bsa_stream_t stream_) {
+  if (!x || !y_poly || !y_mufu || !y_ref || n < 2 || (n & 1)) return BSA_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const int pairs = n / 2;
+  exp2_selftest_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(x, y_poly, y_mufu, y_ref, n);
+  BSA_CUDA(cudaGetLastError());
+  return BSA_OK;
+}
 
 int bsa_set_test_hooks(int64_t wait_limit_ns, int32_t fault_flags) {
   if (wait_limit_ns < 0) return BSA_ERR_INVALID_ARG;

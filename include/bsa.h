@@ -190,6 +190,16 @@ const char *bsa_last_cuda_error(void);
 int bsa_set_test_hooks(int64_t wait_limit_ns, int32_t fault_flags);
 
 /*
+ * Self-test of the exponentials the attention softmax uses. For each of the n
+ * (even) device floats x, writes 2^x from the FMA-pipe polynomial path
+ * (y_poly), from the hardware ex2.approx path (y_mufu) and from CUDA's exp2f
+ * (y_ref). Not part of the computation; used by the tests to bound the
+ * polynomial's error. Asynchronous.
+ */
+int bsa_selftest_exp2(const float *x, float *y_poly, float *y_mufu, float *y_ref, int32_t n,
+                      bsa_stream_t stream);
+
+/*
  * Allocation-free variant of bsa_attn_fwd. The pages have no counterpart: this
  * entry point exists for callers that cannot allocate device memory, such as a
  * plugin that its host framework hands only input and output buffers and no
