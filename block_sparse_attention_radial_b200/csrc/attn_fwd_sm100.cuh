@@ -17,7 +17,8 @@
 //   warp 5     MMA issuer (one thread): S = Q K^T into one of two TMEM S
 //              buffers, then O += P V with P read from TMEM.
 //
-// TMEM columns (512 allocated): S0 [0,128), S1 [128,256), O [256, 256+D).
+// TMEM columns (512 allocated): S0 [0,128), S1 [128,256), O [256, 256+D),
+// Q [384, 384+D/2) (copied from shared memory once per item).
 // Per block g (global counter) the MMA warp issues QK(g+1) before PV(g), so
 // the tensor core computes the next scores while the softmax warps work.
 //
@@ -54,15 +55,25 @@ struct FwdCfg {
   static constexpr int BM = 128;                 // tile rows (MMA M)
   static constexpr int NCB = D / 64;             // 128-byte column blocks per row
   static constexpr int Q_BYTES = BM * D * 2;
-  static constexpr int KV_BYTES = BN * D * 2;    // one K or V tile
-  static constexpr int NS_FIT = (kSmemLimit - 1024 - 512 - Q_BYTES) / KV_BYTES;
+  // A ring stage holds two consecutive key blocks of K (or of V), loaded by
+  // one TMA box of 2*BN rows: the TMA unit's cost is mostly per box, and
+  // radial lists are made of runs of consecutive blocks. A lone block still
+  // takes a whole stage (its second half is simply not used). Layout: D/64
+  // column blocks of [2*BN rows][128 B], block h of the pair at h*BN rows.
+  static constexpr int SEG = 2;                  // key blocks per stage
+  static constexpr int STAGE_ROWS = SEG * BN;
+  static constexpr int CB_BYTES = STAGE_ROWS * 128;  // one 64-column block of a stage
+  static constexpr int STAGE_BYTES = STAGE_ROWS * D * 2;
+  static constexpr int NS_FIT = (kSmemLimit - 1024 - 512 - Q_BYTES) / STAGE_BYTES;
   static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
   // At least 120 KB so that a second CTA never fits on an SM: every CTA then
   // owns its SM's tensor memory and the persistent grid covers all SMs.
-  static constexpr int DSMEM_USED = 1024 + Q_BYTES + NS * KV_BYTES;
+  static constexpr int DSMEM_USED = 1024 + Q_BYTES + NS * STAGE_BYTES;
   static constexpr int DSMEM = DSMEM_USED > 122880 ? DSMEM_USED : 122880;
   static constexpr uint32_t S_COL = 0;           // S buffer b at S_COL + 128 b
   static constexpr uint32_t O_COL = 256;
+  static constexpr uint32_t Q_COL = 384;         // Q as bf16 pairs, D/2 columns
+  static constexpr uint32_t P_COL = 448;         // P as bf16 pairs, BN/2 columns
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int THREADS = 192;
   static_assert(NS >= 2, "K/V ring needs at least two stages");
@@ -73,7 +84,7 @@ struct FwdCfg {
 enum : int { kRoleProducer = 1, kRoleMma = 2, kRoleSoftmax = 3 };
 enum : int {
   kBarKvFull = 1, kBarKvEmpty, kBarQFull, kBarQEmpty, kBarSFull, kBarPFull, kBarODone,
-  kBarOEmpty, kBarFinal
+  kBarOEmpty, kBarFinal, kBarSFree
 };
 
 struct WaitCtx {
@@ -148,6 +159,53 @@ __device__ __forceinline__ int key_block(const FwdParams &p, int e) {
   return min(max(p.col_idx[e], 0), p.nkb - 1);
 }
 
+// A warp's register cache of one row's key blocks: lane i holds entry
+// base + i, and the next 32 entries are already in flight, so reading the
+// list costs a shuffle instead of a dependent global load on the critical
+// path. Lookups must be warp-uniform and non-decreasing in b.
+struct ListCache {
+  int base, cur, nxt;
+  __device__ __forceinline__ static int load(const FwdParams &p, int a, int len, int chunk) {
+    const int i = chunk + static_cast<int>(threadIdx.x & 31);
+    return i < len ? min(max(__ldg(p.col_idx + a + i), 0), p.nkb - 1) : 0;
+  }
+  __device__ __forceinline__ void reset(const FwdParams &p, int a, int len) {
+    base = 0;
+    cur = load(p, a, len, 0);
+    nxt = load(p, a, len, 32);
+  }
+  __device__ __forceinline__ int get(const FwdParams &p, int a, int len, int b) {
+    while (b >= base + 32) {
+      base += 32;
+      cur = nxt;
+      nxt = load(p, a, len, base + 32);
+    }
+    return __shfl_sync(0xffffffffu, cur, b - base);
+  }
+};
+
+// Walks a row's key blocks as segments of one or two consecutive blocks (the
+// unit one ring stage holds). The producer and the MMA warp run identical
+// walkers, so they agree on which ring position holds which block.
+struct SegWalker {
+  int first = 0, count = 0, kb = 0;
+  ListCache cache;
+  __device__ __forceinline__ void reset(const FwdParams &p, int a, int len) {
+    first = 0;
+    count = 0;
+    cache.reset(p, a, len);
+  }
+  // True when block b opens a new segment (b is past the current one).
+  __device__ __forceinline__ bool advance(const FwdParams &p, int a, int len, int b) {
+    if (b < first + count) return false;
+    first = b;
+    kb = cache.get(p, a, len, b);
+    const int next = b + 1 < len ? cache.get(p, a, len, b + 1) : -1;
+    count = next == kb + 1 ? 2 : 1;
+    return true;
+  }
+};
+
 #ifndef BSA_EMU_PAIRS
 #define BSA_EMU_PAIRS 0
 #endif
@@ -190,8 +248,9 @@ __global__ void __launch_bounds__(192, 1)
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t bar_kv_full[C::NS];
   __shared__ __align__(8) uint64_t bar_kv_empty[C::NS];
-  __shared__ __align__(8) uint64_t bar_q_full, bar_q_empty, bar_o_done, bar_o_empty, bar_final;
-  __shared__ __align__(8) uint64_t bar_s_full[2], bar_p_full[2];
+  __shared__ __align__(8) uint64_t bar_q_full, bar_q_empty, bar_o_empty, bar_final;
+  __shared__ __align__(8) uint64_t bar_o_done[2];
+  __shared__ __align__(8) uint64_t bar_s_full[2], bar_s_free[2], bar_p_full;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -210,13 +269,14 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(&bar_q_full, 1);
     mbar_init(&bar_q_empty, 1);
-    mbar_init(&bar_o_done, 1);
     mbar_init(&bar_o_empty, 128);
     mbar_init(&bar_final, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar_s_full[b], 1);
-      mbar_init(&bar_p_full[b], 128);
+      mbar_init(&bar_s_free[b], 128);
+      mbar_init(&bar_o_done[b], 1);
     }
+    mbar_init(&bar_p_full, 128);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -254,40 +314,40 @@ __global__ void __launch_bounds__(192, 1)
       if (!(ok = warp_wait(&bar_q_empty, (qcount & 1u) ^ 1u, wc, kBarQEmpty, qcount))) break;
       if (leader) {
         mbar_arrive_expect_tx(&bar_q_full, C::Q_BYTES);
-#pragma unroll
-        for (int cb = 0; cb < C::NCB; ++cb)
-          tma_load_3d(sQ + cb * C::BM * 128, &tm_q, &bar_q_full, cb * 64, it.qb * BN, it.bh);
+        tma_load_4d(sQ, &tm_q, &bar_q_full, 0, it.qb * BN, 0, it.bh);
       }
       ++qcount;
-      // K0, then (K(j+1), V(j)) for every j: the order the MMA warp consumes them
-      for (int t = 0; ok && t <= 2 * it.len; ++t) {
-        // t = 0: K0; then t = 2j+1: K(j+1), t = 2j+2: V(j)
-        bool is_k = true;
-        int j = 0;
-        if (t > 0) {
-          is_k = ((t - 1) & 1) == 0;
-          j = ((t - 1) >> 1) + (is_k ? 1 : 0);
-        }
-        if (is_k && j >= it.len) continue;  // no K beyond the row
-        const uint32_t s = ring % C::NS;
-        if (!(ok = warp_wait(&bar_kv_empty[s], ((ring / C::NS) & 1u) ^ 1u, wc, kBarKvEmpty, ring)))
-          break;
-        if (is_k && skip_next_k) {  // test hook: this stage's barrier never gets its arrival
-          skip_next_k = false;
-          skipped_ring = static_cast<int>(ring);
-          ++ring;
-          continue;
-        }
-        if (leader) {
-          const int kb = key_block(p, it.a + j);
-          mbar_arrive_expect_tx(&bar_kv_full[s], C::KV_BYTES);
-          uint8_t *dst = sKV + s * C::KV_BYTES;
-          const CUtensorMap *map = is_k ? &tm_k : &tm_v;
+      // Walk the blocks as the MMA warp does (step j: QK(j+1), then PV(j),
+      // after QK(0)) and load each K or V segment at its first use, so the
+      // ring fills in exactly the order the MMA warp consumes it.
+      SegWalker ks, vs;
+      ks.reset(p, it.a, it.len);
+      vs.reset(p, it.a, it.len);
+      for (int t = -1; ok && t < it.len; ++t) {
 #pragma unroll
-          for (int cb = 0; cb < C::NCB; ++cb)
-            tma_load_3d(dst + cb * BN * 128, map, &bar_kv_full[s], cb * 64, kb * BN, it.bh);
+        for (int side = 0; side < 2; ++side) {
+          const bool is_k = side == 0;
+          const int b = is_k ? t + 1 : t;
+          if (is_k ? b >= it.len : t < 0) continue;
+          SegWalker &w = is_k ? ks : vs;
+          if (!w.advance(p, it.a, it.len, b)) continue;
+          const uint32_t s = ring % C::NS;
+          if (!(ok = warp_wait(&bar_kv_empty[s], ((ring / C::NS) & 1u) ^ 1u, wc, kBarKvEmpty,
+                               ring)))
+            break;
+          if (is_k && skip_next_k) {  // test hook: this stage's barrier never gets its arrival
+            skip_next_k = false;
+            skipped_ring = static_cast<int>(ring);
+            ++ring;
+            continue;
+          }
+          if (leader) {
+            mbar_arrive_expect_tx(&bar_kv_full[s], C::STAGE_BYTES);
+            tma_load_4d(sKV + s * C::STAGE_BYTES, is_k ? &tm_k : &tm_v, &bar_kv_full[s], 0,
+                        w.kb * BN, 0, it.bh);
+          }
+          ++ring;
         }
-        ++ring;
       }
     }
     // Copies still in flight must land before the CTA exits: wait for the
@@ -318,7 +378,7 @@ __global__ void __launch_bounds__(192, 1)
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
     constexpr uint32_t kHi = (1024u >> 4) | (1u << 14) | (2u << 29);
     constexpr uint32_t kLboK = 1u << 16;                          // 16 B (unused for K-major SW128)
-    constexpr uint32_t kLboV = static_cast<uint32_t>(BN * 128 / 16) << 16;  // 64-wide D chunks
+    constexpr uint32_t kLboV = static_cast<uint32_t>(C::CB_BYTES / 16) << 16;  // 64-wide D chunks
     const uint32_t q_lo = (smem_addr(sQ) >> 4) | kLboK;
     const uint32_t kv_base = smem_addr(sKV) >> 4;
     uint32_t ring = 0, qcount = 0, g = 0, items_done = 0;
@@ -331,57 +391,86 @@ __global__ void __launch_bounds__(192, 1)
       if (it.len == 0) continue;
       if (!(ok = warp_wait(&bar_q_full, qcount & 1u, wc, kBarQFull, qcount))) break;
       tc_fence_after();
-      for (int t = 0; ok && t <= it.len; ++t) {
-        // step t: QK(t) if t < len, then PV(t-1) if t > 0
-        if (t < it.len) {
-          const uint32_t gg = g + t;
-          const uint32_t s = ring % C::NS;
-          if (!(ok = warp_wait(&bar_kv_full[s], (ring / C::NS) & 1u, wc, kBarKvFull, ring))) break;
-          tc_fence_after();
+      if (leader) {
+        // Q moves into TMEM once per item (after the previous item's MMAs, in
+        // issue order), so the QK MMAs read only K from shared memory; the
+        // shared Q buffer is free as soon as the copies complete.
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off_a = (kk >> 2) * (C::BM * 128 >> 4) + (kk & 3) * 2;
+          tmem_cp_128x256b(tmem + C::Q_COL + kk * 8, q_lo + off_a, kHi);
+        }
+        mma_commit(&bar_q_empty);
+      }
+      SegWalker ks, vs;
+      ks.reset(p, it.a, it.len);
+      vs.reset(p, it.a, it.len);
+      uint32_t kstage = 0, vstage = 0;
+      // Step t (from -1): QK(t+1) as soon as its S buffer has been read by
+      // the softmax, then PV(t) once P(t) is ready. QK for the next block
+      // thus never waits on a PV, and the softmax finds S ready.
+      for (int t = -1; ok && t < it.len; ++t) {
+        const int bq = t + 1;
+        if (bq < it.len) {
+          const uint32_t gq = g + bq;
+          if (gq >= 2) {  // S buffer of block gq-2 must have been loaded by the softmax
+            if (!(ok = warp_wait(&bar_s_free[gq & 1u], ((gq - 2) >> 1) & 1u, wc, kBarSFree, gq)))
+              break;
+            tc_fence_after();
+          }
+          if (ks.advance(p, it.a, it.len, bq)) {
+            kstage = ring % C::NS;
+            if (!(ok = warp_wait(&bar_kv_full[kstage], (ring / C::NS) & 1u, wc, kBarKvFull, ring)))
+              break;
+            tc_fence_after();
+            ++ring;
+          }
           if (leader) {
-            const uint32_t d_tmem = tmem + C::S_COL + (gg & 1u) * 128u;
-            const uint32_t k_lo = (kv_base + s * (C::KV_BYTES >> 4)) | kLboK;
+            const uint32_t d_tmem = tmem + C::S_COL + (gq & 1u) * 128u;
+            const uint32_t k_lo = (kv_base + kstage * (C::STAGE_BYTES >> 4) +
+                                   (bq - ks.first) * (BN * 128 >> 4)) | kLboK;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off_a = (kk >> 2) * (C::BM * 128 >> 4) + (kk & 3) * 2;
-              const uint32_t off_b = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
-              mma_ss_lh(d_tmem, q_lo + off_a, kHi, k_lo + off_b, kHi, idesc_qk, kk > 0 ? 1u : 0u);
+              const uint32_t off_b = (kk >> 2) * (C::CB_BYTES >> 4) + (kk & 3) * 2;
+              mma_ts_lh(d_tmem, tmem + C::Q_COL + kk * 8, k_lo + off_b, kHi, idesc_qk,
+                        kk > 0 ? 1u : 0u);
             }
-            mma_commit(&bar_kv_empty[s]);
-            mma_commit(&bar_s_full[gg & 1u]);
-            if (t == it.len - 1) mma_commit(&bar_q_empty);
+            if (bq == ks.first + ks.count - 1) mma_commit(&bar_kv_empty[kstage]);
+            mma_commit(&bar_s_full[gq & 1u]);
           }
           __syncwarp();
-          ++ring;
         }
-        if (t > 0) {
-          const int j = t - 1;
+        if (t >= 0) {
+          const int j = t;
           const uint32_t gg = g + j;
-          if (!(ok = warp_wait(&bar_p_full[gg & 1u], (gg >> 1) & 1u, wc, kBarPFull, gg))) break;
+          if (!(ok = warp_wait(&bar_p_full, gg & 1u, wc, kBarPFull, gg))) break;
           tc_fence_after();
           if (j == 0 && items_done > 0) {
             if (!(ok = warp_wait(&bar_o_empty, (items_done - 1) & 1u, wc, kBarOEmpty, items_done)))
               break;
             tc_fence_after();
           }
-          const uint32_t s = ring % C::NS;
-          if (!(ok = warp_wait(&bar_kv_full[s], (ring / C::NS) & 1u, wc, kBarKvFull, ring))) break;
-          tc_fence_after();
+          if (vs.advance(p, it.a, it.len, j)) {
+            vstage = ring % C::NS;
+            if (!(ok = warp_wait(&bar_kv_full[vstage], (ring / C::NS) & 1u, wc, kBarKvFull, ring)))
+              break;
+            tc_fence_after();
+            ++ring;
+          }
           if (leader) {
-            const uint32_t p_tmem = tmem + C::S_COL + (gg & 1u) * 128u;
-            const uint32_t v_lo = (kv_base + s * (C::KV_BYTES >> 4)) | kLboV;
+            const uint32_t v_lo = (kv_base + vstage * (C::STAGE_BYTES >> 4) +
+                                   (j - vs.first) * (BN * 128 >> 4)) | kLboV;
 #pragma unroll
             for (int kk = 0; kk < BN / 16; ++kk) {
-              // V tile: key rows of 128 bytes (64 head-dim values), 64-wide
-              // head-dim chunks BN*128 bytes apart (MN-major operand)
-              mma_ts_lh(tmem + C::O_COL, p_tmem + kk * 8, v_lo + kk * (16 * 128 >> 4), kHi,
-                        idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+              // V rows of 128 bytes (64 head-dim values); 64-wide head-dim
+              // chunks one stage column block apart (MN-major operand)
+              mma_ts_lh(tmem + C::O_COL, tmem + C::P_COL + kk * 8, v_lo + kk * (16 * 128 >> 4),
+                        kHi, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
             }
-            mma_commit(&bar_kv_empty[s]);
-            mma_commit(&bar_o_done);
+            if (j == vs.first + vs.count - 1) mma_commit(&bar_kv_empty[vstage]);
+            mma_commit(&bar_o_done[gg & 1u]);
           }
           __syncwarp();
-          ++ring;
         }
       }
       g += it.len;
@@ -423,6 +512,8 @@ __global__ void __launch_bounds__(192, 1)
         continue;
       }
       float m_ref = 0.f, l = 0.f;
+      ListCache lc;
+      lc.reset(p, it.a, it.len);
       for (int j = 0; j < it.len; ++j) {
         const uint32_t gg = g + j;
         const uint32_t s_tmem = lane_tmem + C::S_COL + (gg & 1u) * 128u;
@@ -441,7 +532,10 @@ __global__ void __launch_bounds__(192, 1)
             for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(sr[c][i]);
           }
         }
-        const int kb = key_block(p, it.a + j);
+        // S is in registers: its TMEM buffer may take QK(gg+2) right away.
+        tc_fence_before();
+        mbar_arrive(&bar_s_free[gg & 1u]);
+        const int kb = lc.get(p, it.a, it.len, j);
         const int valid = p.n - kb * BN;
         if (valid < BN) {
 #pragma unroll
@@ -475,19 +569,18 @@ __global__ void __launch_bounds__(192, 1)
         const float sum = valid < BN ? exp2_pack_row<BN, 0>(s, sl2, -m_ref, pk)
                                      : exp2_pack_row<BN, kEmuPairsPer8>(s, sl2, -m_ref, pk);
         l = l * alpha + sum;
-        // P (bf16 pairs) overwrites the first BN/2 columns of this S buffer
-#pragma unroll
-        for (int c = 0; c < BN / 64; ++c) {
-          uint32_t r[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = pk[c * 32 + i];
-          tmem_st32(s_tmem + c * 32, r);
-        }
-        // PV(gg-1) must be complete before O is touched and before P(gg) is
-        // released; this also keeps the o_done phase tracking in lockstep.
-        if (gg >= 1 && !(ok = warp_wait(&bar_o_done, (gg - 1) & 1u, wc, kBarODone, gg))) break;
-        if (__any_sync(0xffffffffu, rescale)) {
+        // PV(gg-1) must have finished with the P buffer (and with O, which a
+        // rescale touches) before P(gg) is written. Waiting for it at every
+        // block keeps each o_done wait phase-exact: PV(gg-2) was waited for
+        // at the previous block. PV(gg-1) was issued a whole softmax earlier,
+        // so this rarely stalls.
+        if (gg >= 1) {
+          if (!(ok = warp_wait(&bar_o_done[(gg - 1) & 1u], ((gg - 1) >> 1) & 1u, wc, kBarODone,
+                               gg)))
+            break;
           tc_fence_after();
+        }
+        if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t r[32];
@@ -499,13 +592,21 @@ __global__ void __launch_bounds__(192, 1)
             tmem_st32(lane_tmem + C::O_COL + c * 32, r);
           }
         }
+        // P (bf16 pairs) into its own TMEM columns
+#pragma unroll
+        for (int c = 0; c < BN / 64; ++c) {
+          uint32_t r[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = pk[c * 32 + i];
+          tmem_st32(lane_tmem + C::P_COL + c * 32, r);
+        }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bar_p_full[gg & 1u]);
+        mbar_arrive(&bar_p_full);
       }
       if (!ok) break;
       const uint32_t gl = g + it.len - 1;
-      if (!(ok = warp_wait(&bar_o_done, gl & 1u, wc, kBarODone, gl))) break;
+      if (!(ok = warp_wait(&bar_o_done[gl & 1u], (gl >> 1) & 1u, wc, kBarODone, gl))) break;
       tc_fence_after();
       const float inv_l = 1.f / l;
 #pragma unroll

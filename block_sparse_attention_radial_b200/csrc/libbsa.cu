@@ -87,22 +87,25 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [batch*heads, n, D] bf16 viewed as a 3-D tensor; box of 64 x rows x 1 with
-// 128-byte swizzling (one 128-byte row segment per box row). Rows past n read
-// as zeros.
+// [batch*heads, n, D] bf16 viewed as a 4-D tensor {64 columns, n rows,
+// D/64 column halves, batch*heads}: one box {64, rows, D/64, 1} brings a whole
+// rows x D tile with 128-byte swizzling, laid out in shared memory as D/64
+// consecutive [rows][64] blocks (the K-major layout the MMA descriptors use).
+// One large box per tile instead of one per 64 columns: the TMA unit's cost is
+// mostly per box. Rows past n read as zeros.
 int make_map(CUtensorMap *map, const void *ptr, int bh, int n, int D, int rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) {
     std::snprintf(t_last_error, sizeof(t_last_error), "cuTensorMapEncodeTiled not available");
     return BSA_ERR_CUDA;
   }
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(n),
+  cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(n), static_cast<cuuint64_t>(D / 64),
                         static_cast<cuuint64_t>(bh)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, 128,
                            static_cast<cuuint64_t>(n) * static_cast<cuuint64_t>(D) * 2};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims,
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(rows), static_cast<cuuint32_t>(D / 64), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims,
                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
@@ -158,8 +161,8 @@ int launch_fwd(const void *q, const void *k, const void *v, int32_t bh, int32_t 
   CUtensorMap tq, tk, tv;
   int st;
   if ((st = make_map(&tq, q, bh, n, D, C::BM)) != BSA_OK) return st;
-  if ((st = make_map(&tk, k, bh, n, D, BN)) != BSA_OK) return st;
-  if ((st = make_map(&tv, v, bh, n, D, BN)) != BSA_OK) return st;
+  if ((st = make_map(&tk, k, bh, n, D, C::STAGE_ROWS)) != BSA_OK) return st;
+  if ((st = make_map(&tv, v, bh, n, D, C::STAGE_ROWS)) != BSA_OK) return st;
   {
     std::lock_guard<std::mutex> lk(g_dev_mu);
     if (!dev->attrs_set[slot]) {
