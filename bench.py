@@ -32,7 +32,8 @@ if ROOT not in sys.path:
 
 METRIC = "block-sparse attn fwd ms & effective TFLOP/s vs bf16 peak at 32k–120k tokens"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ("block_sparse_attention_radial_b200/csrc/attn_fwd_sm100.cuh",
+KERNEL_SOURCES = ("block_sparse_attention_radial_b200/csrc/attn_fwd_pair_sm100.cuh",
+                  "block_sparse_attention_radial_b200/csrc/attn_fwd_sm100.cuh",
                   "block_sparse_attention_radial_b200/csrc/ptx_sm100.cuh")
 
 
@@ -386,7 +387,7 @@ def run_ours(args, world, rank, local):
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_kind": f"{peak_kind} bf16 burst",
                          "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
-                         "kernel": "attn_fwd_sm100_kernel<128,128> (+ work-order prepass)",
+                         "kernel": "attn_fwd_pair_sm100_kernel<128> (+ work-order prepass)",
                          "kernel_ms": kernel_ms, "flops_per_launch": flops},
             "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

@@ -1,0 +1,520 @@
+// Block-sparse attention forward for sm_100a, two query tiles per CTA.
+//
+// A work item is a pair of adjacent query blocks (2p, 2p+1) of one
+// (batch, head). The CTA walks the union of the two rows' key-block lists:
+// each K and V tile is loaded once and used by both tiles when both list it,
+// by one tile otherwise, so the L2 -> shared-memory stream per unit of tensor
+// work drops to (union length) / (sum of the two lengths) of a one-tile
+// kernel. Each tile runs its own softmax warpgroup, and while one tile's
+// softmax works the tensor core runs the other tile's MMAs.
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax of tile A (thread = row = TMEM lane)
+//   warps 4-7  softmax of tile B
+//   warp 8     producer: Q_A, Q_B, then the union's K and V tiles (TMA)
+//   warp 9     MMA issuer
+//
+// TMEM: S_A [0,128), S_B [128,256), O_A [256, 256+D), O_B [256+D, 256+2D).
+// P of a tile overwrites the first 64 columns of its S buffer.
+//
+// MMA schedule, per union step j with flags a (tile A lists block j) and b:
+//   PV_A(j-1) if A listed j-1;  QK_A(j) if a;  PV_B(j-1) if B listed j-1;
+//   QK_B(j) if b;  then K(j) and V(j-1) are released.
+// PV_X(prev) is always issued before QK_X(next), so when S_X is complete the
+// previous PV_X is complete too: the softmax can rescale O_X without waiting.
+#pragma once
+
+#include <climits>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "attn_fwd_sm100.cuh"
+
+namespace bsa {
+
+template <int D>
+struct PairCfg {
+  static constexpr int BN = 128;                 // block = tile rows = MMA M and N
+  static constexpr int Q_BYTES = BN * D * 2;     // one tile's Q
+  static constexpr int TILE_BYTES = BN * D * 2;  // one K or V tile (one 4-D TMA box)
+  static constexpr int NS_FIT = (kSmemLimit - 1024 - 512 - 2 * Q_BYTES) / TILE_BYTES;
+  static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
+  static constexpr int DSMEM_USED = 1024 + 2 * Q_BYTES + NS * TILE_BYTES;
+  static constexpr int DSMEM = DSMEM_USED > 122880 ? DSMEM_USED : 122880;
+  static constexpr uint32_t S_COL = 0;           // S of tile t at S_COL + 128 t
+  static constexpr uint32_t O_COL = 256;         // O of tile t at O_COL + D t
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int THREADS = 320;
+  static_assert(NS >= 3, "K/V ring needs at least three stages");
+};
+
+// Key blocks of one query-block pair, walked as the sorted union of the two
+// rows. Warp-uniform; the producer, the MMA warp and nothing else use it.
+struct UnionWalker {
+  ListCache ca, cb;
+  int a0, lenA, b0, lenB, ia, ib;
+  __device__ __forceinline__ void reset(const FwdParams &p, int a0_, int lenA_, int b0_,
+                                        int lenB_) {
+    a0 = a0_;
+    lenA = lenA_;
+    b0 = b0_;
+    lenB = lenB_;
+    ia = 0;
+    ib = 0;
+    ca.reset(p, a0, lenA);
+    cb.reset(p, b0, lenB);
+  }
+  // Next union block: false when both rows are exhausted.
+  __device__ __forceinline__ bool next(const FwdParams &p, int &kb, bool &inA, bool &inB) {
+    if (ia >= lenA && ib >= lenB) return false;
+    const int va = ia < lenA ? ca.get(p, a0, lenA, ia) : INT_MAX;
+    const int vb = ib < lenB ? cb.get(p, b0, lenB, ib) : INT_MAX;
+    kb = min(va, vb);
+    inA = va == kb;
+    inB = vb == kb;
+    ia += inA ? 1 : 0;
+    ib += inB ? 1 : 0;
+    return true;
+  }
+};
+
+struct PairItem {
+  int bh, qa, a0, lenA, b0, lenB;  // tile B absent (lenB = 0) past the last block
+};
+
+__device__ __forceinline__ PairItem decode_pair(int idx, const FwdParams &p, int npairs) {
+  PairItem it;
+  it.bh = idx / npairs;
+  const int rank = idx - it.bh * npairs;
+  const int list = p.num_lists > 1 ? (it.bh % p.heads) : 0;
+  const long long lbase = static_cast<long long>(list) * p.nqb;
+  const int pr = min(max(p.order[static_cast<long long>(list) * npairs + rank], 0), npairs - 1);
+  it.qa = 2 * pr;
+  const int a = min(max(p.row_ptr[lbase + it.qa], 0), p.nnz);
+  const int ae = min(max(p.row_ptr[lbase + it.qa + 1], 0), p.nnz);
+  it.a0 = a;
+  it.lenA = max(ae - a, 0);
+  if (it.qa + 1 < p.nqb) {
+    const int b = min(max(p.row_ptr[lbase + it.qa + 1], 0), p.nnz);
+    const int be = min(max(p.row_ptr[lbase + it.qa + 2], 0), p.nnz);
+    it.b0 = b;
+    it.lenB = max(be - b, 0);
+  } else {
+    it.b0 = 0;
+    it.lenB = 0;
+  }
+  return it;
+}
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    attn_fwd_pair_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                               const __grid_constant__ CUtensorMap tm_k,
+                               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using C = PairCfg<D>;
+  constexpr int BN = C::BN;
+  extern __shared__ uint8_t dsmem[];
+  __shared__ __align__(8) uint64_t bar_kv_full[C::NS];
+  __shared__ __align__(8) uint64_t bar_kv_empty[C::NS];
+  __shared__ __align__(8) uint64_t bar_q_full, bar_q_empty, bar_final;
+  __shared__ __align__(8) uint64_t bar_s_full[2], bar_p_full[2], bar_o_final[2], bar_o_empty[2];
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const uint32_t raw = smem_addr(dsmem);
+  uint8_t *base = dsmem + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t *sQ = base;                      // Q_A, then Q_B at + Q_BYTES
+  uint8_t *sKV = base + 2 * C::Q_BYTES;
+  const int npairs = (p.nqb + 1) / 2;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(&bar_kv_full[s], 1);
+      mbar_init(&bar_kv_empty[s], 1);
+    }
+    mbar_init(&bar_q_full, 1);
+    mbar_init(&bar_q_empty, 1);
+    mbar_init(&bar_final, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bar_s_full[t], 1);
+      mbar_init(&bar_p_full[t], 128);
+      mbar_init(&bar_o_final[t], 1);
+      mbar_init(&bar_o_empty[t], 128);
+    }
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  WaitCtx wc{&abort_flag, p.wait_limit_ns, 0};
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    wc.role = kRoleProducer;
+    const bool leader = lane == 0;
+    if (leader) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+    uint32_t ring = 0, qcount = 0;
+    bool skip_next_k = (p.fault_flags & 1) && blockIdx.x == 0;
+    int skipped_ring = -1;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int idx = snake_item(k, p.total_items);
+      if (idx == -2) break;
+      if (idx < 0) continue;
+      const PairItem it = decode_pair(idx, p, npairs);
+      if (it.lenA == 0 && it.lenB == 0) continue;
+      if (!(ok = warp_wait(&bar_q_empty, (qcount & 1u) ^ 1u, wc, kBarQEmpty, qcount))) break;
+      if (leader) {
+        mbar_arrive_expect_tx(&bar_q_full, 2 * C::Q_BYTES);
+        tma_load_4d(sQ, &tm_q, &bar_q_full, 0, it.qa * BN, 0, it.bh);
+        tma_load_4d(sQ + C::Q_BYTES, &tm_q, &bar_q_full, 0, (it.qa + 1) * BN, 0, it.bh);
+      }
+      ++qcount;
+      // Same walk and same first-use order as the MMA warp: at step j the
+      // MMA warp needs V(j-1) first when tile A listed j-1 or A skips j, and
+      // K(j) first otherwise.
+      UnionWalker uw;
+      uw.reset(p, it.a0, it.lenA, it.b0, it.lenB);
+      bool pa = false, pb = false;
+      int prev_kb = 0;
+      for (int j = 0; ok; ++j) {
+        int kb = 0;
+        bool a = false, b = false;
+        const bool more = uw.next(p, kb, a, b);
+        const bool need_v = pa || pb;
+        if (!more && !need_v) break;
+        const bool v_first = pa || !a;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const bool is_v = (e == 0) == v_first;
+          if (is_v ? !need_v : !more) continue;
+          const uint32_t s = ring % C::NS;
+          if (!(ok = warp_wait(&bar_kv_empty[s], ((ring / C::NS) & 1u) ^ 1u, wc, kBarKvEmpty,
+                               ring)))
+            break;
+          if (!is_v && skip_next_k) {  // test hook: this stage's barrier never gets its arrival
+            skip_next_k = false;
+            skipped_ring = static_cast<int>(ring);
+            ++ring;
+            continue;
+          }
+          if (leader) {
+            mbar_arrive_expect_tx(&bar_kv_full[s], C::TILE_BYTES);
+            tma_load_4d(sKV + s * C::TILE_BYTES, is_v ? &tm_v : &tm_k, &bar_kv_full[s], 0,
+                        (is_v ? prev_kb : kb) * BN, 0, it.bh);
+          }
+          ++ring;
+        }
+        pa = a;
+        pb = b;
+        prev_kb = kb;
+        if (!more) break;
+      }
+    }
+    if (leader) {
+      WaitCtx drain{&abort_flag, p.wait_limit_ns, kRoleProducer};
+      int zero = 0;
+      drain.abort = &zero;
+      const uint32_t first = ring > C::NS ? ring - C::NS : 0;
+      for (uint32_t r = first; r < ring; ++r) {
+        if (static_cast<int>(r) == skipped_ring) continue;
+        wait_bounded(&bar_kv_full[r % C::NS], (r / C::NS) & 1u, drain, kBarKvFull, r);
+      }
+      if (qcount > 0) wait_bounded(&bar_q_full, (qcount - 1) & 1u, drain, kBarQFull, qcount);
+    }
+    __syncwarp();
+  }
+  else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    // Whole warp walks; lane 0 issues. Descriptors as 32-bit halves (see the
+    // one-tile kernel): shared high half, low half = address >> 4 | LBO.
+    wc.role = kRoleMma;
+    const bool leader = lane == 0;
+    constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false);
+    constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+    constexpr uint32_t kHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+    constexpr uint32_t kLboK = 1u << 16;
+    constexpr uint32_t kLboV = static_cast<uint32_t>(BN * 128 / 16) << 16;  // 64-wide D chunks
+    const uint32_t q_lo0 = (smem_addr(sQ) >> 4) | kLboK;
+    const uint32_t kv_base = smem_addr(sKV) >> 4;
+    uint32_t ring = 0, qcount = 0;
+    uint32_t pcnt[2] = {0u, 0u};      // p_full phases consumed, per tile
+    uint32_t items_t[2] = {0u, 0u};   // items in which the tile had blocks
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int idx = snake_item(k, p.total_items);
+      if (idx == -2) break;
+      if (idx < 0) continue;
+      const PairItem it = decode_pair(idx, p, npairs);
+      if (it.lenA == 0 && it.lenB == 0) continue;
+      if (!(ok = warp_wait(&bar_q_full, qcount & 1u, wc, kBarQFull, qcount))) break;
+      tc_fence_after();
+      const int len_t[2] = {it.lenA, it.lenB};
+      UnionWalker uw;
+      uw.reset(p, it.a0, it.lenA, it.b0, it.lenB);
+      bool pend[2] = {false, false}, first_pv[2] = {true, true};
+      bool q_released = false;
+      for (int j = 0; ok; ++j) {
+        int kb = 0;
+        bool in[2] = {false, false};
+        const bool more = uw.next(p, kb, in[0], in[1]);
+        if (!more && !pend[0] && !pend[1]) break;
+        if (!more && !q_released) {  // no QK left in this item: the Q buffers may refill
+          if (leader) mma_commit(&bar_q_empty);
+          q_released = true;
+        }
+        bool have_k = false, have_v = false;
+        uint32_t kstage = 0, vstage = 0;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (!ok) break;
+          if (pend[t]) {
+            if (!(ok = warp_wait(&bar_p_full[t], pcnt[t] & 1u, wc, kBarPFull, pcnt[t]))) break;
+            ++pcnt[t];
+            tc_fence_after();
+            if (first_pv[t] && items_t[t] > 0) {
+              if (!(ok = warp_wait(&bar_o_empty[t], (items_t[t] - 1) & 1u, wc, kBarOEmpty,
+                                   items_t[t])))
+                break;
+              tc_fence_after();
+            }
+            if (!have_v) {
+              vstage = ring % C::NS;
+              if (!(ok = warp_wait(&bar_kv_full[vstage], (ring / C::NS) & 1u, wc, kBarKvFull,
+                                   ring)))
+                break;
+              tc_fence_after();
+              ++ring;
+              have_v = true;
+            }
+            if (leader) {
+              const uint32_t v_lo = (kv_base + vstage * (C::TILE_BYTES >> 4)) | kLboV;
+#pragma unroll
+              for (int kk = 0; kk < BN / 16; ++kk)
+                mma_ts_lh(tmem + C::O_COL + t * D, tmem + C::S_COL + t * 128 + kk * 8,
+                          v_lo + kk * (16 * 128 >> 4), kHi, idesc_pv,
+                          (!first_pv[t] || kk > 0) ? 1u : 0u);
+            }
+            first_pv[t] = false;
+            pend[t] = false;
+          }
+          if (more && in[t]) {
+            if (!have_k) {
+              kstage = ring % C::NS;
+              if (!(ok = warp_wait(&bar_kv_full[kstage], (ring / C::NS) & 1u, wc, kBarKvFull,
+                                   ring)))
+                break;
+              tc_fence_after();
+              ++ring;
+              have_k = true;
+            }
+            if (leader) {
+              const uint32_t q_lo = q_lo0 + t * (C::Q_BYTES >> 4);
+              const uint32_t k_lo = (kv_base + kstage * (C::TILE_BYTES >> 4)) | kLboK;
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
+                mma_ss_lh(tmem + C::S_COL + t * 128, q_lo + off, kHi, k_lo + off, kHi, idesc_qk,
+                          kk > 0 ? 1u : 0u);
+              }
+              mma_commit(&bar_s_full[t]);
+            }
+            pend[t] = true;
+          }
+        }
+        if (!ok) break;
+        if (leader) {
+          if (have_k) mma_commit(&bar_kv_empty[kstage]);
+          if (have_v) mma_commit(&bar_kv_empty[vstage]);
+        }
+        __syncwarp();
+        if (!more) break;
+      }
+      if (!ok) break;
+      if (leader) {
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+          if (len_t[t] > 0) mma_commit(&bar_o_final[t]);
+        if (!q_released) mma_commit(&bar_q_empty);
+      }
+      __syncwarp();
+#pragma unroll
+      for (int t = 0; t < 2; ++t) items_t[t] += len_t[t] > 0 ? 1u : 0u;
+      ++qcount;
+    }
+    if (leader) {
+      mma_commit(&bar_final);
+      WaitCtx drain{&abort_flag, p.wait_limit_ns, kRoleMma};
+      int zero = 0;
+      drain.abort = &zero;
+      wait_bounded(&bar_final, 0, drain, kBarFinal, qcount);
+    }
+    __syncwarp();
+  }
+  else {
+    // ------------------------------------------------------------ softmax
+    // Warpgroup t (warps 4t..4t+3) serves tile t; thread = row = TMEM lane.
+    wc.role = kRoleSoftmax;
+    const int t = warp >> 2;
+    const int wq = warp & 3;
+    const int row_in_tile = wq * 32 + lane;
+    const uint32_t lane_tmem = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const uint32_t s_tmem = lane_tmem + C::S_COL + t * 128;
+    const uint32_t o_tmem = lane_tmem + C::O_COL + t * D;
+    const float sl2 = p.scale_log2;
+    uint32_t scnt = 0, icnt = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int idx = snake_item(k, p.total_items);
+      if (idx == -2) break;
+      if (idx < 0) continue;
+      const PairItem it = decode_pair(idx, p, npairs);
+      const int qb = it.qa + t;
+      if (qb >= p.nqb) continue;
+      const int len = t == 0 ? it.lenA : it.lenB;
+      const int a0 = t == 0 ? it.a0 : it.b0;
+      const int row = qb * BN + row_in_tile;
+      const bool store = row < p.n;
+      const long long orow = static_cast<long long>(it.bh) * p.n + row;
+      if (len == 0) {
+        if (store) {
+          uint4 *dst = reinterpret_cast<uint4 *>(p.out + orow * D);
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+          if (p.lse) p.lse[orow] = -INFINITY;
+        }
+        continue;
+      }
+      ListCache lc;
+      lc.reset(p, a0, len);
+      float m_ref = 0.f, l = 0.f;
+      for (int j = 0; j < len; ++j) {
+        if (!(ok = warp_wait(&bar_s_full[t], scnt & 1u, wc, kBarSFull, scnt))) break;
+        ++scnt;
+        tc_fence_after();
+        float s[BN];
+        {
+          uint32_t sr[BN / 32][32];
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c) tmem_ld32(s_tmem + c * 32, sr[c]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c) {
+            reg_fence32(sr[c]);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(sr[c][i]);
+          }
+        }
+        const int kb = lc.get(p, a0, len, j);
+        const int valid = p.n - kb * BN;
+        if (valid < BN) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (c >= valid) s[c] = -INFINITY;
+        }
+        float m8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = fmaxf(s[i], s[i + 8]);
+#pragma unroll
+        for (int c = 16; c < BN; c += 16) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m8[i] = fmax3(m8[i], s[c + i], s[c + 8 + i]);
+        }
+        const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                               fmaxf(m8[6], m8[7]));
+        const float mblk = mx * sl2;
+        float alpha = 1.f;
+        bool rescale = false;
+        if (j == 0) {
+          m_ref = mblk;
+        } else if (mblk > m_ref + 8.f) {
+          // lazy rescale (the final O / l is exact either way)
+          alpha = ex2_approx(m_ref - mblk);
+          m_ref = mblk;
+          rescale = true;
+        }
+        uint32_t pk[BN / 2];
+        const float sum = valid < BN ? exp2_pack_row<BN, 0>(s, sl2, -m_ref, pk)
+                                     : exp2_pack_row<BN, kEmuPairsPer8>(s, sl2, -m_ref, pk);
+        l = l * alpha + sum;
+        // S being complete means QK of this block is complete, and the
+        // previous PV of this tile was issued before it: O is settled.
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(o_tmem + c * 32, r);
+            tmem_wait_ld();
+            reg_fence32(r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(o_tmem + c * 32, r);
+          }
+        }
+        // P (bf16 pairs) over the first BN/2 columns of this tile's S buffer
+#pragma unroll
+        for (int c = 0; c < BN / 64; ++c) {
+          uint32_t r[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = pk[c * 32 + i];
+          tmem_st32(s_tmem + c * 32, r);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar_p_full[t]);
+      }
+      if (!ok) break;
+      if (!(ok = warp_wait(&bar_o_final[t], icnt & 1u, wc, kBarODone, icnt))) break;
+      ++icnt;
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(o_tmem + c * 32, r);
+        tmem_wait_ld();
+        reg_fence32(r);
+        if (store) {
+          uint4 *dst = reinterpret_cast<uint4 *>(p.out + orow * D + c * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(r[8 * v4 + 0]) * inv_l, __uint_as_float(r[8 * v4 + 1]) * inv_l);
+            w.y = pack_bf16x2(__uint_as_float(r[8 * v4 + 2]) * inv_l, __uint_as_float(r[8 * v4 + 3]) * inv_l);
+            w.z = pack_bf16x2(__uint_as_float(r[8 * v4 + 4]) * inv_l, __uint_as_float(r[8 * v4 + 5]) * inv_l);
+            w.w = pack_bf16x2(__uint_as_float(r[8 * v4 + 6]) * inv_l, __uint_as_float(r[8 * v4 + 7]) * inv_l);
+            dst[v4] = w;
+          }
+        }
+      }
+      if (store && p.lse) p.lse[orow] = (m_ref + log2f(l)) * 0.69314718055994531f;
+      tc_fence_before();
+      mbar_arrive(&bar_o_empty[t]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9) {
+    __syncwarp();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace bsa

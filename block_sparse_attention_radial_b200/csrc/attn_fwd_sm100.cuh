@@ -72,8 +72,7 @@ struct FwdCfg {
   static constexpr int DSMEM = DSMEM_USED > 122880 ? DSMEM_USED : 122880;
   static constexpr uint32_t S_COL = 0;           // S buffer b at S_COL + 128 b
   static constexpr uint32_t O_COL = 256;
-  static constexpr uint32_t Q_COL = 384;         // Q as bf16 pairs, D/2 columns
-  static constexpr uint32_t P_COL = 448;         // P as bf16 pairs, BN/2 columns
+  static constexpr uint32_t P_COL = 384;         // P buffer b at P_COL + 64 b (bf16 pairs)
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int THREADS = 192;
   static_assert(NS >= 2, "K/V ring needs at least two stages");
@@ -250,7 +249,7 @@ __global__ void __launch_bounds__(192, 1)
   __shared__ __align__(8) uint64_t bar_kv_empty[C::NS];
   __shared__ __align__(8) uint64_t bar_q_full, bar_q_empty, bar_o_empty, bar_final;
   __shared__ __align__(8) uint64_t bar_o_done[2];
-  __shared__ __align__(8) uint64_t bar_s_full[2], bar_s_free[2], bar_p_full;
+  __shared__ __align__(8) uint64_t bar_s_full[2], bar_s_free[2], bar_p_full[2];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -275,8 +274,8 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&bar_s_full[b], 1);
       mbar_init(&bar_s_free[b], 128);
       mbar_init(&bar_o_done[b], 1);
+      mbar_init(&bar_p_full[b], 128);
     }
-    mbar_init(&bar_p_full, 128);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -391,17 +390,7 @@ __global__ void __launch_bounds__(192, 1)
       if (it.len == 0) continue;
       if (!(ok = warp_wait(&bar_q_full, qcount & 1u, wc, kBarQFull, qcount))) break;
       tc_fence_after();
-      if (leader) {
-        // Q moves into TMEM once per item (after the previous item's MMAs, in
-        // issue order), so the QK MMAs read only K from shared memory; the
-        // shared Q buffer is free as soon as the copies complete.
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off_a = (kk >> 2) * (C::BM * 128 >> 4) + (kk & 3) * 2;
-          tmem_cp_128x256b(tmem + C::Q_COL + kk * 8, q_lo + off_a, kHi);
-        }
-        mma_commit(&bar_q_empty);
-      }
+
       SegWalker ks, vs;
       ks.reset(p, it.a, it.len);
       vs.reset(p, it.a, it.len);
@@ -431,19 +420,20 @@ __global__ void __launch_bounds__(192, 1)
                                    (bq - ks.first) * (BN * 128 >> 4)) | kLboK;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off_a = (kk >> 2) * (C::BM * 128 >> 4) + (kk & 3) * 2;
               const uint32_t off_b = (kk >> 2) * (C::CB_BYTES >> 4) + (kk & 3) * 2;
-              mma_ts_lh(d_tmem, tmem + C::Q_COL + kk * 8, k_lo + off_b, kHi, idesc_qk,
-                        kk > 0 ? 1u : 0u);
+              mma_ss_lh(d_tmem, q_lo + off_a, kHi, k_lo + off_b, kHi, idesc_qk, kk > 0 ? 1u : 0u);
             }
             if (bq == ks.first + ks.count - 1) mma_commit(&bar_kv_empty[kstage]);
             mma_commit(&bar_s_full[gq & 1u]);
+            if (bq == it.len - 1) mma_commit(&bar_q_empty);  // last QK: Q may refill
           }
           __syncwarp();
         }
         if (t >= 0) {
           const int j = t;
           const uint32_t gg = g + j;
-          if (!(ok = warp_wait(&bar_p_full, gg & 1u, wc, kBarPFull, gg))) break;
+          if (!(ok = warp_wait(&bar_p_full[gg & 1u], (gg >> 1) & 1u, wc, kBarPFull, gg))) break;
           tc_fence_after();
           if (j == 0 && items_done > 0) {
             if (!(ok = warp_wait(&bar_o_empty, (items_done - 1) & 1u, wc, kBarOEmpty, items_done)))
@@ -464,7 +454,8 @@ __global__ void __launch_bounds__(192, 1)
             for (int kk = 0; kk < BN / 16; ++kk) {
               // V rows of 128 bytes (64 head-dim values); 64-wide head-dim
               // chunks one stage column block apart (MN-major operand)
-              mma_ts_lh(tmem + C::O_COL, tmem + C::P_COL + kk * 8, v_lo + kk * (16 * 128 >> 4),
+              mma_ts_lh(tmem + C::O_COL, tmem + C::P_COL + (gg & 1u) * 64u + kk * 8,
+                        v_lo + kk * (16 * 128 >> 4),
                         kHi, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
             }
             if (j == vs.first + vs.count - 1) mma_commit(&bar_kv_empty[vstage]);
@@ -569,18 +560,21 @@ __global__ void __launch_bounds__(192, 1)
         const float sum = valid < BN ? exp2_pack_row<BN, 0>(s, sl2, -m_ref, pk)
                                      : exp2_pack_row<BN, kEmuPairsPer8>(s, sl2, -m_ref, pk);
         l = l * alpha + sum;
-        // PV(gg-1) must have finished with the P buffer (and with O, which a
-        // rescale touches) before P(gg) is written. Waiting for it at every
-        // block keeps each o_done wait phase-exact: PV(gg-2) was waited for
-        // at the previous block. PV(gg-1) was issued a whole softmax earlier,
-        // so this rarely stalls.
-        if (gg >= 1) {
-          if (!(ok = warp_wait(&bar_o_done[(gg - 1) & 1u], ((gg - 1) >> 1) & 1u, wc, kBarODone,
-                               gg)))
+        // P buffer gg&1 was last read by PV(gg-2). Waiting for that PV at
+        // every block keeps each o_done wait phase-exact (PV(gg-4) was waited
+        // for two blocks ago) and is cheap: PV(gg-2) was issued a whole block
+        // earlier. Only a rescale of O also needs PV(gg-1); that wait is
+        // phase-exact too, since PV(gg-3) is complete once PV(gg-2) is.
+        if (gg >= 2) {
+          if (!(ok = warp_wait(&bar_o_done[gg & 1u], ((gg - 2) >> 1) & 1u, wc, kBarODone, gg)))
             break;
           tc_fence_after();
         }
         if (__any_sync(0xffffffffu, rescale)) {
+          if (!(ok = warp_wait(&bar_o_done[(gg - 1) & 1u], ((gg - 1) >> 1) & 1u, wc, kBarODone,
+                               gg)))
+            break;
+          tc_fence_after();
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t r[32];
@@ -592,17 +586,17 @@ __global__ void __launch_bounds__(192, 1)
             tmem_st32(lane_tmem + C::O_COL + c * 32, r);
           }
         }
-        // P (bf16 pairs) into its own TMEM columns
+        // P (bf16 pairs) into its TMEM buffer
 #pragma unroll
         for (int c = 0; c < BN / 64; ++c) {
           uint32_t r[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) r[i] = pk[c * 32 + i];
-          tmem_st32(lane_tmem + C::P_COL + c * 32, r);
+          tmem_st32(lane_tmem + C::P_COL + (gg & 1u) * 64u + c * 32, r);
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bar_p_full);
+        mbar_arrive(&bar_p_full[gg & 1u]);
       }
       if (!ok) break;
       const uint32_t gl = g + it.len - 1;

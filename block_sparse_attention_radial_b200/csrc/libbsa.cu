@@ -15,6 +15,7 @@
 
 #include "bsa.h"
 
+#include "attn_fwd_pair_sm100.cuh"
 #include "attn_fwd_sm100.cuh"
 #include "dense_ref.cuh"
 #include "device_status.cuh"
@@ -41,12 +42,13 @@ int cuda_fail(cudaError_t e, const char *what) {
 std::mutex g_hook_mu;
 unsigned long long g_wait_limit_ns = 2000000000ull;
 int g_fault_flags = 0;
+bool g_force_one_tile = false;  // test hook: run block-128 problems on the one-tile kernel
 
 constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   bool probed = false;
   int cc_major = 0, cc_minor = 0, sms = 0;
-  bool attrs_set[4] = {false, false, false, false};
+  bool attrs_set[8] = {false, false, false, false, false, false, false, false};
   bool ref_attrs_set[4] = {false, false, false, false};
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -198,6 +200,91 @@ int launch_ref(const RefParams &p, int batch, DeviceInfo *dev, int slot, cudaStr
 
 int slot_of(int D, int BN) { return (D == 128 ? 2 : 0) + (BN == 128 ? 1 : 0); }
 
+template <int D>
+int launch_pair(const void *q, const void *k, const void *v, int32_t bh, int32_t n,
+                const FwdParams &p, DeviceInfo *dev, cudaStream_t stream) {
+  using C = PairCfg<D>;
+  CUtensorMap tq, tk, tv;
+  int st;
+  if ((st = make_map(&tq, q, bh, n, D, C::BN)) != BSA_OK) return st;
+  if ((st = make_map(&tk, k, bh, n, D, C::BN)) != BSA_OK) return st;
+  if ((st = make_map(&tv, v, bh, n, D, C::BN)) != BSA_OK) return st;
+  const int slot = 4 + (D == 128 ? 1 : 0);
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!dev->attrs_set[slot]) {
+      BSA_CUDA(cudaFuncSetAttribute(attn_fwd_pair_sm100_kernel<D>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::DSMEM));
+      dev->attrs_set[slot] = true;
+    }
+  }
+  const int grid = p.total_items < dev->sms ? p.total_items : dev->sms;
+  attn_fwd_pair_sm100_kernel<D><<<grid, C::THREADS, C::DSMEM, stream>>>(tq, tk, tv, p);
+  BSA_CUDA(cudaGetLastError());
+  return BSA_OK;
+}
+
+// Work order into `order`, then the attention kernel. Block-128 problems run
+// on the two-tile kernel (adjacent query blocks share K/V loads); block 64 on
+// the one-tile kernel. Arguments were checked by the caller.
+int run_fwd(const void *q, const void *k, const void *v, int32_t batch, int32_t heads,
+            int32_t n, int32_t head_dim, float softmax_scale, const bsa_block_lists *l,
+            void *out, float *lse, int32_t *order, DeviceInfo *dev, int fault_flags,
+            cudaStream_t stream) {
+  const int nqb = l->num_q_blocks;
+  bool pair;
+  {
+    std::lock_guard<std::mutex> lk(g_hook_mu);
+    pair = l->block == 128 && !g_force_one_tile;
+  }
+  if (pair) {
+    const int npairs = (nqb + 1) / 2;
+    const size_t smem = static_cast<size_t>(npairs <= kLptMaxRows ? npairs : 0) * sizeof(int);
+    pair_order_kernel<<<l->num_lists, 1024, smem, stream>>>(l->row_ptr, l->col_idx, nqb, l->nnz,
+                                                           order, kLptMaxRows);
+  } else {
+    const size_t smem = static_cast<size_t>(nqb <= kLptMaxRows ? nqb : 0) * sizeof(int);
+    lpt_order_kernel<<<l->num_lists, 1024, smem, stream>>>(l->row_ptr, nqb, l->nnz, order,
+                                                          kLptMaxRows);
+  }
+  BSA_CUDA(cudaGetLastError());
+
+  FwdParams p;
+  p.row_ptr = l->row_ptr;
+  p.col_idx = l->col_idx;
+  p.order = order;
+  p.out = static_cast<__nv_bfloat16 *>(out);
+  p.lse = lse;
+  p.heads = heads;
+  p.n = n;
+  p.nqb = nqb;
+  p.nkb = l->num_k_blocks;
+  p.num_lists = l->num_lists;
+  p.nnz = l->nnz;
+  p.total_items = batch * heads * (pair ? (nqb + 1) / 2 : nqb);
+  const float scale =
+      softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
+  p.scale_log2 = scale * 1.4426950408889634f;
+  {
+    std::lock_guard<std::mutex> lk(g_hook_mu);
+    p.wait_limit_ns = g_wait_limit_ns;
+  }
+  p.fault_flags = fault_flags;
+  const int bh = batch * heads;
+  if (pair) {
+    if (head_dim == 128) return launch_pair<128>(q, k, v, bh, n, p, dev, stream);
+    return launch_pair<64>(q, k, v, bh, n, p, dev, stream);
+  }
+  const int slot = slot_of(head_dim, l->block);
+  if (head_dim == 128 && l->block == 128)
+    return launch_fwd<128, 128>(q, k, v, bh, n, p, dev, slot, stream);
+  if (head_dim == 128 && l->block == 64)
+    return launch_fwd<128, 64>(q, k, v, bh, n, p, dev, slot, stream);
+  if (head_dim == 64 && l->block == 128)
+    return launch_fwd<64, 128>(q, k, v, bh, n, p, dev, slot, stream);
+  return launch_fwd<64, 64>(q, k, v, bh, n, p, dev, slot, stream);
+}
+
 // Self-test of the two exp2 paths of the attention softmax against exp2f.
 __global__ void exp2_selftest_kernel(const float *x, float *y_poly, float *y_mufu,
                                      float *y_ref, int n) {
@@ -280,43 +367,14 @@ int bsa_attn_fwd(const void *q, const void *k, const void *v, int32_t batch, int
   if ((st = current_device(&dev)) != BSA_OK) return st;
   if (dev->cc_major != 10) return BSA_ERR_UNSUPPORTED;
 
-  const int nqb = l->num_q_blocks;
-  int32_t *order = static_cast<int32_t *>(workspace);
-  const size_t lpt_smem = static_cast<size_t>(nqb <= kLptMaxRows ? nqb : 0) * sizeof(int);
-  lpt_order_kernel<<<l->num_lists, 1024, lpt_smem, stream>>>(l->row_ptr, nqb, l->nnz, order,
-                                                            kLptMaxRows);
-  BSA_CUDA(cudaGetLastError());
-
-  FwdParams p;
-  p.row_ptr = l->row_ptr;
-  p.col_idx = l->col_idx;
-  p.order = order;
-  p.out = static_cast<__nv_bfloat16 *>(out);
-  p.lse = lse;
-  p.heads = heads;
-  p.n = n;
-  p.nqb = nqb;
-  p.nkb = l->num_k_blocks;
-  p.num_lists = l->num_lists;
-  p.nnz = l->nnz;
-  p.total_items = batch * heads * nqb;
-  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
-  p.scale_log2 = scale * 1.4426950408889634f;
+  int fault_flags;
   {
     std::lock_guard<std::mutex> lk(g_hook_mu);
-    p.wait_limit_ns = g_wait_limit_ns;
-    p.fault_flags = g_fault_flags;
+    fault_flags = g_fault_flags;
     g_fault_flags = 0;
   }
-  const int bh = batch * heads;
-  const int slot = slot_of(head_dim, l->block);
-  if (head_dim == 128 && l->block == 128)
-    return launch_fwd<128, 128>(q, k, v, bh, n, p, dev, slot, stream);
-  if (head_dim == 128 && l->block == 64)
-    return launch_fwd<128, 64>(q, k, v, bh, n, p, dev, slot, stream);
-  if (head_dim == 64 && l->block == 128)
-    return launch_fwd<64, 128>(q, k, v, bh, n, p, dev, slot, stream);
-  return launch_fwd<64, 64>(q, k, v, bh, n, p, dev, slot, stream);
+  return run_fwd(q, k, v, batch, heads, n, head_dim, softmax_scale, l, out, lse,
+                 static_cast<int32_t *>(workspace), dev, fault_flags, stream);
 }
 
 int bsa_attn_dense_masked_ref(const void *q, const void *k, const void *v, int32_t batch,
@@ -436,7 +494,8 @@ int bsa_set_test_hooks(int64_t wait_limit_ns, int32_t fault_flags) {
   if (wait_limit_ns < 0) return BSA_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lk(g_hook_mu);
   g_wait_limit_ns = wait_limit_ns == 0 ? 2000000000ull : static_cast<unsigned long long>(wait_limit_ns);
-  g_fault_flags = fault_flags;
+  g_fault_flags = fault_flags & 1;
+  g_force_one_tile = (fault_flags & 2) != 0;
   return BSA_OK;
 }
 
@@ -489,40 +548,6 @@ extern "C" int bsa_attn_fwd_noalloc(const void *q, const void *k, const void *v,
   int32_t *order = nullptr;
   if ((st = noalloc_scratch(&order)) != BSA_OK) return st;
 
-  const int nqb = l->num_q_blocks;
-  const size_t lpt_smem = static_cast<size_t>(nqb <= kLptMaxRows ? nqb : 0) * sizeof(int);
-  lpt_order_kernel<<<l->num_lists, 1024, lpt_smem, stream>>>(l->row_ptr, nqb, l->nnz, order,
-                                                            kLptMaxRows);
-  BSA_CUDA(cudaGetLastError());
-
-  FwdParams p;
-  p.row_ptr = l->row_ptr;
-  p.col_idx = l->col_idx;
-  p.order = order;
-  p.out = static_cast<__nv_bfloat16 *>(out);
-  p.lse = lse;
-  p.heads = heads;
-  p.n = n;
-  p.nqb = nqb;
-  p.nkb = l->num_k_blocks;
-  p.num_lists = l->num_lists;
-  p.nnz = l->nnz;
-  p.total_items = batch * heads * nqb;
-  const float scale =
-      softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
-  p.scale_log2 = scale * 1.4426950408889634f;
-  {
-    std::lock_guard<std::mutex> lk(g_hook_mu);
-    p.wait_limit_ns = g_wait_limit_ns;
-    p.fault_flags = 0;
-  }
-  const int bh = batch * heads;
-  const int slot = slot_of(head_dim, l->block);
-  if (head_dim == 128 && l->block == 128)
-    return launch_fwd<128, 128>(q, k, v, bh, n, p, dev, slot, stream);
-  if (head_dim == 128 && l->block == 64)
-    return launch_fwd<128, 64>(q, k, v, bh, n, p, dev, slot, stream);
-  if (head_dim == 64 && l->block == 128)
-    return launch_fwd<64, 128>(q, k, v, bh, n, p, dev, slot, stream);
-  return launch_fwd<64, 64>(q, k, v, bh, n, p, dev, slot, stream);
+  return run_fwd(q, k, v, batch, heads, n, head_dim, softmax_scale, l, out, lse, order, dev, 0,
+                 stream);
 }

@@ -2,6 +2,7 @@
 // longest-row-first work order used by the attention kernel.
 #pragma once
 
+#include <climits>
 #include <cstdint>
 
 #include "device_status.cuh"
@@ -194,6 +195,51 @@ __global__ void lpt_order_kernel(const int32_t *row_ptr, int nqb, int nnz, int32
     const int c = cost[r];
     int rank = 0;
     for (int o = 0; o < nqb; ++o) {
+      const int co = cost[o];
+      rank += (co > c) || (co == c && o < r);
+    }
+    ord[rank] = r;
+  }
+}
+
+// One CTA per list: order[list * npairs + rank] = query-block pair (2p, 2p+1)
+// with the rank-th longest union of key blocks (ties: lower pair first).
+// Lists whose pair count does not fit in shared memory keep natural order.
+__global__ void pair_order_kernel(const int32_t *row_ptr, const int32_t *col_idx, int nqb,
+                                  int nnz, int32_t *order, int max_smem_rows) {
+  extern __shared__ int cost[];
+  const int list = blockIdx.x;
+  const int npairs = (nqb + 1) / 2;
+  const int32_t *rp = row_ptr + static_cast<long long>(list) * nqb;
+  int32_t *ord = order + static_cast<long long>(list) * npairs;
+  if (npairs > max_smem_rows) {
+    for (int r = threadIdx.x; r < npairs; r += blockDim.x) ord[r] = r;
+    return;
+  }
+  for (int pr = threadIdx.x; pr < npairs; pr += blockDim.x) {
+    const int qa = 2 * pr;
+    int ia = min(max(rp[qa], 0), nnz), ea = min(max(rp[qa + 1], 0), nnz);
+    int ib = 0, eb = 0;
+    if (qa + 1 < nqb) {
+      ib = min(max(rp[qa + 1], 0), nnz);
+      eb = min(max(rp[qa + 2], 0), nnz);
+    }
+    int u = 0;
+    while (ia < ea || ib < eb) {  // merge the two sorted rows
+      const int va = ia < ea ? col_idx[ia] : INT_MAX;
+      const int vb = ib < eb ? col_idx[ib] : INT_MAX;
+      const int m = min(va, vb);
+      ia += va == m;
+      ib += vb == m;
+      ++u;
+    }
+    cost[pr] = u;
+  }
+  __syncthreads();
+  for (int r = threadIdx.x; r < npairs; r += blockDim.x) {
+    const int c = cost[r];
+    int rank = 0;
+    for (int o = 0; o < npairs; ++o) {
       const int co = cost[o];
       rank += (co > c) || (co == c && o < r);
     }

@@ -186,6 +186,9 @@ const char *bsa_last_cuda_error(void);
  * bsa_attn_fwd launch skip its first K-tile load, so that the consumer's
  * bounded wait runs out and the call reports BSA_ERR_DEVICE_TIMEOUT through
  * bsa_get_device_status(); the flag clears itself after one launch.
+ * `fault_flags` bit 1 (sticky until the next call) runs block-128 problems on
+ * the one-tile kernel instead of the two-tile kernel, so that tests can
+ * compare the two schedules; it changes no result beyond rounding order.
  */
 int bsa_set_test_hooks(int64_t wait_limit_ns, int32_t fault_flags);
 

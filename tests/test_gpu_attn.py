@@ -159,3 +159,27 @@ def _check_large(bsa, name):
 @pytest.mark.parametrize("name", ["wan", "hunyuan", "long4x", "generic"])
 def test_full_size_configs(bsa, name):
     _check_large(bsa, name)
+
+
+@pytest.mark.parametrize("B,H,n,D,L,seed", [(1, 2, 640, 128, 1, 21), (2, 1, 1152, 64, 1, 22),
+                                            (1, 3, 1000, 128, 3, 23)])
+def test_one_tile_and_two_tile_schedules_agree(bsa, B, H, n, D, L, seed):
+    """Block-128 problems run on the two-tile kernel by default; hook bit 1
+    routes them to the one-tile kernel. Both match the oracle, and an odd
+    number of query blocks leaves the last pair with a single tile."""
+    blk = 128
+    q, k, v = (t.cuda() for t in make_random_qkv(B, H, n, D, seed))
+    nqb = -(-n // blk)
+    rp, ci = random_block_lists(L * nqb, nqb, 0.45, seed + 7, empty_rows=[1] if L * nqb > 2 else [],
+                                force={0: [nqb - 1]})
+    lists = bsa.block_lists_from_csr(rp, ci, L, nqb, blk)
+    ref_o, ref_l = oracle.masked_attention_fp64(q, k, v, rp, ci, L, blk)
+    o2, l2 = bsa.attention(q, k, v, lists)
+    try:
+        bsa.bsa_set_test_hooks(0, 2)
+        o1, l1 = bsa.attention(q, k, v, lists)
+    finally:
+        bsa.bsa_set_test_hooks(0, 0)
+    assert bsa.bsa_get_device_status() == 0
+    assert_close(o2, ref_o, l2, ref_l, "two-tile vs oracle")
+    assert_close(o1, ref_o, l1, ref_l, "one-tile vs oracle")
