@@ -57,7 +57,7 @@ def load_peaks():
 def load_traffic(workload: str):
     """DRAM bytes per launch of the attention kernel from a committed ncu summary,
     or None when the summary is missing or was taken on different kernel source."""
-    path = os.path.join(ROOT, "profiles", f"attn_fwd_sm100_{workload}_traffic.json")
+    path = os.path.join(ROOT, "profiles", f"attn_fwd_pair_sm100_{workload}_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
