@@ -49,32 +49,44 @@ struct PairCfg {
   static_assert(NS >= 3, "K/V ring needs at least three stages");
 };
 
+// One row's key blocks read in order by a single thread. The next entry is
+// loaded one call ahead, so its latency overlaps the caller's work.
+struct RowReader {
+  const int32_t *ptr;
+  int left, nxt, hi;
+  __device__ __forceinline__ int fetch() const {
+    return left > 0 ? min(max(__ldg(ptr), 0), hi) : INT_MAX;
+  }
+  __device__ __forceinline__ void reset(const FwdParams &p, int a, int len) {
+    ptr = p.col_idx + a;
+    left = len;
+    hi = p.nkb - 1;
+    nxt = fetch();
+  }
+  __device__ __forceinline__ void pop() {
+    ++ptr;
+    --left;
+    nxt = fetch();
+  }
+};
+
 // Key blocks of one query-block pair, walked as the sorted union of the two
-// rows. Warp-uniform; the producer, the MMA warp and nothing else use it.
+// rows by one thread (the producer and the MMA issuer run identical walks).
 struct UnionWalker {
-  ListCache ca, cb;
-  int a0, lenA, b0, lenB, ia, ib;
-  __device__ __forceinline__ void reset(const FwdParams &p, int a0_, int lenA_, int b0_,
-                                        int lenB_) {
-    a0 = a0_;
-    lenA = lenA_;
-    b0 = b0_;
-    lenB = lenB_;
-    ia = 0;
-    ib = 0;
-    ca.reset(p, a0, lenA);
-    cb.reset(p, b0, lenB);
+  RowReader ra, rb;
+  __device__ __forceinline__ void reset(const FwdParams &p, int a0, int lenA, int b0, int lenB) {
+    ra.reset(p, a0, lenA);
+    rb.reset(p, b0, lenB);
   }
   // Next union block: false when both rows are exhausted.
-  __device__ __forceinline__ bool next(const FwdParams &p, int &kb, bool &inA, bool &inB) {
-    if (ia >= lenA && ib >= lenB) return false;
-    const int va = ia < lenA ? ca.get(p, a0, lenA, ia) : INT_MAX;
-    const int vb = ib < lenB ? cb.get(p, b0, lenB, ib) : INT_MAX;
+  __device__ __forceinline__ bool next(int &kb, bool &inA, bool &inB) {
+    const int va = ra.nxt, vb = rb.nxt;
+    if (va == INT_MAX && vb == INT_MAX) return false;
     kb = min(va, vb);
     inA = va == kb;
     inB = vb == kb;
-    ia += inA ? 1 : 0;
-    ib += inB ? 1 : 0;
+    if (inA) ra.pop();
+    if (inB) rb.pop();
     return true;
   }
 };
@@ -161,72 +173,67 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
-    wc.role = kRoleProducer;
-    const bool leader = lane == 0;
-    if (leader) {
+    // One lane: TMA issue needs no warp, and warp-wide bookkeeping between
+    // issues only adds latency.
+    if (lane == 0) {
+      wc.role = kRoleProducer;
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-    }
-    uint32_t ring = 0, qcount = 0;
-    bool skip_next_k = (p.fault_flags & 1) && blockIdx.x == 0;
-    int skipped_ring = -1;
-    bool ok = true;
-    for (int k = 0; ok; ++k) {
-      const int idx = snake_item(k, p.total_items);
-      if (idx == -2) break;
-      if (idx < 0) continue;
-      const PairItem it = decode_pair(idx, p, npairs);
-      if (it.lenA == 0 && it.lenB == 0) continue;
-      if (!(ok = warp_wait(&bar_q_empty, (qcount & 1u) ^ 1u, wc, kBarQEmpty, qcount))) break;
-      if (leader) {
+      uint32_t ring = 0, qcount = 0;
+      bool skip_next_k = (p.fault_flags & 1) && blockIdx.x == 0;
+      int skipped_ring = -1;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int idx = snake_item(k, p.total_items);
+        if (idx == -2) break;
+        if (idx < 0) continue;
+        const PairItem it = decode_pair(idx, p, npairs);
+        if (it.lenA == 0 && it.lenB == 0) continue;
+        if (!(ok = lane_wait(&bar_q_empty, (qcount & 1u) ^ 1u, wc, kBarQEmpty, qcount))) break;
         mbar_arrive_expect_tx(&bar_q_full, 2 * C::Q_BYTES);
         tma_load_4d(sQ, &tm_q, &bar_q_full, 0, it.qa * BN, 0, it.bh);
         tma_load_4d(sQ + C::Q_BYTES, &tm_q, &bar_q_full, 0, (it.qa + 1) * BN, 0, it.bh);
-      }
-      ++qcount;
-      // Same walk and same first-use order as the MMA warp: at step j the
-      // MMA warp needs V(j-1) first when tile A listed j-1 or A skips j, and
-      // K(j) first otherwise.
-      UnionWalker uw;
-      uw.reset(p, it.a0, it.lenA, it.b0, it.lenB);
-      bool pa = false, pb = false;
-      int prev_kb = 0;
-      for (int j = 0; ok; ++j) {
-        int kb = 0;
-        bool a = false, b = false;
-        const bool more = uw.next(p, kb, a, b);
-        const bool need_v = pa || pb;
-        if (!more && !need_v) break;
-        const bool v_first = pa || !a;
+        ++qcount;
+        // Same walk and same first-use order as the MMA issuer: at step j it
+        // needs V(j-1) first when tile A listed j-1 or A skips j, and K(j)
+        // first otherwise.
+        UnionWalker uw;
+        uw.reset(p, it.a0, it.lenA, it.b0, it.lenB);
+        bool pa = false, pb = false;
+        int prev_kb = 0;
+        while (ok) {
+          int kb = 0;
+          bool a = false, b = false;
+          const bool more = uw.next(kb, a, b);
+          const bool need_v = pa || pb;
+          if (!more && !need_v) break;
+          const bool v_first = pa || !a;
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const bool is_v = (e == 0) == v_first;
-          if (is_v ? !need_v : !more) continue;
-          const uint32_t s = ring % C::NS;
-          if (!(ok = warp_wait(&bar_kv_empty[s], ((ring / C::NS) & 1u) ^ 1u, wc, kBarKvEmpty,
-                               ring)))
-            break;
-          if (!is_v && skip_next_k) {  // test hook: this stage's barrier never gets its arrival
-            skip_next_k = false;
-            skipped_ring = static_cast<int>(ring);
-            ++ring;
-            continue;
-          }
-          if (leader) {
+          for (int e = 0; e < 2; ++e) {
+            const bool is_v = (e == 0) == v_first;
+            if (is_v ? !need_v : !more) continue;
+            const uint32_t s = ring % C::NS;
+            if (!(ok = lane_wait(&bar_kv_empty[s], ((ring / C::NS) & 1u) ^ 1u, wc, kBarKvEmpty,
+                                 ring)))
+              break;
+            if (!is_v && skip_next_k) {  // test hook: this stage's barrier never gets its arrival
+              skip_next_k = false;
+              skipped_ring = static_cast<int>(ring);
+              ++ring;
+              continue;
+            }
             mbar_arrive_expect_tx(&bar_kv_full[s], C::TILE_BYTES);
             tma_load_4d(sKV + s * C::TILE_BYTES, is_v ? &tm_v : &tm_k, &bar_kv_full[s], 0,
                         (is_v ? prev_kb : kb) * BN, 0, it.bh);
+            ++ring;
           }
-          ++ring;
+          pa = a;
+          pb = b;
+          prev_kb = kb;
+          if (!more) break;
         }
-        pa = a;
-        pb = b;
-        prev_kb = kb;
-        if (!more) break;
       }
-    }
-    if (leader) {
       WaitCtx drain{&abort_flag, p.wait_limit_ns, kRoleProducer};
       int zero = 0;
       drain.abort = &zero;
@@ -241,89 +248,87 @@ __global__ void __launch_bounds__(320, 1)
   }
   else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    // Whole warp walks; lane 0 issues. Descriptors as 32-bit halves (see the
-    // one-tile kernel): shared high half, low half = address >> 4 | LBO.
-    wc.role = kRoleMma;
-    const bool leader = lane == 0;
-    constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false);
-    constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-    constexpr uint32_t kHi = (1024u >> 4) | (1u << 14) | (2u << 29);
-    constexpr uint32_t kLboK = 1u << 16;
-    constexpr uint32_t kLboV = static_cast<uint32_t>(BN * 128 / 16) << 16;  // 64-wide D chunks
-    const uint32_t q_lo0 = (smem_addr(sQ) >> 4) | kLboK;
-    const uint32_t kv_base = smem_addr(sKV) >> 4;
-    uint32_t ring = 0, qcount = 0;
-    uint32_t pcnt[2] = {0u, 0u};      // p_full phases consumed, per tile
-    uint32_t items_t[2] = {0u, 0u};   // items in which the tile had blocks
-    bool ok = true;
-    for (int k = 0; ok; ++k) {
-      const int idx = snake_item(k, p.total_items);
-      if (idx == -2) break;
-      if (idx < 0) continue;
-      const PairItem it = decode_pair(idx, p, npairs);
-      if (it.lenA == 0 && it.lenB == 0) continue;
-      if (!(ok = warp_wait(&bar_q_full, qcount & 1u, wc, kBarQFull, qcount))) break;
-      tc_fence_after();
-      const int len_t[2] = {it.lenA, it.lenB};
-      UnionWalker uw;
-      uw.reset(p, it.a0, it.lenA, it.b0, it.lenB);
-      bool pend[2] = {false, false}, first_pv[2] = {true, true};
-      bool q_released = false;
-      for (int j = 0; ok; ++j) {
-        int kb = 0;
-        bool in[2] = {false, false};
-        const bool more = uw.next(p, kb, in[0], in[1]);
-        if (!more && !pend[0] && !pend[1]) break;
-        if (!more && !q_released) {  // no QK left in this item: the Q buffers may refill
-          if (leader) mma_commit(&bar_q_empty);
-          q_released = true;
-        }
-        bool have_k = false, have_v = false;
-        uint32_t kstage = 0, vstage = 0;
+    // One lane issues everything. tcgen05.mma and tcgen05.commit issued from
+    // a single thread go back to back; issued under a lane-0 branch of a
+    // whole warp that also votes on its waits, each MMA and commit costs
+    // tens of extra cycles. Descriptors as 32-bit halves (see the one-tile
+    // kernel): shared high half, low half = address >> 4 | LBO.
+    if (lane == 0) {
+      wc.role = kRoleMma;
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+      constexpr uint32_t kHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+      constexpr uint32_t kLboK = 1u << 16;
+      constexpr uint32_t kLboV = static_cast<uint32_t>(BN * 128 / 16) << 16;  // 64-wide D chunks
+      const uint32_t q_lo0 = (smem_addr(sQ) >> 4) | kLboK;
+      const uint32_t kv_base = smem_addr(sKV) >> 4;
+      uint32_t ring = 0, qcount = 0;
+      uint32_t pcnt[2] = {0u, 0u};     // p_full phases consumed, per tile
+      uint32_t items_t[2] = {0u, 0u};  // items in which the tile had blocks
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int idx = snake_item(k, p.total_items);
+        if (idx == -2) break;
+        if (idx < 0) continue;
+        const PairItem it = decode_pair(idx, p, npairs);
+        if (it.lenA == 0 && it.lenB == 0) continue;
+        if (!(ok = lane_wait(&bar_q_full, qcount & 1u, wc, kBarQFull, qcount))) break;
+        tc_fence_after();
+        const int len_t[2] = {it.lenA, it.lenB};
+        UnionWalker uw;
+        uw.reset(p, it.a0, it.lenA, it.b0, it.lenB);
+        bool pend[2] = {false, false}, first_pv[2] = {true, true};
+        bool q_released = false;
+        while (ok) {
+          int kb = 0;
+          bool in[2] = {false, false};
+          const bool more = uw.next(kb, in[0], in[1]);
+          if (!more && !pend[0] && !pend[1]) break;
+          if (!more && !q_released) {  // no QK left in this item: the Q buffers may refill
+            mma_commit(&bar_q_empty);
+            q_released = true;
+          }
+          bool have_k = false, have_v = false;
+          uint32_t kstage = 0, vstage = 0;
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (!ok) break;
-          if (pend[t]) {
-            if (!(ok = warp_wait(&bar_p_full[t], pcnt[t] & 1u, wc, kBarPFull, pcnt[t]))) break;
-            ++pcnt[t];
-            tc_fence_after();
-            if (first_pv[t] && items_t[t] > 0) {
-              if (!(ok = warp_wait(&bar_o_empty[t], (items_t[t] - 1) & 1u, wc, kBarOEmpty,
-                                   items_t[t])))
-                break;
+          for (int t = 0; t < 2; ++t) {
+            if (!ok) break;
+            if (pend[t]) {
+              if (!(ok = lane_wait(&bar_p_full[t], pcnt[t] & 1u, wc, kBarPFull, pcnt[t]))) break;
+              ++pcnt[t];
+              if (first_pv[t] && items_t[t] > 0) {
+                if (!(ok = lane_wait(&bar_o_empty[t], (items_t[t] - 1) & 1u, wc, kBarOEmpty,
+                                     items_t[t])))
+                  break;
+              }
+              if (!have_v) {
+                vstage = ring % C::NS;
+                if (!(ok = lane_wait(&bar_kv_full[vstage], (ring / C::NS) & 1u, wc, kBarKvFull,
+                                     ring)))
+                  break;
+                ++ring;
+                have_v = true;
+              }
               tc_fence_after();
-            }
-            if (!have_v) {
-              vstage = ring % C::NS;
-              if (!(ok = warp_wait(&bar_kv_full[vstage], (ring / C::NS) & 1u, wc, kBarKvFull,
-                                   ring)))
-                break;
-              tc_fence_after();
-              ++ring;
-              have_v = true;
-            }
-            if (leader) {
               const uint32_t v_lo = (kv_base + vstage * (C::TILE_BYTES >> 4)) | kLboV;
 #pragma unroll
               for (int kk = 0; kk < BN / 16; ++kk)
                 mma_ts_lh(tmem + C::O_COL + t * D, tmem + C::S_COL + t * 128 + kk * 8,
                           v_lo + kk * (16 * 128 >> 4), kHi, idesc_pv,
                           (!first_pv[t] || kk > 0) ? 1u : 0u);
+              first_pv[t] = false;
+              pend[t] = false;
             }
-            first_pv[t] = false;
-            pend[t] = false;
-          }
-          if (more && in[t]) {
-            if (!have_k) {
-              kstage = ring % C::NS;
-              if (!(ok = warp_wait(&bar_kv_full[kstage], (ring / C::NS) & 1u, wc, kBarKvFull,
-                                   ring)))
-                break;
-              tc_fence_after();
-              ++ring;
-              have_k = true;
-            }
-            if (leader) {
+            if (more && in[t]) {
+              if (!have_k) {
+                kstage = ring % C::NS;
+                if (!(ok = lane_wait(&bar_kv_full[kstage], (ring / C::NS) & 1u, wc, kBarKvFull,
+                                     ring)))
+                  break;
+                tc_fence_after();
+                ++ring;
+                have_k = true;
+              }
               const uint32_t q_lo = q_lo0 + t * (C::Q_BYTES >> 4);
               const uint32_t k_lo = (kv_base + kstage * (C::TILE_BYTES >> 4)) | kLboK;
 #pragma unroll
@@ -333,31 +338,23 @@ __global__ void __launch_bounds__(320, 1)
                           kk > 0 ? 1u : 0u);
               }
               mma_commit(&bar_s_full[t]);
+              pend[t] = true;
             }
-            pend[t] = true;
           }
-        }
-        if (!ok) break;
-        if (leader) {
+          if (!ok) break;
           if (have_k) mma_commit(&bar_kv_empty[kstage]);
           if (have_v) mma_commit(&bar_kv_empty[vstage]);
+          if (!more) break;
         }
-        __syncwarp();
-        if (!more) break;
-      }
-      if (!ok) break;
-      if (leader) {
+        if (!ok) break;
 #pragma unroll
         for (int t = 0; t < 2; ++t)
           if (len_t[t] > 0) mma_commit(&bar_o_final[t]);
         if (!q_released) mma_commit(&bar_q_empty);
-      }
-      __syncwarp();
 #pragma unroll
-      for (int t = 0; t < 2; ++t) items_t[t] += len_t[t] > 0 ? 1u : 0u;
-      ++qcount;
-    }
-    if (leader) {
+        for (int t = 0; t < 2; ++t) items_t[t] += len_t[t] > 0 ? 1u : 0u;
+        ++qcount;
+      }
       mma_commit(&bar_final);
       WaitCtx drain{&abort_flag, p.wait_limit_ns, kRoleMma};
       int zero = 0;

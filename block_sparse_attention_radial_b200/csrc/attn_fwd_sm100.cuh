@@ -125,6 +125,12 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const 
   return __all_sync(0xffffffffu, r);
 }
 
+// Single-thread wait, for the roles that run on one lane (no warp vote).
+__device__ __forceinline__ bool lane_wait(uint64_t *bar, uint32_t parity, const WaitCtx &w,
+                                          int bar_id, uint32_t counter) {
+  return mbar_try_wait(bar, parity) || wait_bounded(bar, parity, w, bar_id, counter);
+}
+
 // Work item k of this CTA (static snake over the ordered item list); -1 when
 // the CTA has no item k.
 __device__ __forceinline__ int snake_item(int k, int total) {
