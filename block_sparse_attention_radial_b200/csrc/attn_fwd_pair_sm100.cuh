@@ -288,13 +288,32 @@ __global__ void __launch_bounds__(320, 1)
             mma_commit(&bar_q_empty);
             q_released = true;
           }
+          // Ring positions of this step's V(j-1) and K(j), in the producer's
+          // first-use order, and early non-blocking checks of their barriers
+          // and of tile A's P. A check of even a completed mbarrier takes
+          // about as long as two MMAs and the tensor pipe accepts one MMA at a
+          // time, so checks issued together (and ahead of the MMAs that
+          // precede their use) keep that latency off the tensor pipe.
+          const bool need_v = pend[0] || pend[1];
+          const bool need_k = more && (in[0] || in[1]);
+          const bool v_first = pend[0] || !in[0];
+          const uint32_t vpos = ring + ((need_k && !v_first) ? 1u : 0u);
+          const uint32_t kpos = ring + ((need_v && v_first) ? 1u : 0u);
+          ring += (need_v ? 1u : 0u) + (need_k ? 1u : 0u);
+          const uint32_t vstage = vpos % C::NS, kstage = kpos % C::NS;
+          bool p_ready[2];
+          p_ready[0] = pend[0] && mbar_test(&bar_p_full[0], pcnt[0] & 1u);
+          const bool v_ready = need_v && mbar_test(&bar_kv_full[vstage], (vpos / C::NS) & 1u);
+          const bool k_ready = need_k && mbar_test(&bar_kv_full[kstage], (kpos / C::NS) & 1u);
+          p_ready[1] = false;
           bool have_k = false, have_v = false;
-          uint32_t kstage = 0, vstage = 0;
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
             if (!ok) break;
             if (pend[t]) {
-              if (!(ok = lane_wait(&bar_p_full[t], pcnt[t] & 1u, wc, kBarPFull, pcnt[t]))) break;
+              if (!p_ready[t] &&
+                  !(ok = lane_wait(&bar_p_full[t], pcnt[t] & 1u, wc, kBarPFull, pcnt[t])))
+                break;
               ++pcnt[t];
               if (first_pv[t] && items_t[t] > 0) {
                 if (!(ok = lane_wait(&bar_o_empty[t], (items_t[t] - 1) & 1u, wc, kBarOEmpty,
@@ -302,14 +321,14 @@ __global__ void __launch_bounds__(320, 1)
                   break;
               }
               if (!have_v) {
-                vstage = ring % C::NS;
-                if (!(ok = lane_wait(&bar_kv_full[vstage], (ring / C::NS) & 1u, wc, kBarKvFull,
-                                     ring)))
+                if (!v_ready && !(ok = lane_wait(&bar_kv_full[vstage], (vpos / C::NS) & 1u, wc,
+                                                 kBarKvFull, vpos)))
                   break;
-                ++ring;
                 have_v = true;
               }
               tc_fence_after();
+              // tile B's P, checked while tile A's MMAs go out
+              if (t == 0 && pend[1]) p_ready[1] = mbar_test(&bar_p_full[1], pcnt[1] & 1u);
               const uint32_t v_lo = (kv_base + vstage * (C::TILE_BYTES >> 4)) | kLboV;
 #pragma unroll
               for (int kk = 0; kk < BN / 16; ++kk)
@@ -318,15 +337,15 @@ __global__ void __launch_bounds__(320, 1)
                           (!first_pv[t] || kk > 0) ? 1u : 0u);
               first_pv[t] = false;
               pend[t] = false;
+            } else if (t == 0 && pend[1]) {
+              p_ready[1] = mbar_test(&bar_p_full[1], pcnt[1] & 1u);
             }
             if (more && in[t]) {
               if (!have_k) {
-                kstage = ring % C::NS;
-                if (!(ok = lane_wait(&bar_kv_full[kstage], (ring / C::NS) & 1u, wc, kBarKvFull,
-                                     ring)))
+                if (!k_ready && !(ok = lane_wait(&bar_kv_full[kstage], (kpos / C::NS) & 1u, wc,
+                                                 kBarKvFull, kpos)))
                   break;
                 tc_fence_after();
-                ++ring;
                 have_k = true;
               }
               const uint32_t q_lo = q_lo0 + t * (C::Q_BYTES >> 4);
