@@ -416,8 +416,10 @@ __global__ void __launch_bounds__(320, 1)
         }
         continue;
       }
-      ListCache lc;
-      lc.reset(p, a0, len);
+      // Lists are sorted, so only the row's last block can be the ragged
+      // final key block; its valid column count is taken once per item.
+      const int last_kb = min(max(__ldg(p.col_idx + a0 + len - 1), 0), p.nkb - 1);
+      const int last_valid = min(p.n - last_kb * BN, BN);
       float m_ref = 0.f, l = 0.f;
       for (int j = 0; j < len; ++j) {
         if (!(ok = warp_wait(&bar_s_full[t], scnt & 1u, wc, kBarSFull, scnt))) break;
@@ -436,8 +438,7 @@ __global__ void __launch_bounds__(320, 1)
             for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(sr[c][i]);
           }
         }
-        const int kb = lc.get(p, a0, len, j);
-        const int valid = p.n - kb * BN;
+        const int valid = j == len - 1 ? last_valid : BN;
         if (valid < BN) {
 #pragma unroll
           for (int c = 0; c < BN; ++c)

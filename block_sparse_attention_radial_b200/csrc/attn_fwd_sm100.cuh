@@ -94,7 +94,7 @@ struct WaitCtx {
 
 // Bounded parity wait. Returns false when the CTA is aborting or the limit ran
 // out (the first thread to run out records the timeout and raises the flag).
-__device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, const WaitCtx &w,
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, const WaitCtx &w,
                                           int bar_id, uint32_t counter) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
