@@ -119,6 +119,50 @@ __device__ __forceinline__ PairItem decode_pair(int idx, const FwdParams &p, int
   return it;
 }
 
+// Step plans: the producer, which walks the schedule anyway, writes one
+// 32-bit record per step into a small shared ring, so the MMA issuer reads
+// its step instead of walking the lists itself (the issuer's time between
+// MMA groups is tensor-pipe idle time). Record bits:
+//   1 PV of tile A, 2 QK of tile A, 3 PV of tile B, 4 QK of tile B,
+//   5 last step of the item, 8-10 V stage, 11 its fill parity,
+//   12-14 K stage, 15 its fill parity, 24-31 generation tag (never 0).
+// The producer runs at most a few steps ahead (it is held by the K/V ring and
+// by the Q buffers), far less than kPlanN steps, so a record is never
+// overwritten before it is read.
+constexpr int kPlanN = 32;
+
+__device__ __forceinline__ uint32_t plan_tag(uint32_t step) {
+  return ((step / kPlanN) & 0x7fu) + 1u;
+}
+
+// Bounded wait for step `step`'s record.
+__device__ __forceinline__ bool plan_wait(const volatile uint32_t *ring, uint32_t step,
+                                          uint32_t &rec, const WaitCtx &w) {
+  const volatile uint32_t *slot = ring + step % kPlanN;
+  const uint32_t tag = plan_tag(step);
+  rec = *slot;
+  if ((rec >> 24) == tag) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i) {
+      rec = *slot;
+      if ((rec >> 24) == tag) return true;
+    }
+    if (*w.abort) return false;
+    if (global_timer_ns() - t0 > w.limit) {
+      if (atomicCAS(&g_status, 0u, 4u /* BSA_ERR_DEVICE_TIMEOUT */) == 0u) {
+        g_status_detail[0] = w.role;
+        g_status_detail[1] = kBarPlan;
+        g_status_detail[2] = step;
+        g_status_detail[3] = blockIdx.x;
+      }
+      *w.abort = 1;
+      return false;
+    }
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(320, 1)
     attn_fwd_pair_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -133,6 +177,7 @@ __global__ void __launch_bounds__(320, 1)
   __shared__ __align__(8) uint64_t bar_s_full[2], bar_p_full[2], bar_o_final[2], bar_o_empty[2];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
+  __shared__ uint32_t plan_ring[kPlanN];
 
   const uint32_t raw = smem_addr(dsmem);
   uint8_t *base = dsmem + (((raw + 1023u) & ~1023u) - raw);
@@ -143,6 +188,7 @@ __global__ void __launch_bounds__(320, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  if (threadIdx.x < kPlanN) plan_ring[threadIdx.x] = 0u;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(&bar_kv_full[s], 1);
@@ -180,7 +226,8 @@ __global__ void __launch_bounds__(320, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      uint32_t ring = 0, qcount = 0;
+      uint32_t ring = 0, qcount = 0, gstep = 0;
+      volatile uint32_t *plans = plan_ring;
       bool skip_next_k = (p.fault_flags & 1) && blockIdx.x == 0;
       int skipped_ring = -1;
       bool ok = true;
@@ -209,6 +256,17 @@ __global__ void __launch_bounds__(320, 1)
           const bool need_v = pa || pb;
           if (!more && !need_v) break;
           const bool v_first = pa || !a;
+          {
+            const bool need_k = more;
+            const uint32_t vpos = ring + ((need_k && !v_first) ? 1u : 0u);
+            const uint32_t kpos = ring + ((need_v && v_first) ? 1u : 0u);
+            const uint32_t rec =
+                (pa ? 2u : 0u) | (a ? 4u : 0u) | (pb ? 8u : 0u) | (b ? 16u : 0u) |
+                (more ? 0u : 32u) | ((vpos % C::NS) << 8) | (((vpos / C::NS) & 1u) << 11) |
+                ((kpos % C::NS) << 12) | (((kpos / C::NS) & 1u) << 15) | (plan_tag(gstep) << 24);
+            plans[gstep % kPlanN] = rec;
+            ++gstep;
+          }
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const bool is_v = (e == 0) == v_first;
@@ -262,7 +320,9 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t kLboV = static_cast<uint32_t>(BN * 128 / 16) << 16;  // 64-wide D chunks
       const uint32_t q_lo0 = (smem_addr(sQ) >> 4) | kLboK;
       const uint32_t kv_base = smem_addr(sKV) >> 4;
-      uint32_t ring = 0, qcount = 0;
+      uint32_t gstep = 0, qcount = 0;
+      const volatile uint32_t *plans = plan_ring;
+      uint32_t rec_next = 0u;
       uint32_t pcnt[2] = {0u, 0u};     // p_full phases consumed, per tile
       uint32_t items_t[2] = {0u, 0u};  // items in which the tile had blocks
       bool ok = true;
@@ -275,42 +335,41 @@ __global__ void __launch_bounds__(320, 1)
         if (!(ok = lane_wait(&bar_q_full, qcount & 1u, wc, kBarQFull, qcount))) break;
         tc_fence_after();
         const int len_t[2] = {it.lenA, it.lenB};
-        UnionWalker uw;
-        uw.reset(p, it.a0, it.lenA, it.b0, it.lenB);
-        bool pend[2] = {false, false}, first_pv[2] = {true, true};
+        bool first_pv[2] = {true, true};
         bool q_released = false;
         while (ok) {
-          int kb = 0;
-          bool in[2] = {false, false};
-          const bool more = uw.next(kb, in[0], in[1]);
-          if (!more && !pend[0] && !pend[1]) break;
-          if (!more && !q_released) {  // no QK left in this item: the Q buffers may refill
+          // this step's record (usually already there: the producer runs ahead)
+          uint32_t rec = rec_next;
+          if ((rec >> 24) != plan_tag(gstep) && !(ok = plan_wait(plan_ring, gstep, rec, wc)))
+            break;
+          ++gstep;
+          const bool pv[2] = {(rec & 2u) != 0u, (rec & 8u) != 0u};
+          const bool qk[2] = {(rec & 4u) != 0u, (rec & 16u) != 0u};
+          const bool last = (rec & 32u) != 0u;
+          const uint32_t vstage = (rec >> 8) & 7u, vpar = (rec >> 11) & 1u;
+          const uint32_t kstage = (rec >> 12) & 7u, kpar = (rec >> 15) & 1u;
+          if (last && !q_released) {  // no QK left in this item: the Q buffers may refill
             mma_commit(&bar_q_empty);
             q_released = true;
           }
-          // Ring positions of this step's V(j-1) and K(j), in the producer's
-          // first-use order, and early non-blocking checks of their barriers
-          // and of tile A's P. A check of even a completed mbarrier takes
-          // about as long as two MMAs and the tensor pipe accepts one MMA at a
-          // time, so checks issued together (and ahead of the MMAs that
-          // precede their use) keep that latency off the tensor pipe.
-          const bool need_v = pend[0] || pend[1];
-          const bool need_k = more && (in[0] || in[1]);
-          const bool v_first = pend[0] || !in[0];
-          const uint32_t vpos = ring + ((need_k && !v_first) ? 1u : 0u);
-          const uint32_t kpos = ring + ((need_v && v_first) ? 1u : 0u);
-          ring += (need_v ? 1u : 0u) + (need_k ? 1u : 0u);
-          const uint32_t vstage = vpos % C::NS, kstage = kpos % C::NS;
+          // Early non-blocking checks of this step's barriers: a check of
+          // even a completed mbarrier takes about as long as two MMAs and the
+          // tensor pipe accepts one MMA at a time, so checks issued together
+          // (and ahead of the MMAs that precede their use) keep that latency
+          // off the tensor pipe.
+          const bool need_v = pv[0] || pv[1];
+          const bool need_k = qk[0] || qk[1];
           bool p_ready[2];
-          p_ready[0] = pend[0] && mbar_test(&bar_p_full[0], pcnt[0] & 1u);
-          const bool v_ready = need_v && mbar_test(&bar_kv_full[vstage], (vpos / C::NS) & 1u);
-          const bool k_ready = need_k && mbar_test(&bar_kv_full[kstage], (kpos / C::NS) & 1u);
+          p_ready[0] = pv[0] && mbar_test(&bar_p_full[0], pcnt[0] & 1u);
+          const bool v_ready = need_v && mbar_test(&bar_kv_full[vstage], vpar);
+          const bool k_ready = need_k && mbar_test(&bar_kv_full[kstage], kpar);
           p_ready[1] = false;
           bool have_k = false, have_v = false;
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
             if (!ok) break;
-            if (pend[t]) {
+            if (t == 1) rec_next = plans[gstep % kPlanN];  // next step's record, read ahead
+            if (pv[t]) {
               if (!p_ready[t] &&
                   !(ok = lane_wait(&bar_p_full[t], pcnt[t] & 1u, wc, kBarPFull, pcnt[t])))
                 break;
@@ -321,14 +380,14 @@ __global__ void __launch_bounds__(320, 1)
                   break;
               }
               if (!have_v) {
-                if (!v_ready && !(ok = lane_wait(&bar_kv_full[vstage], (vpos / C::NS) & 1u, wc,
-                                                 kBarKvFull, vpos)))
+                if (!v_ready &&
+                    !(ok = lane_wait(&bar_kv_full[vstage], vpar, wc, kBarKvFull, gstep)))
                   break;
                 have_v = true;
               }
               tc_fence_after();
               // tile B's P, checked while tile A's MMAs go out
-              if (t == 0 && pend[1]) p_ready[1] = mbar_test(&bar_p_full[1], pcnt[1] & 1u);
+              if (t == 0 && pv[1]) p_ready[1] = mbar_test(&bar_p_full[1], pcnt[1] & 1u);
               const uint32_t v_lo = (kv_base + vstage * (C::TILE_BYTES >> 4)) | kLboV;
 #pragma unroll
               for (int kk = 0; kk < BN / 16; ++kk)
@@ -336,14 +395,13 @@ __global__ void __launch_bounds__(320, 1)
                           v_lo + kk * (16 * 128 >> 4), kHi, idesc_pv,
                           (!first_pv[t] || kk > 0) ? 1u : 0u);
               first_pv[t] = false;
-              pend[t] = false;
-            } else if (t == 0 && pend[1]) {
+            } else if (t == 0 && pv[1]) {
               p_ready[1] = mbar_test(&bar_p_full[1], pcnt[1] & 1u);
             }
-            if (more && in[t]) {
+            if (qk[t]) {
               if (!have_k) {
-                if (!k_ready && !(ok = lane_wait(&bar_kv_full[kstage], (kpos / C::NS) & 1u, wc,
-                                                 kBarKvFull, kpos)))
+                if (!k_ready &&
+                    !(ok = lane_wait(&bar_kv_full[kstage], kpar, wc, kBarKvFull, gstep)))
                   break;
                 tc_fence_after();
                 have_k = true;
@@ -357,13 +415,12 @@ __global__ void __launch_bounds__(320, 1)
                           kk > 0 ? 1u : 0u);
               }
               mma_commit(&bar_s_full[t]);
-              pend[t] = true;
             }
           }
           if (!ok) break;
           if (have_k) mma_commit(&bar_kv_empty[kstage]);
           if (have_v) mma_commit(&bar_kv_empty[vstage]);
-          if (!more) break;
+          if (last) break;
         }
         if (!ok) break;
 #pragma unroll

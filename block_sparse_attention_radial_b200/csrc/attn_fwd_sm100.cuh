@@ -83,7 +83,7 @@ struct FwdCfg {
 enum : int { kRoleProducer = 1, kRoleMma = 2, kRoleSoftmax = 3 };
 enum : int {
   kBarKvFull = 1, kBarKvEmpty, kBarQFull, kBarQEmpty, kBarSFull, kBarPFull, kBarODone,
-  kBarOEmpty, kBarFinal, kBarSFree
+  kBarOEmpty, kBarFinal, kBarSFree, kBarPlan
 };
 
 struct WaitCtx {
