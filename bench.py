@@ -176,7 +176,7 @@ def blas_threads() -> int:
 
 def oracle_sample_rate(w, lists_host, q, k, v, budget_s: float, head: int = 0):
     """Time the CPU oracle on query rows of one head; returns (TFLOP/s, seconds,
-    rows, flops). Rows are a contiguous run from the middle of the sequence,
+    rows, flops). Rows are a contiguous run around the middle of the sequence,
     sized by a short calibration run to take about ``budget_s``."""
     import numpy as np
 
@@ -195,13 +195,16 @@ def oracle_sample_rate(w, lists_host, q, k, v, budget_s: float, head: int = 0):
         return f
 
     start = (w.n // 2) // w.block * w.block
-    cal = np.arange(start, min(w.n, start + 64))
+    cal = np.arange(start, min(w.n, start + 256))
     for _ in range(2):  # the first call pays one-time costs
         t0 = time.perf_counter()
         oracle.masked_attention_fp64(qh, kh, vh, rp, ci, 1, w.block, rows=cal)
         t_cal = max(time.perf_counter() - t0, 1e-3)
-    nrows = int(min(w.n - start, max(64, cal.size * budget_s / t_cal)))
-    rows = np.arange(start, start + nrows)
+    # a contiguous run centred on the middle of the sequence (all of head 0
+    # at most)
+    nrows = int(min(w.n, max(64, cal.size * budget_s / t_cal)))
+    first = max(0, min(w.n - nrows, w.n // 2 - nrows // 2))
+    rows = np.arange(first, first + nrows)
     t0 = time.perf_counter()
     oracle.masked_attention_fp64(qh, kh, vh, rp, ci, 1, w.block, rows=rows)
     dt = time.perf_counter() - t0
