@@ -23,6 +23,7 @@ Modules:
 * ``radial_mask``: the token-level radial rule and two independent block-list
   constructions (brute force over the token mask; per-token key intervals).
 * ``attention``: masked softmax attention over block lists, in float64.
+* ``attention_backward``: its gradients (dQ, dK, dV), in float64.
 """
 
 from .radial_mask import (  # noqa: F401
@@ -42,4 +43,9 @@ from .attention import (  # noqa: F401
     masked_attention_rows,
     masked_attention_fp64,
     bf16_round,
+)
+from .attention_backward import (  # noqa: F401
+    masked_attention_backward_fp64,
+    masked_attention_dq_rows,
+    masked_attention_dkdv_keys,
 )
