@@ -133,6 +133,27 @@ def bsa_attn_fwd_noalloc(q, k, v, lists: BlockLists, out, lse=None,
     _check(st, "bsa_attn_fwd_noalloc")
 
 
+def bsa_attn_bwd_workspace_bytes(batch: int, heads: int, n: int, lists: BlockLists) -> int:
+    return int(_lib.load().bsa_attn_bwd_workspace_bytes(batch, heads, n,
+                                                         ctypes.byref(lists.c_struct())))
+
+
+def bsa_attn_bwd(q, k, v, out, dout, lse, lists: BlockLists, dq, dk, dv, workspace=None,
+                 softmax_scale: float = 0.0, stream=None) -> None:
+    """Backward pass of :func:`bsa_attn_fwd` on the tensor cores (asynchronous)."""
+    B, H, n, D = q.shape
+    lib = _lib.load()
+    ls = lists.c_struct()
+    if workspace is None:
+        workspace = torch.empty(max(lib.bsa_attn_bwd_workspace_bytes(B, H, n, ctypes.byref(ls)), 16),
+                                dtype=torch.uint8, device=q.device)
+    st = lib.bsa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), B, H, n, D,
+                          float(softmax_scale), ctypes.byref(ls), _ptr(dq), _ptr(dk), _ptr(dv),
+                          _ptr(workspace), workspace.numel() * workspace.element_size(),
+                          _stream(stream))
+    _check(st, "bsa_attn_bwd")
+
+
 def bsa_attn_dense_masked_ref(q, k, v, lists: BlockLists, out, lse=None,
                               softmax_scale: float = 0.0, stream=None) -> None:
     """Same result from the plain fp32 CUDA-core reference kernel (asynchronous)."""
@@ -218,6 +239,14 @@ def attention(q, k, v, lists: BlockLists, softmax_scale: float = 0.0, want_lse: 
     lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device) if want_lse else None
     bsa_attn_fwd(q, k, v, lists, out, lse, workspace, softmax_scale, stream)
     return out, lse
+
+
+def attention_backward(q, k, v, out, dout, lse, lists: BlockLists, softmax_scale: float = 0.0,
+                       workspace=None, stream=None):
+    """Allocate gradients and run :func:`bsa_attn_bwd`; returns ``(dq, dk, dv)``."""
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    bsa_attn_bwd(q, k, v, out, dout, lse, lists, dq, dk, dv, workspace, softmax_scale, stream)
+    return dq, dk, dv
 
 
 def dense_masked_reference(q, k, v, lists: BlockLists, softmax_scale: float = 0.0, stream=None):

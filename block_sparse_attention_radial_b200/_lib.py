@@ -19,6 +19,8 @@ EXPORTS = (
     "bsa_attn_fwd_workspace_bytes",
     "bsa_attn_fwd",
     "bsa_attn_dense_masked_ref",
+    "bsa_attn_bwd",
+    "bsa_attn_bwd_workspace_bytes",
     "bsa_validate_lists",
     "bsa_get_device_status",
     "bsa_get_timeout_detail",
@@ -86,6 +88,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bsa_selftest_exp2": (ctypes.c_int, [vp, vp, vp, vp, i32, vp]),
         "bsa_attn_fwd_noalloc": (ctypes.c_int, [vp, vp, vp, i32, i32, i32, i32, ctypes.c_float,
                                                 lp, vp, vp, vp]),
+        "bsa_attn_bwd": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float,
+                                        lp, vp, vp, vp, vp, sz, vp]),
+        "bsa_attn_bwd_workspace_bytes": (sz, [i32, i32, i32, lp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

@@ -1,0 +1,813 @@
+// Block-sparse attention backward for sm_100a (block 128, head_dim 64/128).
+//
+// Gradients of O = softmax(Q K^T * scale restricted to the listed blocks) V,
+// given dO and the forward's lse (the derivative of the forward definition;
+// the pages fine-tune the radial attention module with LoRA, [RA-skill]
+// Step 4, which runs this pass):
+//   P = exp(S * scale - lse),  dV = P^T dO,  dP = dO V^T,
+//   delta_i = sum_d dO_id O_id,  dS = P * (dP - delta),
+//   dQ = dS K * scale,  dK = dS^T Q * scale.
+//
+// Three steps:
+//   bwd_prep_kernel    delta and lse * log2(e) per query row, padded to whole
+//                      blocks (padding: delta 0, lse +inf, so P = 0 there)
+//   csc_*_kernel       the lists transposed: per key block, its query blocks
+//                      in ascending order (deterministic accumulation order)
+//   attn_bwd_dkdv_kernel  one item = (batch*head, key block): K and V stay in
+//                      shared memory while the key block's query blocks
+//                      stream through; dK and dV accumulate in TMEM
+//   attn_bwd_dq_kernel    one item = (batch*head, query block): Q and dO stay
+//                      in shared memory while the row's key blocks stream
+//                      through; dQ accumulates in TMEM
+// No atomics: every output row is written once by one CTA, so the result is
+// deterministic. dQ recomputes S and dP (7 block products per listed block
+// instead of the 5 an atomic dQ needs).
+//
+// Both kernels use the forward's two MMA shapes (M128 N128 K16 with K-major
+// operands from shared memory; M128 N=D with A from TMEM and an MN-major B),
+// the same 4-D TMA boxes, and the same bounded waits (a timeout records
+// BSA_ERR_DEVICE_TIMEOUT, raises the CTA abort flag and every role leaves).
+#pragma once
+
+#include <climits>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "attn_fwd_sm100.cuh"
+#include "lists.cuh"
+
+namespace bsa {
+
+struct BwdParams {
+  const int32_t *row_ptr, *col_idx;  // lists: query block -> key blocks
+  const int32_t *col_ptr, *row_idx;  // transposed: key block -> query blocks
+  const float *lse2;                 // [bh][nqb * 128]: lse * log2(e), +inf padding
+  const float *delta;                // [bh][nqb * 128]: sum_d dO * O, 0 padding
+  __nv_bfloat16 *dq, *dk, *dv;
+  int32_t heads, n, nqb, nkb, num_lists, nnz;
+  int32_t total_items;
+  float scale, scale_log2;
+  unsigned long long wait_limit_ns;
+};
+
+constexpr int kBwdBlock = 128;
+
+// ------------------------------------------------------------------ prep --
+
+// One thread per padded query row of one (batch*head): delta and lse2.
+template <int D>
+__global__ void bwd_prep_kernel(const __nv_bfloat16 *out, const __nv_bfloat16 *dout,
+                                const float *lse, float *lse2, float *delta, int n, int nqb,
+                                long long rows_total) {
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= rows_total) return;
+  const long long padded = static_cast<long long>(nqb) * kBwdBlock;
+  const long long bh = idx / padded;
+  const int i = static_cast<int>(idx - bh * padded);
+  if (i >= n) {
+    lse2[idx] = INFINITY;
+    delta[idx] = 0.f;
+    return;
+  }
+  const long long row = bh * n + i;
+  const uint4 *o4 = reinterpret_cast<const uint4 *>(out + row * D);
+  const uint4 *d4 = reinterpret_cast<const uint4 *>(dout + row * D);
+  float acc = 0.f;
+#pragma unroll 4
+  for (int c = 0; c < D / 8; ++c) {
+    const uint4 a = o4[c], b = d4[c];
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&aw[w]));
+      const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&bw[w]));
+      acc = fmaf(fa.x, fb.x, acc);
+      acc = fmaf(fa.y, fb.y, acc);
+    }
+  }
+  delta[idx] = acc;
+  const float l = lse[row];
+  lse2[idx] = l > -INFINITY ? l * 1.4426950408889634f : INFINITY;
+}
+
+// ------------------------------------------------------- transposed lists --
+
+// True when the sorted row [a, b) of col_idx holds kb.
+__device__ __forceinline__ bool row_has(const int32_t *col_idx, int a, int b, int kb) {
+  while (a < b) {
+    const int m = (a + b) >> 1;
+    const int v = col_idx[m];
+    if (v == kb) return true;
+    if (v < kb) a = m + 1;
+    else b = m;
+  }
+  return false;
+}
+
+// One CTA per (list, key block): how many query blocks list it.
+__global__ void csc_count_kernel(const int32_t *row_ptr, const int32_t *col_idx, int nqb, int nkb,
+                                 int nnz, int32_t *col_cnt) {
+  __shared__ int scratch[32];
+  const int list = blockIdx.x / nkb, kb = blockIdx.x - list * nkb;
+  const int32_t *rp = row_ptr + static_cast<long long>(list) * nqb;
+  int c = 0;
+  for (int qb = threadIdx.x; qb < nqb; qb += blockDim.x) {
+    const int a = min(max(rp[qb], 0), nnz), b = min(max(rp[qb + 1], 0), nnz);
+    c += row_has(col_idx, a, b, kb) ? 1 : 0;
+  }
+  int total;
+  cta_inclusive_scan(c, scratch, total);
+  if (threadIdx.x == 0) col_cnt[blockIdx.x + 1] = total;
+  if (blockIdx.x == 0 && threadIdx.x == 0) col_cnt[0] = 0;
+}
+
+// One CTA per (list, key block): its query blocks in ascending order, at
+// col_ptr (the inclusive scan of the counts). Writes stay below `cap` (the
+// entries row_idx holds) even for lists the validator would reject.
+__global__ void csc_fill_kernel(const int32_t *row_ptr, const int32_t *col_idx, int nqb, int nkb,
+                                int nnz, const int32_t *col_ptr, int32_t *row_idx, int cap) {
+  __shared__ int scratch[32];
+  const int list = blockIdx.x / nkb, kb = blockIdx.x - list * nkb;
+  const int32_t *rp = row_ptr + static_cast<long long>(list) * nqb;
+  int base = col_ptr[blockIdx.x];
+  const int end = col_ptr[blockIdx.x + 1];
+  for (int q0 = 0; q0 < nqb; q0 += blockDim.x) {
+    const int qb = q0 + threadIdx.x;
+    bool has = false;
+    if (qb < nqb) {
+      const int a = min(max(rp[qb], 0), nnz), b = min(max(rp[qb + 1], 0), nnz);
+      has = row_has(col_idx, a, b, kb);
+    }
+    int total;
+    const int inc = cta_inclusive_scan(has ? 1 : 0, scratch, total);
+    const int pos = base + inc - 1;
+    if (has && pos >= 0 && pos < end && pos < cap) row_idx[pos] = qb;
+    base += total;
+  }
+}
+
+// 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16),
+// completing on `bar`'s transaction count.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,
+                                          uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// ------------------------------------------------------------ dK / dV --
+
+template <int D>
+struct DkdvCfg {
+  static constexpr int T = kBwdBlock * D * 2;        // one 128 x D bf16 tile
+  static constexpr int STAGE = 2 * T + 1024;         // Q, dO, lse2 and delta of a query block
+  static constexpr int NS_FIT = (kSmemLimit - 1024 - 1024 - 2 * T) / STAGE;
+  static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
+  static constexpr int DSMEM = 1024 + 2 * T + NS * STAGE;
+  static constexpr uint32_t ST_COL = 0;              // S^T, then P^T (bf16) over its first 64
+  static constexpr uint32_t DPT_COL = 128;           // dP^T, then dS^T (bf16) over its first 64
+  static constexpr uint32_t DV_COL = 256;
+  static constexpr uint32_t DK_COL = 256 + D;
+  static constexpr int THREADS = 192;
+  static_assert(NS >= 2, "stage ring needs two stages");
+};
+
+struct BwdItem {
+  int bh, blk, a, len;  // rows [a, a + len) of the (transposed) list
+};
+
+// Warps 0-3: elementwise (thread = key row = TMEM lane) and the dK/dV
+// epilogue; warp 4: TMA producer (lane 0); warp 5: MMA issuer (lane 0).
+// Per query block e of the key block's column, the MMA issuer runs
+//   S^T = K Q_e^T,  dP^T = V dO_e^T        (then the elementwise warps write
+//                                           P^T and dS^T as bf16 over them)
+//   dV += P^T dO_e, dK += dS^T Q_e         (issued before the next S^T, so the
+//                                           TMEM they read is not overwritten)
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
+                         const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v,
+                         const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+  using C = DkdvCfg<D>;
+  constexpr int BN = kBwdBlock;
+  extern __shared__ uint8_t dsmem[];
+  __shared__ __align__(8) uint64_t bar_st_full[C::NS], bar_st_empty[C::NS];
+  __shared__ __align__(8) uint64_t bar_kv_full, bar_kv_empty, bar_s_full, bar_p_full;
+  __shared__ __align__(8) uint64_t bar_acc_full, bar_acc_empty, bar_final;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const uint32_t raw = smem_addr(dsmem);
+  uint8_t *base = dsmem + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t *sK = base;
+  uint8_t *sV = base + C::T;
+  uint8_t *sStage = base + 2 * C::T;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long padded = static_cast<long long>(p.nqb) * BN;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(&bar_st_full[s], 1);
+      mbar_init(&bar_st_empty[s], 1);
+    }
+    mbar_init(&bar_kv_full, 1);
+    mbar_init(&bar_kv_empty, 1);
+    mbar_init(&bar_s_full, 1);
+    mbar_init(&bar_p_full, 128);
+    mbar_init(&bar_acc_full, 1);
+    mbar_init(&bar_acc_empty, 128);
+    mbar_init(&bar_final, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  WaitCtx wc{&abort_flag, p.wait_limit_ns, 0};
+
+  // Item k of this CTA: (batch*head, key block) and its column of the
+  // transposed lists.
+  auto decode = [&](int idx) {
+    BwdItem it;
+    it.bh = idx / p.nkb;
+    it.blk = idx - it.bh * p.nkb;
+    const int list = p.num_lists > 1 ? (it.bh % p.heads) : 0;
+    const long long c = static_cast<long long>(list) * p.nkb + it.blk;
+    const int a = min(max(p.col_ptr[c], 0), p.nnz), b = min(max(p.col_ptr[c + 1], 0), p.nnz);
+    it.a = a;
+    it.len = max(b - a, 0);
+    return it;
+  };
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      wc.role = kRoleProducer;
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      uint32_t ring = 0, kvcount = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int idx = snake_item(k, p.total_items);
+        if (idx == -2) break;
+        if (idx < 0) continue;
+        const BwdItem it = decode(idx);
+        if (it.len == 0) continue;
+        if (!(ok = lane_wait(&bar_kv_empty, (kvcount & 1u) ^ 1u, wc, kBarQEmpty, kvcount))) break;
+        mbar_arrive_expect_tx(&bar_kv_full, 2 * C::T);
+        tma_load_4d(sK, &tm_k, &bar_kv_full, 0, it.blk * BN, 0, it.bh);
+        tma_load_4d(sV, &tm_v, &bar_kv_full, 0, it.blk * BN, 0, it.bh);
+        ++kvcount;
+        for (int e = 0; e < it.len && ok; ++e) {
+          const int qb = min(max(__ldg(p.row_idx + it.a + e), 0), p.nqb - 1);
+          const uint32_t s = ring % C::NS;
+          if (!(ok = lane_wait(&bar_st_empty[s], ((ring / C::NS) & 1u) ^ 1u, wc, kBarKvEmpty,
+                               ring)))
+            break;
+          uint8_t *st = sStage + s * C::STAGE;
+          mbar_arrive_expect_tx(&bar_st_full[s], 2 * C::T + 1024);
+          tma_load_4d(st, &tm_q, &bar_st_full[s], 0, qb * BN, 0, it.bh);
+          tma_load_4d(st + C::T, &tm_do, &bar_st_full[s], 0, qb * BN, 0, it.bh);
+          const long long off = static_cast<long long>(it.bh) * padded + static_cast<long long>(qb) * BN;
+          bulk_load(st + 2 * C::T, p.lse2 + off, 512, &bar_st_full[s]);
+          bulk_load(st + 2 * C::T + 512, p.delta + off, 512, &bar_st_full[s]);
+          ++ring;
+        }
+      }
+      WaitCtx drain{&abort_flag, p.wait_limit_ns, kRoleProducer};
+      int zero = 0;
+      drain.abort = &zero;
+      const uint32_t first = ring > C::NS ? ring - C::NS : 0;
+      for (uint32_t r = first; r < ring; ++r)
+        wait_bounded(&bar_st_full[r % C::NS], (r / C::NS) & 1u, drain, kBarKvFull, r);
+      if (kvcount > 0) wait_bounded(&bar_kv_full, (kvcount - 1) & 1u, drain, kBarQFull, kvcount);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      wc.role = kRoleMma;
+      constexpr uint32_t idesc_ss = idesc_bf16_f32(128, BN, false);
+      constexpr uint32_t idesc_ts = idesc_bf16_f32(128, D, true);
+      constexpr uint32_t kHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+      constexpr uint32_t kLboK = 1u << 16;
+      constexpr uint32_t kLboMN = static_cast<uint32_t>(BN * 128 / 16) << 16;
+      const uint32_t k_lo = (smem_addr(sK) >> 4) | kLboK;
+      const uint32_t v_lo = (smem_addr(sV) >> 4) | kLboK;
+      const uint32_t st_base = smem_addr(sStage) >> 4;
+      uint32_t ring = 0, kvcount = 0, pcount = 0, items = 0;
+      bool ok = true;
+      // dV += P^T dO and dK += dS^T Q for the query block in stage `s`
+      auto issue_acc = [&](uint32_t s, bool first) {
+        const uint32_t q_mn = (st_base + s * (C::STAGE >> 4)) | kLboMN;
+        const uint32_t do_mn = (st_base + s * (C::STAGE >> 4) + (C::T >> 4)) | kLboMN;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts_lh(tmem + C::DV_COL, tmem + C::ST_COL + kk * 8, do_mn + kk * (16 * 128 >> 4),
+                    kHi, idesc_ts, (!first || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts_lh(tmem + C::DK_COL, tmem + C::DPT_COL + kk * 8, q_mn + kk * (16 * 128 >> 4),
+                    kHi, idesc_ts, (!first || kk > 0) ? 1u : 0u);
+        mma_commit(&bar_st_empty[s]);
+      };
+      for (int k = 0; ok; ++k) {
+        const int idx = snake_item(k, p.total_items);
+        if (idx == -2) break;
+        if (idx < 0) continue;
+        const BwdItem it = decode(idx);
+        if (it.len == 0) continue;
+        if (!(ok = lane_wait(&bar_kv_full, kvcount & 1u, wc, kBarQFull, kvcount))) break;
+        ++kvcount;
+        tc_fence_after();
+        bool first = true;
+        for (int e = 0; e < it.len; ++e) {
+          const uint32_t s = ring % C::NS;
+          if (!(ok = lane_wait(&bar_st_full[s], (ring / C::NS) & 1u, wc, kBarKvFull, ring))) break;
+          tc_fence_after();
+          if (e > 0) {  // accumulate the previous query block
+            if (!(ok = lane_wait(&bar_p_full, pcount & 1u, wc, kBarPFull, pcount))) break;
+            ++pcount;
+            tc_fence_after();
+            if (first && items > 0) {
+              if (!(ok = lane_wait(&bar_acc_empty, (items - 1) & 1u, wc, kBarOEmpty, items))) break;
+              tc_fence_after();
+            }
+            issue_acc((ring - 1) % C::NS, first);
+            first = false;
+          }
+          const uint32_t q_k = (st_base + s * (C::STAGE >> 4)) | kLboK;
+          const uint32_t do_k = (st_base + s * (C::STAGE >> 4) + (C::T >> 4)) | kLboK;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
+            mma_ss_lh(tmem + C::ST_COL, k_lo + off, kHi, q_k + off, kHi, idesc_ss, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
+            mma_ss_lh(tmem + C::DPT_COL, v_lo + off, kHi, do_k + off, kHi, idesc_ss,
+                      kk > 0 ? 1u : 0u);
+          }
+          if (e == it.len - 1) mma_commit(&bar_kv_empty);  // K and V read for the last time
+          mma_commit(&bar_s_full);
+          ++ring;
+        }
+        if (!ok) break;
+        if (!(ok = lane_wait(&bar_p_full, pcount & 1u, wc, kBarPFull, pcount))) break;
+        ++pcount;
+        tc_fence_after();
+        if (first && items > 0) {
+          if (!(ok = lane_wait(&bar_acc_empty, (items - 1) & 1u, wc, kBarOEmpty, items))) break;
+          tc_fence_after();
+        }
+        issue_acc((ring - 1) % C::NS, first);
+        mma_commit(&bar_acc_full);
+        ++items;
+      }
+      mma_commit(&bar_final);
+      WaitCtx drain{&abort_flag, p.wait_limit_ns, kRoleMma};
+      int zero = 0;
+      drain.abort = &zero;
+      wait_bounded(&bar_final, 0, drain, kBarFinal, items);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ elementwise + epilogue
+    wc.role = kRoleSoftmax;
+    const int r = warp * 32 + lane;  // key row within the tile = TMEM lane
+    const uint32_t lane_tmem = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const float sl2 = p.scale_log2;
+    uint32_t ring = 0, scount = 0, acount = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int idx = snake_item(k, p.total_items);
+      if (idx == -2) break;
+      if (idx < 0) continue;
+      const BwdItem it = decode(idx);
+      const int key = it.blk * BN + r;
+      const bool store = key < p.n;
+      const long long orow = static_cast<long long>(it.bh) * p.n + key;
+      if (it.len == 0) {  // no query attends these keys
+        if (store) {
+          uint4 *a = reinterpret_cast<uint4 *>(p.dk + orow * D);
+          uint4 *b = reinterpret_cast<uint4 *>(p.dv + orow * D);
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) {
+            a[c] = make_uint4(0, 0, 0, 0);
+            b[c] = make_uint4(0, 0, 0, 0);
+          }
+        }
+        continue;
+      }
+      for (int e = 0; e < it.len; ++e) {
+        const uint32_t s = ring % C::NS, spar = (ring / C::NS) & 1u;
+        ++ring;
+        if (!(ok = warp_wait(&bar_s_full, scount & 1u, wc, kBarSFull, scount))) break;
+        ++scount;
+        // the stage's lse2 / delta rows came by TMA: acquire them from the
+        // stage barrier itself (complete long before S^T is; the stage is
+        // not released before this warp's P arrives)
+        if (!(ok = warp_wait(&bar_st_full[s], spar, wc, kBarKvFull, ring))) break;
+        tc_fence_after();
+        const float *lse_s = reinterpret_cast<const float *>(sStage + s * C::STAGE + 2 * C::T);
+        const float *del_s = lse_s + 128;
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t sr[32], dr[32];
+          tmem_ld32(lane_tmem + C::ST_COL + c * 32, sr);
+          tmem_ld32(lane_tmem + C::DPT_COL + c * 32, dr);
+          tmem_wait_ld();
+          reg_fence32(sr);
+          reg_fence32(dr);
+          uint32_t pk[16], dk16[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float4 l4 = *reinterpret_cast<const float4 *>(lse_s + c * 32 + (i & ~1) * 2);
+            const float4 d4 = *reinterpret_cast<const float4 *>(del_s + c * 32 + (i & ~1) * 2);
+            const float la = (i & 1) ? l4.z : l4.x, lb = (i & 1) ? l4.w : l4.y;
+            const float da = (i & 1) ? d4.z : d4.x, db = (i & 1) ? d4.w : d4.y;
+            const float pa = ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -la));
+            const float pb = ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -lb));
+            const float ga = pa * (__uint_as_float(dr[2 * i]) - da);
+            const float gb = pb * (__uint_as_float(dr[2 * i + 1]) - db);
+            pk[i] = pack_bf16x2(pa, pb);
+            dk16[i] = pack_bf16x2(ga, gb);
+          }
+          // chunk c lands on columns [16c, 16c + 16): already read back
+          tmem_st16(lane_tmem + C::ST_COL + c * 16, pk);
+          tmem_st16(lane_tmem + C::DPT_COL + c * 16, dk16);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar_p_full);
+      }
+      if (!ok) break;
+      // epilogue: dV and dK (times scale) of this key row
+      if (!(ok = warp_wait(&bar_acc_full, acount & 1u, wc, kBarODone, acount))) break;
+      ++acount;
+      tc_fence_after();
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        const uint32_t col = part == 0 ? C::DV_COL : C::DK_COL;
+        const float mul = part == 0 ? 1.f : p.scale;
+        __nv_bfloat16 *dst = part == 0 ? p.dv : p.dk;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(lane_tmem + col + c * 32, v);
+          tmem_wait_ld();
+          reg_fence32(v);
+          if (store) {
+            uint4 *o4 = reinterpret_cast<uint4 *>(dst + orow * D + c * 32);
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              uint4 x;
+              x.x = pack_bf16x2(__uint_as_float(v[8 * w + 0]) * mul, __uint_as_float(v[8 * w + 1]) * mul);
+              x.y = pack_bf16x2(__uint_as_float(v[8 * w + 2]) * mul, __uint_as_float(v[8 * w + 3]) * mul);
+              x.z = pack_bf16x2(__uint_as_float(v[8 * w + 4]) * mul, __uint_as_float(v[8 * w + 5]) * mul);
+              x.w = pack_bf16x2(__uint_as_float(v[8 * w + 6]) * mul, __uint_as_float(v[8 * w + 7]) * mul);
+              o4[w] = x;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar_acc_empty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ dQ --
+
+template <int D>
+struct DqCfg {
+  static constexpr int T = kBwdBlock * D * 2;
+  static constexpr int STAGE = 2 * T;                // K and V of a key block
+  static constexpr int NS_FIT = (kSmemLimit - 1024 - 1024 - 2 * T) / STAGE;
+  static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
+  static constexpr int DSMEM = 1024 + 2 * T + NS * STAGE;
+  static constexpr uint32_t S_COL = 0;               // S (scores), read back
+  static constexpr uint32_t DP_COL = 128;            // dP, then dS (bf16) over its first 64
+  static constexpr uint32_t DQ_COL = 256;
+  static constexpr int THREADS = 192;
+  static_assert(NS >= 2, "stage ring needs two stages");
+};
+
+// Warps 0-3: elementwise (thread = query row = TMEM lane) and the dQ
+// epilogue; warp 4: TMA producer (lane 0); warp 5: MMA issuer (lane 0).
+// Per key block e of the row:  S = Q K_e^T, dP = dO V_e^T, the elementwise
+// warps write dS (bf16) over dP, then dQ += dS K_e (issued before the next
+// S, so the TMEM it reads is not overwritten).
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+  using C = DqCfg<D>;
+  constexpr int BN = kBwdBlock;
+  extern __shared__ uint8_t dsmem[];
+  __shared__ __align__(8) uint64_t bar_st_full[C::NS], bar_st_empty[C::NS];
+  __shared__ __align__(8) uint64_t bar_qd_full, bar_qd_empty, bar_s_full, bar_p_full;
+  __shared__ __align__(8) uint64_t bar_acc_full, bar_acc_empty, bar_final;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const uint32_t raw = smem_addr(dsmem);
+  uint8_t *base = dsmem + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t *sQ = base;
+  uint8_t *sDO = base + C::T;
+  uint8_t *sStage = base + 2 * C::T;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long padded = static_cast<long long>(p.nqb) * BN;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(&bar_st_full[s], 1);
+      mbar_init(&bar_st_empty[s], 1);
+    }
+    mbar_init(&bar_qd_full, 1);
+    mbar_init(&bar_qd_empty, 1);
+    mbar_init(&bar_s_full, 1);
+    mbar_init(&bar_p_full, 128);
+    mbar_init(&bar_acc_full, 1);
+    mbar_init(&bar_acc_empty, 128);
+    mbar_init(&bar_final, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  WaitCtx wc{&abort_flag, p.wait_limit_ns, 0};
+
+  auto decode = [&](int idx) {
+    BwdItem it;
+    it.bh = idx / p.nqb;
+    it.blk = idx - it.bh * p.nqb;
+    const int list = p.num_lists > 1 ? (it.bh % p.heads) : 0;
+    const long long r = static_cast<long long>(list) * p.nqb + it.blk;
+    const int a = min(max(p.row_ptr[r], 0), p.nnz), b = min(max(p.row_ptr[r + 1], 0), p.nnz);
+    it.a = a;
+    it.len = max(b - a, 0);
+    return it;
+  };
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      wc.role = kRoleProducer;
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      uint32_t ring = 0, qdcount = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int idx = snake_item(k, p.total_items);
+        if (idx == -2) break;
+        if (idx < 0) continue;
+        const BwdItem it = decode(idx);
+        if (it.len == 0) continue;
+        if (!(ok = lane_wait(&bar_qd_empty, (qdcount & 1u) ^ 1u, wc, kBarQEmpty, qdcount))) break;
+        mbar_arrive_expect_tx(&bar_qd_full, 2 * C::T);
+        tma_load_4d(sQ, &tm_q, &bar_qd_full, 0, it.blk * BN, 0, it.bh);
+        tma_load_4d(sDO, &tm_do, &bar_qd_full, 0, it.blk * BN, 0, it.bh);
+        ++qdcount;
+        for (int e = 0; e < it.len && ok; ++e) {
+          const int kb = min(max(__ldg(p.col_idx + it.a + e), 0), p.nkb - 1);
+          const uint32_t s = ring % C::NS;
+          if (!(ok = lane_wait(&bar_st_empty[s], ((ring / C::NS) & 1u) ^ 1u, wc, kBarKvEmpty,
+                               ring)))
+            break;
+          uint8_t *st = sStage + s * C::STAGE;
+          mbar_arrive_expect_tx(&bar_st_full[s], 2 * C::T);
+          tma_load_4d(st, &tm_k, &bar_st_full[s], 0, kb * BN, 0, it.bh);
+          tma_load_4d(st + C::T, &tm_v, &bar_st_full[s], 0, kb * BN, 0, it.bh);
+          ++ring;
+        }
+      }
+      WaitCtx drain{&abort_flag, p.wait_limit_ns, kRoleProducer};
+      int zero = 0;
+      drain.abort = &zero;
+      const uint32_t first = ring > C::NS ? ring - C::NS : 0;
+      for (uint32_t r = first; r < ring; ++r)
+        wait_bounded(&bar_st_full[r % C::NS], (r / C::NS) & 1u, drain, kBarKvFull, r);
+      if (qdcount > 0) wait_bounded(&bar_qd_full, (qdcount - 1) & 1u, drain, kBarQFull, qdcount);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      wc.role = kRoleMma;
+      constexpr uint32_t idesc_ss = idesc_bf16_f32(128, BN, false);
+      constexpr uint32_t idesc_ts = idesc_bf16_f32(128, D, true);
+      constexpr uint32_t kHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+      constexpr uint32_t kLboK = 1u << 16;
+      constexpr uint32_t kLboMN = static_cast<uint32_t>(BN * 128 / 16) << 16;
+      const uint32_t q_lo = (smem_addr(sQ) >> 4) | kLboK;
+      const uint32_t do_lo = (smem_addr(sDO) >> 4) | kLboK;
+      const uint32_t st_base = smem_addr(sStage) >> 4;
+      uint32_t ring = 0, qdcount = 0, pcount = 0, items = 0;
+      bool ok = true;
+      // dQ += dS K for the key block in stage `s`
+      auto issue_acc = [&](uint32_t s, bool first) {
+        const uint32_t k_mn = (st_base + s * (C::STAGE >> 4)) | kLboMN;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts_lh(tmem + C::DQ_COL, tmem + C::DP_COL + kk * 8, k_mn + kk * (16 * 128 >> 4),
+                    kHi, idesc_ts, (!first || kk > 0) ? 1u : 0u);
+        mma_commit(&bar_st_empty[s]);
+      };
+      for (int k = 0; ok; ++k) {
+        const int idx = snake_item(k, p.total_items);
+        if (idx == -2) break;
+        if (idx < 0) continue;
+        const BwdItem it = decode(idx);
+        if (it.len == 0) continue;
+        if (!(ok = lane_wait(&bar_qd_full, qdcount & 1u, wc, kBarQFull, qdcount))) break;
+        ++qdcount;
+        tc_fence_after();
+        bool first = true;
+        for (int e = 0; e < it.len; ++e) {
+          const uint32_t s = ring % C::NS;
+          if (!(ok = lane_wait(&bar_st_full[s], (ring / C::NS) & 1u, wc, kBarKvFull, ring))) break;
+          tc_fence_after();
+          if (e > 0) {
+            if (!(ok = lane_wait(&bar_p_full, pcount & 1u, wc, kBarPFull, pcount))) break;
+            ++pcount;
+            tc_fence_after();
+            if (first && items > 0) {
+              if (!(ok = lane_wait(&bar_acc_empty, (items - 1) & 1u, wc, kBarOEmpty, items))) break;
+              tc_fence_after();
+            }
+            issue_acc((ring - 1) % C::NS, first);
+            first = false;
+          }
+          const uint32_t k_k = (st_base + s * (C::STAGE >> 4)) | kLboK;
+          const uint32_t v_k = (st_base + s * (C::STAGE >> 4) + (C::T >> 4)) | kLboK;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
+            mma_ss_lh(tmem + C::S_COL, q_lo + off, kHi, k_k + off, kHi, idesc_ss, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
+            mma_ss_lh(tmem + C::DP_COL, do_lo + off, kHi, v_k + off, kHi, idesc_ss,
+                      kk > 0 ? 1u : 0u);
+          }
+          if (e == it.len - 1) mma_commit(&bar_qd_empty);  // Q and dO read for the last time
+          mma_commit(&bar_s_full);
+          ++ring;
+        }
+        if (!ok) break;
+        if (!(ok = lane_wait(&bar_p_full, pcount & 1u, wc, kBarPFull, pcount))) break;
+        ++pcount;
+        tc_fence_after();
+        if (first && items > 0) {
+          if (!(ok = lane_wait(&bar_acc_empty, (items - 1) & 1u, wc, kBarOEmpty, items))) break;
+          tc_fence_after();
+        }
+        issue_acc((ring - 1) % C::NS, first);
+        mma_commit(&bar_acc_full);
+        ++items;
+      }
+      mma_commit(&bar_final);
+      WaitCtx drain{&abort_flag, p.wait_limit_ns, kRoleMma};
+      int zero = 0;
+      drain.abort = &zero;
+      wait_bounded(&bar_final, 0, drain, kBarFinal, items);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ elementwise + epilogue
+    wc.role = kRoleSoftmax;
+    const int r = warp * 32 + lane;  // query row within the tile = TMEM lane
+    const uint32_t lane_tmem = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const float sl2 = p.scale_log2;
+    uint32_t scount = 0, acount = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int idx = snake_item(k, p.total_items);
+      if (idx == -2) break;
+      if (idx < 0) continue;
+      const BwdItem it = decode(idx);
+      const int row = it.blk * BN + r;
+      const bool store = row < p.n;
+      const long long orow = static_cast<long long>(it.bh) * p.n + row;
+      if (it.len == 0) {  // no key: dQ = 0
+        if (store) {
+          uint4 *a = reinterpret_cast<uint4 *>(p.dq + orow * D);
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) a[c] = make_uint4(0, 0, 0, 0);
+        }
+        continue;
+      }
+      const long long prow = static_cast<long long>(it.bh) * padded + static_cast<long long>(it.blk) * BN + r;
+      const float lse2 = p.lse2[prow], del = p.delta[prow];
+      // lists are sorted: only the row's last block can be the ragged final
+      // key block (its columns >= n hold zero keys; they are masked out)
+      const int last_kb = min(max(__ldg(p.col_idx + it.a + it.len - 1), 0), p.nkb - 1);
+      const int last_valid = min(p.n - last_kb * BN, BN);
+      for (int e = 0; e < it.len; ++e) {
+        if (!(ok = warp_wait(&bar_s_full, scount & 1u, wc, kBarSFull, scount))) break;
+        ++scount;
+        tc_fence_after();
+        const int valid = e == it.len - 1 ? last_valid : BN;
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t sr[32], dr[32];
+          tmem_ld32(lane_tmem + C::S_COL + c * 32, sr);
+          tmem_ld32(lane_tmem + C::DP_COL + c * 32, dr);
+          tmem_wait_ld();
+          reg_fence32(sr);
+          reg_fence32(dr);
+          uint32_t g16[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int col = c * 32 + 2 * i;
+            float pa = ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -lse2));
+            float pb = ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -lse2));
+            if (valid < BN) {
+              pa = col < valid ? pa : 0.f;
+              pb = col + 1 < valid ? pb : 0.f;
+            }
+            g16[i] = pack_bf16x2(pa * (__uint_as_float(dr[2 * i]) - del),
+                                 pb * (__uint_as_float(dr[2 * i + 1]) - del));
+          }
+          // chunk c lands on dP columns [16c, 16c + 16): already read back
+          tmem_st16(lane_tmem + C::DP_COL + c * 16, g16);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar_p_full);
+      }
+      if (!ok) break;
+      if (!(ok = warp_wait(&bar_acc_full, acount & 1u, wc, kBarODone, acount))) break;
+      ++acount;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(lane_tmem + C::DQ_COL + c * 32, v);
+        tmem_wait_ld();
+        reg_fence32(v);
+        if (store) {
+          const float mul = p.scale;
+          uint4 *o4 = reinterpret_cast<uint4 *>(p.dq + orow * D + c * 32);
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            uint4 x;
+            x.x = pack_bf16x2(__uint_as_float(v[8 * w + 0]) * mul, __uint_as_float(v[8 * w + 1]) * mul);
+            x.y = pack_bf16x2(__uint_as_float(v[8 * w + 2]) * mul, __uint_as_float(v[8 * w + 3]) * mul);
+            x.z = pack_bf16x2(__uint_as_float(v[8 * w + 4]) * mul, __uint_as_float(v[8 * w + 5]) * mul);
+            x.w = pack_bf16x2(__uint_as_float(v[8 * w + 6]) * mul, __uint_as_float(v[8 * w + 7]) * mul);
+            o4[w] = x;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar_acc_empty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace bsa

@@ -15,6 +15,7 @@
 
 #include "bsa.h"
 
+#include "attn_bwd_sm100.cuh"
 #include "attn_fwd_pair_sm100.cuh"
 #include "attn_fwd_sm100.cuh"
 #include "dense_ref.cuh"
@@ -48,7 +49,8 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   bool probed = false;
   int cc_major = 0, cc_minor = 0, sms = 0;
-  bool attrs_set[8] = {false, false, false, false, false, false, false, false};
+  bool attrs_set[12] = {false, false, false, false, false, false,
+                       false, false, false, false, false, false};
   bool ref_attrs_set[4] = {false, false, false, false};
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -285,6 +287,109 @@ int run_fwd(const void *q, const void *k, const void *v, int32_t batch, int32_t 
   return launch_fwd<64, 64>(q, k, v, bh, n, p, dev, slot, stream);
 }
 
+// ---------------------------------------------------------------- backward
+
+// Workspace of the backward pass: lse2 and delta per padded query row, then
+// the transposed lists. Offsets are 256-byte aligned (the bulk copies of
+// lse2 / delta rows need 16-byte aligned 512-byte rows).
+struct BwdLayout {
+  size_t lse2, delta, col_ptr, row_idx, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+BwdLayout bwd_layout(int32_t batch, int32_t heads, const bsa_block_lists *l) {
+  BwdLayout w;
+  const size_t rows = static_cast<size_t>(batch) * heads * l->num_q_blocks * kBwdBlock;
+  w.lse2 = 0;
+  w.delta = align256(rows * sizeof(float));
+  w.col_ptr = w.delta + align256(rows * sizeof(float));
+  w.row_idx = w.col_ptr +
+              align256((static_cast<size_t>(l->num_lists) * l->num_k_blocks + 1) * sizeof(int32_t));
+  w.total = w.row_idx + align256(static_cast<size_t>(l->nnz > 0 ? l->nnz : 1) * sizeof(int32_t));
+  return w;
+}
+
+template <int D>
+int launch_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout,
+               const float *lse, int32_t bh, int32_t n, float softmax_scale,
+               const bsa_block_lists *l, void *dq, void *dk, void *dv, uint8_t *ws,
+               DeviceInfo *dev, cudaStream_t stream) {
+  const BwdLayout w = bwd_layout(1, bh, l);
+  float *lse2 = reinterpret_cast<float *>(ws + w.lse2);
+  float *delta = reinterpret_cast<float *>(ws + w.delta);
+  int32_t *col_ptr = reinterpret_cast<int32_t *>(ws + w.col_ptr);
+  int32_t *row_idx = reinterpret_cast<int32_t *>(ws + w.row_idx);
+  const int nqb = l->num_q_blocks, nkb = l->num_k_blocks;
+
+  const long long rows = static_cast<long long>(bh) * nqb * kBwdBlock;
+  bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 255) / 256), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16 *>(out), static_cast<const __nv_bfloat16 *>(dout), lse,
+      lse2, delta, n, nqb, rows);
+  BSA_CUDA(cudaGetLastError());
+  const int cols = l->num_lists * nkb;
+  csc_count_kernel<<<cols, 256, 0, stream>>>(l->row_ptr, l->col_idx, nqb, nkb, l->nnz, col_ptr);
+  BSA_CUDA(cudaGetLastError());
+  scan_rows_kernel<<<1, 1024, 0, stream>>>(col_ptr, cols);
+  BSA_CUDA(cudaGetLastError());
+  csc_fill_kernel<<<cols, 256, 0, stream>>>(l->row_ptr, l->col_idx, nqb, nkb, l->nnz, col_ptr,
+                                            row_idx, l->nnz);
+  BSA_CUDA(cudaGetLastError());
+
+  CUtensorMap tq, tk, tv, td;
+  int st;
+  if ((st = make_map(&tq, q, bh, n, D, kBwdBlock)) != BSA_OK) return st;
+  if ((st = make_map(&tk, k, bh, n, D, kBwdBlock)) != BSA_OK) return st;
+  if ((st = make_map(&tv, v, bh, n, D, kBwdBlock)) != BSA_OK) return st;
+  if ((st = make_map(&td, dout, bh, n, D, kBwdBlock)) != BSA_OK) return st;
+  const int slot = 8 + (D == 128 ? 2 : 0);
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!dev->attrs_set[slot]) {
+      BSA_CUDA(cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    DkdvCfg<D>::DSMEM));
+      BSA_CUDA(cudaFuncSetAttribute(attn_bwd_dq_kernel<D>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    DqCfg<D>::DSMEM));
+      dev->attrs_set[slot] = true;
+    }
+  }
+  BwdParams p;
+  p.row_ptr = l->row_ptr;
+  p.col_idx = l->col_idx;
+  p.col_ptr = col_ptr;
+  p.row_idx = row_idx;
+  p.lse2 = lse2;
+  p.delta = delta;
+  p.dq = static_cast<__nv_bfloat16 *>(dq);
+  p.dk = static_cast<__nv_bfloat16 *>(dk);
+  p.dv = static_cast<__nv_bfloat16 *>(dv);
+  p.heads = l->num_lists > 1 ? l->num_lists : 1;
+  p.n = n;
+  p.nqb = nqb;
+  p.nkb = nkb;
+  p.num_lists = l->num_lists;
+  p.nnz = l->nnz;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(D));
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  {
+    std::lock_guard<std::mutex> lk(g_hook_mu);
+    p.wait_limit_ns = g_wait_limit_ns;
+  }
+  p.total_items = bh * nkb;
+  int grid = p.total_items < dev->sms ? p.total_items : dev->sms;
+  attn_bwd_dkdv_kernel<D><<<grid, DkdvCfg<D>::THREADS, DkdvCfg<D>::DSMEM, stream>>>(tq, tk, tv,
+                                                                                     td, p);
+  BSA_CUDA(cudaGetLastError());
+  p.total_items = bh * nqb;
+  grid = p.total_items < dev->sms ? p.total_items : dev->sms;
+  attn_bwd_dq_kernel<D><<<grid, DqCfg<D>::THREADS, DqCfg<D>::DSMEM, stream>>>(tq, tk, tv, td, p);
+  BSA_CUDA(cudaGetLastError());
+  return BSA_OK;
+}
+
 // Self-test of the two exp2 paths of the attention softmax against exp2f.
 __global__ void exp2_selftest_kernel(const float *x, float *y_poly, float *y_mufu,
                                      float *y_ref, int n) {
@@ -375,6 +480,55 @@ int bsa_attn_fwd(const void *q, const void *k, const void *v, int32_t batch, int
   }
   return run_fwd(q, k, v, batch, heads, n, head_dim, softmax_scale, l, out, lse,
                  static_cast<int32_t *>(workspace), dev, fault_flags, stream);
+}
+
+size_t bsa_attn_bwd_workspace_bytes(int32_t batch, int32_t heads, int32_t n,
+                                    const bsa_block_lists *l) {
+  if (!l || batch < 1 || heads < 1 || n < 1 || l->num_q_blocks < 1 || l->num_k_blocks < 1)
+    return 0;
+  if (l->num_lists != 1 && l->num_lists != heads) return 0;
+  if (l->block != kBwdBlock || l->num_q_blocks != ceil_div(n, l->block)) return 0;
+  return bwd_layout(batch, heads, l).total;
+}
+
+int bsa_attn_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout,
+                 const float *lse, int32_t batch, int32_t heads, int32_t n, int32_t head_dim,
+                 float softmax_scale, const bsa_block_lists *l, void *dq, void *dk, void *dv,
+                 void *workspace, size_t workspace_bytes, bsa_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int st = check_attn_args(q, k, v, batch, heads, n, head_dim, l, dq);
+  if (st != BSA_OK) return st;
+  if (l->block != kBwdBlock) return BSA_ERR_UNSUPPORTED;
+  if (!out || !dout || !lse || !dk || !dv) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(dout) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return BSA_ERR_INVALID_ARG;
+  const size_t bytes = static_cast<size_t>(batch) * heads * n * head_dim * 2;
+  const size_t lbytes = static_cast<size_t>(batch) * heads * n * sizeof(float);
+  const void *ins[6] = {q, k, v, out, dout, lse};
+  const size_t in_bytes[6] = {bytes, bytes, bytes, bytes, bytes, lbytes};
+  void *outs[3] = {dq, dk, dv};
+  for (int a = 0; a < 3; ++a) {
+    for (int b = 0; b < 6; ++b)
+      if (overlaps(outs[a], bytes, ins[b], in_bytes[b])) return BSA_ERR_INVALID_ARG;
+    for (int b = a + 1; b < 3; ++b)
+      if (overlaps(outs[a], bytes, outs[b], bytes)) return BSA_ERR_INVALID_ARG;
+  }
+  const size_t need = bwd_layout(batch, heads, l).total;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < need) return BSA_ERR_INVALID_ARG;
+  if (overlaps(workspace, need, ins[0], bytes) || overlaps(workspace, need, dq, bytes) ||
+      overlaps(workspace, need, dk, bytes) || overlaps(workspace, need, dv, bytes))
+    return BSA_ERR_INVALID_ARG;
+  DeviceInfo *dev = nullptr;
+  if ((st = current_device(&dev)) != BSA_OK) return st;
+  if (dev->cc_major != 10) return BSA_ERR_UNSUPPORTED;
+  const int32_t bh = batch * heads;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  if (head_dim == 128)
+    return launch_bwd<128>(q, k, v, out, dout, lse, bh, n, softmax_scale, l, dq, dk, dv, ws, dev,
+                           stream);
+  return launch_bwd<64>(q, k, v, out, dout, lse, bh, n, softmax_scale, l, dq, dk, dv, ws, dev,
+                        stream);
 }
 
 int bsa_attn_dense_masked_ref(const void *q, const void *k, const void *v, int32_t batch,

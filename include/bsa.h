@@ -153,6 +153,44 @@ int bsa_attn_dense_masked_ref(const void *q, const void *k, const void *v,
                               void *out, float *lse, bsa_stream_t stream);
 
 /*
+ * Backward pass of bsa_attn_fwd: the gradients dq, dk, dv of the attention
+ * output with respect to q, k and v, given the output's gradient dout. The
+ * pages fine-tune the radial attention module with LoRA for longer
+ * sequences ("Radial Attention" skill page, Step 4, `loss.backward()`);
+ * this is the derivative of the forward definition, which the pages do not
+ * print:
+ *   P = softmax(Q K^T * scale over the listed blocks),  dV = P^T dO,
+ *   dP = dO V^T,  delta_i = sum_d dO_id O_id,  dS = P * (dP - delta),
+ *   dQ = dS K * scale,  dK = dS^T Q * scale.
+ *
+ * Arguments: q, k, v, out (the forward's output) and dout: bf16
+ * [batch, heads, n, head_dim] contiguous, 16-byte aligned device pointers; lse:
+ * the forward's fp32 [batch, heads, n] log-sum-exp (required); lists and
+ * softmax_scale exactly as given to the forward call; dq, dk, dv: bf16
+ * [batch, heads, n, head_dim] outputs, 16-byte aligned, written in full (rows
+ * of query blocks with no key block get dq = 0, keys no query block lists get
+ * dk = dv = 0), and not overlapping any input. workspace: device scratch of
+ * at least bsa_attn_bwd_workspace_bytes() bytes, 16-byte aligned, owned by the
+ * caller. Supported: block 128, head_dim 64 or 128 (block 64 returns
+ * BSA_ERR_UNSUPPORTED). Deterministic: every output row is written by one
+ * CTA, no atomics. Asynchronous on `stream`; device timeouts are reported
+ * through bsa_get_device_status(). Returns BSA_OK or an argument / CUDA error.
+ */
+int bsa_attn_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout,
+                 const float *lse, int32_t batch, int32_t heads, int32_t n, int32_t head_dim,
+                 float softmax_scale, const bsa_block_lists *lists, void *dq, void *dk, void *dv,
+                 void *workspace, size_t workspace_bytes, bsa_stream_t stream);
+
+/*
+ * Workspace bytes bsa_attn_bwd needs: per query row of every (batch, head),
+ * lse * log2(e) and delta, padded to whole blocks (2 x 4 bytes), plus the
+ * transposed lists (num_lists * num_k_blocks + 1 offsets, nnz entries).
+ * 0 when the arguments are invalid.
+ */
+size_t bsa_attn_bwd_workspace_bytes(int32_t batch, int32_t heads, int32_t n,
+                                    const bsa_block_lists *lists);
+
+/*
  * Check `lists`: row_ptr starts at 0, is non-decreasing and ends at nnz; each
  * row is strictly increasing and in [0, num_k_blocks). Reads no col_idx entry
  * at or beyond nnz. Synchronises `stream`. Returns BSA_OK, BSA_ERR_BAD_LISTS

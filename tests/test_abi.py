@@ -94,3 +94,37 @@ def test_mask_build_argument_checks(lib):
     assert lib.bsa_radial_mask_build(1 << 16, 1 << 16, 128, vp(1 << 20), None, 0, None, None) == 1
     assert lib.bsa_set_test_hooks(-1, 0) == 1
     assert lib.bsa_set_test_hooks(0, 0) == 0
+
+
+def test_backward_workspace_and_host_checks(lib):
+    from block_sparse_attention_radial_b200._lib import BlockListsC
+
+    ls = BlockListsC(1, 256, 256, 128, 1000, 0, 0)
+    # lse2 + delta: 2 x 40 x 256 x 128 floats; offsets 257 ints; 1000 entries
+    expect = 2 * 40 * 256 * 128 * 4 + 1280 + 4096
+    assert lib.bsa_attn_bwd_workspace_bytes(1, 40, 32760, ctypes.byref(ls)) == expect
+    assert lib.bsa_attn_bwd_workspace_bytes(1, 40, 32769, ctypes.byref(ls)) == 0  # nqb mismatch
+    ls64 = BlockListsC(1, 512, 512, 64, 1000, 0, 0)
+    assert lib.bsa_attn_bwd_workspace_bytes(1, 40, 32760, ctypes.byref(ls64)) == 0  # block 64
+    # bad arguments are rejected on the host, before any CUDA call
+    p = ctypes.c_void_p(4096)
+    ls = BlockListsC(1, 8, 8, 128, 10, 4096, 4096)
+    args = [p, p, p, p, p, p, 1, 2, 1000, 128, ctypes.c_float(0.0), ctypes.byref(ls),
+            ctypes.c_void_p(1 << 30), ctypes.c_void_p(1 << 31), ctypes.c_void_p(3 << 30),
+            ctypes.c_void_p(1 << 33), 1 << 30, None]
+    ovl = list(args)
+    ovl[14] = p  # dv on top of the inputs
+    assert lib.bsa_attn_bwd(*ovl) == 1
+    ovl = list(args)
+    ovl[13] = ctypes.c_void_p(1 << 30)  # dk on top of dq
+    assert lib.bsa_attn_bwd(*ovl) == 1
+    ovl = list(args)
+    ovl[16] = 16  # workspace too small
+    assert lib.bsa_attn_bwd(*ovl) == 1
+    bad = list(args)
+    bad[9] = 96
+    assert lib.bsa_attn_bwd(*bad) == 2  # head_dim
+    ls64 = BlockListsC(1, 16, 16, 64, 10, 4096, 4096)
+    bad = list(args)
+    bad[11] = ctypes.byref(ls64)
+    assert lib.bsa_attn_bwd(*bad) == 2  # block 64 unsupported
