@@ -407,6 +407,157 @@ def run_ours(args, world, rank, local):
     return 0
 
 
+METRIC_BWD = "block-sparse attn bwd ms & effective TFLOP/s (2.5x forward FLOPs) at 32k-120k tokens"
+
+
+def run_ours_bwd(args, world, rank, local):
+    """The backward pass (bsa_attn_bwd) on the same workload: a step is one
+    backward call from resident Q, K, V, O, dO and lse (the forward runs once
+    before timing). value counts the algorithmic backward FLOPs, 2.5 x the
+    forward's; the kernels execute 3.5 x (dQ recomputes S and dP), which the
+    roofline uses."""
+    import numpy as np
+    import torch
+
+    import block_sparse_attention_radial_b200 as bsa
+    from workloads import WORKLOADS, make_qkv
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    w = WORKLOADS[args.workload]
+    q, k, v = make_qkv(w, dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed + 1000)
+    do = torch.randn(q.shape, generator=g, device=dev).to(torch.bfloat16)
+    lists = bsa.radial_block_lists(w.frames, w.tokens_per_frame, w.block, device=dev)
+    rp_h, ci_h = lists.row_ptr.cpu().numpy(), lists.col_idx.cpu().numpy()
+    fwd_flops = bsa.computed_flops(rp_h, ci_h, w.n, w.block, w.head_dim, w.batch, w.heads, 1)
+    flops, exec_flops = 2.5 * fwd_flops, 3.5 * fwd_flops
+    out, lse = bsa.attention(q, k, v, lists)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(bsa.bsa_attn_bwd_workspace_bytes(w.batch, w.heads, w.n, lists),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 6  # prep, transposed-list count, scan, fill; dK/dV; dQ
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        bsa.bsa_attn_bwd(q, k, v, out, do, lse, lists, dq, dk, dv, ws, 0.0, stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if bsa.bsa_get_device_status() != 0:
+        raise SystemExit("device status after warm-up")
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid).replace("GPU-", "")
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid) if rank == 0 else None
+    if sampler is not None:
+        time.sleep(0.4)
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(kev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    clocks = sampler.stop() if sampler is not None else None
+    ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
+    kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    if bsa.bsa_get_device_status() != 0:
+        raise SystemExit("device status after the timed region")
+
+    # end to end: pinned host inputs in, gradients back to the host
+    e2e_steps = max(3, min(args.steps, 10))
+    host_in = [t.cpu().pin_memory() for t in (q, k, v, out, do, lse)]
+    dev_in = [torch.empty_like(t) for t in (q, k, v, out, do, lse)]
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
+
+    def e2e_step():
+        for d_, h_ in zip(dev_in, host_in):
+            d_.copy_(h_, non_blocking=True)
+        bsa.bsa_attn_bwd(*dev_in[:5], dev_in[5], lists, dq, dk, dv, ws, 0.0, stream)
+        for h_, d_ in zip(host_out, (dq, dk, dv)):
+            h_.copy_(d_, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        nrows = 1024
+        first = w.n // 2
+        rows = np.arange(first, min(w.n, first + nrows))
+        qh, kh, vh, dh = (t[:, :1].cpu() for t in (q, k, v, do))
+        t0 = time.perf_counter()
+        oracle.masked_attention_dq_rows(qh, kh, vh, dh, rp_h, ci_h, 1, w.block, 0, 0, rows)
+        dt = time.perf_counter() - t0
+        valid = np.minimum(w.block, w.n - np.arange(w.nqb) * w.block)
+        rf = sum(4 * w.head_dim * int(valid[ci_h[rp_h[r // w.block]:rp_h[r // w.block + 1]]].sum())
+                 for r in rows)
+        cpu_baseline = {"value": 2 * rf / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+                        "kind": "oracle",
+                        "sample": f"dQ of head 0, query rows {int(rows[0])}..{int(rows[-1])} "
+                                  f"({rows.size} rows; 2x their forward FLOPs), {dt:.1f} s, fp64 NumPy"}
+
+    if rank == 0:
+        peaks, peak_kind = load_peaks()
+        peak = float(peaks["bf16_tflops"])
+        achieved = exec_flops / (kernel_ms * 1e-3) / 1e12
+        line = {
+            "metric": METRIC_BWD,
+            "value": flops * world * args.steps / (ms * 1e-3) / 1e12,
+            "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(w, nnz=int(rp_h[-1])),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_kind": f"{peak_kind} bf16 burst",
+                         "kernel": "attn_bwd_dkdv_kernel<128> + attn_bwd_dq_kernel<128> "
+                                   "(+ prep and transposed lists)",
+                         "kernel_ms": kernel_ms, "flops_per_launch": exec_flops},
+            "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+            "cpu_baseline": cpu_baseline,
+        }
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -416,12 +567,16 @@ def main(argv=None):
     ap.add_argument("--workload", default="wan", choices=("wan", "hunyuan", "long4x", "tiny"))
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="which", choices=("fwd", "bwd"), default="fwd",
+                    help="time the forward (default, the headline) or the backward pass")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     world, rank, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, world, rank)
+    if args.which == "bwd":
+        return run_ours_bwd(args, world, rank, local)
     return run_ours(args, world, rank, local)
 
 
