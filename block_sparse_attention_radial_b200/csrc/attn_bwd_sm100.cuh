@@ -519,18 +519,22 @@ struct DqCfg {
   static constexpr int NS_FIT = (kSmemLimit - 1024 - 1024 - 2 * T) / STAGE;
   static constexpr int NS = NS_FIT > 4 ? 4 : NS_FIT;
   static constexpr int DSMEM = 1024 + 2 * T + NS * STAGE;
-  static constexpr uint32_t S_COL = 0;               // S (scores), read back
+  static constexpr uint32_t S_COL = 0;               // S of even steps
   static constexpr uint32_t DP_COL = 128;            // dP, then dS (bf16) over its first 64
   static constexpr uint32_t DQ_COL = 256;
+  static constexpr uint32_t S1_COL = 256 + D;        // S of odd steps
   static constexpr int THREADS = 192;
   static_assert(NS >= 2, "stage ring needs two stages");
+  static_assert(S1_COL + 128 <= 512, "TMEM columns");
+  __host__ __device__ static constexpr uint32_t s_col(int e) { return (e & 1) ? S1_COL : S_COL; }
 };
 
 // Warps 0-3: elementwise (thread = query row = TMEM lane) and the dQ
 // epilogue; warp 4: TMA producer (lane 0); warp 5: MMA issuer (lane 0).
-// Per key block e of the row:  S = Q K_e^T, dP = dO V_e^T, the elementwise
-// warps write dS (bf16) over dP, then dQ += dS K_e (issued before the next
-// S, so the TMEM it reads is not overwritten).
+// Per key block e of the row: S_e = Q K_e^T (double-buffered, issued one
+// block ahead so it runs during the previous elementwise step), dP = dO V_e^T,
+// the elementwise warps write dS (bf16) over dP, then dQ += dS K_e (issued
+// before the next dP, which overwrites the dS it reads).
 template <int D>
 __global__ void __launch_bounds__(192, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -669,10 +673,23 @@ __global__ void __launch_bounds__(192, 1)
         ++qdcount;
         tc_fence_after();
         bool first = true;
+        // S_e = Q K_e^T into its buffer; the key block's stage must be full
+        auto issue_s = [&](int e, uint32_t r) -> bool {
+          const uint32_t s = r % C::NS;
+          if (!lane_wait(&bar_st_full[s], (r / C::NS) & 1u, wc, kBarKvFull, r)) return false;
+          tc_fence_after();
+          const uint32_t k_k = (st_base + s * (C::STAGE >> 4)) | kLboK;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
+            mma_ss_lh(tmem + C::s_col(e), q_lo + off, kHi, k_k + off, kHi, idesc_ss,
+                      kk > 0 ? 1u : 0u);
+          }
+          return true;
+        };
+        if (!(ok = issue_s(0, ring))) break;
         for (int e = 0; e < it.len; ++e) {
           const uint32_t s = ring % C::NS;
-          if (!(ok = lane_wait(&bar_st_full[s], (ring / C::NS) & 1u, wc, kBarKvFull, ring))) break;
-          tc_fence_after();
           if (e > 0) {
             if (!(ok = lane_wait(&bar_p_full, pcount & 1u, wc, kBarPFull, pcount))) break;
             ++pcount;
@@ -684,13 +701,7 @@ __global__ void __launch_bounds__(192, 1)
             issue_acc((ring - 1) % C::NS, first);
             first = false;
           }
-          const uint32_t k_k = (st_base + s * (C::STAGE >> 4)) | kLboK;
           const uint32_t v_k = (st_base + s * (C::STAGE >> 4) + (C::T >> 4)) | kLboK;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
-            mma_ss_lh(tmem + C::S_COL, q_lo + off, kHi, k_k + off, kHi, idesc_ss, kk > 0 ? 1u : 0u);
-          }
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
@@ -700,6 +711,9 @@ __global__ void __launch_bounds__(192, 1)
           if (e == it.len - 1) mma_commit(&bar_qd_empty);  // Q and dO read for the last time
           mma_commit(&bar_s_full);
           ++ring;
+          // the next block's S goes into the buffer the elementwise step of
+          // block e - 1 has finished with (its P arrival was waited above)
+          if (e + 1 < it.len && !(ok = issue_s(e + 1, ring))) break;
         }
         if (!ok) break;
         if (!(ok = lane_wait(&bar_p_full, pcount & 1u, wc, kBarPFull, pcount))) break;
@@ -758,7 +772,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t sr[32], dr[32];
-          tmem_ld32(lane_tmem + C::S_COL + c * 32, sr);
+          tmem_ld32(lane_tmem + C::s_col(e) + c * 32, sr);
           tmem_ld32(lane_tmem + C::DP_COL + c * 32, dr);
           tmem_wait_ld();
           reg_fence32(sr);
