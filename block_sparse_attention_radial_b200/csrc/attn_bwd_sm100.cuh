@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(192, 1)
   constexpr int BN = kBwdBlock;
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t bar_st_full[C::NS], bar_st_empty[C::NS];
-  __shared__ __align__(8) uint64_t bar_kv_full, bar_kv_empty, bar_s_full, bar_p_full;
+  __shared__ __align__(8) uint64_t bar_kv_full, bar_kv_empty, bar_s_full, bar_p_half, bar_p_full;
   __shared__ __align__(8) uint64_t bar_acc_full, bar_acc_empty, bar_final;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -230,6 +230,7 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(&bar_kv_full, 1);
     mbar_init(&bar_kv_empty, 1);
     mbar_init(&bar_s_full, 1);
+    mbar_init(&bar_p_half, 128);
     mbar_init(&bar_p_full, 128);
     mbar_init(&bar_acc_full, 1);
     mbar_init(&bar_acc_empty, 128);
@@ -322,18 +323,29 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t ring = 0, kvcount = 0, pcount = 0, items = 0;
       bool ok = true;
       // dV += P^T dO and dK += dS^T Q for the query block in stage `s`
-      auto issue_acc = [&](uint32_t s, bool first) {
+      // The elementwise warps hand P^T and dS^T over in two halves of 64
+      // query columns (p_half, then p_full): the first half's MMAs run while
+      // the second half is computed.
+      auto issue_acc = [&](uint32_t s, bool first) -> bool {
         const uint32_t q_mn = (st_base + s * (C::STAGE >> 4)) | kLboMN;
         const uint32_t do_mn = (st_base + s * (C::STAGE >> 4) + (C::T >> 4)) | kLboMN;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts_lh(tmem + C::DV_COL, tmem + C::ST_COL + kk * 8, do_mn + kk * (16 * 128 >> 4),
-                    kHi, idesc_ts, (!first || kk > 0) ? 1u : 0u);
+        for (int h = 0; h < 2; ++h) {
+          if (!lane_wait(h == 0 ? &bar_p_half : &bar_p_full, pcount & 1u, wc, kBarPFull, pcount))
+            return false;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts_lh(tmem + C::DK_COL, tmem + C::DPT_COL + kk * 8, q_mn + kk * (16 * 128 >> 4),
-                    kHi, idesc_ts, (!first || kk > 0) ? 1u : 0u);
+          for (int kk = h * BN / 32; kk < (h + 1) * BN / 32; ++kk)
+            mma_ts_lh(tmem + C::DV_COL, tmem + C::ST_COL + kk * 8, do_mn + kk * (16 * 128 >> 4),
+                      kHi, idesc_ts, (!first || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = h * BN / 32; kk < (h + 1) * BN / 32; ++kk)
+            mma_ts_lh(tmem + C::DK_COL, tmem + C::DPT_COL + kk * 8, q_mn + kk * (16 * 128 >> 4),
+                      kHi, idesc_ts, (!first || kk > 0) ? 1u : 0u);
+        }
+        ++pcount;
         mma_commit(&bar_st_empty[s]);
+        return true;
       };
       for (int k = 0; ok; ++k) {
         const int idx = snake_item(k, p.total_items);
@@ -350,14 +362,11 @@ __global__ void __launch_bounds__(192, 1)
           if (!(ok = lane_wait(&bar_st_full[s], (ring / C::NS) & 1u, wc, kBarKvFull, ring))) break;
           tc_fence_after();
           if (e > 0) {  // accumulate the previous query block
-            if (!(ok = lane_wait(&bar_p_full, pcount & 1u, wc, kBarPFull, pcount))) break;
-            ++pcount;
-            tc_fence_after();
             if (first && items > 0) {
               if (!(ok = lane_wait(&bar_acc_empty, (items - 1) & 1u, wc, kBarOEmpty, items))) break;
               tc_fence_after();
             }
-            issue_acc((ring - 1) % C::NS, first);
+            if (!(ok = issue_acc((ring - 1) % C::NS, first))) break;
             first = false;
           }
           const uint32_t q_k = (st_base + s * (C::STAGE >> 4)) | kLboK;
@@ -378,14 +387,11 @@ __global__ void __launch_bounds__(192, 1)
           ++ring;
         }
         if (!ok) break;
-        if (!(ok = lane_wait(&bar_p_full, pcount & 1u, wc, kBarPFull, pcount))) break;
-        ++pcount;
-        tc_fence_after();
         if (first && items > 0) {
           if (!(ok = lane_wait(&bar_acc_empty, (items - 1) & 1u, wc, kBarOEmpty, items))) break;
           tc_fence_after();
         }
-        issue_acc((ring - 1) % C::NS, first);
+        if (!(ok = issue_acc((ring - 1) % C::NS, first))) break;
         mma_commit(&bar_acc_full);
         ++items;
       }
@@ -461,6 +467,11 @@ __global__ void __launch_bounds__(192, 1)
           // chunk c lands on columns [16c, 16c + 16): already read back
           tmem_st16(lane_tmem + C::ST_COL + c * 16, pk);
           tmem_st16(lane_tmem + C::DPT_COL + c * 16, dk16);
+          if (c == BN / 64 - 1) {  // first half of the query columns handed over
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bar_p_half);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
@@ -545,7 +556,7 @@ __global__ void __launch_bounds__(192, 1)
   constexpr int BN = kBwdBlock;
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t bar_st_full[C::NS], bar_st_empty[C::NS];
-  __shared__ __align__(8) uint64_t bar_qd_full, bar_qd_empty, bar_s_full, bar_p_full;
+  __shared__ __align__(8) uint64_t bar_qd_full, bar_qd_empty, bar_s_full, bar_p_half, bar_p_full;
   __shared__ __align__(8) uint64_t bar_acc_full, bar_acc_empty, bar_final;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -568,6 +579,7 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(&bar_qd_full, 1);
     mbar_init(&bar_qd_empty, 1);
     mbar_init(&bar_s_full, 1);
+    mbar_init(&bar_p_half, 128);
     mbar_init(&bar_p_full, 128);
     mbar_init(&bar_acc_full, 1);
     mbar_init(&bar_acc_empty, 128);
@@ -655,13 +667,22 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t ring = 0, qdcount = 0, pcount = 0, items = 0;
       bool ok = true;
       // dQ += dS K for the key block in stage `s`
-      auto issue_acc = [&](uint32_t s, bool first) {
+      // dS comes in two halves of 64 key columns (p_half, then p_full)
+      auto issue_acc = [&](uint32_t s, bool first) -> bool {
         const uint32_t k_mn = (st_base + s * (C::STAGE >> 4)) | kLboMN;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts_lh(tmem + C::DQ_COL, tmem + C::DP_COL + kk * 8, k_mn + kk * (16 * 128 >> 4),
-                    kHi, idesc_ts, (!first || kk > 0) ? 1u : 0u);
+        for (int h = 0; h < 2; ++h) {
+          if (!lane_wait(h == 0 ? &bar_p_half : &bar_p_full, pcount & 1u, wc, kBarPFull, pcount))
+            return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = h * BN / 32; kk < (h + 1) * BN / 32; ++kk)
+            mma_ts_lh(tmem + C::DQ_COL, tmem + C::DP_COL + kk * 8, k_mn + kk * (16 * 128 >> 4),
+                      kHi, idesc_ts, (!first || kk > 0) ? 1u : 0u);
+        }
+        ++pcount;
         mma_commit(&bar_st_empty[s]);
+        return true;
       };
       for (int k = 0; ok; ++k) {
         const int idx = snake_item(k, p.total_items);
@@ -691,14 +712,11 @@ __global__ void __launch_bounds__(192, 1)
         for (int e = 0; e < it.len; ++e) {
           const uint32_t s = ring % C::NS;
           if (e > 0) {
-            if (!(ok = lane_wait(&bar_p_full, pcount & 1u, wc, kBarPFull, pcount))) break;
-            ++pcount;
-            tc_fence_after();
             if (first && items > 0) {
               if (!(ok = lane_wait(&bar_acc_empty, (items - 1) & 1u, wc, kBarOEmpty, items))) break;
               tc_fence_after();
             }
-            issue_acc((ring - 1) % C::NS, first);
+            if (!(ok = issue_acc((ring - 1) % C::NS, first))) break;
             first = false;
           }
           const uint32_t v_k = (st_base + s * (C::STAGE >> 4) + (C::T >> 4)) | kLboK;
@@ -716,14 +734,11 @@ __global__ void __launch_bounds__(192, 1)
           if (e + 1 < it.len && !(ok = issue_s(e + 1, ring))) break;
         }
         if (!ok) break;
-        if (!(ok = lane_wait(&bar_p_full, pcount & 1u, wc, kBarPFull, pcount))) break;
-        ++pcount;
-        tc_fence_after();
         if (first && items > 0) {
           if (!(ok = lane_wait(&bar_acc_empty, (items - 1) & 1u, wc, kBarOEmpty, items))) break;
           tc_fence_after();
         }
-        issue_acc((ring - 1) % C::NS, first);
+        if (!(ok = issue_acc((ring - 1) % C::NS, first))) break;
         mma_commit(&bar_acc_full);
         ++items;
       }
@@ -792,6 +807,11 @@ __global__ void __launch_bounds__(192, 1)
           }
           // chunk c lands on dP columns [16c, 16c + 16): already read back
           tmem_st16(lane_tmem + C::DP_COL + c * 16, g16);
+          if (c == BN / 64 - 1) {  // first half of the key columns handed over
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bar_p_half);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
