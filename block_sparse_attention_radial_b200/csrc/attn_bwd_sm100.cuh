@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(192, 1)
   constexpr int BN = kBwdBlock;
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t bar_st_full[C::NS], bar_st_empty[C::NS];
-  __shared__ __align__(8) uint64_t bar_kv_full, bar_kv_empty, bar_s_full, bar_p_half, bar_p_full;
+  __shared__ __align__(8) uint64_t bar_kv_full, bar_kv_empty, bar_s_full, bar_p_part[4];
   __shared__ __align__(8) uint64_t bar_acc_full, bar_acc_empty, bar_final;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -230,8 +230,7 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(&bar_kv_full, 1);
     mbar_init(&bar_kv_empty, 1);
     mbar_init(&bar_s_full, 1);
-    mbar_init(&bar_p_half, 128);
-    mbar_init(&bar_p_full, 128);
+    for (int h = 0; h < 4; ++h) mbar_init(&bar_p_part[h], 128);
     mbar_init(&bar_acc_full, 1);
     mbar_init(&bar_acc_empty, 128);
     mbar_init(&bar_final, 1);
@@ -323,23 +322,22 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t ring = 0, kvcount = 0, pcount = 0, items = 0;
       bool ok = true;
       // dV += P^T dO and dK += dS^T Q for the query block in stage `s`
-      // The elementwise warps hand P^T and dS^T over in two halves of 64
-      // query columns (p_half, then p_full): the first half's MMAs run while
-      // the second half is computed.
+      // The elementwise warps hand P^T and dS^T over in four parts of 32
+      // query columns (p_part[0..3]): a part's MMAs run while the next part
+      // is computed.
       auto issue_acc = [&](uint32_t s, bool first) -> bool {
         const uint32_t q_mn = (st_base + s * (C::STAGE >> 4)) | kLboMN;
         const uint32_t do_mn = (st_base + s * (C::STAGE >> 4) + (C::T >> 4)) | kLboMN;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (!lane_wait(h == 0 ? &bar_p_half : &bar_p_full, pcount & 1u, wc, kBarPFull, pcount))
-            return false;
+        for (int h = 0; h < 4; ++h) {
+          if (!lane_wait(&bar_p_part[h], pcount & 1u, wc, kBarPFull, pcount)) return false;
           tc_fence_after();
 #pragma unroll
-          for (int kk = h * BN / 32; kk < (h + 1) * BN / 32; ++kk)
+          for (int kk = h * BN / 64; kk < (h + 1) * BN / 64; ++kk)
             mma_ts_lh(tmem + C::DV_COL, tmem + C::ST_COL + kk * 8, do_mn + kk * (16 * 128 >> 4),
                       kHi, idesc_ts, (!first || kk > 0) ? 1u : 0u);
 #pragma unroll
-          for (int kk = h * BN / 32; kk < (h + 1) * BN / 32; ++kk)
+          for (int kk = h * BN / 64; kk < (h + 1) * BN / 64; ++kk)
             mma_ts_lh(tmem + C::DK_COL, tmem + C::DPT_COL + kk * 8, q_mn + kk * (16 * 128 >> 4),
                       kHi, idesc_ts, (!first || kk > 0) ? 1u : 0u);
         }
@@ -467,15 +465,10 @@ __global__ void __launch_bounds__(192, 1)
           // chunk c lands on columns [16c, 16c + 16): already read back
           tmem_st16(lane_tmem + C::ST_COL + c * 16, pk);
           tmem_st16(lane_tmem + C::DPT_COL + c * 16, dk16);
-          if (c == BN / 64 - 1) {  // first half of the query columns handed over
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&bar_p_half);
-          }
+          tmem_wait_st();  // part c of the query columns handed over
+          tc_fence_before();
+          mbar_arrive(&bar_p_part[c]);
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bar_p_full);
       }
       if (!ok) break;
       // epilogue: dV and dK (times scale) of this key row
@@ -556,7 +549,7 @@ __global__ void __launch_bounds__(192, 1)
   constexpr int BN = kBwdBlock;
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t bar_st_full[C::NS], bar_st_empty[C::NS];
-  __shared__ __align__(8) uint64_t bar_qd_full, bar_qd_empty, bar_s_full, bar_p_half, bar_p_full;
+  __shared__ __align__(8) uint64_t bar_qd_full, bar_qd_empty, bar_s_full, bar_p_part[4];
   __shared__ __align__(8) uint64_t bar_acc_full, bar_acc_empty, bar_final;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -579,8 +572,7 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(&bar_qd_full, 1);
     mbar_init(&bar_qd_empty, 1);
     mbar_init(&bar_s_full, 1);
-    mbar_init(&bar_p_half, 128);
-    mbar_init(&bar_p_full, 128);
+    for (int h = 0; h < 4; ++h) mbar_init(&bar_p_part[h], 128);
     mbar_init(&bar_acc_full, 1);
     mbar_init(&bar_acc_empty, 128);
     mbar_init(&bar_final, 1);
@@ -667,16 +659,15 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t ring = 0, qdcount = 0, pcount = 0, items = 0;
       bool ok = true;
       // dQ += dS K for the key block in stage `s`
-      // dS comes in two halves of 64 key columns (p_half, then p_full)
+      // dS comes in four parts of 32 key columns (p_part[0..3])
       auto issue_acc = [&](uint32_t s, bool first) -> bool {
         const uint32_t k_mn = (st_base + s * (C::STAGE >> 4)) | kLboMN;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (!lane_wait(h == 0 ? &bar_p_half : &bar_p_full, pcount & 1u, wc, kBarPFull, pcount))
-            return false;
+        for (int h = 0; h < 4; ++h) {
+          if (!lane_wait(&bar_p_part[h], pcount & 1u, wc, kBarPFull, pcount)) return false;
           tc_fence_after();
 #pragma unroll
-          for (int kk = h * BN / 32; kk < (h + 1) * BN / 32; ++kk)
+          for (int kk = h * BN / 64; kk < (h + 1) * BN / 64; ++kk)
             mma_ts_lh(tmem + C::DQ_COL, tmem + C::DP_COL + kk * 8, k_mn + kk * (16 * 128 >> 4),
                       kHi, idesc_ts, (!first || kk > 0) ? 1u : 0u);
         }
@@ -807,15 +798,10 @@ __global__ void __launch_bounds__(192, 1)
           }
           // chunk c lands on dP columns [16c, 16c + 16): already read back
           tmem_st16(lane_tmem + C::DP_COL + c * 16, g16);
-          if (c == BN / 64 - 1) {  // first half of the key columns handed over
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&bar_p_half);
-          }
+          tmem_wait_st();  // part c of the key columns handed over
+          tc_fence_before();
+          mbar_arrive(&bar_p_part[c]);
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bar_p_full);
       }
       if (!ok) break;
       if (!(ok = warp_wait(&bar_acc_full, acount & 1u, wc, kBarODone, acount))) break;
