@@ -207,7 +207,8 @@ __global__ void __launch_bounds__(192, 1)
   constexpr int BN = kBwdBlock;
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t bar_st_full[C::NS], bar_st_empty[C::NS];
-  __shared__ __align__(8) uint64_t bar_kv_full, bar_kv_empty, bar_s_full, bar_p_part[4];
+  __shared__ __align__(8) uint64_t bar_kv_full, bar_kv_empty, bar_s_full, bar_dp_full;
+  __shared__ __align__(8) uint64_t bar_p_part[4], bar_ds_part[4];
   __shared__ __align__(8) uint64_t bar_acc_full, bar_acc_empty, bar_final;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -230,7 +231,11 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(&bar_kv_full, 1);
     mbar_init(&bar_kv_empty, 1);
     mbar_init(&bar_s_full, 1);
-    for (int h = 0; h < 4; ++h) mbar_init(&bar_p_part[h], 128);
+    mbar_init(&bar_dp_full, 1);
+    for (int h = 0; h < 4; ++h) {
+      mbar_init(&bar_p_part[h], 128);
+      mbar_init(&bar_ds_part[h], 128);
+    }
     mbar_init(&bar_acc_full, 1);
     mbar_init(&bar_acc_empty, 128);
     mbar_init(&bar_final, 1);
@@ -321,29 +326,39 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t st_base = smem_addr(sStage) >> 4;
       uint32_t ring = 0, kvcount = 0, pcount = 0, items = 0;
       bool ok = true;
-      // dV += P^T dO and dK += dS^T Q for the query block in stage `s`
-      // The elementwise warps hand P^T and dS^T over in four parts of 32
-      // query columns (p_part[0..3]): a part's MMAs run while the next part
-      // is computed.
-      auto issue_acc = [&](uint32_t s, bool first) -> bool {
-        const uint32_t q_mn = (st_base + s * (C::STAGE >> 4)) | kLboMN;
-        const uint32_t do_mn = (st_base + s * (C::STAGE >> 4) + (C::T >> 4)) | kLboMN;
+      // Schedule per query block e (stage s_e):
+      //   S^T_e, dP^T_e                       (S^T_0, dP^T_0 before the loop)
+      //   dV += P^T_e dO_e   part by part, as the elementwise warps hand
+      //                      P^T over (p_part[0..3]); they compute P^T while
+      //                      dP^T_e is still on the tensor pipe
+      //   S^T_{e+1}          the S^T region is free once the dV MMAs that
+      //                      read P^T_e are issued; it runs while the
+      //                      elementwise warps compute dS^T_e
+      //   dK += dS^T_e Q_e   part by part (ds_part[0..3])
+      //   dP^T_{e+1}         after the dK MMAs that read dS^T_e
+      auto issue_s = [&](uint32_t r) -> bool {  // S^T = K Q^T for ring slot r
+        const uint32_t s = r % C::NS;
+        if (!lane_wait(&bar_st_full[s], (r / C::NS) & 1u, wc, kBarKvFull, r)) return false;
+        tc_fence_after();
+        const uint32_t q_k = (st_base + s * (C::STAGE >> 4)) | kLboK;
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          if (!lane_wait(&bar_p_part[h], pcount & 1u, wc, kBarPFull, pcount)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = h * BN / 64; kk < (h + 1) * BN / 64; ++kk)
-            mma_ts_lh(tmem + C::DV_COL, tmem + C::ST_COL + kk * 8, do_mn + kk * (16 * 128 >> 4),
-                      kHi, idesc_ts, (!first || kk > 0) ? 1u : 0u);
-#pragma unroll
-          for (int kk = h * BN / 64; kk < (h + 1) * BN / 64; ++kk)
-            mma_ts_lh(tmem + C::DK_COL, tmem + C::DPT_COL + kk * 8, q_mn + kk * (16 * 128 >> 4),
-                      kHi, idesc_ts, (!first || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
+          mma_ss_lh(tmem + C::ST_COL, k_lo + off, kHi, q_k + off, kHi, idesc_ss, kk > 0 ? 1u : 0u);
         }
-        ++pcount;
-        mma_commit(&bar_st_empty[s]);
+        mma_commit(&bar_s_full);
         return true;
+      };
+      auto issue_dp = [&](uint32_t r) {  // dP^T = V dO^T (slot already waited)
+        const uint32_t s = r % C::NS;
+        const uint32_t do_k = (st_base + s * (C::STAGE >> 4) + (C::T >> 4)) | kLboK;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
+          mma_ss_lh(tmem + C::DPT_COL, v_lo + off, kHi, do_k + off, kHi, idesc_ss,
+                    kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bar_dp_full);
       };
       for (int k = 0; ok; ++k) {
         const int idx = snake_item(k, p.total_items);
@@ -354,42 +369,48 @@ __global__ void __launch_bounds__(192, 1)
         if (!(ok = lane_wait(&bar_kv_full, kvcount & 1u, wc, kBarQFull, kvcount))) break;
         ++kvcount;
         tc_fence_after();
+        if (!(ok = issue_s(ring))) break;
+        issue_dp(ring);
         bool first = true;
         for (int e = 0; e < it.len; ++e) {
           const uint32_t s = ring % C::NS;
-          if (!(ok = lane_wait(&bar_st_full[s], (ring / C::NS) & 1u, wc, kBarKvFull, ring))) break;
-          tc_fence_after();
-          if (e > 0) {  // accumulate the previous query block
-            if (first && items > 0) {
-              if (!(ok = lane_wait(&bar_acc_empty, (items - 1) & 1u, wc, kBarOEmpty, items))) break;
-              tc_fence_after();
-            }
-            if (!(ok = issue_acc((ring - 1) % C::NS, first))) break;
-            first = false;
-          }
-          const uint32_t q_k = (st_base + s * (C::STAGE >> 4)) | kLboK;
-          const uint32_t do_k = (st_base + s * (C::STAGE >> 4) + (C::T >> 4)) | kLboK;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
-            mma_ss_lh(tmem + C::ST_COL, k_lo + off, kHi, q_k + off, kHi, idesc_ss, kk > 0 ? 1u : 0u);
+          const uint32_t q_mn = (st_base + s * (C::STAGE >> 4)) | kLboMN;
+          const uint32_t do_mn = (st_base + s * (C::STAGE >> 4) + (C::T >> 4)) | kLboMN;
+          if (first && items > 0) {  // the previous item's epilogue has read dV, dK
+            if (!(ok = lane_wait(&bar_acc_empty, (items - 1) & 1u, wc, kBarOEmpty, items))) break;
+            tc_fence_after();
           }
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
-            mma_ss_lh(tmem + C::DPT_COL, v_lo + off, kHi, do_k + off, kHi, idesc_ss,
-                      kk > 0 ? 1u : 0u);
+          for (int h = 0; h < 4; ++h) {
+            if (!(ok = lane_wait(&bar_p_part[h], pcount & 1u, wc, kBarPFull, pcount))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = h * BN / 64; kk < (h + 1) * BN / 64; ++kk)
+              mma_ts_lh(tmem + C::DV_COL, tmem + C::ST_COL + kk * 8,
+                        do_mn + kk * (16 * 128 >> 4), kHi, idesc_ts,
+                        (!first || kk > 0) ? 1u : 0u);
           }
-          if (e == it.len - 1) mma_commit(&bar_kv_empty);  // K and V read for the last time
-          mma_commit(&bar_s_full);
+          if (!ok) break;
+          if (e + 1 < it.len && !(ok = issue_s(ring + 1))) break;
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            if (!(ok = lane_wait(&bar_ds_part[h], pcount & 1u, wc, kBarPFull, pcount))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = h * BN / 64; kk < (h + 1) * BN / 64; ++kk)
+              mma_ts_lh(tmem + C::DK_COL, tmem + C::DPT_COL + kk * 8,
+                        q_mn + kk * (16 * 128 >> 4), kHi, idesc_ts,
+                        (!first || kk > 0) ? 1u : 0u);
+          }
+          if (!ok) break;
+          mma_commit(&bar_st_empty[s]);  // Q_e and dO_e read for the last time
+          ++pcount;
           ++ring;
+          first = false;
+          if (e + 1 < it.len) issue_dp(ring);
         }
         if (!ok) break;
-        if (first && items > 0) {
-          if (!(ok = lane_wait(&bar_acc_empty, (items - 1) & 1u, wc, kBarOEmpty, items))) break;
-          tc_fence_after();
-        }
-        if (!(ok = issue_acc((ring - 1) % C::NS, first))) break;
+        mma_commit(&bar_kv_empty);  // K and V read for the last time
         mma_commit(&bar_acc_full);
         ++items;
       }
@@ -406,7 +427,7 @@ __global__ void __launch_bounds__(192, 1)
     const int r = warp * 32 + lane;  // key row within the tile = TMEM lane
     const uint32_t lane_tmem = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const float sl2 = p.scale_log2;
-    uint32_t ring = 0, scount = 0, acount = 0;
+    uint32_t ring = 0, scount = 0, dcount = 0, acount = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int idx = snake_item(k, p.total_items);
@@ -432,42 +453,59 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t s = ring % C::NS, spar = (ring / C::NS) & 1u;
         ++ring;
         if (!(ok = warp_wait(&bar_s_full, scount & 1u, wc, kBarSFull, scount))) break;
-        ++scount;
         // the stage's lse2 / delta rows came by TMA: acquire them from the
         // stage barrier itself (complete long before S^T is; the stage is
-        // not released before this warp's P arrives)
+        // not released before this warp's dS^T arrives)
         if (!(ok = warp_wait(&bar_st_full[s], spar, wc, kBarKvFull, ring))) break;
         tc_fence_after();
         const float *lse_s = reinterpret_cast<const float *>(sStage + s * C::STAGE + 2 * C::T);
         const float *del_s = lse_s + 128;
+        // P^T (fp32, kept for dS^T), handed over as bf16 in four parts while
+        // dP^T is still being computed
+        float pf[BN];
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
-          uint32_t sr[32], dr[32];
+          uint32_t sr[32];
           tmem_ld32(lane_tmem + C::ST_COL + c * 32, sr);
-          tmem_ld32(lane_tmem + C::DPT_COL + c * 32, dr);
           tmem_wait_ld();
           reg_fence32(sr);
-          reg_fence32(dr);
-          uint32_t pk[16], dk16[16];
+          uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float4 l4 = *reinterpret_cast<const float4 *>(lse_s + c * 32 + (i & ~1) * 2);
-            const float4 d4 = *reinterpret_cast<const float4 *>(del_s + c * 32 + (i & ~1) * 2);
             const float la = (i & 1) ? l4.z : l4.x, lb = (i & 1) ? l4.w : l4.y;
-            const float da = (i & 1) ? d4.z : d4.x, db = (i & 1) ? d4.w : d4.y;
-            const float pa = ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -la));
-            const float pb = ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -lb));
-            const float ga = pa * (__uint_as_float(dr[2 * i]) - da);
-            const float gb = pb * (__uint_as_float(dr[2 * i + 1]) - db);
-            pk[i] = pack_bf16x2(pa, pb);
-            dk16[i] = pack_bf16x2(ga, gb);
+            pf[c * 32 + 2 * i] = ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -la));
+            pf[c * 32 + 2 * i + 1] = ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -lb));
+            pk[i] = pack_bf16x2(pf[c * 32 + 2 * i], pf[c * 32 + 2 * i + 1]);
           }
           // chunk c lands on columns [16c, 16c + 16): already read back
           tmem_st16(lane_tmem + C::ST_COL + c * 16, pk);
-          tmem_st16(lane_tmem + C::DPT_COL + c * 16, dk16);
-          tmem_wait_st();  // part c of the query columns handed over
+          tmem_wait_st();
           tc_fence_before();
           mbar_arrive(&bar_p_part[c]);
+        }
+        ++scount;
+        if (!(ok = warp_wait(&bar_dp_full, dcount & 1u, wc, kBarSFull, dcount))) break;
+        ++dcount;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t dr[32];
+          tmem_ld32(lane_tmem + C::DPT_COL + c * 32, dr);
+          tmem_wait_ld();
+          reg_fence32(dr);
+          uint32_t g16[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float4 d4 = *reinterpret_cast<const float4 *>(del_s + c * 32 + (i & ~1) * 2);
+            const float da = (i & 1) ? d4.z : d4.x, db = (i & 1) ? d4.w : d4.y;
+            g16[i] = pack_bf16x2(pf[c * 32 + 2 * i] * (__uint_as_float(dr[2 * i]) - da),
+                                 pf[c * 32 + 2 * i + 1] * (__uint_as_float(dr[2 * i + 1]) - db));
+          }
+          tmem_st16(lane_tmem + C::DPT_COL + c * 16, g16);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&bar_ds_part[c]);
         }
       }
       if (!ok) break;
@@ -549,7 +587,11 @@ __global__ void __launch_bounds__(192, 1)
   constexpr int BN = kBwdBlock;
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t bar_st_full[C::NS], bar_st_empty[C::NS];
-  __shared__ __align__(8) uint64_t bar_qd_full, bar_qd_empty, bar_s_full, bar_p_part[4];
+  // one S-ready barrier per S buffer: with S issued a block ahead, a single
+  // barrier could complete two phases before the elementwise warps wait for
+  // the first (at an item's start), and a parity wait cannot tell them apart
+  __shared__ __align__(8) uint64_t bar_qd_full, bar_qd_empty, bar_s_full[2], bar_dp_full;
+  __shared__ __align__(8) uint64_t bar_ds_part[4];
   __shared__ __align__(8) uint64_t bar_acc_full, bar_acc_empty, bar_final;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -571,8 +613,10 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(&bar_qd_full, 1);
     mbar_init(&bar_qd_empty, 1);
-    mbar_init(&bar_s_full, 1);
-    for (int h = 0; h < 4; ++h) mbar_init(&bar_p_part[h], 128);
+    mbar_init(&bar_s_full[0], 1);
+    mbar_init(&bar_s_full[1], 1);
+    mbar_init(&bar_dp_full, 1);
+    for (int h = 0; h < 4; ++h) mbar_init(&bar_ds_part[h], 128);
     mbar_init(&bar_acc_full, 1);
     mbar_init(&bar_acc_empty, 128);
     mbar_init(&bar_final, 1);
@@ -658,22 +702,39 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t st_base = smem_addr(sStage) >> 4;
       uint32_t ring = 0, qdcount = 0, pcount = 0, items = 0;
       bool ok = true;
-      // dQ += dS K for the key block in stage `s`
-      // dS comes in four parts of 32 key columns (p_part[0..3])
-      auto issue_acc = [&](uint32_t s, bool first) -> bool {
-        const uint32_t k_mn = (st_base + s * (C::STAGE >> 4)) | kLboMN;
+      // Schedule per key block e (stage s_e):
+      //   S_{e+1}           into the other S buffer (its previous user, the
+      //                     elementwise step of block e-1, is done): runs
+      //                     while block e's elementwise step works
+      //   dQ += dS_e K_e    part by part, as the elementwise warps hand dS
+      //                     over (ds_part[0..3]); they compute P_e from S_e
+      //                     while dP_e is still on the tensor pipe
+      //   dP_{e+1}          after the dQ MMAs that read dS_e from its region
+      // (S_0 and dP_0 before the loop.)
+      auto issue_s = [&](int e, uint32_t r) -> bool {  // S_e = Q K_e^T
+        const uint32_t s = r % C::NS;
+        if (!lane_wait(&bar_st_full[s], (r / C::NS) & 1u, wc, kBarKvFull, r)) return false;
+        tc_fence_after();
+        const uint32_t k_k = (st_base + s * (C::STAGE >> 4)) | kLboK;
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          if (!lane_wait(&bar_p_part[h], pcount & 1u, wc, kBarPFull, pcount)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = h * BN / 64; kk < (h + 1) * BN / 64; ++kk)
-            mma_ts_lh(tmem + C::DQ_COL, tmem + C::DP_COL + kk * 8, k_mn + kk * (16 * 128 >> 4),
-                      kHi, idesc_ts, (!first || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
+          mma_ss_lh(tmem + C::s_col(e), q_lo + off, kHi, k_k + off, kHi, idesc_ss,
+                    kk > 0 ? 1u : 0u);
         }
-        ++pcount;
-        mma_commit(&bar_st_empty[s]);
+        mma_commit(&bar_s_full[e & 1]);
         return true;
+      };
+      auto issue_dp = [&](uint32_t r) {  // dP = dO V^T (slot already waited)
+        const uint32_t s = r % C::NS;
+        const uint32_t v_k = (st_base + s * (C::STAGE >> 4) + (C::T >> 4)) | kLboK;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
+          mma_ss_lh(tmem + C::DP_COL, do_lo + off, kHi, v_k + off, kHi, idesc_ss,
+                    kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bar_dp_full);
       };
       for (int k = 0; ok; ++k) {
         const int idx = snake_item(k, p.total_items);
@@ -684,52 +745,36 @@ __global__ void __launch_bounds__(192, 1)
         if (!(ok = lane_wait(&bar_qd_full, qdcount & 1u, wc, kBarQFull, qdcount))) break;
         ++qdcount;
         tc_fence_after();
-        bool first = true;
-        // S_e = Q K_e^T into its buffer; the key block's stage must be full
-        auto issue_s = [&](int e, uint32_t r) -> bool {
-          const uint32_t s = r % C::NS;
-          if (!lane_wait(&bar_st_full[s], (r / C::NS) & 1u, wc, kBarKvFull, r)) return false;
-          tc_fence_after();
-          const uint32_t k_k = (st_base + s * (C::STAGE >> 4)) | kLboK;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
-            mma_ss_lh(tmem + C::s_col(e), q_lo + off, kHi, k_k + off, kHi, idesc_ss,
-                      kk > 0 ? 1u : 0u);
-          }
-          return true;
-        };
         if (!(ok = issue_s(0, ring))) break;
+        issue_dp(ring);
+        bool first = true;
         for (int e = 0; e < it.len; ++e) {
           const uint32_t s = ring % C::NS;
-          if (e > 0) {
-            if (first && items > 0) {
-              if (!(ok = lane_wait(&bar_acc_empty, (items - 1) & 1u, wc, kBarOEmpty, items))) break;
-              tc_fence_after();
-            }
-            if (!(ok = issue_acc((ring - 1) % C::NS, first))) break;
-            first = false;
+          if (e + 1 < it.len && !(ok = issue_s(e + 1, ring + 1))) break;
+          if (first && items > 0) {  // the previous item's epilogue has read dQ
+            if (!(ok = lane_wait(&bar_acc_empty, (items - 1) & 1u, wc, kBarOEmpty, items))) break;
+            tc_fence_after();
           }
-          const uint32_t v_k = (st_base + s * (C::STAGE >> 4) + (C::T >> 4)) | kLboK;
+          const uint32_t k_mn = (st_base + s * (C::STAGE >> 4)) | kLboMN;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
-            mma_ss_lh(tmem + C::DP_COL, do_lo + off, kHi, v_k + off, kHi, idesc_ss,
-                      kk > 0 ? 1u : 0u);
+          for (int h = 0; h < 4; ++h) {
+            if (!(ok = lane_wait(&bar_ds_part[h], pcount & 1u, wc, kBarPFull, pcount))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = h * BN / 64; kk < (h + 1) * BN / 64; ++kk)
+              mma_ts_lh(tmem + C::DQ_COL, tmem + C::DP_COL + kk * 8,
+                        k_mn + kk * (16 * 128 >> 4), kHi, idesc_ts,
+                        (!first || kk > 0) ? 1u : 0u);
           }
-          if (e == it.len - 1) mma_commit(&bar_qd_empty);  // Q and dO read for the last time
-          mma_commit(&bar_s_full);
+          if (!ok) break;
+          mma_commit(&bar_st_empty[s]);  // K_e and V_e read for the last time
+          ++pcount;
           ++ring;
-          // the next block's S goes into the buffer the elementwise step of
-          // block e - 1 has finished with (its P arrival was waited above)
-          if (e + 1 < it.len && !(ok = issue_s(e + 1, ring))) break;
+          first = false;
+          if (e + 1 < it.len) issue_dp(ring);
         }
         if (!ok) break;
-        if (first && items > 0) {
-          if (!(ok = lane_wait(&bar_acc_empty, (items - 1) & 1u, wc, kBarOEmpty, items))) break;
-          tc_fence_after();
-        }
-        if (!(ok = issue_acc((ring - 1) % C::NS, first))) break;
+        mma_commit(&bar_qd_empty);  // Q and dO read for the last time
         mma_commit(&bar_acc_full);
         ++items;
       }
@@ -746,7 +791,7 @@ __global__ void __launch_bounds__(192, 1)
     const int r = warp * 32 + lane;  // query row within the tile = TMEM lane
     const uint32_t lane_tmem = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const float sl2 = p.scale_log2;
-    uint32_t scount = 0, acount = 0;
+    uint32_t scount[2] = {0u, 0u}, dcount = 0, acount = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int idx = snake_item(k, p.total_items);
@@ -771,36 +816,44 @@ __global__ void __launch_bounds__(192, 1)
       const int last_kb = min(max(__ldg(p.col_idx + it.a + it.len - 1), 0), p.nkb - 1);
       const int last_valid = min(p.n - last_kb * BN, BN);
       for (int e = 0; e < it.len; ++e) {
-        if (!(ok = warp_wait(&bar_s_full, scount & 1u, wc, kBarSFull, scount))) break;
-        ++scount;
+        const int sb = e & 1;
+        if (!(ok = warp_wait(&bar_s_full[sb], scount[sb] & 1u, wc, kBarSFull, scount[sb]))) break;
+        ++scount[sb];
         tc_fence_after();
         const int valid = e == it.len - 1 ? last_valid : BN;
+        // P from S (fp32, kept for dS) while dP is still being computed
+        float pf[BN];
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
-          uint32_t sr[32], dr[32];
+          uint32_t sr[32];
           tmem_ld32(lane_tmem + C::s_col(e) + c * 32, sr);
-          tmem_ld32(lane_tmem + C::DP_COL + c * 32, dr);
           tmem_wait_ld();
           reg_fence32(sr);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float pv = ex2_approx(fmaf(__uint_as_float(sr[i]), sl2, -lse2));
+            pf[c * 32 + i] = (valid < BN && c * 32 + i >= valid) ? 0.f : pv;
+          }
+        }
+        if (!(ok = warp_wait(&bar_dp_full, dcount & 1u, wc, kBarSFull, dcount))) break;
+        ++dcount;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t dr[32];
+          tmem_ld32(lane_tmem + C::DP_COL + c * 32, dr);
+          tmem_wait_ld();
           reg_fence32(dr);
           uint32_t g16[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int col = c * 32 + 2 * i;
-            float pa = ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -lse2));
-            float pb = ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -lse2));
-            if (valid < BN) {
-              pa = col < valid ? pa : 0.f;
-              pb = col + 1 < valid ? pb : 0.f;
-            }
-            g16[i] = pack_bf16x2(pa * (__uint_as_float(dr[2 * i]) - del),
-                                 pb * (__uint_as_float(dr[2 * i + 1]) - del));
-          }
+          for (int i = 0; i < 16; ++i)
+            g16[i] = pack_bf16x2(pf[c * 32 + 2 * i] * (__uint_as_float(dr[2 * i]) - del),
+                                 pf[c * 32 + 2 * i + 1] * (__uint_as_float(dr[2 * i + 1]) - del));
           // chunk c lands on dP columns [16c, 16c + 16): already read back
           tmem_st16(lane_tmem + C::DP_COL + c * 16, g16);
           tmem_wait_st();  // part c of the key columns handed over
           tc_fence_before();
-          mbar_arrive(&bar_p_part[c]);
+          mbar_arrive(&bar_ds_part[c]);
         }
       }
       if (!ok) break;
