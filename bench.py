@@ -32,14 +32,17 @@ if ROOT not in sys.path:
 
 METRIC = "block-sparse attn fwd ms & effective TFLOP/s vs bf16 peak at 32k–120k tokens"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ("block_sparse_attention_radial_b200/csrc/attn_fwd_pair_sm100.cuh",
-                  "block_sparse_attention_radial_b200/csrc/attn_fwd_sm100.cuh",
-                  "block_sparse_attention_radial_b200/csrc/ptx_sm100.cuh")
+CSRC = "block_sparse_attention_radial_b200/csrc/"
+KERNEL_SOURCES = {
+    "fwd": (CSRC + "attn_fwd_pair_sm100.cuh", CSRC + "attn_fwd_sm100.cuh", CSRC + "ptx_sm100.cuh"),
+    "bwd": (CSRC + "attn_bwd_sm100.cuh", CSRC + "attn_fwd_sm100.cuh", CSRC + "ptx_sm100.cuh"),
+}
+TRAFFIC_FILES = {"fwd": "attn_fwd_pair_sm100_{}_traffic.json", "bwd": "attn_bwd_sm100_{}_traffic.json"}
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(which: str = "fwd") -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[which]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -54,15 +57,16 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def load_traffic(workload: str):
-    """DRAM bytes per launch of the attention kernel from a committed ncu summary,
-    or None when the summary is missing or was taken on different kernel source."""
-    path = os.path.join(ROOT, "profiles", f"attn_fwd_pair_sm100_{workload}_traffic.json")
+def load_traffic(workload: str, which: str = "fwd"):
+    """DRAM bytes per launch (per backward call for ``which="bwd"``) of the
+    timed kernels from a committed ncu summary, or None when the summary is
+    missing or was taken on different kernel source."""
+    path = os.path.join(ROOT, "profiles", TRAFFIC_FILES[which].format(workload))
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    if d.get("kernel_source_hash") != kernel_source_hash():
+    if d.get("kernel_source_hash") != kernel_source_hash(which):
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -549,7 +553,7 @@ def run_ours_bwd(args, world, rank, local):
             "dtype": "bf16", "data": "synthetic",
             "config": workload_config(w, nnz=int(rp_h[-1])),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": None,
+                         "frac": achieved / peak, "traffic": load_traffic(w.name, "bwd"),
                          "peak_kind": f"{peak_kind} bf16 burst",
                          "kernel": "attn_bwd_dkdv_kernel<128> + attn_bwd_dq_kernel<128> "
                                    "(+ prep and transposed lists)",
