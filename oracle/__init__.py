@@ -24,6 +24,8 @@ Modules:
   constructions (brute force over the token mask; per-token key intervals).
 * ``attention``: masked softmax attention over block lists, in float64.
 * ``attention_backward``: its gradients (dQ, dK, dV), in float64.
+* ``module``: the RadialAttention module forward (projections, head split,
+  attention, head merge, output projection), in float64.
 """
 
 from .radial_mask import (  # noqa: F401
@@ -48,4 +50,8 @@ from .attention_backward import (  # noqa: F401
     masked_attention_backward_fp64,
     masked_attention_dq_rows,
     masked_attention_dkdv_keys,
+)
+from .module import (  # noqa: F401
+    radial_attention_module_fp64,
+    radial_attention_module_rows,
 )

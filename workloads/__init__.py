@@ -90,6 +90,28 @@ def make_random_qkv(batch, heads, n, head_dim, seed, device="cpu", scale=1.0):
                  .to(torch.bfloat16).contiguous() for _ in range(3))
 
 
+def make_module_inputs(batch, n, heads, head_dim, seed, device="cpu", bias=True):
+    """Seeded bf16 inputs of the radial attention module: ``x [batch, n, C]``
+    ~ N(0, 1); stacked ``w_qkv [3C, C]`` and ``w_out [C, C]`` ~ N(0, 1/C) (unit
+    variance after projection, like a trained layer's scale); biases ~
+    N(0, 0.1^2) or None. ``C = heads * head_dim``. Returns
+    ``(x, w_qkv, b_qkv, w_out, b_out)``."""
+    C = heads * head_dim
+    dev = torch.device(device)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+
+    def draw(shape, std):
+        return (torch.randn(shape, generator=g, device=dev) * std).to(torch.bfloat16).contiguous()
+
+    x = draw((batch, n, C), 1.0)
+    w_qkv = draw((3 * C, C), C ** -0.5)
+    w_out = draw((C, C), C ** -0.5)
+    b_qkv = draw((3 * C,), 0.1) if bias else None
+    b_out = draw((C,), 0.1) if bias else None
+    return x, w_qkv, b_qkv, w_out, b_out
+
+
 # ----------------------------------------------------------------------------
 # Per-head tile patterns for the generic workload (tile = one block).
 # Families: the diagonal, multi-diagonal and vertical-stripe patterns of the
