@@ -572,6 +572,169 @@ def run_ours_bwd(args, world, rank, local):
     return 0
 
 
+METRIC_MODULE = ("radial attention module fwd (q/k/v projection, block-sparse attention, "
+                 "out projection) ms & effective TFLOP/s at 32k-120k tokens")
+
+
+def run_ours_module(args, world, rank, local):
+    """Time bsa_attn_module_fwd: the RadialAttention module forward of the
+    skill page (one stacked q/k/v projection GEMM, the attention on strided
+    views of its output, the output projection GEMM), with random-init
+    weights of the workload's width (C = heads x head_dim). value counts the
+    two GEMMs' FLOPs plus the attention's computed-block FLOPs."""
+    import numpy as np
+    import torch
+
+    import block_sparse_attention_radial_b200 as bsa
+    from workloads import WORKLOADS, make_module_inputs
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    w = WORKLOADS[args.workload]
+    H, D, n = w.heads, w.head_dim, w.n
+    x, wqkv, bqkv, wo, bo = make_module_inputs(w.batch, n, H, D, w.seed, device=dev)
+    lists = bsa.radial_block_lists(w.frames, w.tokens_per_frame, w.block, device=dev)
+    rp_h, ci_h = lists.row_ptr.cpu().numpy(), lists.col_idx.cpu().numpy()
+    att_flops = bsa.computed_flops(rp_h, ci_h, n, w.block, D, w.batch, H, 1)
+    flops = bsa.module_flops(w.batch, n, H, D, att_flops)
+    y = torch.empty_like(x)
+    ws = torch.empty(bsa.bsa_attn_module_workspace_bytes(w.batch, n, H, D, lists),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 2  # work order, attention (the two GEMMs are cuBLASLt's)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        bsa.bsa_attn_module_fwd(x, wqkv, bqkv, wo, bo, H, lists, y, ws, 0.0, stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if bsa.bsa_get_device_status() != 0:
+        raise SystemExit("device status after warm-up")
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid).replace("GPU-", "")
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid) if rank == 0 else None
+    if sampler is not None:
+        time.sleep(0.4)
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(kev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    clocks = sampler.stop() if sampler is not None else None
+    ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
+    kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    if bsa.bsa_get_device_status() != 0:
+        raise SystemExit("device status after the timed region")
+
+    # end to end: x from pinned host memory in, y back to the host
+    e2e_steps = max(3, min(args.steps, 10))
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    x_dev = torch.empty_like(x)
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        bsa.bsa_attn_module_fwd(x_dev, wqkv, bqkv, wo, bo, H, lists, y, ws, 0.0, stream)
+        y_host.copy_(y, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
+    h2d = x_host.numel() * x_host.element_size()
+    d2h = y_host.numel() * y_host.element_size()
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        C = H * D
+        xc, wqc, bqc, woc, boc = (t.cpu() for t in (x, wqkv, bqkv, wo, bo))
+        rows = np.arange(n // 2, min(n, n // 2 + 64))
+        valid = np.minimum(w.block, n - np.arange(w.nqb) * w.block)
+        att_row = sum(4 * D * int(valid[ci_h[rp_h[r // w.block]:rp_h[r // w.block + 1]]].sum())
+                      for r in rows)
+
+        def sample_flops(h):  # K, V projections of h heads, Q rows, attention rows, out_proj
+            return h * (4 * n * C * D + 2 * rows.size * C * D + att_row + 2 * rows.size * D * C)
+
+        for _ in range(2):  # the first call pays one-time costs
+            t0 = time.perf_counter()
+            oracle.radial_attention_module_rows(xc, wqc, bqc, woc, boc, H, rp_h, ci_h, 1,
+                                                w.block, 0, rows, heads_used=[0])
+            t_one = max(time.perf_counter() - t0, 1e-3)
+        hs = int(max(1, min(H, args.cpu_seconds / t_one)))
+        t0 = time.perf_counter()
+        oracle.radial_attention_module_rows(xc, wqc, bqc, woc, boc, H, rp_h, ci_h, 1, w.block, 0,
+                                            rows, heads_used=list(range(hs)))
+        dt = time.perf_counter() - t0
+        cpu_baseline = {"value": sample_flops(hs) / dt / 1e12, "unit": "TFLOP/s",
+                        "cores": blas_threads(), "kind": "oracle",
+                        "sample": f"module output rows {int(rows[0])}..{int(rows[-1])} of batch 0 "
+                                  f"through heads 0..{hs - 1} (their k/v projections of all "
+                                  f"{n} tokens, q rows, attention rows, out_proj columns), "
+                                  f"{dt:.1f} s, fp64 NumPy"}
+
+    if rank == 0:
+        peaks, peak_kind = load_peaks()
+        peak = float(peaks["bf16_tflops"])
+        achieved = flops / (kernel_ms * 1e-3) / 1e12
+        cfg = workload_config(w, nnz=int(rp_h[-1]))
+        cfg["hidden"] = H * D
+        cfg["l2"] = ("x and the q/k/v projection output exceed L2 (126 MB) many times over; "
+                     "no flush")
+        line = {
+            "metric": METRIC_MODULE,
+            "value": flops * world * args.steps / (ms * 1e-3) / 1e12,
+            "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (random-init weights)",
+            "config": cfg,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_kind": f"{peak_kind} bf16 burst",
+                         "kernel": "whole module: cuBLASLt q/k/v GEMM + work order + "
+                                   "attn_fwd_pair_sm100_kernel<128> + cuBLASLt out GEMM",
+                         "kernel_ms": kernel_ms, "flops_per_launch": flops},
+            "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+            "cpu_baseline": cpu_baseline,
+        }
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -581,8 +744,9 @@ def main(argv=None):
     ap.add_argument("--workload", default="wan", choices=("wan", "hunyuan", "long4x", "tiny"))
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="which", choices=("fwd", "bwd"), default="fwd",
-                    help="time the forward (default, the headline) or the backward pass")
+    ap.add_argument("--pass", dest="which", choices=("fwd", "bwd", "module"), default="fwd",
+                    help="time the forward (default, the headline), the backward pass or the "
+                         "whole module forward (projections + attention)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -591,6 +755,8 @@ def main(argv=None):
         return run_reference(args, world, rank)
     if args.which == "bwd":
         return run_ours_bwd(args, world, rank, local)
+    if args.which == "module":
+        return run_ours_module(args, world, rank, local)
     return run_ours(args, world, rank, local)
 
 

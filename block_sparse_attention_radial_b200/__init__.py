@@ -20,7 +20,7 @@ from dataclasses import dataclass
 import torch
 
 from . import _lib
-from ._lib import BlockListsC, STATUS_NAMES
+from ._lib import BlockListsC, LayoutC, STATUS_NAMES
 
 __all__ = [
     "BsaError", "BlockLists", "bsa_radial_mask_build", "bsa_attn_fwd_workspace_bytes",
@@ -28,6 +28,9 @@ __all__ = [
     "bsa_get_timeout_detail", "bsa_status_string", "bsa_last_cuda_error", "bsa_set_test_hooks",
     "radial_block_lists", "block_lists_from_csr", "attention", "dense_masked_reference",
     "computed_flops", "bsa_attn_fwd_noalloc", "bsa_selftest_exp2", "NOALLOC_MAX_ORDER_ENTRIES",
+    "bsa_attn_fwd_strided", "bsa_attn_module_workspace_bytes", "bsa_attn_module_fwd",
+    "attention_module", "module_flops", "bsa_attn_bwd", "bsa_attn_bwd_workspace_bytes",
+    "attention_backward",
 ]
 
 # Size of the fixed scratch array behind bsa_attn_fwd_noalloc (int32 entries).
@@ -116,6 +119,60 @@ def bsa_attn_fwd(q, k, v, lists: BlockLists, out, lse=None, workspace=None,
                           ctypes.byref(ls), _ptr(out), _ptr(lse), _ptr(workspace),
                           workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "bsa_attn_fwd")
+
+
+def _layout(t) -> LayoutC:
+    """bsa_layout of a [batch, heads, n, head_dim] view with a contiguous last axis."""
+    if t.dim() != 4 or t.stride(3) != 1:
+        raise ValueError("expected a [batch, heads, n, head_dim] view with a contiguous last axis")
+    return LayoutC(t.stride(0), t.stride(1), t.stride(2))
+
+
+def bsa_attn_fwd_strided(q, k, v, lists: BlockLists, out, lse=None, workspace=None,
+                         softmax_scale: float = 0.0, stream=None) -> None:
+    """bsa_attn_fwd on strided [B, H, n, D] views (e.g. ``x.view(B, n, H, D).transpose(1, 2)``):
+    the kernels read q, k, v and write out through their strides, no copy."""
+    B, H, n, D = q.shape
+    lib = _lib.load()
+    ls = lists.c_struct()
+    if workspace is None:
+        workspace = torch.empty(max(lib.bsa_attn_fwd_workspace_bytes(B, H, ctypes.byref(ls)), 16),
+                                dtype=torch.uint8, device=q.device)
+    lq, lk, lv, lo = (_layout(t) for t in (q, k, v, out))
+    st = lib.bsa_attn_fwd_strided(_ptr(q), ctypes.byref(lq), _ptr(k), ctypes.byref(lk), _ptr(v),
+                                  ctypes.byref(lv), B, H, n, D, float(softmax_scale),
+                                  ctypes.byref(ls), _ptr(out), ctypes.byref(lo), _ptr(lse),
+                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  _stream(stream))
+    _check(st, "bsa_attn_fwd_strided")
+
+
+def bsa_attn_module_workspace_bytes(batch: int, n: int, heads: int, head_dim: int,
+                                    lists: BlockLists) -> int:
+    return int(_lib.load().bsa_attn_module_workspace_bytes(batch, n, heads, head_dim,
+                                                           ctypes.byref(lists.c_struct())))
+
+
+def bsa_attn_module_fwd(x, w_qkv, b_qkv, w_out, b_out, heads: int, lists: BlockLists, y,
+                        workspace=None, softmax_scale: float = 0.0, stream=None) -> None:
+    """Radial attention module forward (projections, attention, out projection):
+    x, y bf16 [B, n, C]; w_qkv [3C, C]; w_out [C, C]; biases [3C] / [C] or None."""
+    B, n, C = x.shape
+    D = C // heads
+    lib = _lib.load()
+    ls = lists.c_struct()
+    if workspace is None:
+        workspace = torch.empty(lib.bsa_attn_module_workspace_bytes(B, n, heads, D,
+                                                                    ctypes.byref(ls)),
+                                dtype=torch.uint8, device=x.device)
+    for t in (x, w_qkv, b_qkv, w_out, b_out, y):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("bsa_attn_module_fwd takes contiguous tensors")
+    st = lib.bsa_attn_module_fwd(_ptr(x), _ptr(w_qkv), _ptr(b_qkv), _ptr(w_out), _ptr(b_out), B, n,
+                                 heads, D, float(softmax_scale), ctypes.byref(ls), _ptr(y),
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                 _stream(stream))
+    _check(st, "bsa_attn_module_fwd")
 
 
 def bsa_attn_fwd_noalloc(q, k, v, lists: BlockLists, out, lse=None,
@@ -232,13 +289,38 @@ def block_lists_from_csr(row_ptr, col_idx, num_lists: int, num_q_blocks: int, bl
 
 
 def attention(q, k, v, lists: BlockLists, softmax_scale: float = 0.0, want_lse: bool = True,
-              workspace=None, stream=None):
-    """Allocate outputs and run :func:`bsa_attn_fwd`; returns ``(out, lse)``."""
-    B, H, n, _ = q.shape
-    out = torch.empty_like(q)
+              workspace=None, stream=None, out=None):
+    """Run the forward on [B, H, n, D] tensors; returns ``(out, lse)``.
+
+    Contiguous q, k, v (and ``out``, allocated contiguous when not given) go to
+    :func:`bsa_attn_fwd`; strided views (a contiguous last axis, e.g. heads
+    split off a [B, n, H*D] projection by ``view(B, n, H, D).transpose(1, 2)``)
+    to :func:`bsa_attn_fwd_strided`, which reads and writes them in place."""
+    B, H, n, D = q.shape
+    if out is None:
+        out = torch.empty((B, H, n, D), dtype=q.dtype, device=q.device)
     lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device) if want_lse else None
-    bsa_attn_fwd(q, k, v, lists, out, lse, workspace, softmax_scale, stream)
+    if all(t.is_contiguous() for t in (q, k, v, out)):
+        bsa_attn_fwd(q, k, v, lists, out, lse, workspace, softmax_scale, stream)
+    else:
+        bsa_attn_fwd_strided(q, k, v, lists, out, lse, workspace, softmax_scale, stream)
     return out, lse
+
+
+def attention_module(x, w_qkv, b_qkv, w_out, b_out, heads: int, lists: BlockLists,
+                     softmax_scale: float = 0.0, workspace=None, stream=None):
+    """Allocate y and run :func:`bsa_attn_module_fwd`; returns y (bf16 [B, n, C])."""
+    y = torch.empty_like(x)
+    bsa_attn_module_fwd(x, w_qkv, b_qkv, w_out, b_out, heads, lists, y, workspace, softmax_scale,
+                        stream)
+    return y
+
+
+def module_flops(batch: int, n: int, heads: int, head_dim: int, attention_flops: int) -> int:
+    """FLOPs of one module forward: the two projection GEMMs (2*rows*C*3C and
+    2*rows*C*C) plus the attention's computed-block FLOPs."""
+    C = heads * head_dim
+    return 8 * batch * n * C * C + int(attention_flops)
 
 
 def attention_backward(q, k, v, out, dout, lse, lists: BlockLists, softmax_scale: float = 0.0,

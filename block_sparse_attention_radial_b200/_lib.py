@@ -18,6 +18,9 @@ EXPORTS = (
     "bsa_radial_mask_build",
     "bsa_attn_fwd_workspace_bytes",
     "bsa_attn_fwd",
+    "bsa_attn_fwd_strided",
+    "bsa_attn_module_workspace_bytes",
+    "bsa_attn_module_fwd",
     "bsa_attn_dense_masked_ref",
     "bsa_attn_bwd",
     "bsa_attn_bwd_workspace_bytes",
@@ -57,6 +60,16 @@ class BlockListsC(ctypes.Structure):
     ]
 
 
+class LayoutC(ctypes.Structure):
+    """Mirror of ``bsa_layout`` (element strides; head_dim contiguous)."""
+
+    _fields_ = [
+        ("batch_stride", ctypes.c_int64),
+        ("head_stride", ctypes.c_int64),
+        ("token_stride", ctypes.c_int64),
+    ]
+
+
 _lib = None
 
 
@@ -72,11 +85,17 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib = ctypes.CDLL(path)
     i32, i64, vp, sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
     lp = ctypes.POINTER(BlockListsC)
+    yp = ctypes.POINTER(LayoutC)
     sig = {
         "bsa_radial_mask_build": (ctypes.c_int, [i32, i32, i32, vp, vp, i64, ctypes.POINTER(i64), vp]),
         "bsa_attn_fwd_workspace_bytes": (sz, [i32, i32, lp]),
         "bsa_attn_fwd": (ctypes.c_int, [vp, vp, vp, i32, i32, i32, i32, ctypes.c_float, lp,
                                         vp, vp, vp, sz, vp]),
+        "bsa_attn_fwd_strided": (ctypes.c_int, [vp, yp, vp, yp, vp, yp, i32, i32, i32, i32,
+                                                ctypes.c_float, lp, vp, yp, vp, vp, sz, vp]),
+        "bsa_attn_module_workspace_bytes": (sz, [i32, i32, i32, i32, lp]),
+        "bsa_attn_module_fwd": (ctypes.c_int, [vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                               ctypes.c_float, lp, vp, vp, sz, vp]),
         "bsa_attn_dense_masked_ref": (ctypes.c_int, [vp, vp, vp, i32, i32, i32, i32, ctypes.c_float,
                                                      lp, vp, vp, vp]),
         "bsa_validate_lists": (ctypes.c_int, [lp, vp]),

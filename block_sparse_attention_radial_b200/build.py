@@ -12,7 +12,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = [os.path.join(HERE, "csrc", "libbsa.cu")]
+SOURCES = [os.path.join(HERE, "csrc", "libbsa.cu"), os.path.join(HERE, "csrc", "module.cu")]
 OUTPUT = os.path.join(HERE, "libbsa.so")
 GENCODE = "arch=compute_100a,code=sm_100a"
 
@@ -24,10 +24,16 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found")
 
 
+def cuda_lib_dir() -> str:
+    return os.path.join(os.path.dirname(os.path.dirname(os.path.realpath(nvcc_path()))), "lib64")
+
+
 def build(verbose: bool = False, output: str = OUTPUT) -> str:
+    libdir = cuda_lib_dir()
     cmd = [nvcc_path(), "-gencode", GENCODE, "-lineinfo", "-O3", "-std=c++17",
            "-Xcompiler", "-fPIC", "-shared", "-I", os.path.join(ROOT, "include"),
-           "-o", output + ".tmp"] + SOURCES
+           "-o", output + ".tmp"] + SOURCES + [
+           "-L" + libdir, "-lcublasLt", "-Xlinker", "-rpath," + libdir]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     res = subprocess.run(cmd, capture_output=True, text=True)

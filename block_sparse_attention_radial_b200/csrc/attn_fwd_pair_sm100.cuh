@@ -239,8 +239,9 @@ __global__ void __launch_bounds__(320, 1)
         if (it.lenA == 0 && it.lenB == 0) continue;
         if (!(ok = lane_wait(&bar_q_empty, (qcount & 1u) ^ 1u, wc, kBarQEmpty, qcount))) break;
         mbar_arrive_expect_tx(&bar_q_full, 2 * C::Q_BYTES);
-        tma_load_4d(sQ, &tm_q, &bar_q_full, 0, it.qa * BN, 0, it.bh);
-        tma_load_4d(sQ + C::Q_BYTES, &tm_q, &bar_q_full, 0, (it.qa + 1) * BN, 0, it.bh);
+        const int ib = it.bh / p.heads, ih = it.bh - ib * p.heads;
+        tma_load_5d(sQ, &tm_q, &bar_q_full, 0, it.qa * BN, 0, ih, ib);
+        tma_load_5d(sQ + C::Q_BYTES, &tm_q, &bar_q_full, 0, (it.qa + 1) * BN, 0, ih, ib);
         ++qcount;
         // Same walk and same first-use order as the MMA issuer: at step j it
         // needs V(j-1) first when tile A listed j-1 or A skips j, and K(j)
@@ -282,8 +283,8 @@ __global__ void __launch_bounds__(320, 1)
               continue;
             }
             mbar_arrive_expect_tx(&bar_kv_full[s], C::TILE_BYTES);
-            tma_load_4d(sKV + s * C::TILE_BYTES, is_v ? &tm_v : &tm_k, &bar_kv_full[s], 0,
-                        (is_v ? prev_kb : kb) * BN, 0, it.bh);
+            tma_load_5d(sKV + s * C::TILE_BYTES, is_v ? &tm_v : &tm_k, &bar_kv_full[s], 0,
+                        (is_v ? prev_kb : kb) * BN, 0, ih, ib);
             ++ring;
           }
           pa = a;
@@ -464,9 +465,11 @@ __global__ void __launch_bounds__(320, 1)
       const int row = qb * BN + row_in_tile;
       const bool store = row < p.n;
       const long long orow = static_cast<long long>(it.bh) * p.n + row;
+      const int ib = it.bh / p.heads, ih = it.bh - ib * p.heads;
+      __nv_bfloat16 *const orow_ptr = p.out + ib * p.o_sb + ih * p.o_sh + row * p.o_sn;
       if (len == 0) {
         if (store) {
-          uint4 *dst = reinterpret_cast<uint4 *>(p.out + orow * D);
+          uint4 *dst = reinterpret_cast<uint4 *>(orow_ptr);
 #pragma unroll
           for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
           if (p.lse) p.lse[orow] = -INFINITY;
@@ -564,7 +567,7 @@ __global__ void __launch_bounds__(320, 1)
         tmem_wait_ld();
         reg_fence32(r);
         if (store) {
-          uint4 *dst = reinterpret_cast<uint4 *>(p.out + orow * D + c * 32);
+          uint4 *dst = reinterpret_cast<uint4 *>(orow_ptr + c * 32);
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4) {
             uint4 w;

@@ -40,6 +40,8 @@ namespace bsa {
 struct FwdParams {
   const int32_t *row_ptr, *col_idx, *order;
   __nv_bfloat16 *out;
+  // element strides of out's batch, head and token axes (head_dim contiguous)
+  long long o_sb, o_sh, o_sn;
   float *lse;
   int32_t heads, n, nqb, nkb, num_lists, nnz;
   int32_t total_items;
@@ -317,9 +319,10 @@ __global__ void __launch_bounds__(192, 1)
       const Item it = decode_item(idx, p);
       if (it.len == 0) continue;
       if (!(ok = warp_wait(&bar_q_empty, (qcount & 1u) ^ 1u, wc, kBarQEmpty, qcount))) break;
+      const int ib = it.bh / p.heads, ih = it.bh - ib * p.heads;
       if (leader) {
         mbar_arrive_expect_tx(&bar_q_full, C::Q_BYTES);
-        tma_load_4d(sQ, &tm_q, &bar_q_full, 0, it.qb * BN, 0, it.bh);
+        tma_load_5d(sQ, &tm_q, &bar_q_full, 0, it.qb * BN, 0, ih, ib);
       }
       ++qcount;
       // Walk the blocks as the MMA warp does (step j: QK(j+1), then PV(j),
@@ -348,8 +351,8 @@ __global__ void __launch_bounds__(192, 1)
           }
           if (leader) {
             mbar_arrive_expect_tx(&bar_kv_full[s], C::STAGE_BYTES);
-            tma_load_4d(sKV + s * C::STAGE_BYTES, is_k ? &tm_k : &tm_v, &bar_kv_full[s], 0,
-                        w.kb * BN, 0, it.bh);
+            tma_load_5d(sKV + s * C::STAGE_BYTES, is_k ? &tm_k : &tm_v, &bar_kv_full[s], 0,
+                        w.kb * BN, 0, ih, ib);
           }
           ++ring;
         }
@@ -499,9 +502,11 @@ __global__ void __launch_bounds__(192, 1)
       const int row = it.qb * BN + row_in_tile;
       const bool store = row_in_tile < BN && row < p.n;
       const long long orow = static_cast<long long>(it.bh) * p.n + row;
+      const int ib = it.bh / p.heads, ih = it.bh - ib * p.heads;
+      __nv_bfloat16 *const orow_ptr = p.out + ib * p.o_sb + ih * p.o_sh + row * p.o_sn;
       if (it.len == 0) {
         if (store) {
-          uint4 *dst = reinterpret_cast<uint4 *>(p.out + orow * D);
+          uint4 *dst = reinterpret_cast<uint4 *>(orow_ptr);
 #pragma unroll
           for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
           if (p.lse) p.lse[orow] = -INFINITY;
@@ -616,7 +621,7 @@ __global__ void __launch_bounds__(192, 1)
         tmem_wait_ld();
         reg_fence32(r);
         if (store) {
-          uint4 *dst = reinterpret_cast<uint4 *>(p.out + orow * D + c * 32);
+          uint4 *dst = reinterpret_cast<uint4 *>(orow_ptr + c * 32);
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4) {
             uint4 w;

@@ -120,7 +120,89 @@ int make_map(CUtensorMap *map, const void *ptr, int bh, int n, int D, int rows) 
   return BSA_OK;
 }
 
+// A [batch, heads, n, D] bf16 view with arbitrary batch / head / token strides
+// (elements; D contiguous) as a 5-D tensor {64 columns, n rows, D/64 column
+// halves, heads, batch}: the same {64, rows, D/64} box as make_map, with the
+// head and batch coordinates kept apart so that token-major layouts (the
+// [batch, n, heads, D] output of a fused projection) load without a
+// transpose. An axis of extent 1 gets a placeholder stride (never used).
+int make_map_strided(CUtensorMap *map, const void *ptr, const bsa_layout &L, int batch,
+                     int heads, int n, int D, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    std::snprintf(t_last_error, sizeof(t_last_error), "cuTensorMapEncodeTiled not available");
+    return BSA_ERR_CUDA;
+  }
+  cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(n), static_cast<cuuint64_t>(D / 64),
+                        static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[4] = {static_cast<cuuint64_t>(L.token_stride) * 2, 128,
+                           heads > 1 ? static_cast<cuuint64_t>(L.head_stride) * 2 : 128,
+                           batch > 1 ? static_cast<cuuint64_t>(L.batch_stride) * 2 : 128};
+  cuuint32_t box[5] = {64, static_cast<cuuint32_t>(rows), static_cast<cuuint32_t>(D / 64), 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(ptr), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(t_last_error, sizeof(t_last_error), "cuTensorMapEncodeTiled failed (%d)",
+                  static_cast<int>(r));
+    return BSA_ERR_CUDA;
+  }
+  return BSA_OK;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bsa_layout contiguous_layout(int heads, int n, int D) {
+  bsa_layout L;
+  L.token_stride = D;
+  L.head_stride = static_cast<int64_t>(n) * D;
+  L.batch_stride = static_cast<int64_t>(heads) * n * D;
+  return L;
+}
+
+// A layout the kernels can use: every stride of an axis longer than one is
+// positive, a multiple of 8 elements (16 bytes, for TMA and the 16-byte
+// output stores) and below 2^39 elements (TMA's 2^40-byte stride limit).
+bool layout_ok(const bsa_layout &L, int batch, int heads, int n) {
+  const int64_t lim = int64_t(1) << 39;
+  auto good = [&](int64_t st, int extent) {
+    return extent <= 1 || (st > 0 && st % 8 == 0 && st < lim);
+  };
+  return good(L.token_stride, n) && good(L.head_stride, heads) && good(L.batch_stride, batch);
+}
+
+// Bytes from the first to one past the last element a layout addresses.
+size_t layout_span_bytes(const bsa_layout &L, int batch, int heads, int n, int D) {
+  const int64_t last = (batch > 1 ? (batch - 1) * L.batch_stride : 0) +
+                       (heads > 1 ? (heads - 1) * L.head_stride : 0) +
+                       (n > 1 ? (n - 1) * L.token_stride : 0) + D;
+  return static_cast<size_t>(last) * 2;
+}
+
+// No two (batch, head, token) rows of the layout share an element: sorted by
+// stride, each axis steps past everything the inner axes span. Required of
+// the output, whose rows are written concurrently.
+bool layout_disjoint(const bsa_layout &L, int batch, int heads, int n, int D) {
+  struct Ax {
+    int64_t st;
+    int ext;
+  } ax[3] = {{L.token_stride, n}, {L.head_stride, heads}, {L.batch_stride, batch}};
+  for (int i = 0; i < 3; ++i)
+    for (int j = i + 1; j < 3; ++j)
+      if (ax[j].st < ax[i].st) {
+        const Ax t = ax[i];
+        ax[i] = ax[j];
+        ax[j] = t;
+      }
+  int64_t inner = D;  // elements spanned by the axes already placed
+  for (int i = 0; i < 3; ++i) {
+    if (ax[i].ext <= 1) continue;
+    if (ax[i].st < inner) return false;
+    inner = ax[i].st * (ax[i].ext - 1) + inner;
+  }
+  return true;
+}
 
 bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
@@ -152,21 +234,61 @@ int check_attn_args(const void *q, const void *k, const void *v, int32_t batch, 
   return BSA_OK;
 }
 
+// Argument checks of the strided entry point: those of check_attn_args (with
+// the overlap test made layout-aware) plus the layouts themselves.
+int check_strided_args(const void *q, const bsa_layout *lq, const void *k, const bsa_layout *lk,
+                       const void *v, const bsa_layout *lv, int32_t batch, int32_t heads,
+                       int32_t n, int32_t head_dim, const bsa_block_lists *l, const void *out,
+                       const bsa_layout *lo) {
+  if (!lq || !lk || !lv || !lo) return BSA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !out || !l || !l->row_ptr || (l->nnz > 0 && !l->col_idx))
+    return BSA_ERR_INVALID_ARG;
+  if (batch < 1 || heads < 1 || n < 1) return BSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
+  if (l->block != 64 && l->block != 128) return BSA_ERR_UNSUPPORTED;
+  const long long nb = (static_cast<long long>(n) + l->block - 1) / l->block;
+  if (l->num_q_blocks != nb || l->num_k_blocks != nb) return BSA_ERR_INVALID_ARG;
+  if (l->num_lists != 1 && l->num_lists != heads) return BSA_ERR_INVALID_ARG;
+  if (l->nnz < 0) return BSA_ERR_INVALID_ARG;
+  const long long bh = static_cast<long long>(batch) * heads;
+  if (bh * nb > 0x7fffffffLL || bh * n > 0x7fffffffLL) return BSA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return BSA_ERR_INVALID_ARG;
+  for (const bsa_layout *L : {lq, lk, lv, lo})
+    if (!layout_ok(*L, batch, heads, n)) return BSA_ERR_INVALID_ARG;
+  if (!layout_disjoint(*lo, batch, heads, n, head_dim)) return BSA_ERR_INVALID_ARG;
+  const size_t so = layout_span_bytes(*lo, batch, heads, n, head_dim);
+  if (overlaps(out, so, q, layout_span_bytes(*lq, batch, heads, n, head_dim)) ||
+      overlaps(out, so, k, layout_span_bytes(*lk, batch, heads, n, head_dim)) ||
+      overlaps(out, so, v, layout_span_bytes(*lv, batch, heads, n, head_dim)))
+    return BSA_ERR_INVALID_ARG;
+  return BSA_OK;
+}
+
 size_t order_bytes(const bsa_block_lists *l) {
   return (static_cast<size_t>(l->num_lists) * l->num_q_blocks * sizeof(int32_t) + 255) & ~size_t(255);
 }
 
 constexpr int kLptMaxRows = 12288;  // rows whose costs fit in 48 KB of shared memory
 
+// q, k, v, their layouts, batch and heads of one forward call.
+struct QkvViews {
+  const void *q, *k, *v;
+  bsa_layout lq, lk, lv;
+  int batch, heads;
+};
+
 template <int D, int BN>
-int launch_fwd(const void *q, const void *k, const void *v, int32_t bh, int32_t n,
-               const FwdParams &p, DeviceInfo *dev, int slot, cudaStream_t stream) {
+int launch_fwd(const QkvViews &x, int32_t n, const FwdParams &p, DeviceInfo *dev, int slot,
+               cudaStream_t stream) {
   using C = FwdCfg<D, BN>;
   CUtensorMap tq, tk, tv;
   int st;
-  if ((st = make_map(&tq, q, bh, n, D, C::BM)) != BSA_OK) return st;
-  if ((st = make_map(&tk, k, bh, n, D, C::STAGE_ROWS)) != BSA_OK) return st;
-  if ((st = make_map(&tv, v, bh, n, D, C::STAGE_ROWS)) != BSA_OK) return st;
+  if ((st = make_map_strided(&tq, x.q, x.lq, x.batch, x.heads, n, D, C::BM)) != BSA_OK) return st;
+  if ((st = make_map_strided(&tk, x.k, x.lk, x.batch, x.heads, n, D, C::STAGE_ROWS)) != BSA_OK)
+    return st;
+  if ((st = make_map_strided(&tv, x.v, x.lv, x.batch, x.heads, n, D, C::STAGE_ROWS)) != BSA_OK)
+    return st;
   {
     std::lock_guard<std::mutex> lk(g_dev_mu);
     if (!dev->attrs_set[slot]) {
@@ -203,14 +325,14 @@ int launch_ref(const RefParams &p, int batch, DeviceInfo *dev, int slot, cudaStr
 int slot_of(int D, int BN) { return (D == 128 ? 2 : 0) + (BN == 128 ? 1 : 0); }
 
 template <int D>
-int launch_pair(const void *q, const void *k, const void *v, int32_t bh, int32_t n,
-                const FwdParams &p, DeviceInfo *dev, cudaStream_t stream) {
+int launch_pair(const QkvViews &x, int32_t n, const FwdParams &p, DeviceInfo *dev,
+                cudaStream_t stream) {
   using C = PairCfg<D>;
   CUtensorMap tq, tk, tv;
   int st;
-  if ((st = make_map(&tq, q, bh, n, D, C::BN)) != BSA_OK) return st;
-  if ((st = make_map(&tk, k, bh, n, D, C::BN)) != BSA_OK) return st;
-  if ((st = make_map(&tv, v, bh, n, D, C::BN)) != BSA_OK) return st;
+  if ((st = make_map_strided(&tq, x.q, x.lq, x.batch, x.heads, n, D, C::BN)) != BSA_OK) return st;
+  if ((st = make_map_strided(&tk, x.k, x.lk, x.batch, x.heads, n, D, C::BN)) != BSA_OK) return st;
+  if ((st = make_map_strided(&tv, x.v, x.lv, x.batch, x.heads, n, D, C::BN)) != BSA_OK) return st;
   const int slot = 4 + (D == 128 ? 1 : 0);
   {
     std::lock_guard<std::mutex> lk(g_dev_mu);
@@ -229,10 +351,10 @@ int launch_pair(const void *q, const void *k, const void *v, int32_t bh, int32_t
 // Work order into `order`, then the attention kernel. Block-128 problems run
 // on the two-tile kernel (adjacent query blocks share K/V loads); block 64 on
 // the one-tile kernel. Arguments were checked by the caller.
-int run_fwd(const void *q, const void *k, const void *v, int32_t batch, int32_t heads,
-            int32_t n, int32_t head_dim, float softmax_scale, const bsa_block_lists *l,
-            void *out, float *lse, int32_t *order, DeviceInfo *dev, int fault_flags,
-            cudaStream_t stream) {
+int run_fwd(const QkvViews &x, int32_t n, int32_t head_dim, float softmax_scale,
+            const bsa_block_lists *l, void *out, const bsa_layout &lo, float *lse,
+            int32_t *order, DeviceInfo *dev, int fault_flags, cudaStream_t stream) {
+  const int batch = x.batch, heads = x.heads;
   const int nqb = l->num_q_blocks;
   bool pair;
   {
@@ -256,6 +378,9 @@ int run_fwd(const void *q, const void *k, const void *v, int32_t batch, int32_t 
   p.col_idx = l->col_idx;
   p.order = order;
   p.out = static_cast<__nv_bfloat16 *>(out);
+  p.o_sb = lo.batch_stride;
+  p.o_sh = lo.head_stride;
+  p.o_sn = lo.token_stride;
   p.lse = lse;
   p.heads = heads;
   p.n = n;
@@ -272,19 +397,27 @@ int run_fwd(const void *q, const void *k, const void *v, int32_t batch, int32_t 
     p.wait_limit_ns = g_wait_limit_ns;
   }
   p.fault_flags = fault_flags;
-  const int bh = batch * heads;
   if (pair) {
-    if (head_dim == 128) return launch_pair<128>(q, k, v, bh, n, p, dev, stream);
-    return launch_pair<64>(q, k, v, bh, n, p, dev, stream);
+    if (head_dim == 128) return launch_pair<128>(x, n, p, dev, stream);
+    return launch_pair<64>(x, n, p, dev, stream);
   }
   const int slot = slot_of(head_dim, l->block);
-  if (head_dim == 128 && l->block == 128)
-    return launch_fwd<128, 128>(q, k, v, bh, n, p, dev, slot, stream);
-  if (head_dim == 128 && l->block == 64)
-    return launch_fwd<128, 64>(q, k, v, bh, n, p, dev, slot, stream);
-  if (head_dim == 64 && l->block == 128)
-    return launch_fwd<64, 128>(q, k, v, bh, n, p, dev, slot, stream);
-  return launch_fwd<64, 64>(q, k, v, bh, n, p, dev, slot, stream);
+  if (head_dim == 128 && l->block == 128) return launch_fwd<128, 128>(x, n, p, dev, slot, stream);
+  if (head_dim == 128 && l->block == 64) return launch_fwd<128, 64>(x, n, p, dev, slot, stream);
+  if (head_dim == 64 && l->block == 128) return launch_fwd<64, 128>(x, n, p, dev, slot, stream);
+  return launch_fwd<64, 64>(x, n, p, dev, slot, stream);
+}
+
+QkvViews contiguous_views(const void *q, const void *k, const void *v, int batch, int heads,
+                          int n, int D) {
+  QkvViews x;
+  x.q = q;
+  x.k = k;
+  x.v = v;
+  x.lq = x.lk = x.lv = contiguous_layout(heads, n, D);
+  x.batch = batch;
+  x.heads = heads;
+  return x;
 }
 
 // ---------------------------------------------------------------- backward
@@ -478,7 +611,43 @@ int bsa_attn_fwd(const void *q, const void *k, const void *v, int32_t batch, int
     fault_flags = g_fault_flags;
     g_fault_flags = 0;
   }
-  return run_fwd(q, k, v, batch, heads, n, head_dim, softmax_scale, l, out, lse,
+  return run_fwd(contiguous_views(q, k, v, batch, heads, n, head_dim), n, head_dim,
+                 softmax_scale, l, out, contiguous_layout(heads, n, head_dim), lse,
+                 static_cast<int32_t *>(workspace), dev, fault_flags, stream);
+}
+
+int bsa_attn_fwd_strided(const void *q, const bsa_layout *q_layout, const void *k,
+                         const bsa_layout *k_layout, const void *v, const bsa_layout *v_layout,
+                         int32_t batch, int32_t heads, int32_t n, int32_t head_dim,
+                         float softmax_scale, const bsa_block_lists *l, void *out,
+                         const bsa_layout *out_layout, float *lse, void *workspace,
+                         size_t workspace_bytes, bsa_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int st = check_strided_args(q, q_layout, k, k_layout, v, v_layout, batch, heads, n, head_dim,
+                              l, out, out_layout);
+  if (st != BSA_OK) return st;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < order_bytes(l))
+    return BSA_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return BSA_ERR_INVALID_ARG;
+  DeviceInfo *dev = nullptr;
+  if ((st = current_device(&dev)) != BSA_OK) return st;
+  if (dev->cc_major != 10) return BSA_ERR_UNSUPPORTED;
+  int fault_flags;
+  {
+    std::lock_guard<std::mutex> lk(g_hook_mu);
+    fault_flags = g_fault_flags;
+    g_fault_flags = 0;
+  }
+  QkvViews x;
+  x.q = q;
+  x.k = k;
+  x.v = v;
+  x.lq = *q_layout;
+  x.lk = *k_layout;
+  x.lv = *v_layout;
+  x.batch = batch;
+  x.heads = heads;
+  return run_fwd(x, n, head_dim, softmax_scale, l, out, *out_layout, lse,
                  static_cast<int32_t *>(workspace), dev, fault_flags, stream);
 }
 
@@ -702,6 +871,7 @@ extern "C" int bsa_attn_fwd_noalloc(const void *q, const void *k, const void *v,
   int32_t *order = nullptr;
   if ((st = noalloc_scratch(&order)) != BSA_OK) return st;
 
-  return run_fwd(q, k, v, batch, heads, n, head_dim, softmax_scale, l, out, lse, order, dev, 0,
+  return run_fwd(contiguous_views(q, k, v, batch, heads, n, head_dim), n, head_dim,
+                 softmax_scale, l, out, contiguous_layout(heads, n, head_dim), lse, order, dev, 0,
                  stream);
 }

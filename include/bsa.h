@@ -142,6 +142,85 @@ int bsa_attn_fwd(const void *q, const void *k, const void *v,
                  bsa_stream_t stream);
 
 /*
+ * Strides of a [batch, heads, n, head_dim] bf16 tensor view, in elements; the
+ * head_dim axis is contiguous. The contiguous layout of bsa_attn_fwd is
+ * {heads*n*head_dim, n*head_dim, head_dim}. The token-major output of a fused
+ * q/k/v projection, [batch, n, 3, heads, head_dim] (the skill page's
+ * RadialAttention.forward projects x with q_proj, k_proj, v_proj and views the
+ * result as [batch, n, heads, head_dim] before transposing), gives q, k and v
+ * the layout {3*n*heads*head_dim, head_dim, 3*heads*head_dim} at offsets 0,
+ * heads*head_dim and 2*heads*head_dim; an output in [batch, n, heads,
+ * head_dim] order (what out_proj reads after the page's transpose back) is
+ * {n*heads*head_dim, head_dim, heads*head_dim}.
+ */
+typedef struct {
+  int64_t batch_stride;
+  int64_t head_stride;
+  int64_t token_stride;
+} bsa_layout;
+
+/*
+ * bsa_attn_fwd on strided views: the same operation and results, with q, k,
+ * v and out addressed as ptr + b*batch_stride + h*head_stride + i*token_stride
+ * + d. The kernels read the views directly (the TMA descriptors carry the
+ * strides) and write out in place, so no transpose runs before or after.
+ *
+ * Layout rules (BSA_ERR_INVALID_ARG otherwise): every stride of an axis
+ * longer than 1 is positive, a multiple of 8 and below 2^39; the pointers are
+ * 16-byte aligned; out's rows are pairwise disjoint; the span of out (first to
+ * last addressed element) overlaps none of the spans of q, k and v (which may
+ * overlap each other, e.g. as three slices of one projection buffer).
+ * lse stays [batch, heads, n] contiguous (or NULL). Other arguments,
+ * workspace and errors as bsa_attn_fwd. Asynchronous.
+ */
+int bsa_attn_fwd_strided(const void *q, const bsa_layout *q_layout,
+                         const void *k, const bsa_layout *k_layout,
+                         const void *v, const bsa_layout *v_layout,
+                         int32_t batch, int32_t heads, int32_t n, int32_t head_dim,
+                         float softmax_scale, const bsa_block_lists *lists,
+                         void *out, const bsa_layout *out_layout, float *lse,
+                         void *workspace, size_t workspace_bytes, bsa_stream_t stream);
+
+/*
+ * Bytes of device scratch bsa_attn_module_fwd needs: the projected q/k/v
+ * [batch*n, 3*heads*head_dim] bf16, the attention output [batch*n,
+ * heads*head_dim] bf16, the attention's work order and 32 MiB of GEMM
+ * scratch. Returns 0 for invalid arguments.
+ */
+size_t bsa_attn_module_workspace_bytes(int32_t batch, int32_t n, int32_t heads,
+                                       int32_t head_dim, const bsa_block_lists *lists);
+
+/*
+ * The radial attention module forward ("Radial Attention" skill page, Step 2,
+ * RadialAttention.forward):
+ *   q, k, v = q_proj(x), k_proj(x), v_proj(x), split into heads;
+ *   o = block-sparse attention of q, k, v (bsa_attn_fwd's operation);
+ *   y = out_proj(o with the heads merged back).
+ * With C = heads * head_dim:
+ * x      device bf16 [batch, n, C], row-major.
+ * w_qkv  device bf16 [3C, C]: rows [0, C) q_proj.weight, [C, 2C)
+ *        k_proj.weight, [2C, 3C) v_proj.weight (nn.Linear's [out, in]).
+ * b_qkv  device bf16 [3C] (the three biases in the same order), or NULL.
+ * w_out  device bf16 [C, C] out_proj.weight; b_out bf16 [C] or NULL.
+ * y      device bf16 [batch, n, C]; must not overlap x, the weights or the
+ *        workspace.
+ * workspace  device scratch of bsa_attn_module_workspace_bytes(); the
+ *        projected q/k/v and the attention output stay there after the call.
+ * Head h of the split is columns [h*head_dim, (h+1)*head_dim) of each
+ * projection (the page's view(batch, n, heads, head_dim)). The projections
+ * are cuBLASLt GEMMs (bf16 in, fp32 accumulate, bias in the epilogue, bf16
+ * out); the attention reads q, k, v in place from the projection output and
+ * writes o in [batch, n, heads, head_dim] order, out_proj's input layout, so
+ * no transpose runs. Pointers 16-byte aligned; other limits and errors as
+ * bsa_attn_fwd. Asynchronous.
+ */
+int bsa_attn_module_fwd(const void *x, const void *w_qkv, const void *b_qkv,
+                        const void *w_out, const void *b_out,
+                        int32_t batch, int32_t n, int32_t heads, int32_t head_dim,
+                        float softmax_scale, const bsa_block_lists *lists, void *y,
+                        void *workspace, size_t workspace_bytes, bsa_stream_t stream);
+
+/*
  * Same operation, same arguments (no workspace), computed by a plain fp32
  * CUDA-core kernel that scores every key of every listed block with scalar
  * arithmetic. It is the full-tensor checker for sizes where the CPU oracle

@@ -128,3 +128,58 @@ def test_backward_workspace_and_host_checks(lib):
     bad = list(args)
     bad[11] = ctypes.byref(ls64)
     assert lib.bsa_attn_bwd(*bad) == 2  # block 64 unsupported
+
+
+def test_strided_forward_host_checks(lib):
+    """bsa_attn_fwd_strided: layouts are validated on the host (every call
+    below is rejected before any CUDA call)."""
+    from block_sparse_attention_radial_b200._lib import BlockListsC, LayoutC
+
+    vp, ref = ctypes.c_void_p, ctypes.byref
+    B, H, n, D = 2, 4, 1024, 128
+    C = H * D
+    ls = BlockListsC(1, 8, 8, 128, 10, 1 << 22, 1 << 23)
+    base = 1 << 30                            # fake [B, n, 3, H, D] projection buffer
+    lqkv = LayoutC(n * 3 * C, D, 3 * C)
+    lo = LayoutC(n * C, D, C)                 # [B, n, H, D] output
+
+    def call(q=base, k=base + 2 * C, v=base + 4 * C, o=1 << 34, lq=lqkv, lk=lqkv, lv=lqkv,
+             lo_=lo, hd=D, wsb=1 << 12):
+        return lib.bsa_attn_fwd_strided(vp(q), lq and ref(lq), vp(k), ref(lk), vp(v), ref(lv),
+                                        B, H, n, hd, 0.0, ref(ls), vp(o), ref(lo_), None,
+                                        vp(1 << 36), wsb, None)
+
+    assert call(lq=None) == 1                                   # no layout
+    assert call(hd=96) == 2                                     # head_dim
+    assert call(k=base + 2 * C + 8) == 1                        # misaligned k
+    assert call(lk=LayoutC(n * 3 * C, D, 3 * C + 4)) == 1       # token stride not 16-byte
+    assert call(lv=LayoutC(n * 3 * C, 0, 3 * C)) == 1           # zero head stride, heads > 1
+    assert call(lo_=LayoutC(n * C, D, D)) == 1                  # output rows overlap each other
+    assert call(o=base + 6 * C) == 1                            # output inside the q/k/v span
+    assert call(wsb=4) == 1                                     # workspace too small
+
+
+def test_module_workspace_and_host_checks(lib):
+    from block_sparse_attention_radial_b200._lib import BlockListsC
+
+    vp, ref = ctypes.c_void_p, ctypes.byref
+    ls = BlockListsC(1, 256, 256, 128, 1000, 0, 0)
+    # work order (1 KiB) + q/k/v [32760, 15360] + attention out [32760, 5120] bf16 + 32 MiB
+    expect = 1024 + 32760 * 15360 * 2 + 32760 * 5120 * 2 + (32 << 20)
+    assert lib.bsa_attn_module_workspace_bytes(1, 32760, 40, 128, ref(ls)) == expect
+    assert lib.bsa_attn_module_workspace_bytes(1, 32760, 40, 128, None) == 0
+    B, n, H, D = 1, 1000, 2, 64
+    small = BlockListsC(1, 8, 8, 128, 10, 1 << 22, 1 << 23)
+    ws = lib.bsa_attn_module_workspace_bytes(B, n, H, D, ref(small))
+    x, wq, wo, y, w = (vp(a << 30) for a in (1, 2, 3, 4, 8))
+
+    def call(x=x, wq=wq, wo=wo, y=y, hd=D, wsb=ws):
+        return lib.bsa_attn_module_fwd(x, wq, None, wo, None, B, n, H, hd, 0.0, ref(small), y, w,
+                                       wsb, None)
+
+    assert call(wo=vp(0)) == 1                                  # null weight
+    assert call(hd=96) == 2                                     # head_dim
+    assert call(wsb=ws - 1) == 1                                # workspace too small
+    assert call(y=x) == 1                                       # y on top of x
+    assert call(y=vp((8 << 30) + 4096)) == 1                    # y inside the workspace
+    assert call(x=vp((1 << 30) + 8)) == 1                       # misaligned x
