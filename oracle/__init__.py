@@ -21,7 +21,8 @@ Everything is plain NumPy in float64. Pages cited (tag: page title, site):
 Modules:
 
 * ``radial_mask``: the token-level radial rule and two independent block-list
-  constructions (brute force over the token mask; per-token key intervals).
+  constructions (brute force over the token mask; per-token key intervals);
+  the joint text + video lists (text tokens appended, attended globally).
 * ``attention``: masked softmax attention over block lists, in float64.
 * ``attention_backward``: its gradients (dQ, dK, dV), in float64.
 * ``module``: the RadialAttention module forward (projections, head split,
@@ -39,6 +40,9 @@ from .radial_mask import (  # noqa: F401
     radial_block_lists_bruteforce,
     radial_block_lists_intervals,
     radial_block_lists,
+    joint_token_mask,
+    joint_block_lists_bruteforce,
+    joint_block_lists,
 )
 from .attention import (  # noqa: F401
     expand_row_mask,

@@ -180,3 +180,55 @@ def radial_block_lists(F: int, S: int, B: int, method: str = "auto"):
     if method == "bruteforce" or (method == "auto" and F * S <= 4096):
         return radial_block_lists_bruteforce(F, S, B)
     return radial_block_lists_intervals(F, S, B)
+
+
+# ------------------------------------------------- joint text + video tokens --
+#
+# Reading (the pages are silent on text tokens): a video DiT that runs joint
+# attention over its video tokens and T text tokens appends the text tokens
+# after the F*S video tokens. The radial rule applies between video tokens
+# only; a text query attends to every token and every query attends to every
+# text key (text is global context, never thinned). Blocks are cut over the
+# whole joint sequence from token 0, so the block holding the last video
+# tokens may also hold the first text tokens.
+
+
+def joint_token_mask(F: int, S: int, T: int, B: int) -> np.ndarray:
+    """Dense ``[n, n]`` mask, ``n = F*S + T``: the radial token rule among the
+    video tokens, every pair with a text token (row or column) admitted.
+    Brute force; tiny grids only."""
+    nv = F * S
+    mask = np.ones((nv + T, nv + T), dtype=bool)
+    mask[:nv, :nv] = radial_token_mask(F, S, B)
+    return mask
+
+
+def joint_block_lists_bruteforce(F: int, S: int, T: int, B: int):
+    """Joint block lists from the brute-force token mask (tiny grids only)."""
+    return block_lists_from_token_mask(joint_token_mask(F, S, T, B), B)
+
+
+def joint_block_lists(F: int, S: int, T: int, B: int, method: str = "auto"):
+    """Joint block lists for any size.
+
+    Composed from the radial block lists of the video tokens alone: a query
+    block holding only video tokens keeps its radial key blocks and gains
+    every key block that holds a text token (blocks ``>= (F*S) // B``); a
+    query block holding any text token lists every key block.
+    """
+    nv = F * S
+    n = nv + T
+    if method == "bruteforce" or (method == "auto" and n <= 4096):
+        return joint_block_lists_bruteforce(F, S, T, B)
+    # method "compose" (or "auto" above 4096 tokens)
+    nb = -(-n // B)
+    rp_v, ci_v = radial_block_lists(F, S, B)
+    first_text_block = nv // B if T > 0 else nb
+    active = np.zeros((nb, nb), dtype=bool)
+    for qb in range(nb):
+        if min(n, (qb + 1) * B) > nv:  # holds a text query
+            active[qb] = True
+            continue
+        active[qb, ci_v[rp_v[qb]:rp_v[qb + 1]]] = True
+        active[qb, first_text_block:] = True
+    return _csr_from_dense(active)
