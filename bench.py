@@ -230,7 +230,7 @@ def run_reference(args, world, rank):
 
     w = WORKLOADS[args.workload]
     q, k, v = make_qkv(w, "cpu", heads=1)
-    rp, ci = oracle.radial_block_lists(w.frames, w.tokens_per_frame, w.block)
+    rp, ci = oracle.joint_block_lists(w.frames, w.tokens_per_frame, w.text_tokens, w.block)
     per_step = max(0.2, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
     rate, dt, rows, fl = oracle_sample_rate(w, (rp, ci), q, k, v, per_step)
     times = []
@@ -260,8 +260,10 @@ def run_reference(args, world, rank):
 
 
 def workload_config(w, nnz):
+    text = f" + {w.text_tokens} text tokens" if w.text_tokens else ""
     return {"workload": f"{w.name}: B={w.batch} H={w.heads} D={w.head_dim} "
-                        f"{w.frames}x{w.tokens_per_frame} tokens (n={w.n}), radial {w.block}x{w.block} blocks",
+                        f"{w.frames}x{w.tokens_per_frame} tokens{text} (n={w.n}), radial "
+                        f"{w.block}x{w.block} blocks",
             "global_batch": w.batch, "heads": w.heads, "head_dim": w.head_dim, "seq_len": w.n,
             "frames": w.frames, "tokens_per_frame": w.tokens_per_frame, "block": w.block,
             "nnz_blocks_per_head": nnz, "parallelism": "independent problem per GPU",
@@ -284,7 +286,8 @@ def run_ours(args, world, rank, local):
     assert w.radial, "the bench times the radial path"
 
     q, k, v = make_qkv(w, dev)
-    lists = bsa.radial_block_lists(w.frames, w.tokens_per_frame, w.block, device=dev)
+    lists = bsa.radial_block_lists(w.frames, w.tokens_per_frame, w.block, device=dev,
+                                  text_tokens=w.text_tokens)
     rp_h, ci_h = lists.row_ptr.cpu().numpy(), lists.col_idx.cpu().numpy()
     flops = bsa.computed_flops(rp_h, ci_h, w.n, w.block, w.head_dim, w.batch, w.heads, 1)
     dense_flops = 4 * w.head_dim * w.batch * w.heads * w.n * w.n
@@ -436,7 +439,8 @@ def run_ours_bwd(args, world, rank, local):
     g = torch.Generator(device=dev)
     g.manual_seed(w.seed + 1000)
     do = torch.randn(q.shape, generator=g, device=dev).to(torch.bfloat16)
-    lists = bsa.radial_block_lists(w.frames, w.tokens_per_frame, w.block, device=dev)
+    lists = bsa.radial_block_lists(w.frames, w.tokens_per_frame, w.block, device=dev,
+                                  text_tokens=w.text_tokens)
     rp_h, ci_h = lists.row_ptr.cpu().numpy(), lists.col_idx.cpu().numpy()
     fwd_flops = bsa.computed_flops(rp_h, ci_h, w.n, w.block, w.head_dim, w.batch, w.heads, 1)
     flops, exec_flops = 2.5 * fwd_flops, 3.5 * fwd_flops
@@ -596,7 +600,8 @@ def run_ours_module(args, world, rank, local):
     w = WORKLOADS[args.workload]
     H, D, n = w.heads, w.head_dim, w.n
     x, wqkv, bqkv, wo, bo = make_module_inputs(w.batch, n, H, D, w.seed, device=dev)
-    lists = bsa.radial_block_lists(w.frames, w.tokens_per_frame, w.block, device=dev)
+    lists = bsa.radial_block_lists(w.frames, w.tokens_per_frame, w.block, device=dev,
+                                  text_tokens=w.text_tokens)
     rp_h, ci_h = lists.row_ptr.cpu().numpy(), lists.col_idx.cpu().numpy()
     att_flops = bsa.computed_flops(rp_h, ci_h, n, w.block, D, w.batch, H, 1)
     flops = bsa.module_flops(w.batch, n, H, D, att_flops)
@@ -741,7 +746,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", default="wan", choices=("wan", "hunyuan", "long4x", "tiny"))
+    ap.add_argument("--workload", default="wan", choices=("wan", "hunyuan", "long4x", "tiny", "hunyuan_text"))
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--pass", dest="which", choices=("fwd", "bwd", "module"), default="fwd",

@@ -28,7 +28,7 @@ __all__ = [
     "bsa_get_timeout_detail", "bsa_status_string", "bsa_last_cuda_error", "bsa_set_test_hooks",
     "radial_block_lists", "block_lists_from_csr", "attention", "dense_masked_reference",
     "computed_flops", "bsa_attn_fwd_noalloc", "bsa_selftest_exp2", "NOALLOC_MAX_ORDER_ENTRIES",
-    "bsa_attn_fwd_strided", "bsa_attn_module_workspace_bytes", "bsa_attn_module_fwd",
+    "bsa_attn_fwd_strided", "bsa_attn_module_workspace_bytes", "bsa_joint_mask_build", "bsa_attn_module_fwd",
     "attention_module", "module_flops", "bsa_attn_bwd", "bsa_attn_bwd_workspace_bytes",
     "attention_backward",
 ]
@@ -99,6 +99,21 @@ def bsa_radial_mask_build(frames: int, tokens_per_frame: int, block: int, row_pt
                                    col_capacity if col_idx is not None else 0,
                                    ctypes.byref(nnz) if want_nnz else None, _stream(stream))
     _check(st, "bsa_radial_mask_build")
+    return int(nnz.value) if want_nnz else None
+
+
+def bsa_joint_mask_build(frames: int, tokens_per_frame: int, text_tokens: int, block: int,
+                         row_ptr: torch.Tensor, col_idx: torch.Tensor | None = None,
+                         col_capacity: int = 0, want_nnz: bool = True,
+                         stream=None) -> int | None:
+    """Joint text + video block lists (text tokens after the video tokens, attended
+    globally) into caller-owned int32 device tensors; returns nnz when asked."""
+    lib = _lib.load()
+    nnz = ctypes.c_int64(-1)
+    st = lib.bsa_joint_mask_build(frames, tokens_per_frame, text_tokens, block, _ptr(row_ptr),
+                                  _ptr(col_idx), col_capacity if col_idx is not None else 0,
+                                  ctypes.byref(nnz) if want_nnz else None, _stream(stream))
+    _check(st, "bsa_joint_mask_build")
     return int(nnz.value) if want_nnz else None
 
 
@@ -265,16 +280,19 @@ def bsa_set_test_hooks(wait_limit_ns: int = 0, fault_flags: int = 0) -> None:
 # ------------------------------------------------------------- conveniences
 
 def radial_block_lists(frames: int, tokens_per_frame: int, block: int = 128,
-                       device=None, stream=None) -> BlockLists:
-    """Build the radial lists on the GPU (two calls: count, then fill)."""
+                       device=None, stream=None, text_tokens: int = 0) -> BlockLists:
+    """Build the radial lists on the GPU (two calls: count, then fill). With
+    ``text_tokens`` > 0, the joint lists of the video tokens followed by that
+    many text tokens (:func:`bsa_joint_mask_build`)."""
     device = torch.device("cuda") if device is None else torch.device(device)
-    n = frames * tokens_per_frame
+    n = frames * tokens_per_frame + text_tokens
     nqb = -(-n // block)
     row_ptr = torch.empty(nqb + 1, dtype=torch.int32, device=device)
-    nnz = bsa_radial_mask_build(frames, tokens_per_frame, block, row_ptr, stream=stream)
+    nnz = bsa_joint_mask_build(frames, tokens_per_frame, text_tokens, block, row_ptr,
+                               stream=stream)
     col_idx = torch.empty(max(nnz, 1), dtype=torch.int32, device=device)
-    got = bsa_radial_mask_build(frames, tokens_per_frame, block, row_ptr, col_idx, col_idx.numel(),
-                                stream=stream)
+    got = bsa_joint_mask_build(frames, tokens_per_frame, text_tokens, block, row_ptr, col_idx,
+                               col_idx.numel(), stream=stream)
     assert got == nnz
     return BlockLists(row_ptr, col_idx[:nnz], 1, nqb, block)
 

@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(_HERE, "libbsa.so")
 # Names exported by the library; kept in the same order as include/bsa.h.
 EXPORTS = (
     "bsa_radial_mask_build",
+    "bsa_joint_mask_build",
     "bsa_attn_fwd_workspace_bytes",
     "bsa_attn_fwd",
     "bsa_attn_fwd_strided",
@@ -88,6 +89,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     yp = ctypes.POINTER(LayoutC)
     sig = {
         "bsa_radial_mask_build": (ctypes.c_int, [i32, i32, i32, vp, vp, i64, ctypes.POINTER(i64), vp]),
+        "bsa_joint_mask_build": (ctypes.c_int, [i32, i32, i32, i32, vp, vp, i64,
+                                                ctypes.POINTER(i64), vp]),
         "bsa_attn_fwd_workspace_bytes": (sz, [i32, i32, lp]),
         "bsa_attn_fwd": (ctypes.c_int, [vp, vp, vp, i32, i32, i32, i32, ctypes.c_float, lp,
                                         vp, vp, vp, sz, vp]),

@@ -545,13 +545,15 @@ using namespace bsa;
 
 extern "C" {
 
-int bsa_radial_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t block,
-                          int32_t *row_ptr, int32_t *col_idx, int64_t col_capacity,
-                          int64_t *nnz_out, bsa_stream_t stream_) {
+int bsa_joint_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t text_tokens,
+                         int32_t block, int32_t *row_ptr, int32_t *col_idx,
+                         int64_t col_capacity, int64_t *nnz_out, bsa_stream_t stream_) {
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  if (frames < 1 || tokens_per_frame < 1 || !row_ptr) return BSA_ERR_INVALID_ARG;
+  if (frames < 1 || tokens_per_frame < 1 || text_tokens < 0 || !row_ptr)
+    return BSA_ERR_INVALID_ARG;
   if (block != 64 && block != 128) return BSA_ERR_UNSUPPORTED;
-  const long long n = static_cast<long long>(frames) * tokens_per_frame;
+  const long long nv = static_cast<long long>(frames) * tokens_per_frame;
+  const long long n = nv + text_tokens;
   if (n > 0x7fffffffLL) return BSA_ERR_INVALID_ARG;
   const int nb = ceil_div(n, block);
   if (nb > 262144) return BSA_ERR_UNSUPPORTED;
@@ -560,6 +562,7 @@ int bsa_radial_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t bloc
   g.frames = frames;
   g.tpf = tokens_per_frame;
   g.block = block;
+  g.nv = static_cast<int>(nv);
   g.n = static_cast<int>(n);
   g.nb = nb;
   int rs = 0;
@@ -583,6 +586,13 @@ int bsa_radial_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t bloc
     BSA_CUDA(cudaGetLastError());
   }
   return BSA_OK;
+}
+
+int bsa_radial_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t block,
+                          int32_t *row_ptr, int32_t *col_idx, int64_t col_capacity,
+                          int64_t *nnz_out, bsa_stream_t stream_) {
+  return bsa_joint_mask_build(frames, tokens_per_frame, 0, block, row_ptr, col_idx, col_capacity,
+                              nnz_out, stream_);
 }
 
 size_t bsa_attn_fwd_workspace_bytes(int32_t batch, int32_t heads, const bsa_block_lists *l) {

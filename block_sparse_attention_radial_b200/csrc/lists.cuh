@@ -43,8 +43,9 @@ __device__ T cta_inclusive_scan(T x, T *scratch, T &total) {
 
 // ------------------------------------------------------------ radial mask --
 
+// n = nv + text: the frames * tpf video tokens, then `text` text tokens.
 struct RadialGeom {
-  int32_t frames, tpf, block, n, nb, rstar;
+  int32_t frames, tpf, block, n, nb, rstar, nv;
 };
 
 __device__ __forceinline__ int band_of(int d) { return 31 - __clz(d < 1 ? 1 : d); }
@@ -57,9 +58,19 @@ __device__ __forceinline__ int band_of(int d) { return 31 - __clz(d < 1 ? 1 : d)
 // most one per step, so the union over the query block's positions
 // [s_lo, s_hi] in that frame is the single interval [st(s_lo), st(s_hi) + w).
 // Its key blocks are marked; the threads of the CTA share the (f_i, f_j) pairs.
+//
+// Text tokens (after the video tokens) are global: a query block holding a
+// text token lists every key block, and every query block lists the key
+// blocks that hold text tokens.
 __device__ void radial_mark_row(const RadialGeom g, int qb, uint32_t *bits) {
   const int t0 = qb * g.block;
   const int t1 = min(g.n, t0 + g.block);  // query tokens [t0, t1)
+  if (t1 > g.nv) {
+    for (int b = threadIdx.x; b < g.nb; b += blockDim.x) atomicOr(&bits[b >> 5], 1u << (b & 31));
+    return;
+  }
+  for (int b = g.nv / g.block + threadIdx.x; g.nv < g.n && b < g.nb; b += blockDim.x)
+    atomicOr(&bits[b >> 5], 1u << (b & 31));
   const int fa = t0 / g.tpf, fb = (t1 - 1) / g.tpf;
   const int pairs = (fb - fa + 1) * g.frames;
   for (int p = threadIdx.x; p < pairs; p += blockDim.x) {

@@ -110,6 +110,25 @@ int bsa_radial_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t bloc
                           int64_t *nnz_out, bsa_stream_t stream);
 
 /*
+ * bsa_radial_mask_build for a joint sequence of video and text tokens: the
+ * frames * tokens_per_frame video tokens (frame-major) followed by
+ * text_tokens text tokens, n = frames * tokens_per_frame + text_tokens.
+ * The pages describe video tokens only; the reading taken for the text that
+ * video DiTs attend jointly with the video: the radial rule applies between
+ * video tokens; a text query attends to every token and every query attends
+ * to every text key. Blocks are cut over the whole sequence from token 0, so
+ * a block may hold both the last video and the first text tokens; a query
+ * block holding any text token lists every key block, and every row lists
+ * the key blocks from (frames * tokens_per_frame) / block on.
+ * text_tokens = 0 gives bsa_radial_mask_build's lists. Other arguments,
+ * limits, synchronisation and errors as bsa_radial_mask_build
+ * (text_tokens < 0 is BSA_ERR_INVALID_ARG).
+ */
+int bsa_joint_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t text_tokens,
+                         int32_t block, int32_t *row_ptr, int32_t *col_idx,
+                         int64_t col_capacity, int64_t *nnz_out, bsa_stream_t stream);
+
+/*
  * Bytes of device scratch memory bsa_attn_fwd needs for this problem (the
  * longest-row-first work order of every list). Returns 0 for invalid lists.
  */

@@ -92,6 +92,10 @@ def test_mask_build_argument_checks(lib):
     assert lib.bsa_radial_mask_build(4, 256, 64, vp(0), None, 0, None, None) == 1
     assert lib.bsa_radial_mask_build(4, 256, 32, vp(1 << 20), None, 0, None, None) == 2
     assert lib.bsa_radial_mask_build(1 << 16, 1 << 16, 128, vp(1 << 20), None, 0, None, None) == 1
+    assert lib.bsa_joint_mask_build(4, 256, -1, 64, vp(1 << 20), None, 0, None, None) == 1
+    assert lib.bsa_joint_mask_build(4, 256, 77, 32, vp(1 << 20), None, 0, None, None) == 2
+    assert lib.bsa_joint_mask_build(1 << 15, 1 << 16, 1 << 30, 128, vp(1 << 20), None, 0, None,
+                                    None) == 1
     assert lib.bsa_set_test_hooks(-1, 0) == 1
     assert lib.bsa_set_test_hooks(0, 0) == 0
 

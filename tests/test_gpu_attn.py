@@ -128,7 +128,8 @@ def _check_large(bsa, name):
     w = WORKLOADS[name]
     q, k, v = make_qkv(w, "cuda")
     if w.radial:
-        lists = bsa.radial_block_lists(w.frames, w.tokens_per_frame, w.block)
+        lists = bsa.radial_block_lists(w.frames, w.tokens_per_frame, w.block,
+                                       text_tokens=w.text_tokens)
         num_lists = 1
     else:
         rp, ci, _ = make_generic_lists(w.heads, w.nqb)
@@ -140,6 +141,9 @@ def _check_large(bsa, name):
     # sampled rows of three heads against the float64 oracle, for both kernels
     rp, ci = _host_lists(lists)
     rows = sample_rows(w.n, w.block, w.tokens_per_frame, 512, seed=w.seed)
+    if w.text_tokens:  # both sides of the video / text boundary (a mixed block)
+        nv = w.n - w.text_tokens
+        rows = np.unique(np.r_[rows, nv - 16, nv - 1, nv, nv + 1])
     heads = sorted({0, w.heads // 2, w.heads - 1})
     ref_o = np.zeros((1, len(heads), rows.size, w.head_dim))
     ref_l = np.zeros((1, len(heads), rows.size))
@@ -156,7 +160,7 @@ def _check_large(bsa, name):
     assert_close(sel(ro), ref_o, sel(rl), ref_l, f"{name}: fp32 reference vs oracle (sampled)")
 
 
-@pytest.mark.parametrize("name", ["wan", "hunyuan", "long4x", "generic"])
+@pytest.mark.parametrize("name", ["wan", "hunyuan", "long4x", "generic", "hunyuan_text"])
 def test_full_size_configs(bsa, name):
     _check_large(bsa, name)
 

@@ -69,3 +69,17 @@ def test_capacity_too_small(bsa):
     assert bsa.bsa_get_device_status() == 6
     assert bsa.bsa_get_device_status() == 0
     assert np.array_equal(col_idx.cpu().numpy(), ci[:col_idx.numel()])
+
+
+JOINT = [(4, 64, 16, 64), (3, 40, 21, 64), (5, 48, 7, 128), (2, 100, 130, 64), (6, 33, 1, 64),
+         (4, 256, 77, 64), (33, 3600, 256, 128), (21, 1560, 512, 128), (8, 256, 0, 64)]
+
+
+@pytest.mark.parametrize("F,S,T,B", JOINT)
+def test_joint_text_video_lists_bit_exact(bsa, F, S, T, B):
+    lists = bsa.radial_block_lists(F, S, B, device="cuda:0", text_tokens=T)
+    rp, ci = oracle.joint_block_lists(F, S, T, B)
+    assert np.array_equal(lists.row_ptr.cpu().numpy(), rp)
+    assert np.array_equal(lists.col_idx.cpu().numpy(), ci)
+    assert bsa.bsa_get_device_status() == 0
+    assert bsa.bsa_validate_lists(lists) == 0

@@ -19,6 +19,9 @@ The shapes stand in for the video-DiT workloads the pages measure on
                seed 4, one seeded tile pattern per head (diagonal,
                multi-diagonal, vertical stripes + diagonal, or a dual window),
                density 10-40 %.
+* ``hunyuan_text``  the hunyuan grid followed by 256 joint text tokens
+               (n=119056; HunyuanVideo-style joint text + video attention),
+               same value recipe, seed 5.
 """
 
 from __future__ import annotations
@@ -43,6 +46,7 @@ class Workload:
     frames: int = 0            # radial workloads only
     tokens_per_frame: int = 0  # radial workloads only
     radial: bool = True
+    text_tokens: int = 0       # joint text tokens appended after the video tokens
 
     @property
     def nqb(self) -> int:
@@ -55,6 +59,8 @@ WORKLOADS = {
     "hunyuan": Workload("hunyuan", 1, 24, 128, 33 * 3600, 128, 2, "normal_token_scale", 33, 3600),
     "long4x": Workload("long4x", 1, 40, 128, 84 * 1560, 128, 3, "normal", 84, 1560),
     "generic": Workload("generic", 1, 24, 128, 32768, 128, 4, "normal_scaled", radial=False),
+    "hunyuan_text": Workload("hunyuan_text", 1, 24, 128, 33 * 3600 + 256, 128, 5,
+                             "normal_token_scale", 33, 3600, text_tokens=256),
 }
 
 
