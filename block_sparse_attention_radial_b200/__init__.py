@@ -28,7 +28,8 @@ __all__ = [
     "bsa_get_timeout_detail", "bsa_status_string", "bsa_last_cuda_error", "bsa_set_test_hooks",
     "radial_block_lists", "block_lists_from_csr", "attention", "dense_masked_reference",
     "computed_flops", "bsa_attn_fwd_noalloc", "bsa_selftest_exp2", "NOALLOC_MAX_ORDER_ENTRIES",
-    "bsa_attn_fwd_strided", "bsa_attn_module_workspace_bytes", "bsa_joint_mask_build", "bsa_attn_module_fwd",
+    "bsa_attn_fwd_strided", "bsa_attn_module_workspace_bytes", "bsa_joint_mask_build",
+    "bsa_attn_fwd_host", "bsa_attn_fwd_host_workspace_bytes", "bsa_attn_module_fwd",
     "attention_module", "module_flops", "bsa_attn_bwd", "bsa_attn_bwd_workspace_bytes",
     "attention_backward",
 ]
@@ -160,6 +161,34 @@ def bsa_attn_fwd_strided(q, k, v, lists: BlockLists, out, lse=None, workspace=No
                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
                                   _stream(stream))
     _check(st, "bsa_attn_fwd_strided")
+
+
+def bsa_attn_fwd_host_workspace_bytes(batch: int, heads: int, n: int, head_dim: int,
+                                      lists: BlockLists) -> int:
+    return int(_lib.load().bsa_attn_fwd_host_workspace_bytes(batch, heads, n, head_dim,
+                                                             ctypes.byref(lists.c_struct())))
+
+
+def bsa_attn_fwd_host(q, k, v, lists: BlockLists, out, lse=None, workspace=None,
+                      softmax_scale: float = 0.0, stream=None, device=None) -> None:
+    """bsa_attn_fwd on CPU tensors (pin them for copy/compute overlap): q, k, v
+    and out bf16 [B, H, n, D] in host memory, lse float [B, H, n] or None. The
+    copies and kernels are enqueued on ``stream``; synchronise it before
+    reading ``out``."""
+    B, H, n, D = q.shape
+    for t in (q, k, v, out, lse):
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError("bsa_attn_fwd_host takes contiguous host tensors")
+    lib = _lib.load()
+    ls = lists.c_struct()
+    if workspace is None:
+        dev = lists.row_ptr.device if device is None else torch.device(device)
+        workspace = torch.empty(lib.bsa_attn_fwd_host_workspace_bytes(B, H, n, D, ctypes.byref(ls)),
+                                dtype=torch.uint8, device=dev)
+    st = lib.bsa_attn_fwd_host(_ptr(q), _ptr(k), _ptr(v), B, H, n, D, float(softmax_scale),
+                               ctypes.byref(ls), _ptr(out), _ptr(lse), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "bsa_attn_fwd_host")
 
 
 def bsa_attn_module_workspace_bytes(batch: int, n: int, heads: int, head_dim: int,

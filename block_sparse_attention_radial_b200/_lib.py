@@ -20,6 +20,8 @@ EXPORTS = (
     "bsa_attn_fwd_workspace_bytes",
     "bsa_attn_fwd",
     "bsa_attn_fwd_strided",
+    "bsa_attn_fwd_host_workspace_bytes",
+    "bsa_attn_fwd_host",
     "bsa_attn_module_workspace_bytes",
     "bsa_attn_module_fwd",
     "bsa_attn_dense_masked_ref",
@@ -97,6 +99,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bsa_attn_fwd_strided": (ctypes.c_int, [vp, yp, vp, yp, vp, yp, i32, i32, i32, i32,
                                                 ctypes.c_float, lp, vp, yp, vp, vp, sz, vp]),
         "bsa_attn_module_workspace_bytes": (sz, [i32, i32, i32, i32, lp]),
+        "bsa_attn_fwd_host_workspace_bytes": (sz, [i32, i32, i32, i32, lp]),
+        "bsa_attn_fwd_host": (ctypes.c_int, [vp, vp, vp, i32, i32, i32, i32, ctypes.c_float, lp,
+                                             vp, vp, vp, sz, vp]),
         "bsa_attn_module_fwd": (ctypes.c_int, [vp, vp, vp, vp, vp, i32, i32, i32, i32,
                                                ctypes.c_float, lp, vp, vp, sz, vp]),
         "bsa_attn_dense_masked_ref": (ctypes.c_int, [vp, vp, vp, i32, i32, i32, i32, ctypes.c_float,

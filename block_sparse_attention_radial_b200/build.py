@@ -12,7 +12,8 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = [os.path.join(HERE, "csrc", "libbsa.cu"), os.path.join(HERE, "csrc", "module.cu")]
+SOURCES = [os.path.join(HERE, "csrc", name)
+           for name in ("libbsa.cu", "module.cu", "host_pipeline.cu")]
 OUTPUT = os.path.join(HERE, "libbsa.so")
 GENCODE = "arch=compute_100a,code=sm_100a"
 

@@ -1,0 +1,171 @@
+// libbsa: the forward pass on host buffers (bsa_attn_fwd_host).
+//
+// q, k, v live in host memory and the results go back to host memory. The
+// problem is cut into groups of heads; each group's q, k, v are copied in on
+// one stream, its attention runs on the caller's stream as soon as its inputs
+// have landed, and its out / lse are copied back on a third stream as soon as
+// it is done. With pinned host memory the copy engines (one per direction)
+// and the SMs work at the same time, so a call takes about the longest of
+// the three (usually the host-to-device copy over PCIe) instead of their sum.
+//
+// Uses only the public entry points (bsa_attn_fwd) and the CUDA runtime; the
+// device staging buffers are the caller's workspace.
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "bsa.h"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kTargetGroups = 8;
+
+// Per-device copy streams and events. An event is waited on right after each
+// record, and a wait binds to the record that precedes it, so one event per
+// kind serves every group.
+struct PipeState {
+  bool ready = false;
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t entry = nullptr, landed = nullptr, computed = nullptr, done = nullptr;
+};
+std::mutex g_pipe_mu;  // one caller at a time enqueues on the shared streams
+PipeState g_pipe[kMaxDevices];
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Staging layout inside the workspace: the attention's own scratch, then q,
+// k, v, out and lse for the whole problem.
+struct HostLayout {
+  size_t attn_ws, q, k, v, out, lse, total;
+};
+
+HostLayout host_layout(int32_t batch, int32_t heads, int32_t n, int32_t head_dim,
+                       const bsa_block_lists *l) {
+  HostLayout w;
+  const size_t t = static_cast<size_t>(batch) * heads * n * head_dim * 2;
+  w.attn_ws = align256(bsa_attn_fwd_workspace_bytes(batch, heads, l));
+  w.q = w.attn_ws;
+  w.k = w.q + align256(t);
+  w.v = w.k + align256(t);
+  w.out = w.v + align256(t);
+  w.lse = w.out + align256(t);
+  w.total = w.lse + align256(static_cast<size_t>(batch) * heads * n * sizeof(float));
+  return w;
+}
+
+int pipe_state(PipeState **st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSA_ERR_CUDA;
+  PipeState &s = g_pipe[dev];
+  if (!s.ready) {
+    const unsigned fl = cudaEventDisableTiming;
+    if (cudaStreamCreateWithFlags(&s.in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&s.out, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&s.entry, fl) != cudaSuccess ||
+        cudaEventCreateWithFlags(&s.landed, fl) != cudaSuccess ||
+        cudaEventCreateWithFlags(&s.computed, fl) != cudaSuccess ||
+        cudaEventCreateWithFlags(&s.done, fl) != cudaSuccess)
+      return BSA_ERR_CUDA;
+    s.ready = true;
+  }
+  *st = &s;
+  return BSA_OK;
+}
+
+#define PIPE_CUDA(call)                          \
+  do {                                           \
+    if ((call) != cudaSuccess) return BSA_ERR_CUDA; \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+size_t bsa_attn_fwd_host_workspace_bytes(int32_t batch, int32_t heads, int32_t n,
+                                         int32_t head_dim, const bsa_block_lists *l) {
+  if (!l || batch < 1 || heads < 1 || n < 1 || head_dim < 1) return 0;
+  if (bsa_attn_fwd_workspace_bytes(batch, heads, l) == 0) return 0;
+  return host_layout(batch, heads, n, head_dim, l).total;
+}
+
+int bsa_attn_fwd_host(const void *q_host, const void *k_host, const void *v_host,
+                      int32_t batch, int32_t heads, int32_t n, int32_t head_dim,
+                      float softmax_scale, const bsa_block_lists *l, void *out_host,
+                      float *lse_host, void *workspace, size_t workspace_bytes,
+                      bsa_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!q_host || !k_host || !v_host || !out_host || !l || !workspace) return BSA_ERR_INVALID_ARG;
+  if (batch < 1 || heads < 1 || n < 1) return BSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
+  if (bsa_attn_fwd_workspace_bytes(batch, heads, l) == 0) return BSA_ERR_INVALID_ARG;
+  const HostLayout w = host_layout(batch, heads, n, head_dim, l);
+  if (workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return BSA_ERR_INVALID_ARG;
+
+  // Groups of whole heads inside one batch item (a group of per-head lists is
+  // then a contiguous run of lists), about kTargetGroups of them in all.
+  const long long bh = static_cast<long long>(batch) * heads;
+  long long gsl = (bh + kTargetGroups - 1) / kTargetGroups;
+  const int gs = static_cast<int>(gsl > heads ? heads : gsl);
+  const int groups_per_item = (heads + gs - 1) / gs;
+
+  std::lock_guard<std::mutex> lk(g_pipe_mu);
+  PipeState *ps = nullptr;
+  int st = pipe_state(&ps);
+  if (st != BSA_OK) return st;
+
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const size_t row = static_cast<size_t>(n) * head_dim * 2;  // bytes of one (b, h) slice
+  const size_t lrow = static_cast<size_t>(n) * sizeof(float);
+  const int nqb = l->num_q_blocks;
+
+  // everything already on the caller's stream (e.g. the lists) comes first
+  PIPE_CUDA(cudaEventRecord(ps->entry, stream));
+  PIPE_CUDA(cudaStreamWaitEvent(ps->in, ps->entry, 0));
+  PIPE_CUDA(cudaStreamWaitEvent(ps->out, ps->entry, 0));
+
+  for (int b = 0; b < batch; ++b) {
+    for (int gi = 0; gi < groups_per_item; ++gi) {
+      const int h0 = gi * gs;
+      const int hn = heads - h0 < gs ? heads - h0 : gs;
+      const size_t off = (static_cast<size_t>(b) * heads + h0) * row;
+      const size_t bytes = static_cast<size_t>(hn) * row;
+      PIPE_CUDA(cudaMemcpyAsync(ws + w.q + off, static_cast<const uint8_t *>(q_host) + off, bytes,
+                                cudaMemcpyHostToDevice, ps->in));
+      PIPE_CUDA(cudaMemcpyAsync(ws + w.k + off, static_cast<const uint8_t *>(k_host) + off, bytes,
+                                cudaMemcpyHostToDevice, ps->in));
+      PIPE_CUDA(cudaMemcpyAsync(ws + w.v + off, static_cast<const uint8_t *>(v_host) + off, bytes,
+                                cudaMemcpyHostToDevice, ps->in));
+      PIPE_CUDA(cudaEventRecord(ps->landed, ps->in));
+      PIPE_CUDA(cudaStreamWaitEvent(stream, ps->landed, 0));
+
+      bsa_block_lists sub = *l;
+      if (l->num_lists > 1) {  // this group's heads use lists h0 .. h0 + hn - 1
+        sub.num_lists = hn;
+        sub.row_ptr = l->row_ptr + static_cast<size_t>(h0) * nqb;
+      }
+      const size_t loff = (static_cast<size_t>(b) * heads + h0) * lrow;
+      st = bsa_attn_fwd(ws + w.q + off, ws + w.k + off, ws + w.v + off, 1, hn, n, head_dim,
+                        softmax_scale, &sub, ws + w.out + off,
+                        reinterpret_cast<float *>(ws + w.lse + loff), ws, w.attn_ws, stream_);
+      if (st != BSA_OK) return st;
+      PIPE_CUDA(cudaEventRecord(ps->computed, stream));
+      PIPE_CUDA(cudaStreamWaitEvent(ps->out, ps->computed, 0));
+      PIPE_CUDA(cudaMemcpyAsync(static_cast<uint8_t *>(out_host) + off, ws + w.out + off, bytes,
+                                cudaMemcpyDeviceToHost, ps->out));
+      if (lse_host)
+        PIPE_CUDA(cudaMemcpyAsync(reinterpret_cast<uint8_t *>(lse_host) + loff, ws + w.lse + loff,
+                                  static_cast<size_t>(hn) * lrow, cudaMemcpyDeviceToHost, ps->out));
+    }
+  }
+  // the caller's stream orders after the last copy back
+  PIPE_CUDA(cudaEventRecord(ps->done, ps->out));
+  PIPE_CUDA(cudaStreamWaitEvent(stream, ps->done, 0));
+  return BSA_OK;
+}
+
+}  // extern "C"

@@ -161,6 +161,42 @@ int bsa_attn_fwd(const void *q, const void *k, const void *v,
                  bsa_stream_t stream);
 
 /*
+ * Bytes of device workspace bsa_attn_fwd_host needs: device copies of q, k,
+ * v, out and lse plus bsa_attn_fwd's own scratch. Returns 0 for invalid
+ * arguments.
+ */
+size_t bsa_attn_fwd_host_workspace_bytes(int32_t batch, int32_t heads, int32_t n,
+                                         int32_t head_dim, const bsa_block_lists *lists);
+
+/*
+ * bsa_attn_fwd on HOST buffers: q_host, k_host, v_host (bf16 [batch, heads,
+ * n, head_dim], contiguous) are copied to the device, the attention runs, and
+ * out_host (same layout) and lse_host (float [batch, heads, n], or NULL) are
+ * copied back. The problem is cut into about eight groups of whole heads
+ * (never across batch items); group g's inputs are copied in on an internal
+ * stream while group g-1 computes on `stream` and group g-2's results are
+ * copied out on a second internal stream, so with pinned (page-locked) host
+ * memory the copies in both directions overlap the kernels; pageable memory
+ * works but serialises.
+ * lists        device lists as for bsa_attn_fwd (already built, or built
+ *              earlier on `stream`: the call orders after the work already
+ *              enqueued on `stream`).
+ * workspace    device memory of bsa_attn_fwd_host_workspace_bytes(),
+ *              256-byte aligned; holds the device copies.
+ * Asynchronous: the host buffers must stay valid, and out_host / lse_host
+ * must not be read, until `stream` has been synchronised (work enqueued on
+ * `stream` afterwards also orders after the last copy back). Calls are
+ * serialised on the internal streams (one staging area per call). Errors as
+ * bsa_attn_fwd; an error from a group's launch is returned after the groups
+ * before it were enqueued (their results are then incomplete).
+ */
+int bsa_attn_fwd_host(const void *q_host, const void *k_host, const void *v_host,
+                      int32_t batch, int32_t heads, int32_t n, int32_t head_dim,
+                      float softmax_scale, const bsa_block_lists *lists, void *out_host,
+                      float *lse_host, void *workspace, size_t workspace_bytes,
+                      bsa_stream_t stream);
+
+/*
  * Strides of a [batch, heads, n, head_dim] bf16 tensor view, in elements; the
  * head_dim axis is contiguous. The contiguous layout of bsa_attn_fwd is
  * {heads*n*head_dim, n*head_dim, head_dim}. The token-major output of a fused
