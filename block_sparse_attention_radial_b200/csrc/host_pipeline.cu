@@ -107,11 +107,12 @@ int bsa_attn_fwd_host(const void *q_host, const void *k_host, const void *v_host
     return BSA_ERR_INVALID_ARG;
 
   // Groups of whole heads inside one batch item (a group of per-head lists is
-  // then a contiguous run of lists), about kTargetGroups of them in all.
+  // then a contiguous run of lists), about kTargetGroups of them in all. The
+  // first and the last group hold one head: the first group's copy is the
+  // only one no kernel overlaps, and the last group's kernel and copy back
+  // are the only ones no copy in overlaps.
   const long long bh = static_cast<long long>(batch) * heads;
-  long long gsl = (bh + kTargetGroups - 1) / kTargetGroups;
-  const int gs = static_cast<int>(gsl > heads ? heads : gsl);
-  const int groups_per_item = (heads + gs - 1) / gs;
+  const long long mid = bh > 2 ? (bh - 2 + kTargetGroups - 3) / (kTargetGroups - 2) : 1;
 
   std::lock_guard<std::mutex> lk(g_pipe_mu);
   PipeState *ps = nullptr;
@@ -128,10 +129,15 @@ int bsa_attn_fwd_host(const void *q_host, const void *k_host, const void *v_host
   PIPE_CUDA(cudaStreamWaitEvent(ps->in, ps->entry, 0));
   PIPE_CUDA(cudaStreamWaitEvent(ps->out, ps->entry, 0));
 
-  for (int b = 0; b < batch; ++b) {
-    for (int gi = 0; gi < groups_per_item; ++gi) {
-      const int h0 = gi * gs;
-      const int hn = heads - h0 < gs ? heads - h0 : gs;
+  for (long long idx = 0; idx < bh;) {
+    {
+      const int b = static_cast<int>(idx / heads), h0 = static_cast<int>(idx % heads);
+      long long size = (idx == 0 || idx == bh - 1) ? 1 : mid;
+      if (size > heads - h0) size = heads - h0;             // stay inside the batch item
+      if (idx > 0 && idx + size > bh - 1) size = bh - 1 - idx;  // keep the last head apart
+      if (size < 1) size = 1;
+      const int hn = static_cast<int>(size);
+      idx += size;
       const size_t off = (static_cast<size_t>(b) * heads + h0) * row;
       const size_t bytes = static_cast<size_t>(hn) * row;
       PIPE_CUDA(cudaMemcpyAsync(ws + w.q + off, static_cast<const uint8_t *>(q_host) + off, bytes,
