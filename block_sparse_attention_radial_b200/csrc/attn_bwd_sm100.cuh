@@ -45,6 +45,12 @@ struct BwdParams {
   const float *lse2;                 // [bh][nqb * 128]: lse * log2(e), +inf padding
   const float *delta;                // [bh][nqb * 128]: sum_d dO * O, 0 padding
   __nv_bfloat16 *dq, *dk, *dv;
+  // Block-64 lists run as 128-row tiles: a 4-bit mask per list entry, bit
+  // qi * 2 + kj set when 64-row query block qi of the tile lists 64-key block
+  // kj of the key tile (rmask per CSR entry, cmask per transposed entry).
+  // Both null for block-128 lists (every pair of the tile is listed); read
+  // only by the MASKED instances of the kernels.
+  const uint8_t *rmask, *cmask;
   int32_t heads, n, nqb, nkb, num_lists, nnz;
   int32_t total_items;
   float scale, scale_log2;
@@ -93,16 +99,20 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16 *out, const __nv_bfloat16 *d
 
 // ------------------------------------------------------- transposed lists --
 
-// True when the sorted row [a, b) of col_idx holds kb.
-__device__ __forceinline__ bool row_has(const int32_t *col_idx, int a, int b, int kb) {
+// Position of kb in the sorted row [a, b) of col_idx, or -1.
+__device__ __forceinline__ int row_find(const int32_t *col_idx, int a, int b, int kb) {
   while (a < b) {
     const int m = (a + b) >> 1;
     const int v = col_idx[m];
-    if (v == kb) return true;
+    if (v == kb) return m;
     if (v < kb) a = m + 1;
     else b = m;
   }
-  return false;
+  return -1;
+}
+
+__device__ __forceinline__ bool row_has(const int32_t *col_idx, int a, int b, int kb) {
+  return row_find(col_idx, a, b, kb) >= 0;
 }
 
 // One CTA per (list, key block): how many query blocks list it.
@@ -123,10 +133,12 @@ __global__ void csc_count_kernel(const int32_t *row_ptr, const int32_t *col_idx,
 }
 
 // One CTA per (list, key block): its query blocks in ascending order, at
-// col_ptr (the inclusive scan of the counts). Writes stay below `cap` (the
-// entries row_idx holds) even for lists the validator would reject.
+// col_ptr (the inclusive scan of the counts), and with rmask given each
+// entry's mask into cmask. Writes stay below `cap` (the entries row_idx
+// holds) even for lists the validator would reject.
 __global__ void csc_fill_kernel(const int32_t *row_ptr, const int32_t *col_idx, int nqb, int nkb,
-                                int nnz, const int32_t *col_ptr, int32_t *row_idx, int cap) {
+                                int nnz, const int32_t *col_ptr, int32_t *row_idx, int cap,
+                                const uint8_t *rmask, uint8_t *cmask) {
   __shared__ int scratch[32];
   const int list = blockIdx.x / nkb, kb = blockIdx.x - list * nkb;
   const int32_t *rp = row_ptr + static_cast<long long>(list) * nqb;
@@ -134,17 +146,86 @@ __global__ void csc_fill_kernel(const int32_t *row_ptr, const int32_t *col_idx, 
   const int end = col_ptr[blockIdx.x + 1];
   for (int q0 = 0; q0 < nqb; q0 += blockDim.x) {
     const int qb = q0 + threadIdx.x;
-    bool has = false;
+    int at = -1;
     if (qb < nqb) {
       const int a = min(max(rp[qb], 0), nnz), b = min(max(rp[qb + 1], 0), nnz);
-      has = row_has(col_idx, a, b, kb);
+      at = row_find(col_idx, a, b, kb);
     }
+    const bool has = at >= 0;
     int total;
     const int inc = cta_inclusive_scan(has ? 1 : 0, scratch, total);
     const int pos = base + inc - 1;
-    if (has && pos >= 0 && pos < end && pos < cap) row_idx[pos] = qb;
+    if (has && pos >= 0 && pos < end && pos < cap) {
+      row_idx[pos] = qb;
+      if (rmask) cmask[pos] = rmask[at];
+    }
     base += total;
   }
+}
+
+// ------------------------------------------------- block-64 lists as tiles --
+//
+// The backward kernels work on 128 x 128 tiles. Lists at block 64 become tile
+// lists: tile row t covers query blocks 2t and 2t+1, tile column u key blocks
+// 2u and 2u+1; entry (t, u) exists when any of its four pairs is listed and
+// carries the 4-bit mask of the listed pairs (bit qi * 2 + kj). One thread
+// per tile row merges the two sorted rows; counts first, then (after a scan
+// of the counts) the entries.
+__device__ int merge_tile_row(const int32_t *col_idx, int a0, int a1, int b0, int b1, int nkb,
+                              int32_t *cols, uint8_t *masks, long long cap) {
+  int cnt = 0;
+  while (a0 < a1 || b0 < b1) {
+    const int ka = a0 < a1 ? min(max(col_idx[a0], 0), nkb - 1) >> 1 : 0x7fffffff;
+    const int kb = b0 < b1 ? min(max(col_idx[b0], 0), nkb - 1) >> 1 : 0x7fffffff;
+    const int u = min(ka, kb);
+    uint32_t bits = 0;
+    while (a0 < a1 && (min(max(col_idx[a0], 0), nkb - 1) >> 1) == u) {
+      bits |= 1u << (min(max(col_idx[a0], 0), nkb - 1) & 1);
+      ++a0;
+    }
+    while (b0 < b1 && (min(max(col_idx[b0], 0), nkb - 1) >> 1) == u) {
+      bits |= 1u << (2 + (min(max(col_idx[b0], 0), nkb - 1) & 1));
+      ++b0;
+    }
+    if (cols && cnt < cap) {
+      cols[cnt] = u;
+      masks[cnt] = static_cast<uint8_t>(bits);
+    }
+    ++cnt;
+  }
+  return cnt;
+}
+
+// rows = num_lists * nt tile rows; nqb, nkb count 64-blocks.
+__global__ void tile_count_kernel(const int32_t *row_ptr, const int32_t *col_idx, int nqb, int nkb,
+                                  int nnz, int nt, int rows, int32_t *tile_ptr) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i == 0) tile_ptr[0] = 0;
+  if (i >= rows) return;
+  const int list = i / nt, t = i - list * nt;
+  const int32_t *rp = row_ptr + static_cast<long long>(list) * nqb;
+  const int q0 = 2 * t, q1 = 2 * t + 1;
+  const int a0 = min(max(rp[q0], 0), nnz), a1 = min(max(rp[q0 + 1], 0), nnz);
+  const int b0 = q1 < nqb ? min(max(rp[q1], 0), nnz) : 0;
+  const int b1 = q1 < nqb ? min(max(rp[q1 + 1], 0), nnz) : 0;
+  tile_ptr[i + 1] = merge_tile_row(col_idx, a0, max(a0, a1), b0, max(b0, b1), nkb, nullptr,
+                                   nullptr, 0);
+}
+
+__global__ void tile_fill_kernel(const int32_t *row_ptr, const int32_t *col_idx, int nqb, int nkb,
+                                 int nnz, int nt, int rows, const int32_t *tile_ptr,
+                                 int32_t *tile_col, uint8_t *tile_mask, long long cap) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= rows) return;
+  const int list = i / nt, t = i - list * nt;
+  const int32_t *rp = row_ptr + static_cast<long long>(list) * nqb;
+  const int q0 = 2 * t, q1 = 2 * t + 1;
+  const int a0 = min(max(rp[q0], 0), nnz), a1 = min(max(rp[q0 + 1], 0), nnz);
+  const int b0 = q1 < nqb ? min(max(rp[q1], 0), nnz) : 0;
+  const int b1 = q1 < nqb ? min(max(rp[q1 + 1], 0), nnz) : 0;
+  const long long at = tile_ptr[i];
+  merge_tile_row(col_idx, a0, max(a0, a1), b0, max(b0, b1), nkb, tile_col + at, tile_mask + at,
+                 cap - at);
 }
 
 // tcgen05.st of 16 columns (32x32b shape: thread t writes TMEM lane t).
@@ -197,7 +278,7 @@ struct BwdItem {
 //                                           P^T and dS^T as bf16 over them)
 //   dV += P^T dO_e, dK += dS^T Q_e         (issued before the next S^T, so the
 //                                           TMEM they read is not overwritten)
-template <int D>
+template <int D, bool MASKED>
 __global__ void __launch_bounds__(192, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
@@ -460,6 +541,9 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
         const float *lse_s = reinterpret_cast<const float *>(sStage + s * C::STAGE + 2 * C::T);
         const float *del_s = lse_s + 128;
+        // listed (query half, key half) pairs of this tile pair; this thread's
+        // key half is warp / 2, chunk c's query half c / 2
+        const uint32_t bits = MASKED ? __ldg(p.cmask + it.a + e) : 0xFu;
         // P^T (fp32, kept for dS^T), handed over as bf16 in four parts while
         // dP^T is still being computed
         float pf[BN];
@@ -469,13 +553,16 @@ __global__ void __launch_bounds__(192, 1)
           tmem_ld32(lane_tmem + C::ST_COL + c * 32, sr);
           tmem_wait_ld();
           reg_fence32(sr);
+          const bool on = !MASKED || ((bits >> ((c >> 1) * 2 + (warp >> 1))) & 1u);
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float4 l4 = *reinterpret_cast<const float4 *>(lse_s + c * 32 + (i & ~1) * 2);
             const float la = (i & 1) ? l4.z : l4.x, lb = (i & 1) ? l4.w : l4.y;
-            pf[c * 32 + 2 * i] = ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -la));
-            pf[c * 32 + 2 * i + 1] = ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -lb));
+            const float pa = ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -la));
+            const float pb = ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -lb));
+            pf[c * 32 + 2 * i] = on ? pa : 0.f;
+            pf[c * 32 + 2 * i + 1] = on ? pb : 0.f;
             pk[i] = pack_bf16x2(pf[c * 32 + 2 * i], pf[c * 32 + 2 * i + 1]);
           }
           // chunk c lands on columns [16c, 16c + 16): already read back
@@ -577,7 +664,7 @@ struct DqCfg {
 // block ahead so it runs during the previous elementwise step), dP = dO V_e^T,
 // the elementwise warps write dS (bf16) over dP, then dQ += dS K_e (issued
 // before the next dP, which overwrites the dS it reads).
-template <int D>
+template <int D, bool MASKED>
 __global__ void __launch_bounds__(192, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -821,6 +908,9 @@ __global__ void __launch_bounds__(192, 1)
         ++scount[sb];
         tc_fence_after();
         const int valid = e == it.len - 1 ? last_valid : BN;
+        // listed (query half, key half) pairs of this tile pair; this thread's
+        // query half is warp / 2, chunk c's key half c / 2
+        const uint32_t bits = MASKED ? __ldg(p.rmask + it.a + e) : 0xFu;
         // P from S (fp32, kept for dS) while dP is still being computed
         float pf[BN];
 #pragma unroll
@@ -829,10 +919,11 @@ __global__ void __launch_bounds__(192, 1)
           tmem_ld32(lane_tmem + C::s_col(e) + c * 32, sr);
           tmem_wait_ld();
           reg_fence32(sr);
+          const bool on = !MASKED || ((bits >> ((warp >> 1) * 2 + (c >> 1))) & 1u);
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float pv = ex2_approx(fmaf(__uint_as_float(sr[i]), sl2, -lse2));
-            pf[c * 32 + i] = (valid < BN && c * 32 + i >= valid) ? 0.f : pv;
+            pf[c * 32 + i] = (!on || (valid < BN && c * 32 + i >= valid)) ? 0.f : pv;
           }
         }
         if (!(ok = warp_wait(&bar_dp_full, dcount & 1u, wc, kBarSFull, dcount))) break;

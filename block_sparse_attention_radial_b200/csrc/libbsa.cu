@@ -423,36 +423,77 @@ QkvViews contiguous_views(const void *q, const void *k, const void *v, int batch
 // ---------------------------------------------------------------- backward
 
 // Workspace of the backward pass: lse2 and delta per padded query row, then
-// the transposed lists. Offsets are 256-byte aligned (the bulk copies of
-// lse2 / delta rows need 16-byte aligned 512-byte rows).
+// the transposed lists; for block-64 lists also the per-entry masks of the
+// transposed lists and the 128-row tile lists (pointers, entries, masks).
+// Offsets are 256-byte aligned (the bulk copies of lse2 / delta rows need
+// 16-byte aligned 512-byte rows).
 struct BwdLayout {
-  size_t lse2, delta, col_ptr, row_idx, total;
+  size_t lse2, delta, col_ptr, row_idx, cmask, tile_ptr, tile_col, tile_mask, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-BwdLayout bwd_layout(int32_t batch, int32_t heads, const bsa_block_lists *l) {
+BwdLayout bwd_layout(int32_t batch, int32_t heads, int32_t n, const bsa_block_lists *l) {
   BwdLayout w;
-  const size_t rows = static_cast<size_t>(batch) * heads * l->num_q_blocks * kBwdBlock;
+  const size_t nt = static_cast<size_t>(ceil_div(n, kBwdBlock));  // 128-row tiles
+  const size_t rows = static_cast<size_t>(batch) * heads * nt * kBwdBlock;
+  const size_t ptrs = (static_cast<size_t>(l->num_lists) * nt + 1) * sizeof(int32_t);
+  const size_t entries = static_cast<size_t>(l->nnz > 0 ? l->nnz : 1);
   w.lse2 = 0;
   w.delta = align256(rows * sizeof(float));
   w.col_ptr = w.delta + align256(rows * sizeof(float));
-  w.row_idx = w.col_ptr +
-              align256((static_cast<size_t>(l->num_lists) * l->num_k_blocks + 1) * sizeof(int32_t));
-  w.total = w.row_idx + align256(static_cast<size_t>(l->nnz > 0 ? l->nnz : 1) * sizeof(int32_t));
+  w.row_idx = w.col_ptr + align256(ptrs);
+  w.cmask = w.tile_ptr = w.tile_col = w.tile_mask = w.total =
+      w.row_idx + align256(entries * sizeof(int32_t));
+  if (l->block != kBwdBlock) {
+    w.tile_ptr = w.cmask + align256(entries);
+    w.tile_col = w.tile_ptr + align256(ptrs);
+    w.tile_mask = w.tile_col + align256(entries * sizeof(int32_t));
+    w.total = w.tile_mask + align256(entries);
+  }
   return w;
 }
 
 template <int D>
 int launch_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout,
                const float *lse, int32_t bh, int32_t n, float softmax_scale,
-               const bsa_block_lists *l, void *dq, void *dk, void *dv, uint8_t *ws,
+               const bsa_block_lists *l_in, void *dq, void *dk, void *dv, uint8_t *ws,
                DeviceInfo *dev, cudaStream_t stream) {
-  const BwdLayout w = bwd_layout(1, bh, l);
+  const BwdLayout w = bwd_layout(1, bh, n, l_in);
   float *lse2 = reinterpret_cast<float *>(ws + w.lse2);
   float *delta = reinterpret_cast<float *>(ws + w.delta);
   int32_t *col_ptr = reinterpret_cast<int32_t *>(ws + w.col_ptr);
   int32_t *row_idx = reinterpret_cast<int32_t *>(ws + w.row_idx);
+  // The kernels walk 128 x 128 tiles. Block-64 lists become tile lists with a
+  // 4-bit mask per entry (the listed 64 x 64 pairs of the tile pair).
+  bsa_block_lists tiles = *l_in;
+  const bsa_block_lists *l = &tiles;
+  const uint8_t *rmask = nullptr;
+  uint8_t *cmask = nullptr;
+  if (l_in->block != kBwdBlock) {
+    const int nt = ceil_div(n, kBwdBlock);
+    const int rows_t = l_in->num_lists * nt;
+    int32_t *tile_ptr = reinterpret_cast<int32_t *>(ws + w.tile_ptr);
+    int32_t *tile_col = reinterpret_cast<int32_t *>(ws + w.tile_col);
+    uint8_t *tile_mask = ws + w.tile_mask;
+    const long long cap = l_in->nnz > 0 ? l_in->nnz : 1;
+    tile_count_kernel<<<(rows_t + 127) / 128, 128, 0, stream>>>(
+        l_in->row_ptr, l_in->col_idx, l_in->num_q_blocks, l_in->num_k_blocks, l_in->nnz, nt,
+        rows_t, tile_ptr);
+    BSA_CUDA(cudaGetLastError());
+    scan_rows_kernel<<<1, 1024, 0, stream>>>(tile_ptr, rows_t);
+    BSA_CUDA(cudaGetLastError());
+    tile_fill_kernel<<<(rows_t + 127) / 128, 128, 0, stream>>>(
+        l_in->row_ptr, l_in->col_idx, l_in->num_q_blocks, l_in->num_k_blocks, l_in->nnz, nt,
+        rows_t, tile_ptr, tile_col, tile_mask, cap);
+    BSA_CUDA(cudaGetLastError());
+    tiles.num_q_blocks = tiles.num_k_blocks = nt;
+    tiles.block = kBwdBlock;
+    tiles.row_ptr = tile_ptr;
+    tiles.col_idx = tile_col;  // nnz stays the 64-list size: a bound on the tile entries
+    rmask = tile_mask;
+    cmask = ws + w.cmask;
+  }
   const int nqb = l->num_q_blocks, nkb = l->num_k_blocks;
 
   const long long rows = static_cast<long long>(bh) * nqb * kBwdBlock;
@@ -466,7 +507,7 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *out, con
   scan_rows_kernel<<<1, 1024, 0, stream>>>(col_ptr, cols);
   BSA_CUDA(cudaGetLastError());
   csc_fill_kernel<<<cols, 256, 0, stream>>>(l->row_ptr, l->col_idx, nqb, nkb, l->nnz, col_ptr,
-                                            row_idx, l->nnz);
+                                            row_idx, l->nnz > 0 ? l->nnz : 1, rmask, cmask);
   BSA_CUDA(cudaGetLastError());
 
   CUtensorMap tq, tk, tv, td;
@@ -475,16 +516,26 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *out, con
   if ((st = make_map(&tk, k, bh, n, D, kBwdBlock)) != BSA_OK) return st;
   if ((st = make_map(&tv, v, bh, n, D, kBwdBlock)) != BSA_OK) return st;
   if ((st = make_map(&td, dout, bh, n, D, kBwdBlock)) != BSA_OK) return st;
-  const int slot = 8 + (D == 128 ? 2 : 0);
+  const bool masked = rmask != nullptr;
+  const int slot = 8 + (D == 128 ? 2 : 0) + (masked ? 1 : 0);
   {
     std::lock_guard<std::mutex> lk(g_dev_mu);
     if (!dev->attrs_set[slot]) {
-      BSA_CUDA(cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    DkdvCfg<D>::DSMEM));
-      BSA_CUDA(cudaFuncSetAttribute(attn_bwd_dq_kernel<D>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    DqCfg<D>::DSMEM));
+      if (masked) {
+        BSA_CUDA(cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D, true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      DkdvCfg<D>::DSMEM));
+        BSA_CUDA(cudaFuncSetAttribute(attn_bwd_dq_kernel<D, true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      DqCfg<D>::DSMEM));
+      } else {
+        BSA_CUDA(cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D, false>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      DkdvCfg<D>::DSMEM));
+        BSA_CUDA(cudaFuncSetAttribute(attn_bwd_dq_kernel<D, false>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      DqCfg<D>::DSMEM));
+      }
       dev->attrs_set[slot] = true;
     }
   }
@@ -493,6 +544,8 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *out, con
   p.col_idx = l->col_idx;
   p.col_ptr = col_ptr;
   p.row_idx = row_idx;
+  p.rmask = rmask;
+  p.cmask = cmask;
   p.lse2 = lse2;
   p.delta = delta;
   p.dq = static_cast<__nv_bfloat16 *>(dq);
@@ -513,12 +566,21 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *out, con
   }
   p.total_items = bh * nkb;
   int grid = p.total_items < dev->sms ? p.total_items : dev->sms;
-  attn_bwd_dkdv_kernel<D><<<grid, DkdvCfg<D>::THREADS, DkdvCfg<D>::DSMEM, stream>>>(tq, tk, tv,
-                                                                                     td, p);
+  if (masked)
+    attn_bwd_dkdv_kernel<D, true><<<grid, DkdvCfg<D>::THREADS, DkdvCfg<D>::DSMEM, stream>>>(
+        tq, tk, tv, td, p);
+  else
+    attn_bwd_dkdv_kernel<D, false><<<grid, DkdvCfg<D>::THREADS, DkdvCfg<D>::DSMEM, stream>>>(
+        tq, tk, tv, td, p);
   BSA_CUDA(cudaGetLastError());
   p.total_items = bh * nqb;
   grid = p.total_items < dev->sms ? p.total_items : dev->sms;
-  attn_bwd_dq_kernel<D><<<grid, DqCfg<D>::THREADS, DqCfg<D>::DSMEM, stream>>>(tq, tk, tv, td, p);
+  if (masked)
+    attn_bwd_dq_kernel<D, true><<<grid, DqCfg<D>::THREADS, DqCfg<D>::DSMEM, stream>>>(tq, tk, tv,
+                                                                                      td, p);
+  else
+    attn_bwd_dq_kernel<D, false><<<grid, DqCfg<D>::THREADS, DqCfg<D>::DSMEM, stream>>>(tq, tk,
+                                                                                       tv, td, p);
   BSA_CUDA(cudaGetLastError());
   return BSA_OK;
 }
@@ -666,8 +728,8 @@ size_t bsa_attn_bwd_workspace_bytes(int32_t batch, int32_t heads, int32_t n,
   if (!l || batch < 1 || heads < 1 || n < 1 || l->num_q_blocks < 1 || l->num_k_blocks < 1)
     return 0;
   if (l->num_lists != 1 && l->num_lists != heads) return 0;
-  if (l->block != kBwdBlock || l->num_q_blocks != ceil_div(n, l->block)) return 0;
-  return bwd_layout(batch, heads, l).total;
+  if ((l->block != 64 && l->block != 128) || l->num_q_blocks != ceil_div(n, l->block)) return 0;
+  return bwd_layout(batch, heads, n, l).total;
 }
 
 int bsa_attn_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout,
@@ -677,7 +739,6 @@ int bsa_attn_bwd(const void *q, const void *k, const void *v, const void *out, c
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   int st = check_attn_args(q, k, v, batch, heads, n, head_dim, l, dq);
   if (st != BSA_OK) return st;
-  if (l->block != kBwdBlock) return BSA_ERR_UNSUPPORTED;
   if (!out || !dout || !lse || !dk || !dv) return BSA_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(dout) || !aligned16(dk) || !aligned16(dv) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u))
@@ -693,7 +754,7 @@ int bsa_attn_bwd(const void *q, const void *k, const void *v, const void *out, c
     for (int b = a + 1; b < 3; ++b)
       if (overlaps(outs[a], bytes, outs[b], bytes)) return BSA_ERR_INVALID_ARG;
   }
-  const size_t need = bwd_layout(batch, heads, l).total;
+  const size_t need = bwd_layout(batch, heads, n, l).total;
   if (!workspace || !aligned16(workspace) || workspace_bytes < need) return BSA_ERR_INVALID_ARG;
   if (overlaps(workspace, need, ins[0], bytes) || overlaps(workspace, need, dq, bytes) ||
       overlaps(workspace, need, dk, bytes) || overlaps(workspace, need, dv, bytes))

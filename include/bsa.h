@@ -305,8 +305,9 @@ int bsa_attn_dense_masked_ref(const void *q, const void *k, const void *v,
  * of query blocks with no key block get dq = 0, keys no query block lists get
  * dk = dv = 0), and not overlapping any input. workspace: device scratch of
  * at least bsa_attn_bwd_workspace_bytes() bytes, 16-byte aligned, owned by the
- * caller. Supported: block 128, head_dim 64 or 128 (block 64 returns
- * BSA_ERR_UNSUPPORTED). Deterministic: every output row is written by one
+ * caller. Supported: block 64 or 128, head_dim 64 or 128 (block-64 lists
+ * run as 128-row tiles with a mask of the listed 64 x 64 quarters).
+ * Deterministic: every output row is written by one
  * CTA, no atomics. Asynchronous on `stream`; device timeouts are reported
  * through bsa_get_device_status(). Returns BSA_OK or an argument / CUDA error.
  */
@@ -317,9 +318,10 @@ int bsa_attn_bwd(const void *q, const void *k, const void *v, const void *out, c
 
 /*
  * Workspace bytes bsa_attn_bwd needs: per query row of every (batch, head),
- * lse * log2(e) and delta, padded to whole blocks (2 x 4 bytes), plus the
- * transposed lists (num_lists * num_k_blocks + 1 offsets, nnz entries).
- * 0 when the arguments are invalid.
+ * lse * log2(e) and delta, padded to whole 128-row tiles (2 x 4 bytes), plus
+ * the transposed lists (num_lists * ceil(n / 128) + 1 offsets, nnz entries);
+ * at block 64 also the 128-row tile lists (offsets, entries) and one mask
+ * byte per tile and per transposed entry. 0 when the arguments are invalid.
  */
 size_t bsa_attn_bwd_workspace_bytes(int32_t batch, int32_t heads, int32_t n,
                                     const bsa_block_lists *lists);

@@ -108,8 +108,11 @@ def test_backward_workspace_and_host_checks(lib):
     expect = 2 * 40 * 256 * 128 * 4 + 1280 + 4096
     assert lib.bsa_attn_bwd_workspace_bytes(1, 40, 32760, ctypes.byref(ls)) == expect
     assert lib.bsa_attn_bwd_workspace_bytes(1, 40, 32769, ctypes.byref(ls)) == 0  # nqb mismatch
+    # block 64: the same plus masks of the transposed entries and the 128-row tile lists
     ls64 = BlockListsC(1, 512, 512, 64, 1000, 0, 0)
-    assert lib.bsa_attn_bwd_workspace_bytes(1, 40, 32760, ctypes.byref(ls64)) == 0  # block 64
+    expect64 = expect + 1024 + 1280 + 4096 + 1024
+    assert lib.bsa_attn_bwd_workspace_bytes(1, 40, 32760, ctypes.byref(ls64)) == expect64
+    assert lib.bsa_attn_bwd_workspace_bytes(1, 40, 32769, ctypes.byref(ls64)) == 0  # nqb mismatch
     # bad arguments are rejected on the host, before any CUDA call
     p = ctypes.c_void_p(4096)
     ls = BlockListsC(1, 8, 8, 128, 10, 4096, 4096)
@@ -128,10 +131,10 @@ def test_backward_workspace_and_host_checks(lib):
     bad = list(args)
     bad[9] = 96
     assert lib.bsa_attn_bwd(*bad) == 2  # head_dim
-    ls64 = BlockListsC(1, 16, 16, 64, 10, 4096, 4096)
+    bad32 = BlockListsC(1, 32, 32, 32, 10, 4096, 4096)
     bad = list(args)
-    bad[11] = ctypes.byref(ls64)
-    assert lib.bsa_attn_bwd(*bad) == 2  # block 64 unsupported
+    bad[11] = ctypes.byref(bad32)
+    assert lib.bsa_attn_bwd(*bad) == 2  # block 32 unsupported
 
 
 def test_strided_forward_host_checks(lib):

@@ -71,7 +71,25 @@ CASES = [
 
 @pytest.mark.parametrize("B,H,n,D,L,seed", CASES)
 def test_random_lists_full(bsa, B, H, n, D, L, seed):
-    blk = 128
+    _random_case(bsa, B, H, n, D, L, seed, 128)
+
+
+CASES_64 = [
+    # block 64: the kernels run 128-row tiles with a per-entry mask of the
+    # listed 64 x 64 pairs
+    (1, 1, 256, 64, 1, 31),
+    (1, 2, 1000, 128, 2, 32),    # per-head lists, ragged
+    (2, 2, 1050, 64, 1, 33),     # odd number of 64-blocks, batch > 1
+    (1, 3, 640, 128, 3, 34),
+]
+
+
+@pytest.mark.parametrize("B,H,n,D,L,seed", CASES_64)
+def test_random_lists_full_block64(bsa, B, H, n, D, L, seed):
+    _random_case(bsa, B, H, n, D, L, seed, 64)
+
+
+def _random_case(bsa, B, H, n, D, L, seed, blk):
     q, k, v = (t.cuda() for t in make_random_qkv(B, H, n, D, seed))
     nqb = -(-n // blk)
     rp, ci = random_block_lists(L * nqb, nqb, 0.5, seed + 100,
@@ -81,6 +99,20 @@ def test_random_lists_full(bsa, B, H, n, D, L, seed):
     do = _dout((B, H, n, D), seed + 7).cuda()
     dq, dk, dv = _run(bsa, q, k, v, lists, do)
     rq, rk, rv = oracle.masked_attention_backward_fp64(q, k, v, do, rp, ci, L, blk)
+    _close(dq.float().cpu(), rq, "dq")
+    _close(dk.float().cpu(), rk, "dk")
+    _close(dv.float().cpu(), rv, "dv")
+
+
+def test_tiny_radial_block64(bsa):
+    """The tiny radial configuration (4 x 256 tokens, block 64, D = 64)."""
+    w = WORKLOADS["tiny"]
+    q, k, v = (t.cuda() for t in make_qkv(w, "cpu"))
+    lists = bsa.radial_block_lists(w.frames, w.tokens_per_frame, w.block)
+    rp, ci = oracle.radial_block_lists(w.frames, w.tokens_per_frame, w.block)
+    do = _dout(q.shape, 51).cuda()
+    dq, dk, dv = _run(bsa, q, k, v, lists, do)
+    rq, rk, rv = oracle.masked_attention_backward_fp64(q, k, v, do, rp, ci, 1, w.block)
     _close(dq.float().cpu(), rq, "dq")
     _close(dk.float().cpu(), rk, "dk")
     _close(dv.float().cpu(), rv, "dv")
