@@ -29,7 +29,7 @@ __all__ = [
     "radial_block_lists", "block_lists_from_csr", "attention", "dense_masked_reference",
     "computed_flops", "bsa_attn_fwd_noalloc", "bsa_selftest_exp2", "NOALLOC_MAX_ORDER_ENTRIES",
     "bsa_attn_fwd_strided", "bsa_attn_module_workspace_bytes", "bsa_joint_mask_build",
-    "bsa_attn_fwd_host", "bsa_attn_fwd_host_workspace_bytes", "bsa_attn_module_fwd",
+    "bsa_attn_fwd_host", "bsa_attn_fwd_host_workspace_bytes", "bsa_attn_bwd_strided", "bsa_attn_module_fwd",
     "attention_module", "module_flops", "bsa_attn_bwd", "bsa_attn_bwd_workspace_bytes",
     "attention_backward",
 ]
@@ -255,6 +255,26 @@ def bsa_attn_bwd(q, k, v, out, dout, lse, lists: BlockLists, dq, dk, dv, workspa
     _check(st, "bsa_attn_bwd")
 
 
+def bsa_attn_bwd_strided(q, k, v, out, dout, lse, lists: BlockLists, dq, dk, dv, workspace=None,
+                         softmax_scale: float = 0.0, stream=None) -> None:
+    """bsa_attn_bwd on strided [B, H, n, D] views (contiguous last axis): reads
+    and writes every tensor through its strides, no copy."""
+    B, H, n, D = q.shape
+    lib = _lib.load()
+    ls = lists.c_struct()
+    if workspace is None:
+        workspace = torch.empty(max(lib.bsa_attn_bwd_workspace_bytes(B, H, n, ctypes.byref(ls)), 16),
+                                dtype=torch.uint8, device=q.device)
+    lay = [_layout(t) for t in (q, k, v, out, dout, dq, dk, dv)]
+    st = lib.bsa_attn_bwd_strided(
+        _ptr(q), ctypes.byref(lay[0]), _ptr(k), ctypes.byref(lay[1]), _ptr(v), ctypes.byref(lay[2]),
+        _ptr(out), ctypes.byref(lay[3]), _ptr(dout), ctypes.byref(lay[4]), _ptr(lse), B, H, n, D,
+        float(softmax_scale), ctypes.byref(ls), _ptr(dq), ctypes.byref(lay[5]), _ptr(dk),
+        ctypes.byref(lay[6]), _ptr(dv), ctypes.byref(lay[7]), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "bsa_attn_bwd_strided")
+
+
 def bsa_attn_dense_masked_ref(q, k, v, lists: BlockLists, out, lse=None,
                               softmax_scale: float = 0.0, stream=None) -> None:
     """Same result from the plain fp32 CUDA-core reference kernel (asynchronous)."""
@@ -371,10 +391,20 @@ def module_flops(batch: int, n: int, heads: int, head_dim: int, attention_flops:
 
 
 def attention_backward(q, k, v, out, dout, lse, lists: BlockLists, softmax_scale: float = 0.0,
-                       workspace=None, stream=None):
-    """Allocate gradients and run :func:`bsa_attn_bwd`; returns ``(dq, dk, dv)``."""
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    bsa_attn_bwd(q, k, v, out, dout, lse, lists, dq, dk, dv, workspace, softmax_scale, stream)
+                       workspace=None, stream=None, grads=None):
+    """Gradients of :func:`attention`; returns ``(dq, dk, dv)``. ``grads`` may
+    give the three output tensors (any views with a contiguous last axis);
+    otherwise they are allocated contiguous. All-contiguous calls go to
+    :func:`bsa_attn_bwd`, others to :func:`bsa_attn_bwd_strided`."""
+    if grads is None:
+        shape = tuple(q.shape)
+        grads = tuple(torch.empty(shape, dtype=q.dtype, device=q.device) for _ in range(3))
+    dq, dk, dv = grads
+    if all(t.is_contiguous() for t in (q, k, v, out, dout, dq, dk, dv)):
+        bsa_attn_bwd(q, k, v, out, dout, lse, lists, dq, dk, dv, workspace, softmax_scale, stream)
+    else:
+        bsa_attn_bwd_strided(q, k, v, out, dout, lse, lists, dq, dk, dv, workspace, softmax_scale,
+                             stream)
     return dq, dk, dv
 
 

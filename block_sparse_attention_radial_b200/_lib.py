@@ -26,6 +26,7 @@ EXPORTS = (
     "bsa_attn_module_fwd",
     "bsa_attn_dense_masked_ref",
     "bsa_attn_bwd",
+    "bsa_attn_bwd_strided",
     "bsa_attn_bwd_workspace_bytes",
     "bsa_validate_lists",
     "bsa_get_device_status",
@@ -118,6 +119,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bsa_attn_bwd": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float,
                                         lp, vp, vp, vp, vp, sz, vp]),
         "bsa_attn_bwd_workspace_bytes": (sz, [i32, i32, i32, lp]),
+        "bsa_attn_bwd_strided": (ctypes.c_int, [vp, yp, vp, yp, vp, yp, vp, yp, vp, yp, vp, i32,
+                                                i32, i32, i32, ctypes.c_float, lp, vp, yp, vp, yp,
+                                                vp, yp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

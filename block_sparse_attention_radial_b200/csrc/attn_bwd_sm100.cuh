@@ -45,13 +45,15 @@ struct BwdParams {
   const float *lse2;                 // [bh][nqb * 128]: lse * log2(e), +inf padding
   const float *delta;                // [bh][nqb * 128]: sum_d dO * O, 0 padding
   __nv_bfloat16 *dq, *dk, *dv;
+  // element strides (batch, head, token) of dq, dk, dv; head_dim contiguous
+  long long dq_s[3], dk_s[3], dv_s[3];
   // Block-64 lists run as 128-row tiles: a 4-bit mask per list entry, bit
   // qi * 2 + kj set when 64-row query block qi of the tile lists 64-key block
   // kj of the key tile (rmask per CSR entry, cmask per transposed entry).
   // Both null for block-128 lists (every pair of the tile is listed); read
   // only by the MASKED instances of the kernels.
   const uint8_t *rmask, *cmask;
-  int32_t heads, n, nqb, nkb, num_lists, nnz;
+  int32_t heads, n, nqb, nkb, num_lists, nnz;  // heads: per batch item
   int32_t total_items;
   float scale, scale_log2;
   unsigned long long wait_limit_ns;
@@ -62,9 +64,12 @@ constexpr int kBwdBlock = 128;
 // ------------------------------------------------------------------ prep --
 
 // One thread per padded query row of one (batch*head): delta and lse2.
+// out and dout are read through their (batch, head, token) element strides.
 template <int D>
 __global__ void bwd_prep_kernel(const __nv_bfloat16 *out, const __nv_bfloat16 *dout,
                                 const float *lse, float *lse2, float *delta, int n, int nqb,
+                                int heads, long long o_sb, long long o_sh, long long o_sn,
+                                long long d_sb, long long d_sh, long long d_sn,
                                 long long rows_total) {
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= rows_total) return;
@@ -77,8 +82,9 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16 *out, const __nv_bfloat16 *d
     return;
   }
   const long long row = bh * n + i;
-  const uint4 *o4 = reinterpret_cast<const uint4 *>(out + row * D);
-  const uint4 *d4 = reinterpret_cast<const uint4 *>(dout + row * D);
+  const long long b = bh / heads, h = bh - b * heads;
+  const uint4 *o4 = reinterpret_cast<const uint4 *>(out + b * o_sb + h * o_sh + i * o_sn);
+  const uint4 *d4 = reinterpret_cast<const uint4 *>(dout + b * d_sb + h * d_sh + i * d_sn);
   float acc = 0.f;
 #pragma unroll 4
   for (int c = 0; c < D / 8; ++c) {
@@ -365,8 +371,9 @@ __global__ void __launch_bounds__(192, 1)
         if (it.len == 0) continue;
         if (!(ok = lane_wait(&bar_kv_empty, (kvcount & 1u) ^ 1u, wc, kBarQEmpty, kvcount))) break;
         mbar_arrive_expect_tx(&bar_kv_full, 2 * C::T);
-        tma_load_4d(sK, &tm_k, &bar_kv_full, 0, it.blk * BN, 0, it.bh);
-        tma_load_4d(sV, &tm_v, &bar_kv_full, 0, it.blk * BN, 0, it.bh);
+        const int ib = it.bh / p.heads, ih = it.bh - ib * p.heads;
+        tma_load_5d(sK, &tm_k, &bar_kv_full, 0, it.blk * BN, 0, ih, ib);
+        tma_load_5d(sV, &tm_v, &bar_kv_full, 0, it.blk * BN, 0, ih, ib);
         ++kvcount;
         for (int e = 0; e < it.len && ok; ++e) {
           const int qb = min(max(__ldg(p.row_idx + it.a + e), 0), p.nqb - 1);
@@ -376,8 +383,8 @@ __global__ void __launch_bounds__(192, 1)
             break;
           uint8_t *st = sStage + s * C::STAGE;
           mbar_arrive_expect_tx(&bar_st_full[s], 2 * C::T + 1024);
-          tma_load_4d(st, &tm_q, &bar_st_full[s], 0, qb * BN, 0, it.bh);
-          tma_load_4d(st + C::T, &tm_do, &bar_st_full[s], 0, qb * BN, 0, it.bh);
+          tma_load_5d(st, &tm_q, &bar_st_full[s], 0, qb * BN, 0, ih, ib);
+          tma_load_5d(st + C::T, &tm_do, &bar_st_full[s], 0, qb * BN, 0, ih, ib);
           const long long off = static_cast<long long>(it.bh) * padded + static_cast<long long>(qb) * BN;
           bulk_load(st + 2 * C::T, p.lse2 + off, 512, &bar_st_full[s]);
           bulk_load(st + 2 * C::T + 512, p.delta + off, 512, &bar_st_full[s]);
@@ -517,11 +524,13 @@ __global__ void __launch_bounds__(192, 1)
       const BwdItem it = decode(idx);
       const int key = it.blk * BN + r;
       const bool store = key < p.n;
-      const long long orow = static_cast<long long>(it.bh) * p.n + key;
+      const long long ib = it.bh / p.heads, ih = it.bh - ib * p.heads;
+      __nv_bfloat16 *const dk_row = p.dk + ib * p.dk_s[0] + ih * p.dk_s[1] + key * p.dk_s[2];
+      __nv_bfloat16 *const dv_row = p.dv + ib * p.dv_s[0] + ih * p.dv_s[1] + key * p.dv_s[2];
       if (it.len == 0) {  // no query attends these keys
         if (store) {
-          uint4 *a = reinterpret_cast<uint4 *>(p.dk + orow * D);
-          uint4 *b = reinterpret_cast<uint4 *>(p.dv + orow * D);
+          uint4 *a = reinterpret_cast<uint4 *>(dk_row);
+          uint4 *b = reinterpret_cast<uint4 *>(dv_row);
 #pragma unroll
           for (int c = 0; c < D / 8; ++c) {
             a[c] = make_uint4(0, 0, 0, 0);
@@ -604,7 +613,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int part = 0; part < 2; ++part) {
         const uint32_t col = part == 0 ? C::DV_COL : C::DK_COL;
         const float mul = part == 0 ? 1.f : p.scale;
-        __nv_bfloat16 *dst = part == 0 ? p.dv : p.dk;
+        __nv_bfloat16 *dst = part == 0 ? dv_row : dk_row;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
@@ -612,7 +621,7 @@ __global__ void __launch_bounds__(192, 1)
           tmem_wait_ld();
           reg_fence32(v);
           if (store) {
-            uint4 *o4 = reinterpret_cast<uint4 *>(dst + orow * D + c * 32);
+            uint4 *o4 = reinterpret_cast<uint4 *>(dst + c * 32);
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
               uint4 x;
@@ -750,8 +759,9 @@ __global__ void __launch_bounds__(192, 1)
         if (it.len == 0) continue;
         if (!(ok = lane_wait(&bar_qd_empty, (qdcount & 1u) ^ 1u, wc, kBarQEmpty, qdcount))) break;
         mbar_arrive_expect_tx(&bar_qd_full, 2 * C::T);
-        tma_load_4d(sQ, &tm_q, &bar_qd_full, 0, it.blk * BN, 0, it.bh);
-        tma_load_4d(sDO, &tm_do, &bar_qd_full, 0, it.blk * BN, 0, it.bh);
+        const int ib = it.bh / p.heads, ih = it.bh - ib * p.heads;
+        tma_load_5d(sQ, &tm_q, &bar_qd_full, 0, it.blk * BN, 0, ih, ib);
+        tma_load_5d(sDO, &tm_do, &bar_qd_full, 0, it.blk * BN, 0, ih, ib);
         ++qdcount;
         for (int e = 0; e < it.len && ok; ++e) {
           const int kb = min(max(__ldg(p.col_idx + it.a + e), 0), p.nkb - 1);
@@ -761,8 +771,8 @@ __global__ void __launch_bounds__(192, 1)
             break;
           uint8_t *st = sStage + s * C::STAGE;
           mbar_arrive_expect_tx(&bar_st_full[s], 2 * C::T);
-          tma_load_4d(st, &tm_k, &bar_st_full[s], 0, kb * BN, 0, it.bh);
-          tma_load_4d(st + C::T, &tm_v, &bar_st_full[s], 0, kb * BN, 0, it.bh);
+          tma_load_5d(st, &tm_k, &bar_st_full[s], 0, kb * BN, 0, ih, ib);
+          tma_load_5d(st + C::T, &tm_v, &bar_st_full[s], 0, kb * BN, 0, ih, ib);
           ++ring;
         }
       }
@@ -887,10 +897,11 @@ __global__ void __launch_bounds__(192, 1)
       const BwdItem it = decode(idx);
       const int row = it.blk * BN + r;
       const bool store = row < p.n;
-      const long long orow = static_cast<long long>(it.bh) * p.n + row;
+      const long long ib = it.bh / p.heads, ih = it.bh - ib * p.heads;
+      __nv_bfloat16 *const dq_row = p.dq + ib * p.dq_s[0] + ih * p.dq_s[1] + row * p.dq_s[2];
       if (it.len == 0) {  // no key: dQ = 0
         if (store) {
-          uint4 *a = reinterpret_cast<uint4 *>(p.dq + orow * D);
+          uint4 *a = reinterpret_cast<uint4 *>(dq_row);
 #pragma unroll
           for (int c = 0; c < D / 8; ++c) a[c] = make_uint4(0, 0, 0, 0);
         }
@@ -959,7 +970,7 @@ __global__ void __launch_bounds__(192, 1)
         reg_fence32(v);
         if (store) {
           const float mul = p.scale;
-          uint4 *o4 = reinterpret_cast<uint4 *>(p.dq + orow * D + c * 32);
+          uint4 *o4 = reinterpret_cast<uint4 *>(dq_row + c * 32);
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
             uint4 x;

@@ -265,6 +265,32 @@ int check_strided_args(const void *q, const bsa_layout *lq, const void *k, const
   return BSA_OK;
 }
 
+// Whether two [batch, heads, n, D] views share no element. Exact for what
+// callers use: spans that do not overlap, or identical token-major layouts
+// (the heads of a token inside one token row, token rows of every batch item
+// one after another) whose bases sit at least one row footprint apart inside
+// a token row, as the q / k / v slices of one [batch, n, 3, heads, D] buffer
+// do. Anything else counts as overlapping.
+bool views_disjoint(const void *a, const bsa_layout &La, const void *b, const bsa_layout &Lb,
+                    int batch, int heads, int n, int D) {
+  if (!overlaps(a, layout_span_bytes(La, batch, heads, n, D), b,
+                layout_span_bytes(Lb, batch, heads, n, D)))
+    return true;
+  if (La.batch_stride != Lb.batch_stride || La.head_stride != Lb.head_stride ||
+      La.token_stride != Lb.token_stride)
+    return false;
+  const int64_t sn = La.token_stride;
+  const int64_t foot = (heads > 1 ? (heads - 1) * La.head_stride : 0) + D;
+  if (heads > 1 && La.head_stride < D) return false;
+  if (batch > 1 && La.batch_stride != static_cast<int64_t>(n) * sn) return false;
+  if (foot > sn) return false;
+  const int64_t bytes = static_cast<int64_t>(reinterpret_cast<uintptr_t>(b)) -
+                        static_cast<int64_t>(reinterpret_cast<uintptr_t>(a));
+  if (bytes % 2) return false;
+  const int64_t r = ((bytes / 2) % sn + sn) % sn;
+  return r >= foot && sn - r >= foot;
+}
+
 size_t order_bytes(const bsa_block_lists *l) {
   return (static_cast<size_t>(l->num_lists) * l->num_q_blocks * sizeof(int32_t) + 255) & ~size_t(255);
 }
@@ -454,11 +480,18 @@ BwdLayout bwd_layout(int32_t batch, int32_t heads, int32_t n, const bsa_block_li
   return w;
 }
 
+// Inputs, outputs and their layouts of one backward call.
+struct BwdViews {
+  const void *q, *k, *v, *out, *dout;
+  void *dq, *dk, *dv;
+  bsa_layout lq, lk, lv, lo, ldo, ldq, ldk, ldv;
+  int batch, heads;
+};
+
 template <int D>
-int launch_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout,
-               const float *lse, int32_t bh, int32_t n, float softmax_scale,
-               const bsa_block_lists *l_in, void *dq, void *dk, void *dv, uint8_t *ws,
-               DeviceInfo *dev, cudaStream_t stream) {
+int launch_bwd(const BwdViews &x, const float *lse, int32_t n, float softmax_scale,
+               const bsa_block_lists *l_in, uint8_t *ws, DeviceInfo *dev, cudaStream_t stream) {
+  const int32_t bh = x.batch * x.heads;
   const BwdLayout w = bwd_layout(1, bh, n, l_in);
   float *lse2 = reinterpret_cast<float *>(ws + w.lse2);
   float *delta = reinterpret_cast<float *>(ws + w.delta);
@@ -498,8 +531,9 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *out, con
 
   const long long rows = static_cast<long long>(bh) * nqb * kBwdBlock;
   bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 255) / 256), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16 *>(out), static_cast<const __nv_bfloat16 *>(dout), lse,
-      lse2, delta, n, nqb, rows);
+      static_cast<const __nv_bfloat16 *>(x.out), static_cast<const __nv_bfloat16 *>(x.dout), lse,
+      lse2, delta, n, nqb, x.heads, x.lo.batch_stride, x.lo.head_stride, x.lo.token_stride,
+      x.ldo.batch_stride, x.ldo.head_stride, x.ldo.token_stride, rows);
   BSA_CUDA(cudaGetLastError());
   const int cols = l->num_lists * nkb;
   csc_count_kernel<<<cols, 256, 0, stream>>>(l->row_ptr, l->col_idx, nqb, nkb, l->nnz, col_ptr);
@@ -512,10 +546,14 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *out, con
 
   CUtensorMap tq, tk, tv, td;
   int st;
-  if ((st = make_map(&tq, q, bh, n, D, kBwdBlock)) != BSA_OK) return st;
-  if ((st = make_map(&tk, k, bh, n, D, kBwdBlock)) != BSA_OK) return st;
-  if ((st = make_map(&tv, v, bh, n, D, kBwdBlock)) != BSA_OK) return st;
-  if ((st = make_map(&td, dout, bh, n, D, kBwdBlock)) != BSA_OK) return st;
+  if ((st = make_map_strided(&tq, x.q, x.lq, x.batch, x.heads, n, D, kBwdBlock)) != BSA_OK)
+    return st;
+  if ((st = make_map_strided(&tk, x.k, x.lk, x.batch, x.heads, n, D, kBwdBlock)) != BSA_OK)
+    return st;
+  if ((st = make_map_strided(&tv, x.v, x.lv, x.batch, x.heads, n, D, kBwdBlock)) != BSA_OK)
+    return st;
+  if ((st = make_map_strided(&td, x.dout, x.ldo, x.batch, x.heads, n, D, kBwdBlock)) != BSA_OK)
+    return st;
   const bool masked = rmask != nullptr;
   const int slot = 8 + (D == 128 ? 2 : 0) + (masked ? 1 : 0);
   {
@@ -548,10 +586,17 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *out, con
   p.cmask = cmask;
   p.lse2 = lse2;
   p.delta = delta;
-  p.dq = static_cast<__nv_bfloat16 *>(dq);
-  p.dk = static_cast<__nv_bfloat16 *>(dk);
-  p.dv = static_cast<__nv_bfloat16 *>(dv);
-  p.heads = l->num_lists > 1 ? l->num_lists : 1;
+  p.dq = static_cast<__nv_bfloat16 *>(x.dq);
+  p.dk = static_cast<__nv_bfloat16 *>(x.dk);
+  p.dv = static_cast<__nv_bfloat16 *>(x.dv);
+  const bsa_layout *outl[3] = {&x.ldq, &x.ldk, &x.ldv};
+  long long *outs[3] = {p.dq_s, p.dk_s, p.dv_s};
+  for (int i = 0; i < 3; ++i) {
+    outs[i][0] = outl[i]->batch_stride;
+    outs[i][1] = outl[i]->head_stride;
+    outs[i][2] = outl[i]->token_stride;
+  }
+  p.heads = x.heads;
   p.n = n;
   p.nqb = nqb;
   p.nkb = nkb;
@@ -723,6 +768,81 @@ int bsa_attn_fwd_strided(const void *q, const bsa_layout *q_layout, const void *
                  static_cast<int32_t *>(workspace), dev, fault_flags, stream);
 }
 
+int bsa_attn_bwd_strided(const void *q, const bsa_layout *q_layout, const void *k,
+                         const bsa_layout *k_layout, const void *v, const bsa_layout *v_layout,
+                         const void *out, const bsa_layout *out_layout, const void *dout,
+                         const bsa_layout *dout_layout, const float *lse, int32_t batch,
+                         int32_t heads, int32_t n, int32_t head_dim, float softmax_scale,
+                         const bsa_block_lists *l, void *dq, const bsa_layout *dq_layout,
+                         void *dk, const bsa_layout *dk_layout, void *dv,
+                         const bsa_layout *dv_layout, void *workspace, size_t workspace_bytes,
+                         bsa_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const bsa_layout *lays[8] = {q_layout, k_layout,  v_layout,  out_layout,
+                               dout_layout, dq_layout, dk_layout, dv_layout};
+  const void *ptrs[8] = {q, k, v, out, dout, dq, dk, dv};
+  for (int i = 0; i < 8; ++i)
+    if (!lays[i] || !ptrs[i]) return BSA_ERR_INVALID_ARG;
+  if (!lse || !l || !l->row_ptr || (l->nnz > 0 && !l->col_idx)) return BSA_ERR_INVALID_ARG;
+  if (batch < 1 || heads < 1 || n < 1) return BSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
+  if (l->block != 64 && l->block != 128) return BSA_ERR_UNSUPPORTED;
+  const long long nb = (static_cast<long long>(n) + l->block - 1) / l->block;
+  if (l->num_q_blocks != nb || l->num_k_blocks != nb) return BSA_ERR_INVALID_ARG;
+  if (l->num_lists != 1 && l->num_lists != heads) return BSA_ERR_INVALID_ARG;
+  if (l->nnz < 0) return BSA_ERR_INVALID_ARG;
+  const long long bhl = static_cast<long long>(batch) * heads;
+  if (bhl * nb > 0x7fffffffLL || bhl * n > 0x7fffffffLL) return BSA_ERR_UNSUPPORTED;
+  for (int i = 0; i < 8; ++i) {
+    if (!aligned16(ptrs[i])) return BSA_ERR_INVALID_ARG;
+    if (!layout_ok(*lays[i], batch, heads, n)) return BSA_ERR_INVALID_ARG;
+  }
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return BSA_ERR_INVALID_ARG;
+  size_t span[8];
+  for (int i = 0; i < 8; ++i) span[i] = layout_span_bytes(*lays[i], batch, heads, n, head_dim);
+  const size_t lbytes = static_cast<size_t>(bhl) * n * sizeof(float);
+  for (int a = 5; a < 8; ++a) {  // the gradients
+    if (!layout_disjoint(*lays[a], batch, heads, n, head_dim)) return BSA_ERR_INVALID_ARG;
+    for (int b = 0; b < 5; ++b)
+      if (overlaps(ptrs[a], span[a], ptrs[b], span[b])) return BSA_ERR_INVALID_ARG;
+    if (overlaps(ptrs[a], span[a], lse, lbytes)) return BSA_ERR_INVALID_ARG;
+    for (int b = a + 1; b < 8; ++b)
+      if (!views_disjoint(ptrs[a], *lays[a], ptrs[b], *lays[b], batch, heads, n, head_dim))
+        return BSA_ERR_INVALID_ARG;
+  }
+  const size_t need = bwd_layout(batch, heads, n, l).total;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < need) return BSA_ERR_INVALID_ARG;
+  for (int i = 0; i < 8; ++i)
+    if (overlaps(workspace, need, ptrs[i], span[i])) return BSA_ERR_INVALID_ARG;
+  if (overlaps(workspace, need, lse, lbytes)) return BSA_ERR_INVALID_ARG;
+  DeviceInfo *dev = nullptr;
+  int st;
+  if ((st = current_device(&dev)) != BSA_OK) return st;
+  if (dev->cc_major != 10) return BSA_ERR_UNSUPPORTED;
+  BwdViews x;
+  x.q = q;
+  x.k = k;
+  x.v = v;
+  x.out = out;
+  x.dout = dout;
+  x.dq = dq;
+  x.dk = dk;
+  x.dv = dv;
+  x.lq = *q_layout;
+  x.lk = *k_layout;
+  x.lv = *v_layout;
+  x.lo = *out_layout;
+  x.ldo = *dout_layout;
+  x.ldq = *dq_layout;
+  x.ldk = *dk_layout;
+  x.ldv = *dv_layout;
+  x.batch = batch;
+  x.heads = heads;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  if (head_dim == 128) return launch_bwd<128>(x, lse, n, softmax_scale, l, ws, dev, stream);
+  return launch_bwd<64>(x, lse, n, softmax_scale, l, ws, dev, stream);
+}
+
 size_t bsa_attn_bwd_workspace_bytes(int32_t batch, int32_t heads, int32_t n,
                                     const bsa_block_lists *l) {
   if (!l || batch < 1 || heads < 1 || n < 1 || l->num_q_blocks < 1 || l->num_k_blocks < 1)
@@ -762,13 +882,22 @@ int bsa_attn_bwd(const void *q, const void *k, const void *v, const void *out, c
   DeviceInfo *dev = nullptr;
   if ((st = current_device(&dev)) != BSA_OK) return st;
   if (dev->cc_major != 10) return BSA_ERR_UNSUPPORTED;
-  const int32_t bh = batch * heads;
+  BwdViews x;
+  x.q = q;
+  x.k = k;
+  x.v = v;
+  x.out = out;
+  x.dout = dout;
+  x.dq = dq;
+  x.dk = dk;
+  x.dv = dv;
+  x.lq = x.lk = x.lv = x.lo = x.ldo = x.ldq = x.ldk = x.ldv =
+      contiguous_layout(heads, n, head_dim);
+  x.batch = batch;
+  x.heads = heads;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
-  if (head_dim == 128)
-    return launch_bwd<128>(q, k, v, out, dout, lse, bh, n, softmax_scale, l, dq, dk, dv, ws, dev,
-                           stream);
-  return launch_bwd<64>(q, k, v, out, dout, lse, bh, n, softmax_scale, l, dq, dk, dv, ws, dev,
-                        stream);
+  if (head_dim == 128) return launch_bwd<128>(x, lse, n, softmax_scale, l, ws, dev, stream);
+  return launch_bwd<64>(x, lse, n, softmax_scale, l, ws, dev, stream);
 }
 
 int bsa_attn_dense_masked_ref(const void *q, const void *k, const void *v, int32_t batch,

@@ -317,6 +317,33 @@ int bsa_attn_bwd(const void *q, const void *k, const void *v, const void *out, c
                  void *workspace, size_t workspace_bytes, bsa_stream_t stream);
 
 /*
+ * bsa_attn_bwd on strided views (bsa_layout, as for bsa_attn_fwd_strided):
+ * the same gradients, with q, k, v, out, dout read and dq, dk, dv written
+ * through their strides (the kernels' TMA descriptors and stores carry
+ * them), so the gradients of a fused projection's q / k / v slices land in
+ * one [batch, n, 3, heads, head_dim] buffer without a transpose. lse stays
+ * [batch, heads, n] contiguous.
+ * Layout rules (BSA_ERR_INVALID_ARG otherwise): those of
+ * bsa_attn_fwd_strided for every view; each gradient's rows pairwise
+ * disjoint; the gradients share no element with each other (disjoint spans,
+ * or identical token-major layouts offset inside a token row by at least the
+ * row's head footprint, like three column slices of one buffer) and their
+ * spans overlap no input span, lse or the workspace. Workspace, limits,
+ * determinism and errors as bsa_attn_bwd. Asynchronous.
+ */
+int bsa_attn_bwd_strided(const void *q, const bsa_layout *q_layout,
+                         const void *k, const bsa_layout *k_layout,
+                         const void *v, const bsa_layout *v_layout,
+                         const void *out, const bsa_layout *out_layout,
+                         const void *dout, const bsa_layout *dout_layout,
+                         const float *lse, int32_t batch, int32_t heads, int32_t n,
+                         int32_t head_dim, float softmax_scale, const bsa_block_lists *lists,
+                         void *dq, const bsa_layout *dq_layout,
+                         void *dk, const bsa_layout *dk_layout,
+                         void *dv, const bsa_layout *dv_layout,
+                         void *workspace, size_t workspace_bytes, bsa_stream_t stream);
+
+/*
  * Workspace bytes bsa_attn_bwd needs: per query row of every (batch, head),
  * lse * log2(e) and delta, padded to whole 128-row tiles (2 x 4 bytes), plus
  * the transposed lists (num_lists * ceil(n / 128) + 1 offsets, nnz entries);

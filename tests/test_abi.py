@@ -190,3 +190,30 @@ def test_module_workspace_and_host_checks(lib):
     assert call(y=x) == 1                                       # y on top of x
     assert call(y=vp((8 << 30) + 4096)) == 1                    # y inside the workspace
     assert call(x=vp((1 << 30) + 8)) == 1                       # misaligned x
+
+
+def test_strided_backward_host_checks(lib):
+    """bsa_attn_bwd_strided rejects bad layouts on the host; the gradient
+    slices of one [B, n, 3, H, D] buffer are accepted as disjoint (checked
+    through the forward's identical rules for a gradient that would overlap)."""
+    from block_sparse_attention_radial_b200._lib import BlockListsC, LayoutC
+
+    vp, ref = ctypes.c_void_p, ctypes.byref
+    B, H, n, D = 1, 4, 1024, 64
+    C = H * D
+    ls = BlockListsC(1, 8, 8, 128, 10, 1 << 22, 1 << 23)
+    lqkv = LayoutC(n * 3 * C, D, 3 * C)
+    ltok = LayoutC(n * C, D, C)
+    qkv, attn, dattn, dqkv = 1 << 30, 1 << 32, 3 << 32, 1 << 34
+
+    def call(dq=dqkv, dk=dqkv + 2 * C, dv=dqkv + 4 * C, ldq=lqkv, ldk=lqkv, ldv=lqkv, wsb=16):
+        return lib.bsa_attn_bwd_strided(
+            vp(qkv), ref(lqkv), vp(qkv + 2 * C), ref(lqkv), vp(qkv + 4 * C), ref(lqkv),
+            vp(attn), ref(ltok), vp(dattn), ref(ltok), vp(5 << 32), B, H, n, D, 0.0, ref(ls),
+            vp(dq), ref(ldq), vp(dk), ref(ldk), vp(dv), ref(ldv), vp(1 << 36), wsb, None)
+
+    assert call() == 1                                   # workspace too small (layouts fine)
+    assert call(dk=dqkv + 2 * C - 64) == 1               # dk's rows reach into dq's
+    assert call(ldv=LayoutC(n * 3 * C, D, 3 * C + 8)) == 1  # different layout, shared span
+    assert call(dq=qkv) == 1                              # dq on top of the inputs
+    assert call(ldq=LayoutC(n * 3 * C, 8, 3 * C)) == 1   # dq's own rows overlap

@@ -184,3 +184,28 @@ def test_wan_sampled_rows_and_keys(bsa):
     rk, rv = oracle.masked_attention_dkdv_keys(qc, kc, vc, dc, rp, ci, 1, w.block, 0, 0, keys)
     _close(dk[0, 0, keys].float().cpu(), rk, "dk head 0")
     _close(dv[0, 0, keys].float().cpu(), rv, "dv head 0")
+
+
+@pytest.mark.parametrize("B,H,n,D,blk,L,seed", [(1, 3, 1000, 128, 128, 1, 61),
+                                                (2, 2, 700, 64, 64, 2, 62)])
+def test_strided_views_match_contiguous_bit_for_bit(bsa, B, H, n, D, blk, L, seed):
+    """q, k, v as slices of a [B, n, 3, H, D] projection buffer, out and dout
+    token-major, gradients into the slices of a second such buffer: the same
+    bits as the contiguous entry point."""
+    q, k, v = (t.cuda() for t in make_random_qkv(B, H, n, D, seed))
+    nqb = -(-n // blk)
+    rp, ci = random_block_lists(L * nqb, nqb, 0.5, seed + 100, force={0: [nqb - 1]})
+    lists = bsa.block_lists_from_csr(rp, ci, L, nqb, blk)
+    do = _dout((B, H, n, D), seed + 7).cuda()
+    out, lse = bsa.attention(q, k, v, lists)
+    ref = bsa.attention_backward(q, k, v, out, do, lse, lists)
+    tok = lambda t: t.transpose(1, 2).contiguous().transpose(1, 2)  # noqa: E731
+    buf = torch.stack([t.transpose(1, 2) for t in (q, k, v)], dim=2).contiguous()
+    qv, kv, vv = (buf[:, :, i].transpose(1, 2) for i in range(3))
+    gbuf = torch.full((B, n, 3, H, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    grads = tuple(gbuf[:, :, i].transpose(1, 2) for i in range(3))
+    got = bsa.attention_backward(qv, kv, vv, tok(out), tok(do), lse, lists, grads=grads)
+    assert bsa.bsa_get_device_status() == 0
+    for name, a, b in zip(("dq", "dk", "dv"), got, ref):
+        assert torch.equal(a, b), name
+    assert not torch.isnan(gbuf.float()).any()
