@@ -57,5 +57,6 @@ from .attention_backward import (  # noqa: F401
 )
 from .module import (  # noqa: F401
     radial_attention_module_fp64,
+    radial_attention_module_backward_fp64,
     radial_attention_module_rows,
 )

@@ -1,4 +1,4 @@
-"""Oracle: the radial attention module forward, in float64.
+"""Oracle: the radial attention module, forward and backward, in float64.
 
 TEST INFRASTRUCTURE ONLY (see the package docstring).
 
@@ -24,6 +24,9 @@ Functions:
 
 * ``radial_attention_module_fp64``: ``y [batch, n, C]`` of whole problems
   (small n).
+* ``radial_attention_module_backward_fp64``: the gradients of the output
+  with respect to x and to the four layers' weights and biases, given dy
+  (small n): the chain rule through the same steps in reverse order.
 * ``radial_attention_module_rows``: ``y`` of selected tokens of one batch
   item (any n). It writes ``out_proj`` as the sum over heads of
   ``O_h W_out[:, cols_h]^T`` (the same product, split by the columns of the
@@ -37,6 +40,7 @@ from __future__ import annotations
 import numpy as np
 
 from .attention import _as_f64, expand_row_mask, masked_attention_fp64, masked_attention_rows
+from .attention_backward import masked_attention_backward_fp64
 
 
 def _linear(x, w, b):
@@ -104,3 +108,53 @@ def radial_attention_module_rows(x, w_qkv, b_qkv, w_out, b_out, heads: int, row_
         o_h, _ = masked_attention_rows(q_h, k_h, v_h, adm, scale)
         y += o_h @ wo[:, cq].T
     return y
+
+
+def radial_attention_module_backward_fp64(x, w_qkv, b_qkv, w_out, b_out, dy, heads: int, row_ptr,
+                                          col_idx, num_lists: int, block: int,
+                                          scale: float | None = None):
+    """Gradients of ``radial_attention_module_fp64``'s output, given ``dy``
+    (``[batch, n, C]``). Returns ``(dx, dw_qkv, db_qkv, dw_out, db_out)`` with
+    the shapes of ``x``, ``w_qkv``, ``[3C]``, ``w_out``, ``[C]`` (the bias
+    gradients also when the biases are None: the layer's bias gradient).
+
+    Reverse order of the forward's steps:
+
+    * ``out_proj`` (``y = A W_out^T + b_out``): ``dA = dy W_out``,
+      ``dW_out = sum over tokens of dy^T A``, ``db_out = sum of dy``;
+    * head merge and split are reshapes: their gradients reshape back;
+    * the attention: ``masked_attention_backward_fp64``;
+    * each projection (``P = x W^T + b``): ``dW = dP^T x``, ``db = sum of dP``,
+      and ``dx`` sums ``dP W`` over the three projections.
+    """
+    x = _as_f64(x)
+    Bt, n, C = x.shape
+    D = C // heads
+    (wq, wk, wv), (bq, bk, bv) = _split_qkv(w_qkv, b_qkv, C)
+    wo = _as_f64(w_out)
+    dy = _as_f64(dy)
+
+    def heads_first(t):
+        return t.reshape(Bt, n, heads, D).transpose(0, 2, 1, 3)
+
+    def heads_merged(t):
+        return t.transpose(0, 2, 1, 3).reshape(Bt, n, C)
+
+    q = heads_first(_linear(x, wq, bq))
+    k = heads_first(_linear(x, wk, bk))
+    v = heads_first(_linear(x, wv, bv))
+    o, _ = masked_attention_fp64(q, k, v, row_ptr, col_idx, num_lists, block, scale)
+    a = heads_merged(o)
+    # out_proj
+    da = dy @ wo
+    dw_out = np.einsum("bni,bnj->ij", dy, a)
+    db_out = dy.sum(axis=(0, 1))
+    # attention
+    dq, dk, dv = masked_attention_backward_fp64(q, k, v, heads_first(da), row_ptr, col_idx,
+                                                num_lists, block, scale)
+    dqm, dkm, dvm = heads_merged(dq), heads_merged(dk), heads_merged(dv)
+    # projections
+    dw_qkv = np.concatenate([np.einsum("bno,bni->oi", g, x) for g in (dqm, dkm, dvm)], axis=0)
+    db_qkv = np.concatenate([g.sum(axis=(0, 1)) for g in (dqm, dkm, dvm)])
+    dx = dqm @ wq + dkm @ wk + dvm @ wv
+    return dx, dw_qkv, db_qkv, dw_out, db_out

@@ -114,3 +114,80 @@ def test_planted_head_split_slip_is_caught():
     y_wrong = o.transpose(0, 2, 1, 3).reshape(B, n, C) @ wo.float().double().numpy().T \
         + bo.float().double().numpy()
     assert np.abs(y_wrong - good).max() > 1e-2
+
+
+
+def _torch_mha_grads(x, w_qkv, b_qkv, w_out, b_out, dy, heads, allowed):
+    """float64 autograd through torch's multi_head_attention_forward."""
+    leaves = [_f64(t).clone().requires_grad_() for t in (x, w_qkv, b_qkv, w_out, b_out)]
+    xl, wq, bq, wo, bo = leaves
+    xt = xl.transpose(0, 1)
+    C = xt.shape[-1]
+    y, _ = torch.nn.functional.multi_head_attention_forward(
+        xt, xt, xt, C, heads, wq, bq, None, None, False, 0.0, wo, bo, training=False,
+        need_weights=False, attn_mask=torch.from_numpy(~allowed))
+    (y.transpose(0, 1) * _f64(dy)).sum().backward()
+    return [t.grad.numpy() for t in leaves]
+
+
+@pytest.mark.parametrize("B,n,H,D,blk,L,seed", [(2, 70, 2, 8, 16, 1, 61), (1, 100, 3, 4, 32, 3, 62)])
+def test_backward_matches_torch_autograd(B, n, H, D, blk, L, seed):
+    x, wqkv, bqkv, wo, bo = make_module_inputs(B, n, H, D, seed)
+    dy, _, _, _, _ = make_module_inputs(B, n, H, D, seed + 1, bias=False)
+    nqb = -(-n // blk)
+    rp, ci = random_block_lists(L * nqb, nqb, 0.5, seed + 10)
+    empty = np.nonzero(np.diff(rp) == 0)[0]
+    rp, ci = random_block_lists(L * nqb, nqb, 0.5, seed + 10,
+                                force={int(r): [int(r) % nqb] for r in empty})
+    got = oracle.radial_attention_module_backward_fp64(x, wqkv, bqkv, wo, bo, dy, H, rp, ci, L,
+                                                       blk)
+    rows = np.arange(n)
+    if L == 1:
+        allowed = oracle.expand_row_mask(rp, ci, 0, rows, n, blk)
+    else:
+        per_head = [oracle.expand_row_mask(rp, ci, h * nqb, rows, n, blk) for h in range(H)]
+        allowed = np.stack([per_head[h] for _ in range(B) for h in range(H)])
+    ref = _torch_mha_grads(x, wqkv, bqkv, wo, bo, dy, H, allowed)
+    for name, g, r in zip(("dx", "dw_qkv", "db_qkv", "dw_out", "db_out"), got, ref):
+        np.testing.assert_allclose(g, r, rtol=1e-9, atol=1e-10, err_msg=name)
+
+
+def test_backward_finite_differences():
+    """Central differences of the forward oracle on sampled entries of every
+    gradient (rows with empty lists included)."""
+    B, n, H, D, blk = 1, 24, 2, 4, 8
+    x, wqkv, bqkv, wo, bo = (t.float().double().numpy()
+                             for t in make_module_inputs(B, n, H, D, 71))
+    dy = np.random.default_rng(72).standard_normal((B, n, H * D))
+    nqb = n // blk
+    rp, ci = random_block_lists(nqb, nqb, 0.5, 73, empty_rows=[1], force={0: [2]})
+    grads = oracle.radial_attention_module_backward_fp64(x, wqkv, bqkv, wo, bo, dy, H, rp, ci, 1,
+                                                         blk)
+    params = [x, wqkv, bqkv, wo, bo]
+
+    def loss(ps):
+        return float((oracle.radial_attention_module_fp64(*ps, H, rp, ci, 1, blk) * dy).sum())
+
+    rng = np.random.default_rng(74)
+    eps = 1e-6
+    for i, (p_, g) in enumerate(zip(params, grads)):
+        for _ in range(6):
+            idx = tuple(int(rng.integers(0, s)) for s in p_.shape)
+            hi = [q.copy() for q in params]
+            lo = [q.copy() for q in params]
+            hi[i][idx] += eps
+            lo[i][idx] -= eps
+            fd = (loss(hi) - loss(lo)) / (2 * eps)
+            np.testing.assert_allclose(g[idx], fd, rtol=1e-5, atol=1e-7)
+
+
+def test_backward_planted_slip_is_caught():
+    """Taking dw_out as A^T dy (transposed) is caught by the autograd pin's tolerance."""
+    B, n, H, D, blk = 1, 32, 2, 4, 8
+    x, wqkv, bqkv, wo, bo = make_module_inputs(B, n, H, D, 81)
+    dy, _, _, _, _ = make_module_inputs(B, n, H, D, 82, bias=False)
+    nqb = n // blk
+    rp, ci = random_block_lists(nqb, nqb, 0.6, 83, force={0: [0]})
+    _, _, _, dwo, _ = oracle.radial_attention_module_backward_fp64(x, wqkv, bqkv, wo, bo, dy, H, rp,
+                                                                   ci, 1, blk)
+    assert np.abs(dwo - dwo.T).max() > 1e-3
