@@ -29,7 +29,8 @@ __all__ = [
     "radial_block_lists", "block_lists_from_csr", "attention", "dense_masked_reference",
     "computed_flops", "bsa_attn_fwd_noalloc", "bsa_selftest_exp2", "NOALLOC_MAX_ORDER_ENTRIES",
     "bsa_attn_fwd_strided", "bsa_attn_module_workspace_bytes", "bsa_joint_mask_build",
-    "bsa_attn_fwd_host", "bsa_attn_fwd_host_workspace_bytes", "bsa_attn_bwd_strided", "bsa_attn_module_fwd",
+    "bsa_attn_fwd_host", "bsa_attn_fwd_host_workspace_bytes", "bsa_attn_bwd_strided",
+    "bsa_attn_module_bwd", "bsa_attn_module_bwd_workspace_bytes", "attention_module_backward", "bsa_attn_module_fwd",
     "attention_module", "module_flops", "bsa_attn_bwd", "bsa_attn_bwd_workspace_bytes",
     "attention_backward",
 ]
@@ -219,6 +220,37 @@ def bsa_attn_module_fwd(x, w_qkv, b_qkv, w_out, b_out, heads: int, lists: BlockL
     _check(st, "bsa_attn_module_fwd")
 
 
+def bsa_attn_module_bwd_workspace_bytes(batch: int, n: int, heads: int, head_dim: int,
+                                        lists: BlockLists) -> int:
+    return int(_lib.load().bsa_attn_module_bwd_workspace_bytes(batch, n, heads, head_dim,
+                                                               ctypes.byref(lists.c_struct())))
+
+
+def bsa_attn_module_bwd(x, w_qkv, w_out, dy, heads: int, lists: BlockLists, fwd_workspace,
+                        dx, dw_qkv, db_qkv, dw_out, db_out, workspace=None,
+                        softmax_scale: float = 0.0, stream=None) -> None:
+    """Gradients of the module forward whose workspace is ``fwd_workspace``:
+    dx [B, n, C], dw_qkv [3C, C], db_qkv [3C] (or None), dw_out [C, C],
+    db_out [C] (or None), all bf16."""
+    B, n, C = x.shape
+    D = C // heads
+    lib = _lib.load()
+    ls = lists.c_struct()
+    if workspace is None:
+        workspace = torch.empty(lib.bsa_attn_module_bwd_workspace_bytes(B, n, heads, D,
+                                                                        ctypes.byref(ls)),
+                                dtype=torch.uint8, device=x.device)
+    for t in (x, w_qkv, w_out, dy, dx, dw_qkv, db_qkv, dw_out, db_out):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("bsa_attn_module_bwd takes contiguous tensors")
+    st = lib.bsa_attn_module_bwd(
+        _ptr(x), _ptr(w_qkv), _ptr(w_out), _ptr(dy), B, n, heads, D, float(softmax_scale),
+        ctypes.byref(ls), _ptr(fwd_workspace), fwd_workspace.numel() * fwd_workspace.element_size(),
+        _ptr(dx), _ptr(dw_qkv), _ptr(db_qkv), _ptr(dw_out), _ptr(db_out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "bsa_attn_module_bwd")
+
+
 def bsa_attn_fwd_noalloc(q, k, v, lists: BlockLists, out, lse=None,
                          softmax_scale: float = 0.0, stream=None) -> None:
     """bsa_attn_fwd without a workspace, for callers that cannot allocate device
@@ -376,11 +408,28 @@ def attention(q, k, v, lists: BlockLists, softmax_scale: float = 0.0, want_lse: 
 
 def attention_module(x, w_qkv, b_qkv, w_out, b_out, heads: int, lists: BlockLists,
                      softmax_scale: float = 0.0, workspace=None, stream=None):
-    """Allocate y and run :func:`bsa_attn_module_fwd`; returns y (bf16 [B, n, C])."""
+    """Allocate y and run :func:`bsa_attn_module_fwd`; returns y (bf16 [B, n, C]).
+    Pass ``workspace`` (of :func:`bsa_attn_module_workspace_bytes`) to keep the
+    saved q/k/v, attention output and lse for :func:`attention_module_backward`."""
     y = torch.empty_like(x)
     bsa_attn_module_fwd(x, w_qkv, b_qkv, w_out, b_out, heads, lists, y, workspace, softmax_scale,
                         stream)
     return y
+
+
+def attention_module_backward(x, w_qkv, w_out, dy, heads: int, lists: BlockLists, fwd_workspace,
+                              softmax_scale: float = 0.0, biases: bool = True, workspace=None,
+                              stream=None):
+    """Allocate the gradients and run :func:`bsa_attn_module_bwd`; returns
+    ``(dx, dw_qkv, db_qkv, dw_out, db_out)`` (the bias gradients None when
+    ``biases`` is False)."""
+    C = x.shape[-1]
+    dx, dwq, dwo = torch.empty_like(x), torch.empty_like(w_qkv), torch.empty_like(w_out)
+    dbq = torch.empty(3 * C, dtype=x.dtype, device=x.device) if biases else None
+    dbo = torch.empty(C, dtype=x.dtype, device=x.device) if biases else None
+    bsa_attn_module_bwd(x, w_qkv, w_out, dy, heads, lists, fwd_workspace, dx, dwq, dbq, dwo, dbo,
+                        workspace, softmax_scale, stream)
+    return dx, dwq, dbq, dwo, dbo
 
 
 def module_flops(batch: int, n: int, heads: int, head_dim: int, attention_flops: int) -> int:

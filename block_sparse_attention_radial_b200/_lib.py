@@ -24,6 +24,8 @@ EXPORTS = (
     "bsa_attn_fwd_host",
     "bsa_attn_module_workspace_bytes",
     "bsa_attn_module_fwd",
+    "bsa_attn_module_bwd_workspace_bytes",
+    "bsa_attn_module_bwd",
     "bsa_attn_dense_masked_ref",
     "bsa_attn_bwd",
     "bsa_attn_bwd_strided",
@@ -101,6 +103,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                                 ctypes.c_float, lp, vp, yp, vp, vp, sz, vp]),
         "bsa_attn_module_workspace_bytes": (sz, [i32, i32, i32, i32, lp]),
         "bsa_attn_fwd_host_workspace_bytes": (sz, [i32, i32, i32, i32, lp]),
+        "bsa_attn_module_bwd_workspace_bytes": (sz, [i32, i32, i32, i32, lp]),
+        "bsa_attn_module_bwd": (ctypes.c_int, [vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float,
+                                               lp, vp, sz, vp, vp, vp, vp, vp, vp, sz, vp]),
         "bsa_attn_fwd_host": (ctypes.c_int, [vp, vp, vp, i32, i32, i32, i32, ctypes.c_float, lp,
                                              vp, vp, vp, sz, vp]),
         "bsa_attn_module_fwd": (ctypes.c_int, [vp, vp, vp, vp, vp, i32, i32, i32, i32,

@@ -260,7 +260,8 @@ size_t bsa_attn_module_workspace_bytes(int32_t batch, int32_t n, int32_t heads,
  * y      device bf16 [batch, n, C]; must not overlap x, the weights or the
  *        workspace.
  * workspace  device scratch of bsa_attn_module_workspace_bytes(); the
- *        projected q/k/v and the attention output stay there after the call.
+ *        projected q/k/v, the attention output and its lse stay there after
+ *        the call (bsa_attn_module_bwd reads them).
  * Head h of the split is columns [h*head_dim, (h+1)*head_dim) of each
  * projection (the page's view(batch, n, heads, head_dim)). The projections
  * are cuBLASLt GEMMs (bf16 in, fp32 accumulate, bias in the epilogue, bf16
@@ -273,6 +274,44 @@ int bsa_attn_module_fwd(const void *x, const void *w_qkv, const void *b_qkv,
                         const void *w_out, const void *b_out,
                         int32_t batch, int32_t n, int32_t heads, int32_t head_dim,
                         float softmax_scale, const bsa_block_lists *lists, void *y,
+                        void *workspace, size_t workspace_bytes, bsa_stream_t stream);
+
+/*
+ * Bytes of device scratch bsa_attn_module_bwd needs: the attention output's
+ * gradient [batch*n, C] and the q/k/v gradients [batch*n, 3C] (bf16), the
+ * attention backward's workspace, bias-gradient partial sums and 32 MiB of
+ * GEMM scratch. Returns 0 for invalid arguments.
+ */
+size_t bsa_attn_module_bwd_workspace_bytes(int32_t batch, int32_t n, int32_t heads,
+                                           int32_t head_dim, const bsa_block_lists *lists);
+
+/*
+ * Backward of bsa_attn_module_fwd: given dy = dL/dy (bf16 [batch, n, C]),
+ * the gradients of x and of the four nn.Linear layers' weights and biases
+ * (the LoRA fine-tuning of the "Radial Attention" skill page, Step 4, runs
+ * loss.backward() through this module). With the forward's A = the attention
+ * output, heads merged ([batch*n, C]) and QKV = the stacked projection:
+ *   dA = dy w_out,            dw_out = dy^T A,        db_out = column sums of dy,
+ *   dQKV = attention backward (bsa_attn_bwd's operation) of dA, laid out as
+ *          QKV's q / k / v column slices,
+ *   dw_qkv = dQKV^T x,        db_qkv = column sums of dQKV,   dx = dQKV w_qkv.
+ * x, w_qkv, w_out, lists, softmax_scale: exactly as given to the forward.
+ * fwd_workspace: the forward call's workspace, unchanged since (q/k/v, A and
+ *   lse are read from it).
+ * dx [batch, n, C], dw_qkv [3C, C], dw_out [C, C]: bf16 outputs; db_qkv [3C]
+ *   and db_out [C]: bf16 outputs or NULL (not computed). No output may
+ *   overlap an input, a workspace or another output.
+ * workspace: bsa_attn_module_bwd_workspace_bytes() of device scratch.
+ * GEMMs on cuBLASLt (bf16 in, fp32 accumulate, bf16 out); bias gradients by a
+ * fixed-order two-pass column sum (fp32), so the whole backward is
+ * deterministic. 16-byte aligned pointers; limits and errors as bsa_attn_bwd.
+ * Asynchronous.
+ */
+int bsa_attn_module_bwd(const void *x, const void *w_qkv, const void *w_out, const void *dy,
+                        int32_t batch, int32_t n, int32_t heads, int32_t head_dim,
+                        float softmax_scale, const bsa_block_lists *lists,
+                        const void *fwd_workspace, size_t fwd_workspace_bytes,
+                        void *dx, void *dw_qkv, void *db_qkv, void *dw_out, void *db_out,
                         void *workspace, size_t workspace_bytes, bsa_stream_t stream);
 
 /*

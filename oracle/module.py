@@ -147,14 +147,15 @@ def radial_attention_module_backward_fp64(x, w_qkv, b_qkv, w_out, b_out, dy, hea
     a = heads_merged(o)
     # out_proj
     da = dy @ wo
-    dw_out = np.einsum("bni,bnj->ij", dy, a)
+    dw_out = dy.reshape(-1, C).T @ a.reshape(-1, C)  # sum over (batch, token) of dy^T A
     db_out = dy.sum(axis=(0, 1))
     # attention
     dq, dk, dv = masked_attention_backward_fp64(q, k, v, heads_first(da), row_ptr, col_idx,
                                                 num_lists, block, scale)
     dqm, dkm, dvm = heads_merged(dq), heads_merged(dk), heads_merged(dv)
     # projections
-    dw_qkv = np.concatenate([np.einsum("bno,bni->oi", g, x) for g in (dqm, dkm, dvm)], axis=0)
+    xr = x.reshape(-1, C)
+    dw_qkv = np.concatenate([g.reshape(-1, C).T @ xr for g in (dqm, dkm, dvm)], axis=0)
     db_qkv = np.concatenate([g.sum(axis=(0, 1)) for g in (dqm, dkm, dvm)])
     dx = dqm @ wq + dkm @ wk + dvm @ wv
     return dx, dw_qkv, db_qkv, dw_out, db_out

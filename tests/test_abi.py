@@ -171,9 +171,15 @@ def test_module_workspace_and_host_checks(lib):
 
     vp, ref = ctypes.c_void_p, ctypes.byref
     ls = BlockListsC(1, 256, 256, 128, 1000, 0, 0)
-    # work order (1 KiB) + q/k/v [32760, 15360] + attention out [32760, 5120] bf16 + 32 MiB
-    expect = 1024 + 32760 * 15360 * 2 + 32760 * 5120 * 2 + (32 << 20)
+    # work order (1 KiB) + q/k/v [32760, 15360] + attention out [32760, 5120] bf16
+    # + lse [40, 32760] fp32 + 32 MiB
+    expect = 1024 + 32760 * 15360 * 2 + 32760 * 5120 * 2 + 40 * 32760 * 4 + (32 << 20)
     assert lib.bsa_attn_module_workspace_bytes(1, 32760, 40, 128, ref(ls)) == expect
+    # backward: dA [32760, 5120] + dQKV [32760, 15360] bf16 + the attention
+    # backward's workspace + 32 x 15360 fp32 partial sums + 32 MiB
+    attn_bwd = lib.bsa_attn_bwd_workspace_bytes(1, 40, 32760, ref(ls))
+    expect_b = 32760 * 5120 * 2 + 32760 * 15360 * 2 + attn_bwd + 32 * 15360 * 4 + (32 << 20)
+    assert lib.bsa_attn_module_bwd_workspace_bytes(1, 32760, 40, 128, ref(ls)) == expect_b
     assert lib.bsa_attn_module_workspace_bytes(1, 32760, 40, 128, None) == 0
     B, n, H, D = 1, 1000, 2, 64
     small = BlockListsC(1, 8, 8, 128, 10, 1 << 22, 1 << 23)
