@@ -580,14 +580,21 @@ def run_ours_bwd(args, world, rank, local):
 
 METRIC_MODULE = ("radial attention module fwd (q/k/v projection, block-sparse attention, "
                  "out projection) ms & effective TFLOP/s at 32k-120k tokens")
+METRIC_MODULE_BWD = ("radial attention module bwd (dx, dW, db of the four projections through the "
+                     "block-sparse attention backward) ms & effective TFLOP/s at 32k-120k tokens")
 
 
-def run_ours_module(args, world, rank, local):
+def run_ours_module(args, world, rank, local, backward=False):
     """Time bsa_attn_module_fwd: the RadialAttention module forward of the
     skill page (one stacked q/k/v projection GEMM, the attention on strided
     views of its output, the output projection GEMM), with random-init
     weights of the workload's width (C = heads x head_dim). value counts the
-    two GEMMs' FLOPs plus the attention's computed-block FLOPs."""
+    two GEMMs' FLOPs plus the attention's computed-block FLOPs.
+
+    With ``backward``, time bsa_attn_module_bwd instead (after one forward
+    that fills the saved q/k/v, attention output and lse): four GEMMs
+    (16 n C^2 FLOPs), the attention backward (counted as 2.5 x the forward's
+    computed-block FLOPs; it executes 3.5 x) and two column sums."""
     import numpy as np
     import torch
 
@@ -607,16 +614,36 @@ def run_ours_module(args, world, rank, local):
     rp_h, ci_h = lists.row_ptr.cpu().numpy(), lists.col_idx.cpu().numpy()
     att_flops = bsa.computed_flops(rp_h, ci_h, n, w.block, D, w.batch, H, 1)
     flops = bsa.module_flops(w.batch, n, H, D, att_flops)
+    exec_flops = flops
     y = torch.empty_like(x)
     ws = torch.empty(bsa.bsa_attn_module_workspace_bytes(w.batch, n, H, D, lists),
                      dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     launches_per_step = 2  # work order, attention (the two GEMMs are cuBLASLt's)
+    if backward:
+        C = H * D
+        flops = 16 * w.batch * n * C * C + 2.5 * att_flops
+        exec_flops = 16 * w.batch * n * C * C + 3.5 * att_flops
+        g = torch.Generator(device=dev)
+        g.manual_seed(w.seed + 2000)
+        dy = torch.randn(x.shape, generator=g, device=dev).to(torch.bfloat16)
+        grads = (torch.empty_like(x), torch.empty_like(wqkv),
+                 torch.empty(3 * C, dtype=x.dtype, device=dev), torch.empty_like(wo),
+                 torch.empty(C, dtype=x.dtype, device=dev))
+        bws = torch.empty(bsa.bsa_attn_module_bwd_workspace_bytes(w.batch, n, H, D, lists),
+                          dtype=torch.uint8, device=dev)
+        bsa.bsa_attn_module_fwd(x, wqkv, bqkv, wo, bo, H, lists, y, ws, 0.0, stream)
+        # attention backward: prep, transposed-list count, scan, fill, dK/dV, dQ;
+        # two column-sum passes for each bias gradient (the GEMMs are cuBLASLt's)
+        launches_per_step = 6 + 4
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        bsa.bsa_attn_module_fwd(x, wqkv, bqkv, wo, bo, H, lists, y, ws, 0.0, stream)
+        if backward:
+            bsa.bsa_attn_module_bwd(x, wqkv, wo, dy, H, lists, ws, *grads, bws, 0.0, stream)
+        else:
+            bsa.bsa_attn_module_fwd(x, wqkv, bqkv, wo, bo, H, lists, y, ws, 0.0, stream)
         if ev is not None:
             ev[1].record(stream)
 
@@ -650,16 +677,27 @@ def run_ours_module(args, world, rank, local):
     if bsa.bsa_get_device_status() != 0:
         raise SystemExit("device status after the timed region")
 
-    # end to end: x from pinned host memory in, y back to the host
+    # end to end: x (backward: dy) from pinned host memory in, y (backward:
+    # every gradient) back to the host
     e2e_steps = max(3, min(args.steps, 10))
-    x_host = x.cpu().pin_memory()
-    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-    x_dev = torch.empty_like(x)
+    if backward:
+        x_host = dy.cpu().pin_memory()
+        x_dev = torch.empty_like(dy)
+        out_dev = grads
+    else:
+        x_host = x.cpu().pin_memory()
+        x_dev = torch.empty_like(x)
+        out_dev = (y,)
+    out_host = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in out_dev]
 
     def e2e_step():
         x_dev.copy_(x_host, non_blocking=True)
-        bsa.bsa_attn_module_fwd(x_dev, wqkv, bqkv, wo, bo, H, lists, y, ws, 0.0, stream)
-        y_host.copy_(y, non_blocking=True)
+        if backward:
+            bsa.bsa_attn_module_bwd(x, wqkv, wo, x_dev, H, lists, ws, *grads, bws, 0.0, stream)
+        else:
+            bsa.bsa_attn_module_fwd(x_dev, wqkv, bqkv, wo, bo, H, lists, y, ws, 0.0, stream)
+        for h_, d_ in zip(out_host, out_dev):
+            h_.copy_(d_, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize(dev)
@@ -672,10 +710,10 @@ def run_ours_module(args, world, rank, local):
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
     h2d = x_host.numel() * x_host.element_size()
-    d2h = y_host.numel() * y_host.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in out_host)
 
     cpu_baseline = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not backward:
         import oracle
 
         C = H * D
@@ -708,13 +746,13 @@ def run_ours_module(args, world, rank, local):
     if rank == 0:
         peaks, peak_kind = load_peaks()
         peak = float(peaks["bf16_tflops"])
-        achieved = flops / (kernel_ms * 1e-3) / 1e12
+        achieved = exec_flops / (kernel_ms * 1e-3) / 1e12
         cfg = workload_config(w, nnz=int(rp_h[-1]))
         cfg["hidden"] = H * D
         cfg["l2"] = ("x and the q/k/v projection output exceed L2 (126 MB) many times over; "
                      "no flush")
         line = {
-            "metric": METRIC_MODULE,
+            "metric": METRIC_MODULE_BWD if backward else METRIC_MODULE,
             "value": flops * world * args.steps / (ms * 1e-3) / 1e12,
             "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -725,9 +763,12 @@ def run_ours_module(args, world, rank, local):
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": None,
                          "peak_kind": f"{peak_kind} bf16 burst",
-                         "kernel": "whole module: cuBLASLt q/k/v GEMM + work order + "
-                                   "attn_fwd_pair_sm100_kernel<128> + cuBLASLt out GEMM",
-                         "kernel_ms": kernel_ms, "flops_per_launch": flops},
+                         "kernel": ("whole module backward: four cuBLASLt GEMMs + attention "
+                                    "backward (attn_bwd_dkdv/dq_kernel<128>) + column sums")
+                         if backward else
+                         ("whole module: cuBLASLt q/k/v GEMM + work order + "
+                          "attn_fwd_pair_sm100_kernel<128> + cuBLASLt out GEMM"),
+                         "kernel_ms": kernel_ms, "flops_per_launch": exec_flops},
             "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
@@ -751,9 +792,10 @@ def main(argv=None):
     ap.add_argument("--workload", default="wan", choices=("wan", "hunyuan", "long4x", "tiny", "hunyuan_text"))
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="which", choices=("fwd", "bwd", "module"), default="fwd",
-                    help="time the forward (default, the headline), the backward pass or the "
-                         "whole module forward (projections + attention)")
+    ap.add_argument("--pass", dest="which", choices=("fwd", "bwd", "module", "module_bwd"),
+                    default="fwd",
+                    help="time the forward (default, the headline), the backward pass, or the "
+                         "whole module forward / backward (projections + attention)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -762,8 +804,8 @@ def main(argv=None):
         return run_reference(args, world, rank)
     if args.which == "bwd":
         return run_ours_bwd(args, world, rank, local)
-    if args.which == "module":
-        return run_ours_module(args, world, rank, local)
+    if args.which in ("module", "module_bwd"):
+        return run_ours_module(args, world, rank, local, backward=args.which == "module_bwd")
     return run_ours(args, world, rank, local)
 
 
