@@ -227,24 +227,31 @@ __global__ void pair_order_kernel(const int32_t *row_ptr, const int32_t *col_idx
     for (int r = threadIdx.x; r < npairs; r += blockDim.x) ord[r] = r;
     return;
   }
-  for (int pr = threadIdx.x; pr < npairs; pr += blockDim.x) {
+  // one warp per pair: |A u B| = |A| + |B| - |A n B|, the lanes looking
+  // A's entries up in B (sorted) by binary search
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int pr = warp; pr < npairs; pr += nwarps) {
     const int qa = 2 * pr;
-    int ia = min(max(rp[qa], 0), nnz), ea = min(max(rp[qa + 1], 0), nnz);
+    const int ia = min(max(rp[qa], 0), nnz), ea = max(ia, min(max(rp[qa + 1], 0), nnz));
     int ib = 0, eb = 0;
     if (qa + 1 < nqb) {
       ib = min(max(rp[qa + 1], 0), nnz);
-      eb = min(max(rp[qa + 2], 0), nnz);
+      eb = max(ib, min(max(rp[qa + 2], 0), nnz));
     }
-    int u = 0;
-    while (ia < ea || ib < eb) {  // merge the two sorted rows
-      const int va = ia < ea ? col_idx[ia] : INT_MAX;
-      const int vb = ib < eb ? col_idx[ib] : INT_MAX;
-      const int m = min(va, vb);
-      ia += va == m;
-      ib += vb == m;
-      ++u;
+    int common = 0;
+    for (int e = ia + lane; e < ea; e += 32) {
+      const int v = col_idx[e];
+      int lo = ib, hi = eb;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (col_idx[mid] < v) lo = mid + 1;
+        else hi = mid;
+      }
+      common += (lo < eb && col_idx[lo] == v) ? 1 : 0;
     }
-    cost[pr] = u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) common += __shfl_xor_sync(0xffffffffu, common, o);
+    if (lane == 0) cost[pr] = (ea - ia) + (eb - ib) - common;
   }
   __syncthreads();
   for (int r = threadIdx.x; r < npairs; r += blockDim.x) {
