@@ -91,6 +91,8 @@ struct UnionWalker {
   }
 };
 
+constexpr int kItemN = 4;  // work items in flight between the producer and the consumers
+
 struct PairItem {
   int bh, qa, a0, lenA, b0, lenB;  // tile B absent (lenB = 0) past the last block
 };
@@ -178,6 +180,12 @@ __global__ void __launch_bounds__(320, 1)
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   __shared__ uint32_t plan_ring[kPlanN];
+  // Work items are taken from a global counter by the producer, in the work
+  // order, and handed to the MMA issuer and the softmax warps through this
+  // ring (a longest-first order served dynamically keeps the CTAs' finishing
+  // times within about one item of each other).
+  __shared__ int item_ring[kItemN];
+  __shared__ __align__(8) uint64_t bar_item_full[kItemN], bar_item_empty[kItemN];
 
   const uint32_t raw = smem_addr(dsmem);
   uint8_t *base = dsmem + (((raw + 1023u) & ~1023u) - raw);
@@ -202,6 +210,10 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&bar_p_full[t], 128);
       mbar_init(&bar_o_final[t], 1);
       mbar_init(&bar_o_empty[t], 128);
+    }
+    for (int i = 0; i < kItemN; ++i) {
+      mbar_init(&bar_item_full[i], 1);
+      mbar_init(&bar_item_empty[i], 9);  // the MMA lane and one lane per softmax warp
     }
     abort_flag = 0;
     fence_barrier_init();
@@ -232,9 +244,14 @@ __global__ void __launch_bounds__(320, 1)
       int skipped_ring = -1;
       bool ok = true;
       for (int k = 0; ok; ++k) {
-        const int idx = snake_item(k, p.total_items);
-        if (idx == -2) break;
-        if (idx < 0) continue;
+        const int slot = k % kItemN;
+        if (!(ok = lane_wait(&bar_item_empty[slot], ((k / kItemN) & 1) ^ 1, wc, kBarItem, k)))
+          break;
+        int idx = atomicAdd(p.item_counter, 1);
+        if (idx >= p.total_items) idx = -1;
+        item_ring[slot] = idx;
+        mbar_arrive(&bar_item_full[slot]);
+        if (idx < 0) break;
         const PairItem it = decode_pair(idx, p, npairs);
         if (it.lenA == 0 && it.lenB == 0) continue;
         if (!(ok = lane_wait(&bar_q_empty, (qcount & 1u) ^ 1u, wc, kBarQEmpty, qcount))) break;
@@ -328,9 +345,11 @@ __global__ void __launch_bounds__(320, 1)
       uint32_t items_t[2] = {0u, 0u};  // items in which the tile had blocks
       bool ok = true;
       for (int k = 0; ok; ++k) {
-        const int idx = snake_item(k, p.total_items);
-        if (idx == -2) break;
-        if (idx < 0) continue;
+        const int slot = k % kItemN;
+        if (!(ok = lane_wait(&bar_item_full[slot], (k / kItemN) & 1, wc, kBarItem, k))) break;
+        const int idx = *static_cast<volatile int *>(&item_ring[slot]);
+        mbar_arrive(&bar_item_empty[slot]);
+        if (idx < 0) break;
         const PairItem it = decode_pair(idx, p, npairs);
         if (it.lenA == 0 && it.lenB == 0) continue;
         if (!(ok = lane_wait(&bar_q_full, qcount & 1u, wc, kBarQFull, qcount))) break;
@@ -454,9 +473,12 @@ __global__ void __launch_bounds__(320, 1)
     uint32_t scnt = 0, icnt = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int idx = snake_item(k, p.total_items);
-      if (idx == -2) break;
-      if (idx < 0) continue;
+      const int slot = k % kItemN;
+      if (!(ok = warp_wait(&bar_item_full[slot], (k / kItemN) & 1, wc, kBarItem, k))) break;
+      const int idx = *static_cast<volatile int *>(&item_ring[slot]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_item_empty[slot]);
+      if (idx < 0) break;
       const PairItem it = decode_pair(idx, p, npairs);
       const int qb = it.qa + t;
       if (qb >= p.nqb) continue;

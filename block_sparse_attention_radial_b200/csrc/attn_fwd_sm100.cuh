@@ -39,6 +39,7 @@ namespace bsa {
 
 struct FwdParams {
   const int32_t *row_ptr, *col_idx, *order;
+  int32_t *item_counter;  // next work item (two-tile kernel); zeroed by the work-order kernel
   __nv_bfloat16 *out;
   // element strides of out's batch, head and token axes (head_dim contiguous)
   long long o_sb, o_sh, o_sn;
@@ -85,7 +86,7 @@ struct FwdCfg {
 enum : int { kRoleProducer = 1, kRoleMma = 2, kRoleSoftmax = 3 };
 enum : int {
   kBarKvFull = 1, kBarKvEmpty, kBarQFull, kBarQEmpty, kBarSFull, kBarPFull, kBarODone,
-  kBarOEmpty, kBarFinal, kBarSFree, kBarPlan
+  kBarOEmpty, kBarFinal, kBarSFree, kBarPlan, kBarItem
 };
 
 struct WaitCtx {

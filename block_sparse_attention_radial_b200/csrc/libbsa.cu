@@ -91,41 +91,16 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [batch*heads, n, D] bf16 viewed as a 4-D tensor {64 columns, n rows,
-// D/64 column halves, batch*heads}: one box {64, rows, D/64, 1} brings a whole
-// rows x D tile with 128-byte swizzling, laid out in shared memory as D/64
-// consecutive [rows][64] blocks (the K-major layout the MMA descriptors use).
-// One large box per tile instead of one per 64 columns: the TMA unit's cost is
-// mostly per box. Rows past n read as zeros.
-int make_map(CUtensorMap *map, const void *ptr, int bh, int n, int D, int rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) {
-    std::snprintf(t_last_error, sizeof(t_last_error), "cuTensorMapEncodeTiled not available");
-    return BSA_ERR_CUDA;
-  }
-  cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(n), static_cast<cuuint64_t>(D / 64),
-                        static_cast<cuuint64_t>(bh)};
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, 128,
-                           static_cast<cuuint64_t>(n) * static_cast<cuuint64_t>(D) * 2};
-  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(rows), static_cast<cuuint32_t>(D / 64), 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims,
-                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) {
-    std::snprintf(t_last_error, sizeof(t_last_error), "cuTensorMapEncodeTiled failed (%d)",
-                  static_cast<int>(r));
-    return BSA_ERR_CUDA;
-  }
-  return BSA_OK;
-}
-
 // A [batch, heads, n, D] bf16 view with arbitrary batch / head / token strides
 // (elements; D contiguous) as a 5-D tensor {64 columns, n rows, D/64 column
-// halves, heads, batch}: the same {64, rows, D/64} box as make_map, with the
-// head and batch coordinates kept apart so that token-major layouts (the
-// [batch, n, heads, D] output of a fused projection) load without a
-// transpose. An axis of extent 1 gets a placeholder stride (never used).
+// halves, heads, batch}. One box {64, rows, D/64, 1, 1} brings a whole
+// rows x D tile with 128-byte swizzling, laid out in shared memory as D/64
+// consecutive [rows][64] blocks (the K-major layout the MMA descriptors use):
+// one large box per tile, since the TMA unit's cost is mostly per box. Rows
+// past n read as zeros. Head and batch stay separate coordinates, so
+// token-major layouts (the [batch, n, heads, D] output of a fused projection)
+// load without a transpose. An axis of extent 1 gets a placeholder stride
+// (never used).
 int make_map_strided(CUtensorMap *map, const void *ptr, const bsa_layout &L, int batch,
                      int heads, int n, int D, int rows) {
   EncodeTiledFn fn = encode_fn();
@@ -291,9 +266,12 @@ bool views_disjoint(const void *a, const bsa_layout &La, const void *b, const bs
   return r >= foot && sn - r >= foot;
 }
 
-size_t order_bytes(const bsa_block_lists *l) {
+// Forward scratch: the work order, then (256 bytes on) the work counter.
+size_t order_only_bytes(const bsa_block_lists *l) {
   return (static_cast<size_t>(l->num_lists) * l->num_q_blocks * sizeof(int32_t) + 255) & ~size_t(255);
 }
+
+size_t order_bytes(const bsa_block_lists *l) { return order_only_bytes(l) + 256; }
 
 constexpr int kLptMaxRows = 12288;  // rows whose costs fit in 48 KB of shared memory
 
@@ -379,7 +357,8 @@ int launch_pair(const QkvViews &x, int32_t n, const FwdParams &p, DeviceInfo *de
 // the one-tile kernel. Arguments were checked by the caller.
 int run_fwd(const QkvViews &x, int32_t n, int32_t head_dim, float softmax_scale,
             const bsa_block_lists *l, void *out, const bsa_layout &lo, float *lse,
-            int32_t *order, DeviceInfo *dev, int fault_flags, cudaStream_t stream) {
+            int32_t *order, int32_t *item_counter, DeviceInfo *dev, int fault_flags,
+            cudaStream_t stream) {
   const int batch = x.batch, heads = x.heads;
   const int nqb = l->num_q_blocks;
   bool pair;
@@ -391,7 +370,7 @@ int run_fwd(const QkvViews &x, int32_t n, int32_t head_dim, float softmax_scale,
     const int npairs = (nqb + 1) / 2;
     const size_t smem = static_cast<size_t>(npairs <= kLptMaxRows ? npairs : 0) * sizeof(int);
     pair_order_kernel<<<l->num_lists, 1024, smem, stream>>>(l->row_ptr, l->col_idx, nqb, l->nnz,
-                                                           order, kLptMaxRows);
+                                                           order, kLptMaxRows, item_counter);
   } else {
     const size_t smem = static_cast<size_t>(nqb <= kLptMaxRows ? nqb : 0) * sizeof(int);
     lpt_order_kernel<<<l->num_lists, 1024, smem, stream>>>(l->row_ptr, nqb, l->nnz, order,
@@ -403,6 +382,7 @@ int run_fwd(const QkvViews &x, int32_t n, int32_t head_dim, float softmax_scale,
   p.row_ptr = l->row_ptr;
   p.col_idx = l->col_idx;
   p.order = order;
+  p.item_counter = item_counter;
   p.out = static_cast<__nv_bfloat16 *>(out);
   p.o_sb = lo.batch_stride;
   p.o_sh = lo.head_stride;
@@ -728,9 +708,12 @@ int bsa_attn_fwd(const void *q, const void *k, const void *v, int32_t batch, int
     fault_flags = g_fault_flags;
     g_fault_flags = 0;
   }
+  int32_t *order = static_cast<int32_t *>(workspace);
+  int32_t *counter = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) +
+                                                 order_only_bytes(l));
   return run_fwd(contiguous_views(q, k, v, batch, heads, n, head_dim), n, head_dim,
-                 softmax_scale, l, out, contiguous_layout(heads, n, head_dim), lse,
-                 static_cast<int32_t *>(workspace), dev, fault_flags, stream);
+                 softmax_scale, l, out, contiguous_layout(heads, n, head_dim), lse, order,
+                 counter, dev, fault_flags, stream);
 }
 
 int bsa_attn_fwd_strided(const void *q, const bsa_layout *q_layout, const void *k,
@@ -764,8 +747,11 @@ int bsa_attn_fwd_strided(const void *q, const bsa_layout *q_layout, const void *
   x.lv = *v_layout;
   x.batch = batch;
   x.heads = heads;
-  return run_fwd(x, n, head_dim, softmax_scale, l, out, *out_layout, lse,
-                 static_cast<int32_t *>(workspace), dev, fault_flags, stream);
+  int32_t *order = static_cast<int32_t *>(workspace);
+  int32_t *counter = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) +
+                                                 order_only_bytes(l));
+  return run_fwd(x, n, head_dim, softmax_scale, l, out, *out_layout, lse, order, counter, dev,
+                 fault_flags, stream);
 }
 
 int bsa_attn_bwd_strided(const void *q, const bsa_layout *q_layout, const void *k,
@@ -1025,13 +1011,13 @@ int bsa_set_test_hooks(int64_t wait_limit_ns, int32_t fault_flags) {
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
-// Allocation-free entry point. Its scratch (the work order) is this fixed
-// array instead of a caller-provided workspace. In host code `g_noalloc_order`
+// Allocation-free entry point. Its scratch (the work order, then the work
+// counter) is this fixed array instead of a caller-provided workspace. In host code `g_noalloc_order`
 // names a host-side stand-in, not device memory, so the device address is
 // resolved once per device with cudaGetSymbolAddress and cached.
 // ---------------------------------------------------------------------------
 
-static __device__ __align__(256) int32_t g_noalloc_order[BSA_NOALLOC_MAX_ORDER_ENTRIES];
+static __device__ __align__(256) int32_t g_noalloc_order[BSA_NOALLOC_MAX_ORDER_ENTRIES + 64];
 
 namespace bsa {
 namespace {
@@ -1072,6 +1058,6 @@ extern "C" int bsa_attn_fwd_noalloc(const void *q, const void *k, const void *v,
   if ((st = noalloc_scratch(&order)) != BSA_OK) return st;
 
   return run_fwd(contiguous_views(q, k, v, batch, heads, n, head_dim), n, head_dim,
-                 softmax_scale, l, out, contiguous_layout(heads, n, head_dim), lse, order, dev, 0,
-                 stream);
+                 softmax_scale, l, out, contiguous_layout(heads, n, head_dim), lse, order,
+                 order + BSA_NOALLOC_MAX_ORDER_ENTRIES, dev, 0, stream);
 }

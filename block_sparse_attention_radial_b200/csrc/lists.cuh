@@ -216,9 +216,13 @@ __global__ void lpt_order_kernel(const int32_t *row_ptr, int nqb, int nnz, int32
 // One CTA per list: order[list * npairs + rank] = query-block pair (2p, 2p+1)
 // with the rank-th longest union of key blocks (ties: lower pair first).
 // Lists whose pair count does not fit in shared memory keep natural order.
+// Also zeroes `item_counter`, the attention kernel's work counter (this
+// kernel runs before it in stream order).
 __global__ void pair_order_kernel(const int32_t *row_ptr, const int32_t *col_idx, int nqb,
-                                  int nnz, int32_t *order, int max_smem_rows) {
+                                  int nnz, int32_t *order, int max_smem_rows,
+                                  int32_t *item_counter) {
   extern __shared__ int cost[];
+  if (blockIdx.x == 0 && threadIdx.x == 0) *item_counter = 0;
   const int list = blockIdx.x;
   const int npairs = (nqb + 1) / 2;
   const int32_t *rp = row_ptr + static_cast<long long>(list) * nqb;

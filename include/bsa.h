@@ -130,7 +130,8 @@ int bsa_joint_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t text_
 
 /*
  * Bytes of device scratch memory bsa_attn_fwd needs for this problem (the
- * longest-row-first work order of every list). Returns 0 for invalid lists.
+ * longest-row-first work order of every list and a work counter the kernel's
+ * CTAs take items from). Returns 0 for invalid lists.
  */
 size_t bsa_attn_fwd_workspace_bytes(int32_t batch, int32_t heads, const bsa_block_lists *lists);
 
@@ -451,8 +452,9 @@ int bsa_selftest_exp2(const float *x, float *y_poly, float *y_mufu, float *y_ref
  *
  * Same operation, arguments and results as bsa_attn_fwd, minus the workspace:
  * the scratch it needs (the longest-row-first work order, one int32 per query
- * block per list) lives in a fixed array compiled into the library, of
- * BSA_NOALLOC_MAX_ORDER_ENTRIES int32 entries (256 KiB). Every GPU that loads
+ * block per list, and the work counter) lives in a fixed array compiled into
+ * the library, of BSA_NOALLOC_MAX_ORDER_ENTRIES + 64 int32 entries (256 KiB +
+ * 256 B). Every GPU that loads
  * the library holds that array until the process exits.
  *
  * - Returns BSA_ERR_SCRATCH_LIMIT, launching nothing, when

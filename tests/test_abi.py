@@ -55,10 +55,12 @@ def test_status_strings(lib):
 def test_workspace_bytes(lib):
     from block_sparse_attention_radial_b200._lib import BlockListsC
 
+    # the work order (one int per query block and list, 256-byte aligned) and
+    # 256 bytes for the work counter
     ls = BlockListsC(1, 256, 256, 128, 1000, 0, 0)
-    assert lib.bsa_attn_fwd_workspace_bytes(1, 40, ctypes.byref(ls)) == 1024
+    assert lib.bsa_attn_fwd_workspace_bytes(1, 40, ctypes.byref(ls)) == 1024 + 256
     ls = BlockListsC(24, 256, 256, 128, 1000, 0, 0)
-    assert lib.bsa_attn_fwd_workspace_bytes(1, 24, ctypes.byref(ls)) == 24 * 256 * 4
+    assert lib.bsa_attn_fwd_workspace_bytes(1, 24, ctypes.byref(ls)) == 24 * 256 * 4 + 256
     ls = BlockListsC(3, 256, 256, 128, 1000, 0, 0)   # neither 1 nor heads
     assert lib.bsa_attn_fwd_workspace_bytes(1, 24, ctypes.byref(ls)) == 0
 
@@ -171,9 +173,9 @@ def test_module_workspace_and_host_checks(lib):
 
     vp, ref = ctypes.c_void_p, ctypes.byref
     ls = BlockListsC(1, 256, 256, 128, 1000, 0, 0)
-    # work order (1 KiB) + q/k/v [32760, 15360] + attention out [32760, 5120] bf16
-    # + lse [40, 32760] fp32 + 32 MiB
-    expect = 1024 + 32760 * 15360 * 2 + 32760 * 5120 * 2 + 40 * 32760 * 4 + (32 << 20)
+    # work order and counter (1 KiB + 256) + q/k/v [32760, 15360] + attention out
+    # [32760, 5120] bf16 + lse [40, 32760] fp32 + 32 MiB
+    expect = 1280 + 32760 * 15360 * 2 + 32760 * 5120 * 2 + 40 * 32760 * 4 + (32 << 20)
     assert lib.bsa_attn_module_workspace_bytes(1, 32760, 40, 128, ref(ls)) == expect
     # backward: dA [32760, 5120] + dQKV [32760, 15360] bf16 + the attention
     # backward's workspace + 32 x 15360 fp32 partial sums + 32 MiB
