@@ -55,11 +55,13 @@ struct BwdParams {
   const uint8_t *rmask, *cmask;
   int32_t heads, n, nqb, nkb, num_lists, nnz;  // heads: per batch item
   int32_t total_items;
+  int32_t *item_counter;  // next work item; zeroed by bwd_prep_kernel
   float scale, scale_log2;
   unsigned long long wait_limit_ns;
 };
 
 constexpr int kBwdBlock = 128;
+constexpr int kBwdItemN = 4;  // work items in flight between the producer and the consumers
 
 // ------------------------------------------------------------------ prep --
 
@@ -70,8 +72,9 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16 *out, const __nv_bfloat16 *d
                                 const float *lse, float *lse2, float *delta, int n, int nqb,
                                 int heads, long long o_sb, long long o_sh, long long o_sn,
                                 long long d_sb, long long d_sh, long long d_sn,
-                                long long rows_total) {
+                                long long rows_total, int32_t *item_counters) {
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx < 2) item_counters[idx] = 0;  // the dK/dV and the dQ kernel's work counters
   if (idx >= rows_total) return;
   const long long padded = static_cast<long long>(nqb) * kBwdBlock;
   const long long bh = idx / padded;
@@ -299,6 +302,11 @@ __global__ void __launch_bounds__(192, 1)
   __shared__ __align__(8) uint64_t bar_acc_full, bar_acc_empty, bar_final;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
+  // work items from the global counter (natural order, served dynamically):
+  // the producer takes them and hands them to the MMA issuer and the four
+  // elementwise warps
+  __shared__ int item_ring[kBwdItemN];
+  __shared__ __align__(8) uint64_t bar_item_full[kBwdItemN], bar_item_empty[kBwdItemN];
 
   const uint32_t raw = smem_addr(dsmem);
   uint8_t *base = dsmem + (((raw + 1023u) & ~1023u) - raw);
@@ -326,6 +334,10 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(&bar_acc_full, 1);
     mbar_init(&bar_acc_empty, 128);
     mbar_init(&bar_final, 1);
+    for (int i = 0; i < kBwdItemN; ++i) {
+      mbar_init(&bar_item_full[i], 1);
+      mbar_init(&bar_item_empty[i], 5);  // the MMA lane and one lane per elementwise warp
+    }
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -364,9 +376,14 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t ring = 0, kvcount = 0;
       bool ok = true;
       for (int k = 0; ok; ++k) {
-        const int idx = snake_item(k, p.total_items);
-        if (idx == -2) break;
-        if (idx < 0) continue;
+        const int slot = k % kBwdItemN;
+        if (!(ok = lane_wait(&bar_item_empty[slot], ((k / kBwdItemN) & 1) ^ 1, wc, kBarItem, k)))
+          break;
+        int idx = atomicAdd(p.item_counter, 1);
+        if (idx >= p.total_items) idx = -1;
+        item_ring[slot] = idx;
+        mbar_arrive(&bar_item_full[slot]);
+        if (idx < 0) break;
         const BwdItem it = decode(idx);
         if (it.len == 0) continue;
         if (!(ok = lane_wait(&bar_kv_empty, (kvcount & 1u) ^ 1u, wc, kBarQEmpty, kvcount))) break;
@@ -449,9 +466,11 @@ __global__ void __launch_bounds__(192, 1)
         mma_commit(&bar_dp_full);
       };
       for (int k = 0; ok; ++k) {
-        const int idx = snake_item(k, p.total_items);
-        if (idx == -2) break;
-        if (idx < 0) continue;
+        const int slot = k % kBwdItemN;
+        if (!(ok = lane_wait(&bar_item_full[slot], (k / kBwdItemN) & 1, wc, kBarItem, k))) break;
+        const int idx = *static_cast<volatile int *>(&item_ring[slot]);
+        mbar_arrive(&bar_item_empty[slot]);
+        if (idx < 0) break;
         const BwdItem it = decode(idx);
         if (it.len == 0) continue;
         if (!(ok = lane_wait(&bar_kv_full, kvcount & 1u, wc, kBarQFull, kvcount))) break;
@@ -518,9 +537,12 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t ring = 0, scount = 0, dcount = 0, acount = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int idx = snake_item(k, p.total_items);
-      if (idx == -2) break;
-      if (idx < 0) continue;
+      const int slot = k % kBwdItemN;
+      if (!(ok = warp_wait(&bar_item_full[slot], (k / kBwdItemN) & 1, wc, kBarItem, k))) break;
+      const int idx = *static_cast<volatile int *>(&item_ring[slot]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_item_empty[slot]);
+      if (idx < 0) break;
       const BwdItem it = decode(idx);
       const int key = it.blk * BN + r;
       const bool store = key < p.n;
@@ -691,6 +713,11 @@ __global__ void __launch_bounds__(192, 1)
   __shared__ __align__(8) uint64_t bar_acc_full, bar_acc_empty, bar_final;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
+  // work items from the global counter (natural order, served dynamically):
+  // the producer takes them and hands them to the MMA issuer and the four
+  // elementwise warps
+  __shared__ int item_ring[kBwdItemN];
+  __shared__ __align__(8) uint64_t bar_item_full[kBwdItemN], bar_item_empty[kBwdItemN];
 
   const uint32_t raw = smem_addr(dsmem);
   uint8_t *base = dsmem + (((raw + 1023u) & ~1023u) - raw);
@@ -716,6 +743,10 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(&bar_acc_full, 1);
     mbar_init(&bar_acc_empty, 128);
     mbar_init(&bar_final, 1);
+    for (int i = 0; i < kBwdItemN; ++i) {
+      mbar_init(&bar_item_full[i], 1);
+      mbar_init(&bar_item_empty[i], 5);  // the MMA lane and one lane per elementwise warp
+    }
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -752,9 +783,14 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t ring = 0, qdcount = 0;
       bool ok = true;
       for (int k = 0; ok; ++k) {
-        const int idx = snake_item(k, p.total_items);
-        if (idx == -2) break;
-        if (idx < 0) continue;
+        const int slot = k % kBwdItemN;
+        if (!(ok = lane_wait(&bar_item_empty[slot], ((k / kBwdItemN) & 1) ^ 1, wc, kBarItem, k)))
+          break;
+        int idx = atomicAdd(p.item_counter, 1);
+        if (idx >= p.total_items) idx = -1;
+        item_ring[slot] = idx;
+        mbar_arrive(&bar_item_full[slot]);
+        if (idx < 0) break;
         const BwdItem it = decode(idx);
         if (it.len == 0) continue;
         if (!(ok = lane_wait(&bar_qd_empty, (qdcount & 1u) ^ 1u, wc, kBarQEmpty, qdcount))) break;
@@ -834,9 +870,11 @@ __global__ void __launch_bounds__(192, 1)
         mma_commit(&bar_dp_full);
       };
       for (int k = 0; ok; ++k) {
-        const int idx = snake_item(k, p.total_items);
-        if (idx == -2) break;
-        if (idx < 0) continue;
+        const int slot = k % kBwdItemN;
+        if (!(ok = lane_wait(&bar_item_full[slot], (k / kBwdItemN) & 1, wc, kBarItem, k))) break;
+        const int idx = *static_cast<volatile int *>(&item_ring[slot]);
+        mbar_arrive(&bar_item_empty[slot]);
+        if (idx < 0) break;
         const BwdItem it = decode(idx);
         if (it.len == 0) continue;
         if (!(ok = lane_wait(&bar_qd_full, qdcount & 1u, wc, kBarQFull, qdcount))) break;
@@ -891,9 +929,12 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t scount[2] = {0u, 0u}, dcount = 0, acount = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int idx = snake_item(k, p.total_items);
-      if (idx == -2) break;
-      if (idx < 0) continue;
+      const int slot = k % kBwdItemN;
+      if (!(ok = warp_wait(&bar_item_full[slot], (k / kBwdItemN) & 1, wc, kBarItem, k))) break;
+      const int idx = *static_cast<volatile int *>(&item_ring[slot]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_item_empty[slot]);
+      if (idx < 0) break;
       const BwdItem it = decode(idx);
       const int row = it.blk * BN + r;
       const bool store = row < p.n;

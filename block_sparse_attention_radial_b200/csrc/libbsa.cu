@@ -434,7 +434,7 @@ QkvViews contiguous_views(const void *q, const void *k, const void *v, int batch
 // Offsets are 256-byte aligned (the bulk copies of lse2 / delta rows need
 // 16-byte aligned 512-byte rows).
 struct BwdLayout {
-  size_t lse2, delta, col_ptr, row_idx, cmask, tile_ptr, tile_col, tile_mask, total;
+  size_t lse2, delta, counters, col_ptr, row_idx, cmask, tile_ptr, tile_col, tile_mask, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -447,7 +447,8 @@ BwdLayout bwd_layout(int32_t batch, int32_t heads, int32_t n, const bsa_block_li
   const size_t entries = static_cast<size_t>(l->nnz > 0 ? l->nnz : 1);
   w.lse2 = 0;
   w.delta = align256(rows * sizeof(float));
-  w.col_ptr = w.delta + align256(rows * sizeof(float));
+  w.counters = w.delta + align256(rows * sizeof(float));  // the two kernels' work counters
+  w.col_ptr = w.counters + 256;
   w.row_idx = w.col_ptr + align256(ptrs);
   w.cmask = w.tile_ptr = w.tile_col = w.tile_mask = w.total =
       w.row_idx + align256(entries * sizeof(int32_t));
@@ -513,7 +514,8 @@ int launch_bwd(const BwdViews &x, const float *lse, int32_t n, float softmax_sca
   bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 255) / 256), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16 *>(x.out), static_cast<const __nv_bfloat16 *>(x.dout), lse,
       lse2, delta, n, nqb, x.heads, x.lo.batch_stride, x.lo.head_stride, x.lo.token_stride,
-      x.ldo.batch_stride, x.ldo.head_stride, x.ldo.token_stride, rows);
+      x.ldo.batch_stride, x.ldo.head_stride, x.ldo.token_stride, rows,
+      reinterpret_cast<int32_t *>(ws + w.counters));
   BSA_CUDA(cudaGetLastError());
   const int cols = l->num_lists * nkb;
   csc_count_kernel<<<cols, 256, 0, stream>>>(l->row_ptr, l->col_idx, nqb, nkb, l->nnz, col_ptr);
@@ -589,7 +591,9 @@ int launch_bwd(const BwdViews &x, const float *lse, int32_t n, float softmax_sca
     std::lock_guard<std::mutex> lk(g_hook_mu);
     p.wait_limit_ns = g_wait_limit_ns;
   }
+  int32_t *counters = reinterpret_cast<int32_t *>(ws + w.counters);
   p.total_items = bh * nkb;
+  p.item_counter = counters;
   int grid = p.total_items < dev->sms ? p.total_items : dev->sms;
   if (masked)
     attn_bwd_dkdv_kernel<D, true><<<grid, DkdvCfg<D>::THREADS, DkdvCfg<D>::DSMEM, stream>>>(
@@ -599,6 +603,7 @@ int launch_bwd(const BwdViews &x, const float *lse, int32_t n, float softmax_sca
         tq, tk, tv, td, p);
   BSA_CUDA(cudaGetLastError());
   p.total_items = bh * nqb;
+  p.item_counter = counters + 1;
   grid = p.total_items < dev->sms ? p.total_items : dev->sms;
   if (masked)
     attn_bwd_dq_kernel<D, true><<<grid, DqCfg<D>::THREADS, DqCfg<D>::DSMEM, stream>>>(tq, tk, tv,

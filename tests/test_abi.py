@@ -106,8 +106,9 @@ def test_backward_workspace_and_host_checks(lib):
     from block_sparse_attention_radial_b200._lib import BlockListsC
 
     ls = BlockListsC(1, 256, 256, 128, 1000, 0, 0)
-    # lse2 + delta: 2 x 40 x 256 x 128 floats; offsets 257 ints; 1000 entries
-    expect = 2 * 40 * 256 * 128 * 4 + 1280 + 4096
+    # lse2 + delta: 2 x 40 x 256 x 128 floats; 256 bytes of work counters;
+    # offsets 257 ints; 1000 entries
+    expect = 2 * 40 * 256 * 128 * 4 + 256 + 1280 + 4096
     assert lib.bsa_attn_bwd_workspace_bytes(1, 40, 32760, ctypes.byref(ls)) == expect
     assert lib.bsa_attn_bwd_workspace_bytes(1, 40, 32769, ctypes.byref(ls)) == 0  # nqb mismatch
     # block 64: the same plus masks of the transposed entries and the 128-row tile lists
