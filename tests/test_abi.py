@@ -226,3 +226,28 @@ def test_strided_backward_host_checks(lib):
     assert call(ldv=LayoutC(n * 3 * C, D, 3 * C + 8)) == 1  # different layout, shared span
     assert call(dq=qkv) == 1                              # dq on top of the inputs
     assert call(ldq=LayoutC(n * 3 * C, 8, 3 * C)) == 1   # dq's own rows overlap
+
+
+def test_host_buffer_forward_host_checks(lib):
+    """bsa_attn_fwd_host: workspace size formula and argument checks on the
+    host (all rejected before any CUDA call)."""
+    from block_sparse_attention_radial_b200._lib import BlockListsC
+
+    vp, ref = ctypes.c_void_p, ctypes.byref
+    ls = BlockListsC(1, 256, 256, 128, 1000, 0, 0)
+    t = 1 * 40 * 32760 * 128 * 2
+    # attention scratch (order + counter) + q, k, v, out (bf16) + lse (fp32)
+    expect = 1280 + 4 * t + 40 * 32760 * 4
+    assert lib.bsa_attn_fwd_host_workspace_bytes(1, 40, 32760, 128, ref(ls)) == expect
+    small = BlockListsC(1, 8, 8, 128, 10, 1 << 22, 1 << 23)
+    ws = lib.bsa_attn_fwd_host_workspace_bytes(1, 2, 1000, 64, ref(small))
+    h = vp(1 << 20)
+
+    def call(q=h, hd=64, w=vp(1 << 32), wsb=ws):
+        return lib.bsa_attn_fwd_host(q, h, h, 1, 2, 1000, hd, 0.0, ref(small), h, None, w, wsb,
+                                     None)
+
+    assert call(q=vp(0)) == 1                       # null input
+    assert call(hd=96) == 2                         # head_dim
+    assert call(wsb=ws - 1) == 1                    # workspace too small
+    assert call(w=vp((1 << 32) + 16)) == 1          # workspace not 256-byte aligned
