@@ -526,30 +526,78 @@ __global__ void __launch_bounds__(320, 1)
           for (int c = 0; c < BN; ++c)
             if (c >= valid) s[c] = -INFINITY;
         }
-        float m8[8];
+        auto row_max = [&]() {
+          float m8[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = fmaxf(s[i], s[i + 8]);
+          for (int i = 0; i < 8; ++i) m8[i] = fmaxf(s[i], s[i + 8]);
 #pragma unroll
-        for (int c = 16; c < BN; c += 16) {
+          for (int c = 16; c < BN; c += 16) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) m8[i] = fmax3(m8[i], s[c + i], s[c + 8 + i]);
-        }
-        const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
-                               fmaxf(m8[6], m8[7]));
-        const float mblk = mx * sl2;
+            for (int i = 0; i < 8; ++i) m8[i] = fmax3(m8[i], s[c + i], s[c + 8 + i]);
+          }
+          return fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                       fmaxf(m8[6], m8[7]));
+        };
+        uint32_t pk[BN / 2];
+        auto exp_row = [&]() {
+          return valid < BN ? exp2_pack_row<BN, 0>(s, sl2, -m_ref, pk)
+                            : exp2_pack_row<BN, kEmuPairsPer8>(s, sl2, -m_ref, pk);
+        };
         float alpha = 1.f;
         bool rescale = false;
+        float sum;
         if (j == 0) {
-          m_ref = mblk;
-        } else if (mblk > m_ref + 8.f) {
-          // lazy rescale (the final O / l is exact either way)
-          alpha = ex2_approx(m_ref - mblk);
-          m_ref = mblk;
-          rescale = true;
+          m_ref = row_max() * sl2;
+          sum = exp_row();
+        } else {
+          // The reference stays the first block's maximum: P may exceed 1 by
+          // far (bf16 keeps its relative precision and the fp32 sums stay
+          // finite), so the row maximum is only taken again when the row sum
+          // leaves [0, 2^64]; then O and l are rescaled (the final O / l and
+          // lse are exact either way).
+          sum = exp_row();
+          // Warp-uniform: the TMEM reads below are warp-collective
+          // (.sync.aligned), so when any row of the warp needs the rescale
+          // every lane takes this path (a rescale is valid for any row).
+          if (__any_sync(0xffffffffu, !(sum <= 0x1p64f))) {
+            // S is still in TMEM (P has not been stored over it yet): take the
+            // row maximum from it, then recompute P 32 columns at a time, so
+            // that no more than one chunk of scores is live next to P
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c) {
+              uint32_t sr[32];
+              tmem_ld32(s_tmem + c * 32, sr);
+              tmem_wait_ld();
+              reg_fence32(sr);
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (c * 32 + i < valid) mx = fmaxf(mx, __uint_as_float(sr[i]));
+            }
+            const float m_new = fmaxf(m_ref, mx * sl2);
+            alpha = ex2_approx(m_ref - m_new);
+            m_ref = m_new;
+            rescale = true;
+            float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c) {
+              uint32_t sr[32];
+              tmem_ld32(s_tmem + c * 32, sr);
+              tmem_wait_ld();
+              reg_fence32(sr);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int col = c * 32 + 2 * i;
+                const float a = col < valid ? ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -m_ref)) : 0.f;
+                const float b = col + 1 < valid ? ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -m_ref)) : 0.f;
+                acc.x += a;
+                acc.y += b;
+                pk[c * 16 + i] = pack_bf16x2(a, b);
+              }
+            }
+            sum = acc.x + acc.y;
+          }
         }
-        uint32_t pk[BN / 2];
-        const float sum = valid < BN ? exp2_pack_row<BN, 0>(s, sl2, -m_ref, pk)
-                                     : exp2_pack_row<BN, kEmuPairsPer8>(s, sl2, -m_ref, pk);
         l = l * alpha + sum;
         // S being complete means QK of this block is complete, and the
         // previous PV of this tile was issued before it: O is settled.

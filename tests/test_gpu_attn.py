@@ -104,6 +104,30 @@ def test_running_max_jumps_trigger_rescale(bsa):
     assert_close(ro, ref_o, rl, ref_l, "fp32 reference vs oracle")
 
 
+@pytest.mark.parametrize("top", [12.0, 40.0])
+def test_running_max_jump_forces_a_rescale(bsa, top):
+    """Scores of later key blocks exceed the first block's maximum by tens of
+    log2 units: with the smaller ramp P grows to about 2^50 against the first
+    block's reference (no rescale needed); with the larger one a row sum
+    leaves [0, 2^64] or overflows to inf, and the kernels take the row
+    maximum again and rescale O and l."""
+    n, D, blk = 1024, 128, 128
+    q, k, v = make_random_qkv(1, 2, n, D, seed=32)
+    ramp = torch.linspace(0.2, top, n).view(1, 1, n, 1)
+    k = (k.float() * ramp).to(torch.bfloat16)
+    # such peaked rows return about one V row each: V at a quarter of unit
+    # scale keeps |out| (and its bf16 rounding) inside the absolute bound
+    v = (v.float() * 0.25).to(torch.bfloat16)
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    nqb = n // blk
+    rp = np.arange(nqb + 1, dtype=np.int32) * nqb
+    ci = np.tile(np.arange(nqb, dtype=np.int32), nqb)
+    lists = bsa.block_lists_from_csr(rp, ci, 1, nqb, blk)
+    out, lse, ro, rl = _run(bsa, q, k, v, lists)
+    ref_o, ref_l = oracle.masked_attention_fp64(q, k, v, rp, ci, 1, blk)
+    assert_close(out, ref_o, lse, ref_l, "tcgen05 vs oracle")
+
+
 def test_explicit_scale_and_no_lse(bsa):
     n, D, blk = 512, 64, 64
     q, k, v = (t.cuda() for t in make_random_qkv(1, 1, n, D, seed=41))
