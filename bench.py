@@ -40,11 +40,22 @@ KERNEL_SOURCES = {
 TRAFFIC_FILES = {"fwd": "attn_fwd_pair_sm100_{}_traffic.json", "bwd": "attn_bwd_sm100_{}_traffic.json"}
 
 
+def _code_only(text: str) -> str:
+    """C++ source without comments and blank lines: what the compiler sees."""
+    import re
+
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_source_hash(which: str = "fwd") -> str:
+    """Hash of the kernels' source code (comments excluded), recorded with an
+    ncu capture so that a changed kernel invalidates its traffic figure."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES[which]:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

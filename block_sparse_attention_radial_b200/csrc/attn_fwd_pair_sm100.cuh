@@ -22,6 +22,13 @@
 //   QK_B(j) if b;  then K(j) and V(j-1) are released.
 // PV_X(prev) is always issued before QK_X(next), so when S_X is complete the
 // previous PV_X is complete too: the softmax can rescale O_X without waiting.
+//
+// Work items come from a global counter, in the longest-first order of
+// pair_order_kernel: the producer takes each index and passes it to the MMA
+// issuer and the softmax warps through a small ring in shared memory.
+// Softmax: the row maximum of an item's first block is the reference for
+// the whole item; later blocks rescale only when a row sum of P leaves
+// [0, 2^64].
 #pragma once
 
 #include <climits>
@@ -37,7 +44,7 @@ template <int D>
 struct PairCfg {
   static constexpr int BN = 128;                 // block = tile rows = MMA M and N
   static constexpr int Q_BYTES = BN * D * 2;     // one tile's Q
-  static constexpr int TILE_BYTES = BN * D * 2;  // one K or V tile (one 4-D TMA box)
+  static constexpr int TILE_BYTES = BN * D * 2;  // one K or V tile (one TMA box)
   static constexpr int NS_FIT = (kSmemLimit - 1024 - 512 - 2 * Q_BYTES) / TILE_BYTES;
   static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
   static constexpr int DSMEM_USED = 1024 + 2 * Q_BYTES + NS * TILE_BYTES;
