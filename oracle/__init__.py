@@ -27,6 +27,8 @@ Modules:
 * ``attention_backward``: its gradients (dQ, dK, dV), in float64.
 * ``module``: the RadialAttention module forward (projections, head split,
   attention, head merge, output projection), in float64.
+* ``tile_patterns``: per-head tile patterns (diagonal and multi-diagonal
+  bands, vertical stripes, dual windows) expanded into block lists.
 """
 
 from .radial_mask import (  # noqa: F401
@@ -54,6 +56,10 @@ from .attention_backward import (  # noqa: F401
     masked_attention_backward_fp64,
     masked_attention_dq_rows,
     masked_attention_dkdv_keys,
+)
+from .tile_patterns import (  # noqa: F401
+    tile_pattern_mask,
+    tile_pattern_lists,
 )
 from .module import (  # noqa: F401
     radial_attention_module_fp64,

@@ -125,21 +125,33 @@ def make_module_inputs(batch, n, heads, head_dim, seed, device="cpu", bias=True)
 # (local band plus an axial stripe) family of the Compact Attention abstract.
 # ----------------------------------------------------------------------------
 
-def _pattern(rng: np.random.Generator, nb: int) -> tuple[str, np.ndarray]:
+def _pattern(rng: np.random.Generator, nb: int) -> tuple[str, np.ndarray, dict]:
+    """One seeded draw: ``(kind, mask, descriptor)``. The descriptor states the
+    same pattern as data (``bands`` of ``kb - qb`` offsets, ``axial`` period
+    and half-width, stripe ``columns``) for the device-side pattern builder."""
     qb = np.arange(nb)[:, None]
     kb = np.arange(nb)[None, :]
     kind = ("dual_window", "diagonal", "multi_diagonal", "stripe_diagonal")[rng.integers(4)]
+    desc = {"bands": [], "axial": None, "columns": []}
     if kind == "diagonal":
         w = int(rng.integers(8, 64))
         m = np.abs(qb - kb) <= w
+        desc["bands"].append((-w, w))
     elif kind == "multi_diagonal":
-        m = np.abs(qb - kb) <= int(rng.integers(1, 4))
+        c = int(rng.integers(1, 4))
+        m = np.abs(qb - kb) <= c
+        desc["bands"].append((-c, c))
         for off in rng.integers(-nb // 2, nb // 2, size=int(rng.integers(3, 9))):
-            m |= np.abs(kb - qb - int(off)) <= int(rng.integers(2, 9))
+            h = int(rng.integers(2, 9))
+            m |= np.abs(kb - qb - int(off)) <= h
+            desc["bands"].append((int(off) - h, int(off) + h))
     elif kind == "stripe_diagonal":
-        m = np.abs(qb - kb) <= int(rng.integers(1, 5))
+        c = int(rng.integers(1, 5))
+        m = np.abs(qb - kb) <= c
         cols = rng.choice(nb, size=int(rng.integers(20, 90)), replace=False)
         m |= np.isin(kb, cols)
+        desc["bands"].append((-c, c))
+        desc["columns"] = sorted(int(x) for x in cols)
     else:  # dual window: local band of total width 2..16 tiles plus an axial stripe
         width = int(rng.integers(2, 17))
         period = int(rng.choice([8, 16, 32]))
@@ -148,7 +160,23 @@ def _pattern(rng: np.random.Generator, nb: int) -> tuple[str, np.ndarray]:
         m = (rel >= -(width // 2)) & (rel < width - width // 2)
         md = np.mod(rel, period)
         m |= (md <= a) | (md >= period - a)
-    return kind, np.broadcast_to(m, (nb, nb)).copy()
+        desc["bands"].append((-(width // 2), width - width // 2 - 1))
+        desc["axial"] = (period, a)
+    return kind, np.broadcast_to(m, (nb, nb)).copy(), desc
+
+
+def _draw_generic(heads: int, nqb: int, seed_base: int, density):
+    draws = []
+    for h in range(heads):
+        rng = np.random.default_rng(seed_base + h)
+        while True:
+            kind, m, desc = _pattern(rng, nqb)
+            if density[0] <= m.mean() <= density[1]:
+                break
+        m[np.arange(nqb), np.arange(nqb)] = True
+        desc["bands"].append((0, 0))  # the diagonal tile every row keeps
+        draws.append((kind, m, desc))
+    return draws
 
 
 def make_generic_lists(heads: int, nqb: int, seed_base: int = 1000,
@@ -159,23 +187,20 @@ def make_generic_lists(heads: int, nqb: int, seed_base: int = 1000,
     ``h``'s rows start at ``h * nqb``. Every row keeps its diagonal tile, so no
     row is empty.
     """
-    dense = []
-    kinds = []
-    for h in range(heads):
-        rng = np.random.default_rng(seed_base + h)
-        while True:
-            kind, m = _pattern(rng, nqb)
-            if density[0] <= m.mean() <= density[1]:
-                break
-        m[np.arange(nqb), np.arange(nqb)] = True
-        dense.append(m)
-        kinds.append(kind)
-    allm = np.concatenate(dense, axis=0)
+    draws = _draw_generic(heads, nqb, seed_base, density)
+    allm = np.concatenate([m for _, m, _ in draws], axis=0)
     counts = allm.sum(axis=1)
     row_ptr = np.zeros(allm.shape[0] + 1, dtype=np.int64)
     row_ptr[1:] = np.cumsum(counts)
     _, cols = np.nonzero(allm)
-    return row_ptr.astype(np.int32), cols.astype(np.int32), kinds
+    return row_ptr.astype(np.int32), cols.astype(np.int32), [k for k, _, _ in draws]
+
+
+def generic_tile_patterns(heads: int, nqb: int, seed_base: int = 1000,
+                          density=(0.10, 0.40)) -> list[dict]:
+    """The descriptors of :func:`make_generic_lists`'s patterns (same draws),
+    diagonal tile included, for building the same lists from the patterns."""
+    return [d for _, _, d in _draw_generic(heads, nqb, seed_base, density)]
 
 
 def random_block_lists(num_rows: int, nkb: int, density: float, seed: int,
