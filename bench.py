@@ -241,7 +241,8 @@ def run_reference(args, world, rank):
 
     w = WORKLOADS[args.workload]
     q, k, v = make_qkv(w, "cpu", heads=1)
-    rp, ci = oracle.joint_block_lists(w.frames, w.tokens_per_frame, w.text_tokens, w.block)
+    rp_all, ci_all, _ = host_lists(w)
+    rp, ci = rp_all[:w.nqb + 1], ci_all[:rp_all[w.nqb]]   # head 0's list
     per_step = max(0.2, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
     rate, dt, rows, fl = oracle_sample_rate(w, (rp, ci), q, k, v, per_step)
     times = []
@@ -260,7 +261,7 @@ def run_reference(args, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": total / len(times) * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w, nnz=int(rp[-1])),
+        "config": workload_config(w, nnz=int(rp_all[-1])),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -271,14 +272,35 @@ def run_reference(args, world, rank):
 
 
 def workload_config(w, nnz):
-    text = f" + {w.text_tokens} text tokens" if w.text_tokens else ""
-    return {"workload": f"{w.name}: B={w.batch} H={w.heads} D={w.head_dim} "
-                        f"{w.frames}x{w.tokens_per_frame} tokens{text} (n={w.n}), radial "
-                        f"{w.block}x{w.block} blocks",
+    if w.radial:
+        text = f" + {w.text_tokens} text tokens" if w.text_tokens else ""
+        desc = (f"{w.name}: B={w.batch} H={w.heads} D={w.head_dim} "
+                f"{w.frames}x{w.tokens_per_frame} tokens{text} (n={w.n}), radial "
+                f"{w.block}x{w.block} blocks")
+    else:
+        desc = (f"{w.name}: B={w.batch} H={w.heads} D={w.head_dim} n={w.n}, one seeded tile "
+                f"pattern per head (diagonal, multi-diagonal, stripes, dual window), "
+                f"{w.block}x{w.block} blocks")
+    return {"workload": desc,
             "global_batch": w.batch, "heads": w.heads, "head_dim": w.head_dim, "seq_len": w.n,
             "frames": w.frames, "tokens_per_frame": w.tokens_per_frame, "block": w.block,
-            "nnz_blocks_per_head": nnz, "parallelism": "independent problem per GPU",
+            ("nnz_blocks_per_head" if w.radial else "nnz_blocks_all_heads"): nnz,
+            "parallelism": "independent problem per GPU",
             "l2": "inputs larger than L2 (Q, K, V per problem exceed 126 MB); no flush"}
+
+
+def host_lists(w):
+    """The workload's block lists on the host from the oracle: ``(row_ptr,
+    col_idx, num_lists)`` (head 0's list first)."""
+    import oracle
+
+    if w.radial:
+        rp, ci = oracle.joint_block_lists(w.frames, w.tokens_per_frame, w.text_tokens, w.block)
+        return rp, ci, 1
+    from workloads import generic_tile_patterns
+
+    rp, ci = oracle.tile_pattern_lists(generic_tile_patterns(w.heads, w.nqb), w.nqb)
+    return rp, ci, w.heads
 
 
 def run_ours(args, world, rank, local):
@@ -294,25 +316,41 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     init_dist(world, "nccl")
     w = WORKLOADS[args.workload]
-    assert w.radial, "the bench times the radial path"
 
     q, k, v = make_qkv(w, dev)
-    lists = bsa.radial_block_lists(w.frames, w.tokens_per_frame, w.block, device=dev,
-                                  text_tokens=w.text_tokens)
+    stream = torch.cuda.current_stream(dev)
+    if w.radial:
+        num_lists = 1
+        lists = bsa.radial_block_lists(w.frames, w.tokens_per_frame, w.block, device=dev,
+                                      text_tokens=w.text_tokens)
+    else:  # per-head tile patterns, expanded on the GPU
+        from workloads import generic_tile_patterns
+
+        num_lists = w.heads
+        pats = generic_tile_patterns(w.heads, w.nqb)
+        pat_raw, pat_cols = bsa.pack_tile_patterns(pats, dev)
+        lists = bsa.tile_pattern_block_lists(pats, w.nqb, w.block, device=dev)
     rp_h, ci_h = lists.row_ptr.cpu().numpy(), lists.col_idx.cpu().numpy()
-    flops = bsa.computed_flops(rp_h, ci_h, w.n, w.block, w.head_dim, w.batch, w.heads, 1)
+    flops = bsa.computed_flops(rp_h, ci_h, w.n, w.block, w.head_dim, w.batch, w.heads, num_lists)
     dense_flops = 4 * w.head_dim * w.batch * w.heads * w.n * w.n
     out = torch.empty_like(q)
     lse = torch.empty((w.batch, w.heads, w.n), dtype=torch.float32, device=dev)
     ws = torch.empty(max(bsa.bsa_attn_fwd_workspace_bytes(w.batch, w.heads, lists), 16),
                      dtype=torch.uint8, device=dev)
     row_ptr, col_idx = lists.row_ptr, lists.col_idx
-    stream = torch.cuda.current_stream(dev)
-    launches_per_step = 5  # mask count, scan, fill; work order; attention
+    launches_per_step = 5  # list count, scan, fill; work order; attention
+
+    def build_lists():
+        if w.radial:
+            bsa.bsa_joint_mask_build(w.frames, w.tokens_per_frame, w.text_tokens, w.block,
+                                     row_ptr, col_idx, col_idx.numel(), want_nnz=False,
+                                     stream=stream)
+        else:
+            bsa.bsa_tile_pattern_lists_build(w.heads, w.nqb, pat_raw, pat_cols, row_ptr, col_idx,
+                                             col_idx.numel(), want_nnz=False, stream=stream)
 
     def step(ev=None):
-        bsa.bsa_joint_mask_build(w.frames, w.tokens_per_frame, w.text_tokens, w.block, row_ptr,
-                                 col_idx, col_idx.numel(), want_nnz=False, stream=stream)
+        build_lists()
         if ev is not None:
             ev[0].record(stream)
         bsa.bsa_attn_fwd(q, k, v, lists, out, lse, ws, 0.0, stream)
@@ -368,8 +406,7 @@ def run_ours(args, world, rank, local):
                           dtype=torch.uint8, device=dev)
 
     def e2e_step():
-        bsa.bsa_joint_mask_build(w.frames, w.tokens_per_frame, w.text_tokens, w.block, row_ptr,
-                                 col_idx, col_idx.numel(), want_nnz=False, stream=stream)
+        build_lists()
         bsa.bsa_attn_fwd_host(qh, kh, vh, lists, oh, lh, ws_host, 0.0, stream)
 
     e2e_step()
@@ -387,7 +424,8 @@ def run_ours(args, world, rank, local):
 
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, dt, rows, fl = oracle_sample_rate(w, (rp_h, ci_h), q, k, v, args.cpu_seconds)
+        head0 = (rp_h[:w.nqb + 1], ci_h[:rp_h[w.nqb]])
+        rate, dt, rows, fl = oracle_sample_rate(w, head0, q, k, v, args.cpu_seconds)
         cpu_baseline = {"value": rate, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                         "sample": f"head 0, {rows.size} query rows ({int(rows[0])}..{int(rows[-1])}) "
                                   f"of the {w.name} problem, {dt:.1f} s, fp64 NumPy"}
@@ -800,7 +838,9 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", default="wan", choices=("wan", "hunyuan", "long4x", "tiny", "hunyuan_text"))
+    ap.add_argument("--workload", default="wan",
+                    choices=("wan", "hunyuan", "long4x", "tiny", "hunyuan_text", "generic"),
+                    help="generic: per-head tile patterns built on the GPU (forward only)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--pass", dest="which", choices=("fwd", "bwd", "module", "module_bwd"),
@@ -810,6 +850,8 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.workload == "generic" and args.which != "fwd":
+        ap.error("the generic workload is timed for the forward pass only")
     world, rank, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, world, rank)

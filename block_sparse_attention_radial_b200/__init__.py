@@ -20,7 +20,7 @@ from dataclasses import dataclass
 import torch
 
 from . import _lib
-from ._lib import BlockListsC, LayoutC, STATUS_NAMES
+from ._lib import TILE_PATTERN_MAX_BANDS, BlockListsC, LayoutC, STATUS_NAMES, TilePatternC
 
 __all__ = [
     "BsaError", "BlockLists", "bsa_radial_mask_build", "bsa_attn_fwd_workspace_bytes",
@@ -32,7 +32,8 @@ __all__ = [
     "bsa_attn_fwd_host", "bsa_attn_fwd_host_workspace_bytes", "bsa_attn_bwd_strided",
     "bsa_attn_module_bwd", "bsa_attn_module_bwd_workspace_bytes", "attention_module_backward", "bsa_attn_module_fwd",
     "attention_module", "module_flops", "bsa_attn_bwd", "bsa_attn_bwd_workspace_bytes",
-    "attention_backward",
+    "attention_backward", "bsa_tile_pattern_lists_build", "tile_pattern_block_lists",
+    "pack_tile_patterns",
 ]
 
 # Size of the fixed scratch array behind bsa_attn_fwd_noalloc (int32 entries).
@@ -116,6 +117,28 @@ def bsa_joint_mask_build(frames: int, tokens_per_frame: int, text_tokens: int, b
                                   _ptr(col_idx), col_capacity if col_idx is not None else 0,
                                   ctypes.byref(nnz) if want_nnz else None, _stream(stream))
     _check(st, "bsa_joint_mask_build")
+    return int(nnz.value) if want_nnz else None
+
+
+def bsa_tile_pattern_lists_build(num_lists: int, num_q_blocks: int, patterns: torch.Tensor,
+                                 columns: torch.Tensor | None, row_ptr: torch.Tensor,
+                                 col_idx: torch.Tensor | None = None, col_capacity: int = 0,
+                                 want_nnz: bool = True, stream=None) -> int | None:
+    """Per-head tile-pattern lists into caller-owned int32 device tensors.
+
+    ``patterns``: device bytes of ``bsa_tile_pattern[num_lists]`` (see
+    :func:`pack_tile_patterns`); ``columns``: device int32 stripe columns or
+    None. Returns nnz when asked (that synchronises the stream)."""
+    lib = _lib.load()
+    nnz = ctypes.c_int64(-1)
+    ncols = 0 if columns is None else int(columns.numel())
+    st = lib.bsa_tile_pattern_lists_build(num_lists, num_q_blocks, _ptr(patterns),
+                                          _ptr(columns if ncols else None), ncols, _ptr(row_ptr),
+                                          _ptr(col_idx),
+                                          col_capacity if col_idx is not None else 0,
+                                          ctypes.byref(nnz) if want_nnz else None,
+                                          _stream(stream))
+    _check(st, "bsa_tile_pattern_lists_build")
     return int(nnz.value) if want_nnz else None
 
 
@@ -376,6 +399,51 @@ def radial_block_lists(frames: int, tokens_per_frame: int, block: int = 128,
                                col_idx.numel(), stream=stream)
     assert got == nnz
     return BlockLists(row_ptr, col_idx[:nnz], 1, nqb, block)
+
+
+def pack_tile_patterns(patterns, device=None):
+    """Lay out per-head pattern descriptors as ``bsa_tile_pattern[]`` and the
+    shared stripe-column array, both on ``device``.
+
+    Each descriptor is a dict with ``bands`` (list of ``(lo, hi)`` offsets
+    ``kb - qb``, at most 16), ``axial`` (``None`` or ``(period, halfwidth)``)
+    and ``columns`` (stripe key blocks). Returns ``(patterns_u8, columns_i32
+    or None)``."""
+    device = torch.device("cuda") if device is None else torch.device(device)
+    arr = (TilePatternC * len(patterns))()
+    cols: list[int] = []
+    for c, p in zip(arr, patterns):
+        bands = list(p.get("bands", ()))
+        if len(bands) > TILE_PATTERN_MAX_BANDS:
+            raise ValueError(f"at most {TILE_PATTERN_MAX_BANDS} bands per pattern")
+        c.num_bands = len(bands)
+        for t, (lo, hi) in enumerate(bands):
+            c.band_lo[t], c.band_hi[t] = int(lo), int(hi)
+        axial = p.get("axial")
+        c.axial_period, c.axial_halfwidth = (0, 0) if axial is None else (int(axial[0]), int(axial[1]))
+        c.columns_begin = len(cols)
+        cols.extend(int(x) for x in p.get("columns", ()))
+        c.columns_end = len(cols)
+    raw = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8).to(device)
+    col_t = torch.tensor(cols, dtype=torch.int32, device=device) if cols else None
+    return raw, col_t
+
+
+def tile_pattern_block_lists(patterns, num_q_blocks: int, block: int = 128, device=None,
+                             stream=None) -> BlockLists:
+    """Build one list per head from its tile pattern on the GPU (two calls:
+    count, then fill); ``num_lists = len(patterns)``."""
+    device = torch.device("cuda") if device is None else torch.device(device)
+    raw, cols = pack_tile_patterns(patterns, device)
+    rows = len(patterns) * num_q_blocks
+    row_ptr = torch.empty(rows + 1, dtype=torch.int32, device=device)
+    nnz = bsa_tile_pattern_lists_build(len(patterns), num_q_blocks, raw, cols, row_ptr,
+                                       stream=stream)
+    col_idx = torch.empty(max(nnz, 1), dtype=torch.int32, device=device)
+    got = bsa_tile_pattern_lists_build(len(patterns), num_q_blocks, raw, cols, row_ptr, col_idx,
+                                       col_idx.numel(), stream=stream)
+    assert got == nnz
+    return BlockLists(row_ptr, col_idx[:nnz], len(patterns), num_q_blocks, block)
 
 
 def block_lists_from_csr(row_ptr, col_idx, num_lists: int, num_q_blocks: int, block: int,

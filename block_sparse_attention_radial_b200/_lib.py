@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libbsa.so")
 EXPORTS = (
     "bsa_radial_mask_build",
     "bsa_joint_mask_build",
+    "bsa_tile_pattern_lists_build",
     "bsa_attn_fwd_workspace_bytes",
     "bsa_attn_fwd",
     "bsa_attn_fwd_strided",
@@ -50,6 +51,23 @@ STATUS_NAMES = {
     6: "BSA_ERR_CAPACITY",
     7: "BSA_ERR_SCRATCH_LIMIT",
 }
+
+
+TILE_PATTERN_MAX_BANDS = 16
+
+
+class TilePatternC(ctypes.Structure):
+    """Mirror of ``bsa_tile_pattern``."""
+
+    _fields_ = [
+        ("num_bands", ctypes.c_int32),
+        ("band_lo", ctypes.c_int32 * TILE_PATTERN_MAX_BANDS),
+        ("band_hi", ctypes.c_int32 * TILE_PATTERN_MAX_BANDS),
+        ("axial_period", ctypes.c_int32),
+        ("axial_halfwidth", ctypes.c_int32),
+        ("columns_begin", ctypes.c_int32),
+        ("columns_end", ctypes.c_int32),
+    ]
 
 
 class BlockListsC(ctypes.Structure):
@@ -96,6 +114,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bsa_radial_mask_build": (ctypes.c_int, [i32, i32, i32, vp, vp, i64, ctypes.POINTER(i64), vp]),
         "bsa_joint_mask_build": (ctypes.c_int, [i32, i32, i32, i32, vp, vp, i64,
                                                 ctypes.POINTER(i64), vp]),
+        "bsa_tile_pattern_lists_build": (ctypes.c_int, [i32, i32, vp, vp, i64, vp, vp, i64,
+                                                        ctypes.POINTER(i64), vp]),
         "bsa_attn_fwd_workspace_bytes": (sz, [i32, i32, lp]),
         "bsa_attn_fwd": (ctypes.c_int, [vp, vp, vp, i32, i32, i32, i32, ctypes.c_float, lp,
                                         vp, vp, vp, sz, vp]),

@@ -21,6 +21,7 @@
 #include "dense_ref.cuh"
 #include "device_status.cuh"
 #include "lists.cuh"
+#include "patterns.cuh"
 
 namespace bsa {
 namespace {
@@ -685,6 +686,46 @@ int bsa_radial_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t bloc
                           int64_t *nnz_out, bsa_stream_t stream_) {
   return bsa_joint_mask_build(frames, tokens_per_frame, 0, block, row_ptr, col_idx, col_capacity,
                               nnz_out, stream_);
+}
+
+static_assert(sizeof(bsa_tile_pattern) == (5 + 2 * BSA_TILE_PATTERN_MAX_BANDS) * sizeof(int32_t),
+              "bsa_tile_pattern is a plain array of int32 fields");
+
+int bsa_tile_pattern_lists_build(int32_t num_lists, int32_t num_q_blocks,
+                                 const bsa_tile_pattern *patterns, const int32_t *columns,
+                                 int64_t num_columns, int32_t *row_ptr, int32_t *col_idx,
+                                 int64_t col_capacity, int64_t *nnz_out, bsa_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (num_lists < 1 || num_q_blocks < 1 || !patterns || !row_ptr || num_columns < 0 ||
+      (num_columns > 0 && !columns))
+    return BSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(patterns) | reinterpret_cast<uintptr_t>(row_ptr) |
+       reinterpret_cast<uintptr_t>(columns) | reinterpret_cast<uintptr_t>(col_idx)) & 3u)
+    return BSA_ERR_INVALID_ARG;
+  if (num_q_blocks > 262144) return BSA_ERR_UNSUPPORTED;
+  const long long rows = static_cast<long long>(num_lists) * num_q_blocks;
+  if (rows >= 0x7fffffffLL) return BSA_ERR_INVALID_ARG;
+  if (col_idx && col_capacity < 0) return BSA_ERR_INVALID_ARG;
+  const size_t smem = static_cast<size_t>((num_q_blocks + 31) / 32) * sizeof(uint32_t);
+  pattern_count_kernel<<<static_cast<unsigned>(rows), 128, smem, stream>>>(
+      patterns, columns, num_columns, num_q_blocks, row_ptr);
+  BSA_CUDA(cudaGetLastError());
+  scan_rows_kernel<<<1, 1024, 0, stream>>>(row_ptr, static_cast<int>(rows));
+  BSA_CUDA(cudaGetLastError());
+  if (nnz_out) {
+    int32_t last = 0;
+    BSA_CUDA(cudaMemcpyAsync(&last, row_ptr + rows, sizeof(int32_t), cudaMemcpyDeviceToHost,
+                             stream));
+    BSA_CUDA(cudaStreamSynchronize(stream));
+    *nnz_out = last;
+    if (col_idx && last > col_capacity) return BSA_ERR_CAPACITY;
+  }
+  if (col_idx) {
+    pattern_fill_kernel<<<static_cast<unsigned>(rows), 128, smem, stream>>>(
+        patterns, columns, num_columns, num_q_blocks, row_ptr, col_idx, col_capacity);
+    BSA_CUDA(cudaGetLastError());
+  }
+  return BSA_OK;
 }
 
 size_t bsa_attn_fwd_workspace_bytes(int32_t batch, int32_t heads, const bsa_block_lists *l) {

@@ -130,22 +130,19 @@ __global__ void scan_rows_kernel(int32_t *row_ptr, int rows) {
   }
 }
 
-// One CTA per query block: write the row's key blocks in ascending order.
-__global__ void radial_fill_kernel(RadialGeom g, const int32_t *row_ptr, int32_t *col_idx,
-                                   long long capacity) {
-  extern __shared__ uint32_t bits[];
-  __shared__ int scratch[32];
-  const int words = (g.nb + 31) >> 5;
-  radial_row_bitmap(g, blockIdx.x, bits, words);
-  // each thread owns a contiguous run of words, so ascending thread order is
-  // ascending block order
+// Writes the set bits of a row bitmap (`words` words) as ascending key-block
+// indices from col_idx[start]; entries at or beyond `capacity` are not written
+// and record BSA_ERR_CAPACITY. Each thread owns a contiguous run of words, so
+// ascending thread order is ascending block order. `scratch` holds 32 ints.
+__device__ void write_row_ascending(const uint32_t *bits, int words, long long start,
+                                    int32_t *col_idx, long long capacity, int *scratch) {
   const int per = (words + blockDim.x - 1) / blockDim.x;
   const int w0 = min(words, threadIdx.x * per), w1 = min(words, w0 + per);
   int c = 0;
   for (int i = w0; i < w1; ++i) c += __popc(bits[i]);
   int total;
   const int inc = cta_inclusive_scan(c, scratch, total);
-  long long pos = static_cast<long long>(row_ptr[blockIdx.x]) + (inc - c);
+  long long pos = start + (inc - c);
   for (int i = w0; i < w1; ++i) {
     uint32_t b = bits[i];
     while (b) {
@@ -159,6 +156,16 @@ __global__ void radial_fill_kernel(RadialGeom g, const int32_t *row_ptr, int32_t
       ++pos;
     }
   }
+}
+
+// One CTA per query block: write the row's key blocks in ascending order.
+__global__ void radial_fill_kernel(RadialGeom g, const int32_t *row_ptr, int32_t *col_idx,
+                                   long long capacity) {
+  extern __shared__ uint32_t bits[];
+  __shared__ int scratch[32];
+  const int words = (g.nb + 31) >> 5;
+  radial_row_bitmap(g, blockIdx.x, bits, words);
+  write_row_ascending(bits, words, row_ptr[blockIdx.x], col_idx, capacity, scratch);
 }
 
 // ------------------------------------------------------------- validation --

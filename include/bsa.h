@@ -128,6 +128,62 @@ int bsa_joint_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t text_
                          int32_t block, int32_t *row_ptr, int32_t *col_idx,
                          int64_t col_capacity, int64_t *nnz_out, bsa_stream_t stream);
 
+#define BSA_TILE_PATTERN_MAX_BANDS 16
+
+/*
+ * One head's tile pattern: the union of its terms over tiles (query block qb,
+ * key block kb, rel = kb - qb). It covers the families of the Sparse-vDiT
+ * skill page, "Sparse attention patterns" (diagonal window |rel| <= w;
+ * multi-diagonal bands at chosen offsets; vertical stripes, fixed key columns
+ * in every row; mixed = their union), and the dual window (local plus axial)
+ * of the Compact Attention abstract.
+ *
+ * num_bands        0..BSA_TILE_PATTERN_MAX_BANDS band terms: band t holds
+ *                  band_lo[t] <= rel <= band_hi[t] (empty when lo > hi).
+ * axial_period     0 (no axial term) or P >= 1: the term holds when rel is
+ *                  congruent modulo P to some t with |t| <= axial_halfwidth
+ *                  (the axial window read on a video's tile sequence: tiles
+ *                  about a whole number of frame periods away).
+ * axial_halfwidth  >= 0.
+ * columns_begin,   this pattern's vertical-stripe key blocks are
+ * columns_end      columns[columns_begin .. columns_end) of the shared
+ *                  `columns` array (any order, repeats allowed).
+ * Key blocks outside [0, num_q_blocks) do not exist; a row may be empty.
+ */
+typedef struct {
+  int32_t num_bands;
+  int32_t band_lo[BSA_TILE_PATTERN_MAX_BANDS];
+  int32_t band_hi[BSA_TILE_PATTERN_MAX_BANDS];
+  int32_t axial_period;
+  int32_t axial_halfwidth;
+  int32_t columns_begin;
+  int32_t columns_end;
+} bsa_tile_pattern;
+
+/*
+ * Expand one tile pattern per list into CSR block lists on the device
+ * (num_k_blocks = num_q_blocks): list h's rows start at h * num_q_blocks and
+ * each row holds its key blocks in ascending order, as bsa_attn_fwd takes
+ * them with num_lists = heads.
+ *
+ * patterns     device bsa_tile_pattern[num_lists].
+ * columns      device int32[num_columns], the stripe columns of every
+ *              pattern; NULL when num_columns is 0.
+ * row_ptr      device int32[num_lists * num_q_blocks + 1], written.
+ * col_idx, col_capacity, nnz_out: as bsa_radial_mask_build (NULL col_idx =
+ *              count only; nnz_out given = synchronise and check capacity).
+ * Limits: num_lists >= 1, 1 <= num_q_blocks <= 262144,
+ * num_lists * num_q_blocks < 2^31 - 1. A malformed pattern (num_bands
+ * outside [0, 16], negative period or half-width, a column range outside
+ * [0, num_columns]) or a stripe column outside [0, num_q_blocks) is found on
+ * the device: its rows (for a bad column, just that column) are left out and
+ * bsa_get_device_status() reports BSA_ERR_INVALID_ARG.
+ */
+int bsa_tile_pattern_lists_build(int32_t num_lists, int32_t num_q_blocks,
+                                 const bsa_tile_pattern *patterns, const int32_t *columns,
+                                 int64_t num_columns, int32_t *row_ptr, int32_t *col_idx,
+                                 int64_t col_capacity, int64_t *nnz_out, bsa_stream_t stream);
+
 /*
  * Bytes of device scratch memory bsa_attn_fwd needs for this problem (the
  * longest-row-first work order of every list and a work counter the kernel's

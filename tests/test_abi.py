@@ -102,6 +102,28 @@ def test_mask_build_argument_checks(lib):
     assert lib.bsa_set_test_hooks(0, 0) == 0
 
 
+def test_tile_pattern_build_argument_checks(lib):
+    """Bad tile-pattern build arguments are rejected before any launch."""
+    import ctypes
+
+    from block_sparse_attention_radial_b200._lib import TilePatternC
+
+    assert ctypes.sizeof(TilePatternC) == (5 + 2 * 16) * 4
+    vp = ctypes.c_void_p
+    pat, rp, cols = vp(1 << 20), vp(2 << 20), vp(3 << 20)
+    f = lib.bsa_tile_pattern_lists_build
+    assert f(0, 16, pat, None, 0, rp, None, 0, None, None) == 1          # no lists
+    assert f(2, 0, pat, None, 0, rp, None, 0, None, None) == 1           # no rows
+    assert f(2, 16, None, None, 0, rp, None, 0, None, None) == 1         # no patterns
+    assert f(2, 16, pat, None, 0, None, None, 0, None, None) == 1        # no row_ptr
+    assert f(2, 16, pat, None, 5, rp, None, 0, None, None) == 1          # columns missing
+    assert f(2, 16, pat, cols, -1, rp, None, 0, None, None) == 1         # negative count
+    assert f(2, 16, vp((1 << 20) + 2), None, 0, rp, None, 0, None, None) == 1  # misaligned
+    assert f(2, 16, pat, None, 0, rp, vp(4 << 20), -1, None, None) == 1  # negative capacity
+    assert f(2, 262145, pat, None, 0, rp, None, 0, None, None) == 2      # too many blocks
+    assert f(1 << 14, 1 << 17, pat, None, 0, rp, None, 0, None, None) == 1  # rows >= 2^31 - 1
+
+
 def test_backward_workspace_and_host_checks(lib):
     from block_sparse_attention_radial_b200._lib import BlockListsC
 
