@@ -539,18 +539,18 @@ def run_ours_bwd(args, world, rank, local):
     if bsa.bsa_get_device_status() != 0:
         raise SystemExit("device status after the timed region")
 
-    # end to end: pinned host inputs in, gradients back to the host
+    # end to end through the C ABI on host buffers: bsa_attn_bwd_host copies
+    # pinned q, k, v, out, dout, lse in and dq, dk, dv back, pipelined with the
+    # kernels by head group
     e2e_steps = max(3, min(args.steps, 10))
     host_in = [t.cpu().pin_memory() for t in (q, k, v, out, do, lse)]
-    dev_in = [torch.empty_like(t) for t in (q, k, v, out, do, lse)]
     host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
+    ws_host = torch.empty(bsa.bsa_attn_bwd_host_workspace_bytes(w.batch, w.heads, w.n,
+                                                                w.head_dim, lists),
+                          dtype=torch.uint8, device=dev)
 
     def e2e_step():
-        for d_, h_ in zip(dev_in, host_in):
-            d_.copy_(h_, non_blocking=True)
-        bsa.bsa_attn_bwd(*dev_in[:5], dev_in[5], lists, dq, dk, dv, ws, 0.0, stream)
-        for h_, d_ in zip(host_out, (dq, dk, dv)):
-            h_.copy_(d_, non_blocking=True)
+        bsa.bsa_attn_bwd_host(*host_in, lists, *host_out, ws_host, 0.0, stream)
 
     e2e_step()
     torch.cuda.synchronize(dev)

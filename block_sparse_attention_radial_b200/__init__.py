@@ -33,7 +33,7 @@ __all__ = [
     "bsa_attn_module_bwd", "bsa_attn_module_bwd_workspace_bytes", "attention_module_backward", "bsa_attn_module_fwd",
     "attention_module", "module_flops", "bsa_attn_bwd", "bsa_attn_bwd_workspace_bytes",
     "attention_backward", "bsa_tile_pattern_lists_build", "tile_pattern_block_lists",
-    "pack_tile_patterns",
+    "pack_tile_patterns", "bsa_attn_bwd_host", "bsa_attn_bwd_host_workspace_bytes",
 ]
 
 # Size of the fixed scratch array behind bsa_attn_fwd_noalloc (int32 entries).
@@ -308,6 +308,35 @@ def bsa_attn_bwd(q, k, v, out, dout, lse, lists: BlockLists, dq, dk, dv, workspa
                           _ptr(workspace), workspace.numel() * workspace.element_size(),
                           _stream(stream))
     _check(st, "bsa_attn_bwd")
+
+
+def bsa_attn_bwd_host_workspace_bytes(batch: int, heads: int, n: int, head_dim: int,
+                                      lists: BlockLists) -> int:
+    return int(_lib.load().bsa_attn_bwd_host_workspace_bytes(batch, heads, n, head_dim,
+                                                             ctypes.byref(lists.c_struct())))
+
+
+def bsa_attn_bwd_host(q, k, v, out, dout, lse, lists: BlockLists, dq, dk, dv, workspace=None,
+                      softmax_scale: float = 0.0, stream=None, device=None) -> None:
+    """bsa_attn_bwd on CPU tensors (pin them for copy/compute overlap): q, k, v,
+    out, dout and the gradients dq, dk, dv bf16 [B, H, n, D], lse float
+    [B, H, n], all contiguous in host memory. Enqueued on ``stream``;
+    synchronise it before reading the gradients."""
+    B, H, n, D = q.shape
+    for t in (q, k, v, out, dout, lse, dq, dk, dv):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("bsa_attn_bwd_host takes contiguous host tensors")
+    lib = _lib.load()
+    ls = lists.c_struct()
+    if workspace is None:
+        dev = lists.row_ptr.device if device is None else torch.device(device)
+        workspace = torch.empty(lib.bsa_attn_bwd_host_workspace_bytes(B, H, n, D, ctypes.byref(ls)),
+                                dtype=torch.uint8, device=dev)
+    st = lib.bsa_attn_bwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), B, H, n,
+                               D, float(softmax_scale), ctypes.byref(ls), _ptr(dq), _ptr(dk),
+                               _ptr(dv), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "bsa_attn_bwd_host")
 
 
 def bsa_attn_bwd_strided(q, k, v, out, dout, lse, lists: BlockLists, dq, dk, dv, workspace=None,

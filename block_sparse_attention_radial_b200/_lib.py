@@ -31,6 +31,8 @@ EXPORTS = (
     "bsa_attn_bwd",
     "bsa_attn_bwd_strided",
     "bsa_attn_bwd_workspace_bytes",
+    "bsa_attn_bwd_host_workspace_bytes",
+    "bsa_attn_bwd_host",
     "bsa_validate_lists",
     "bsa_get_device_status",
     "bsa_get_timeout_detail",
@@ -144,6 +146,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bsa_attn_bwd": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float,
                                         lp, vp, vp, vp, vp, sz, vp]),
         "bsa_attn_bwd_workspace_bytes": (sz, [i32, i32, i32, lp]),
+        "bsa_attn_bwd_host_workspace_bytes": (sz, [i32, i32, i32, i32, lp]),
+        "bsa_attn_bwd_host": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                             ctypes.c_float, lp, vp, vp, vp, vp, sz, vp]),
         "bsa_attn_bwd_strided": (ctypes.c_int, [vp, yp, vp, yp, vp, yp, vp, yp, vp, yp, vp, i32,
                                                 i32, i32, i32, ctypes.c_float, lp, vp, yp, vp, yp,
                                                 vp, yp, vp, sz, vp]),

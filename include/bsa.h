@@ -450,6 +450,43 @@ size_t bsa_attn_bwd_workspace_bytes(int32_t batch, int32_t heads, int32_t n,
                                     const bsa_block_lists *lists);
 
 /*
+ * Bytes of device workspace bsa_attn_bwd_host needs: device copies of q, k,
+ * v, out, dout, lse, dq, dk and dv plus bsa_attn_bwd's own scratch for the
+ * largest head group. Returns 0 for invalid arguments.
+ */
+size_t bsa_attn_bwd_host_workspace_bytes(int32_t batch, int32_t heads, int32_t n,
+                                         int32_t head_dim, const bsa_block_lists *lists);
+
+/*
+ * bsa_attn_bwd on HOST buffers: q_host, k_host, v_host, out_host, dout_host
+ * (bf16 [batch, heads, n, head_dim], contiguous) and lse_host (float
+ * [batch, heads, n], required) are copied to the device, the backward runs,
+ * and dq_host, dk_host, dv_host (bf16, same layout; not overlapping any
+ * input) are copied back. Head groups and streams as bsa_attn_fwd_host:
+ * group g's inputs are copied in on an internal stream while group g-1's
+ * backward runs on `stream` (one bsa_attn_bwd call per group, on that
+ * group's heads and lists) and group g-2's gradients are copied out on a
+ * second internal stream. The gradients are bit-identical to one
+ * bsa_attn_bwd call on the whole problem: every (batch, head) slice is
+ * computed by the same kernels in the same order either way.
+ * lists        device lists as for bsa_attn_bwd (built, or enqueued on
+ *              `stream` before this call).
+ * workspace    device memory of bsa_attn_bwd_host_workspace_bytes(),
+ *              256-byte aligned; holds the device copies.
+ * Asynchronous, with the same rules as bsa_attn_fwd_host: host buffers stay
+ * valid and the gradients unread until `stream` has been synchronised; calls
+ * of both host entries are serialised on the internal streams. Errors as
+ * bsa_attn_bwd; an error from a group's launch is returned after the groups
+ * before it were enqueued (their results are then incomplete).
+ */
+int bsa_attn_bwd_host(const void *q_host, const void *k_host, const void *v_host,
+                      const void *out_host, const void *dout_host, const float *lse_host,
+                      int32_t batch, int32_t heads, int32_t n, int32_t head_dim,
+                      float softmax_scale, const bsa_block_lists *lists, void *dq_host,
+                      void *dk_host, void *dv_host, void *workspace, size_t workspace_bytes,
+                      bsa_stream_t stream);
+
+/*
  * Check `lists`: row_ptr starts at 0, is non-decreasing and ends at nnz; each
  * row is strictly increasing and in [0, num_k_blocks). Reads no col_idx entry
  * at or beyond nnz. Synchronises `stream`. Returns BSA_OK, BSA_ERR_BAD_LISTS

@@ -273,3 +273,37 @@ def test_host_buffer_forward_host_checks(lib):
     assert call(hd=96) == 2                         # head_dim
     assert call(wsb=ws - 1) == 1                    # workspace too small
     assert call(w=vp((1 << 32) + 16)) == 1          # workspace not 256-byte aligned
+
+
+def test_host_buffer_backward_host_checks(lib):
+    """bsa_attn_bwd_host: workspace size formula and argument checks on the
+    host (all rejected before any CUDA call)."""
+    from block_sparse_attention_radial_b200._lib import BlockListsC
+
+    vp, ref = ctypes.c_void_p, ctypes.byref
+    ls = BlockListsC(1, 256, 256, 128, 1000, 0, 0)
+    t = 1 * 40 * 32760 * 128 * 2
+    # 40 heads in groups of at most 7: the backward's scratch for 7 heads
+    # (lse2 and delta per 128-row tile row, work counters, transposed offsets
+    # and entries), then q, k, v, out, dout, dq, dk, dv (bf16) and lse (fp32)
+    scratch = 2 * 7 * 256 * 128 * 4 + 256 + 1280 + 4096
+    expect = scratch + 8 * t + 40 * 32760 * 4
+    assert lib.bsa_attn_bwd_host_workspace_bytes(1, 40, 32760, 128, ref(ls)) == expect
+    assert lib.bsa_attn_bwd_host_workspace_bytes(1, 40, 0, 128, ref(ls)) == 0
+    bad = BlockListsC(3, 256, 256, 128, 1000, 0, 0)      # 3 lists for 40 heads
+    assert lib.bsa_attn_bwd_host_workspace_bytes(1, 40, 32760, 128, ref(bad)) == 0
+    small = BlockListsC(2, 8, 8, 128, 10, 1 << 22, 1 << 23)
+    ws = lib.bsa_attn_bwd_host_workspace_bytes(1, 2, 1000, 64, ref(small))
+    assert ws > 0
+    h = vp(1 << 20)
+
+    def call(q=h, lse=h, dv=h, hd=64, w=vp(1 << 32), wsb=ws):
+        return lib.bsa_attn_bwd_host(q, h, h, h, h, lse, 1, 2, 1000, hd, 0.0, ref(small), h, h, dv,
+                                     w, wsb, None)
+
+    assert call(q=vp(0)) == 1                       # null input
+    assert call(lse=None) == 1                      # lse is required
+    assert call(dv=None) == 1                       # null output
+    assert call(hd=96) == 2                         # head_dim
+    assert call(wsb=ws - 1) == 1                    # workspace too small
+    assert call(w=vp((1 << 32) + 16)) == 1          # workspace not 256-byte aligned
