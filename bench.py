@@ -852,6 +852,9 @@ def main(argv=None):
         ap.error("--warmup must be at least 3")
     if args.workload == "generic" and args.which != "fwd":
         ap.error("the generic workload is timed for the forward pass only")
+    if args.impl == "reference" and args.which != "fwd":
+        ap.error("the reference arm times the forward oracle only (the backward and module "
+                 "passes report their own oracle samples as cpu_baseline)")
     world, rank, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, world, rank)
