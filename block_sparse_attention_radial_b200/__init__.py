@@ -449,6 +449,8 @@ def pack_tile_patterns(patterns, device=None):
         for t, (lo, hi) in enumerate(bands):
             c.band_lo[t], c.band_hi[t] = int(lo), int(hi)
         axial = p.get("axial")
+        if axial is not None and (int(axial[0]) < 1 or int(axial[1]) < 0):
+            raise ValueError("axial term needs a period >= 1 and a half-width >= 0 (None: no term)")
         c.axial_period, c.axial_halfwidth = (0, 0) if axial is None else (int(axial[0]), int(axial[1]))
         c.columns_begin = len(cols)
         cols.extend(int(x) for x in p.get("columns", ()))

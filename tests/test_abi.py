@@ -307,3 +307,28 @@ def test_host_buffer_backward_host_checks(lib):
     assert call(hd=96) == 2                         # head_dim
     assert call(wsb=ws - 1) == 1                    # workspace too small
     assert call(w=vp((1 << 32) + 16)) == 1          # workspace not 256-byte aligned
+
+
+def test_tile_pattern_packing():
+    """Descriptors are laid out as bsa_tile_pattern[] (stripe columns in one
+    shared array, each pattern's range recorded); malformed terms are refused
+    on the host."""
+    import pytest
+    import torch
+
+    import block_sparse_attention_radial_b200 as bsa
+
+    pats = [{"bands": [(-2, 3), (7, 7)], "axial": (8, 1), "columns": [5, 1]}, {},
+            {"columns": [9]}]
+    raw, cols = bsa.pack_tile_patterns(pats, device="cpu")
+    words = raw.view(torch.int32).view(3, 37)
+    assert words[0, 0] == 2 and words[0, 1:3].tolist() == [-2, 7]
+    assert words[0, 17:19].tolist() == [3, 7]
+    assert words[0, 33:37].tolist() == [8, 1, 0, 2]
+    assert words[1].tolist() == [0] * 35 + [2, 2]      # empty range at offset 2
+    assert words[2, 35:37].tolist() == [2, 3]
+    assert cols.tolist() == [5, 1, 9]
+    with pytest.raises(ValueError):
+        bsa.pack_tile_patterns([{"bands": [(0, 0)] * 17}], device="cpu")
+    with pytest.raises(ValueError):
+        bsa.pack_tile_patterns([{"axial": (0, 1)}], device="cpu")
