@@ -118,3 +118,27 @@ def test_generic_workload_descriptors_reproduce_its_lists():
     np.testing.assert_array_equal(rp, rq)
     np.testing.assert_array_equal(ci, cq)
     assert set(kinds) == {"dual_window", "diagonal", "multi_diagonal", "stripe_diagonal"}
+
+
+def test_random_descriptors_against_loops():
+    """Random unions of every term, including bands outside the row, inverted
+    bands and repeated columns, against a per-tile loop (the axial term by the
+    explicit search over period multiples)."""
+    rng = np.random.default_rng(7)
+    for _ in range(30):
+        n = int(rng.integers(1, 40))
+        pat = {"bands": [], "axial": None, "columns": []}
+        for _ in range(int(rng.integers(0, 5))):
+            o, h = int(rng.integers(-n - 3, n + 3)), int(rng.integers(-2, 6))
+            pat["bands"].append((o - h, o + h))
+        if rng.random() < 0.6:
+            pat["axial"] = (int(rng.integers(1, 12)), int(rng.integers(0, 4)))
+        if rng.random() < 0.6:
+            pat["columns"] = rng.integers(0, n, size=int(rng.integers(0, 6))).tolist()
+        want = np.zeros((n, n), dtype=bool)
+        ax = _axial_bruteforce(n, *pat["axial"]) if pat["axial"] else np.zeros((n, n), bool)
+        for qb in range(n):
+            for kb in range(n):
+                want[qb, kb] = (any(lo <= kb - qb <= hi for lo, hi in pat["bands"])
+                                or ax[qb, kb] or kb in pat["columns"])
+        np.testing.assert_array_equal(oracle.tile_pattern_mask(pat, n), want)
