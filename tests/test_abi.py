@@ -332,3 +332,41 @@ def test_tile_pattern_packing():
         bsa.pack_tile_patterns([{"bands": [(0, 0)] * 17}], device="cpu")
     with pytest.raises(ValueError):
         bsa.pack_tile_patterns([{"axial": (0, 1)}], device="cpu")
+
+
+def test_plain_c_caller(lib, tmp_path):
+    """A C99 program compiled against include/bsa.h and linked to libbsa.so
+    calls host-only entry points: the header is plain C and the symbols link
+    without C++ name mangling."""
+    import shutil
+    import subprocess
+
+    from block_sparse_attention_radial_b200 import _lib
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "caller.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include "bsa.h"
+int main(void) {
+  bsa_block_lists l = {1, 256, 256, 128, 1000, (const int32_t *)0, (const int32_t *)0};
+  bsa_tile_pattern p = {0};
+  printf("%zu\n", bsa_attn_fwd_workspace_bytes(1, 40, &l));
+  printf("%s\n", bsa_status_string(BSA_ERR_CAPACITY));
+  printf("%d\n", bsa_tile_pattern_lists_build(0, 16, &p, 0, 0, 0, 0, 0, 0, 0));
+  printf("%zu\n", sizeof(bsa_tile_pattern));
+  return 0;
+}
+""")
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), "-L" + libdir, "-l:libbsa.so",
+                    "-Wl,-rpath," + libdir], check=True, capture_output=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    assert out[0] == "1280"                      # 128 pair entries, aligned, + the work counter
+    assert out[1] == lib.bsa_status_string(6).decode()
+    assert out[2] == "1"                         # BSA_ERR_INVALID_ARG, found on the host
+    assert out[3] == str(37 * 4)
