@@ -1,0 +1,57 @@
+"""bench.py's host-side pieces on the CPU: the workloads' host lists (head 0
+first, one list per head for the per-head tile patterns), the config block of
+the JSON line, argument checks, and the kernel-source hash that ties a
+committed DRAM-traffic figure to the code it was measured on."""
+
+import json
+import os
+
+import numpy as np
+import pytest
+
+import bench
+from workloads import WORKLOADS
+
+
+def test_host_lists_radial_and_generic():
+    rp, ci, nl = bench.host_lists(WORKLOADS["tiny"])
+    assert nl == 1 and rp.size == WORKLOADS["tiny"].nqb + 1 and rp[-1] == ci.size == 220
+    w = WORKLOADS["generic"]
+    rp, ci, nl = bench.host_lists(w)
+    assert nl == w.heads and rp.size == w.heads * w.nqb + 1 and rp[-1] == ci.size
+    assert np.all(np.diff(rp) >= 1)              # every row keeps its diagonal tile
+
+
+def test_workload_config_names_the_workload():
+    c = bench.workload_config(WORKLOADS["wan"], nnz=31248)
+    assert c["workload"].startswith("wan:") and "21x1560" in c["workload"]
+    assert c["nnz_blocks_per_head"] == 31248 and c["seq_len"] == 32760
+    g = bench.workload_config(WORKLOADS["generic"], nnz=287806)
+    assert g["workload"].startswith("generic:") and g["nnz_blocks_all_heads"] == 287806
+    json.dumps(c), json.dumps(g)
+
+
+@pytest.mark.parametrize("argv", [["--warmup", "2"], ["--workload", "generic", "--pass", "bwd"],
+                                  ["--impl", "reference", "--pass", "module"]])
+def test_argument_checks(argv):
+    with pytest.raises(SystemExit) as e:
+        bench.main(argv)
+    assert e.value.code == 2
+
+
+def test_traffic_figure_follows_the_kernel_source_hash():
+    """A committed capture's DRAM bytes are reported only while the kernel
+    source it was taken on is unchanged (comments aside); otherwise null."""
+    for which, name in (("fwd", "attn_fwd_pair_sm100_wan_traffic.json"),
+                        ("bwd", "attn_bwd_sm100_wan_traffic.json")):
+        with open(os.path.join(bench.ROOT, "profiles", name)) as f:
+            d = json.load(f)
+        same = d["kernel_source_hash"] == bench.kernel_source_hash(which)
+        assert bench.load_traffic("wan", which) == (d["dram_bytes_per_launch"] if same else None)
+    assert bench.load_traffic("generic") is None   # no capture for that workload
+
+
+def test_source_hash_ignores_comments():
+    code = "int f(int x) {\n  return x + 1;  // one\n}\n"
+    assert bench._code_only(code) == bench._code_only("/* doc */\n" + code.replace("one", "two"))
+    assert bench._code_only(code) != bench._code_only(code.replace("+ 1", "+ 2"))
