@@ -55,3 +55,26 @@ def test_source_hash_ignores_comments():
     code = "int f(int x) {\n  return x + 1;  // one\n}\n"
     assert bench._code_only(code) == bench._code_only("/* doc */\n" + code.replace("one", "two"))
     assert bench._code_only(code) != bench._code_only(code.replace("+ 1", "+ 2"))
+
+
+def test_computed_flops_counts_valid_rows_and_columns():
+    """4 * D * (valid rows x valid columns) over every listed block, per head
+    and batch item, against a per-token loop (ragged last block included)."""
+    import block_sparse_attention_radial_b200 as bsa
+
+    n, blk, D, B, H = 300, 64, 32, 2, 3
+    nqb = -(-n // blk)
+    rng = np.random.default_rng(3)
+    for L in (1, H):
+        m = rng.random((L * nqb, nqb)) < 0.5
+        rp = np.zeros(L * nqb + 1, dtype=np.int64)
+        rp[1:] = np.cumsum(m.sum(axis=1))
+        ci = np.nonzero(m)[1]
+        pairs = 0
+        for r in range(L * nqb):
+            qb = r % nqb
+            for kb in ci[rp[r]:rp[r + 1]]:
+                pairs += sum(1 for i in range(qb * blk, min(n, qb * blk + blk))
+                             for j in range(kb * blk, min(n, kb * blk + blk)))
+        per_list_heads = H if L == 1 else 1
+        assert bsa.computed_flops(rp, ci, n, blk, D, B, H, L) == 4 * D * B * per_list_heads * pairs
