@@ -544,18 +544,24 @@ int bsa_selftest_exp2(const float *x, float *y_poly, float *y_mufu, float *y_ref
  * later allocations. Those callers cannot provide bsa_attn_fwd's workspace.
  *
  * Same operation, arguments and results as bsa_attn_fwd, minus the workspace:
- * the scratch it needs (the longest-row-first work order, one int32 per query
- * block per list, and the work counter) lives in a fixed array compiled into
- * the library, of BSA_NOALLOC_MAX_ORDER_ENTRIES + 64 int32 entries (256 KiB +
- * 256 B). Every GPU that loads
- * the library holds that array until the process exits.
+ * the scratch it needs (the longest-first work order and the work counter)
+ * lives in a fixed array compiled into the library, of
+ * BSA_NOALLOC_MAX_ORDER_ENTRIES + 64 int32 entries (256 KiB + 256 B). The work
+ * order takes one int32 per query block per list at block 64 and one per pair
+ * of query blocks (ceil(num_q_blocks / 2) per list) at block 128; the limit
+ * below is checked against the larger of the two, so at block 128 it is
+ * conservative by a factor of two. Every GPU that loads the library holds
+ * that array until the process exits.
  *
  * - Returns BSA_ERR_SCRATCH_LIMIT, launching nothing, when
  *   lists->num_lists * lists->num_q_blocks exceeds the maximum.
  * - Calls no cudaMalloc, cudaFree or other allocating routine.
  * - The first call on each device resolves the array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   (cudaGetSymbolAddress) with that device current and keeps it for the
+ *   rest of the process; make that first call before any stream capture.
+ *   A device reset (cudaDeviceReset) unloads the library's device code and
+ *   leaves the kept address stale: do not call this entry point on a device
+ *   after resetting it in the same process.
  * - All calls share the one array and each call overwrites the entries it
  *   uses (nothing in it has to start at zero). Calls whose kernels overlap on
  *   the GPU (for example on two streams at once) race on it; serialise them.

@@ -8,9 +8,9 @@ and dQ, dK, dV are rounded to bf16 on output (2^-9). The gradient of a row
 is a sum of many such terms with independent rounding, so the relative RMS
 error stays near a few 2^-9; dS = P (dP - delta) loses relative accuracy where
 dP is close to delta, which the max-abs bound (relative to the tensor's
-largest entry) absorbs. Bars: relative RMS <= 1e-2, max-abs <= 2.5e-2 of the
-oracle's largest entry, per tensor (measured: about 2.4e-3 and 4e-3 on the
-random cases).
+largest entry) absorbs. Bars: the forward's relative RMS 5e-3 and max-abs
+2e-2, the max-abs taken relative to the oracle's largest entry, per tensor
+(measured: about 2.4e-3 and 4e-3 on the random cases).
 """
 
 import numpy as np
@@ -22,8 +22,8 @@ from workloads import WORKLOADS, make_qkv, make_random_qkv, random_block_lists
 
 pytestmark = pytest.mark.gpu
 
-REL_RMS = 1e-2
-MAX_REL = 2.5e-2
+REL_RMS = 5e-3
+MAX_REL = 2e-2
 
 
 @pytest.fixture(scope="module")
