@@ -303,12 +303,154 @@ def host_lists(w):
     return rp, ci, w.heads
 
 
+def _gpu_uuid(dev):
+    import torch
+
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid).replace("GPU-", "")
+    except Exception:
+        return None
+
+
+class FwdProblem:
+    """One forward workload resident on the device: inputs, lists, outputs and
+    the step that rebuilds the lists and runs the attention."""
+
+    def __init__(self, w, dev, stream):
+        import torch
+
+        import block_sparse_attention_radial_b200 as bsa
+        from workloads import make_qkv
+
+        self.w, self.dev, self.stream, self.bsa = w, dev, stream, bsa
+        self.q, self.k, self.v = make_qkv(w, dev)
+        if w.radial:
+            self.num_lists = 1
+            self.lists = bsa.radial_block_lists(w.frames, w.tokens_per_frame, w.block, device=dev,
+                                                text_tokens=w.text_tokens)
+        else:  # per-head tile patterns, expanded on the GPU
+            from workloads import generic_tile_patterns
+
+            self.num_lists = w.heads
+            pats = generic_tile_patterns(w.heads, w.nqb)
+            self.pat_raw, self.pat_cols = bsa.pack_tile_patterns(pats, dev)
+            self.lists = bsa.tile_pattern_block_lists(pats, w.nqb, w.block, device=dev)
+        self.rp_h = self.lists.row_ptr.cpu().numpy()
+        self.ci_h = self.lists.col_idx.cpu().numpy()
+        self.flops = bsa.computed_flops(self.rp_h, self.ci_h, w.n, w.block, w.head_dim, w.batch,
+                                        w.heads, self.num_lists)
+        self.dense_flops = 4 * w.head_dim * w.batch * w.heads * w.n * w.n
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty((w.batch, w.heads, w.n), dtype=torch.float32, device=dev)
+        self.ws = torch.empty(max(bsa.bsa_attn_fwd_workspace_bytes(w.batch, w.heads, self.lists),
+                                  16), dtype=torch.uint8, device=dev)
+        self.launches_per_step = 5  # list count, scan, fill; work order; attention
+
+    def build_lists(self):
+        w, l, bsa = self.w, self.lists, self.bsa
+        if w.radial:
+            bsa.bsa_joint_mask_build(w.frames, w.tokens_per_frame, w.text_tokens, w.block,
+                                     l.row_ptr, l.col_idx, l.col_idx.numel(), want_nnz=False,
+                                     stream=self.stream)
+        else:
+            bsa.bsa_tile_pattern_lists_build(w.heads, w.nqb, self.pat_raw, self.pat_cols,
+                                             l.row_ptr, l.col_idx, l.col_idx.numel(),
+                                             want_nnz=False, stream=self.stream)
+
+    def step(self, ev=None):
+        self.build_lists()
+        if ev is not None:
+            ev[0].record(self.stream)
+        self.bsa.bsa_attn_fwd(self.q, self.k, self.v, self.lists, self.out, self.lse, self.ws,
+                              0.0, self.stream)
+        if ev is not None:
+            ev[1].record(self.stream)
+
+    def timed(self, steps, warmup, rank):
+        """W untimed steps, then K steps bracketed by a barrier and a device
+        synchronisation, with the clocks sampled meanwhile. Returns (ms over
+        all K steps, max over ranks; mean attention-kernel ms; clocks)."""
+        import numpy as np
+        import torch
+
+        bsa, dev, stream = self.bsa, self.dev, self.stream
+        for _ in range(warmup):
+            self.step()
+        torch.cuda.synchronize(dev)
+        status = bsa.bsa_get_device_status()
+        if status != 0:
+            raise SystemExit(f"device status {status} after warm-up")
+        sampler = ClockSampler(_gpu_uuid(dev)) if rank == 0 else None
+        if sampler is not None:
+            time.sleep(0.4)   # let the sampler start before the timed region
+        kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(dev)
+        torch.cuda.synchronize(dev)
+        t_start.record(stream)
+        for i in range(steps):
+            self.step(kev[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(dev)
+        clocks = sampler.stop() if sampler is not None else None
+        ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
+        kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+        status = bsa.bsa_get_device_status()
+        if status != 0:
+            raise SystemExit(f"device status {status} after the timed region")
+        # the lists rebuilt inside every step are the ones the FLOPs were counted on
+        if not (np.array_equal(self.lists.row_ptr.cpu().numpy(), self.rp_h)
+                and np.array_equal(self.lists.col_idx.cpu().numpy(), self.ci_h)):
+            raise SystemExit("lists rebuilt in the timed steps differ from the counted lists")
+        return ms, kernel_ms, clocks
+
+    def roofline(self, kernel_ms, peaks, peak_kind):
+        peak = float(peaks["bf16_tflops"])
+        achieved = self.flops / (kernel_ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": load_traffic(self.w.name),
+                "peak_kind": f"{peak_kind} bf16 burst",
+                "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
+                "kernel": "attn_fwd_pair_sm100_kernel<128> (+ work-order prepass)",
+                "kernel_ms": kernel_ms, "flops_per_launch": self.flops}
+
+
+# The other configurations of the metric's 32k-131k token range, timed in the
+# same default run after the headline one (one GPU only).
+PER_CONFIG = ("hunyuan", "long4x", "generic")
+
+
+def per_config_records(args, dev, stream, rank, peaks, peak_kind):
+    import torch
+
+    from workloads import WORKLOADS
+
+    recs = {}
+    steps, warmup = max(3, min(args.steps, args.per_config_steps)), 3
+    for name in PER_CONFIG:
+        prob = FwdProblem(WORKLOADS[name], dev, stream)
+        ms, kernel_ms, clocks = prob.timed(steps, warmup, rank)
+        recs[name] = {
+            "value": prob.flops * steps / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": ms / steps, "steps": steps, "warmup": warmup,
+            "config": workload_config(prob.w, nnz=int(prob.rp_h[-1])),
+            "roofline": prob.roofline(kernel_ms, peaks, peak_kind),
+            "gpu_launches": prob.launches_per_step * steps,
+            "dense_equivalent_tflops": prob.dense_flops * steps / (ms * 1e-3) / 1e12,
+            "clocks": clocks,
+        }
+        del prob
+        torch.cuda.empty_cache()
+    return recs
+
+
 def run_ours(args, world, rank, local):
-    import numpy as np
     import torch
 
     import block_sparse_attention_radial_b200 as bsa
-    from workloads import WORKLOADS, make_qkv
+    from workloads import WORKLOADS
 
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
@@ -316,97 +458,24 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     init_dist(world, "nccl")
     w = WORKLOADS[args.workload]
-
-    q, k, v = make_qkv(w, dev)
     stream = torch.cuda.current_stream(dev)
-    if w.radial:
-        num_lists = 1
-        lists = bsa.radial_block_lists(w.frames, w.tokens_per_frame, w.block, device=dev,
-                                      text_tokens=w.text_tokens)
-    else:  # per-head tile patterns, expanded on the GPU
-        from workloads import generic_tile_patterns
-
-        num_lists = w.heads
-        pats = generic_tile_patterns(w.heads, w.nqb)
-        pat_raw, pat_cols = bsa.pack_tile_patterns(pats, dev)
-        lists = bsa.tile_pattern_block_lists(pats, w.nqb, w.block, device=dev)
-    rp_h, ci_h = lists.row_ptr.cpu().numpy(), lists.col_idx.cpu().numpy()
-    flops = bsa.computed_flops(rp_h, ci_h, w.n, w.block, w.head_dim, w.batch, w.heads, num_lists)
-    dense_flops = 4 * w.head_dim * w.batch * w.heads * w.n * w.n
-    out = torch.empty_like(q)
-    lse = torch.empty((w.batch, w.heads, w.n), dtype=torch.float32, device=dev)
-    ws = torch.empty(max(bsa.bsa_attn_fwd_workspace_bytes(w.batch, w.heads, lists), 16),
-                     dtype=torch.uint8, device=dev)
-    row_ptr, col_idx = lists.row_ptr, lists.col_idx
-    launches_per_step = 5  # list count, scan, fill; work order; attention
-
-    def build_lists():
-        if w.radial:
-            bsa.bsa_joint_mask_build(w.frames, w.tokens_per_frame, w.text_tokens, w.block,
-                                     row_ptr, col_idx, col_idx.numel(), want_nnz=False,
-                                     stream=stream)
-        else:
-            bsa.bsa_tile_pattern_lists_build(w.heads, w.nqb, pat_raw, pat_cols, row_ptr, col_idx,
-                                             col_idx.numel(), want_nnz=False, stream=stream)
-
-    def step(ev=None):
-        build_lists()
-        if ev is not None:
-            ev[0].record(stream)
-        bsa.bsa_attn_fwd(q, k, v, lists, out, lse, ws, 0.0, stream)
-        if ev is not None:
-            ev[1].record(stream)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    status = bsa.bsa_get_device_status()
-    if status != 0:
-        raise SystemExit(f"device status {status} after warm-up")
-
-    uuid = None
-    try:
-        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid).replace("GPU-", "")
-    except Exception:
-        pass
-    sampler = ClockSampler(uuid) if rank == 0 else None
-    if sampler is not None:
-        time.sleep(0.4)   # let the sampler start before the timed region
-    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(dev)
-    torch.cuda.synchronize(dev)
-    t_start.record(stream)
-    for i in range(args.steps):
-        step(kev[i])
-    t_end.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(dev)
-    clocks = sampler.stop() if sampler is not None else None
-    ms_local = t_start.elapsed_time(t_end)
-    ms = max_over_ranks(ms_local, dev)
-    kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
-    status = bsa.bsa_get_device_status()
-    if status != 0:
-        raise SystemExit(f"device status {status} after the timed region")
-    # the lists rebuilt inside every step are the ones the FLOPs were counted on
-    if not (np.array_equal(row_ptr.cpu().numpy(), rp_h)
-            and np.array_equal(col_idx.cpu().numpy(), ci_h)):
-        raise SystemExit("lists rebuilt in the timed steps differ from the counted lists")
+    prob = FwdProblem(w, dev, stream)
+    q, k, v, lists = prob.q, prob.k, prob.v, prob.lists
+    rp_h, ci_h, flops = prob.rp_h, prob.ci_h, prob.flops
+    ms, kernel_ms, clocks = prob.timed(args.steps, args.warmup, rank)
 
     # ---- end to end through the C ABI on host buffers: bsa_attn_fwd_host copies
     # pinned q, k, v in and out / lse back, pipelined with the kernels by head group
     e2e_steps = max(3, min(args.steps, 10))
     qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
-    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    oh = torch.empty(prob.out.shape, dtype=prob.out.dtype).pin_memory()
+    lh = torch.empty(prob.lse.shape, dtype=prob.lse.dtype).pin_memory()
     ws_host = torch.empty(bsa.bsa_attn_fwd_host_workspace_bytes(w.batch, w.heads, w.n,
                                                                 w.head_dim, lists),
                           dtype=torch.uint8, device=dev)
 
     def e2e_step():
-        build_lists()
+        prob.build_lists()
         bsa.bsa_attn_fwd_host(qh, kh, vh, lists, oh, lh, ws_host, 0.0, stream)
 
     e2e_step()
@@ -429,12 +498,17 @@ def run_ours(args, world, rank, local):
         cpu_baseline = {"value": rate, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                         "sample": f"head 0, {rows.size} query rows ({int(rows[0])}..{int(rows[-1])}) "
                                   f"of the {w.name} problem, {dt:.1f} s, fp64 NumPy"}
+    del qh, kh, vh, oh, lh, ws_host
 
+    peaks, peak_kind = load_peaks()
+    roofline = prob.roofline(kernel_ms, peaks, peak_kind)
+    dense_flops, launches_per_step = prob.dense_flops, prob.launches_per_step
+    per_config = None
+    if world == 1 and args.workload == "wan" and args.per_config_steps > 0:
+        del prob, q, k, v, lists
+        torch.cuda.empty_cache()
+        per_config = per_config_records(args, dev, stream, rank, peaks, peak_kind)
     if rank == 0:
-        peaks, peak_kind = load_peaks()
-        peak = float(peaks["bf16_tflops"])
-        achieved = flops / (kernel_ms * 1e-3) / 1e12
-        traffic = load_traffic(w.name)
         line = {
             "metric": METRIC,
             "value": flops * world * args.steps / (ms * 1e-3) / 1e12,
@@ -444,18 +518,14 @@ def run_ours(args, world, rank, local):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": workload_config(w, nnz=int(rp_h[-1])),
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": traffic,
-                         "peak_kind": f"{peak_kind} bf16 burst",
-                         "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
-                         "kernel": "attn_fwd_pair_sm100_kernel<128> (+ work-order prepass)",
-                         "kernel_ms": kernel_ms, "flops_per_launch": flops},
+            "roofline": roofline,
             "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
             "dense_equivalent_tflops": dense_flops * world * args.steps / (ms * 1e-3) / 1e12,
             "clocks": clocks,
             "cpu_baseline": cpu_baseline,
+            "per_config": per_config,
         }
         print(json.dumps(line), flush=True)
     import torch.distributed as dist
@@ -843,6 +913,9 @@ def main(argv=None):
                     help="generic: per-head tile patterns built on the GPU (forward only)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--per-config-steps", type=int, default=10,
+                    help="timed steps for each of the other forward configurations recorded "
+                         "under per_config in the default (wan, one GPU) run; 0 skips them")
     ap.add_argument("--pass", dest="which", choices=("fwd", "bwd", "module", "module_bwd"),
                     default="fwd",
                     help="time the forward (default, the headline), the backward pass, or the "

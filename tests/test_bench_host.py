@@ -78,3 +78,13 @@ def test_computed_flops_counts_valid_rows_and_columns():
                              for j in range(kb * blk, min(n, kb * blk + blk)))
         per_list_heads = H if L == 1 else 1
         assert bsa.computed_flops(rp, ci, n, blk, D, B, H, L) == 4 * D * B * per_list_heads * pairs
+
+
+def test_per_config_names_cover_the_metric_range():
+    # the default run records the other forward configurations beside wan
+    names = bench.PER_CONFIG
+    assert set(names) == {"hunyuan", "long4x", "generic"}
+    for name in names:
+        w = WORKLOADS[name]
+        assert w.n >= 32 * 1024 and w.block == 128 and w.head_dim == 128
+    assert max(WORKLOADS[n].n for n in names) == 84 * 1560
