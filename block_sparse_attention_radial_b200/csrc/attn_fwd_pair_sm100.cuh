@@ -8,11 +8,20 @@
 // kernel. Each tile runs its own softmax warpgroup, and while one tile's
 // softmax works the tensor core runs the other tile's MMAs.
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax of tile A (thread = row = TMEM lane)
 //   warps 4-7  softmax of tile B
 //   warp 8     producer: Q_A, Q_B, then the union's K and V tiles (TMA)
 //   warp 9     MMA issuer
+//   warps 10-11 no role (they complete the third warpgroup)
+// Register budgets: each SM sub-partition holds one warp of each warpgroup,
+// launched at 168 registers per thread. The third warpgroup gives up all but
+// 88 and the two softmax warpgroups take 208 each (208 + 208 + 88 = 3 x 168),
+// so a softmax thread keeps its 128 scores and the packed P in registers
+// without spilling, and the producer and MMA lanes still fit theirs. Each
+// budget change sits inside its role's branch: the compiler allocates the
+// code a change dominates within that budget, and code after a join of the
+// branches would get the smallest one.
 //
 // TMEM: S_A [0,128), S_B [128,256), O_A [256, 256+D), O_B [256+D, 256+2D).
 // P of a tile overwrites the first 64 columns of its S buffer.
@@ -52,7 +61,11 @@ struct PairCfg {
   static constexpr uint32_t S_COL = 0;           // S of tile t at S_COL + 128 t
   static constexpr uint32_t O_COL = 256;         // O of tile t at O_COL + D t
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 384;
+  static constexpr uint32_t REGS_LAUNCH = 168;  // 65536 / 384, rounded down to a multiple of 8
+  static constexpr uint32_t REGS_SOFTMAX = 208;
+  static constexpr uint32_t REGS_OTHER = 88;
+  static_assert(2 * REGS_SOFTMAX + REGS_OTHER <= 3 * REGS_LAUNCH, "register budgets");
   static_assert(NS >= 3, "K/V ring needs at least three stages");
 };
 
@@ -173,7 +186,7 @@ __device__ __forceinline__ bool plan_wait(const volatile uint32_t *ring, uint32_
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_fwd_pair_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k,
                                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -236,239 +249,247 @@ __global__ void __launch_bounds__(320, 1)
 
   WaitCtx wc{&abort_flag, p.wait_limit_ns, 0};
 
-  if (warp == 8) {
-    // ------------------------------------------------------------ producer
-    // One lane: TMA issue needs no warp, and warp-wide bookkeeping between
-    // issues only adds latency.
-    if (lane == 0) {
-      wc.role = kRoleProducer;
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      uint32_t ring = 0, qcount = 0, gstep = 0;
-      volatile uint32_t *plans = plan_ring;
-      bool skip_next_k = (p.fault_flags & 1) && blockIdx.x == 0;
-      int skipped_ring = -1;
-      bool ok = true;
-      for (int k = 0; ok; ++k) {
-        const int slot = k % kItemN;
-        if (!(ok = lane_wait(&bar_item_empty[slot], ((k / kItemN) & 1) ^ 1, wc, kBarItem, k)))
-          break;
-        int idx = atomicAdd(p.item_counter, 1);
-        if (idx >= p.total_items) idx = -1;
-        item_ring[slot] = idx;
-        mbar_arrive(&bar_item_full[slot]);
-        if (idx < 0) break;
-        const PairItem it = decode_pair(idx, p, npairs);
-        if (it.lenA == 0 && it.lenB == 0) continue;
-        if (!(ok = lane_wait(&bar_q_empty, (qcount & 1u) ^ 1u, wc, kBarQEmpty, qcount))) break;
-        mbar_arrive_expect_tx(&bar_q_full, 2 * C::Q_BYTES);
-        const int ib = it.bh / p.heads, ih = it.bh - ib * p.heads;
-        tma_load_5d(sQ, &tm_q, &bar_q_full, 0, it.qa * BN, 0, ih, ib);
-        tma_load_5d(sQ + C::Q_BYTES, &tm_q, &bar_q_full, 0, (it.qa + 1) * BN, 0, ih, ib);
-        ++qcount;
-        // Same walk and same first-use order as the MMA issuer: at step j it
-        // needs V(j-1) first when tile A listed j-1 or A skips j, and K(j)
-        // first otherwise.
-        UnionWalker uw;
-        uw.reset(p, it.a0, it.lenA, it.b0, it.lenB);
-        bool pa = false, pb = false;
-        int prev_kb = 0;
-        while (ok) {
-          int kb = 0;
-          bool a = false, b = false;
-          const bool more = uw.next(kb, a, b);
-          const bool need_v = pa || pb;
-          if (!more && !need_v) break;
-          const bool v_first = pa || !a;
-          {
-            const bool need_k = more;
-            const uint32_t vpos = ring + ((need_k && !v_first) ? 1u : 0u);
-            const uint32_t kpos = ring + ((need_v && v_first) ? 1u : 0u);
-            const uint32_t rec =
-                (pa ? 2u : 0u) | (a ? 4u : 0u) | (pb ? 8u : 0u) | (b ? 16u : 0u) |
-                (more ? 0u : 32u) | ((vpos % C::NS) << 8) | (((vpos / C::NS) & 1u) << 11) |
-                ((kpos % C::NS) << 12) | (((kpos / C::NS) & 1u) << 15) | (plan_tag(gstep) << 24);
-            plans[gstep % kPlanN] = rec;
-            ++gstep;
-          }
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const bool is_v = (e == 0) == v_first;
-            if (is_v ? !need_v : !more) continue;
-            const uint32_t s = ring % C::NS;
-            if (!(ok = lane_wait(&bar_kv_empty[s], ((ring / C::NS) & 1u) ^ 1u, wc, kBarKvEmpty,
-                                 ring)))
-              break;
-            if (!is_v && skip_next_k) {  // test hook: this stage's barrier never gets its arrival
-              skip_next_k = false;
-              skipped_ring = static_cast<int>(ring);
-              ++ring;
-              continue;
-            }
-            mbar_arrive_expect_tx(&bar_kv_full[s], C::TILE_BYTES);
-            tma_load_5d(sKV + s * C::TILE_BYTES, is_v ? &tm_v : &tm_k, &bar_kv_full[s], 0,
-                        (is_v ? prev_kb : kb) * BN, 0, ih, ib);
-            ++ring;
-          }
-          pa = a;
-          pb = b;
-          prev_kb = kb;
-          if (!more) break;
-        }
-      }
-      WaitCtx drain{&abort_flag, p.wait_limit_ns, kRoleProducer};
-      int zero = 0;
-      drain.abort = &zero;
-      const uint32_t first = ring > C::NS ? ring - C::NS : 0;
-      for (uint32_t r = first; r < ring; ++r) {
-        if (static_cast<int>(r) == skipped_ring) continue;
-        wait_bounded(&bar_kv_full[r % C::NS], (r / C::NS) & 1u, drain, kBarKvFull, r);
-      }
-      if (qcount > 0) wait_bounded(&bar_q_full, (qcount - 1) & 1u, drain, kBarQFull, qcount);
-    }
-    __syncwarp();
-  }
-  else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    // One lane issues everything. tcgen05.mma and tcgen05.commit issued from
-    // a single thread go back to back; issued under a lane-0 branch of a
-    // whole warp that also votes on its waits, each MMA and commit costs
-    // tens of extra cycles. Descriptors as 32-bit halves (see the one-tile
-    // kernel): shared high half, low half = address >> 4 | LBO.
-    if (lane == 0) {
-      wc.role = kRoleMma;
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-      constexpr uint32_t kHi = (1024u >> 4) | (1u << 14) | (2u << 29);
-      constexpr uint32_t kLboK = 1u << 16;
-      constexpr uint32_t kLboV = static_cast<uint32_t>(BN * 128 / 16) << 16;  // 64-wide D chunks
-      const uint32_t q_lo0 = (smem_addr(sQ) >> 4) | kLboK;
-      const uint32_t kv_base = smem_addr(sKV) >> 4;
-      uint32_t gstep = 0, qcount = 0;
-      const volatile uint32_t *plans = plan_ring;
-      uint32_t rec_next = 0u;
-      uint32_t pcnt[2] = {0u, 0u};     // p_full phases consumed, per tile
-      uint32_t items_t[2] = {0u, 0u};  // items in which the tile had blocks
-      bool ok = true;
-      for (int k = 0; ok; ++k) {
-        const int slot = k % kItemN;
-        if (!(ok = lane_wait(&bar_item_full[slot], (k / kItemN) & 1, wc, kBarItem, k))) break;
-        const int idx = *static_cast<volatile int *>(&item_ring[slot]);
-        mbar_arrive(&bar_item_empty[slot]);
-        if (idx < 0) break;
-        const PairItem it = decode_pair(idx, p, npairs);
-        if (it.lenA == 0 && it.lenB == 0) continue;
-        if (!(ok = lane_wait(&bar_q_full, qcount & 1u, wc, kBarQFull, qcount))) break;
-        tc_fence_after();
-        const int len_t[2] = {it.lenA, it.lenB};
-        bool first_pv[2] = {true, true};
-        bool q_released = false;
-        while (ok) {
-          // this step's record (usually already there: the producer runs ahead)
-          uint32_t rec = rec_next;
-          if ((rec >> 24) != plan_tag(gstep) && !(ok = plan_wait(plan_ring, gstep, rec, wc)))
+  // Each budget change sits inside its role's branch, so that the role's code
+  // is dominated by it and the compiler allocates that role's registers
+  // within its own budget (after a join of the branches it would have to
+  // assume the smallest).
+  if (warp >= 8) {
+    regs_shrink<C::REGS_OTHER>();
+    if (warp == 8) {
+      // ------------------------------------------------------------ producer
+      // One lane: TMA issue needs no warp, and warp-wide bookkeeping between
+      // issues only adds latency.
+      if (lane == 0) {
+        wc.role = kRoleProducer;
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        uint32_t ring = 0, qcount = 0, gstep = 0;
+        volatile uint32_t *plans = plan_ring;
+        bool skip_next_k = (p.fault_flags & 1) && blockIdx.x == 0;
+        int skipped_ring = -1;
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+          const int slot = k % kItemN;
+          if (!(ok = lane_wait(&bar_item_empty[slot], ((k / kItemN) & 1) ^ 1, wc, kBarItem, k)))
             break;
-          ++gstep;
-          const bool pv[2] = {(rec & 2u) != 0u, (rec & 8u) != 0u};
-          const bool qk[2] = {(rec & 4u) != 0u, (rec & 16u) != 0u};
-          const bool last = (rec & 32u) != 0u;
-          const uint32_t vstage = (rec >> 8) & 7u, vpar = (rec >> 11) & 1u;
-          const uint32_t kstage = (rec >> 12) & 7u, kpar = (rec >> 15) & 1u;
-          if (last && !q_released) {  // no QK left in this item: the Q buffers may refill
-            mma_commit(&bar_q_empty);
-            q_released = true;
-          }
-          // Early non-blocking checks of this step's barriers: a check of
-          // even a completed mbarrier takes about as long as two MMAs and the
-          // tensor pipe accepts one MMA at a time, so checks issued together
-          // (and ahead of the MMAs that precede their use) keep that latency
-          // off the tensor pipe.
-          const bool need_v = pv[0] || pv[1];
-          const bool need_k = qk[0] || qk[1];
-          bool p_ready[2];
-          p_ready[0] = pv[0] && mbar_test(&bar_p_full[0], pcnt[0] & 1u);
-          const bool v_ready = need_v && mbar_test(&bar_kv_full[vstage], vpar);
-          const bool k_ready = need_k && mbar_test(&bar_kv_full[kstage], kpar);
-          p_ready[1] = false;
-          bool have_k = false, have_v = false;
+          int idx = atomicAdd(p.item_counter, 1);
+          if (idx >= p.total_items) idx = -1;
+          item_ring[slot] = idx;
+          mbar_arrive(&bar_item_full[slot]);
+          if (idx < 0) break;
+          const PairItem it = decode_pair(idx, p, npairs);
+          if (it.lenA == 0 && it.lenB == 0) continue;
+          if (!(ok = lane_wait(&bar_q_empty, (qcount & 1u) ^ 1u, wc, kBarQEmpty, qcount))) break;
+          mbar_arrive_expect_tx(&bar_q_full, 2 * C::Q_BYTES);
+          const int ib = it.bh / p.heads, ih = it.bh - ib * p.heads;
+          tma_load_5d(sQ, &tm_q, &bar_q_full, 0, it.qa * BN, 0, ih, ib);
+          tma_load_5d(sQ + C::Q_BYTES, &tm_q, &bar_q_full, 0, (it.qa + 1) * BN, 0, ih, ib);
+          ++qcount;
+          // Same walk and same first-use order as the MMA issuer: at step j it
+          // needs V(j-1) first when tile A listed j-1 or A skips j, and K(j)
+          // first otherwise.
+          UnionWalker uw;
+          uw.reset(p, it.a0, it.lenA, it.b0, it.lenB);
+          bool pa = false, pb = false;
+          int prev_kb = 0;
+          while (ok) {
+            int kb = 0;
+            bool a = false, b = false;
+            const bool more = uw.next(kb, a, b);
+            const bool need_v = pa || pb;
+            if (!more && !need_v) break;
+            const bool v_first = pa || !a;
+            {
+              const bool need_k = more;
+              const uint32_t vpos = ring + ((need_k && !v_first) ? 1u : 0u);
+              const uint32_t kpos = ring + ((need_v && v_first) ? 1u : 0u);
+              const uint32_t rec =
+                  (pa ? 2u : 0u) | (a ? 4u : 0u) | (pb ? 8u : 0u) | (b ? 16u : 0u) |
+                  (more ? 0u : 32u) | ((vpos % C::NS) << 8) | (((vpos / C::NS) & 1u) << 11) |
+                  ((kpos % C::NS) << 12) | (((kpos / C::NS) & 1u) << 15) | (plan_tag(gstep) << 24);
+              plans[gstep % kPlanN] = rec;
+              ++gstep;
+            }
 #pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            if (!ok) break;
-            if (t == 1) rec_next = plans[gstep % kPlanN];  // next step's record, read ahead
-            if (pv[t]) {
-              if (!p_ready[t] &&
-                  !(ok = lane_wait(&bar_p_full[t], pcnt[t] & 1u, wc, kBarPFull, pcnt[t])))
+            for (int e = 0; e < 2; ++e) {
+              const bool is_v = (e == 0) == v_first;
+              if (is_v ? !need_v : !more) continue;
+              const uint32_t s = ring % C::NS;
+              if (!(ok = lane_wait(&bar_kv_empty[s], ((ring / C::NS) & 1u) ^ 1u, wc, kBarKvEmpty,
+                                   ring)))
                 break;
-              ++pcnt[t];
-              if (first_pv[t] && items_t[t] > 0) {
-                if (!(ok = lane_wait(&bar_o_empty[t], (items_t[t] - 1) & 1u, wc, kBarOEmpty,
-                                     items_t[t])))
-                  break;
+              if (!is_v && skip_next_k) {  // test hook: this stage's barrier never gets its arrival
+                skip_next_k = false;
+                skipped_ring = static_cast<int>(ring);
+                ++ring;
+                continue;
               }
-              if (!have_v) {
-                if (!v_ready &&
-                    !(ok = lane_wait(&bar_kv_full[vstage], vpar, wc, kBarKvFull, gstep)))
-                  break;
-                have_v = true;
-              }
-              tc_fence_after();
-              // tile B's P, checked while tile A's MMAs go out
-              if (t == 0 && pv[1]) p_ready[1] = mbar_test(&bar_p_full[1], pcnt[1] & 1u);
-              const uint32_t v_lo = (kv_base + vstage * (C::TILE_BYTES >> 4)) | kLboV;
-#pragma unroll
-              for (int kk = 0; kk < BN / 16; ++kk)
-                mma_ts_lh(tmem + C::O_COL + t * D, tmem + C::S_COL + t * 128 + kk * 8,
-                          v_lo + kk * (16 * 128 >> 4), kHi, idesc_pv,
-                          (!first_pv[t] || kk > 0) ? 1u : 0u);
-              first_pv[t] = false;
-            } else if (t == 0 && pv[1]) {
-              p_ready[1] = mbar_test(&bar_p_full[1], pcnt[1] & 1u);
+              mbar_arrive_expect_tx(&bar_kv_full[s], C::TILE_BYTES);
+              tma_load_5d(sKV + s * C::TILE_BYTES, is_v ? &tm_v : &tm_k, &bar_kv_full[s], 0,
+                          (is_v ? prev_kb : kb) * BN, 0, ih, ib);
+              ++ring;
             }
-            if (qk[t]) {
-              if (!have_k) {
-                if (!k_ready &&
-                    !(ok = lane_wait(&bar_kv_full[kstage], kpar, wc, kBarKvFull, gstep)))
+            pa = a;
+            pb = b;
+            prev_kb = kb;
+            if (!more) break;
+          }
+        }
+        WaitCtx drain{&abort_flag, p.wait_limit_ns, kRoleProducer};
+        int zero = 0;
+        drain.abort = &zero;
+        const uint32_t first = ring > C::NS ? ring - C::NS : 0;
+        for (uint32_t r = first; r < ring; ++r) {
+          if (static_cast<int>(r) == skipped_ring) continue;
+          wait_bounded(&bar_kv_full[r % C::NS], (r / C::NS) & 1u, drain, kBarKvFull, r);
+        }
+        if (qcount > 0) wait_bounded(&bar_q_full, (qcount - 1) & 1u, drain, kBarQFull, qcount);
+      }
+      __syncwarp();
+    }
+    else if (warp == 9) {
+      // ------------------------------------------------------------ MMA issuer
+      // One lane issues everything. tcgen05.mma and tcgen05.commit issued from
+      // a single thread go back to back; issued under a lane-0 branch of a
+      // whole warp that also votes on its waits, each MMA and commit costs
+      // tens of extra cycles. Descriptors as 32-bit halves (see the one-tile
+      // kernel): shared high half, low half = address >> 4 | LBO.
+      if (lane == 0) {
+        wc.role = kRoleMma;
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+        constexpr uint32_t kHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+        constexpr uint32_t kLboK = 1u << 16;
+        constexpr uint32_t kLboV = static_cast<uint32_t>(BN * 128 / 16) << 16;  // 64-wide D chunks
+        const uint32_t q_lo0 = (smem_addr(sQ) >> 4) | kLboK;
+        const uint32_t kv_base = smem_addr(sKV) >> 4;
+        uint32_t gstep = 0, qcount = 0;
+        const volatile uint32_t *plans = plan_ring;
+        uint32_t rec_next = 0u;
+        uint32_t pcnt[2] = {0u, 0u};     // p_full phases consumed, per tile
+        uint32_t items_t[2] = {0u, 0u};  // items in which the tile had blocks
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+          const int slot = k % kItemN;
+          if (!(ok = lane_wait(&bar_item_full[slot], (k / kItemN) & 1, wc, kBarItem, k))) break;
+          const int idx = *static_cast<volatile int *>(&item_ring[slot]);
+          mbar_arrive(&bar_item_empty[slot]);
+          if (idx < 0) break;
+          const PairItem it = decode_pair(idx, p, npairs);
+          if (it.lenA == 0 && it.lenB == 0) continue;
+          if (!(ok = lane_wait(&bar_q_full, qcount & 1u, wc, kBarQFull, qcount))) break;
+          tc_fence_after();
+          const int len_t[2] = {it.lenA, it.lenB};
+          bool first_pv[2] = {true, true};
+          bool q_released = false;
+          while (ok) {
+            // this step's record (usually already there: the producer runs ahead)
+            uint32_t rec = rec_next;
+            if ((rec >> 24) != plan_tag(gstep) && !(ok = plan_wait(plan_ring, gstep, rec, wc)))
+              break;
+            ++gstep;
+            const bool pv[2] = {(rec & 2u) != 0u, (rec & 8u) != 0u};
+            const bool qk[2] = {(rec & 4u) != 0u, (rec & 16u) != 0u};
+            const bool last = (rec & 32u) != 0u;
+            const uint32_t vstage = (rec >> 8) & 7u, vpar = (rec >> 11) & 1u;
+            const uint32_t kstage = (rec >> 12) & 7u, kpar = (rec >> 15) & 1u;
+            if (last && !q_released) {  // no QK left in this item: the Q buffers may refill
+              mma_commit(&bar_q_empty);
+              q_released = true;
+            }
+            // Early non-blocking checks of this step's barriers: a check of
+            // even a completed mbarrier takes about as long as two MMAs and the
+            // tensor pipe accepts one MMA at a time, so checks issued together
+            // (and ahead of the MMAs that precede their use) keep that latency
+            // off the tensor pipe.
+            const bool need_v = pv[0] || pv[1];
+            const bool need_k = qk[0] || qk[1];
+            bool p_ready[2];
+            p_ready[0] = pv[0] && mbar_test(&bar_p_full[0], pcnt[0] & 1u);
+            const bool v_ready = need_v && mbar_test(&bar_kv_full[vstage], vpar);
+            const bool k_ready = need_k && mbar_test(&bar_kv_full[kstage], kpar);
+            p_ready[1] = false;
+            bool have_k = false, have_v = false;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (!ok) break;
+              if (t == 1) rec_next = plans[gstep % kPlanN];  // next step's record, read ahead
+              if (pv[t]) {
+                if (!p_ready[t] &&
+                    !(ok = lane_wait(&bar_p_full[t], pcnt[t] & 1u, wc, kBarPFull, pcnt[t])))
                   break;
+                ++pcnt[t];
+                if (first_pv[t] && items_t[t] > 0) {
+                  if (!(ok = lane_wait(&bar_o_empty[t], (items_t[t] - 1) & 1u, wc, kBarOEmpty,
+                                       items_t[t])))
+                    break;
+                }
+                if (!have_v) {
+                  if (!v_ready &&
+                      !(ok = lane_wait(&bar_kv_full[vstage], vpar, wc, kBarKvFull, gstep)))
+                    break;
+                  have_v = true;
+                }
                 tc_fence_after();
-                have_k = true;
-              }
-              const uint32_t q_lo = q_lo0 + t * (C::Q_BYTES >> 4);
-              const uint32_t k_lo = (kv_base + kstage * (C::TILE_BYTES >> 4)) | kLboK;
+                // tile B's P, checked while tile A's MMAs go out
+                if (t == 0 && pv[1]) p_ready[1] = mbar_test(&bar_p_full[1], pcnt[1] & 1u);
+                const uint32_t v_lo = (kv_base + vstage * (C::TILE_BYTES >> 4)) | kLboV;
 #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
-                mma_ss_lh(tmem + C::S_COL + t * 128, q_lo + off, kHi, k_lo + off, kHi, idesc_qk,
-                          kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < BN / 16; ++kk)
+                  mma_ts_lh(tmem + C::O_COL + t * D, tmem + C::S_COL + t * 128 + kk * 8,
+                            v_lo + kk * (16 * 128 >> 4), kHi, idesc_pv,
+                            (!first_pv[t] || kk > 0) ? 1u : 0u);
+                first_pv[t] = false;
+              } else if (t == 0 && pv[1]) {
+                p_ready[1] = mbar_test(&bar_p_full[1], pcnt[1] & 1u);
               }
-              mma_commit(&bar_s_full[t]);
+              if (qk[t]) {
+                if (!have_k) {
+                  if (!k_ready &&
+                      !(ok = lane_wait(&bar_kv_full[kstage], kpar, wc, kBarKvFull, gstep)))
+                    break;
+                  tc_fence_after();
+                  have_k = true;
+                }
+                const uint32_t q_lo = q_lo0 + t * (C::Q_BYTES >> 4);
+                const uint32_t k_lo = (kv_base + kstage * (C::TILE_BYTES >> 4)) | kLboK;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                  const uint32_t off = (kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2;
+                  mma_ss_lh(tmem + C::S_COL + t * 128, q_lo + off, kHi, k_lo + off, kHi, idesc_qk,
+                            kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&bar_s_full[t]);
+              }
             }
+            if (!ok) break;
+            if (have_k) mma_commit(&bar_kv_empty[kstage]);
+            if (have_v) mma_commit(&bar_kv_empty[vstage]);
+            if (last) break;
           }
           if (!ok) break;
-          if (have_k) mma_commit(&bar_kv_empty[kstage]);
-          if (have_v) mma_commit(&bar_kv_empty[vstage]);
-          if (last) break;
+#pragma unroll
+          for (int t = 0; t < 2; ++t)
+            if (len_t[t] > 0) mma_commit(&bar_o_final[t]);
+          if (!q_released) mma_commit(&bar_q_empty);
+#pragma unroll
+          for (int t = 0; t < 2; ++t) items_t[t] += len_t[t] > 0 ? 1u : 0u;
+          ++qcount;
         }
-        if (!ok) break;
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-          if (len_t[t] > 0) mma_commit(&bar_o_final[t]);
-        if (!q_released) mma_commit(&bar_q_empty);
-#pragma unroll
-        for (int t = 0; t < 2; ++t) items_t[t] += len_t[t] > 0 ? 1u : 0u;
-        ++qcount;
+        mma_commit(&bar_final);
+        WaitCtx drain{&abort_flag, p.wait_limit_ns, kRoleMma};
+        int zero = 0;
+        drain.abort = &zero;
+        wait_bounded(&bar_final, 0, drain, kBarFinal, qcount);
       }
-      mma_commit(&bar_final);
-      WaitCtx drain{&abort_flag, p.wait_limit_ns, kRoleMma};
-      int zero = 0;
-      drain.abort = &zero;
-      wait_bounded(&bar_final, 0, drain, kBarFinal, qcount);
+      __syncwarp();
     }
-    __syncwarp();
-  }
-  else {
+    // warps 10 and 11 have no role: they wait at the final barrier
+  } else {
     // ------------------------------------------------------------ softmax
     // Warpgroup t (warps 4t..4t+3) serves tile t; thread = row = TMEM lane.
+    regs_grow<C::REGS_SOFTMAX>();
     wc.role = kRoleSoftmax;
     const int t = warp >> 2;
     const int wq = warp & 3;

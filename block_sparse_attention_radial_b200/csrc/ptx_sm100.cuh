@@ -273,6 +273,20 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, bo
          ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
+// ------------------------------------------------------- register budgets --
+
+// Per-warp register budget changes. Every warp of a warpgroup executes the
+// same one; an increase waits until decreases elsewhere in the CTA have freed
+// enough registers, so the sums must balance against the launch allocation.
+template <uint32_t N>
+__device__ __forceinline__ void regs_shrink() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_grow() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------------- math --
 
 __device__ __forceinline__ float ex2_approx(float x) {
