@@ -738,7 +738,7 @@ def run_ours_module(args, world, rank, local, backward=False):
     ws = torch.empty(bsa.bsa_attn_module_workspace_bytes(w.batch, n, H, D, lists),
                      dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = 2  # work order, attention (the two GEMMs are cuBLASLt's)
+    launches_per_step = 4  # q/k/v GEMM, work order, attention, out GEMM
     if backward:
         C = H * D
         flops = 16 * w.batch * n * C * C + 2.5 * att_flops
@@ -752,9 +752,9 @@ def run_ours_module(args, world, rank, local, backward=False):
         bws = torch.empty(bsa.bsa_attn_module_bwd_workspace_bytes(w.batch, n, H, D, lists),
                           dtype=torch.uint8, device=dev)
         bsa.bsa_attn_module_fwd(x, wqkv, bqkv, wo, bo, H, lists, y, ws, 0.0, stream)
-        # attention backward: prep, transposed-list count, scan, fill, dK/dV, dQ;
-        # two column-sum passes for each bias gradient (the GEMMs are cuBLASLt's)
-        launches_per_step = 6 + 4
+        # four GEMMs; attention backward: prep, transposed-list count, scan,
+        # fill, dK/dV, dQ; two column-sum passes for each bias gradient
+        launches_per_step = 4 + 6 + 4
 
     def step(ev=None):
         if ev is not None:
@@ -882,11 +882,11 @@ def run_ours_module(args, world, rank, local, backward=False):
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": None,
                          "peak_kind": f"{peak_kind} bf16 burst",
-                         "kernel": ("whole module backward: four cuBLASLt GEMMs + attention "
+                         "kernel": ("whole module backward: four gemm_bf16_sm100 GEMMs + attention "
                                     "backward (attn_bwd_dkdv/dq_kernel<128>) + column sums")
                          if backward else
-                         ("whole module: cuBLASLt q/k/v GEMM + work order + "
-                          "attn_fwd_pair_sm100_kernel<128> + cuBLASLt out GEMM"),
+                         ("whole module: gemm_bf16_sm100 q/k/v GEMM + work order + "
+                          "attn_fwd_pair_sm100_kernel<128> + gemm_bf16_sm100 out GEMM"),
                          "kernel_ms": kernel_ms, "flops_per_launch": exec_flops},
             "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

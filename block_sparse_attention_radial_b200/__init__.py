@@ -28,6 +28,7 @@ __all__ = [
     "bsa_get_timeout_detail", "bsa_status_string", "bsa_last_cuda_error", "bsa_set_test_hooks",
     "radial_block_lists", "block_lists_from_csr", "attention", "dense_masked_reference",
     "computed_flops", "bsa_attn_fwd_noalloc", "bsa_selftest_exp2", "NOALLOC_MAX_ORDER_ENTRIES",
+    "bsa_gemm_bf16",
     "bsa_attn_fwd_strided", "bsa_attn_module_workspace_bytes", "bsa_joint_mask_build",
     "bsa_attn_fwd_host", "bsa_attn_fwd_host_workspace_bytes", "bsa_attn_bwd_strided",
     "bsa_attn_module_bwd", "bsa_attn_module_bwd_workspace_bytes", "attention_module_backward", "bsa_attn_module_fwd",
@@ -396,6 +397,22 @@ def bsa_status_string(status: int) -> str:
 
 def bsa_last_cuda_error() -> str:
     return _lib.load().bsa_last_cuda_error().decode()
+
+
+def bsa_gemm_bf16(a, b, out, bias=None, a_mn_major: bool = False, b_mn_major: bool = False,
+                  stream=None) -> None:
+    """out[m, n] = A[m, k] B[k, n] (+ bias[n]) on the library's tcgen05 GEMM.
+
+    ``a`` is A stored as [m, k] (``a_mn_major=False``) or as its transpose
+    [k, m]; ``b`` is B stored as [n, k] (``b_mn_major=False``, an nn.Linear
+    weight) or as [k, n]. 2-D bf16 device tensors with a contiguous last axis;
+    the row strides are passed through."""
+    m, n = out.shape
+    k = a.shape[0] if a_mn_major else a.shape[1]
+    st = _lib.load().bsa_gemm_bf16(_ptr(a), a.stride(0), int(a_mn_major), _ptr(b), b.stride(0),
+                                   int(b_mn_major), _ptr(bias), _ptr(out), out.stride(0), m, n, k,
+                                   _stream(stream))
+    _check(st, "bsa_gemm_bf16")
 
 
 def bsa_selftest_exp2(x: torch.Tensor):

@@ -27,6 +27,7 @@ EXPORTS = (
     "bsa_attn_module_fwd",
     "bsa_attn_module_bwd_workspace_bytes",
     "bsa_attn_module_bwd",
+    "bsa_gemm_bf16",
     "bsa_attn_dense_masked_ref",
     "bsa_attn_bwd",
     "bsa_attn_bwd_strided",
@@ -140,6 +141,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "bsa_last_cuda_error": (ctypes.c_char_p, []),
         "bsa_set_test_hooks": (ctypes.c_int, [i64, i32]),
+        "bsa_gemm_bf16": (ctypes.c_int, [vp, i64, i32, vp, i64, i32, vp, vp, i64, i64, i64, i64,
+                                         vp]),
         "bsa_selftest_exp2": (ctypes.c_int, [vp, vp, vp, vp, i32, vp]),
         "bsa_attn_fwd_noalloc": (ctypes.c_int, [vp, vp, vp, i32, i32, i32, i32, ctypes.c_float,
                                                 lp, vp, vp, vp]),

@@ -25,16 +25,10 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def cuda_lib_dir() -> str:
-    return os.path.join(os.path.dirname(os.path.dirname(os.path.realpath(nvcc_path()))), "lib64")
-
-
 def build(verbose: bool = False, output: str = OUTPUT) -> str:
-    libdir = cuda_lib_dir()
     cmd = [nvcc_path(), "-gencode", GENCODE, "-lineinfo", "-O3", "-std=c++17",
            "-Xcompiler", "-fPIC", "-shared", "-I", os.path.join(ROOT, "include"),
-           "-o", output + ".tmp"] + SOURCES + [
-           "-L" + libdir, "-lcublasLt", "-Xlinker", "-rpath," + libdir]
+           "-o", output + ".tmp"] + SOURCES
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     res = subprocess.run(cmd, capture_output=True, text=True)

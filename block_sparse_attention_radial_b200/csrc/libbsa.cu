@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdint>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -20,6 +21,8 @@
 #include "attn_fwd_sm100.cuh"
 #include "dense_ref.cuh"
 #include "device_status.cuh"
+#include "gemm.h"
+#include "gemm_sm100.cuh"
 #include "lists.cuh"
 #include "patterns.cuh"
 
@@ -53,6 +56,7 @@ struct DeviceInfo {
   bool attrs_set[12] = {false, false, false, false, false, false,
                        false, false, false, false, false, false};
   bool ref_attrs_set[4] = {false, false, false, false};
+  bool gemm_attrs_set[4] = {false, false, false, false};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -631,7 +635,108 @@ __global__ void exp2_selftest_kernel(const float *x, float *y_poly, float *y_muf
   y_ref[2 * i + 1] = exp2f(v.y);
 }
 
+// A row-major bf16 matrix [outer][inner] (row stride `stride` elements) as a
+// 2-D tensor map with 128-byte swizzling and box {64, box_outer}: a K-major
+// operand tile (64 K values per row) or one 64-wide chunk of an MN-major one.
+// Out-of-range rows and columns read as zeros.
+int make_map_2d(CUtensorMap *map, const void *ptr, int64_t inner, int64_t outer, int64_t stride,
+                int box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    std::snprintf(t_last_error, sizeof(t_last_error), "cuTensorMapEncodeTiled not available");
+    return BSA_ERR_CUDA;
+  }
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(stride) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_outer)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(t_last_error, sizeof(t_last_error), "cuTensorMapEncodeTiled failed (%d)",
+                  static_cast<int>(r));
+    return BSA_ERR_CUDA;
+  }
+  return BSA_OK;
+}
+
+template <bool A_MN, bool B_MN>
+int launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
+                DeviceInfo *dev, cudaStream_t stream) {
+  const int slot = (A_MN ? 2 : 0) + (B_MN ? 1 : 0);
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!dev->gemm_attrs_set[slot]) {
+      BSA_CUDA(cudaFuncSetAttribute(gemm_bf16_sm100_kernel<A_MN, B_MN>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg::DSMEM));
+      dev->gemm_attrs_set[slot] = true;
+    }
+  }
+  const int grid = p.total_tiles < dev->sms ? p.total_tiles : dev->sms;
+  gemm_bf16_sm100_kernel<A_MN, B_MN><<<grid, GemmCfg::THREADS, GemmCfg::DSMEM, stream>>>(ta, tb,
+                                                                                       p);
+  BSA_CUDA(cudaGetLastError());
+  return BSA_OK;
+}
+
 }  // namespace
+
+int gemm_bf16(const void *a, int64_t lda, bool a_mn_major, const void *b, int64_t ldb,
+              bool b_mn_major, const void *bias, void *d, int64_t ldd, int64_t m, int64_t n,
+              int64_t k, cudaStream_t stream) {
+  if (!a || !b || !d) return BSA_ERR_INVALID_ARG;
+  constexpr int64_t kMaxDim = (int64_t(1) << 31) - 256;
+  if (m < 1 || n < 1 || k < 1 || m > kMaxDim || n > kMaxDim || k > kMaxDim)
+    return BSA_ERR_INVALID_ARG;
+  // 16-byte aligned bases and row strides (TMA, 16-byte output vectors);
+  // output rows hold whole 8-element vectors
+  if (!aligned16(a) || !aligned16(b) || !aligned16(d) || (lda & 7) || (ldb & 7) || (ldd & 7) ||
+      (n & 7))
+    return BSA_ERR_INVALID_ARG;
+  if (lda < (a_mn_major ? m : k) || ldb < (b_mn_major ? n : k) || ldd < n)
+    return BSA_ERR_INVALID_ARG;
+  if (lda >= (int64_t(1) << 39) || ldb >= (int64_t(1) << 39)) return BSA_ERR_INVALID_ARG;
+  const size_t a_span = static_cast<size_t>(((a_mn_major ? k : m) - 1) * lda + (a_mn_major ? m : k)) * 2;
+  const size_t b_span = static_cast<size_t>(((b_mn_major ? k : n) - 1) * ldb + (b_mn_major ? n : k)) * 2;
+  const size_t d_span = static_cast<size_t>((m - 1) * ldd + n) * 2;
+  if (overlaps(d, d_span, a, a_span) || overlaps(d, d_span, b, b_span) ||
+      (bias && overlaps(d, d_span, bias, static_cast<size_t>(n) * 2)))
+    return BSA_ERR_INVALID_ARG;
+  DeviceInfo *dev = nullptr;
+  int st;
+  if ((st = current_device(&dev)) != BSA_OK) return st;
+  if (dev->cc_major != 10) return BSA_ERR_UNSUPPORTED;
+  CUtensorMap ta, tb;
+  if ((st = a_mn_major ? make_map_2d(&ta, a, m, k, lda, GemmCfg::BK)
+                       : make_map_2d(&ta, a, k, m, lda, GemmCfg::BM)) != BSA_OK)
+    return st;
+  if ((st = b_mn_major ? make_map_2d(&tb, b, n, k, ldb, GemmCfg::BK)
+                       : make_map_2d(&tb, b, k, n, ldb, GemmCfg::BN)) != BSA_OK)
+    return st;
+  GemmParams p;
+  p.M = static_cast<int>(m);
+  p.N = static_cast<int>(n);
+  p.K = static_cast<int>(k);
+  p.d = static_cast<__nv_bfloat16 *>(d);
+  p.ldd = ldd;
+  p.bias = static_cast<const __nv_bfloat16 *>(bias);
+  p.tiles_m = static_cast<int>((m + GemmCfg::BM - 1) / GemmCfg::BM);
+  p.tiles_n = static_cast<int>((n + GemmCfg::BN - 1) / GemmCfg::BN);
+  if (static_cast<int64_t>(p.tiles_m) * p.tiles_n > INT32_MAX) return BSA_ERR_INVALID_ARG;
+  p.total_tiles = p.tiles_m * p.tiles_n;
+  p.k_blocks = static_cast<int>((k + GemmCfg::BK - 1) / GemmCfg::BK);
+  {
+    std::lock_guard<std::mutex> lk(g_hook_mu);
+    p.wait_limit_ns = g_wait_limit_ns;
+  }
+  if (a_mn_major)
+    return b_mn_major ? launch_gemm<true, true>(ta, tb, p, dev, stream)
+                      : launch_gemm<true, false>(ta, tb, p, dev, stream);
+  return b_mn_major ? launch_gemm<false, true>(ta, tb, p, dev, stream)
+                    : launch_gemm<false, false>(ta, tb, p, dev, stream);
+}
+
 }  // namespace bsa
 
 using namespace bsa;
@@ -1043,6 +1148,13 @@ int bsa_selftest_exp2(const float *x, float *y_poly, float *y_mufu, float *y_ref
   exp2_selftest_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(x, y_poly, y_mufu, y_ref, n);
   BSA_CUDA(cudaGetLastError());
   return BSA_OK;
+}
+
+int bsa_gemm_bf16(const void *a, int64_t lda, int32_t a_mn_major, const void *b, int64_t ldb,
+                  int32_t b_mn_major, const void *bias, void *d, int64_t ldd, int64_t m,
+                  int64_t n, int64_t k, bsa_stream_t stream) {
+  return gemm_bf16(a, lda, a_mn_major != 0, b, ldb, b_mn_major != 0, bias, d, ldd, m, n, k,
+                   reinterpret_cast<cudaStream_t>(stream));
 }
 
 int bsa_set_test_hooks(int64_t wait_limit_ns, int32_t fault_flags) {

@@ -1,4 +1,5 @@
-// libbsa: the radial attention module forward (bsa_attn_module_fwd).
+// libbsa: the radial attention module forward and backward
+// (bsa_attn_module_fwd, bsa_attn_module_bwd).
 //
 // The skill page's RadialAttention module ("Radial Attention" skill page,
 // Step 2, RadialAttention.__init__ / forward) projects x with three
@@ -12,36 +13,29 @@
 // through strided TMA descriptors; the attention writes its output in
 // [batch, n, heads, head_dim] order, which is already the row-major
 // [batch*n, C] operand of out_proj. No transpose or copy runs between the
-// three launches. The two projections are plain dense GEMMs and run on
-// cuBLASLt (bf16 inputs, fp32 accumulation, bf16 output).
+// three launches. Every GEMM, forward and backward, is the library's tcgen05
+// GEMM (gemm_sm100.cuh: bf16 inputs, fp32 accumulation in tensor memory,
+// bf16 output), which reads either operand in either orientation, so the
+// backward's transposed products need no transposed copies either.
 
-#include <cublasLt.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
 #include <cstdio>
-#include <map>
-#include <mutex>
-#include <tuple>
 
 #include "bsa.h"
+#include "gemm.h"
 
 namespace {
-
-constexpr size_t kGemmScratch = size_t(32) << 20;  // cuBLASLt workspace
-constexpr int kMaxDevices = 64;
-
-std::mutex g_lt_mu;
-cublasLtHandle_t g_lt[kMaxDevices] = {};
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Scratch layout inside the caller's forward workspace: the attention's work
 // order, the q/k/v projection, the attention output and lse (kept for the
-// backward), the GEMM scratch.
+// backward).
 struct ModuleLayout {
-  size_t order, qkv, attn, lse, gemm, total;
+  size_t order, qkv, attn, lse, total;
 };
 
 ModuleLayout module_layout(int32_t batch, int32_t n, int32_t heads, int32_t head_dim,
@@ -53,18 +47,17 @@ ModuleLayout module_layout(int32_t batch, int32_t n, int32_t heads, int32_t head
   w.qkv = align256(bsa_attn_fwd_workspace_bytes(batch, heads, l));
   w.attn = w.qkv + align256(rows * 3 * C * 2);
   w.lse = w.attn + align256(rows * C * 2);
-  w.gemm = w.lse + align256(rows * heads * sizeof(float));
-  w.total = w.gemm + kGemmScratch;
+  w.total = w.lse + align256(rows * heads * sizeof(float));
   return w;
 }
 
 // Scratch layout of the backward's own workspace: the attention output's
 // gradient, the q/k/v gradients, the attention backward's scratch, the
-// column-sum partials, the GEMM scratch.
+// column-sum partials.
 constexpr int kColsumChunks = 32;  // row chunks of the bias-gradient sums
 
 struct ModuleBwdLayout {
-  size_t dattn, dqkv, attn_ws, partial, gemm, total;
+  size_t dattn, dqkv, attn_ws, partial, total;
 };
 
 ModuleBwdLayout module_bwd_layout(int32_t batch, int32_t n, int32_t heads, int32_t head_dim,
@@ -76,8 +69,7 @@ ModuleBwdLayout module_bwd_layout(int32_t batch, int32_t n, int32_t heads, int32
   w.dqkv = align256(rows * C * 2);
   w.attn_ws = w.dqkv + align256(rows * 3 * C * 2);
   w.partial = w.attn_ws + align256(bsa_attn_bwd_workspace_bytes(batch, heads, n, l));
-  w.gemm = w.partial + align256(static_cast<size_t>(kColsumChunks) * 3 * C * sizeof(float));
-  w.total = w.gemm + kGemmScratch;
+  w.total = w.partial + align256(static_cast<size_t>(kColsumChunks) * 3 * C * sizeof(float));
   return w;
 }
 
@@ -155,110 +147,11 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int lt_handle(cublasLtHandle_t *h) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSA_ERR_CUDA;
-  std::lock_guard<std::mutex> lk(g_lt_mu);
-  if (!g_lt[dev] && cublasLtCreate(&g_lt[dev]) != CUBLAS_STATUS_SUCCESS) return BSA_ERR_CUDA;
-  *h = g_lt[dev];
-  return BSA_OK;
-}
-
-// Column-major GEMM on cuBLASLt: D (m x n, leading dimension ldd) =
-// op(A) (m x k) * op(B) (k x n) [+ bias[m] on every column], bf16 operands,
-// fp32 accumulation, bf16 D. Row-major matrices are their transposes in
-// these terms (see the callers).
-//
-// The descriptors and the algorithm cuBLASLt's heuristic picks are built once
-// per (device, shape, transposes, bias or not) and reused, so a call costs one
-// enqueue on the host (the heuristic query alone takes longer than a small
-// GEMM).
-struct GemmPlan {
-  int status = BSA_ERR_CUDA;
-  cublasLtMatmulDesc_t op = nullptr;
-  cublasLtMatrixLayout_t la = nullptr, lb = nullptr, lc = nullptr;
-  cublasLtMatmulAlgo_t algo;
-};
-
-struct GemmKey {
-  int dev;
-  bool ta, tb, bias;
-  int64_t m, n, k, lda, ldb, ldd;
-  bool operator<(const GemmKey &o) const {
-    return std::tie(dev, ta, tb, bias, m, n, k, lda, ldb, ldd) <
-           std::tie(o.dev, o.ta, o.tb, o.bias, o.m, o.n, o.k, o.lda, o.ldb, o.ldd);
-  }
-};
-
-std::mutex g_plan_mu;
-std::map<GemmKey, GemmPlan> g_plans;
-
-GemmPlan make_plan(cublasLtHandle_t h, const GemmKey &g) {
-  GemmPlan p;
-  if (cublasLtMatmulDescCreate(&p.op, CUBLAS_COMPUTE_32F, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS)
-    return p;
-  const cublasOperation_t tA = g.ta ? CUBLAS_OP_T : CUBLAS_OP_N;
-  const cublasOperation_t tB = g.tb ? CUBLAS_OP_T : CUBLAS_OP_N;
-  cublasLtMatmulDescSetAttribute(p.op, CUBLASLT_MATMUL_DESC_TRANSA, &tA, sizeof(tA));
-  cublasLtMatmulDescSetAttribute(p.op, CUBLASLT_MATMUL_DESC_TRANSB, &tB, sizeof(tB));
-  if (g.bias) {
-    const cublasLtEpilogue_t ep = CUBLASLT_EPILOGUE_BIAS;
-    const cudaDataType_t bt = CUDA_R_16BF;
-    cublasLtMatmulDescSetAttribute(p.op, CUBLASLT_MATMUL_DESC_EPILOGUE, &ep, sizeof(ep));
-    cublasLtMatmulDescSetAttribute(p.op, CUBLASLT_MATMUL_DESC_BIAS_DATA_TYPE, &bt, sizeof(bt));
-  }
-  // stored shapes: A is (ta ? k x m : m x k), B is (tb ? n x k : k x n)
-  if (cublasLtMatrixLayoutCreate(&p.la, CUDA_R_16BF, g.ta ? g.k : g.m, g.ta ? g.m : g.k, g.lda) !=
-          CUBLAS_STATUS_SUCCESS ||
-      cublasLtMatrixLayoutCreate(&p.lb, CUDA_R_16BF, g.tb ? g.n : g.k, g.tb ? g.k : g.n, g.ldb) !=
-          CUBLAS_STATUS_SUCCESS ||
-      cublasLtMatrixLayoutCreate(&p.lc, CUDA_R_16BF, g.m, g.n, g.ldd) != CUBLAS_STATUS_SUCCESS)
-    return p;
-  cublasLtMatmulPreference_t pref = nullptr;
-  if (cublasLtMatmulPreferenceCreate(&pref) != CUBLAS_STATUS_SUCCESS) return p;
-  const size_t scratch = kGemmScratch;
-  cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &scratch,
-                                       sizeof(scratch));
-  cublasLtMatmulHeuristicResult_t res;
-  int found = 0;
-  const cublasStatus_t hs =
-      cublasLtMatmulAlgoGetHeuristic(h, p.op, p.la, p.lb, p.lc, p.lc, pref, 1, &res, &found);
-  cublasLtMatmulPreferenceDestroy(pref);
-  if (hs != CUBLAS_STATUS_SUCCESS || found < 1) {
-    p.status = BSA_ERR_UNSUPPORTED;
-    return p;
-  }
-  p.algo = res.algo;
-  p.status = BSA_OK;
-  return p;
-}
-
-int gemm_bf16(cublasLtHandle_t h, bool ta, bool tb, int64_t m, int64_t n, int64_t k,
-              const void *A, int64_t lda, const void *B, int64_t ldb, void *D, int64_t ldd,
-              const void *bias, void *scratch, cudaStream_t stream) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
-  std::lock_guard<std::mutex> lk(g_plan_mu);  // the bias pointer is set on the shared desc
-  const GemmKey key{dev, ta, tb, bias != nullptr, m, n, k, lda, ldb, ldd};
-  auto it = g_plans.find(key);
-  if (it == g_plans.end()) it = g_plans.emplace(key, make_plan(h, key)).first;
-  GemmPlan &p = it->second;
-  if (p.status != BSA_OK) return p.status;
-  if (bias)
-    cublasLtMatmulDescSetAttribute(p.op, CUBLASLT_MATMUL_DESC_BIAS_POINTER, &bias, sizeof(bias));
-  const float alpha = 1.f, beta = 0.f;
-  if (cublasLtMatmul(h, p.op, &alpha, A, p.la, B, p.lb, &beta, D, p.lc, D, p.lc, &p.algo, scratch,
-                     kGemmScratch, stream) != CUBLAS_STATUS_SUCCESS)
-    return BSA_ERR_CUDA;
-  return BSA_OK;
-}
-
 // out[rows, m] (row-major) = a[rows, k] (row-major) * w[m, k]^T + bias[m]:
-// column-major out^T (m x rows) = op_T(w^T) * a^T, w's row-major storage being
-// the k x m column-major matrix w^T.
-int linear_bf16(cublasLtHandle_t h, const void *a, const void *w, const void *bias, void *out,
-                int64_t rows, int64_t m, int64_t k, void *scratch, cudaStream_t stream) {
-  return gemm_bf16(h, true, false, m, rows, k, w, k, a, k, out, m, bias, scratch, stream);
+// an nn.Linear layer, weight [out, in].
+int linear_bf16(const void *a, const void *w, const void *bias, void *out, int64_t rows,
+                int64_t m, int64_t k, cudaStream_t stream) {
+  return bsa::gemm_bf16(a, k, false, w, k, false, bias, out, m, rows, m, k, stream);
 }
 
 }  // namespace
@@ -300,14 +193,10 @@ int bsa_attn_module_fwd(const void *x, const void *w_qkv, const void *b_qkv, con
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   uint16_t *qkv = reinterpret_cast<uint16_t *>(ws + w.qkv);
   void *attn = ws + w.attn;
-  cublasLtHandle_t h;
   int st;
-  if ((st = lt_handle(&h)) != BSA_OK) return st;
 
   // (1) qkv[b*n + i, :] = x[b, i, :] [q_proj; k_proj; v_proj]^T + bias
-  if ((st = linear_bf16(h, x, w_qkv, b_qkv, qkv, rows, 3 * C, C, ws + w.gemm, stream)) !=
-      BSA_OK)
-    return st;
+  if ((st = linear_bf16(x, w_qkv, b_qkv, qkv, rows, 3 * C, C, stream)) != BSA_OK) return st;
   // (2) attention on the q / k / v column slices of qkv, output token-major
   bsa_layout lqkv, lo;
   lqkv.batch_stride = static_cast<int64_t>(n) * 3 * C;
@@ -322,7 +211,7 @@ int bsa_attn_module_fwd(const void *x, const void *w_qkv, const void *b_qkv, con
                                  stream_)) != BSA_OK)
     return st;
   // (3) y = attn out_proj^T + bias
-  return linear_bf16(h, attn, w_out, b_out, y, rows, C, C, ws + w.gemm, stream);
+  return linear_bf16(attn, w_out, b_out, y, rows, C, C, stream);
 }
 
 size_t bsa_attn_module_bwd_workspace_bytes(int32_t batch, int32_t n, int32_t heads,
@@ -382,19 +271,16 @@ int bsa_attn_module_bwd(const void *x, const void *w_qkv, const void *w_out, con
   uint16_t *dattn = reinterpret_cast<uint16_t *>(ws + w.dattn);
   uint16_t *dqkv = reinterpret_cast<uint16_t *>(ws + w.dqkv);
   float *partial = reinterpret_cast<float *>(ws + w.partial);
-  void *scratch = ws + w.gemm;
-  cublasLtHandle_t h;
   int st;
-  if ((st = lt_handle(&h)) != BSA_OK) return st;
 
-  // Row-major [r, c] matrices are column-major [c, r] below.
-  // (1) d_attn = dy w_out            : d_attn^T (C x rows) = w_out^T dy^T
-  if ((st = gemm_bf16(h, false, false, C, rows, C, w_out, C, dy, C, dattn, C, nullptr, scratch,
-                      stream)) != BSA_OK)
+  // Row-major products; "MN-major" operands are read transposed in place.
+  // (1) d_attn[rows, C] = dy[rows, C] w_out[C, C]
+  if ((st = bsa::gemm_bf16(dy, C, false, w_out, C, true, nullptr, dattn, C, rows, C, C,
+                           stream)) != BSA_OK)
     return st;
-  // (2) dw_out = dy^T attn           : dw_out^T (C x C) = attn^T dy
-  if ((st = gemm_bf16(h, false, true, C, C, rows, attn, C, dy, C, dw_out, C, nullptr, scratch,
-                      stream)) != BSA_OK)
+  // (2) dw_out[C, C] = dy^T attn   (both read from their [rows, C] storage)
+  if ((st = bsa::gemm_bf16(dy, C, true, attn, C, true, nullptr, dw_out, C, C, C, rows,
+                           stream)) != BSA_OK)
     return st;
   // (3) db_out = column sums of dy
   if (db_out && (st = colsum_bf16(dy, rows, static_cast<int>(C), partial, db_out, stream)) != BSA_OK)
@@ -413,17 +299,17 @@ int bsa_attn_module_bwd(const void *x, const void *w_qkv, const void *w_out, con
                                  dqkv, &lqkv, dqkv + C, &lqkv, dqkv + 2 * C, &lqkv,
                                  ws + w.attn_ws, w.partial - w.attn_ws, stream_)) != BSA_OK)
     return st;
-  // (5) dw_qkv = dqkv^T x            : dw_qkv^T (C x 3C) = x^T dqkv
-  if ((st = gemm_bf16(h, false, true, C, 3 * C, rows, x, C, dqkv, 3 * C, dw_qkv, C, nullptr,
-                      scratch, stream)) != BSA_OK)
+  // (5) dw_qkv[3C, C] = dqkv^T x   (both read from their [rows, .] storage)
+  if ((st = bsa::gemm_bf16(dqkv, 3 * C, true, x, C, true, nullptr, dw_qkv, C, 3 * C, C, rows,
+                           stream)) != BSA_OK)
     return st;
   // (6) db_qkv = column sums of dqkv
   if (db_qkv &&
       (st = colsum_bf16(dqkv, rows, static_cast<int>(3 * C), partial, db_qkv, stream)) != BSA_OK)
     return st;
-  // (7) dx = dqkv w_qkv              : dx^T (C x rows) = w_qkv^T dqkv^T
-  return gemm_bf16(h, false, false, C, rows, 3 * C, w_qkv, C, dqkv, 3 * C, dx, C, nullptr,
-                   scratch, stream);
+  // (7) dx[rows, C] = dqkv[rows, 3C] w_qkv[3C, C]
+  return bsa::gemm_bf16(dqkv, 3 * C, false, w_qkv, C, true, nullptr, dx, C, rows, C, 3 * C,
+                        stream);
 }
 
 }  // extern "C"

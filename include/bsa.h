@@ -296,8 +296,8 @@ int bsa_attn_fwd_strided(const void *q, const bsa_layout *q_layout,
 /*
  * Bytes of device scratch bsa_attn_module_fwd needs: the projected q/k/v
  * [batch*n, 3*heads*head_dim] bf16, the attention output [batch*n,
- * heads*head_dim] bf16, the attention's work order and 32 MiB of GEMM
- * scratch. Returns 0 for invalid arguments.
+ * heads*head_dim] bf16, its lse and the attention's work order. Returns 0
+ * for invalid arguments.
  */
 size_t bsa_attn_module_workspace_bytes(int32_t batch, int32_t n, int32_t heads,
                                        int32_t head_dim, const bsa_block_lists *lists);
@@ -321,8 +321,9 @@ size_t bsa_attn_module_workspace_bytes(int32_t batch, int32_t n, int32_t heads,
  *        the call (bsa_attn_module_bwd reads them).
  * Head h of the split is columns [h*head_dim, (h+1)*head_dim) of each
  * projection (the page's view(batch, n, heads, head_dim)). The projections
- * are cuBLASLt GEMMs (bf16 in, fp32 accumulate, bias in the epilogue, bf16
- * out); the attention reads q, k, v in place from the projection output and
+ * run on the library's tcgen05 GEMM (bsa_gemm_bf16: bf16 in, fp32
+ * accumulate, bias in the epilogue, bf16 out); the attention reads q, k, v in
+ * place from the projection output and
  * writes o in [batch, n, heads, head_dim] order, out_proj's input layout, so
  * no transpose runs. Pointers 16-byte aligned; other limits and errors as
  * bsa_attn_fwd. Asynchronous.
@@ -336,8 +337,8 @@ int bsa_attn_module_fwd(const void *x, const void *w_qkv, const void *b_qkv,
 /*
  * Bytes of device scratch bsa_attn_module_bwd needs: the attention output's
  * gradient [batch*n, C] and the q/k/v gradients [batch*n, 3C] (bf16), the
- * attention backward's workspace, bias-gradient partial sums and 32 MiB of
- * GEMM scratch. Returns 0 for invalid arguments.
+ * attention backward's workspace and the bias-gradient partial sums. Returns
+ * 0 for invalid arguments.
  */
 size_t bsa_attn_module_bwd_workspace_bytes(int32_t batch, int32_t n, int32_t heads,
                                            int32_t head_dim, const bsa_block_lists *lists);
@@ -359,9 +360,10 @@ size_t bsa_attn_module_bwd_workspace_bytes(int32_t batch, int32_t n, int32_t hea
  *   and db_out [C]: bf16 outputs or NULL (not computed). No output may
  *   overlap an input, a workspace or another output.
  * workspace: bsa_attn_module_bwd_workspace_bytes() of device scratch.
- * GEMMs on cuBLASLt (bf16 in, fp32 accumulate, bf16 out); bias gradients by a
- * fixed-order two-pass column sum (fp32), so the whole backward is
- * deterministic. 16-byte aligned pointers; limits and errors as bsa_attn_bwd.
+ * GEMMs on the library's tcgen05 GEMM (bsa_gemm_bf16: bf16 in, fp32
+ * accumulate, bf16 out; each output element is summed in one fixed order);
+ * bias gradients by a fixed-order two-pass column sum (fp32), so the whole
+ * backward is deterministic. 16-byte aligned pointers; limits and errors as bsa_attn_bwd.
  * Asynchronous.
  */
 int bsa_attn_module_bwd(const void *x, const void *w_qkv, const void *w_out, const void *dy,
@@ -370,6 +372,35 @@ int bsa_attn_module_bwd(const void *x, const void *w_qkv, const void *w_out, con
                         const void *fwd_workspace, size_t fwd_workspace_bytes,
                         void *dx, void *dw_qkv, void *db_qkv, void *dw_out, void *db_out,
                         void *workspace, size_t workspace_bytes, bsa_stream_t stream);
+
+/*
+ * Dense bf16 matrix product of the module's linear layers ("Radial Attention"
+ * skill page, Step 2: q_proj, k_proj, v_proj and out_proj are nn.Linear
+ * layers, y = x W^T + b; the backward multiplies by W and by the transposed
+ * activations):
+ *   D[m, n] = A[m, k] B[k, n] (+ bias[n] on every row),
+ * bf16 operands, fp32 accumulation on the tensor cores (tcgen05, TMEM
+ * accumulators), rounded to bf16 once on output.
+ * a, lda, a_mn_major  A stored row-major as [m][k] (a_mn_major = 0, row stride
+ *        lda >= k) or as its transpose [k][m] (a_mn_major = 1, lda >= m).
+ * b, ldb, b_mn_major  B stored as [n][k] (b_mn_major = 0, ldb >= k: an
+ *        nn.Linear weight [out, in], giving x W^T) or as [k][n]
+ *        (b_mn_major = 1, ldb >= n).
+ * bias   device bf16 [n] or NULL.
+ * d, ldd device bf16 output [m][n], row stride ldd >= n; must not overlap a,
+ *        b or bias.
+ * Device pointers 16-byte aligned; lda, ldb, ldd and n multiples of 8;
+ * m, n, k in [1, 2^31 - 256]. Every output element is the sum over k in one
+ * fixed order (results are reproducible bit for bit). Returns
+ * BSA_ERR_INVALID_ARG for bad arguments (nothing launched),
+ * BSA_ERR_UNSUPPORTED on a device other than sm_100, BSA_ERR_CUDA on a launch
+ * error; a device-side wait that runs out is reported through
+ * bsa_get_device_status(). Asynchronous on `stream`.
+ */
+int bsa_gemm_bf16(const void *a, int64_t lda, int32_t a_mn_major,
+                  const void *b, int64_t ldb, int32_t b_mn_major,
+                  const void *bias, void *d, int64_t ldd,
+                  int64_t m, int64_t n, int64_t k, bsa_stream_t stream);
 
 /*
  * Same operation, same arguments (no workspace), computed by a plain fp32

@@ -197,13 +197,13 @@ def test_module_workspace_and_host_checks(lib):
     vp, ref = ctypes.c_void_p, ctypes.byref
     ls = BlockListsC(1, 256, 256, 128, 1000, 0, 0)
     # work order and counter (1 KiB + 256) + q/k/v [32760, 15360] + attention out
-    # [32760, 5120] bf16 + lse [40, 32760] fp32 + 32 MiB
-    expect = 1280 + 32760 * 15360 * 2 + 32760 * 5120 * 2 + 40 * 32760 * 4 + (32 << 20)
+    # [32760, 5120] bf16 + lse [40, 32760] fp32 (the GEMMs need no scratch)
+    expect = 1280 + 32760 * 15360 * 2 + 32760 * 5120 * 2 + 40 * 32760 * 4
     assert lib.bsa_attn_module_workspace_bytes(1, 32760, 40, 128, ref(ls)) == expect
     # backward: dA [32760, 5120] + dQKV [32760, 15360] bf16 + the attention
-    # backward's workspace + 32 x 15360 fp32 partial sums + 32 MiB
+    # backward's workspace + 32 x 15360 fp32 partial sums
     attn_bwd = lib.bsa_attn_bwd_workspace_bytes(1, 40, 32760, ref(ls))
-    expect_b = 32760 * 5120 * 2 + 32760 * 15360 * 2 + attn_bwd + 32 * 15360 * 4 + (32 << 20)
+    expect_b = 32760 * 5120 * 2 + 32760 * 15360 * 2 + attn_bwd + 32 * 15360 * 4
     assert lib.bsa_attn_module_bwd_workspace_bytes(1, 32760, 40, 128, ref(ls)) == expect_b
     assert lib.bsa_attn_module_workspace_bytes(1, 32760, 40, 128, None) == 0
     B, n, H, D = 1, 1000, 2, 64
@@ -370,3 +370,29 @@ int main(void) {
     assert out[1] == lib.bsa_status_string(6).decode()
     assert out[2] == "1"                         # BSA_ERR_INVALID_ARG, found on the host
     assert out[3] == str(37 * 4)
+
+
+def test_gemm_host_checks(lib):
+    """bsa_gemm_bf16 rejects bad shapes, strides, alignment and overlapping
+    output on the host, before any CUDA call."""
+    vp = ctypes.c_void_p
+    a, b, d, bias = (vp(x << 30) for x in (1, 2, 3, 4))
+
+    def call(a=a, lda=256, amn=0, b=b, ldb=256, bmn=0, bias=None, d=d, ldd=512, m=100, n=512,
+             k=256):
+        return lib.bsa_gemm_bf16(a, lda, amn, b, ldb, bmn, bias, d, ldd, m, n, k, None)
+
+    assert call(m=0) == 1 and call(n=0) == 1 and call(k=0) == 1
+    assert call(n=500, ldd=504) == 1                 # n not a multiple of 8
+    assert call(lda=252, k=250) == 1                 # lda not a multiple of 8
+    assert call(lda=128) == 1                        # K-major A: lda < k
+    assert call(amn=1, lda=96) == 1                  # MN-major A: lda < m
+    assert call(ldb=128) == 1                        # B stored [n][k]: ldb < k
+    assert call(bmn=1, ldb=256) == 1                 # B stored [k][n]: ldb < n
+    assert call(ldd=256) == 1                        # ldd < n
+    assert call(a=vp((1 << 30) + 8)) == 1            # misaligned A
+    assert call(d=vp((3 << 30) + 2)) == 1            # misaligned D
+    assert call(d=vp((1 << 30) + 1024)) == 1         # D inside A's span
+    assert call(d=vp((2 << 30) + 4096)) == 1         # D inside B's span
+    assert call(bias=vp((3 << 30) + 64)) == 1        # bias inside D's span
+    assert call(a=None) == 1
