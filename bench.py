@@ -902,6 +902,78 @@ def run_ours_module(args, world, rank, local, backward=False):
     return 0
 
 
+METRIC_GEMM = "bf16 GEMM ms & TFLOP/s of the module's linear layers (Wan width)"
+GEMM_SHAPES = {  # name: (m, n, k, A MN-major, B MN-major), rows = 21 x 1560 tokens, C = 5120
+    "qkv": (32760, 15360, 5120, False, False),
+    "out": (32760, 5120, 5120, False, False),
+    "dattn": (32760, 5120, 5120, False, True),
+    "dw_out": (5120, 5120, 32760, True, True),
+    "dw_qkv": (15360, 5120, 32760, True, True),
+    "dx": (32760, 5120, 15360, False, True),
+}
+
+
+def run_gemm(args, world, rank, local):
+    """The module's six GEMM shapes (forward projections and backward
+    products) through bsa_gemm_bf16, each timed with CUDA events; with
+    --gemm-vs-torch also torch.matmul on the same operands, for context."""
+    import torch
+
+    import block_sparse_attention_radial_b200 as bsa
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    names = list(GEMM_SHAPES) if args.gemm_shape == "all" else [args.gemm_shape]
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    res = {}
+    for name in names:
+        m, n, k, amn, bmn = GEMM_SHAPES[name]
+        a = torch.randn((k, m) if amn else (m, k), generator=g, device=dev).to(torch.bfloat16)
+        b = torch.randn((k, n) if bmn else (n, k), generator=g, device=dev).to(torch.bfloat16)
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        arms = [("ours", lambda: bsa.bsa_gemm_bf16(a, b, out, None, amn, bmn))]
+        if args.gemm_vs_torch:
+            arms.append(("torch_matmul", lambda: torch.matmul(a.t() if amn else a,
+                                                              b if bmn else b.t(), out=out)))
+        r = {"m": m, "n": n, "k": k, "a_mn_major": amn, "b_mn_major": bmn}
+        for tag, fn in arms:
+            for _ in range(args.warmup):
+                fn()
+            torch.cuda.synchronize(dev)
+            ts = []
+            for _ in range(args.steps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize(dev)
+                ts.append(e0.elapsed_time(e1))
+            ms = statistics.median(ts)
+            r[tag] = {"ms": ms, "tflops": 2 * m * n * k / ms / 1e9}
+        if bsa.bsa_get_device_status() != 0:
+            raise SystemExit("device status after the GEMMs")
+        res[name] = r
+        del a, b, out
+        torch.cuda.empty_cache()
+    head = names[0]
+    achieved = res[head]["ours"]["tflops"]
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC_GEMM, "value": achieved, "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "dtype": "bf16", "data": "synthetic", "config": {"workload": f"gemm {head}"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "peak_kind": f"{peak_kind} bf16 burst",
+                         "kernel": "gemm_bf16_sm100_kernel"},
+            "shapes": res}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -916,10 +988,16 @@ def main(argv=None):
     ap.add_argument("--per-config-steps", type=int, default=10,
                     help="timed steps for each of the other forward configurations recorded "
                          "under per_config in the default (wan, one GPU) run; 0 skips them")
-    ap.add_argument("--pass", dest="which", choices=("fwd", "bwd", "module", "module_bwd"),
+    ap.add_argument("--gemm-shape", default="all", choices=("all",) + tuple(GEMM_SHAPES),
+                    help="--pass gemm: one of the module's GEMM shapes, or all six")
+    ap.add_argument("--gemm-vs-torch", action="store_true",
+                    help="--pass gemm: also time torch.matmul on the same operands")
+    ap.add_argument("--pass", dest="which",
+                    choices=("fwd", "bwd", "module", "module_bwd", "gemm"),
                     default="fwd",
-                    help="time the forward (default, the headline), the backward pass, or the "
-                         "whole module forward / backward (projections + attention)")
+                    help="time the forward (default, the headline), the backward pass, the "
+                         "whole module forward / backward (projections + attention), or the "
+                         "module's GEMMs alone")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -935,6 +1013,8 @@ def main(argv=None):
         return run_ours_bwd(args, world, rank, local)
     if args.which in ("module", "module_bwd"):
         return run_ours_module(args, world, rank, local, backward=args.which == "module_bwd")
+    if args.which == "gemm":
+        return run_gemm(args, world, rank, local)
     return run_ours(args, world, rank, local)
 
 

@@ -88,3 +88,11 @@ def test_per_config_names_cover_the_metric_range():
         w = WORKLOADS[name]
         assert w.n >= 32 * 1024 and w.block == 128 and w.head_dim == 128
     assert max(WORKLOADS[n].n for n in names) == 84 * 1560
+
+
+def test_gemm_shapes_are_the_module_products():
+    rows, C = 21 * 1560, 40 * 128
+    s = bench.GEMM_SHAPES
+    assert s["qkv"][:3] == (rows, 3 * C, C) and s["out"][:3] == (rows, C, C)
+    assert s["dw_qkv"][:3] == (3 * C, C, rows) and s["dx"][:3] == (rows, C, 3 * C)
+    assert all(m % 8 == 0 or not amn for m, n, k, amn, bmn in s.values())
