@@ -28,7 +28,8 @@ __all__ = [
     "bsa_get_timeout_detail", "bsa_status_string", "bsa_last_cuda_error", "bsa_set_test_hooks",
     "radial_block_lists", "block_lists_from_csr", "attention", "dense_masked_reference",
     "computed_flops", "bsa_attn_fwd_noalloc", "bsa_selftest_exp2", "NOALLOC_MAX_ORDER_ENTRIES",
-    "bsa_gemm_bf16",
+    "bsa_gemm_bf16", "bsa_joint_mask_build_varlen", "bsa_attn_fwd_varlen",
+    "bsa_attn_fwd_varlen_workspace_bytes", "radial_block_lists_varlen", "attention_varlen",
     "bsa_attn_fwd_strided", "bsa_attn_module_workspace_bytes", "bsa_joint_mask_build",
     "bsa_attn_fwd_host", "bsa_attn_fwd_host_workspace_bytes", "bsa_attn_bwd_strided",
     "bsa_attn_module_bwd", "bsa_attn_module_bwd_workspace_bytes", "attention_module_backward", "bsa_attn_module_fwd",
@@ -75,10 +76,11 @@ class BlockLists:
     num_lists: int
     num_q_blocks: int
     block: int
+    k_blocks: int = 0           # key blocks when they differ from num_q_blocks (varlen: the widest item)
 
     @property
     def num_k_blocks(self) -> int:
-        return self.num_q_blocks
+        return self.k_blocks or self.num_q_blocks
 
     @property
     def nnz(self) -> int:
@@ -118,6 +120,23 @@ def bsa_joint_mask_build(frames: int, tokens_per_frame: int, text_tokens: int, b
                                   _ptr(col_idx), col_capacity if col_idx is not None else 0,
                                   ctypes.byref(nnz) if want_nnz else None, _stream(stream))
     _check(st, "bsa_joint_mask_build")
+    return int(nnz.value) if want_nnz else None
+
+
+def bsa_joint_mask_build_varlen(items, block: int, row_ptr: torch.Tensor,
+                                col_idx: torch.Tensor | None = None, col_capacity: int = 0,
+                                want_nnz: bool = True, stream=None) -> int | None:
+    """Concatenated joint lists of a variable-length batch: ``items`` is a list of
+    (frames, tokens_per_frame, text_tokens); returns nnz when asked."""
+    lib = _lib.load()
+    k = len(items)
+    arr = ctypes.c_int32 * max(k, 1)
+    fr, tp, tx = (arr(*[int(it[i]) for it in items]) for i in range(3))
+    nnz = ctypes.c_int64(-1)
+    st = lib.bsa_joint_mask_build_varlen(k, fr, tp, tx, block, _ptr(row_ptr), _ptr(col_idx),
+                                         col_capacity if col_idx is not None else 0,
+                                         ctypes.byref(nnz) if want_nnz else None, _stream(stream))
+    _check(st, "bsa_joint_mask_build_varlen")
     return int(nnz.value) if want_nnz else None
 
 
@@ -186,6 +205,43 @@ def bsa_attn_fwd_strided(q, k, v, lists: BlockLists, out, lse=None, workspace=No
                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
                                   _stream(stream))
     _check(st, "bsa_attn_fwd_strided")
+
+
+def _cu_array(cu_seqlens):
+    cu = [int(c) for c in cu_seqlens]
+    return len(cu) - 1, (ctypes.c_int32 * len(cu))(*cu)
+
+
+def bsa_attn_fwd_varlen_workspace_bytes(cu_seqlens, heads: int, lists: BlockLists) -> int:
+    k, cu = _cu_array(cu_seqlens)
+    return int(_lib.load().bsa_attn_fwd_varlen_workspace_bytes(k, cu, heads,
+                                                               ctypes.byref(lists.c_struct())))
+
+
+def bsa_attn_fwd_varlen(q, k, v, cu_seqlens, lists: BlockLists, out, lse=None, workspace=None,
+                        softmax_scale: float = 0.0, stream=None) -> None:
+    """Variable-length batch forward on packed [total, heads, head_dim] tensors
+    (item b = tokens cu_seqlens[b]..cu_seqlens[b+1]); lse is [heads, total]."""
+    total, H, D = q.shape
+    lib = _lib.load()
+    ls = lists.c_struct()
+    nitems, cu = _cu_array(cu_seqlens)
+    if workspace is None:
+        workspace = torch.empty(max(lib.bsa_attn_fwd_varlen_workspace_bytes(
+            nitems, cu, H, ctypes.byref(ls)), 16), dtype=torch.uint8, device=q.device)
+
+    def lay(t):
+        if t.dim() != 3 or t.stride(2) != 1:
+            raise ValueError("expected a [total, heads, head_dim] view with a contiguous last axis")
+        return LayoutC(0, t.stride(1), t.stride(0))
+
+    lq, lk, lv, lo = (lay(t) for t in (q, k, v, out))
+    st = lib.bsa_attn_fwd_varlen(_ptr(q), ctypes.byref(lq), _ptr(k), ctypes.byref(lk), _ptr(v),
+                                 ctypes.byref(lv), nitems, cu, H, D, float(softmax_scale),
+                                 ctypes.byref(ls), _ptr(out), ctypes.byref(lo), _ptr(lse),
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                 _stream(stream))
+    _check(st, "bsa_attn_fwd_varlen")
 
 
 def bsa_attn_fwd_host_workspace_bytes(batch: int, heads: int, n: int, head_dim: int,
@@ -445,6 +501,31 @@ def radial_block_lists(frames: int, tokens_per_frame: int, block: int = 128,
                                col_idx.numel(), stream=stream)
     assert got == nnz
     return BlockLists(row_ptr, col_idx[:nnz], 1, nqb, block)
+
+
+def radial_block_lists_varlen(items, block: int = 128, device=None, stream=None) -> BlockLists:
+    """Concatenated joint lists of a variable-length batch on the GPU; ``items``
+    is a list of (frames, tokens_per_frame, text_tokens)."""
+    device = torch.device("cuda") if device is None else torch.device(device)
+    nqbs = [-(-(f * s + t) // block) for f, s, t in items]
+    row_ptr = torch.empty(sum(nqbs) + 1, dtype=torch.int32, device=device)
+    nnz = bsa_joint_mask_build_varlen(items, block, row_ptr, stream=stream)
+    col_idx = torch.empty(max(nnz, 1), dtype=torch.int32, device=device)
+    got = bsa_joint_mask_build_varlen(items, block, row_ptr, col_idx, col_idx.numel(),
+                                      stream=stream)
+    assert got == nnz
+    return BlockLists(row_ptr, col_idx[:nnz], 1, sum(nqbs), block, k_blocks=max(nqbs))
+
+
+def attention_varlen(q, k, v, cu_seqlens, lists: BlockLists, softmax_scale: float = 0.0,
+                     want_lse: bool = True, stream=None):
+    """Variable-length batch on packed [total, heads, head_dim] q, k, v; returns
+    ``(out [total, heads, head_dim], lse [heads, total])``."""
+    total, H, D = q.shape
+    out = torch.empty_like(q)
+    lse = torch.empty((H, total), dtype=torch.float32, device=q.device) if want_lse else None
+    bsa_attn_fwd_varlen(q, k, v, cu_seqlens, lists, out, lse, None, softmax_scale, stream)
+    return out, lse
 
 
 def pack_tile_patterns(patterns, device=None):

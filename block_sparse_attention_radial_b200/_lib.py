@@ -17,10 +17,13 @@ LIB_PATH = os.path.join(_HERE, "libbsa.so")
 EXPORTS = (
     "bsa_radial_mask_build",
     "bsa_joint_mask_build",
+    "bsa_joint_mask_build_varlen",
     "bsa_tile_pattern_lists_build",
     "bsa_attn_fwd_workspace_bytes",
     "bsa_attn_fwd",
     "bsa_attn_fwd_strided",
+    "bsa_attn_fwd_varlen_workspace_bytes",
+    "bsa_attn_fwd_varlen",
     "bsa_attn_fwd_host_workspace_bytes",
     "bsa_attn_fwd_host",
     "bsa_attn_module_workspace_bytes",
@@ -119,6 +122,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                                 ctypes.POINTER(i64), vp]),
         "bsa_tile_pattern_lists_build": (ctypes.c_int, [i32, i32, vp, vp, i64, vp, vp, i64,
                                                         ctypes.POINTER(i64), vp]),
+        "bsa_joint_mask_build_varlen": (ctypes.c_int, [i32, vp, vp, vp, i32, vp, vp, i64,
+                                                       ctypes.POINTER(i64), vp]),
+        "bsa_attn_fwd_varlen_workspace_bytes": (sz, [i32, vp, i32, lp]),
+        "bsa_attn_fwd_varlen": (ctypes.c_int, [vp, yp, vp, yp, vp, yp, i32, vp, i32, i32,
+                                               ctypes.c_float, lp, vp, yp, vp, vp, sz, vp]),
         "bsa_attn_fwd_workspace_bytes": (sz, [i32, i32, lp]),
         "bsa_attn_fwd": (ctypes.c_int, [vp, vp, vp, i32, i32, i32, i32, ctypes.c_float, lp,
                                         vp, vp, vp, sz, vp]),

@@ -77,10 +77,10 @@ struct RowReader {
   __device__ __forceinline__ int fetch() const {
     return left > 0 ? min(max(__ldg(ptr), 0), hi) : INT_MAX;
   }
-  __device__ __forceinline__ void reset(const FwdParams &p, int a, int len) {
+  __device__ __forceinline__ void reset(const FwdParams &p, int a, int len, int nkb) {
     ptr = p.col_idx + a;
     left = len;
-    hi = p.nkb - 1;
+    hi = nkb - 1;
     nxt = fetch();
   }
   __device__ __forceinline__ void pop() {
@@ -94,9 +94,10 @@ struct RowReader {
 // rows by one thread (the producer and the MMA issuer run identical walks).
 struct UnionWalker {
   RowReader ra, rb;
-  __device__ __forceinline__ void reset(const FwdParams &p, int a0, int lenA, int b0, int lenB) {
-    ra.reset(p, a0, lenA);
-    rb.reset(p, b0, lenB);
+  __device__ __forceinline__ void reset(const FwdParams &p, int a0, int lenA, int b0, int lenB,
+                                        int nkb) {
+    ra.reset(p, a0, lenA, nkb);
+    rb.reset(p, b0, lenB, nkb);
   }
   // Next union block: false when both rows are exhausted.
   __device__ __forceinline__ bool next(int &kb, bool &inA, bool &inB) {
@@ -113,23 +114,34 @@ struct UnionWalker {
 
 constexpr int kItemN = 4;  // work items in flight between the producer and the consumers
 
-struct PairItem {
-  int bh, qa, a0, lenA, b0, lenB;  // tile B absent (lenB = 0) past the last block
+// Variable-length batches: the batch is one packed token sequence (batch
+// extent 1 in the views) holding num_items items one after the other; item b
+// owns tokens [tok0[b], tok0[b+1]), query-block rows [row0[b], row0[b+1]) of
+// every list (its key blocks counted from 0 inside the item), work-order
+// entries [pair0[b], pair0[b+1]) of every list and work items
+// [work0[b], work0[b+1]) (heads x its query-block pairs). Passed by value as
+// a kernel parameter.
+constexpr int kMaxVarlenItems = 64;
+struct VarlenTable {
+  int32_t num_items;
+  int32_t tok0[kMaxVarlenItems + 1];
+  int32_t row0[kMaxVarlenItems + 1];
+  int32_t pair0[kMaxVarlenItems + 1];
+  int32_t work0[kMaxVarlenItems + 1];
 };
 
-__device__ __forceinline__ PairItem decode_pair(int idx, const FwdParams &p, int npairs) {
-  PairItem it;
-  it.bh = idx / npairs;
-  const int rank = idx - it.bh * npairs;
-  const int list = p.num_lists > 1 ? (it.bh % p.heads) : 0;
-  const long long lbase = static_cast<long long>(list) * p.nqb;
-  const int pr = min(max(p.order[static_cast<long long>(list) * npairs + rank], 0), npairs - 1);
-  it.qa = 2 * pr;
+struct PairItem {
+  int bh, qa, a0, lenA, b0, lenB;  // tile B absent (lenB = 0) past the last block
+  int n, nqb, nkb, tok0;           // the item's tokens, query and key blocks, first token
+};
+
+// Rows qa and qa + 1 (when it exists) of the list starting at row lbase.
+__device__ __forceinline__ void pair_rows(const FwdParams &p, long long lbase, PairItem &it) {
   const int a = min(max(p.row_ptr[lbase + it.qa], 0), p.nnz);
   const int ae = min(max(p.row_ptr[lbase + it.qa + 1], 0), p.nnz);
   it.a0 = a;
   it.lenA = max(ae - a, 0);
-  if (it.qa + 1 < p.nqb) {
+  if (it.qa + 1 < it.nqb) {
     const int b = min(max(p.row_ptr[lbase + it.qa + 1], 0), p.nnz);
     const int be = min(max(p.row_ptr[lbase + it.qa + 2], 0), p.nnz);
     it.b0 = b;
@@ -138,6 +150,53 @@ __device__ __forceinline__ PairItem decode_pair(int idx, const FwdParams &p, int
     it.b0 = 0;
     it.lenB = 0;
   }
+}
+
+template <bool VARLEN>
+__device__ __forceinline__ PairItem decode_pair(int idx, const FwdParams &p, int npairs,
+                                                const VarlenTable &vt) {
+  PairItem it;
+  if (!VARLEN) {
+    it.n = p.n;
+    it.nqb = p.nqb;
+    it.nkb = p.nkb;
+    it.tok0 = 0;
+    it.bh = idx / npairs;
+    const int rank = idx - it.bh * npairs;
+    const int list = p.num_lists > 1 ? (it.bh % p.heads) : 0;
+    const long long lbase = static_cast<long long>(list) * p.nqb;
+    const int pr = min(max(p.order[static_cast<long long>(list) * npairs + rank], 0), npairs - 1);
+    it.qa = 2 * pr;
+    pair_rows(p, lbase, it);
+    return it;
+  }
+  // the item holding work index idx: the last b with work0[b] <= idx (items
+  // without work share their work0 with the next item and are skipped)
+  int lo = 0, hi = vt.num_items - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (vt.work0[mid] <= idx)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  const int b = lo;
+  it.tok0 = vt.tok0[b];
+  it.n = vt.tok0[b + 1] - it.tok0;
+  it.nqb = vt.row0[b + 1] - vt.row0[b];
+  it.nkb = it.nqb;
+  const int np = vt.pair0[b + 1] - vt.pair0[b];
+  const int local = idx - vt.work0[b];
+  it.bh = local / np;  // the head (batch extent 1)
+  const int rank = local - it.bh * np;
+  const int list = p.num_lists > 1 ? it.bh : 0;
+  const long long lbase = static_cast<long long>(p.num_lists) * vt.row0[b] +
+                          static_cast<long long>(list) * it.nqb;
+  const long long obase = static_cast<long long>(p.num_lists) * vt.pair0[b] +
+                          static_cast<long long>(list) * np;
+  const int pr = min(max(p.order[obase + rank], 0), np - 1);
+  it.qa = 2 * pr;
+  pair_rows(p, lbase, it);
   return it;
 }
 
@@ -185,11 +244,12 @@ __device__ __forceinline__ bool plan_wait(const volatile uint32_t *ring, uint32_
   }
 }
 
-template <int D>
+template <int D, bool VARLEN>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_pair_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k,
-                               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                               const __grid_constant__ CUtensorMap tm_v, const FwdParams p,
+                               const __grid_constant__ VarlenTable vt) {
   using C = PairCfg<D>;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t dsmem[];
@@ -278,19 +338,20 @@ __global__ void __launch_bounds__(384, 1)
           item_ring[slot] = idx;
           mbar_arrive(&bar_item_full[slot]);
           if (idx < 0) break;
-          const PairItem it = decode_pair(idx, p, npairs);
+          const PairItem it = decode_pair<VARLEN>(idx, p, npairs, vt);
           if (it.lenA == 0 && it.lenB == 0) continue;
           if (!(ok = lane_wait(&bar_q_empty, (qcount & 1u) ^ 1u, wc, kBarQEmpty, qcount))) break;
           mbar_arrive_expect_tx(&bar_q_full, 2 * C::Q_BYTES);
           const int ib = it.bh / p.heads, ih = it.bh - ib * p.heads;
-          tma_load_5d(sQ, &tm_q, &bar_q_full, 0, it.qa * BN, 0, ih, ib);
-          tma_load_5d(sQ + C::Q_BYTES, &tm_q, &bar_q_full, 0, (it.qa + 1) * BN, 0, ih, ib);
+          tma_load_5d(sQ, &tm_q, &bar_q_full, 0, it.tok0 + it.qa * BN, 0, ih, ib);
+          tma_load_5d(sQ + C::Q_BYTES, &tm_q, &bar_q_full, 0, it.tok0 + (it.qa + 1) * BN, 0, ih,
+                      ib);
           ++qcount;
           // Same walk and same first-use order as the MMA issuer: at step j it
           // needs V(j-1) first when tile A listed j-1 or A skips j, and K(j)
           // first otherwise.
           UnionWalker uw;
-          uw.reset(p, it.a0, it.lenA, it.b0, it.lenB);
+          uw.reset(p, it.a0, it.lenA, it.b0, it.lenB, it.nkb);
           bool pa = false, pb = false;
           int prev_kb = 0;
           while (ok) {
@@ -327,7 +388,7 @@ __global__ void __launch_bounds__(384, 1)
               }
               mbar_arrive_expect_tx(&bar_kv_full[s], C::TILE_BYTES);
               tma_load_5d(sKV + s * C::TILE_BYTES, is_v ? &tm_v : &tm_k, &bar_kv_full[s], 0,
-                          (is_v ? prev_kb : kb) * BN, 0, ih, ib);
+                          it.tok0 + (is_v ? prev_kb : kb) * BN, 0, ih, ib);
               ++ring;
             }
             pa = a;
@@ -376,7 +437,7 @@ __global__ void __launch_bounds__(384, 1)
           const int idx = *static_cast<volatile int *>(&item_ring[slot]);
           mbar_arrive(&bar_item_empty[slot]);
           if (idx < 0) break;
-          const PairItem it = decode_pair(idx, p, npairs);
+          const PairItem it = decode_pair<VARLEN>(idx, p, npairs, vt);
           if (it.lenA == 0 && it.lenB == 0) continue;
           if (!(ok = lane_wait(&bar_q_full, qcount & 1u, wc, kBarQFull, qcount))) break;
           tc_fence_after();
@@ -507,16 +568,17 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_item_empty[slot]);
       if (idx < 0) break;
-      const PairItem it = decode_pair(idx, p, npairs);
+      const PairItem it = decode_pair<VARLEN>(idx, p, npairs, vt);
       const int qb = it.qa + t;
-      if (qb >= p.nqb) continue;
+      if (qb >= it.nqb) continue;
       const int len = t == 0 ? it.lenA : it.lenB;
       const int a0 = t == 0 ? it.a0 : it.b0;
       const int row = qb * BN + row_in_tile;
-      const bool store = row < p.n;
-      const long long orow = static_cast<long long>(it.bh) * p.n + row;
+      const bool store = row < it.n;
+      const long long orow = static_cast<long long>(it.bh) * p.n + it.tok0 + row;
       const int ib = it.bh / p.heads, ih = it.bh - ib * p.heads;
-      __nv_bfloat16 *const orow_ptr = p.out + ib * p.o_sb + ih * p.o_sh + row * p.o_sn;
+      __nv_bfloat16 *const orow_ptr =
+          p.out + ib * p.o_sb + ih * p.o_sh + static_cast<long long>(it.tok0 + row) * p.o_sn;
       if (len == 0) {
         if (store) {
           uint4 *dst = reinterpret_cast<uint4 *>(orow_ptr);
@@ -528,8 +590,8 @@ __global__ void __launch_bounds__(384, 1)
       }
       // Lists are sorted, so only the row's last block can be the ragged
       // final key block; its valid column count is taken once per item.
-      const int last_kb = min(max(__ldg(p.col_idx + a0 + len - 1), 0), p.nkb - 1);
-      const int last_valid = min(p.n - last_kb * BN, BN);
+      const int last_kb = min(max(__ldg(p.col_idx + a0 + len - 1), 0), it.nkb - 1);
+      const int last_valid = min(it.n - last_kb * BN, BN);
       float m_ref = 0.f, l = 0.f;
       for (int j = 0; j < len; ++j) {
         if (!(ok = warp_wait(&bar_s_full[t], scnt & 1u, wc, kBarSFull, scnt))) break;

@@ -333,26 +333,40 @@ int launch_ref(const RefParams &p, int batch, DeviceInfo *dev, int slot, cudaStr
 
 int slot_of(int D, int BN) { return (D == 128 ? 2 : 0) + (BN == 128 ? 1 : 0); }
 
+// The two-tile kernel; `vt` (variable-length batches) or null (a regular
+// batch). For a variable-length batch, x.batch is 1 and n the total tokens.
 template <int D>
 int launch_pair(const QkvViews &x, int32_t n, const FwdParams &p, DeviceInfo *dev,
-                cudaStream_t stream) {
+                const VarlenTable *vt, cudaStream_t stream) {
   using C = PairCfg<D>;
   CUtensorMap tq, tk, tv;
   int st;
   if ((st = make_map_strided(&tq, x.q, x.lq, x.batch, x.heads, n, D, C::BN)) != BSA_OK) return st;
   if ((st = make_map_strided(&tk, x.k, x.lk, x.batch, x.heads, n, D, C::BN)) != BSA_OK) return st;
   if ((st = make_map_strided(&tv, x.v, x.lv, x.batch, x.heads, n, D, C::BN)) != BSA_OK) return st;
-  const int slot = 4 + (D == 128 ? 1 : 0);
+  const int slot = (vt ? 6 : 4) + (D == 128 ? 1 : 0);
   {
     std::lock_guard<std::mutex> lk(g_dev_mu);
     if (!dev->attrs_set[slot]) {
-      BSA_CUDA(cudaFuncSetAttribute(attn_fwd_pair_sm100_kernel<D>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::DSMEM));
+      if (vt)
+        BSA_CUDA(cudaFuncSetAttribute(attn_fwd_pair_sm100_kernel<D, true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, C::DSMEM));
+      else
+        BSA_CUDA(cudaFuncSetAttribute(attn_fwd_pair_sm100_kernel<D, false>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, C::DSMEM));
       dev->attrs_set[slot] = true;
     }
   }
   const int grid = p.total_items < dev->sms ? p.total_items : dev->sms;
-  attn_fwd_pair_sm100_kernel<D><<<grid, C::THREADS, C::DSMEM, stream>>>(tq, tk, tv, p);
+  if (vt) {
+    attn_fwd_pair_sm100_kernel<D, true><<<grid, C::THREADS, C::DSMEM, stream>>>(tq, tk, tv, p,
+                                                                                *vt);
+  } else {
+    VarlenTable none;
+    none.num_items = 0;
+    attn_fwd_pair_sm100_kernel<D, false><<<grid, C::THREADS, C::DSMEM, stream>>>(tq, tk, tv, p,
+                                                                                 none);
+  }
   BSA_CUDA(cudaGetLastError());
   return BSA_OK;
 }
@@ -409,14 +423,50 @@ int run_fwd(const QkvViews &x, int32_t n, int32_t head_dim, float softmax_scale,
   }
   p.fault_flags = fault_flags;
   if (pair) {
-    if (head_dim == 128) return launch_pair<128>(x, n, p, dev, stream);
-    return launch_pair<64>(x, n, p, dev, stream);
+    if (head_dim == 128) return launch_pair<128>(x, n, p, dev, nullptr, stream);
+    return launch_pair<64>(x, n, p, dev, nullptr, stream);
   }
   const int slot = slot_of(head_dim, l->block);
   if (head_dim == 128 && l->block == 128) return launch_fwd<128, 128>(x, n, p, dev, slot, stream);
   if (head_dim == 128 && l->block == 64) return launch_fwd<128, 64>(x, n, p, dev, slot, stream);
   if (head_dim == 64 && l->block == 128) return launch_fwd<64, 128>(x, n, p, dev, slot, stream);
   return launch_fwd<64, 64>(x, n, p, dev, slot, stream);
+}
+
+// ----------------------------------------------------- variable-length batches
+
+// Per-item table of a variable-length batch from the host's cu_seqlens
+// (item b = tokens [cu[b], cu[b+1])), for block-128 lists with `heads`
+// work-item rows per query-block pair. Returns BSA_ERR_INVALID_ARG for a
+// malformed cu_seqlens.
+int varlen_table(int32_t num_items, const int32_t *cu, int32_t heads, int block, VarlenTable *vt,
+                 int32_t *max_nqb) {
+  if (num_items < 1 || num_items > kMaxVarlenItems || !cu || cu[0] != 0) return BSA_ERR_INVALID_ARG;
+  long long rows = 0, pairs = 0, work = 0;
+  int mx = 0;
+  vt->num_items = num_items;
+  for (int b = 0; b <= num_items; ++b) {
+    if (b > 0 && cu[b] < cu[b - 1]) return BSA_ERR_INVALID_ARG;
+    vt->tok0[b] = cu[b];
+    vt->row0[b] = static_cast<int32_t>(rows);
+    vt->pair0[b] = static_cast<int32_t>(pairs);
+    vt->work0[b] = static_cast<int32_t>(work);
+    if (b == num_items) break;
+    const int nqb = ceil_div(static_cast<long long>(cu[b + 1]) - cu[b], block);
+    mx = nqb > mx ? nqb : mx;
+    rows += nqb;
+    pairs += (nqb + 1) / 2;
+    work += static_cast<long long>(heads) * ((nqb + 1) / 2);
+    if (work > 0x7fffffffLL) return BSA_ERR_UNSUPPORTED;
+  }
+  if (cu[num_items] < 1) return BSA_ERR_INVALID_ARG;
+  *max_nqb = mx;
+  return BSA_OK;
+}
+
+size_t varlen_order_bytes(const VarlenTable &vt, int num_lists) {
+  return ((static_cast<size_t>(num_lists) * vt.pair0[vt.num_items] * sizeof(int32_t) + 255) &
+          ~size_t(255)) + 256;
 }
 
 QkvViews contiguous_views(const void *q, const void *k, const void *v, int batch, int heads,
@@ -768,7 +818,7 @@ int bsa_joint_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t text_
     while ((tokens_per_frame >> (rs + 1)) >= block) ++rs;
   g.rstar = rs;
   const size_t smem = static_cast<size_t>((nb + 31) / 32) * sizeof(uint32_t);
-  radial_count_kernel<<<nb, 128, smem, stream>>>(g, row_ptr);
+  radial_count_kernel<<<nb, 128, smem, stream>>>(g, row_ptr, 0);
   BSA_CUDA(cudaGetLastError());
   scan_rows_kernel<<<1, 1024, 0, stream>>>(row_ptr, nb);
   BSA_CUDA(cudaGetLastError());
@@ -780,8 +830,69 @@ int bsa_joint_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t text_
     if (col_idx && last > col_capacity) return BSA_ERR_CAPACITY;
   }
   if (col_idx) {
-    radial_fill_kernel<<<nb, 128, smem, stream>>>(g, row_ptr, col_idx, col_capacity);
+    radial_fill_kernel<<<nb, 128, smem, stream>>>(g, row_ptr, 0, col_idx, col_capacity);
     BSA_CUDA(cudaGetLastError());
+  }
+  return BSA_OK;
+}
+
+int bsa_joint_mask_build_varlen(int32_t num_items, const int32_t *frames,
+                                const int32_t *tokens_per_frame, const int32_t *text_tokens,
+                                int32_t block, int32_t *row_ptr, int32_t *col_idx,
+                                int64_t col_capacity, int64_t *nnz_out, bsa_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (num_items < 1 || num_items > kMaxVarlenItems || !frames || !tokens_per_frame || !row_ptr)
+    return BSA_ERR_INVALID_ARG;
+  if (block != 64 && block != 128) return BSA_ERR_UNSUPPORTED;
+  if (col_idx && col_capacity < 0) return BSA_ERR_INVALID_ARG;
+  RadialGeom g[kMaxVarlenItems];
+  int row0[kMaxVarlenItems + 1];
+  long long rows = 0;
+  for (int b = 0; b < num_items; ++b) {
+    const int T = text_tokens ? text_tokens[b] : 0;
+    if (frames[b] < 1 || tokens_per_frame[b] < 1 || T < 0) return BSA_ERR_INVALID_ARG;
+    const long long nv = static_cast<long long>(frames[b]) * tokens_per_frame[b];
+    const long long n = nv + T;
+    if (n > 0x7fffffffLL) return BSA_ERR_INVALID_ARG;
+    const int nb = ceil_div(n, block);
+    if (nb > 262144) return BSA_ERR_UNSUPPORTED;
+    g[b].frames = frames[b];
+    g[b].tpf = tokens_per_frame[b];
+    g[b].block = block;
+    g[b].nv = static_cast<int>(nv);
+    g[b].n = static_cast<int>(n);
+    g[b].nb = nb;
+    int rs = 0;
+    if (tokens_per_frame[b] >= block)
+      while ((tokens_per_frame[b] >> (rs + 1)) >= block) ++rs;
+    g[b].rstar = rs;
+    row0[b] = static_cast<int>(rows);
+    rows += nb;
+    if (rows > 0x7fffffffLL - 1) return BSA_ERR_UNSUPPORTED;
+  }
+  row0[num_items] = static_cast<int>(rows);
+  for (int b = 0; b < num_items; ++b) {
+    const size_t smem = static_cast<size_t>((g[b].nb + 31) / 32) * sizeof(uint32_t);
+    radial_count_kernel<<<g[b].nb, 128, smem, stream>>>(g[b], row_ptr, row0[b]);
+    BSA_CUDA(cudaGetLastError());
+  }
+  scan_rows_kernel<<<1, 1024, 0, stream>>>(row_ptr, row0[num_items]);
+  BSA_CUDA(cudaGetLastError());
+  if (nnz_out) {
+    int32_t last = 0;
+    BSA_CUDA(cudaMemcpyAsync(&last, row_ptr + row0[num_items], sizeof(int32_t),
+                             cudaMemcpyDeviceToHost, stream));
+    BSA_CUDA(cudaStreamSynchronize(stream));
+    *nnz_out = last;
+    if (col_idx && last > col_capacity) return BSA_ERR_CAPACITY;
+  }
+  if (col_idx) {
+    for (int b = 0; b < num_items; ++b) {
+      const size_t smem = static_cast<size_t>((g[b].nb + 31) / 32) * sizeof(uint32_t);
+      radial_fill_kernel<<<g[b].nb, 128, smem, stream>>>(g[b], row_ptr, row0[b], col_idx,
+                                                         col_capacity);
+      BSA_CUDA(cudaGetLastError());
+    }
   }
   return BSA_OK;
 }
@@ -903,6 +1014,121 @@ int bsa_attn_fwd_strided(const void *q, const bsa_layout *q_layout, const void *
                                                  order_only_bytes(l));
   return run_fwd(x, n, head_dim, softmax_scale, l, out, *out_layout, lse, order, counter, dev,
                  fault_flags, stream);
+}
+
+size_t bsa_attn_fwd_varlen_workspace_bytes(int32_t num_items, const int32_t *cu_seqlens,
+                                           int32_t heads, const bsa_block_lists *l) {
+  if (!l || heads < 1 || (l->num_lists != 1 && l->num_lists != heads)) return 0;
+  VarlenTable vt;
+  int32_t mx = 0;
+  if (varlen_table(num_items, cu_seqlens, heads, 128, &vt, &mx) != BSA_OK) return 0;
+  return varlen_order_bytes(vt, l->num_lists);
+}
+
+int bsa_attn_fwd_varlen(const void *q, const bsa_layout *q_layout, const void *k,
+                        const bsa_layout *k_layout, const void *v, const bsa_layout *v_layout,
+                        int32_t num_items, const int32_t *cu_seqlens, int32_t heads,
+                        int32_t head_dim, float softmax_scale, const bsa_block_lists *l,
+                        void *out, const bsa_layout *out_layout, float *lse, void *workspace,
+                        size_t workspace_bytes, bsa_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!q_layout || !k_layout || !v_layout || !out_layout) return BSA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !out || !l || !l->row_ptr || (l->nnz > 0 && !l->col_idx))
+    return BSA_ERR_INVALID_ARG;
+  if (heads < 1) return BSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
+  if (l->block != 128) return BSA_ERR_UNSUPPORTED;
+  if (l->num_lists != 1 && l->num_lists != heads) return BSA_ERR_INVALID_ARG;
+  if (l->nnz < 0) return BSA_ERR_INVALID_ARG;
+  VarlenTable vt;
+  int32_t max_nqb = 0;
+  int st;
+  if ((st = varlen_table(num_items, cu_seqlens, heads, l->block, &vt, &max_nqb)) != BSA_OK)
+    return st;
+  const int32_t total = cu_seqlens[num_items];
+  if (l->num_q_blocks != vt.row0[num_items] || l->num_k_blocks != max_nqb)
+    return BSA_ERR_INVALID_ARG;
+  if (static_cast<long long>(heads) * total > 0x7fffffffLL ||
+      static_cast<long long>(l->num_lists) * l->num_q_blocks > 0x7fffffffLL)
+    return BSA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return BSA_ERR_INVALID_ARG;
+  // the packed sequence is a batch of one: [1, heads, total, head_dim] views
+  for (const bsa_layout *L : {q_layout, k_layout, v_layout, out_layout})
+    if (!layout_ok(*L, 1, heads, total)) return BSA_ERR_INVALID_ARG;
+  if (!layout_disjoint(*out_layout, 1, heads, total, head_dim)) return BSA_ERR_INVALID_ARG;
+  const size_t so = layout_span_bytes(*out_layout, 1, heads, total, head_dim);
+  if (overlaps(out, so, q, layout_span_bytes(*q_layout, 1, heads, total, head_dim)) ||
+      overlaps(out, so, k, layout_span_bytes(*k_layout, 1, heads, total, head_dim)) ||
+      overlaps(out, so, v, layout_span_bytes(*v_layout, 1, heads, total, head_dim)))
+    return BSA_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace) ||
+      workspace_bytes < varlen_order_bytes(vt, l->num_lists))
+    return BSA_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return BSA_ERR_INVALID_ARG;
+  DeviceInfo *dev = nullptr;
+  if ((st = current_device(&dev)) != BSA_OK) return st;
+  if (dev->cc_major != 10) return BSA_ERR_UNSUPPORTED;
+  int fault_flags;
+  {
+    std::lock_guard<std::mutex> lk(g_hook_mu);
+    fault_flags = g_fault_flags;
+    g_fault_flags = 0;
+  }
+  const int L = l->num_lists;
+  int32_t *order = static_cast<int32_t *>(workspace);
+  int32_t *counter = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) +
+                                                 varlen_order_bytes(vt, L) - 256);
+  // work order per item: each item's pairs longest union first, per list;
+  // the first launch also zeroes the work counter
+  bool first = true;
+  for (int b = 0; b < num_items; ++b) {
+    const int nqb = vt.row0[b + 1] - vt.row0[b];
+    if (nqb == 0) continue;
+    const int npairs = (nqb + 1) / 2;
+    const size_t smem = static_cast<size_t>(npairs <= kLptMaxRows ? npairs : 0) * sizeof(int);
+    pair_order_kernel<<<L, 1024, smem, stream>>>(
+        l->row_ptr + static_cast<long long>(L) * vt.row0[b], l->col_idx, nqb, l->nnz,
+        order + static_cast<long long>(L) * vt.pair0[b], kLptMaxRows, first ? counter : nullptr);
+    BSA_CUDA(cudaGetLastError());
+    first = false;
+  }
+  FwdParams p;
+  p.row_ptr = l->row_ptr;
+  p.col_idx = l->col_idx;
+  p.order = order;
+  p.item_counter = counter;
+  p.out = static_cast<__nv_bfloat16 *>(out);
+  p.o_sb = out_layout->batch_stride;
+  p.o_sh = out_layout->head_stride;
+  p.o_sn = out_layout->token_stride;
+  p.lse = lse;
+  p.heads = heads;
+  p.n = total;
+  p.nqb = l->num_q_blocks;
+  p.nkb = l->num_k_blocks;
+  p.num_lists = L;
+  p.nnz = l->nnz;
+  p.total_items = vt.work0[num_items];
+  const float scale =
+      softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
+  p.scale_log2 = scale * 1.4426950408889634f;
+  {
+    std::lock_guard<std::mutex> lk(g_hook_mu);
+    p.wait_limit_ns = g_wait_limit_ns;
+  }
+  p.fault_flags = fault_flags;
+  QkvViews x;
+  x.q = q;
+  x.k = k;
+  x.v = v;
+  x.lq = *q_layout;
+  x.lk = *k_layout;
+  x.lv = *v_layout;
+  x.batch = 1;
+  x.heads = heads;
+  if (head_dim == 128) return launch_pair<128>(x, total, p, dev, &vt, stream);
+  return launch_pair<64>(x, total, p, dev, &vt, stream);
 }
 
 int bsa_attn_bwd_strided(const void *q, const bsa_layout *q_layout, const void *k,

@@ -96,8 +96,10 @@ __device__ void radial_row_bitmap(const RadialGeom g, int qb, uint32_t *bits, in
   __syncthreads();
 }
 
-// One CTA per query block: row length into row_ptr[qb + 1].
-__global__ void radial_count_kernel(RadialGeom g, int32_t *row_ptr) {
+// One CTA per query block: row length into row_ptr[row0 + qb + 1]. `row0` is
+// the first row of this mask in a concatenation of several items' lists (0
+// for a single mask).
+__global__ void radial_count_kernel(RadialGeom g, int32_t *row_ptr, int row0) {
   extern __shared__ uint32_t bits[];
   __shared__ int scratch[32];
   const int words = (g.nb + 31) >> 5;
@@ -107,8 +109,8 @@ __global__ void radial_count_kernel(RadialGeom g, int32_t *row_ptr) {
   int total;
   cta_inclusive_scan(c, scratch, total);
   if (threadIdx.x == 0) {
-    row_ptr[blockIdx.x + 1] = total;
-    if (blockIdx.x == 0) row_ptr[0] = 0;
+    row_ptr[row0 + blockIdx.x + 1] = total;
+    if (row0 == 0 && blockIdx.x == 0) row_ptr[0] = 0;
   }
 }
 
@@ -158,14 +160,15 @@ __device__ void write_row_ascending(const uint32_t *bits, int words, long long s
   }
 }
 
-// One CTA per query block: write the row's key blocks in ascending order.
-__global__ void radial_fill_kernel(RadialGeom g, const int32_t *row_ptr, int32_t *col_idx,
-                                   long long capacity) {
+// One CTA per query block: write the row's key blocks in ascending order
+// (key blocks of this mask's own item, from 0).
+__global__ void radial_fill_kernel(RadialGeom g, const int32_t *row_ptr, int row0,
+                                   int32_t *col_idx, long long capacity) {
   extern __shared__ uint32_t bits[];
   __shared__ int scratch[32];
   const int words = (g.nb + 31) >> 5;
   radial_row_bitmap(g, blockIdx.x, bits, words);
-  write_row_ascending(bits, words, row_ptr[blockIdx.x], col_idx, capacity, scratch);
+  write_row_ascending(bits, words, row_ptr[row0 + blockIdx.x], col_idx, capacity, scratch);
 }
 
 // ------------------------------------------------------------- validation --
@@ -223,13 +226,13 @@ __global__ void lpt_order_kernel(const int32_t *row_ptr, int nqb, int nnz, int32
 // One CTA per list: order[list * npairs + rank] = query-block pair (2p, 2p+1)
 // with the rank-th longest union of key blocks (ties: lower pair first).
 // Lists whose pair count does not fit in shared memory keep natural order.
-// Also zeroes `item_counter`, the attention kernel's work counter (this
-// kernel runs before it in stream order).
+// Also zeroes `item_counter` (when given), the attention kernel's work
+// counter (this kernel runs before it in stream order).
 __global__ void pair_order_kernel(const int32_t *row_ptr, const int32_t *col_idx, int nqb,
                                   int nnz, int32_t *order, int max_smem_rows,
                                   int32_t *item_counter) {
   extern __shared__ int cost[];
-  if (blockIdx.x == 0 && threadIdx.x == 0) *item_counter = 0;
+  if (item_counter && blockIdx.x == 0 && threadIdx.x == 0) *item_counter = 0;
   const int list = blockIdx.x;
   const int npairs = (nqb + 1) / 2;
   const int32_t *rp = row_ptr + static_cast<long long>(list) * nqb;

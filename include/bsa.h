@@ -128,6 +128,29 @@ int bsa_joint_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t text_
                          int32_t block, int32_t *row_ptr, int32_t *col_idx,
                          int64_t col_capacity, int64_t *nnz_out, bsa_stream_t stream);
 
+/*
+ * Block lists of a variable-length batch: item b is a video of frames[b] x
+ * tokens_per_frame[b] tokens followed by text_tokens[b] text tokens (NULL:
+ * none), with the joint rule of bsa_joint_mask_build. The pages describe one
+ * video at a time and say nothing of batches; batching items of different
+ * lengths (prompts with different text lengths, clips with different frame
+ * counts) in one launch is this library's reading, and each item keeps
+ * exactly its own lists.
+ * The lists of the items are concatenated: item b's nqb_b = ceil(n_b / block)
+ * query-block rows follow those of items 0..b-1 (row_ptr holds
+ * sum_b nqb_b + 1 entries, values are offsets into one col_idx), and its
+ * column indices count key blocks from 0 inside the item. The result is the
+ * bsa_block_lists of bsa_attn_fwd_varlen with num_lists = 1,
+ * num_q_blocks = sum_b nqb_b and num_k_blocks = max_b nqb_b.
+ * num_items in [1, 64]; frames, tokens_per_frame, text_tokens are host
+ * arrays of num_items entries. Other arguments, synchronisation and errors
+ * as bsa_joint_mask_build.
+ */
+int bsa_joint_mask_build_varlen(int32_t num_items, const int32_t *frames,
+                                const int32_t *tokens_per_frame, const int32_t *text_tokens,
+                                int32_t block, int32_t *row_ptr, int32_t *col_idx,
+                                int64_t col_capacity, int64_t *nnz_out, bsa_stream_t stream);
+
 #define BSA_TILE_PATTERN_MAX_BANDS 16
 
 /*
@@ -292,6 +315,51 @@ int bsa_attn_fwd_strided(const void *q, const bsa_layout *q_layout,
                          float softmax_scale, const bsa_block_lists *lists,
                          void *out, const bsa_layout *out_layout, float *lse,
                          void *workspace, size_t workspace_bytes, bsa_stream_t stream);
+
+/*
+ * Bytes of device scratch bsa_attn_fwd_varlen needs (the per-item work order
+ * and the work counter); 0 for invalid arguments.
+ */
+size_t bsa_attn_fwd_varlen_workspace_bytes(int32_t num_items, const int32_t *cu_seqlens,
+                                           int32_t heads, const bsa_block_lists *lists);
+
+/*
+ * bsa_attn_fwd's operation on a variable-length batch in one launch: the
+ * items' tokens are packed one after another, item b owning tokens
+ * [cu_seqlens[b], cu_seqlens[b+1]) of q, k, v and out, and attention runs
+ * inside each item only, over that item's block lists (the pages treat one
+ * sequence at a time; batching sequences of different lengths is this
+ * library's reading).
+ * q, k, v, out  device bf16 views of [1, heads, total, head_dim] described by
+ *        their bsa_layout (batch_stride unused), total = cu_seqlens[num_items];
+ *        e.g. packed [total, heads, head_dim] (token_stride = heads*head_dim,
+ *        head_stride = head_dim) or [heads, total, head_dim]. Layout rules as
+ *        bsa_attn_fwd_strided. Every element must be finite (an item's last
+ *        key block may read the next item's tokens, which enter with weight 0).
+ * num_items, cu_seqlens  number of items in [1, 64] and a host array of
+ *        num_items + 1 token offsets: cu_seqlens[0] = 0, non-decreasing, total
+ *        >= 1 (empty items are allowed).
+ * lists  the items' lists concatenated as bsa_joint_mask_build_varlen writes
+ *        them: block 128; num_q_blocks = sum_b ceil(n_b / 128); num_k_blocks
+ *        = max_b ceil(n_b / 128); num_lists 1 (each item's list shared by its
+ *        heads) or heads (item b's rows hold its lists for heads 0..heads-1,
+ *        one after another, nqb_b rows each); column indices count key blocks
+ *        inside the item.
+ * lse    device fp32 [heads, total] (natural log, -inf for a row without
+ *        keys), or NULL.
+ * workspace  bsa_attn_fwd_varlen_workspace_bytes() bytes of device scratch.
+ * Results for each item equal bsa_attn_fwd on that item alone, bit for bit.
+ * Returns BSA_ERR_UNSUPPORTED for block 64 or head_dim other than 64 / 128;
+ * other errors as bsa_attn_fwd. Asynchronous.
+ */
+int bsa_attn_fwd_varlen(const void *q, const bsa_layout *q_layout,
+                        const void *k, const bsa_layout *k_layout,
+                        const void *v, const bsa_layout *v_layout,
+                        int32_t num_items, const int32_t *cu_seqlens,
+                        int32_t heads, int32_t head_dim, float softmax_scale,
+                        const bsa_block_lists *lists,
+                        void *out, const bsa_layout *out_layout, float *lse,
+                        void *workspace, size_t workspace_bytes, bsa_stream_t stream);
 
 /*
  * Bytes of device scratch bsa_attn_module_fwd needs: the projected q/k/v

@@ -29,6 +29,8 @@ Modules:
   attention, head merge, output projection), in float64.
 * ``tile_patterns``: per-head tile patterns (diagonal and multi-diagonal
   bands, vertical stripes, dual windows) expanded into block lists.
+* ``varlen``: variable-length batches (items with their own lists,
+  concatenated; attention item by item).
 """
 
 from .radial_mask import (  # noqa: F401
@@ -60,6 +62,11 @@ from .attention_backward import (  # noqa: F401
 from .tile_patterns import (  # noqa: F401
     tile_pattern_mask,
     tile_pattern_lists,
+)
+from .varlen import (  # noqa: F401
+    varlen_block_lists,
+    split_item_lists,
+    varlen_masked_attention_fp64,
 )
 from .module import (  # noqa: F401
     radial_attention_module_fp64,

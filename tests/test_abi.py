@@ -396,3 +396,44 @@ def test_gemm_host_checks(lib):
     assert call(d=vp((2 << 30) + 4096)) == 1         # D inside B's span
     assert call(bias=vp((3 << 30) + 64)) == 1        # bias inside D's span
     assert call(a=None) == 1
+
+
+def test_varlen_host_checks(lib):
+    """bsa_attn_fwd_varlen and its list builder reject malformed per-item
+    arguments on the host, before any CUDA call."""
+    from block_sparse_attention_radial_b200._lib import BlockListsC, LayoutC
+
+    vp, ref = ctypes.c_void_p, ctypes.byref
+    H, D = 2, 128
+    cu_ok = (ctypes.c_int32 * 4)(0, 300, 300, 700)        # nqb 3, 0, 4 at block 128
+    lay = LayoutC(0, D, H * D)                            # packed [total, H, D]
+    q, k, v, o, w = (vp(a << 30) for a in (1, 2, 3, 4, 8))
+
+    def lists(nq=7, nk=4, block=128, L=1):
+        return BlockListsC(L, nq, nk, block, 10, 1 << 22, 1 << 23)
+
+    def call(ls=None, cu=cu_ok, items=3, wsb=1 << 20, out=o, hd=D):
+        ls = lists() if ls is None else ls
+        return lib.bsa_attn_fwd_varlen(q, ref(lay), k, ref(lay), v, ref(lay), items, cu, H, hd,
+                                       0.0, ref(ls), out, ref(lay), None, w, wsb, None)
+
+    assert lib.bsa_attn_fwd_varlen_workspace_bytes(3, cu_ok, H, ref(lists())) == 256 + 256
+    assert call(items=0) == 1 and call(items=65) == 1
+    assert call(cu=(ctypes.c_int32 * 4)(1, 300, 300, 700)) == 1      # cu[0] != 0
+    assert call(cu=(ctypes.c_int32 * 4)(0, 300, 200, 700)) == 1      # decreasing
+    assert call(cu=(ctypes.c_int32 * 2)(0, 0), items=1) == 1          # no tokens at all
+    assert call(ls=lists(nq=6)) == 1                                  # row count mismatch
+    assert call(ls=lists(nk=7)) == 1                                  # widest item is 4
+    assert call(ls=lists(block=64, nq=14, nk=7)) == 2                 # block 64 unsupported
+    assert call(ls=lists(L=3)) == 1                                   # num_lists not 1 or H
+    assert call(hd=96) == 2
+    assert call(wsb=256) == 1                                         # workspace too small
+    assert call(out=vp((4 << 30) + 8)) == 1                           # misaligned out
+    assert call(out=vp((1 << 30) + 4096)) == 1                        # out inside q's span
+    # list builder: bad item geometry, too many items
+    fr, tp, tx = ((ctypes.c_int32 * 2)(*x) for x in ((2, 0), (100, 100), (0, 0)))
+    rp = vp(1 << 22)
+    assert lib.bsa_joint_mask_build_varlen(2, fr, tp, tx, 128, rp, None, 0, None, None) == 1
+    fr2 = (ctypes.c_int32 * 2)(2, 3)
+    assert lib.bsa_joint_mask_build_varlen(65, fr2, tp, tx, 128, rp, None, 0, None, None) == 1
+    assert lib.bsa_joint_mask_build_varlen(2, fr2, tp, tx, 96, rp, None, 0, None, None) == 2

@@ -1,0 +1,129 @@
+"""Variable-length batches on the GPU: the concatenated list builder
+(bsa_joint_mask_build_varlen) bit-exact against the oracle, and the varlen
+forward (bsa_attn_fwd_varlen) against the float64 oracle item by item and,
+bit for bit, against the regular entry run on each item alone.
+
+Items differ in frame count, tokens per frame and text length, so their token
+counts, query-block counts and lists all differ; one launch serves them all.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import assert_close
+from workloads import random_block_lists
+
+pytestmark = pytest.mark.gpu
+
+ITEMS = [(4, 320, 0), (3, 256, 77), (5, 200, 130)]   # (frames, tokens_per_frame, text)
+
+
+@pytest.fixture(scope="module")
+def bsa():
+    import block_sparse_attention_radial_b200 as m
+
+    torch.cuda.set_device(0)
+    return m
+
+
+def _cu(lengths):
+    return np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+
+
+def _packed(total, H, D, seed):
+    g = torch.Generator().manual_seed(seed)
+    return [torch.randn((total, H, D), generator=g).to(torch.bfloat16) for _ in range(3)]
+
+
+def _item_view(x, t0, t1):
+    """[1, H, n_b, D] contiguous copy of item tokens t0..t1 of a packed tensor."""
+    return x[t0:t1].permute(1, 0, 2).unsqueeze(0).contiguous()
+
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_varlen_lists_bit_exact(bsa, block):
+    items = ITEMS + [(1, 50, 0), (21, 1560, 256)]
+    lists = bsa.radial_block_lists_varlen(items, block)
+    rp, ci = oracle.varlen_block_lists(items, block)
+    assert bsa.bsa_get_device_status() == 0
+    assert np.array_equal(lists.row_ptr.cpu().numpy(), rp)
+    assert np.array_equal(lists.col_idx.cpu().numpy(), ci)
+    nqbs = [-(-(f * s + t) // block) for f, s, t in items]
+    assert lists.num_q_blocks == sum(nqbs) and lists.num_k_blocks == max(nqbs)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_varlen_radial_against_oracle_and_single_items(bsa, D):
+    H = 3
+    lengths = [f * s + t for f, s, t in ITEMS]
+    cu = _cu(lengths)
+    q, k, v = _packed(int(cu[-1]), H, D, seed=D)
+    lists = bsa.radial_block_lists_varlen(ITEMS, 128)
+    out, lse = bsa.attention_varlen(q.cuda(), k.cuda(), v.cuda(), cu, lists)
+    assert bsa.bsa_get_device_status() == 0
+    rp, ci = oracle.varlen_block_lists(ITEMS, 128)
+    nqbs = [-(-n // 128) for n in lengths]
+    item_lists = oracle.split_item_lists(rp, ci, nqbs)
+    ref_o, ref_l = oracle.varlen_masked_attention_fp64(q.float().numpy(), k.float().numpy(),
+                                                       v.float().numpy(), cu, item_lists, 1, 128)
+    o, l_ = out.cpu(), lse.cpu()
+    for b, (f, s, t) in enumerate(ITEMS):
+        t0, t1 = int(cu[b]), int(cu[b + 1])
+        assert_close(o[t0:t1].float().numpy(), ref_o[t0:t1], l_[:, t0:t1].numpy(),
+                     ref_l[:, t0:t1], f"varlen item {b} ({f}x{s}+{t})")
+        # the same item through the regular entry, alone: identical bits
+        one = bsa.radial_block_lists(f, s, 128, text_tokens=t)
+        qi, ki, vi = (_item_view(x, t0, t1).cuda() for x in (q, k, v))
+        oi, li = bsa.attention(qi, ki, vi, one)
+        assert torch.equal(oi[0].permute(1, 0, 2).cpu(), o[t0:t1]), f"item {b} output differs"
+        assert torch.equal(li[0].cpu(), l_[:, t0:t1]), f"item {b} lse differs"
+
+
+def test_varlen_per_head_lists_and_an_empty_item(bsa):
+    H, D, blk = 4, 128, 128
+    lengths = [500, 0, 1, 383, 1024]
+    cu = _cu(lengths)
+    q, k, v = _packed(int(cu[-1]), H, D, seed=7)
+    nqbs = [-(-n // blk) for n in lengths]
+    rps, cis, item_lists, off = [], [], [], 0
+    for b, nqb in enumerate(nqbs):
+        if nqb == 0:
+            item_lists.append((np.zeros(1, dtype=np.int64), np.zeros(0, dtype=np.int64)))
+            continue
+        rp, ci = random_block_lists(H * nqb, nqb, 0.5, seed=20 + b)
+        item_lists.append((rp, ci))
+        rps.append(np.asarray(rp[:-1]) + off)
+        cis.append(np.asarray(ci))
+        off += int(rp[-1])
+    row_ptr = np.concatenate(rps + [np.array([off])])
+    col_idx = np.concatenate(cis)
+    lists = bsa.block_lists_from_csr(row_ptr, col_idx, H, sum(nqbs), blk)
+    lists.k_blocks = max(nqbs)
+    out, lse = bsa.attention_varlen(q.cuda(), k.cuda(), v.cuda(), cu, lists)
+    assert bsa.bsa_get_device_status() == 0
+    ref_o, ref_l = oracle.varlen_masked_attention_fp64(q.float().numpy(), k.float().numpy(),
+                                                       v.float().numpy(), cu, item_lists, H, blk)
+    assert_close(out.cpu().float().numpy(), ref_o, lse.cpu().numpy(), ref_l, "per-head varlen")
+
+
+def test_varlen_medium_batch_matches_single_items(bsa):
+    # larger items, many work items per launch: every item bit-identical to
+    # its own regular call (itself checked against the oracle elsewhere)
+    items = [(8, 1560, 256), (5, 3600, 0), (12, 780, 64)]
+    H, D = 8, 128
+    lengths = [f * s + t for f, s, t in items]
+    cu = _cu(lengths)
+    g = torch.Generator(device="cuda").manual_seed(3)
+    q, k, v = (torch.randn((int(cu[-1]), H, D), generator=g, device="cuda").to(torch.bfloat16)
+               for _ in range(3))
+    lists = bsa.radial_block_lists_varlen(items, 128)
+    out, lse = bsa.attention_varlen(q, k, v, cu, lists)
+    assert bsa.bsa_get_device_status() == 0
+    for b, (f, s, t) in enumerate(items):
+        t0, t1 = int(cu[b]), int(cu[b + 1])
+        one = bsa.radial_block_lists(f, s, 128, text_tokens=t)
+        oi, li = bsa.attention(*(_item_view(x, t0, t1) for x in (q, k, v)), one)
+        assert torch.equal(oi[0].permute(1, 0, 2), out[t0:t1]), f"item {b} output differs"
+        assert torch.equal(li[0], lse[:, t0:t1]), f"item {b} lse differs"
