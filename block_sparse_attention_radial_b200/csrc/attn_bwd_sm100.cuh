@@ -328,11 +328,11 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(&bar_s_full, 1);
     mbar_init(&bar_dp_full, 1);
     for (int h = 0; h < 4; ++h) {
-      mbar_init(&bar_p_part[h], 128);
-      mbar_init(&bar_ds_part[h], 128);
+      mbar_init(&bar_p_part[h], 4);  // one arrival per elementwise warp
+      mbar_init(&bar_ds_part[h], 4);
     }
     mbar_init(&bar_acc_full, 1);
-    mbar_init(&bar_acc_empty, 128);
+    mbar_init(&bar_acc_empty, 4);
     mbar_init(&bar_final, 1);
     for (int i = 0; i < kBwdItemN; ++i) {
       mbar_init(&bar_item_full[i], 1);
@@ -600,7 +600,8 @@ __global__ void __launch_bounds__(192, 1)
           tmem_st16(lane_tmem + C::ST_COL + c * 16, pk);
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(&bar_p_part[c]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar_p_part[c]);
         }
         ++scount;
         if (!(ok = warp_wait(&bar_dp_full, dcount & 1u, wc, kBarSFull, dcount))) break;
@@ -623,7 +624,8 @@ __global__ void __launch_bounds__(192, 1)
           tmem_st16(lane_tmem + C::DPT_COL + c * 16, g16);
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(&bar_ds_part[c]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar_ds_part[c]);
         }
       }
       if (!ok) break;
@@ -657,7 +659,8 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&bar_acc_empty);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_acc_empty);
     }
   }
 
@@ -739,9 +742,9 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(&bar_s_full[0], 1);
     mbar_init(&bar_s_full[1], 1);
     mbar_init(&bar_dp_full, 1);
-    for (int h = 0; h < 4; ++h) mbar_init(&bar_ds_part[h], 128);
+    for (int h = 0; h < 4; ++h) mbar_init(&bar_ds_part[h], 4);
     mbar_init(&bar_acc_full, 1);
-    mbar_init(&bar_acc_empty, 128);
+    mbar_init(&bar_acc_empty, 4);
     mbar_init(&bar_final, 1);
     for (int i = 0; i < kBwdItemN; ++i) {
       mbar_init(&bar_item_full[i], 1);
@@ -996,7 +999,8 @@ __global__ void __launch_bounds__(192, 1)
           tmem_st16(lane_tmem + C::DP_COL + c * 16, g16);
           tmem_wait_st();  // part c of the key columns handed over
           tc_fence_before();
-          mbar_arrive(&bar_ds_part[c]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar_ds_part[c]);
         }
       }
       if (!ok) break;
@@ -1024,7 +1028,8 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&bar_acc_empty);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_acc_empty);
     }
   }
 

@@ -287,9 +287,9 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&bar_final, 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bar_s_full[t], 1);
-      mbar_init(&bar_p_full[t], 128);
+      mbar_init(&bar_p_full[t], 4);   // one arrival per softmax warp
       mbar_init(&bar_o_final[t], 1);
-      mbar_init(&bar_o_empty[t], 128);
+      mbar_init(&bar_o_empty[t], 4);
     }
     for (int i = 0; i < kItemN; ++i) {
       mbar_init(&bar_item_full[i], 1);
@@ -711,9 +711,12 @@ __global__ void __launch_bounds__(384, 1)
           for (int i = 0; i < 32; ++i) r[i] = pk[c * 32 + i];
           tmem_st32(s_tmem + c * 32, r);
         }
+        // the warp-collective wait covers every lane's stores; one arrival
+        // per warp (128 arrivals on one barrier would serialise)
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bar_p_full[t]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_p_full[t]);
       }
       if (!ok) break;
       if (!(ok = warp_wait(&bar_o_final[t], icnt & 1u, wc, kBarODone, icnt))) break;
@@ -741,7 +744,8 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (store && p.lse) p.lse[orow] = (m_ref + log2f(l)) * 0.69314718055994531f;
       tc_fence_before();
-      mbar_arrive(&bar_o_empty[t]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_o_empty[t]);
     }
   }
 

@@ -277,13 +277,13 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(&bar_q_full, 1);
     mbar_init(&bar_q_empty, 1);
-    mbar_init(&bar_o_empty, 128);
+    mbar_init(&bar_o_empty, 4);  // one arrival per softmax warp
     mbar_init(&bar_final, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar_s_full[b], 1);
-      mbar_init(&bar_s_free[b], 128);
+      mbar_init(&bar_s_free[b], 4);
       mbar_init(&bar_o_done[b], 1);
-      mbar_init(&bar_p_full[b], 128);
+      mbar_init(&bar_p_full[b], 4);
     }
     abort_flag = 0;
     fence_barrier_init();
@@ -537,7 +537,8 @@ __global__ void __launch_bounds__(192, 1)
         }
         // S is in registers: its TMEM buffer may take QK(gg+2) right away.
         tc_fence_before();
-        mbar_arrive(&bar_s_free[gg & 1u]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_s_free[gg & 1u]);
         const int kb = lc.get(p, it.a, it.len, j);
         const int valid = p.n - kb * BN;
         if (valid < BN) {
@@ -608,7 +609,8 @@ __global__ void __launch_bounds__(192, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bar_p_full[gg & 1u]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_p_full[gg & 1u]);
       }
       if (!ok) break;
       const uint32_t gl = g + it.len - 1;
@@ -636,7 +638,8 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (store && p.lse) p.lse[orow] = (m_ref + log2f(l)) * 0.69314718055994531f;
       tc_fence_before();
-      mbar_arrive(&bar_o_empty);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_o_empty);
       g += it.len;
     }
   }

@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar_acc_full[b], 1);
-      mbar_init(&bar_acc_empty[b], 128);
+      mbar_init(&bar_acc_empty[b], 4);  // one arrival per epilogue warp
     }
     mbar_init(&bar_final, 1);
     abort_flag = 0;
@@ -249,7 +249,8 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&bar_acc_empty[buf]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_acc_empty[buf]);
     }
     (void)ok;
   }
