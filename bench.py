@@ -316,13 +316,14 @@ class FwdProblem:
     """One forward workload resident on the device: inputs, lists, outputs and
     the step that rebuilds the lists and runs the attention."""
 
-    def __init__(self, w, dev, stream):
+    def __init__(self, w, dev, stream, generated: bool = False):
         import torch
 
         import block_sparse_attention_radial_b200 as bsa
         from workloads import make_qkv
 
         self.w, self.dev, self.stream, self.bsa = w, dev, stream, bsa
+        self.generated = generated
         self.q, self.k, self.v = make_qkv(w, dev)
         if w.radial:
             self.num_lists = 1
@@ -345,6 +346,15 @@ class FwdProblem:
         self.ws = torch.empty(max(bsa.bsa_attn_fwd_workspace_bytes(w.batch, w.heads, self.lists),
                                   16), dtype=torch.uint8, device=dev)
         self.launches_per_step = 5  # list count, scan, fill; work order; attention
+        if generated:  # rows generated in the kernel: count, scan, work order, attention
+            self.launches_per_step = 4
+            if w.radial:
+                nbytes = bsa._lib.load().bsa_attn_fwd_radial_workspace_bytes(
+                    w.frames, w.tokens_per_frame, w.text_tokens)
+            else:
+                self.pat_raw, self.pat_cols = bsa.pack_tile_patterns(pats, dev)
+                nbytes = bsa._lib.load().bsa_attn_fwd_patterns_workspace_bytes(w.heads, w.nqb)
+            self.gws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
 
     def build_lists(self):
         w, l, bsa = self.w, self.lists, self.bsa
@@ -358,11 +368,26 @@ class FwdProblem:
                                              want_nnz=False, stream=self.stream)
 
     def step(self, ev=None):
+        w, bsa = self.w, self.bsa
+        if self.generated:
+            # the whole entry is timed: row lengths, work order and attention
+            if ev is not None:
+                ev[0].record(self.stream)
+            if w.radial:
+                bsa.bsa_attn_fwd_radial(self.q, self.k, self.v, w.frames, w.tokens_per_frame,
+                                        self.out, self.lse, w.text_tokens, self.gws, 0.0,
+                                        self.stream)
+            else:
+                bsa.bsa_attn_fwd_patterns(self.q, self.k, self.v, self.pat_raw, self.pat_cols,
+                                          self.out, self.lse, None, self.gws, 0.0, self.stream)
+            if ev is not None:
+                ev[1].record(self.stream)
+            return
         self.build_lists()
         if ev is not None:
             ev[0].record(self.stream)
-        self.bsa.bsa_attn_fwd(self.q, self.k, self.v, self.lists, self.out, self.lse, self.ws,
-                              0.0, self.stream)
+        bsa.bsa_attn_fwd(self.q, self.k, self.v, self.lists, self.out, self.lse, self.ws,
+                         0.0, self.stream)
         if ev is not None:
             ev[1].record(self.stream)
 
@@ -401,7 +426,7 @@ class FwdProblem:
         if status != 0:
             raise SystemExit(f"device status {status} after the timed region")
         # the lists rebuilt inside every step are the ones the FLOPs were counted on
-        if not (np.array_equal(self.lists.row_ptr.cpu().numpy(), self.rp_h)
+        if not self.generated and not (np.array_equal(self.lists.row_ptr.cpu().numpy(), self.rp_h)
                 and np.array_equal(self.lists.col_idx.cpu().numpy(), self.ci_h)):
             raise SystemExit("lists rebuilt in the timed steps differ from the counted lists")
         return ms, kernel_ms, clocks
@@ -409,12 +434,15 @@ class FwdProblem:
     def roofline(self, kernel_ms, peaks, peak_kind):
         peak = float(peaks["bf16_tflops"])
         achieved = self.flops / (kernel_ms * 1e-3) / 1e12
+        kernel = ("attn_fwd_pair_sm100_kernel<128> (+ work-order prepass)" if not self.generated
+                  else "attn_fwd_pair_sm100_kernel<128>, rows generated in the kernel "
+                       "(+ row-length count, scan and work order, all timed)")
         return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": load_traffic(self.w.name),
+                "frac": achieved / peak,
+                "traffic": None if self.generated else load_traffic(self.w.name),
                 "peak_kind": f"{peak_kind} bf16 burst",
                 "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
-                "kernel": "attn_fwd_pair_sm100_kernel<128> (+ work-order prepass)",
-                "kernel_ms": kernel_ms, "flops_per_launch": self.flops}
+                "kernel": kernel, "kernel_ms": kernel_ms, "flops_per_launch": self.flops}
 
 
 # The other configurations of the metric's 32k-131k token range, timed in the
@@ -459,7 +487,7 @@ def run_ours(args, world, rank, local):
     init_dist(world, "nccl")
     w = WORKLOADS[args.workload]
     stream = torch.cuda.current_stream(dev)
-    prob = FwdProblem(w, dev, stream)
+    prob = FwdProblem(w, dev, stream, generated=args.rows == "generated")
     q, k, v, lists = prob.q, prob.k, prob.v, prob.lists
     rp_h, ci_h, flops = prob.rp_h, prob.ci_h, prob.flops
     ms, kernel_ms, clocks = prob.timed(args.steps, args.warmup, rank)
@@ -504,7 +532,7 @@ def run_ours(args, world, rank, local):
     roofline = prob.roofline(kernel_ms, peaks, peak_kind)
     dense_flops, launches_per_step = prob.dense_flops, prob.launches_per_step
     per_config = None
-    if world == 1 and args.workload == "wan" and args.per_config_steps > 0:
+    if world == 1 and args.workload == "wan" and args.rows == "lists" and args.per_config_steps > 0:
         del prob, q, k, v, lists
         torch.cuda.empty_cache()
         per_config = per_config_records(args, dev, stream, rank, peaks, peak_kind)
@@ -527,6 +555,8 @@ def run_ours(args, world, rank, local):
             "cpu_baseline": cpu_baseline,
             "per_config": per_config,
         }
+        line["config"]["rows"] = ("generated in the kernel" if args.rows == "generated"
+                                  else "block lists rebuilt every step")
         print(json.dumps(line), flush=True)
     import torch.distributed as dist
 
@@ -988,6 +1018,10 @@ def main(argv=None):
     ap.add_argument("--per-config-steps", type=int, default=10,
                     help="timed steps for each of the other forward configurations recorded "
                          "under per_config in the default (wan, one GPU) run; 0 skips them")
+    ap.add_argument("--rows", choices=("lists", "generated"), default="lists",
+                    help="forward: read the block lists (default), or generate every row's key "
+                         "blocks inside the attention kernel from the radial geometry / the "
+                         "tile patterns (bsa_attn_fwd_radial / bsa_attn_fwd_patterns)")
     ap.add_argument("--gemm-shape", default="all", choices=("all",) + tuple(GEMM_SHAPES),
                     help="--pass gemm: one of the module's GEMM shapes, or all six")
     ap.add_argument("--gemm-vs-torch", action="store_true",

@@ -30,6 +30,7 @@ __all__ = [
     "computed_flops", "bsa_attn_fwd_noalloc", "bsa_selftest_exp2", "NOALLOC_MAX_ORDER_ENTRIES",
     "bsa_gemm_bf16", "bsa_joint_mask_build_varlen", "bsa_attn_fwd_varlen",
     "bsa_attn_fwd_varlen_workspace_bytes", "radial_block_lists_varlen", "attention_varlen",
+    "bsa_attn_fwd_patterns", "bsa_attn_fwd_radial",
     "bsa_attn_fwd_strided", "bsa_attn_module_workspace_bytes", "bsa_joint_mask_build",
     "bsa_attn_fwd_host", "bsa_attn_fwd_host_workspace_bytes", "bsa_attn_bwd_strided",
     "bsa_attn_module_bwd", "bsa_attn_module_bwd_workspace_bytes", "attention_module_backward", "bsa_attn_module_fwd",
@@ -205,6 +206,43 @@ def bsa_attn_fwd_strided(q, k, v, lists: BlockLists, out, lse=None, workspace=No
                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
                                   _stream(stream))
     _check(st, "bsa_attn_fwd_strided")
+
+
+def bsa_attn_fwd_patterns(q, k, v, patterns, columns, out, lse=None, head_pattern=None,
+                          workspace=None, softmax_scale: float = 0.0, stream=None) -> None:
+    """Forward over per-head tile patterns generated inside the kernel (no
+    column list): ``patterns`` / ``columns`` as packed by
+    :func:`pack_tile_patterns`; ``head_pattern`` an int32 device tensor mapping
+    heads to patterns, or None (one pattern, or one per head)."""
+    B, H, n, D = q.shape
+    lib = _lib.load()
+    L = int(patterns.numel() * patterns.element_size() // ctypes.sizeof(TilePatternC))
+    nqb = -(-n // 128)
+    if workspace is None:
+        workspace = torch.empty(max(lib.bsa_attn_fwd_patterns_workspace_bytes(L, nqb), 16),
+                                dtype=torch.uint8, device=q.device)
+    st = lib.bsa_attn_fwd_patterns(_ptr(q), _ptr(k), _ptr(v), B, H, n, D, float(softmax_scale),
+                                   L, _ptr(patterns), _ptr(columns),
+                                   0 if columns is None else columns.numel(), _ptr(head_pattern),
+                                   _ptr(out), _ptr(lse), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "bsa_attn_fwd_patterns")
+
+
+def bsa_attn_fwd_radial(q, k, v, frames: int, tokens_per_frame: int, out, lse=None,
+                        text_tokens: int = 0, workspace=None, softmax_scale: float = 0.0,
+                        stream=None) -> None:
+    """Forward over the (joint) radial mask generated inside the kernel."""
+    B, H, n, D = q.shape
+    lib = _lib.load()
+    if workspace is None:
+        workspace = torch.empty(max(lib.bsa_attn_fwd_radial_workspace_bytes(
+            frames, tokens_per_frame, text_tokens), 16), dtype=torch.uint8, device=q.device)
+    st = lib.bsa_attn_fwd_radial(_ptr(q), _ptr(k), _ptr(v), B, H, frames, tokens_per_frame,
+                                 text_tokens, D, float(softmax_scale), _ptr(out), _ptr(lse),
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                 _stream(stream))
+    _check(st, "bsa_attn_fwd_radial")
 
 
 def _cu_array(cu_seqlens):

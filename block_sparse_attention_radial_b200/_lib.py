@@ -22,6 +22,10 @@ EXPORTS = (
     "bsa_attn_fwd_workspace_bytes",
     "bsa_attn_fwd",
     "bsa_attn_fwd_strided",
+    "bsa_attn_fwd_patterns_workspace_bytes",
+    "bsa_attn_fwd_patterns",
+    "bsa_attn_fwd_radial_workspace_bytes",
+    "bsa_attn_fwd_radial",
     "bsa_attn_fwd_varlen_workspace_bytes",
     "bsa_attn_fwd_varlen",
     "bsa_attn_fwd_host_workspace_bytes",
@@ -125,6 +129,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bsa_joint_mask_build_varlen": (ctypes.c_int, [i32, vp, vp, vp, i32, vp, vp, i64,
                                                        ctypes.POINTER(i64), vp]),
         "bsa_attn_fwd_varlen_workspace_bytes": (sz, [i32, vp, i32, lp]),
+        "bsa_attn_fwd_patterns_workspace_bytes": (sz, [i32, i32]),
+        "bsa_attn_fwd_patterns": (ctypes.c_int, [vp, vp, vp, i32, i32, i32, i32, ctypes.c_float,
+                                                 i32, vp, vp, i64, vp, vp, vp, vp, sz, vp]),
+        "bsa_attn_fwd_radial_workspace_bytes": (sz, [i32, i32, i32]),
+        "bsa_attn_fwd_radial": (ctypes.c_int, [vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                               ctypes.c_float, vp, vp, vp, sz, vp]),
         "bsa_attn_fwd_varlen": (ctypes.c_int, [vp, yp, vp, yp, vp, yp, i32, vp, i32, i32,
                                                ctypes.c_float, lp, vp, yp, vp, vp, sz, vp]),
         "bsa_attn_fwd_workspace_bytes": (sz, [i32, i32, lp]),

@@ -46,6 +46,7 @@
 #include <cuda_bf16.h>
 
 #include "attn_fwd_sm100.cuh"
+#include "rowgen.cuh"
 
 namespace bsa {
 
@@ -90,24 +91,86 @@ struct RowReader {
   }
 };
 
+// Where the rows' key blocks come from: the CSR lists (col_idx), or
+// generated in the kernel from per-list tile patterns or the radial geometry.
+enum : int { kModeLists = 0, kModeVarlen = 1, kModePatterns = 2, kModeRadial = 3 };
+
+// One row's key blocks in ascending order, by mode; next() returns INT_MAX
+// past the end.
+template <int MODE>
+struct RowSource;
+
+template <>
+struct RowSource<kModeLists> {
+  RowReader r;
+  __device__ __forceinline__ void reset(const FwdParams &p, int list, int qb, int a0, int len,
+                                        int nkb, const bsa_tile_pattern *) {
+    r.reset(p, a0, len, nkb);
+  }
+  __device__ __forceinline__ int next() {
+    const int v = r.nxt;
+    if (v != INT_MAX) r.pop();
+    return v;
+  }
+};
+
+template <>
+struct RowSource<kModeVarlen> : RowSource<kModeLists> {};
+
+template <>
+struct RowSource<kModePatterns> {
+  PatternRow r;
+  int left;  // the row's length from the count pass: never walk past it
+  // `pat`: the item's pattern, staged in shared memory by the producer
+  __device__ __forceinline__ void reset(const FwdParams &p, int list, int qb, int a0, int len,
+                                        int nkb, const bsa_tile_pattern *pat) {
+    r.reset(pat, p.pattern_columns, p.num_pattern_columns, qb, nkb);
+    left = len;
+  }
+  __device__ __forceinline__ int next() {
+    if (left <= 0) return INT_MAX;
+    --left;
+    return r.next();
+  }
+};
+
+template <>
+struct RowSource<kModeRadial> {
+  RadialRow r;
+  int left;
+  __device__ __forceinline__ void reset(const FwdParams &p, int list, int qb, int a0, int len,
+                                        int nkb, const bsa_tile_pattern *) {
+    r.reset(p.radial, qb);
+    left = len;
+  }
+  __device__ __forceinline__ int next() {
+    if (left <= 0) return INT_MAX;
+    --left;
+    return r.next();
+  }
+};
+
 // Key blocks of one query-block pair, walked as the sorted union of the two
-// rows by one thread (the producer and the MMA issuer run identical walks).
+// rows by one thread (the producer; the MMA issuer reads its step plans).
+template <int MODE>
 struct UnionWalker {
-  RowReader ra, rb;
-  __device__ __forceinline__ void reset(const FwdParams &p, int a0, int lenA, int b0, int lenB,
-                                        int nkb) {
-    ra.reset(p, a0, lenA, nkb);
-    rb.reset(p, b0, lenB, nkb);
+  RowSource<MODE> ra, rb;
+  int va, vb;
+  __device__ __forceinline__ void reset(const FwdParams &p, int list, int qa, int a0, int lenA,
+                                        int b0, int lenB, int nkb, const bsa_tile_pattern *pat) {
+    ra.reset(p, list, qa, a0, lenA, nkb, pat);
+    rb.reset(p, list, qa + 1, b0, lenB, nkb, pat);
+    va = ra.next();
+    vb = rb.next();
   }
   // Next union block: false when both rows are exhausted.
   __device__ __forceinline__ bool next(int &kb, bool &inA, bool &inB) {
-    const int va = ra.nxt, vb = rb.nxt;
     if (va == INT_MAX && vb == INT_MAX) return false;
     kb = min(va, vb);
     inA = va == kb;
     inB = vb == kb;
-    if (inA) ra.pop();
-    if (inB) rb.pop();
+    if (inA) va = ra.next();
+    if (inB) vb = rb.next();
     return true;
   }
 };
@@ -133,6 +196,7 @@ struct VarlenTable {
 struct PairItem {
   int bh, qa, a0, lenA, b0, lenB;  // tile B absent (lenB = 0) past the last block
   int n, nqb, nkb, tok0;           // the item's tokens, query and key blocks, first token
+  int list;                        // the list (pattern) the item's rows belong to
 };
 
 // Rows qa and qa + 1 (when it exists) of the list starting at row lbase.
@@ -152,18 +216,21 @@ __device__ __forceinline__ void pair_rows(const FwdParams &p, long long lbase, P
   }
 }
 
-template <bool VARLEN>
+template <int MODE>
 __device__ __forceinline__ PairItem decode_pair(int idx, const FwdParams &p, int npairs,
                                                 const VarlenTable &vt) {
   PairItem it;
-  if (!VARLEN) {
+  if (MODE != kModeVarlen) {
     it.n = p.n;
     it.nqb = p.nqb;
     it.nkb = p.nkb;
     it.tok0 = 0;
     it.bh = idx / npairs;
     const int rank = idx - it.bh * npairs;
-    const int list = p.num_lists > 1 ? (it.bh % p.heads) : 0;
+    const int h = it.bh % p.heads;
+    const int list = p.head_list ? min(max(p.head_list[h], 0), p.num_lists - 1)
+                                 : (p.num_lists > 1 ? h : 0);
+    it.list = list;
     const long long lbase = static_cast<long long>(list) * p.nqb;
     const int pr = min(max(p.order[static_cast<long long>(list) * npairs + rank], 0), npairs - 1);
     it.qa = 2 * pr;
@@ -190,6 +257,7 @@ __device__ __forceinline__ PairItem decode_pair(int idx, const FwdParams &p, int
   it.bh = local / np;  // the head (batch extent 1)
   const int rank = local - it.bh * np;
   const int list = p.num_lists > 1 ? it.bh : 0;
+  it.list = list;
   const long long lbase = static_cast<long long>(p.num_lists) * vt.row0[b] +
                           static_cast<long long>(list) * it.nqb;
   const long long obase = static_cast<long long>(p.num_lists) * vt.pair0[b] +
@@ -244,7 +312,7 @@ __device__ __forceinline__ bool plan_wait(const volatile uint32_t *ring, uint32_
   }
 }
 
-template <int D, bool VARLEN>
+template <int D, int MODE>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_pair_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k,
@@ -265,6 +333,9 @@ __global__ void __launch_bounds__(384, 1)
   // ring (a longest-first order served dynamically keeps the CTAs' finishing
   // times within about one item of each other).
   __shared__ int item_ring[kItemN];
+  // the producer's copy of the current item's tile pattern (rows generated
+  // from tile patterns only)
+  __shared__ bsa_tile_pattern prod_pat;
   __shared__ __align__(8) uint64_t bar_item_full[kItemN], bar_item_empty[kItemN];
 
   const uint32_t raw = smem_addr(dsmem);
@@ -338,7 +409,7 @@ __global__ void __launch_bounds__(384, 1)
           item_ring[slot] = idx;
           mbar_arrive(&bar_item_full[slot]);
           if (idx < 0) break;
-          const PairItem it = decode_pair<VARLEN>(idx, p, npairs, vt);
+          const PairItem it = decode_pair<MODE>(idx, p, npairs, vt);
           if (it.lenA == 0 && it.lenB == 0) continue;
           if (!(ok = lane_wait(&bar_q_empty, (qcount & 1u) ^ 1u, wc, kBarQEmpty, qcount))) break;
           mbar_arrive_expect_tx(&bar_q_full, 2 * C::Q_BYTES);
@@ -350,8 +421,9 @@ __global__ void __launch_bounds__(384, 1)
           // Same walk and same first-use order as the MMA issuer: at step j it
           // needs V(j-1) first when tile A listed j-1 or A skips j, and K(j)
           // first otherwise.
-          UnionWalker uw;
-          uw.reset(p, it.a0, it.lenA, it.b0, it.lenB, it.nkb);
+          if (MODE == kModePatterns) prod_pat = p.patterns[it.list];
+          UnionWalker<MODE> uw;
+          uw.reset(p, it.list, it.qa, it.a0, it.lenA, it.b0, it.lenB, it.nkb, &prod_pat);
           bool pa = false, pb = false;
           int prev_kb = 0;
           while (ok) {
@@ -437,7 +509,7 @@ __global__ void __launch_bounds__(384, 1)
           const int idx = *static_cast<volatile int *>(&item_ring[slot]);
           mbar_arrive(&bar_item_empty[slot]);
           if (idx < 0) break;
-          const PairItem it = decode_pair<VARLEN>(idx, p, npairs, vt);
+          const PairItem it = decode_pair<MODE>(idx, p, npairs, vt);
           if (it.lenA == 0 && it.lenB == 0) continue;
           if (!(ok = lane_wait(&bar_q_full, qcount & 1u, wc, kBarQFull, qcount))) break;
           tc_fence_after();
@@ -568,7 +640,7 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_item_empty[slot]);
       if (idx < 0) break;
-      const PairItem it = decode_pair<VARLEN>(idx, p, npairs, vt);
+      const PairItem it = decode_pair<MODE>(idx, p, npairs, vt);
       const int qb = it.qa + t;
       if (qb >= it.nqb) continue;
       const int len = t == 0 ? it.lenA : it.lenB;
@@ -590,8 +662,25 @@ __global__ void __launch_bounds__(384, 1)
       }
       // Lists are sorted, so only the row's last block can be the ragged
       // final key block; its valid column count is taken once per item.
-      const int last_kb = min(max(__ldg(p.col_idx + a0 + len - 1), 0), it.nkb - 1);
-      const int last_valid = min(it.n - last_kb * BN, BN);
+      int last_valid;
+      if (MODE == kModeLists || MODE == kModeVarlen) {
+        const int last_kb = min(max(__ldg(p.col_idx + a0 + len - 1), 0), it.nkb - 1);
+        last_valid = min(it.n - last_kb * BN, BN);
+      } else {
+        // generated rows: the last block is ragged iff the row holds the
+        // final key block
+        bool has_final;
+        if (MODE == kModePatterns) {
+          PatternRow r;
+          r.reset(p.patterns + it.list, p.pattern_columns, p.num_pattern_columns, qb, it.nkb);
+          has_final = r.has(it.nkb - 1);
+        } else {
+          RadialRow r;
+          r.reset(p.radial, qb);
+          has_final = r.has(it.nkb - 1);
+        }
+        last_valid = has_final ? min(it.n - (it.nkb - 1) * BN, BN) : BN;
+      }
       float m_ref = 0.f, l = 0.f;
       for (int j = 0; j < len; ++j) {
         if (!(ok = warp_wait(&bar_s_full[t], scnt & 1u, wc, kBarSFull, scnt))) break;

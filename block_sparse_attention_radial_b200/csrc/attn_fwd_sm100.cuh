@@ -32,7 +32,9 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "bsa.h"
 #include "device_status.cuh"
+#include "lists.cuh"
 #include "ptx_sm100.cuh"
 
 namespace bsa {
@@ -49,6 +51,14 @@ struct FwdParams {
   float scale_log2;  // softmax_scale * log2(e)
   unsigned long long wait_limit_ns;
   int32_t fault_flags;
+  // Rows generated in the kernel instead of read from col_idx (two-tile
+  // kernel): per-list tile patterns (list of head h = head_list[h] when given)
+  // or the radial geometry shared by every head.
+  const bsa_tile_pattern *patterns = nullptr;
+  const int32_t *pattern_columns = nullptr;
+  long long num_pattern_columns = 0;
+  const int32_t *head_list = nullptr;
+  RadialGeom radial = {};
 };
 
 constexpr int kSmemLimit = 232448;  // 227 KB dynamic + static per CTA on sm_100

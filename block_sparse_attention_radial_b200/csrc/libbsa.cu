@@ -57,6 +57,7 @@ struct DeviceInfo {
                        false, false, false, false, false, false};
   bool ref_attrs_set[4] = {false, false, false, false};
   bool gemm_attrs_set[4] = {false, false, false, false};
+  bool pair_attrs_set[8] = {false, false, false, false, false, false, false, false};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -333,10 +334,31 @@ int launch_ref(const RefParams &p, int batch, DeviceInfo *dev, int slot, cudaStr
 
 int slot_of(int D, int BN) { return (D == 128 ? 2 : 0) + (BN == 128 ? 1 : 0); }
 
-// The two-tile kernel; `vt` (variable-length batches) or null (a regular
-// batch). For a variable-length batch, x.batch is 1 and n the total tokens.
+// The two-tile kernel in one of its row modes (kModeLists, kModeVarlen with
+// `vt`, kModePatterns, kModeRadial). For a variable-length batch, x.batch is 1
+// and n the total tokens.
+template <int D, int MODE>
+int launch_pair_mode(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                     const FwdParams &p, DeviceInfo *dev, const VarlenTable &vt,
+                     cudaStream_t stream) {
+  using C = PairCfg<D>;
+  const int slot = MODE * 2 + (D == 128 ? 1 : 0);
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!dev->pair_attrs_set[slot]) {
+      BSA_CUDA(cudaFuncSetAttribute(attn_fwd_pair_sm100_kernel<D, MODE>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::DSMEM));
+      dev->pair_attrs_set[slot] = true;
+    }
+  }
+  const int grid = p.total_items < dev->sms ? p.total_items : dev->sms;
+  attn_fwd_pair_sm100_kernel<D, MODE><<<grid, C::THREADS, C::DSMEM, stream>>>(tq, tk, tv, p, vt);
+  BSA_CUDA(cudaGetLastError());
+  return BSA_OK;
+}
+
 template <int D>
-int launch_pair(const QkvViews &x, int32_t n, const FwdParams &p, DeviceInfo *dev,
+int launch_pair(const QkvViews &x, int32_t n, const FwdParams &p, DeviceInfo *dev, int mode,
                 const VarlenTable *vt, cudaStream_t stream) {
   using C = PairCfg<D>;
   CUtensorMap tq, tk, tv;
@@ -344,31 +366,15 @@ int launch_pair(const QkvViews &x, int32_t n, const FwdParams &p, DeviceInfo *de
   if ((st = make_map_strided(&tq, x.q, x.lq, x.batch, x.heads, n, D, C::BN)) != BSA_OK) return st;
   if ((st = make_map_strided(&tk, x.k, x.lk, x.batch, x.heads, n, D, C::BN)) != BSA_OK) return st;
   if ((st = make_map_strided(&tv, x.v, x.lv, x.batch, x.heads, n, D, C::BN)) != BSA_OK) return st;
-  const int slot = (vt ? 6 : 4) + (D == 128 ? 1 : 0);
-  {
-    std::lock_guard<std::mutex> lk(g_dev_mu);
-    if (!dev->attrs_set[slot]) {
-      if (vt)
-        BSA_CUDA(cudaFuncSetAttribute(attn_fwd_pair_sm100_kernel<D, true>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, C::DSMEM));
-      else
-        BSA_CUDA(cudaFuncSetAttribute(attn_fwd_pair_sm100_kernel<D, false>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, C::DSMEM));
-      dev->attrs_set[slot] = true;
-    }
+  VarlenTable none;
+  none.num_items = 0;
+  const VarlenTable &t = vt ? *vt : none;
+  switch (mode) {
+    case kModeVarlen: return launch_pair_mode<D, kModeVarlen>(tq, tk, tv, p, dev, t, stream);
+    case kModePatterns: return launch_pair_mode<D, kModePatterns>(tq, tk, tv, p, dev, t, stream);
+    case kModeRadial: return launch_pair_mode<D, kModeRadial>(tq, tk, tv, p, dev, t, stream);
+    default: return launch_pair_mode<D, kModeLists>(tq, tk, tv, p, dev, t, stream);
   }
-  const int grid = p.total_items < dev->sms ? p.total_items : dev->sms;
-  if (vt) {
-    attn_fwd_pair_sm100_kernel<D, true><<<grid, C::THREADS, C::DSMEM, stream>>>(tq, tk, tv, p,
-                                                                                *vt);
-  } else {
-    VarlenTable none;
-    none.num_items = 0;
-    attn_fwd_pair_sm100_kernel<D, false><<<grid, C::THREADS, C::DSMEM, stream>>>(tq, tk, tv, p,
-                                                                                 none);
-  }
-  BSA_CUDA(cudaGetLastError());
-  return BSA_OK;
 }
 
 // Work order into `order`, then the attention kernel. Block-128 problems run
@@ -423,8 +429,8 @@ int run_fwd(const QkvViews &x, int32_t n, int32_t head_dim, float softmax_scale,
   }
   p.fault_flags = fault_flags;
   if (pair) {
-    if (head_dim == 128) return launch_pair<128>(x, n, p, dev, nullptr, stream);
-    return launch_pair<64>(x, n, p, dev, nullptr, stream);
+    if (head_dim == 128) return launch_pair<128>(x, n, p, dev, kModeLists, nullptr, stream);
+    return launch_pair<64>(x, n, p, dev, kModeLists, nullptr, stream);
   }
   const int slot = slot_of(head_dim, l->block);
   if (head_dim == 128 && l->block == 128) return launch_fwd<128, 128>(x, n, p, dev, slot, stream);
@@ -467,6 +473,61 @@ int varlen_table(int32_t num_items, const int32_t *cu, int32_t heads, int block,
 size_t varlen_order_bytes(const VarlenTable &vt, int num_lists) {
   return ((static_cast<size_t>(num_lists) * vt.pair0[vt.num_items] * sizeof(int32_t) + 255) &
           ~size_t(255)) + 256;
+}
+
+// ------------------------------------------------ rows generated in-kernel
+
+// Scratch of the generated-row entries: row lengths (row_ptr of the count
+// pass), the work order and the work counter.
+constexpr int kMaxGeneratedLists = 4096;
+struct GeneratedLayout {
+  size_t row_ptr, order, cost, counter, total;
+};
+GeneratedLayout generated_layout(int num_lists, int nqb) {
+  GeneratedLayout w;
+  const size_t pairs = static_cast<size_t>(num_lists) * ((nqb + 1) / 2) * sizeof(int32_t);
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  w.row_ptr = 0;
+  w.order = up((static_cast<size_t>(num_lists) * nqb + 1) * sizeof(int32_t));
+  w.cost = w.order + up(pairs);
+  w.counter = w.cost + up(pairs);
+  w.total = w.counter + 256;
+  return w;
+}
+
+// Parameters of the two-tile kernel for rows generated in the kernel
+// (contiguous [batch, heads, n, head_dim] views, block 128).
+FwdParams generated_params(int batch, int heads, int n, int nqb, int num_lists,
+                           const int32_t *row_ptr, const int32_t *order, int32_t *counter,
+                           void *out, int head_dim, float *lse, float softmax_scale) {
+  FwdParams p;
+  p.row_ptr = row_ptr;
+  p.col_idx = nullptr;
+  p.order = order;
+  p.item_counter = counter;
+  p.out = static_cast<__nv_bfloat16 *>(out);
+  const bsa_layout lo = contiguous_layout(heads, n, head_dim);
+  p.o_sb = lo.batch_stride;
+  p.o_sh = lo.head_stride;
+  p.o_sn = lo.token_stride;
+  p.lse = lse;
+  p.heads = heads;
+  p.n = n;
+  p.nqb = nqb;
+  p.nkb = nqb;
+  p.num_lists = num_lists;
+  p.nnz = 0x7fffffff;  // row_ptr comes from this call's own count pass
+  p.total_items = batch * heads * ((nqb + 1) / 2);
+  const float scale =
+      softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
+  p.scale_log2 = scale * 1.4426950408889634f;
+  {
+    std::lock_guard<std::mutex> lk(g_hook_mu);
+    p.wait_limit_ns = g_wait_limit_ns;
+    p.fault_flags = g_fault_flags;
+    g_fault_flags = 0;
+  }
+  return p;
 }
 
 QkvViews contiguous_views(const void *q, const void *k, const void *v, int batch, int heads,
@@ -1127,8 +1188,148 @@ int bsa_attn_fwd_varlen(const void *q, const bsa_layout *q_layout, const void *k
   x.lv = *v_layout;
   x.batch = 1;
   x.heads = heads;
-  if (head_dim == 128) return launch_pair<128>(x, total, p, dev, &vt, stream);
-  return launch_pair<64>(x, total, p, dev, &vt, stream);
+  if (head_dim == 128) return launch_pair<128>(x, total, p, dev, kModeVarlen, &vt, stream);
+  return launch_pair<64>(x, total, p, dev, kModeVarlen, &vt, stream);
+}
+
+size_t bsa_attn_fwd_patterns_workspace_bytes(int32_t num_patterns, int32_t num_q_blocks) {
+  if (num_patterns < 1 || num_q_blocks < 1) return 0;
+  return generated_layout(num_patterns, num_q_blocks).total;
+}
+
+int bsa_attn_fwd_patterns(const void *q, const void *k, const void *v, int32_t batch,
+                          int32_t heads, int32_t n, int32_t head_dim, float softmax_scale,
+                          int32_t num_patterns, const bsa_tile_pattern *patterns,
+                          const int32_t *columns, int64_t num_columns,
+                          const int32_t *head_pattern, void *out, float *lse, void *workspace,
+                          size_t workspace_bytes, bsa_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!patterns || num_columns < 0 || (num_columns > 0 && !columns)) return BSA_ERR_INVALID_ARG;
+  if (num_patterns < 1 || num_patterns > kMaxGeneratedLists) return BSA_ERR_INVALID_ARG;
+  if (!head_pattern && num_patterns != 1 && num_patterns != heads) return BSA_ERR_INVALID_ARG;
+  if (n < 1) return BSA_ERR_INVALID_ARG;
+  const int nqb = ceil_div(n, 128);
+  // the argument checks of bsa_attn_fwd, on stand-in lists of the same shape
+  bsa_block_lists shape;
+  shape.num_lists = 1;
+  shape.num_q_blocks = nqb;
+  shape.num_k_blocks = nqb;
+  shape.block = 128;
+  shape.nnz = 0;
+  shape.row_ptr = static_cast<const int32_t *>(workspace);
+  shape.col_idx = nullptr;
+  int st = check_attn_args(q, k, v, batch, heads, n, head_dim, &shape, out);
+  if (st != BSA_OK) return st;
+  const GeneratedLayout w = generated_layout(num_patterns, nqb);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < w.total) return BSA_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return BSA_ERR_INVALID_ARG;
+  if (static_cast<long long>(num_patterns) * nqb > 0x7fffffffLL) return BSA_ERR_UNSUPPORTED;
+  DeviceInfo *dev = nullptr;
+  if ((st = current_device(&dev)) != BSA_OK) return st;
+  if (dev->cc_major != 10) return BSA_ERR_UNSUPPORTED;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  int32_t *row_ptr = reinterpret_cast<int32_t *>(ws + w.row_ptr);
+  int32_t *order = reinterpret_cast<int32_t *>(ws + w.order);
+  int32_t *counter = reinterpret_cast<int32_t *>(ws + w.counter);
+  // row lengths of every pattern (the count pass of the list builder), then
+  // the work order from the generated rows; no column list is written
+  const int rows = num_patterns * nqb;
+  const size_t bits = static_cast<size_t>((nqb + 31) / 32) * sizeof(uint32_t);
+  pattern_count_kernel<<<rows, 128, bits, stream>>>(patterns, columns, num_columns, nqb, row_ptr);
+  BSA_CUDA(cudaGetLastError());
+  scan_rows_kernel<<<1, 1024, 0, stream>>>(row_ptr, rows);
+  BSA_CUDA(cudaGetLastError());
+  const int npairs = (nqb + 1) / 2;
+  int32_t *cost = reinterpret_cast<int32_t *>(ws + w.cost);
+  pattern_pair_union_kernel<<<num_patterns * npairs, 128, 2 * bits, stream>>>(
+      patterns, columns, num_columns, nqb, cost);
+  BSA_CUDA(cudaGetLastError());
+  const size_t smem = static_cast<size_t>(npairs <= kLptMaxRows ? npairs : 0) * sizeof(int);
+  rank_pairs_kernel<<<num_patterns, 1024, smem, stream>>>(cost, npairs, order, kLptMaxRows,
+                                                          counter);
+  BSA_CUDA(cudaGetLastError());
+  FwdParams p = generated_params(batch, heads, n, nqb, num_patterns, row_ptr, order, counter,
+                                 out, head_dim, lse, softmax_scale);
+  p.patterns = patterns;
+  p.pattern_columns = columns;
+  p.num_pattern_columns = num_columns;
+  p.head_list = head_pattern;
+  const QkvViews x = contiguous_views(q, k, v, batch, heads, n, head_dim);
+  if (head_dim == 128) return launch_pair<128>(x, n, p, dev, kModePatterns, nullptr, stream);
+  return launch_pair<64>(x, n, p, dev, kModePatterns, nullptr, stream);
+}
+
+size_t bsa_attn_fwd_radial_workspace_bytes(int32_t frames, int32_t tokens_per_frame,
+                                           int32_t text_tokens) {
+  if (frames < 1 || tokens_per_frame < 1 || text_tokens < 0) return 0;
+  const long long n = static_cast<long long>(frames) * tokens_per_frame + text_tokens;
+  if (n > 0x7fffffffLL) return 0;
+  return generated_layout(1, ceil_div(n, 128)).total;
+}
+
+int bsa_attn_fwd_radial(const void *q, const void *k, const void *v, int32_t batch,
+                        int32_t heads, int32_t frames, int32_t tokens_per_frame,
+                        int32_t text_tokens, int32_t head_dim, float softmax_scale, void *out,
+                        float *lse, void *workspace, size_t workspace_bytes,
+                        bsa_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (frames < 1 || tokens_per_frame < 1 || text_tokens < 0) return BSA_ERR_INVALID_ARG;
+  // a key frame must fit the generator's 64-block window: it touches at most
+  // (tokens_per_frame - 1) / 128 + 2 key blocks
+  if ((tokens_per_frame - 1) / 128 + 2 > 64) return BSA_ERR_UNSUPPORTED;
+  const long long nl = static_cast<long long>(frames) * tokens_per_frame + text_tokens;
+  if (nl > 0x7fffffffLL) return BSA_ERR_INVALID_ARG;
+  const int n = static_cast<int>(nl);
+  const int nqb = ceil_div(n, 128);
+  bsa_block_lists shape;
+  shape.num_lists = 1;
+  shape.num_q_blocks = nqb;
+  shape.num_k_blocks = nqb;
+  shape.block = 128;
+  shape.nnz = 0;
+  shape.row_ptr = static_cast<const int32_t *>(workspace);
+  shape.col_idx = nullptr;
+  int st = check_attn_args(q, k, v, batch, heads, n, head_dim, &shape, out);
+  if (st != BSA_OK) return st;
+  const GeneratedLayout w = generated_layout(1, nqb);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < w.total) return BSA_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return BSA_ERR_INVALID_ARG;
+  DeviceInfo *dev = nullptr;
+  if ((st = current_device(&dev)) != BSA_OK) return st;
+  if (dev->cc_major != 10) return BSA_ERR_UNSUPPORTED;
+  RadialGeom g;
+  g.frames = frames;
+  g.tpf = tokens_per_frame;
+  g.block = 128;
+  g.nv = frames * tokens_per_frame;
+  g.n = n;
+  g.nb = nqb;
+  int rs = 0;
+  if (tokens_per_frame >= 128)
+    while ((tokens_per_frame >> (rs + 1)) >= 128) ++rs;
+  g.rstar = rs;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  int32_t *row_ptr = reinterpret_cast<int32_t *>(ws + w.row_ptr);
+  int32_t *order = reinterpret_cast<int32_t *>(ws + w.order);
+  int32_t *counter = reinterpret_cast<int32_t *>(ws + w.counter);
+  const size_t bits = static_cast<size_t>((nqb + 31) / 32) * sizeof(uint32_t);
+  radial_count_kernel<<<nqb, 128, bits, stream>>>(g, row_ptr, 0);
+  BSA_CUDA(cudaGetLastError());
+  scan_rows_kernel<<<1, 1024, 0, stream>>>(row_ptr, nqb);
+  BSA_CUDA(cudaGetLastError());
+  const int npairs = (nqb + 1) / 2;
+  int32_t *cost = reinterpret_cast<int32_t *>(ws + w.cost);
+  radial_pair_union_kernel<<<npairs, 128, bits, stream>>>(g, cost);
+  BSA_CUDA(cudaGetLastError());
+  const size_t smem = static_cast<size_t>(npairs <= kLptMaxRows ? npairs : 0) * sizeof(int);
+  rank_pairs_kernel<<<1, 1024, smem, stream>>>(cost, npairs, order, kLptMaxRows, counter);
+  BSA_CUDA(cudaGetLastError());
+  FwdParams p = generated_params(batch, heads, n, nqb, 1, row_ptr, order, counter, out,
+                                 head_dim, lse, softmax_scale);
+  p.radial = g;
+  const QkvViews x = contiguous_views(q, k, v, batch, heads, n, head_dim);
+  if (head_dim == 128) return launch_pair<128>(x, n, p, dev, kModeRadial, nullptr, stream);
+  return launch_pair<64>(x, n, p, dev, kModeRadial, nullptr, stream);
 }
 
 int bsa_attn_bwd_strided(const void *q, const bsa_layout *q_layout, const void *k,

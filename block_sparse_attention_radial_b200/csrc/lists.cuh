@@ -193,6 +193,21 @@ __global__ void validate_cols_kernel(const int32_t *row_ptr, const int32_t *col_
 
 // ------------------------------------------------------------ work order --
 
+// ord[rank] = the index with the rank-th largest cost (ties: lower index
+// first), ranked by counting so the order is deterministic. The CTA's threads
+// share the work; `cost` is complete before the call.
+__device__ __forceinline__ void rank_by_cost(const int *cost, int count, int32_t *ord) {
+  for (int r = threadIdx.x; r < count; r += blockDim.x) {
+    const int c = cost[r];
+    int rank = 0;
+    for (int o = 0; o < count; ++o) {
+      const int co = cost[o];
+      rank += (co > c) || (co == c && o < r);
+    }
+    ord[rank] = r;
+  }
+}
+
 // One CTA per list. order[list * nqb + rank] = query block with the rank-th
 // longest row (ties: lower block first). Rows are ranked by counting, which
 // keeps the order deterministic. Lists with more rows than fit in shared
@@ -268,15 +283,7 @@ __global__ void pair_order_kernel(const int32_t *row_ptr, const int32_t *col_idx
     if (lane == 0) cost[pr] = (ea - ia) + (eb - ib) - common;
   }
   __syncthreads();
-  for (int r = threadIdx.x; r < npairs; r += blockDim.x) {
-    const int c = cost[r];
-    int rank = 0;
-    for (int o = 0; o < npairs; ++o) {
-      const int co = cost[o];
-      rank += (co > c) || (co == c && o < r);
-    }
-    ord[rank] = r;
-  }
+  rank_by_cost(cost, npairs, ord);
 }
 
 }  // namespace bsa

@@ -317,6 +317,64 @@ int bsa_attn_fwd_strided(const void *q, const bsa_layout *q_layout,
                          void *workspace, size_t workspace_bytes, bsa_stream_t stream);
 
 /*
+ * Rows generated inside the attention kernel. The two entries below compute
+ * bsa_attn_fwd's operation over lists that are never written out: each
+ * query-block row's key blocks are generated by the attention kernel's
+ * producer from the analytic description (the Sparse-vDiT skill page, "CUDA
+ * kernel invocation (pseudo-code)", dispatches pattern-specialised kernels;
+ * the Compact Attention abstract's tile-aligned windows; the radial rule of
+ * the "Radial Attention" skill page, Step 1, and the thismoment.ai blog, "How
+ * Radial Attention Works"). Only the row lengths are computed first (the
+ * builders' count pass), for the work order and the softmax; no column list
+ * exists. Results are bit-identical to bsa_attn_fwd on the lists that
+ * bsa_tile_pattern_lists_build / bsa_joint_mask_build would build. Block
+ * 128; q, k, v, out contiguous bf16 [batch, heads, n, head_dim] as for
+ * bsa_attn_fwd, lse fp32 [batch, heads, n] or NULL; other limits and errors
+ * as bsa_attn_fwd. Asynchronous.
+ */
+
+/* Bytes of device scratch bsa_attn_fwd_patterns needs (row lengths, work
+ * order, work counter); 0 for invalid arguments. */
+size_t bsa_attn_fwd_patterns_workspace_bytes(int32_t num_patterns, int32_t num_q_blocks);
+
+/*
+ * Per-head tile patterns generated in the kernel. patterns: device array of
+ * num_patterns descriptors (as for bsa_tile_pattern_lists_build, whose
+ * columns array and num_columns they index). head_pattern: device int32
+ * [heads], the pattern of each head (heads sharing a pattern share one set of
+ * row lengths and one work order: Sparse-vDiT's head fusion), or NULL when
+ * num_patterns is 1 (every head) or heads (head h uses pattern h); entries are
+ * clamped into [0, num_patterns). num_patterns in [1, 4096]. A malformed
+ * descriptor or out-of-range column is reported through
+ * bsa_get_device_status() (BSA_ERR_INVALID_ARG), as by the list builder.
+ */
+int bsa_attn_fwd_patterns(const void *q, const void *k, const void *v,
+                          int32_t batch, int32_t heads, int32_t n, int32_t head_dim,
+                          float softmax_scale, int32_t num_patterns,
+                          const bsa_tile_pattern *patterns, const int32_t *columns,
+                          int64_t num_columns, const int32_t *head_pattern,
+                          void *out, float *lse, void *workspace, size_t workspace_bytes,
+                          bsa_stream_t stream);
+
+/* Bytes of device scratch bsa_attn_fwd_radial needs; 0 for invalid
+ * arguments. */
+size_t bsa_attn_fwd_radial_workspace_bytes(int32_t frames, int32_t tokens_per_frame,
+                                           int32_t text_tokens);
+
+/*
+ * The joint radial mask (bsa_joint_mask_build's rule; text_tokens = 0 is the
+ * plain radial mask) generated in the kernel, shared by every head:
+ * n = frames * tokens_per_frame + text_tokens. tokens_per_frame at most
+ * 8063 (a key frame then touches at most 64 key blocks, the generator's
+ * window), BSA_ERR_UNSUPPORTED beyond.
+ */
+int bsa_attn_fwd_radial(const void *q, const void *k, const void *v,
+                        int32_t batch, int32_t heads, int32_t frames,
+                        int32_t tokens_per_frame, int32_t text_tokens, int32_t head_dim,
+                        float softmax_scale, void *out, float *lse, void *workspace,
+                        size_t workspace_bytes, bsa_stream_t stream);
+
+/*
  * Bytes of device scratch bsa_attn_fwd_varlen needs (the per-item work order
  * and the work counter); 0 for invalid arguments.
  */

@@ -437,3 +437,37 @@ def test_varlen_host_checks(lib):
     fr2 = (ctypes.c_int32 * 2)(2, 3)
     assert lib.bsa_joint_mask_build_varlen(65, fr2, tp, tx, 128, rp, None, 0, None, None) == 1
     assert lib.bsa_joint_mask_build_varlen(2, fr2, tp, tx, 96, rp, None, 0, None, None) == 2
+
+
+def test_generated_rows_host_checks(lib):
+    """bsa_attn_fwd_patterns / bsa_attn_fwd_radial reject bad arguments on the
+    host, before any CUDA call."""
+    vp = ctypes.c_void_p
+    B, H, n, D = 1, 4, 1000, 128
+    q, k, v, o, pat, cols, w = (vp(a << 30) for a in (1, 2, 3, 4, 5, 6, 8))
+    ws = lib.bsa_attn_fwd_patterns_workspace_bytes(2, 8)
+    # row lengths (2*8+1 ints -> 256 B) + order (2*4 ints -> 256 B) + counter
+    assert ws == 256 + 256 + 256
+    assert lib.bsa_attn_fwd_patterns_workspace_bytes(0, 8) == 0
+
+    def pcall(L=H, p=pat, c=cols, nc=10, hp=None, wsb=1 << 20, hd=D, nn=n):
+        return lib.bsa_attn_fwd_patterns(q, k, v, B, H, nn, hd, 0.0, L, p, c, nc, hp, o, None, w,
+                                         wsb, None)
+
+    assert pcall(L=0) == 1 and pcall(L=4097) == 1
+    assert pcall(L=3) == 1                       # neither 1 nor heads, and no head map
+    assert pcall(p=None) == 1
+    assert pcall(c=None) == 1                    # columns missing while num_columns > 0
+    assert pcall(nc=-1) == 1
+    assert pcall(wsb=256) == 1
+    assert pcall(hd=96) == 2
+    assert pcall(nn=0) == 1
+
+    def rcall(F=4, S=250, T=0, wsb=1 << 20):
+        return lib.bsa_attn_fwd_radial(q, k, v, B, H, F, S, T, D, 0.0, o, None, w, wsb, None)
+
+    assert rcall(F=0) == 1 and rcall(S=0) == 1 and rcall(T=-1) == 1
+    assert rcall(S=9000) == 2                    # a frame wider than the generator's window
+    assert rcall(wsb=256) == 1
+    assert lib.bsa_attn_fwd_radial_workspace_bytes(4, 250, 0) > 0
+    assert lib.bsa_attn_fwd_radial_workspace_bytes(0, 250, 0) == 0
