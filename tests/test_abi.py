@@ -446,8 +446,9 @@ def test_generated_rows_host_checks(lib):
     B, H, n, D = 1, 4, 1000, 128
     q, k, v, o, pat, cols, w = (vp(a << 30) for a in (1, 2, 3, 4, 5, 6, 8))
     ws = lib.bsa_attn_fwd_patterns_workspace_bytes(2, 8)
-    # row lengths (2*8+1 ints -> 256 B) + order (2*4 ints -> 256 B) + counter
-    assert ws == 256 + 256 + 256
+    # row lengths (2*8+1 ints -> 256 B) + order and pair costs (2*4 ints -> 256 B
+    # each) + counter
+    assert ws == 256 + 256 + 256 + 256
     assert lib.bsa_attn_fwd_patterns_workspace_bytes(0, 8) == 0
 
     def pcall(L=H, p=pat, c=cols, nc=10, hp=None, wsb=1 << 20, hd=D, nn=n):
