@@ -34,7 +34,8 @@ METRIC = "block-sparse attn fwd ms & effective TFLOP/s vs bf16 peak at 32k–120
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 CSRC = "block_sparse_attention_radial_b200/csrc/"
 KERNEL_SOURCES = {
-    "fwd": (CSRC + "attn_fwd_pair_sm100.cuh", CSRC + "attn_fwd_sm100.cuh", CSRC + "ptx_sm100.cuh"),
+    "fwd": (CSRC + "attn_fwd_pair_sm100.cuh", CSRC + "attn_fwd_sm100.cuh", CSRC + "ptx_sm100.cuh",
+            CSRC + "rowgen.cuh"),
     "bwd": (CSRC + "attn_bwd_sm100.cuh", CSRC + "attn_fwd_sm100.cuh", CSRC + "ptx_sm100.cuh"),
 }
 TRAFFIC_FILES = {"fwd": "attn_fwd_pair_sm100_{}_traffic.json", "bwd": "attn_bwd_sm100_{}_traffic.json"}
