@@ -1012,7 +1012,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="wan",
-                    choices=("wan", "hunyuan", "long4x", "tiny", "hunyuan_text", "generic"),
+                    choices=("wan", "hunyuan", "long4x", "tiny", "hunyuan_text", "generic",
+                             "wan_b64"),
                     help="generic: per-head tile patterns built on the GPU (forward only)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -93,7 +93,11 @@ struct RowReader {
 
 // Where the rows' key blocks come from: the CSR lists (col_idx), or
 // generated in the kernel from per-list tile patterns or the radial geometry.
-enum : int { kModeLists = 0, kModeVarlen = 1, kModePatterns = 2, kModeRadial = 3 };
+// kModeQuarters: block-64 lists merged into 128-row tile lists, each entry
+// with the mask of its listed 64 x 64 quarters (the softmax masks the rest).
+enum : int {
+  kModeLists = 0, kModeVarlen = 1, kModePatterns = 2, kModeRadial = 3, kModeQuarters = 4
+};
 
 // One row's key blocks in ascending order, by mode; next() returns INT_MAX
 // past the end.
@@ -116,6 +120,9 @@ struct RowSource<kModeLists> {
 
 template <>
 struct RowSource<kModeVarlen> : RowSource<kModeLists> {};
+
+template <>
+struct RowSource<kModeQuarters> : RowSource<kModeLists> {};
 
 template <>
 struct RowSource<kModePatterns> {
@@ -663,7 +670,7 @@ __global__ void __launch_bounds__(384, 1)
       // Lists are sorted, so only the row's last block can be the ragged
       // final key block; its valid column count is taken once per item.
       int last_valid;
-      if (MODE == kModeLists || MODE == kModeVarlen) {
+      if (MODE == kModeLists || MODE == kModeVarlen || MODE == kModeQuarters) {
         const int last_kb = min(max(__ldg(p.col_idx + a0 + len - 1), 0), it.nkb - 1);
         last_valid = min(it.n - last_kb * BN, BN);
       } else {
@@ -681,8 +688,14 @@ __global__ void __launch_bounds__(384, 1)
         }
         last_valid = has_final ? min(it.n - (it.nkb - 1) * BN, BN) : BN;
       }
-      float m_ref = 0.f, l = 0.f;
+      // With quarter masks a row half may have nothing listed in its first
+      // blocks: it then carries no reference maximum (-inf) until it does.
+      float m_ref = MODE == kModeQuarters ? -INFINITY : 0.f, l = 0.f;
+      const int qhalf = wq >> 1;  // the 64-row half of the tile this warp's rows are in
       for (int j = 0; j < len; ++j) {
+        // this block's listed key halves for the warp's query half
+        const uint32_t qbits =
+            MODE == kModeQuarters ? (__ldg(p.tile_mask + a0 + j) >> (2 * qhalf)) & 3u : 3u;
         if (!(ok = warp_wait(&bar_s_full[t], scnt & 1u, wc, kBarSFull, scnt))) break;
         ++scnt;
         tc_fence_after();
@@ -705,6 +718,13 @@ __global__ void __launch_bounds__(384, 1)
           for (int c = 0; c < BN; ++c)
             if (c >= valid) s[c] = -INFINITY;
         }
+        if (MODE == kModeQuarters && qbits != 3u) {  // an unlisted key half
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (!((qbits >> (c >> 6)) & 1u)) s[c] = -INFINITY;
+        }
+        // a column the row attends in this block (used when S is re-read)
+        auto col_ok = [&](int c) { return c < valid && ((qbits >> (c >> 6)) & 1u); };
         auto row_max = [&]() {
           float m8[8];
 #pragma unroll
@@ -725,16 +745,30 @@ __global__ void __launch_bounds__(384, 1)
         float alpha = 1.f;
         bool rescale = false;
         float sum;
-        if (j == 0) {
+        if (MODE == kModeQuarters) {
+          // rows without a reference yet take this block's maximum (still
+          // -inf when none of the row's columns here is listed); the vote
+          // keeps the branch warp-uniform
+          if (__any_sync(0xffffffffu, m_ref == -INFINITY)) {
+            const float mb = row_max() * sl2;
+            if (m_ref == -INFINITY) m_ref = mb;
+          }
+        } else if (j == 0) {
           m_ref = row_max() * sl2;
-          sum = exp_row();
+        }
+        if (MODE == kModeQuarters && m_ref == -INFINITY) {  // nothing listed yet: P = 0
+          sum = 0.f;
+#pragma unroll
+          for (int i = 0; i < BN / 2; ++i) pk[i] = 0u;
         } else {
+          sum = exp_row();
+        }
+        if (j > 0 || MODE == kModeQuarters) {
           // The reference stays the first block's maximum: P may exceed 1 by
           // far (bf16 keeps its relative precision and the fp32 sums stay
           // finite), so the row maximum is only taken again when the row sum
           // leaves [0, 2^64]; then O and l are rescaled (the final O / l and
           // lse are exact either way).
-          sum = exp_row();
           // Warp-uniform: the TMEM reads below are warp-collective
           // (.sync.aligned), so when any row of the warp needs the rescale
           // every lane takes this path (a rescale is valid for any row).
@@ -751,12 +785,14 @@ __global__ void __launch_bounds__(384, 1)
               reg_fence32(sr);
 #pragma unroll
               for (int i = 0; i < 32; ++i)
-                if (c * 32 + i < valid) mx = fmaxf(mx, __uint_as_float(sr[i]));
+                if (col_ok(c * 32 + i)) mx = fmaxf(mx, __uint_as_float(sr[i]));
             }
             const float m_new = fmaxf(m_ref, mx * sl2);
-            alpha = ex2_approx(m_ref - m_new);
+            // (a row with nothing listed so far keeps P = 0 and alpha = 1)
+            const bool has_ref = m_new != -INFINITY;
+            alpha = has_ref ? ex2_approx(m_ref - m_new) : 1.f;
             m_ref = m_new;
-            rescale = true;
+            rescale = has_ref;
             float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
             for (int c = 0; c < BN / 32; ++c) {
@@ -767,8 +803,12 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
                 const int col = c * 32 + 2 * i;
-                const float a = col < valid ? ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -m_ref)) : 0.f;
-                const float b = col + 1 < valid ? ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -m_ref)) : 0.f;
+                const float a = has_ref && col_ok(col)
+                                    ? ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -m_ref))
+                                    : 0.f;
+                const float b = has_ref && col_ok(col + 1)
+                                    ? ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -m_ref))
+                                    : 0.f;
                 acc.x += a;
                 acc.y += b;
                 pk[c * 16 + i] = pack_bf16x2(a, b);
@@ -811,7 +851,9 @@ __global__ void __launch_bounds__(384, 1)
       if (!(ok = warp_wait(&bar_o_final[t], icnt & 1u, wc, kBarODone, icnt))) break;
       ++icnt;
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      // l = 0 only for a row with nothing listed in any block (a row half
+      // whose quarters are all unlisted): out 0, lse -inf, like an empty row
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
@@ -831,7 +873,8 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
-      if (store && p.lse) p.lse[orow] = (m_ref + log2f(l)) * 0.69314718055994531f;
+      if (store && p.lse)
+        p.lse[orow] = l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_o_empty[t]);

@@ -59,6 +59,9 @@ struct FwdParams {
   long long num_pattern_columns = 0;
   const int32_t *head_list = nullptr;
   RadialGeom radial = {};
+  // Block-64 lists packed as 128-row tiles (two-tile kernel): per tile-list
+  // entry, bit qi * 2 + kj set when query half qi lists key half kj.
+  const uint8_t *tile_mask = nullptr;
 };
 
 constexpr int kSmemLimit = 232448;  // 227 KB dynamic + static per CTA on sm_100

@@ -57,7 +57,7 @@ struct DeviceInfo {
                        false, false, false, false, false, false};
   bool ref_attrs_set[4] = {false, false, false, false};
   bool gemm_attrs_set[4] = {false, false, false, false};
-  bool pair_attrs_set[8] = {false, false, false, false, false, false, false, false};
+  bool pair_attrs_set[10] = {};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -272,12 +272,32 @@ bool views_disjoint(const void *a, const bsa_layout &La, const void *b, const bs
   return r >= foot && sn - r >= foot;
 }
 
-// Forward scratch: the work order, then (256 bytes on) the work counter.
+// Forward scratch: the work order, then (256 bytes on) the work counter;
+// at block 64 then the 128-row tile lists the two-tile kernel runs on (tile
+// row pointers, tile columns, quarter masks).
 size_t order_only_bytes(const bsa_block_lists *l) {
   return (static_cast<size_t>(l->num_lists) * l->num_q_blocks * sizeof(int32_t) + 255) & ~size_t(255);
 }
 
-size_t order_bytes(const bsa_block_lists *l) { return order_only_bytes(l) + 256; }
+struct TileScratch {
+  size_t ptr, col, mask, total;  // offsets from the start of the tile lists
+};
+
+TileScratch tile_scratch(const bsa_block_lists *l) {
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t nt = (static_cast<size_t>(l->num_q_blocks) + 1) / 2;
+  const size_t cap = l->nnz > 0 ? static_cast<size_t>(l->nnz) : 1;
+  TileScratch t;
+  t.ptr = 0;
+  t.col = up((static_cast<size_t>(l->num_lists) * nt + 1) * sizeof(int32_t));
+  t.mask = t.col + up(cap * sizeof(int32_t));
+  t.total = t.mask + up(cap);
+  return t;
+}
+
+size_t order_bytes(const bsa_block_lists *l) {
+  return order_only_bytes(l) + 256 + (l->block == 64 ? tile_scratch(l).total : 0);
+}
 
 constexpr int kLptMaxRows = 12288;  // rows whose costs fit in 48 KB of shared memory
 
@@ -373,6 +393,7 @@ int launch_pair(const QkvViews &x, int32_t n, const FwdParams &p, DeviceInfo *de
     case kModeVarlen: return launch_pair_mode<D, kModeVarlen>(tq, tk, tv, p, dev, t, stream);
     case kModePatterns: return launch_pair_mode<D, kModePatterns>(tq, tk, tv, p, dev, t, stream);
     case kModeRadial: return launch_pair_mode<D, kModeRadial>(tq, tk, tv, p, dev, t, stream);
+    case kModeQuarters: return launch_pair_mode<D, kModeQuarters>(tq, tk, tv, p, dev, t, stream);
     default: return launch_pair_mode<D, kModeLists>(tq, tk, tv, p, dev, t, stream);
   }
 }
@@ -383,13 +404,69 @@ int launch_pair(const QkvViews &x, int32_t n, const FwdParams &p, DeviceInfo *de
 int run_fwd(const QkvViews &x, int32_t n, int32_t head_dim, float softmax_scale,
             const bsa_block_lists *l, void *out, const bsa_layout &lo, float *lse,
             int32_t *order, int32_t *item_counter, DeviceInfo *dev, int fault_flags,
-            cudaStream_t stream) {
+            cudaStream_t stream, uint8_t *tile_lists = nullptr) {
   const int batch = x.batch, heads = x.heads;
   const int nqb = l->num_q_blocks;
-  bool pair;
+  bool pair, force_one_tile;
   {
     std::lock_guard<std::mutex> lk(g_hook_mu);
-    pair = l->block == 128 && !g_force_one_tile;
+    force_one_tile = g_force_one_tile;
+    pair = l->block == 128 && !force_one_tile;
+  }
+  if (l->block == 64 && tile_lists && !force_one_tile) {
+    // Block 64 on the two-tile kernel: the lists merged into 128-row tile
+    // lists (each entry with its listed 64 x 64 quarters), the work order over
+    // tile-row pairs, then the kernel masking the unlisted quarters.
+    const TileScratch ts = tile_scratch(l);
+    int32_t *tile_ptr = reinterpret_cast<int32_t *>(tile_lists + ts.ptr);
+    int32_t *tile_col = reinterpret_cast<int32_t *>(tile_lists + ts.col);
+    uint8_t *tile_mask = tile_lists + ts.mask;
+    const int nt = (nqb + 1) / 2, ntk = (l->num_k_blocks + 1) / 2;
+    const int rows_t = l->num_lists * nt;
+    const long long cap = l->nnz > 0 ? l->nnz : 1;
+    tile_count_kernel<<<(rows_t + 127) / 128, 128, 0, stream>>>(
+        l->row_ptr, l->col_idx, nqb, l->num_k_blocks, l->nnz, nt, rows_t, tile_ptr);
+    BSA_CUDA(cudaGetLastError());
+    scan_rows_kernel<<<1, 1024, 0, stream>>>(tile_ptr, rows_t);
+    BSA_CUDA(cudaGetLastError());
+    tile_fill_kernel<<<(rows_t + 127) / 128, 128, 0, stream>>>(
+        l->row_ptr, l->col_idx, nqb, l->num_k_blocks, l->nnz, nt, rows_t, tile_ptr, tile_col,
+        tile_mask, cap);
+    BSA_CUDA(cudaGetLastError());
+    const int npairs = (nt + 1) / 2;
+    const size_t smem = static_cast<size_t>(npairs <= kLptMaxRows ? npairs : 0) * sizeof(int);
+    pair_order_kernel<<<l->num_lists, 1024, smem, stream>>>(tile_ptr, tile_col, nt,
+                                                           static_cast<int>(cap), order,
+                                                           kLptMaxRows, item_counter);
+    BSA_CUDA(cudaGetLastError());
+    FwdParams p;
+    p.row_ptr = tile_ptr;
+    p.col_idx = tile_col;
+    p.tile_mask = tile_mask;
+    p.order = order;
+    p.item_counter = item_counter;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.o_sb = lo.batch_stride;
+    p.o_sh = lo.head_stride;
+    p.o_sn = lo.token_stride;
+    p.lse = lse;
+    p.heads = heads;
+    p.n = n;
+    p.nqb = nt;
+    p.nkb = ntk;
+    p.num_lists = l->num_lists;
+    p.nnz = static_cast<int32_t>(cap);
+    p.total_items = batch * heads * npairs;
+    const float scale =
+        softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
+    p.scale_log2 = scale * 1.4426950408889634f;
+    {
+      std::lock_guard<std::mutex> lk(g_hook_mu);
+      p.wait_limit_ns = g_wait_limit_ns;
+    }
+    p.fault_flags = fault_flags;
+    if (head_dim == 128) return launch_pair<128>(x, n, p, dev, kModeQuarters, nullptr, stream);
+    return launch_pair<64>(x, n, p, dev, kModeQuarters, nullptr, stream);
   }
   if (pair) {
     const int npairs = (nqb + 1) / 2;
@@ -1036,7 +1113,8 @@ int bsa_attn_fwd(const void *q, const void *k, const void *v, int32_t batch, int
                                                  order_only_bytes(l));
   return run_fwd(contiguous_views(q, k, v, batch, heads, n, head_dim), n, head_dim,
                  softmax_scale, l, out, contiguous_layout(heads, n, head_dim), lse, order,
-                 counter, dev, fault_flags, stream);
+                 counter, dev, fault_flags, stream,
+                 static_cast<uint8_t *>(workspace) + order_only_bytes(l) + 256);
 }
 
 int bsa_attn_fwd_strided(const void *q, const bsa_layout *q_layout, const void *k,
@@ -1074,7 +1152,7 @@ int bsa_attn_fwd_strided(const void *q, const bsa_layout *q_layout, const void *
   int32_t *counter = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) +
                                                  order_only_bytes(l));
   return run_fwd(x, n, head_dim, softmax_scale, l, out, *out_layout, lse, order, counter, dev,
-                 fault_flags, stream);
+                 fault_flags, stream, static_cast<uint8_t *>(workspace) + order_only_bytes(l) + 256);
 }
 
 size_t bsa_attn_fwd_varlen_workspace_bytes(int32_t num_items, const int32_t *cu_seqlens,

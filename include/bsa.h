@@ -210,7 +210,9 @@ int bsa_tile_pattern_lists_build(int32_t num_lists, int32_t num_q_blocks,
 /*
  * Bytes of device scratch memory bsa_attn_fwd needs for this problem (the
  * longest-row-first work order of every list and a work counter the kernel's
- * CTAs take items from). Returns 0 for invalid lists.
+ * CTAs take items from; at block 64 also the lists merged into 128-row tile
+ * lists, about 5 bytes per list entry, on which block-64 problems run).
+ * Returns 0 for invalid lists.
  */
 size_t bsa_attn_fwd_workspace_bytes(int32_t batch, int32_t heads, const bsa_block_lists *lists);
 
@@ -677,9 +679,10 @@ const char *bsa_last_cuda_error(void);
  * bsa_attn_fwd launch skip its first K-tile load, so that the consumer's
  * bounded wait runs out and the call reports BSA_ERR_DEVICE_TIMEOUT through
  * bsa_get_device_status(); the flag clears itself after one launch.
- * `fault_flags` bit 1 (sticky until the next call) runs block-128 problems on
- * the one-tile kernel instead of the two-tile kernel, so that tests can
- * compare the two schedules; it changes no result beyond rounding order.
+ * `fault_flags` bit 1 (sticky until the next call) runs every problem on the
+ * one-tile kernel instead of the two-tile kernel (block 128 directly, block
+ * 64 without packing its blocks into 128-row tiles), so that tests can compare
+ * the two schedules; it changes no result beyond rounding order.
  */
 int bsa_set_test_hooks(int64_t wait_limit_ns, int32_t fault_flags);
 
@@ -700,7 +703,9 @@ int bsa_selftest_exp2(const float *x, float *y_poly, float *y_mufu, float *y_ref
  * allocator, or a runtime whose memory plan is fixed at start-up and forbids
  * later allocations. Those callers cannot provide bsa_attn_fwd's workspace.
  *
- * Same operation, arguments and results as bsa_attn_fwd, minus the workspace:
+ * Same operation, arguments and results as bsa_attn_fwd, minus the workspace
+ * (block-64 problems run on the one-tile kernel here, without the tile
+ * lists that would need more scratch):
  * the scratch it needs (the longest-first work order and the work counter)
  * lives in a fixed array compiled into the library, of
  * BSA_NOALLOC_MAX_ORDER_ENTRIES + 64 int32 entries (256 KiB + 256 B). The work

@@ -8,7 +8,8 @@ shared by every call. These tests call it through the C ABI on several
 problems in a row, so later calls reuse the array earlier ones filled, and
 compare each result with bsa_attn_fwd on the same inputs. Both entries run the
 same kernels on the same lists in the same order, so the results must be
-bit-identical. The file is collected last so that a run stopping at the first
+bit-identical (at block 64 the allocation-free entry runs the one-tile kernel,
+and the reference is taken on that kernel too). The file is collected last so that a run stopping at the first
 failure has already run everything else; it also passes alone in a fresh
 process.
 """
@@ -92,7 +93,15 @@ def test_noalloc_at_the_scratch_limit(bsa):
     # query blocks fills the whole array, and the work counter sits after it.
     nqb = bsa.NOALLOC_MAX_ORDER_ENTRIES
     q, k, v, lists = _long_sequence(bsa, nqb)
-    ref = bsa.attention(q, k, v, lists)
+    # the workspace entry packs block-64 problems into 128-row tiles on the
+    # two-tile kernel; the allocation-free entry has no room for those tile
+    # lists and runs the one-tile kernel, so the reference takes that kernel
+    # too (test hook bit 1) and the results must again be identical
+    try:
+        bsa.bsa_set_test_hooks(0, 2)
+        ref = bsa.attention(q, k, v, lists)
+    finally:
+        bsa.bsa_set_test_hooks(0, 0)
     got = _run_noalloc(bsa, q, k, v, lists)
     assert bsa.bsa_get_device_status() == 0
     _assert_identical(got, ref, "noalloc at the limit (block 64, one list)")

@@ -22,6 +22,8 @@ The shapes stand in for the video-DiT workloads the pages measure on
 * ``hunyuan_text``  the hunyuan grid followed by 256 joint text tokens
                (n=119056; HunyuanVideo-style joint text + video attention),
                same value recipe, seed 5.
+* ``wan_b64``  the wan problem (same tensors, seed 1) with the radial mask cut
+               at block 64.
 """
 
 from __future__ import annotations
@@ -61,6 +63,7 @@ WORKLOADS = {
     "generic": Workload("generic", 1, 24, 128, 32768, 128, 4, "normal_scaled", radial=False),
     "hunyuan_text": Workload("hunyuan_text", 1, 24, 128, 33 * 3600 + 256, 128, 5,
                              "normal_token_scale", 33, 3600, text_tokens=256),
+    "wan_b64": Workload("wan_b64", 1, 40, 128, 21 * 1560, 64, 1, "normal_scaled", 21, 1560),
 }
 
 
