@@ -30,6 +30,7 @@ __all__ = [
     "computed_flops", "bsa_attn_fwd_noalloc", "bsa_selftest_exp2", "NOALLOC_MAX_ORDER_ENTRIES",
     "bsa_gemm_bf16", "bsa_joint_mask_build_varlen", "bsa_attn_fwd_varlen",
     "bsa_attn_fwd_varlen_workspace_bytes", "radial_block_lists_varlen", "attention_varlen",
+    "bsa_attn_bwd_varlen", "bsa_attn_bwd_varlen_workspace_bytes", "attention_varlen_backward",
     "bsa_attn_fwd_patterns", "bsa_attn_fwd_radial",
     "bsa_attn_fwd_strided", "bsa_attn_module_workspace_bytes", "bsa_joint_mask_build",
     "bsa_attn_fwd_host", "bsa_attn_fwd_host_workspace_bytes", "bsa_attn_bwd_strided",
@@ -250,6 +251,13 @@ def _cu_array(cu_seqlens):
     return len(cu) - 1, (ctypes.c_int32 * len(cu))(*cu)
 
 
+def _packed_layout(t):
+    """Layout of a packed [total, heads, head_dim] view (contiguous last axis)."""
+    if t.dim() != 3 or t.stride(2) != 1:
+        raise ValueError("expected a [total, heads, head_dim] view with a contiguous last axis")
+    return LayoutC(0, t.stride(1), t.stride(0))
+
+
 def bsa_attn_fwd_varlen_workspace_bytes(cu_seqlens, heads: int, lists: BlockLists) -> int:
     k, cu = _cu_array(cu_seqlens)
     return int(_lib.load().bsa_attn_fwd_varlen_workspace_bytes(k, cu, heads,
@@ -268,18 +276,40 @@ def bsa_attn_fwd_varlen(q, k, v, cu_seqlens, lists: BlockLists, out, lse=None, w
         workspace = torch.empty(max(lib.bsa_attn_fwd_varlen_workspace_bytes(
             nitems, cu, H, ctypes.byref(ls)), 16), dtype=torch.uint8, device=q.device)
 
-    def lay(t):
-        if t.dim() != 3 or t.stride(2) != 1:
-            raise ValueError("expected a [total, heads, head_dim] view with a contiguous last axis")
-        return LayoutC(0, t.stride(1), t.stride(0))
-
-    lq, lk, lv, lo = (lay(t) for t in (q, k, v, out))
+    lq, lk, lv, lo = (_packed_layout(t) for t in (q, k, v, out))
     st = lib.bsa_attn_fwd_varlen(_ptr(q), ctypes.byref(lq), _ptr(k), ctypes.byref(lk), _ptr(v),
                                  ctypes.byref(lv), nitems, cu, H, D, float(softmax_scale),
                                  ctypes.byref(ls), _ptr(out), ctypes.byref(lo), _ptr(lse),
                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
                                  _stream(stream))
     _check(st, "bsa_attn_fwd_varlen")
+
+
+def bsa_attn_bwd_varlen_workspace_bytes(cu_seqlens, heads: int, lists: BlockLists) -> int:
+    k, cu = _cu_array(cu_seqlens)
+    return int(_lib.load().bsa_attn_bwd_varlen_workspace_bytes(k, cu, heads,
+                                                               ctypes.byref(lists.c_struct())))
+
+
+def bsa_attn_bwd_varlen(q, k, v, out, dout, lse, cu_seqlens, lists: BlockLists, dq, dk, dv,
+                        workspace=None, softmax_scale: float = 0.0, stream=None) -> None:
+    """Variable-length batch backward on packed [total, heads, head_dim] tensors;
+    lse is the forward's [heads, total]."""
+    total, H, D = q.shape
+    lib = _lib.load()
+    ls = lists.c_struct()
+    nitems, cu = _cu_array(cu_seqlens)
+    if workspace is None:
+        workspace = torch.empty(max(lib.bsa_attn_bwd_varlen_workspace_bytes(
+            nitems, cu, H, ctypes.byref(ls)), 16), dtype=torch.uint8, device=q.device)
+    lay = [_packed_layout(t) for t in (q, k, v, out, dout, dq, dk, dv)]
+    st = lib.bsa_attn_bwd_varlen(
+        _ptr(q), ctypes.byref(lay[0]), _ptr(k), ctypes.byref(lay[1]), _ptr(v), ctypes.byref(lay[2]),
+        _ptr(out), ctypes.byref(lay[3]), _ptr(dout), ctypes.byref(lay[4]), _ptr(lse), nitems, cu,
+        H, D, float(softmax_scale), ctypes.byref(ls), _ptr(dq), ctypes.byref(lay[5]), _ptr(dk),
+        ctypes.byref(lay[6]), _ptr(dv), ctypes.byref(lay[7]), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "bsa_attn_bwd_varlen")
 
 
 def bsa_attn_fwd_host_workspace_bytes(batch: int, heads: int, n: int, head_dim: int,
@@ -564,6 +594,16 @@ def attention_varlen(q, k, v, cu_seqlens, lists: BlockLists, softmax_scale: floa
     lse = torch.empty((H, total), dtype=torch.float32, device=q.device) if want_lse else None
     bsa_attn_fwd_varlen(q, k, v, cu_seqlens, lists, out, lse, None, softmax_scale, stream)
     return out, lse
+
+
+def attention_varlen_backward(q, k, v, out, dout, lse, cu_seqlens, lists: BlockLists,
+                              softmax_scale: float = 0.0, stream=None):
+    """Gradients ``(dq, dk, dv)`` of :func:`attention_varlen` (packed
+    [total, heads, head_dim]; lse [heads, total] from the forward)."""
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    bsa_attn_bwd_varlen(q, k, v, out, dout, lse, cu_seqlens, lists, dq, dk, dv, None,
+                        softmax_scale, stream)
+    return dq, dk, dv
 
 
 def pack_tile_patterns(patterns, device=None):

@@ -38,6 +38,8 @@ EXPORTS = (
     "bsa_attn_dense_masked_ref",
     "bsa_attn_bwd",
     "bsa_attn_bwd_strided",
+    "bsa_attn_bwd_varlen_workspace_bytes",
+    "bsa_attn_bwd_varlen",
     "bsa_attn_bwd_workspace_bytes",
     "bsa_attn_bwd_host_workspace_bytes",
     "bsa_attn_bwd_host",
@@ -173,6 +175,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bsa_attn_bwd_strided": (ctypes.c_int, [vp, yp, vp, yp, vp, yp, vp, yp, vp, yp, vp, i32,
                                                 i32, i32, i32, ctypes.c_float, lp, vp, yp, vp, yp,
                                                 vp, yp, vp, sz, vp]),
+        "bsa_attn_bwd_varlen_workspace_bytes": (sz, [i32, vp, i32, lp]),
+        "bsa_attn_bwd_varlen": (ctypes.c_int, [vp, yp, vp, yp, vp, yp, vp, yp, vp, yp, vp, i32,
+                                               vp, i32, i32, ctypes.c_float, lp, vp, yp, vp, yp,
+                                               vp, yp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

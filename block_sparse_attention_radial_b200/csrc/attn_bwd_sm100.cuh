@@ -66,13 +66,14 @@ constexpr int kBwdItemN = 4;  // work items in flight between the producer and t
 // ------------------------------------------------------------------ prep --
 
 // One thread per padded query row of one (batch*head): delta and lse2.
-// out and dout are read through their (batch, head, token) element strides.
+// out and dout are read through their (batch, head, token) element strides,
+// lse through its (batch, head) strides l_sb, l_sh (rows contiguous).
 template <int D>
 __global__ void bwd_prep_kernel(const __nv_bfloat16 *out, const __nv_bfloat16 *dout,
                                 const float *lse, float *lse2, float *delta, int n, int nqb,
                                 int heads, long long o_sb, long long o_sh, long long o_sn,
-                                long long d_sb, long long d_sh, long long d_sn,
-                                long long rows_total, int32_t *item_counters) {
+                                long long d_sb, long long d_sh, long long d_sn, long long l_sb,
+                                long long l_sh, long long rows_total, int32_t *item_counters) {
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx < 2) item_counters[idx] = 0;  // the dK/dV and the dQ kernel's work counters
   if (idx >= rows_total) return;
@@ -84,8 +85,8 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16 *out, const __nv_bfloat16 *d
     delta[idx] = 0.f;
     return;
   }
-  const long long row = bh * n + i;
   const long long b = bh / heads, h = bh - b * heads;
+  const long long row = b * l_sb + h * l_sh + i;
   const uint4 *o4 = reinterpret_cast<const uint4 *>(out + b * o_sb + h * o_sh + i * o_sn);
   const uint4 *d4 = reinterpret_cast<const uint4 *>(dout + b * d_sb + h * d_sh + i * d_sn);
   float acc = 0.f;

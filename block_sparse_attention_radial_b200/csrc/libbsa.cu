@@ -660,6 +660,7 @@ struct BwdViews {
   void *dq, *dk, *dv;
   bsa_layout lq, lk, lv, lo, ldo, ldq, ldk, ldv;
   int batch, heads;
+  long long lse_sb = -1, lse_sh = -1;  // lse's batch / head strides; -1: contiguous [B, H, n]
 };
 
 template <int D>
@@ -704,10 +705,12 @@ int launch_bwd(const BwdViews &x, const float *lse, int32_t n, float softmax_sca
   const int nqb = l->num_q_blocks, nkb = l->num_k_blocks;
 
   const long long rows = static_cast<long long>(bh) * nqb * kBwdBlock;
+  const long long l_sh = x.lse_sh >= 0 ? x.lse_sh : n;
+  const long long l_sb = x.lse_sb >= 0 ? x.lse_sb : static_cast<long long>(x.heads) * n;
   bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 255) / 256), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16 *>(x.out), static_cast<const __nv_bfloat16 *>(x.dout), lse,
       lse2, delta, n, nqb, x.heads, x.lo.batch_stride, x.lo.head_stride, x.lo.token_stride,
-      x.ldo.batch_stride, x.ldo.head_stride, x.ldo.token_stride, rows,
+      x.ldo.batch_stride, x.ldo.head_stride, x.ldo.token_stride, l_sb, l_sh, rows,
       reinterpret_cast<int32_t *>(ws + w.counters));
   BSA_CUDA(cudaGetLastError());
   const int cols = l->num_lists * nkb;
@@ -1410,6 +1413,89 @@ int bsa_attn_fwd_radial(const void *q, const void *k, const void *v, int32_t bat
   return launch_pair<64>(x, n, p, dev, kModeRadial, nullptr, stream);
 }
 
+}  // extern "C"
+
+namespace {
+
+// Argument checks shared by the strided and variable-length backward entries:
+// the eight views of [batch, heads, n, head_dim] (q, k, v, out, dout, dq, dk,
+// dv), lse (lbytes bytes) and `need` bytes of workspace.
+int check_bwd_views(const void *const ptrs[8], const bsa_layout *const lays[8], const float *lse,
+                    int32_t batch, int32_t heads, int32_t n, int32_t head_dim, size_t lbytes,
+                    const void *workspace, size_t workspace_bytes, size_t need) {
+  for (int i = 0; i < 8; ++i) {
+    if (!aligned16(ptrs[i])) return BSA_ERR_INVALID_ARG;
+    if (!layout_ok(*lays[i], batch, heads, n)) return BSA_ERR_INVALID_ARG;
+  }
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return BSA_ERR_INVALID_ARG;
+  size_t span[8];
+  for (int i = 0; i < 8; ++i) span[i] = layout_span_bytes(*lays[i], batch, heads, n, head_dim);
+  for (int a = 5; a < 8; ++a) {  // the gradients
+    if (!layout_disjoint(*lays[a], batch, heads, n, head_dim)) return BSA_ERR_INVALID_ARG;
+    for (int b = 0; b < 5; ++b)
+      if (overlaps(ptrs[a], span[a], ptrs[b], span[b])) return BSA_ERR_INVALID_ARG;
+    if (overlaps(ptrs[a], span[a], lse, lbytes)) return BSA_ERR_INVALID_ARG;
+    for (int b = a + 1; b < 8; ++b)
+      if (!views_disjoint(ptrs[a], *lays[a], ptrs[b], *lays[b], batch, heads, n, head_dim))
+        return BSA_ERR_INVALID_ARG;
+  }
+  if (!workspace || !aligned16(workspace) || workspace_bytes < need) return BSA_ERR_INVALID_ARG;
+  for (int i = 0; i < 8; ++i)
+    if (overlaps(workspace, need, ptrs[i], span[i])) return BSA_ERR_INVALID_ARG;
+  if (overlaps(workspace, need, lse, lbytes)) return BSA_ERR_INVALID_ARG;
+  return BSA_OK;
+}
+
+BwdViews bwd_views(const void *const ptrs[8], const bsa_layout *const lays[8], int batch,
+                   int heads) {
+  BwdViews x;
+  x.q = ptrs[0];
+  x.k = ptrs[1];
+  x.v = ptrs[2];
+  x.out = ptrs[3];
+  x.dout = ptrs[4];
+  x.dq = const_cast<void *>(ptrs[5]);
+  x.dk = const_cast<void *>(ptrs[6]);
+  x.dv = const_cast<void *>(ptrs[7]);
+  x.lq = *lays[0];
+  x.lk = *lays[1];
+  x.lv = *lays[2];
+  x.lo = *lays[3];
+  x.ldo = *lays[4];
+  x.ldq = *lays[5];
+  x.ldk = *lays[6];
+  x.ldv = *lays[7];
+  x.batch = batch;
+  x.heads = heads;
+  return x;
+}
+
+// Item b's share of concatenated variable-length lists: its L * nqb_b rows
+// (offsets into the shared col_idx), nqb_b query and key blocks.
+bsa_block_lists varlen_item_lists(const bsa_block_lists *l, const VarlenTable &vt, int b) {
+  bsa_block_lists sub = *l;
+  const int nqb = vt.row0[b + 1] - vt.row0[b];
+  sub.row_ptr = l->row_ptr + static_cast<long long>(l->num_lists) * vt.row0[b];
+  sub.num_q_blocks = sub.num_k_blocks = nqb;
+  return sub;
+}
+
+size_t varlen_bwd_bytes(const VarlenTable &vt, int heads, const bsa_block_lists *l) {
+  size_t mx = 256;
+  for (int b = 0; b < vt.num_items; ++b) {
+    const int n_b = vt.tok0[b + 1] - vt.tok0[b];
+    if (n_b == 0) continue;
+    const bsa_block_lists sub = varlen_item_lists(l, vt, b);
+    const size_t t = bwd_layout(1, heads, n_b, &sub).total;
+    mx = t > mx ? t : mx;
+  }
+  return mx;
+}
+
+}  // namespace
+
+extern "C" {
+
 int bsa_attn_bwd_strided(const void *q, const bsa_layout *q_layout, const void *k,
                          const bsa_layout *k_layout, const void *v, const bsa_layout *v_layout,
                          const void *out, const bsa_layout *out_layout, const void *dout,
@@ -1435,54 +1521,91 @@ int bsa_attn_bwd_strided(const void *q, const bsa_layout *q_layout, const void *
   if (l->nnz < 0) return BSA_ERR_INVALID_ARG;
   const long long bhl = static_cast<long long>(batch) * heads;
   if (bhl * nb > 0x7fffffffLL || bhl * n > 0x7fffffffLL) return BSA_ERR_UNSUPPORTED;
-  for (int i = 0; i < 8; ++i) {
-    if (!aligned16(ptrs[i])) return BSA_ERR_INVALID_ARG;
-    if (!layout_ok(*lays[i], batch, heads, n)) return BSA_ERR_INVALID_ARG;
-  }
-  if (reinterpret_cast<uintptr_t>(lse) & 3u) return BSA_ERR_INVALID_ARG;
-  size_t span[8];
-  for (int i = 0; i < 8; ++i) span[i] = layout_span_bytes(*lays[i], batch, heads, n, head_dim);
   const size_t lbytes = static_cast<size_t>(bhl) * n * sizeof(float);
-  for (int a = 5; a < 8; ++a) {  // the gradients
-    if (!layout_disjoint(*lays[a], batch, heads, n, head_dim)) return BSA_ERR_INVALID_ARG;
-    for (int b = 0; b < 5; ++b)
-      if (overlaps(ptrs[a], span[a], ptrs[b], span[b])) return BSA_ERR_INVALID_ARG;
-    if (overlaps(ptrs[a], span[a], lse, lbytes)) return BSA_ERR_INVALID_ARG;
-    for (int b = a + 1; b < 8; ++b)
-      if (!views_disjoint(ptrs[a], *lays[a], ptrs[b], *lays[b], batch, heads, n, head_dim))
-        return BSA_ERR_INVALID_ARG;
-  }
   const size_t need = bwd_layout(batch, heads, n, l).total;
-  if (!workspace || !aligned16(workspace) || workspace_bytes < need) return BSA_ERR_INVALID_ARG;
-  for (int i = 0; i < 8; ++i)
-    if (overlaps(workspace, need, ptrs[i], span[i])) return BSA_ERR_INVALID_ARG;
-  if (overlaps(workspace, need, lse, lbytes)) return BSA_ERR_INVALID_ARG;
+  int st = check_bwd_views(ptrs, lays, lse, batch, heads, n, head_dim, lbytes, workspace,
+                           workspace_bytes, need);
+  if (st != BSA_OK) return st;
   DeviceInfo *dev = nullptr;
-  int st;
   if ((st = current_device(&dev)) != BSA_OK) return st;
   if (dev->cc_major != 10) return BSA_ERR_UNSUPPORTED;
-  BwdViews x;
-  x.q = q;
-  x.k = k;
-  x.v = v;
-  x.out = out;
-  x.dout = dout;
-  x.dq = dq;
-  x.dk = dk;
-  x.dv = dv;
-  x.lq = *q_layout;
-  x.lk = *k_layout;
-  x.lv = *v_layout;
-  x.lo = *out_layout;
-  x.ldo = *dout_layout;
-  x.ldq = *dq_layout;
-  x.ldk = *dk_layout;
-  x.ldv = *dv_layout;
-  x.batch = batch;
-  x.heads = heads;
+  const BwdViews x = bwd_views(ptrs, lays, batch, heads);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   if (head_dim == 128) return launch_bwd<128>(x, lse, n, softmax_scale, l, ws, dev, stream);
   return launch_bwd<64>(x, lse, n, softmax_scale, l, ws, dev, stream);
+}
+
+size_t bsa_attn_bwd_varlen_workspace_bytes(int32_t num_items, const int32_t *cu_seqlens,
+                                           int32_t heads, const bsa_block_lists *l) {
+  if (!l || heads < 1 || l->block != 128 || (l->num_lists != 1 && l->num_lists != heads))
+    return 0;
+  VarlenTable vt;
+  int32_t mx = 0;
+  if (varlen_table(num_items, cu_seqlens, heads, 128, &vt, &mx) != BSA_OK) return 0;
+  return varlen_bwd_bytes(vt, heads, l);
+}
+
+int bsa_attn_bwd_varlen(const void *q, const bsa_layout *q_layout, const void *k,
+                        const bsa_layout *k_layout, const void *v, const bsa_layout *v_layout,
+                        const void *out, const bsa_layout *out_layout, const void *dout,
+                        const bsa_layout *dout_layout, const float *lse, int32_t num_items,
+                        const int32_t *cu_seqlens, int32_t heads, int32_t head_dim,
+                        float softmax_scale, const bsa_block_lists *l, void *dq,
+                        const bsa_layout *dq_layout, void *dk, const bsa_layout *dk_layout,
+                        void *dv, const bsa_layout *dv_layout, void *workspace,
+                        size_t workspace_bytes, bsa_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const bsa_layout *lays[8] = {q_layout, k_layout,  v_layout,  out_layout,
+                               dout_layout, dq_layout, dk_layout, dv_layout};
+  const void *ptrs[8] = {q, k, v, out, dout, dq, dk, dv};
+  for (int i = 0; i < 8; ++i)
+    if (!lays[i] || !ptrs[i]) return BSA_ERR_INVALID_ARG;
+  if (!lse || !l || !l->row_ptr || (l->nnz > 0 && !l->col_idx)) return BSA_ERR_INVALID_ARG;
+  if (heads < 1) return BSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
+  if (l->block != 128) return BSA_ERR_UNSUPPORTED;
+  if (l->num_lists != 1 && l->num_lists != heads) return BSA_ERR_INVALID_ARG;
+  if (l->nnz < 0) return BSA_ERR_INVALID_ARG;
+  VarlenTable vt;
+  int32_t max_nqb = 0;
+  int st;
+  if ((st = varlen_table(num_items, cu_seqlens, heads, l->block, &vt, &max_nqb)) != BSA_OK)
+    return st;
+  const int32_t total = cu_seqlens[num_items];
+  if (l->num_q_blocks != vt.row0[num_items] || l->num_k_blocks != max_nqb)
+    return BSA_ERR_INVALID_ARG;
+  if (static_cast<long long>(heads) * total > 0x7fffffffLL ||
+      static_cast<long long>(l->num_lists) * l->num_q_blocks > 0x7fffffffLL ||
+      static_cast<long long>(heads) * max_nqb * kBwdBlock > 0x7fffffffLL)
+    return BSA_ERR_UNSUPPORTED;
+  // the packed sequence is a batch of one: [1, heads, total, head_dim] views
+  const size_t lbytes = static_cast<size_t>(heads) * total * sizeof(float);
+  const size_t need = varlen_bwd_bytes(vt, heads, l);
+  if ((st = check_bwd_views(ptrs, lays, lse, 1, heads, total, head_dim, lbytes, workspace,
+                            workspace_bytes, need)) != BSA_OK)
+    return st;
+  DeviceInfo *dev = nullptr;
+  if ((st = current_device(&dev)) != BSA_OK) return st;
+  if (dev->cc_major != 10) return BSA_ERR_UNSUPPORTED;
+  // one backward per item on its slice of the packed views; the items run
+  // one after another on `stream` and reuse the workspace
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  for (int b = 0; b < num_items; ++b) {
+    const int32_t t0 = vt.tok0[b], n_b = vt.tok0[b + 1] - t0;
+    if (n_b == 0) continue;
+    const void *item[8];
+    for (int i = 0; i < 8; ++i)
+      item[i] = static_cast<const uint8_t *>(ptrs[i]) +
+                static_cast<long long>(t0) * lays[i]->token_stride * 2;
+    BwdViews x = bwd_views(item, lays, 1, heads);
+    x.lse_sb = static_cast<long long>(heads) * total;
+    x.lse_sh = total;
+    const bsa_block_lists sub = varlen_item_lists(l, vt, b);
+    st = head_dim == 128 ? launch_bwd<128>(x, lse + t0, n_b, softmax_scale, &sub, ws, dev, stream)
+                         : launch_bwd<64>(x, lse + t0, n_b, softmax_scale, &sub, ws, dev, stream);
+    if (st != BSA_OK) return st;
+  }
+  return BSA_OK;
 }
 
 size_t bsa_attn_bwd_workspace_bytes(int32_t batch, int32_t heads, int32_t n,

@@ -599,6 +599,48 @@ int bsa_attn_bwd_strided(const void *q, const bsa_layout *q_layout,
                          void *workspace, size_t workspace_bytes, bsa_stream_t stream);
 
 /*
+ * Bytes of device scratch bsa_attn_bwd_varlen needs: the largest item's
+ * bsa_attn_bwd scratch (the items reuse it one after another). 0 for invalid
+ * arguments.
+ */
+size_t bsa_attn_bwd_varlen_workspace_bytes(int32_t num_items, const int32_t *cu_seqlens,
+                                           int32_t heads, const bsa_block_lists *lists);
+
+/*
+ * bsa_attn_bwd on a variable-length batch packed as for bsa_attn_fwd_varlen:
+ * item b owns tokens [cu_seqlens[b], cu_seqlens[b+1]) of q, k, v, out, dout,
+ * dq, dk and dv, and its gradients are those of bsa_attn_bwd on that item
+ * alone with its own lists (the pages treat one sequence at a time; batching
+ * sequences of different lengths is this library's reading).
+ * q, k, v, out, dout, dq, dk, dv  device bf16 views of [1, heads, total,
+ *        head_dim] (batch_stride unused), total = cu_seqlens[num_items]; layout
+ *        rules as bsa_attn_bwd_strided with batch 1 and n = total.
+ * lse    the forward's fp32 [heads, total] log-sum-exp (required), as
+ *        bsa_attn_fwd_varlen writes it.
+ * num_items, cu_seqlens, lists  as for bsa_attn_fwd_varlen (block 128).
+ * workspace  bsa_attn_bwd_varlen_workspace_bytes() bytes of device scratch,
+ *        16-byte aligned, overlapping no view and not lse.
+ * The items run one after another on `stream` (six launches each: prep,
+ * the three passes of the transposed lists, dK/dV, dQ); tokens of empty
+ * items are not touched. Each item's gradients are bit-identical to
+ * bsa_attn_bwd on that item alone. Deterministic. Returns
+ * BSA_ERR_UNSUPPORTED for block 64 or head_dim other than 64 / 128; other
+ * errors as bsa_attn_bwd_strided. Asynchronous.
+ */
+int bsa_attn_bwd_varlen(const void *q, const bsa_layout *q_layout,
+                        const void *k, const bsa_layout *k_layout,
+                        const void *v, const bsa_layout *v_layout,
+                        const void *out, const bsa_layout *out_layout,
+                        const void *dout, const bsa_layout *dout_layout,
+                        const float *lse, int32_t num_items, const int32_t *cu_seqlens,
+                        int32_t heads, int32_t head_dim, float softmax_scale,
+                        const bsa_block_lists *lists,
+                        void *dq, const bsa_layout *dq_layout,
+                        void *dk, const bsa_layout *dk_layout,
+                        void *dv, const bsa_layout *dv_layout,
+                        void *workspace, size_t workspace_bytes, bsa_stream_t stream);
+
+/*
  * Workspace bytes bsa_attn_bwd needs: per query row of every (batch, head),
  * lse * log2(e) and delta, padded to whole 128-row tiles (2 x 4 bytes), plus
  * the transposed lists (num_lists * ceil(n / 128) + 1 offsets, nnz entries);

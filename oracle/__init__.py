@@ -30,7 +30,7 @@ Modules:
 * ``tile_patterns``: per-head tile patterns (diagonal and multi-diagonal
   bands, vertical stripes, dual windows) expanded into block lists.
 * ``varlen``: variable-length batches (items with their own lists,
-  concatenated; attention item by item).
+  concatenated; attention and its gradients item by item).
 """
 
 from .radial_mask import (  # noqa: F401
@@ -67,6 +67,7 @@ from .varlen import (  # noqa: F401
     varlen_block_lists,
     split_item_lists,
     varlen_masked_attention_fp64,
+    varlen_masked_attention_backward_fp64,
 )
 from .module import (  # noqa: F401
     radial_attention_module_fp64,

@@ -16,6 +16,7 @@ from __future__ import annotations
 import numpy as np
 
 from .attention import masked_attention_fp64
+from .attention_backward import masked_attention_backward_fp64
 from .radial_mask import joint_block_lists
 
 
@@ -71,3 +72,24 @@ def varlen_masked_attention_fp64(q, k, v, cu_seqlens, item_lists, num_lists: int
         out[sl] = np.transpose(o[0], (1, 0, 2))
         lse[:, sl] = l_[0]
     return out, lse
+
+
+def varlen_masked_attention_backward_fp64(q, k, v, do, cu_seqlens, item_lists, num_lists: int,
+                                          block: int, scale: float | None = None):
+    """Gradients of ``varlen_masked_attention_fp64``: item by item, the
+    single-problem gradients (dQ, dK, dV) on the item's tokens; packed
+    ``[total, heads, D]`` float64 arrays, zero on no token."""
+    q, k, v, do = (np.asarray(x, dtype=np.float64) for x in (q, k, v, do))
+    total, H, D = q.shape
+    grads = [np.zeros((total, H, D)) for _ in range(3)]
+    for b, (rp, ci) in enumerate(item_lists):
+        t0, t1 = int(cu_seqlens[b]), int(cu_seqlens[b + 1])
+        if t1 == t0:
+            continue
+        sl = slice(t0, t1)
+        as_bhnd = lambda x: np.transpose(x[sl], (1, 0, 2))[None]  # noqa: E731
+        gs = masked_attention_backward_fp64(as_bhnd(q), as_bhnd(k), as_bhnd(v), as_bhnd(do), rp,
+                                            ci, num_lists, block, scale=scale)
+        for g, gi in zip(grads, gs):
+            g[sl] = np.transpose(gi[0], (1, 0, 2))
+    return tuple(grads)

@@ -439,6 +439,52 @@ def test_varlen_host_checks(lib):
     assert lib.bsa_joint_mask_build_varlen(2, fr2, tp, tx, 96, rp, None, 0, None, None) == 2
 
 
+def test_varlen_backward_host_checks(lib):
+    """bsa_attn_bwd_varlen rejects malformed arguments on the host, before any
+    CUDA call."""
+    from block_sparse_attention_radial_b200._lib import BlockListsC, LayoutC
+
+    vp, ref = ctypes.c_void_p, ctypes.byref
+    H, D = 2, 128
+    cu_ok = (ctypes.c_int32 * 4)(0, 300, 300, 700)        # nqb 3, 0, 4 at block 128
+    lay = LayoutC(0, D, H * D)                            # packed [total, H, D]
+    bufs = [vp(a << 30) for a in range(1, 9)]             # q k v out dout dq dk dv
+    lse, w = vp(9 << 30), vp(10 << 30)
+
+    def lists(nq=7, nk=4, block=128, L=1):
+        return BlockListsC(L, nq, nk, block, 10, 1 << 22, 1 << 23)
+
+    def call(ls=None, cu=cu_ok, items=3, wsb=1 << 24, hd=D, lse_=lse, dq=None):
+        ls = lists() if ls is None else ls
+        p = list(bufs)
+        if dq is not None:
+            p[5] = dq
+        return lib.bsa_attn_bwd_varlen(p[0], ref(lay), p[1], ref(lay), p[2], ref(lay), p[3],
+                                       ref(lay), p[4], ref(lay), lse_, items, cu, H, hd, 0.0,
+                                       ref(ls), p[5], ref(lay), p[6], ref(lay), p[7], ref(lay), w,
+                                       wsb, None)
+
+    ws = lib.bsa_attn_bwd_varlen_workspace_bytes(3, cu_ok, H, ref(lists()))
+    # the largest item (400 tokens, 4 tiles): lse2 + delta for 2 x 512 rows,
+    # counters, 4 + 1 column pointers, 10 entries, 256-byte aligned
+    assert ws == 4096 + 4096 + 256 + 256 + 256
+    assert lib.bsa_attn_bwd_varlen_workspace_bytes(3, cu_ok, H, ref(lists(block=64))) == 0
+    assert call(items=0) == 1 and call(items=65) == 1
+    assert call(cu=(ctypes.c_int32 * 4)(1, 300, 300, 700)) == 1      # cu[0] != 0
+    assert call(cu=(ctypes.c_int32 * 4)(0, 300, 200, 700)) == 1      # decreasing
+    assert call(ls=lists(nq=6)) == 1                                  # row count mismatch
+    assert call(ls=lists(nk=5)) == 1                                  # widest item is 4
+    assert call(ls=lists(block=64, nq=14, nk=7)) == 2                 # block 64 unsupported
+    assert call(ls=lists(L=3)) == 1                                   # num_lists not 1 or H
+    assert call(hd=96) == 2
+    assert call(lse_=None) == 1                                       # lse required
+    assert call(lse_=vp((9 << 30) + 2)) == 1                          # misaligned lse
+    assert call(wsb=ws - 1) == 1                                      # workspace too small
+    assert call(dq=vp((6 << 30) + 8)) == 1                            # misaligned dq
+    assert call(dq=vp((1 << 30) + 4096)) == 1                         # dq inside q's span
+    assert call(dq=bufs[6]) == 1                                      # dq and dk the same
+
+
 def test_generated_rows_host_checks(lib):
     """bsa_attn_fwd_patterns / bsa_attn_fwd_radial reject bad arguments on the
     host, before any CUDA call."""

@@ -3,8 +3,9 @@
 The pages batch nothing of different lengths; the reading is that each item is
 its own problem. These checks tie the oracle to constructions that do not go
 through it: dense softmax attention with a block-diagonal mask over the packed
-sequence (torch SDPA in float64, the mask built here), the batched oracle for
-items of equal length, and the items' own lists split back out.
+sequence (torch SDPA in float64, the mask built here; its gradients by torch
+autograd), the batched oracle for items of equal length, and the items' own
+lists split back out.
 """
 
 import numpy as np
@@ -82,3 +83,55 @@ def test_a_token_never_sees_another_item():
                                                 block)
     assert np.array_equal(o1[:90], o2[:90]) and np.array_equal(o1[170:], o2[170:])
     assert not np.allclose(o1[90:170], o2[90:170])
+
+
+def _token_mask(rp, ci, n, block):
+    """Dense [n, n] mask of one item's single-list block lists (built here)."""
+    m = np.zeros((n, n), dtype=bool)
+    for qb in range(len(rp) - 1):
+        for kb in ci[rp[qb]:rp[qb + 1]]:
+            m[qb * block:(qb + 1) * block, kb * block:(kb + 1) * block] = True
+    return m
+
+
+def test_backward_equals_autograd_of_block_diagonal_masked_attention():
+    # radial items of different lengths, an empty one, and a query block whose
+    # row is empty (no key admitted: zero output, zero gradient)
+    items = [(3, 40, 10), (0, 0, 0), (4, 48, 0), (2, 30, 5)]
+    block, H, D = 32, 2, 8
+    lengths = [f * s + t for f, s, t in items]
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    total = int(cu[-1])
+    lists = []
+    for (f, s, t), n in zip(items, lengths):
+        lists.append(oracle.joint_block_lists(f, s, t, block) if n else
+                     (np.zeros(1, dtype=np.int64), np.zeros(0, dtype=np.int64)))
+    rp0, ci0 = lists[2]
+    ci0 = np.array(ci0)
+    keep = np.ones(ci0.size, dtype=bool)
+    keep[rp0[1]:rp0[2]] = False                      # item 2's query block 1: no keys
+    counts = np.diff(rp0)
+    counts[1] = 0
+    lists[2] = (np.concatenate([[0], np.cumsum(counts)]), ci0[keep])
+    q, k, v = _packed(total, H, D, 5)
+    do = torch.randn((total, H, D), generator=torch.Generator().manual_seed(6),
+                     dtype=torch.float64)
+    dq, dk, dv = oracle.varlen_masked_attention_backward_fp64(q.numpy(), k.numpy(), v.numpy(),
+                                                              do.numpy(), cu, lists, 1, block)
+    mask = np.zeros((total, total), dtype=bool)
+    for b, n in enumerate(lengths):
+        if n:
+            t0 = int(cu[b])
+            mask[t0:t0 + n, t0:t0 + n] = _token_mask(*lists[b], n, block)
+    mask = torch.as_tensor(mask)
+    qa, ka, va = (x.clone().requires_grad_(True) for x in (q, k, v))
+    s = torch.einsum("thd,shd->hts", qa, ka) * D ** -0.5
+    s = s.masked_fill(~mask, float("-inf"))
+    p = torch.softmax(s, dim=-1).nan_to_num(0.0)     # rows with no key: all zero
+    o = torch.einsum("hts,shd->thd", p, va)
+    (o * do).sum().backward()
+    for got, ref, name in ((dq, qa.grad, "dq"), (dk, ka.grad, "dk"), (dv, va.grad, "dv")):
+        assert np.allclose(got, ref.numpy(), atol=1e-12, rtol=1e-10), name
+    t0 = int(cu[2]) + block
+    assert np.all(dq[t0:t0 + block] == 0)            # the row with no keys
+    assert np.any(dq[int(cu[0]):int(cu[1])] != 0)
