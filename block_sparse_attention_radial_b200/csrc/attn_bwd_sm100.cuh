@@ -126,8 +126,10 @@ __device__ __forceinline__ bool row_has(const int32_t *col_idx, int a, int b, in
 }
 
 // One CTA per (list, key block): how many query blocks list it.
+// (first: also write col_cnt[0] = 0; later segments of a concatenation
+// leave the entry before them alone)
 __global__ void csc_count_kernel(const int32_t *row_ptr, const int32_t *col_idx, int nqb, int nkb,
-                                 int nnz, int32_t *col_cnt) {
+                                 int nnz, int32_t *col_cnt, int first) {
   __shared__ int scratch[32];
   const int list = blockIdx.x / nkb, kb = blockIdx.x - list * nkb;
   const int32_t *rp = row_ptr + static_cast<long long>(list) * nqb;
@@ -139,7 +141,7 @@ __global__ void csc_count_kernel(const int32_t *row_ptr, const int32_t *col_idx,
   int total;
   cta_inclusive_scan(c, scratch, total);
   if (threadIdx.x == 0) col_cnt[blockIdx.x + 1] = total;
-  if (blockIdx.x == 0 && threadIdx.x == 0) col_cnt[0] = 0;
+  if (first && blockIdx.x == 0 && threadIdx.x == 0) col_cnt[0] = 0;
 }
 
 // One CTA per (list, key block): its query blocks in ascending order, at
@@ -278,8 +280,51 @@ struct DkdvCfg {
 };
 
 struct BwdItem {
-  int bh, blk, a, len;  // rows [a, a + len) of the (transposed) list
+  int blk, a, len;           // block; rows [a, a + len) of the (transposed) list
+  int ib, ih;                // batch item and head of the views
+  int n, nqb, nkb, tok0;     // the problem's tokens, query and key blocks, first token
+  long long lbase;           // lse2 / delta index of the problem's first query row
 };
+
+// Work item idx (one per (batch*head, block) of `nblk` blocks) of a regular
+// call, or of a variable-length batch (one per (item, head, block); items
+// from the table, each its own problem of nqb_b = nkb_b blocks): everything
+// but the list rows. Returns the list row (query-block row, or transposed
+// key-block column) that the item's entries are at.
+template <bool VARLEN>
+__device__ __forceinline__ long long bwd_decode(int idx, bool by_key, const BwdParams &p,
+                                                const VarlenTable &vt, BwdItem &it) {
+  long long lrow;
+  if (!VARLEN) {
+    const int nblk = by_key ? p.nkb : p.nqb;
+    const int bh = idx / nblk;
+    it.blk = idx - bh * nblk;
+    it.ib = bh / p.heads;
+    it.ih = bh - it.ib * p.heads;
+    it.n = p.n;
+    it.nqb = p.nqb;
+    it.nkb = p.nkb;
+    it.tok0 = 0;
+    it.lbase = static_cast<long long>(bh) * p.nqb * kBwdBlock;
+    lrow = 0;
+  } else {
+    const int b = varlen_item_of_row(vt, idx / p.heads);
+    const int nq = vt.row0[b + 1] - vt.row0[b];
+    const int local = idx - p.heads * vt.row0[b];
+    it.ih = local / nq;
+    it.blk = local - it.ih * nq;
+    it.ib = 0;
+    it.tok0 = vt.tok0[b];
+    it.n = vt.tok0[b + 1] - it.tok0;
+    it.nqb = it.nkb = nq;
+    // lse2 / delta: per item, per head, its padded rows
+    it.lbase = (static_cast<long long>(p.heads) * vt.row0[b] + static_cast<long long>(it.ih) * nq) *
+               kBwdBlock;
+    lrow = static_cast<long long>(p.num_lists) * vt.row0[b];
+  }
+  const int list = p.num_lists > 1 ? it.ih : 0;
+  return lrow + static_cast<long long>(list) * (by_key ? it.nkb : it.nqb) + it.blk;
+}
 
 // Warps 0-3: elementwise (thread = key row = TMEM lane) and the dK/dV
 // epilogue; warp 4: TMA producer (lane 0); warp 5: MMA issuer (lane 0).
@@ -288,12 +333,13 @@ struct BwdItem {
 //                                           P^T and dS^T as bf16 over them)
 //   dV += P^T dO_e, dK += dS^T Q_e         (issued before the next S^T, so the
 //                                           TMEM they read is not overwritten)
-template <int D, bool MASKED>
+template <int D, bool MASKED, bool VARLEN>
 __global__ void __launch_bounds__(192, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v,
-                         const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+                         const __grid_constant__ CUtensorMap tm_do, const BwdParams p,
+                         const __grid_constant__ VarlenTable vt) {
   using C = DkdvCfg<D>;
   constexpr int BN = kBwdBlock;
   extern __shared__ uint8_t dsmem[];
@@ -317,7 +363,6 @@ __global__ void __launch_bounds__(192, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const long long padded = static_cast<long long>(p.nqb) * BN;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) {
@@ -356,10 +401,7 @@ __global__ void __launch_bounds__(192, 1)
   // transposed lists.
   auto decode = [&](int idx) {
     BwdItem it;
-    it.bh = idx / p.nkb;
-    it.blk = idx - it.bh * p.nkb;
-    const int list = p.num_lists > 1 ? (it.bh % p.heads) : 0;
-    const long long c = static_cast<long long>(list) * p.nkb + it.blk;
+    const long long c = bwd_decode<VARLEN>(idx, true, p, vt, it);
     const int a = min(max(p.col_ptr[c], 0), p.nnz), b = min(max(p.col_ptr[c + 1], 0), p.nnz);
     it.a = a;
     it.len = max(b - a, 0);
@@ -389,21 +431,21 @@ __global__ void __launch_bounds__(192, 1)
         if (it.len == 0) continue;
         if (!(ok = lane_wait(&bar_kv_empty, (kvcount & 1u) ^ 1u, wc, kBarQEmpty, kvcount))) break;
         mbar_arrive_expect_tx(&bar_kv_full, 2 * C::T);
-        const int ib = it.bh / p.heads, ih = it.bh - ib * p.heads;
-        tma_load_5d(sK, &tm_k, &bar_kv_full, 0, it.blk * BN, 0, ih, ib);
-        tma_load_5d(sV, &tm_v, &bar_kv_full, 0, it.blk * BN, 0, ih, ib);
+        const int ib = it.ib, ih = it.ih;
+        tma_load_5d(sK, &tm_k, &bar_kv_full, 0, it.tok0 + it.blk * BN, 0, ih, ib);
+        tma_load_5d(sV, &tm_v, &bar_kv_full, 0, it.tok0 + it.blk * BN, 0, ih, ib);
         ++kvcount;
         for (int e = 0; e < it.len && ok; ++e) {
-          const int qb = min(max(__ldg(p.row_idx + it.a + e), 0), p.nqb - 1);
+          const int qb = min(max(__ldg(p.row_idx + it.a + e), 0), it.nqb - 1);
           const uint32_t s = ring % C::NS;
           if (!(ok = lane_wait(&bar_st_empty[s], ((ring / C::NS) & 1u) ^ 1u, wc, kBarKvEmpty,
                                ring)))
             break;
           uint8_t *st = sStage + s * C::STAGE;
           mbar_arrive_expect_tx(&bar_st_full[s], 2 * C::T + 1024);
-          tma_load_5d(st, &tm_q, &bar_st_full[s], 0, qb * BN, 0, ih, ib);
-          tma_load_5d(st + C::T, &tm_do, &bar_st_full[s], 0, qb * BN, 0, ih, ib);
-          const long long off = static_cast<long long>(it.bh) * padded + static_cast<long long>(qb) * BN;
+          tma_load_5d(st, &tm_q, &bar_st_full[s], 0, it.tok0 + qb * BN, 0, ih, ib);
+          tma_load_5d(st + C::T, &tm_do, &bar_st_full[s], 0, it.tok0 + qb * BN, 0, ih, ib);
+          const long long off = it.lbase + static_cast<long long>(qb) * BN;
           bulk_load(st + 2 * C::T, p.lse2 + off, 512, &bar_st_full[s]);
           bulk_load(st + 2 * C::T + 512, p.delta + off, 512, &bar_st_full[s]);
           ++ring;
@@ -546,10 +588,10 @@ __global__ void __launch_bounds__(192, 1)
       if (idx < 0) break;
       const BwdItem it = decode(idx);
       const int key = it.blk * BN + r;
-      const bool store = key < p.n;
-      const long long ib = it.bh / p.heads, ih = it.bh - ib * p.heads;
-      __nv_bfloat16 *const dk_row = p.dk + ib * p.dk_s[0] + ih * p.dk_s[1] + key * p.dk_s[2];
-      __nv_bfloat16 *const dv_row = p.dv + ib * p.dv_s[0] + ih * p.dv_s[1] + key * p.dv_s[2];
+      const bool store = key < it.n;
+      const long long ib = it.ib, ih = it.ih, tk = it.tok0 + key;
+      __nv_bfloat16 *const dk_row = p.dk + ib * p.dk_s[0] + ih * p.dk_s[1] + tk * p.dk_s[2];
+      __nv_bfloat16 *const dv_row = p.dv + ib * p.dv_s[0] + ih * p.dv_s[1] + tk * p.dv_s[2];
       if (it.len == 0) {  // no query attends these keys
         if (store) {
           uint4 *a = reinterpret_cast<uint4 *>(dk_row);
@@ -699,12 +741,13 @@ struct DqCfg {
 // block ahead so it runs during the previous elementwise step), dP = dO V_e^T,
 // the elementwise warps write dS (bf16) over dP, then dQ += dS K_e (issued
 // before the next dP, which overwrites the dS it reads).
-template <int D, bool MASKED>
+template <int D, bool MASKED, bool VARLEN>
 __global__ void __launch_bounds__(192, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v,
-                       const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+                       const __grid_constant__ CUtensorMap tm_do, const BwdParams p,
+                       const __grid_constant__ VarlenTable vt) {
   using C = DqCfg<D>;
   constexpr int BN = kBwdBlock;
   extern __shared__ uint8_t dsmem[];
@@ -731,7 +774,6 @@ __global__ void __launch_bounds__(192, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const long long padded = static_cast<long long>(p.nqb) * BN;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) {
@@ -766,10 +808,7 @@ __global__ void __launch_bounds__(192, 1)
 
   auto decode = [&](int idx) {
     BwdItem it;
-    it.bh = idx / p.nqb;
-    it.blk = idx - it.bh * p.nqb;
-    const int list = p.num_lists > 1 ? (it.bh % p.heads) : 0;
-    const long long r = static_cast<long long>(list) * p.nqb + it.blk;
+    const long long r = bwd_decode<VARLEN>(idx, false, p, vt, it);
     const int a = min(max(p.row_ptr[r], 0), p.nnz), b = min(max(p.row_ptr[r + 1], 0), p.nnz);
     it.a = a;
     it.len = max(b - a, 0);
@@ -799,20 +838,20 @@ __global__ void __launch_bounds__(192, 1)
         if (it.len == 0) continue;
         if (!(ok = lane_wait(&bar_qd_empty, (qdcount & 1u) ^ 1u, wc, kBarQEmpty, qdcount))) break;
         mbar_arrive_expect_tx(&bar_qd_full, 2 * C::T);
-        const int ib = it.bh / p.heads, ih = it.bh - ib * p.heads;
-        tma_load_5d(sQ, &tm_q, &bar_qd_full, 0, it.blk * BN, 0, ih, ib);
-        tma_load_5d(sDO, &tm_do, &bar_qd_full, 0, it.blk * BN, 0, ih, ib);
+        const int ib = it.ib, ih = it.ih;
+        tma_load_5d(sQ, &tm_q, &bar_qd_full, 0, it.tok0 + it.blk * BN, 0, ih, ib);
+        tma_load_5d(sDO, &tm_do, &bar_qd_full, 0, it.tok0 + it.blk * BN, 0, ih, ib);
         ++qdcount;
         for (int e = 0; e < it.len && ok; ++e) {
-          const int kb = min(max(__ldg(p.col_idx + it.a + e), 0), p.nkb - 1);
+          const int kb = min(max(__ldg(p.col_idx + it.a + e), 0), it.nkb - 1);
           const uint32_t s = ring % C::NS;
           if (!(ok = lane_wait(&bar_st_empty[s], ((ring / C::NS) & 1u) ^ 1u, wc, kBarKvEmpty,
                                ring)))
             break;
           uint8_t *st = sStage + s * C::STAGE;
           mbar_arrive_expect_tx(&bar_st_full[s], 2 * C::T);
-          tma_load_5d(st, &tm_k, &bar_st_full[s], 0, kb * BN, 0, ih, ib);
-          tma_load_5d(st + C::T, &tm_v, &bar_st_full[s], 0, kb * BN, 0, ih, ib);
+          tma_load_5d(st, &tm_k, &bar_st_full[s], 0, it.tok0 + kb * BN, 0, ih, ib);
+          tma_load_5d(st + C::T, &tm_v, &bar_st_full[s], 0, it.tok0 + kb * BN, 0, ih, ib);
           ++ring;
         }
       }
@@ -941,9 +980,9 @@ __global__ void __launch_bounds__(192, 1)
       if (idx < 0) break;
       const BwdItem it = decode(idx);
       const int row = it.blk * BN + r;
-      const bool store = row < p.n;
-      const long long ib = it.bh / p.heads, ih = it.bh - ib * p.heads;
-      __nv_bfloat16 *const dq_row = p.dq + ib * p.dq_s[0] + ih * p.dq_s[1] + row * p.dq_s[2];
+      const bool store = row < it.n;
+      const long long ib = it.ib, ih = it.ih, tq = it.tok0 + row;
+      __nv_bfloat16 *const dq_row = p.dq + ib * p.dq_s[0] + ih * p.dq_s[1] + tq * p.dq_s[2];
       if (it.len == 0) {  // no key: dQ = 0
         if (store) {
           uint4 *a = reinterpret_cast<uint4 *>(dq_row);
@@ -952,12 +991,13 @@ __global__ void __launch_bounds__(192, 1)
         }
         continue;
       }
-      const long long prow = static_cast<long long>(it.bh) * padded + static_cast<long long>(it.blk) * BN + r;
+      const long long prow = it.lbase + static_cast<long long>(it.blk) * BN + r;
       const float lse2 = p.lse2[prow], del = p.delta[prow];
       // lists are sorted: only the row's last block can be the ragged final
-      // key block (its columns >= n hold zero keys; they are masked out)
-      const int last_kb = min(max(__ldg(p.col_idx + it.a + it.len - 1), 0), p.nkb - 1);
-      const int last_valid = min(p.n - last_kb * BN, BN);
+      // key block (its columns >= n hold zero keys, or the next item's keys
+      // in a variable-length batch; they are masked out)
+      const int last_kb = min(max(__ldg(p.col_idx + it.a + it.len - 1), 0), it.nkb - 1);
+      const int last_valid = min(it.n - last_kb * BN, BN);
       for (int e = 0; e < it.len; ++e) {
         const int sb = e & 1;
         if (!(ok = warp_wait(&bar_s_full[sb], scount[sb] & 1u, wc, kBarSFull, scount[sb]))) break;

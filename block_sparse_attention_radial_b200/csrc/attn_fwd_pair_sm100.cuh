@@ -184,22 +184,6 @@ struct UnionWalker {
 
 constexpr int kItemN = 4;  // work items in flight between the producer and the consumers
 
-// Variable-length batches: the batch is one packed token sequence (batch
-// extent 1 in the views) holding num_items items one after the other; item b
-// owns tokens [tok0[b], tok0[b+1]), query-block rows [row0[b], row0[b+1]) of
-// every list (its key blocks counted from 0 inside the item), work-order
-// entries [pair0[b], pair0[b+1]) of every list and work items
-// [work0[b], work0[b+1]) (heads x its query-block pairs). Passed by value as
-// a kernel parameter.
-constexpr int kMaxVarlenItems = 64;
-struct VarlenTable {
-  int32_t num_items;
-  int32_t tok0[kMaxVarlenItems + 1];
-  int32_t row0[kMaxVarlenItems + 1];
-  int32_t pair0[kMaxVarlenItems + 1];
-  int32_t work0[kMaxVarlenItems + 1];
-};
-
 struct PairItem {
   int bh, qa, a0, lenA, b0, lenB;  // tile B absent (lenB = 0) past the last block
   int n, nqb, nkb, tok0;           // the item's tokens, query and key blocks, first token
@@ -739,8 +723,11 @@ __global__ void __launch_bounds__(384, 1)
         };
         uint32_t pk[BN / 2];
         auto exp_row = [&]() {
-          return valid < BN ? exp2_pack_row<BN, 0>(s, sl2, -m_ref, pk)
-                            : exp2_pack_row<BN, kEmuPairsPer8>(s, sl2, -m_ref, pk);
+          // a row without a reference maximum has every column at -inf here
+          // (its block maximum is -inf): any finite bias gives P = 0, sum 0
+          const float bias = MODE == kModeQuarters && m_ref == -INFINITY ? 0.f : -m_ref;
+          return valid < BN ? exp2_pack_row<BN, 0>(s, sl2, bias, pk)
+                            : exp2_pack_row<BN, kEmuPairsPer8>(s, sl2, bias, pk);
         };
         float alpha = 1.f;
         bool rescale = false;
@@ -756,14 +743,10 @@ __global__ void __launch_bounds__(384, 1)
         } else if (j == 0) {
           m_ref = row_max() * sl2;
         }
-        if (MODE == kModeQuarters && m_ref == -INFINITY) {  // nothing listed yet: P = 0
-          sum = 0.f;
-#pragma unroll
-          for (int i = 0; i < BN / 2; ++i) pk[i] = 0u;
-        } else {
-          sum = exp_row();
-        }
-        if (j > 0 || MODE == kModeQuarters) {
+        sum = exp_row();
+        // (at j = 0, and at a row's first block with a reference, the
+        // reference is the block's own maximum: every P <= 1, no rescale)
+        if (j > 0) {
           // The reference stays the first block's maximum: P may exceed 1 by
           // far (bf16 keeps its relative precision and the fp32 sums stay
           // finite), so the row maximum is only taken again when the row sum

@@ -39,6 +39,38 @@
 
 namespace bsa {
 
+// Variable-length batches: the batch is one packed token sequence (batch
+// extent 1 in the views) holding num_items items one after the other; item b
+// owns tokens [tok0[b], tok0[b+1]), query-block rows [row0[b], row0[b+1]) of
+// every list (its key blocks counted from 0 inside the item), work-order
+// entries [pair0[b], pair0[b+1]) of every list and work items
+// [work0[b], work0[b+1]) (heads x its query-block pairs; the backward
+// derives its own work items from row0). Passed by value as a kernel
+// parameter.
+constexpr int kMaxVarlenItems = 64;
+struct VarlenTable {
+  int32_t num_items;
+  int32_t tok0[kMaxVarlenItems + 1];
+  int32_t row0[kMaxVarlenItems + 1];
+  int32_t pair0[kMaxVarlenItems + 1];
+  int32_t work0[kMaxVarlenItems + 1];
+};
+
+// The item holding query-block row r of a variable-length batch: the last b
+// with row0[b] <= r (an item without rows shares its row0 with the next item
+// and is skipped).
+__device__ __forceinline__ int varlen_item_of_row(const VarlenTable &vt, int r) {
+  int lo = 0, hi = vt.num_items - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (vt.row0[mid] <= r)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
 struct FwdParams {
   const int32_t *row_ptr, *col_idx, *order;
   int32_t *item_counter;  // next work item (two-tile kernel); zeroed by the work-order kernel

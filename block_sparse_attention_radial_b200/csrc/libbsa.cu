@@ -53,8 +53,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   bool probed = false;
   int cc_major = 0, cc_minor = 0, sms = 0;
-  bool attrs_set[12] = {false, false, false, false, false, false,
-                       false, false, false, false, false, false};
+  bool attrs_set[14] = {};
   bool ref_attrs_set[4] = {false, false, false, false};
   bool gemm_attrs_set[4] = {false, false, false, false};
   bool pair_attrs_set[10] = {};
@@ -663,6 +662,94 @@ struct BwdViews {
   long long lse_sb = -1, lse_sh = -1;  // lse's batch / head strides; -1: contiguous [B, H, n]
 };
 
+// The dK/dV and dQ kernels of one backward call, once the prep and the
+// transposed lists are in place: TMA maps over the views ([batch, heads,
+// n_map] tokens), the instance for the masks and for a variable-length
+// batch (vt non-null: its items are the problems), dkdv_items and dq_items
+// work items.
+template <int D>
+int launch_bwd_kernels(const BwdViews &x, int32_t n_map, BwdParams &p, bool masked,
+                       const VarlenTable *vt, long long dkdv_items, long long dq_items,
+                       DeviceInfo *dev, cudaStream_t stream) {
+  CUtensorMap tq, tk, tv, td;
+  int st;
+  if ((st = make_map_strided(&tq, x.q, x.lq, x.batch, x.heads, n_map, D, kBwdBlock)) != BSA_OK)
+    return st;
+  if ((st = make_map_strided(&tk, x.k, x.lk, x.batch, x.heads, n_map, D, kBwdBlock)) != BSA_OK)
+    return st;
+  if ((st = make_map_strided(&tv, x.v, x.lv, x.batch, x.heads, n_map, D, kBwdBlock)) != BSA_OK)
+    return st;
+  if ((st = make_map_strided(&td, x.dout, x.ldo, x.batch, x.heads, n_map, D, kBwdBlock)) != BSA_OK)
+    return st;
+  const bool varlen = vt != nullptr;
+  using DkdvFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, BwdParams,
+                          VarlenTable);
+  DkdvFn dkdv = varlen   ? attn_bwd_dkdv_kernel<D, false, true>
+                : masked ? attn_bwd_dkdv_kernel<D, true, false>
+                         : attn_bwd_dkdv_kernel<D, false, false>;
+  DkdvFn dq = varlen   ? attn_bwd_dq_kernel<D, false, true>
+              : masked ? attn_bwd_dq_kernel<D, true, false>
+                       : attn_bwd_dq_kernel<D, false, false>;
+  const int slot = 8 + (D == 128 ? 3 : 0) + (varlen ? 2 : masked ? 1 : 0);
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!dev->attrs_set[slot]) {
+      BSA_CUDA(cudaFuncSetAttribute(dkdv, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    DkdvCfg<D>::DSMEM));
+      BSA_CUDA(cudaFuncSetAttribute(dq, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    DqCfg<D>::DSMEM));
+      dev->attrs_set[slot] = true;
+    }
+  }
+  static const VarlenTable kNoItems{};
+  const VarlenTable &table = varlen ? *vt : kNoItems;
+  int32_t *counters = p.item_counter;
+  p.total_items = static_cast<int32_t>(dkdv_items);
+  int grid = p.total_items < dev->sms ? p.total_items : dev->sms;
+  if (grid > 0) {
+    dkdv<<<grid, DkdvCfg<D>::THREADS, DkdvCfg<D>::DSMEM, stream>>>(tq, tk, tv, td, p, table);
+    BSA_CUDA(cudaGetLastError());
+  }
+  p.total_items = static_cast<int32_t>(dq_items);
+  p.item_counter = counters + 1;
+  grid = p.total_items < dev->sms ? p.total_items : dev->sms;
+  if (grid > 0) {
+    dq<<<grid, DqCfg<D>::THREADS, DqCfg<D>::DSMEM, stream>>>(tq, tk, tv, td, p, table);
+    BSA_CUDA(cudaGetLastError());
+  }
+  p.item_counter = counters;
+  return BSA_OK;
+}
+
+// Parameters shared by every backward launch of a call.
+template <int D>
+BwdParams bwd_params(const BwdViews &x, const bsa_block_lists *l, float softmax_scale) {
+  BwdParams p;
+  p.row_ptr = l->row_ptr;
+  p.col_idx = l->col_idx;
+  p.dq = static_cast<__nv_bfloat16 *>(x.dq);
+  p.dk = static_cast<__nv_bfloat16 *>(x.dk);
+  p.dv = static_cast<__nv_bfloat16 *>(x.dv);
+  const bsa_layout *outl[3] = {&x.ldq, &x.ldk, &x.ldv};
+  long long *outs[3] = {p.dq_s, p.dk_s, p.dv_s};
+  for (int i = 0; i < 3; ++i) {
+    outs[i][0] = outl[i]->batch_stride;
+    outs[i][1] = outl[i]->head_stride;
+    outs[i][2] = outl[i]->token_stride;
+  }
+  p.heads = x.heads;
+  p.num_lists = l->num_lists;
+  p.nnz = l->nnz;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(D));
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  {
+    std::lock_guard<std::mutex> lk(g_hook_mu);
+    p.wait_limit_ns = g_wait_limit_ns;
+  }
+  return p;
+}
+
 template <int D>
 int launch_bwd(const BwdViews &x, const float *lse, int32_t n, float softmax_scale,
                const bsa_block_lists *l_in, uint8_t *ws, DeviceInfo *dev, cudaStream_t stream) {
@@ -714,7 +801,8 @@ int launch_bwd(const BwdViews &x, const float *lse, int32_t n, float softmax_sca
       reinterpret_cast<int32_t *>(ws + w.counters));
   BSA_CUDA(cudaGetLastError());
   const int cols = l->num_lists * nkb;
-  csc_count_kernel<<<cols, 256, 0, stream>>>(l->row_ptr, l->col_idx, nqb, nkb, l->nnz, col_ptr);
+  csc_count_kernel<<<cols, 256, 0, stream>>>(l->row_ptr, l->col_idx, nqb, nkb, l->nnz, col_ptr,
+                                             1);
   BSA_CUDA(cudaGetLastError());
   scan_rows_kernel<<<1, 1024, 0, stream>>>(col_ptr, cols);
   BSA_CUDA(cudaGetLastError());
@@ -722,93 +810,83 @@ int launch_bwd(const BwdViews &x, const float *lse, int32_t n, float softmax_sca
                                             row_idx, l->nnz > 0 ? l->nnz : 1, rmask, cmask);
   BSA_CUDA(cudaGetLastError());
 
-  CUtensorMap tq, tk, tv, td;
-  int st;
-  if ((st = make_map_strided(&tq, x.q, x.lq, x.batch, x.heads, n, D, kBwdBlock)) != BSA_OK)
-    return st;
-  if ((st = make_map_strided(&tk, x.k, x.lk, x.batch, x.heads, n, D, kBwdBlock)) != BSA_OK)
-    return st;
-  if ((st = make_map_strided(&tv, x.v, x.lv, x.batch, x.heads, n, D, kBwdBlock)) != BSA_OK)
-    return st;
-  if ((st = make_map_strided(&td, x.dout, x.ldo, x.batch, x.heads, n, D, kBwdBlock)) != BSA_OK)
-    return st;
-  const bool masked = rmask != nullptr;
-  const int slot = 8 + (D == 128 ? 2 : 0) + (masked ? 1 : 0);
-  {
-    std::lock_guard<std::mutex> lk(g_dev_mu);
-    if (!dev->attrs_set[slot]) {
-      if (masked) {
-        BSA_CUDA(cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D, true>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      DkdvCfg<D>::DSMEM));
-        BSA_CUDA(cudaFuncSetAttribute(attn_bwd_dq_kernel<D, true>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      DqCfg<D>::DSMEM));
-      } else {
-        BSA_CUDA(cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D, false>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      DkdvCfg<D>::DSMEM));
-        BSA_CUDA(cudaFuncSetAttribute(attn_bwd_dq_kernel<D, false>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      DqCfg<D>::DSMEM));
-      }
-      dev->attrs_set[slot] = true;
-    }
-  }
-  BwdParams p;
-  p.row_ptr = l->row_ptr;
-  p.col_idx = l->col_idx;
+  BwdParams p = bwd_params<D>(x, l, softmax_scale);
   p.col_ptr = col_ptr;
   p.row_idx = row_idx;
   p.rmask = rmask;
   p.cmask = cmask;
   p.lse2 = lse2;
   p.delta = delta;
-  p.dq = static_cast<__nv_bfloat16 *>(x.dq);
-  p.dk = static_cast<__nv_bfloat16 *>(x.dk);
-  p.dv = static_cast<__nv_bfloat16 *>(x.dv);
-  const bsa_layout *outl[3] = {&x.ldq, &x.ldk, &x.ldv};
-  long long *outs[3] = {p.dq_s, p.dk_s, p.dv_s};
-  for (int i = 0; i < 3; ++i) {
-    outs[i][0] = outl[i]->batch_stride;
-    outs[i][1] = outl[i]->head_stride;
-    outs[i][2] = outl[i]->token_stride;
-  }
-  p.heads = x.heads;
   p.n = n;
   p.nqb = nqb;
   p.nkb = nkb;
-  p.num_lists = l->num_lists;
-  p.nnz = l->nnz;
-  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(D));
-  p.scale = scale;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  {
-    std::lock_guard<std::mutex> lk(g_hook_mu);
-    p.wait_limit_ns = g_wait_limit_ns;
-  }
+  p.row_ptr = l->row_ptr;
+  p.col_idx = l->col_idx;
+  p.item_counter = reinterpret_cast<int32_t *>(ws + w.counters);
+  return launch_bwd_kernels<D>(x, n, p, rmask != nullptr, nullptr,
+                               static_cast<long long>(bh) * nkb, static_cast<long long>(bh) * nqb,
+                               dev, stream);
+}
+
+// Backward of a variable-length batch (block-128 lists concatenated item by
+// item, packed [1, heads, total] views, lse [heads, total]): per item the
+// prep (lse2 / delta laid out item by item, head by head) and the item's
+// columns of the transposed lists (one scan over all of them); then one
+// dK/dV and one dQ launch over every item's work.
+template <int D>
+int launch_bwd_varlen(const BwdViews &x, const float *lse, int32_t total, float softmax_scale,
+                      const bsa_block_lists *l, const VarlenTable &vt, uint8_t *ws,
+                      DeviceInfo *dev, cudaStream_t stream) {
+  const int R = vt.row0[vt.num_items];
+  const BwdLayout w = bwd_layout(1, x.heads, R * kBwdBlock, l);
+  float *lse2 = reinterpret_cast<float *>(ws + w.lse2);
+  float *delta = reinterpret_cast<float *>(ws + w.delta);
+  int32_t *col_ptr = reinterpret_cast<int32_t *>(ws + w.col_ptr);
+  int32_t *row_idx = reinterpret_cast<int32_t *>(ws + w.row_idx);
   int32_t *counters = reinterpret_cast<int32_t *>(ws + w.counters);
-  p.total_items = bh * nkb;
+  const int L = l->num_lists;
+  bool first = true;
+  for (int b = 0; b < vt.num_items; ++b) {
+    const int nq = vt.row0[b + 1] - vt.row0[b];
+    if (nq == 0) continue;
+    const int32_t t0 = vt.tok0[b], n_b = vt.tok0[b + 1] - t0;
+    const long long base = static_cast<long long>(x.heads) * vt.row0[b] * kBwdBlock;
+    const long long rows = static_cast<long long>(x.heads) * nq * kBwdBlock;
+    bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 255) / 256), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(x.out) + static_cast<long long>(t0) * x.lo.token_stride,
+        static_cast<const __nv_bfloat16 *>(x.dout) + static_cast<long long>(t0) * x.ldo.token_stride,
+        lse + t0, lse2 + base, delta + base, n_b, nq, x.heads, 0, x.lo.head_stride,
+        x.lo.token_stride, 0, x.ldo.head_stride, x.ldo.token_stride, 0, total, rows, counters);
+    BSA_CUDA(cudaGetLastError());
+    const long long lr = static_cast<long long>(L) * vt.row0[b];
+    csc_count_kernel<<<L * nq, 256, 0, stream>>>(l->row_ptr + lr, l->col_idx, nq, nq, l->nnz,
+                                                 col_ptr + lr, first ? 1 : 0);
+    BSA_CUDA(cudaGetLastError());
+    first = false;
+  }
+  const int cols = L * R;
+  scan_rows_kernel<<<1, 1024, 0, stream>>>(col_ptr, cols);
+  BSA_CUDA(cudaGetLastError());
+  for (int b = 0; b < vt.num_items; ++b) {
+    const int nq = vt.row0[b + 1] - vt.row0[b];
+    if (nq == 0) continue;
+    const long long lr = static_cast<long long>(L) * vt.row0[b];
+    csc_fill_kernel<<<L * nq, 256, 0, stream>>>(l->row_ptr + lr, l->col_idx, nq, nq, l->nnz,
+                                                col_ptr + lr, row_idx, l->nnz > 0 ? l->nnz : 1,
+                                                nullptr, nullptr);
+    BSA_CUDA(cudaGetLastError());
+  }
+  BwdParams p = bwd_params<D>(x, l, softmax_scale);
+  p.col_ptr = col_ptr;
+  p.row_idx = row_idx;
+  p.rmask = p.cmask = nullptr;
+  p.lse2 = lse2;
+  p.delta = delta;
+  p.n = total;
+  p.nqb = p.nkb = 0;  // per item, from the table
   p.item_counter = counters;
-  int grid = p.total_items < dev->sms ? p.total_items : dev->sms;
-  if (masked)
-    attn_bwd_dkdv_kernel<D, true><<<grid, DkdvCfg<D>::THREADS, DkdvCfg<D>::DSMEM, stream>>>(
-        tq, tk, tv, td, p);
-  else
-    attn_bwd_dkdv_kernel<D, false><<<grid, DkdvCfg<D>::THREADS, DkdvCfg<D>::DSMEM, stream>>>(
-        tq, tk, tv, td, p);
-  BSA_CUDA(cudaGetLastError());
-  p.total_items = bh * nqb;
-  p.item_counter = counters + 1;
-  grid = p.total_items < dev->sms ? p.total_items : dev->sms;
-  if (masked)
-    attn_bwd_dq_kernel<D, true><<<grid, DqCfg<D>::THREADS, DqCfg<D>::DSMEM, stream>>>(tq, tk, tv,
-                                                                                      td, p);
-  else
-    attn_bwd_dq_kernel<D, false><<<grid, DqCfg<D>::THREADS, DqCfg<D>::DSMEM, stream>>>(tq, tk,
-                                                                                       tv, td, p);
-  BSA_CUDA(cudaGetLastError());
-  return BSA_OK;
+  const long long items = static_cast<long long>(x.heads) * R;
+  return launch_bwd_kernels<D>(x, total, p, false, &vt, items, items, dev, stream);
 }
 
 // Self-test of the two exp2 paths of the attention softmax against exp2f.
@@ -1470,26 +1548,10 @@ BwdViews bwd_views(const void *const ptrs[8], const bsa_layout *const lays[8], i
   return x;
 }
 
-// Item b's share of concatenated variable-length lists: its L * nqb_b rows
-// (offsets into the shared col_idx), nqb_b query and key blocks.
-bsa_block_lists varlen_item_lists(const bsa_block_lists *l, const VarlenTable &vt, int b) {
-  bsa_block_lists sub = *l;
-  const int nqb = vt.row0[b + 1] - vt.row0[b];
-  sub.row_ptr = l->row_ptr + static_cast<long long>(l->num_lists) * vt.row0[b];
-  sub.num_q_blocks = sub.num_k_blocks = nqb;
-  return sub;
-}
-
+// lse2 / delta for every item's padded rows (item by item, head by head),
+// the transposed lists of all items, the work counters.
 size_t varlen_bwd_bytes(const VarlenTable &vt, int heads, const bsa_block_lists *l) {
-  size_t mx = 256;
-  for (int b = 0; b < vt.num_items; ++b) {
-    const int n_b = vt.tok0[b + 1] - vt.tok0[b];
-    if (n_b == 0) continue;
-    const bsa_block_lists sub = varlen_item_lists(l, vt, b);
-    const size_t t = bwd_layout(1, heads, n_b, &sub).total;
-    mx = t > mx ? t : mx;
-  }
-  return mx;
+  return bwd_layout(1, heads, vt.row0[vt.num_items] * kBwdBlock, l).total;
 }
 
 }  // namespace
@@ -1542,6 +1604,7 @@ size_t bsa_attn_bwd_varlen_workspace_bytes(int32_t num_items, const int32_t *cu_
   VarlenTable vt;
   int32_t mx = 0;
   if (varlen_table(num_items, cu_seqlens, heads, 128, &vt, &mx) != BSA_OK) return 0;
+  if (static_cast<long long>(heads) * vt.row0[num_items] * kBwdBlock > 0x7fffffffLL) return 0;
   return varlen_bwd_bytes(vt, heads, l);
 }
 
@@ -1576,7 +1639,7 @@ int bsa_attn_bwd_varlen(const void *q, const bsa_layout *q_layout, const void *k
     return BSA_ERR_INVALID_ARG;
   if (static_cast<long long>(heads) * total > 0x7fffffffLL ||
       static_cast<long long>(l->num_lists) * l->num_q_blocks > 0x7fffffffLL ||
-      static_cast<long long>(heads) * max_nqb * kBwdBlock > 0x7fffffffLL)
+      static_cast<long long>(heads) * l->num_q_blocks * kBwdBlock > 0x7fffffffLL)
     return BSA_ERR_UNSUPPORTED;
   // the packed sequence is a batch of one: [1, heads, total, head_dim] views
   const size_t lbytes = static_cast<size_t>(heads) * total * sizeof(float);
@@ -1587,25 +1650,11 @@ int bsa_attn_bwd_varlen(const void *q, const bsa_layout *q_layout, const void *k
   DeviceInfo *dev = nullptr;
   if ((st = current_device(&dev)) != BSA_OK) return st;
   if (dev->cc_major != 10) return BSA_ERR_UNSUPPORTED;
-  // one backward per item on its slice of the packed views; the items run
-  // one after another on `stream` and reuse the workspace
+  const BwdViews x = bwd_views(ptrs, lays, 1, heads);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
-  for (int b = 0; b < num_items; ++b) {
-    const int32_t t0 = vt.tok0[b], n_b = vt.tok0[b + 1] - t0;
-    if (n_b == 0) continue;
-    const void *item[8];
-    for (int i = 0; i < 8; ++i)
-      item[i] = static_cast<const uint8_t *>(ptrs[i]) +
-                static_cast<long long>(t0) * lays[i]->token_stride * 2;
-    BwdViews x = bwd_views(item, lays, 1, heads);
-    x.lse_sb = static_cast<long long>(heads) * total;
-    x.lse_sh = total;
-    const bsa_block_lists sub = varlen_item_lists(l, vt, b);
-    st = head_dim == 128 ? launch_bwd<128>(x, lse + t0, n_b, softmax_scale, &sub, ws, dev, stream)
-                         : launch_bwd<64>(x, lse + t0, n_b, softmax_scale, &sub, ws, dev, stream);
-    if (st != BSA_OK) return st;
-  }
-  return BSA_OK;
+  if (head_dim == 128)
+    return launch_bwd_varlen<128>(x, lse, total, softmax_scale, l, vt, ws, dev, stream);
+  return launch_bwd_varlen<64>(x, lse, total, softmax_scale, l, vt, ws, dev, stream);
 }
 
 size_t bsa_attn_bwd_workspace_bytes(int32_t batch, int32_t heads, int32_t n,

@@ -599,9 +599,10 @@ int bsa_attn_bwd_strided(const void *q, const bsa_layout *q_layout,
                          void *workspace, size_t workspace_bytes, bsa_stream_t stream);
 
 /*
- * Bytes of device scratch bsa_attn_bwd_varlen needs: the largest item's
- * bsa_attn_bwd scratch (the items reuse it one after another). 0 for invalid
- * arguments.
+ * Bytes of device scratch bsa_attn_bwd_varlen needs: lse * log2(e) and delta
+ * for every item's query rows padded to whole 128-row blocks, per head (2 x 4
+ * bytes each), the transposed lists of all items (num_lists * sum_b nqb_b + 1
+ * offsets, nnz entries) and two work counters. 0 for invalid arguments.
  */
 size_t bsa_attn_bwd_varlen_workspace_bytes(int32_t num_items, const int32_t *cu_seqlens,
                                            int32_t heads, const bsa_block_lists *lists);
@@ -620,10 +621,14 @@ size_t bsa_attn_bwd_varlen_workspace_bytes(int32_t num_items, const int32_t *cu_
  * num_items, cu_seqlens, lists  as for bsa_attn_fwd_varlen (block 128).
  * workspace  bsa_attn_bwd_varlen_workspace_bytes() bytes of device scratch,
  *        16-byte aligned, overlapping no view and not lse.
- * The items run one after another on `stream` (six launches each: prep,
- * the three passes of the transposed lists, dK/dV, dQ); tokens of empty
- * items are not touched. Each item's gradients are bit-identical to
- * bsa_attn_bwd on that item alone. Deterministic. Returns
+ * Per item a prep launch (delta, lse * log2(e)) and the item's columns of
+ * the transposed lists (count, fill; one scan over all items between them),
+ * then ONE dK/dV and ONE dQ launch serve every item (their work items are
+ * (item, head, block), decoded from a per-item table). Tokens of empty items
+ * are not touched. Each item's gradients are bit-identical to bsa_attn_bwd
+ * on that item alone. Every element of the views must be finite (an item's
+ * last blocks read the next item's tokens, which enter with weight 0).
+ * Deterministic. Returns
  * BSA_ERR_UNSUPPORTED for block 64 or head_dim other than 64 / 128; other
  * errors as bsa_attn_bwd_strided. Asynchronous.
  */

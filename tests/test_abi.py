@@ -465,9 +465,10 @@ def test_varlen_backward_host_checks(lib):
                                        wsb, None)
 
     ws = lib.bsa_attn_bwd_varlen_workspace_bytes(3, cu_ok, H, ref(lists()))
-    # the largest item (400 tokens, 4 tiles): lse2 + delta for 2 x 512 rows,
-    # counters, 4 + 1 column pointers, 10 entries, 256-byte aligned
-    assert ws == 4096 + 4096 + 256 + 256 + 256
+    # every item's padded rows (7 blocks of 128, 2 heads): lse2 + delta for
+    # 1792 rows each, counters, 7 + 1 column pointers, 10 entries, each part
+    # 256-byte aligned
+    assert ws == 7168 + 7168 + 256 + 256 + 256
     assert lib.bsa_attn_bwd_varlen_workspace_bytes(3, cu_ok, H, ref(lists(block=64))) == 0
     assert call(items=0) == 1 and call(items=65) == 1
     assert call(cu=(ctypes.c_int32 * 4)(1, 300, 300, 700)) == 1      # cu[0] != 0
