@@ -574,7 +574,8 @@ def run_ours_bwd(args, world, rank, local):
     backward call from resident Q, K, V, O, dO and lse (the forward runs once
     before timing). value counts the algorithmic backward FLOPs, 2.5 x the
     forward's; the kernels execute 3.5 x (dQ recomputes S and dP), which the
-    roofline uses."""
+    roofline uses. --bwd-kernel one_pass times bsa_attn_bwd_one_pass instead
+    (one kernel, 2.5 x executed, dQ parts added in row order)."""
     import numpy as np
     import torch
 
@@ -595,18 +596,23 @@ def run_ours_bwd(args, world, rank, local):
                                   text_tokens=w.text_tokens)
     rp_h, ci_h = lists.row_ptr.cpu().numpy(), lists.col_idx.cpu().numpy()
     fwd_flops = bsa.computed_flops(rp_h, ci_h, w.n, w.block, w.head_dim, w.batch, w.heads, 1)
-    flops, exec_flops = 2.5 * fwd_flops, 3.5 * fwd_flops
+    one_pass = args.bwd_kernel == "one_pass"
+    flops, exec_flops = 2.5 * fwd_flops, (2.5 if one_pass else 3.5) * fwd_flops
     out, lse = bsa.attention(q, k, v, lists)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = torch.empty(bsa.bsa_attn_bwd_workspace_bytes(w.batch, w.heads, w.n, lists),
-                     dtype=torch.uint8, device=dev)
+    ws_bytes = (bsa.bsa_attn_bwd_one_pass_workspace_bytes if one_pass else
+                bsa.bsa_attn_bwd_workspace_bytes)(w.batch, w.heads, w.n, lists)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = 6  # prep, transposed-list count, scan, fill; dK/dV; dQ
+    # prep, transposed-list count, scan, fill; dK/dV and dQ (or the one-pass
+    # kernel and its initialisation)
+    launches_per_step = 6
+    bwd_call = bsa.bsa_attn_bwd_one_pass if one_pass else bsa.bsa_attn_bwd
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        bsa.bsa_attn_bwd(q, k, v, out, do, lse, lists, dq, dk, dv, ws, 0.0, stream)
+        bwd_call(q, k, v, out, do, lse, lists, dq, dk, dv, ws, 0.0, stream)
         if ev is not None:
             ev[1].record(stream)
 
@@ -707,12 +713,15 @@ def run_ours_bwd(args, world, rank, local):
             "ms_per_step": ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(w, nnz=int(rp_h[-1])),
+            "config": dict(workload_config(w, nnz=int(rp_h[-1])), bwd_kernel=args.bwd_kernel),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": load_traffic(w.name, "bwd"),
+                         "frac": achieved / peak,
+                         "traffic": None if one_pass else load_traffic(w.name, "bwd"),
                          "peak_kind": f"{peak_kind} bf16 burst",
-                         "kernel": "attn_bwd_dkdv_kernel<128> + attn_bwd_dq_kernel<128> "
-                                   "(+ prep and transposed lists)",
+                         "kernel": ("attn_bwd_fused_kernel<128> (+ prep, transposed lists, "
+                                    "counter initialisation)" if one_pass else
+                                    "attn_bwd_dkdv_kernel<128> + attn_bwd_dq_kernel<128> "
+                                    "(+ prep and transposed lists)"),
                          "kernel_ms": kernel_ms, "flops_per_launch": exec_flops},
             "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -1020,6 +1029,8 @@ def main(argv=None):
     ap.add_argument("--per-config-steps", type=int, default=10,
                     help="timed steps for each of the other forward configurations recorded "
                          "under per_config in the default (wan, one GPU) run; 0 skips them")
+    ap.add_argument("--bwd-kernel", choices=("two", "one_pass"), default="two",
+                    help="--pass bwd: bsa_attn_bwd (dK/dV + dQ kernels) or bsa_attn_bwd_one_pass")
     ap.add_argument("--rows", choices=("lists", "generated"), default="lists",
                     help="forward: read the block lists (default), or generate every row's key "
                          "blocks inside the attention kernel from the radial geometry / the "

@@ -31,6 +31,7 @@ __all__ = [
     "bsa_gemm_bf16", "bsa_joint_mask_build_varlen", "bsa_attn_fwd_varlen",
     "bsa_attn_fwd_varlen_workspace_bytes", "radial_block_lists_varlen", "attention_varlen",
     "bsa_attn_bwd_varlen", "bsa_attn_bwd_varlen_workspace_bytes", "attention_varlen_backward",
+    "bsa_attn_bwd_one_pass", "bsa_attn_bwd_one_pass_workspace_bytes",
     "bsa_attn_fwd_patterns", "bsa_attn_fwd_radial",
     "bsa_attn_fwd_strided", "bsa_attn_module_workspace_bytes", "bsa_joint_mask_build",
     "bsa_attn_fwd_host", "bsa_attn_fwd_host_workspace_bytes", "bsa_attn_bwd_strided",
@@ -462,6 +463,28 @@ def bsa_attn_bwd_host(q, k, v, out, dout, lse, lists: BlockLists, dq, dk, dv, wo
                                _ptr(dv), _ptr(workspace),
                                workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "bsa_attn_bwd_host")
+
+
+def bsa_attn_bwd_one_pass_workspace_bytes(batch: int, heads: int, n: int,
+                                          lists: BlockLists) -> int:
+    return int(_lib.load().bsa_attn_bwd_one_pass_workspace_bytes(batch, heads, n,
+                                                                 ctypes.byref(lists.c_struct())))
+
+
+def bsa_attn_bwd_one_pass(q, k, v, out, dout, lse, lists: BlockLists, dq, dk, dv, workspace=None,
+                          softmax_scale: float = 0.0, stream=None) -> None:
+    """The backward from one kernel (block 128; dQ parts added in row order)."""
+    B, H, n, D = q.shape
+    lib = _lib.load()
+    ls = lists.c_struct()
+    if workspace is None:
+        workspace = torch.empty(max(lib.bsa_attn_bwd_one_pass_workspace_bytes(
+            B, H, n, ctypes.byref(ls)), 16), dtype=torch.uint8, device=q.device)
+    st = lib.bsa_attn_bwd_one_pass(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), B,
+                                   H, n, D, float(softmax_scale), ctypes.byref(ls), _ptr(dq),
+                                   _ptr(dk), _ptr(dv), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "bsa_attn_bwd_one_pass")
 
 
 def bsa_attn_bwd_strided(q, k, v, out, dout, lse, lists: BlockLists, dq, dk, dv, workspace=None,

@@ -41,6 +41,8 @@ EXPORTS = (
     "bsa_attn_bwd_varlen_workspace_bytes",
     "bsa_attn_bwd_varlen",
     "bsa_attn_bwd_workspace_bytes",
+    "bsa_attn_bwd_one_pass_workspace_bytes",
+    "bsa_attn_bwd_one_pass",
     "bsa_attn_bwd_host_workspace_bytes",
     "bsa_attn_bwd_host",
     "bsa_validate_lists",
@@ -169,6 +171,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bsa_attn_bwd": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, ctypes.c_float,
                                         lp, vp, vp, vp, vp, sz, vp]),
         "bsa_attn_bwd_workspace_bytes": (sz, [i32, i32, i32, lp]),
+        "bsa_attn_bwd_one_pass_workspace_bytes": (sz, [i32, i32, i32, lp]),
+        "bsa_attn_bwd_one_pass": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                                 ctypes.c_float, lp, vp, vp, vp, vp, sz, vp]),
         "bsa_attn_bwd_host_workspace_bytes": (sz, [i32, i32, i32, i32, lp]),
         "bsa_attn_bwd_host": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
                                              ctypes.c_float, lp, vp, vp, vp, vp, sz, vp]),

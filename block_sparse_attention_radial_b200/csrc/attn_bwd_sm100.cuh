@@ -58,6 +58,12 @@ struct BwdParams {
   int32_t *item_counter;  // next work item; zeroed by bwd_prep_kernel
   float scale, scale_log2;
   unsigned long long wait_limit_ns;
+  // one-pass kernel only: the dQ accumulator rows ([bh][nqb * 128][D] fp32),
+  // the part counters ([bh][nqb][4]) and, per transposed entry, the key
+  // block's position in its query block's row
+  float *dq_acc = nullptr;
+  int32_t *dq_sem = nullptr;
+  const int32_t *row_pos = nullptr;
 };
 
 constexpr int kBwdBlock = 128;
@@ -146,11 +152,12 @@ __global__ void csc_count_kernel(const int32_t *row_ptr, const int32_t *col_idx,
 
 // One CTA per (list, key block): its query blocks in ascending order, at
 // col_ptr (the inclusive scan of the counts), and with rmask given each
-// entry's mask into cmask. Writes stay below `cap` (the entries row_idx
-// holds) even for lists the validator would reject.
+// entry's mask into cmask and (row_pos non-null) the key block's position in
+// the query block's row into row_pos. Writes stay below `cap` (the entries
+// row_idx holds) even for lists the validator would reject.
 __global__ void csc_fill_kernel(const int32_t *row_ptr, const int32_t *col_idx, int nqb, int nkb,
                                 int nnz, const int32_t *col_ptr, int32_t *row_idx, int cap,
-                                const uint8_t *rmask, uint8_t *cmask) {
+                                const uint8_t *rmask, uint8_t *cmask, int32_t *row_pos) {
   __shared__ int scratch[32];
   const int list = blockIdx.x / nkb, kb = blockIdx.x - list * nkb;
   const int32_t *rp = row_ptr + static_cast<long long>(list) * nqb;
@@ -158,9 +165,10 @@ __global__ void csc_fill_kernel(const int32_t *row_ptr, const int32_t *col_idx, 
   const int end = col_ptr[blockIdx.x + 1];
   for (int q0 = 0; q0 < nqb; q0 += blockDim.x) {
     const int qb = q0 + threadIdx.x;
-    int at = -1;
+    int at = -1, a = 0;
     if (qb < nqb) {
-      const int a = min(max(rp[qb], 0), nnz), b = min(max(rp[qb + 1], 0), nnz);
+      a = min(max(rp[qb], 0), nnz);
+      const int b = min(max(rp[qb + 1], 0), nnz);
       at = row_find(col_idx, a, b, kb);
     }
     const bool has = at >= 0;
@@ -170,6 +178,7 @@ __global__ void csc_fill_kernel(const int32_t *row_ptr, const int32_t *col_idx, 
     if (has && pos >= 0 && pos < end && pos < cap) {
       row_idx[pos] = qb;
       if (rmask) cmask[pos] = rmask[at];
+      if (row_pos) row_pos[pos] = at - a;
     }
     base += total;
   }

@@ -16,6 +16,7 @@
 
 #include "bsa.h"
 
+#include "attn_bwd_fused_sm100.cuh"
 #include "attn_bwd_sm100.cuh"
 #include "attn_fwd_pair_sm100.cuh"
 #include "attn_fwd_sm100.cuh"
@@ -53,7 +54,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   bool probed = false;
   int cc_major = 0, cc_minor = 0, sms = 0;
-  bool attrs_set[14] = {};
+  bool attrs_set[16] = {};
   bool ref_attrs_set[4] = {false, false, false, false};
   bool gemm_attrs_set[4] = {false, false, false, false};
   bool pair_attrs_set[10] = {};
@@ -622,16 +623,21 @@ QkvViews contiguous_views(const void *q, const void *k, const void *v, int batch
 
 // Workspace of the backward pass: lse2 and delta per padded query row, then
 // the transposed lists; for block-64 lists also the per-entry masks of the
-// transposed lists and the 128-row tile lists (pointers, entries, masks).
-// Offsets are 256-byte aligned (the bulk copies of lse2 / delta rows need
-// 16-byte aligned 512-byte rows).
+// transposed lists and the 128-row tile lists (pointers, entries, masks); for
+// block-128 lists of a regular call (the one-pass kernel) the key blocks'
+// positions in their query rows, the dQ part counters and the fp32 dQ
+// accumulator rows (sized for head_dim 128, the largest). Offsets are
+// 256-byte aligned (the bulk copies of lse2 / delta rows need 16-byte
+// aligned 512-byte rows).
 struct BwdLayout {
-  size_t lse2, delta, counters, col_ptr, row_idx, cmask, tile_ptr, tile_col, tile_mask, total;
+  size_t lse2, delta, counters, col_ptr, row_idx, cmask, tile_ptr, tile_col, tile_mask;
+  size_t row_pos, dq_sem, dq_acc, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-BwdLayout bwd_layout(int32_t batch, int32_t heads, int32_t n, const bsa_block_lists *l) {
+BwdLayout bwd_layout(int32_t batch, int32_t heads, int32_t n, const bsa_block_lists *l,
+                     bool one_pass = false) {
   BwdLayout w;
   const size_t nt = static_cast<size_t>(ceil_div(n, kBwdBlock));  // 128-row tiles
   const size_t rows = static_cast<size_t>(batch) * heads * nt * kBwdBlock;
@@ -649,6 +655,13 @@ BwdLayout bwd_layout(int32_t batch, int32_t heads, int32_t n, const bsa_block_li
     w.tile_col = w.tile_ptr + align256(ptrs);
     w.tile_mask = w.tile_col + align256(entries * sizeof(int32_t));
     w.total = w.tile_mask + align256(entries);
+  }
+  w.row_pos = w.dq_sem = w.dq_acc = w.total;
+  if (one_pass && l->block == kBwdBlock) {
+    const size_t qblocks = static_cast<size_t>(batch) * heads * nt;
+    w.dq_sem = w.row_pos + align256(entries * sizeof(int32_t));
+    w.dq_acc = w.dq_sem + align256(qblocks * 4 * sizeof(int32_t));
+    w.total = w.dq_acc + align256(qblocks * kBwdBlock * 128 * sizeof(float));
   }
   return w;
 }
@@ -721,6 +734,47 @@ int launch_bwd_kernels(const BwdViews &x, int32_t n_map, BwdParams &p, bool mask
   return BSA_OK;
 }
 
+// The one-pass backward (block 128): counters and dq of empty rows
+// initialised, then one kernel for dK, dV and dQ over `items` (batch*head,
+// key block) work items; rows = batch*heads*nqb*128 padded query rows.
+template <int D>
+int launch_bwd_one_pass(const BwdViews &x, int32_t n_map, BwdParams &p, long long items,
+                        long long rows, DeviceInfo *dev, cudaStream_t stream) {
+  CUtensorMap tq, tk, tv, td;
+  int st;
+  if ((st = make_map_strided(&tq, x.q, x.lq, x.batch, x.heads, n_map, D, kBwdBlock)) != BSA_OK)
+    return st;
+  if ((st = make_map_strided(&tk, x.k, x.lk, x.batch, x.heads, n_map, D, kBwdBlock)) != BSA_OK)
+    return st;
+  if ((st = make_map_strided(&tv, x.v, x.lv, x.batch, x.heads, n_map, D, kBwdBlock)) != BSA_OK)
+    return st;
+  if ((st = make_map_strided(&td, x.dout, x.ldo, x.batch, x.heads, n_map, D, kBwdBlock)) != BSA_OK)
+    return st;
+  const int slot = 14 + (D == 128 ? 1 : 0);
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!dev->attrs_set[slot]) {
+      BSA_CUDA(cudaFuncSetAttribute(attn_bwd_fused_kernel<D>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    FusedCfg<D>::DSMEM));
+      dev->attrs_set[slot] = true;
+    }
+  }
+  const long long sems = rows / kBwdBlock * 4;
+  const long long threads = rows > sems ? rows : sems;
+  fused_init_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
+      p, rows, sems);
+  BSA_CUDA(cudaGetLastError());
+  p.total_items = static_cast<int32_t>(items);
+  const int grid = p.total_items < dev->sms ? p.total_items : dev->sms;
+  if (grid > 0) {
+    attn_bwd_fused_kernel<D><<<grid, FusedCfg<D>::THREADS, FusedCfg<D>::DSMEM, stream>>>(
+        tq, tk, tv, td, p);
+    BSA_CUDA(cudaGetLastError());
+  }
+  return BSA_OK;
+}
+
 // Parameters shared by every backward launch of a call.
 template <int D>
 BwdParams bwd_params(const BwdViews &x, const bsa_block_lists *l, float softmax_scale) {
@@ -750,11 +804,14 @@ BwdParams bwd_params(const BwdViews &x, const bsa_block_lists *l, float softmax_
   return p;
 }
 
+// one_pass (block 128 only): dK, dV and dQ from the one-pass kernel with the
+// dQ parts added in order; otherwise the dK/dV and dQ kernels.
 template <int D>
 int launch_bwd(const BwdViews &x, const float *lse, int32_t n, float softmax_scale,
-               const bsa_block_lists *l_in, uint8_t *ws, DeviceInfo *dev, cudaStream_t stream) {
+               const bsa_block_lists *l_in, uint8_t *ws, DeviceInfo *dev, cudaStream_t stream,
+               bool one_pass = false) {
   const int32_t bh = x.batch * x.heads;
-  const BwdLayout w = bwd_layout(1, bh, n, l_in);
+  const BwdLayout w = bwd_layout(1, bh, n, l_in, one_pass);
   float *lse2 = reinterpret_cast<float *>(ws + w.lse2);
   float *delta = reinterpret_cast<float *>(ws + w.delta);
   int32_t *col_ptr = reinterpret_cast<int32_t *>(ws + w.col_ptr);
@@ -806,8 +863,10 @@ int launch_bwd(const BwdViews &x, const float *lse, int32_t n, float softmax_sca
   BSA_CUDA(cudaGetLastError());
   scan_rows_kernel<<<1, 1024, 0, stream>>>(col_ptr, cols);
   BSA_CUDA(cudaGetLastError());
+  int32_t *row_pos = one_pass ? reinterpret_cast<int32_t *>(ws + w.row_pos) : nullptr;
   csc_fill_kernel<<<cols, 256, 0, stream>>>(l->row_ptr, l->col_idx, nqb, nkb, l->nnz, col_ptr,
-                                            row_idx, l->nnz > 0 ? l->nnz : 1, rmask, cmask);
+                                            row_idx, l->nnz > 0 ? l->nnz : 1, rmask, cmask,
+                                            row_pos);
   BSA_CUDA(cudaGetLastError());
 
   BwdParams p = bwd_params<D>(x, l, softmax_scale);
@@ -823,6 +882,12 @@ int launch_bwd(const BwdViews &x, const float *lse, int32_t n, float softmax_sca
   p.row_ptr = l->row_ptr;
   p.col_idx = l->col_idx;
   p.item_counter = reinterpret_cast<int32_t *>(ws + w.counters);
+  if (one_pass) {
+    p.row_pos = row_pos;
+    p.dq_sem = reinterpret_cast<int32_t *>(ws + w.dq_sem);
+    p.dq_acc = reinterpret_cast<float *>(ws + w.dq_acc);
+    return launch_bwd_one_pass<D>(x, n, p, static_cast<long long>(bh) * nkb, rows, dev, stream);
+  }
   return launch_bwd_kernels<D>(x, n, p, rmask != nullptr, nullptr,
                                static_cast<long long>(bh) * nkb, static_cast<long long>(bh) * nqb,
                                dev, stream);
@@ -873,7 +938,7 @@ int launch_bwd_varlen(const BwdViews &x, const float *lse, int32_t total, float 
     const long long lr = static_cast<long long>(L) * vt.row0[b];
     csc_fill_kernel<<<L * nq, 256, 0, stream>>>(l->row_ptr + lr, l->col_idx, nq, nq, l->nnz,
                                                 col_ptr + lr, row_idx, l->nnz > 0 ? l->nnz : 1,
-                                                nullptr, nullptr);
+                                                nullptr, nullptr, nullptr);
     BSA_CUDA(cudaGetLastError());
   }
   BwdParams p = bwd_params<D>(x, l, softmax_scale);
@@ -1666,10 +1731,17 @@ size_t bsa_attn_bwd_workspace_bytes(int32_t batch, int32_t heads, int32_t n,
   return bwd_layout(batch, heads, n, l).total;
 }
 
-int bsa_attn_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout,
-                 const float *lse, int32_t batch, int32_t heads, int32_t n, int32_t head_dim,
-                 float softmax_scale, const bsa_block_lists *l, void *dq, void *dk, void *dv,
-                 void *workspace, size_t workspace_bytes, bsa_stream_t stream_) {
+}  // extern "C"
+
+namespace {
+
+// bsa_attn_bwd and bsa_attn_bwd_one_pass: contiguous views, the two-kernel
+// or (one_pass, block 128) the one-pass backward.
+int attn_bwd_contiguous(const void *q, const void *k, const void *v, const void *out,
+                        const void *dout, const float *lse, int32_t batch, int32_t heads,
+                        int32_t n, int32_t head_dim, float softmax_scale,
+                        const bsa_block_lists *l, void *dq, void *dk, void *dv, void *workspace,
+                        size_t workspace_bytes, bsa_stream_t stream_, bool one_pass) {
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   int st = check_attn_args(q, k, v, batch, heads, n, head_dim, l, dq);
   if (st != BSA_OK) return st;
@@ -1688,7 +1760,8 @@ int bsa_attn_bwd(const void *q, const void *k, const void *v, const void *out, c
     for (int b = a + 1; b < 3; ++b)
       if (overlaps(outs[a], bytes, outs[b], bytes)) return BSA_ERR_INVALID_ARG;
   }
-  const size_t need = bwd_layout(batch, heads, n, l).total;
+  if (one_pass && l->block != kBwdBlock) return BSA_ERR_UNSUPPORTED;
+  const size_t need = bwd_layout(batch, heads, n, l, one_pass).total;
   if (!workspace || !aligned16(workspace) || workspace_bytes < need) return BSA_ERR_INVALID_ARG;
   if (overlaps(workspace, need, ins[0], bytes) || overlaps(workspace, need, dq, bytes) ||
       overlaps(workspace, need, dk, bytes) || overlaps(workspace, need, dv, bytes))
@@ -1710,8 +1783,36 @@ int bsa_attn_bwd(const void *q, const void *k, const void *v, const void *out, c
   x.batch = batch;
   x.heads = heads;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
-  if (head_dim == 128) return launch_bwd<128>(x, lse, n, softmax_scale, l, ws, dev, stream);
-  return launch_bwd<64>(x, lse, n, softmax_scale, l, ws, dev, stream);
+  if (head_dim == 128)
+    return launch_bwd<128>(x, lse, n, softmax_scale, l, ws, dev, stream, one_pass);
+  return launch_bwd<64>(x, lse, n, softmax_scale, l, ws, dev, stream, one_pass);
+}
+
+}  // namespace
+
+extern "C" {
+
+int bsa_attn_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout,
+                 const float *lse, int32_t batch, int32_t heads, int32_t n, int32_t head_dim,
+                 float softmax_scale, const bsa_block_lists *l, void *dq, void *dk, void *dv,
+                 void *workspace, size_t workspace_bytes, bsa_stream_t stream) {
+  return attn_bwd_contiguous(q, k, v, out, dout, lse, batch, heads, n, head_dim, softmax_scale, l,
+                             dq, dk, dv, workspace, workspace_bytes, stream, false);
+}
+
+size_t bsa_attn_bwd_one_pass_workspace_bytes(int32_t batch, int32_t heads, int32_t n,
+                                             const bsa_block_lists *l) {
+  if (bsa_attn_bwd_workspace_bytes(batch, heads, n, l) == 0 || l->block != kBwdBlock) return 0;
+  return bwd_layout(batch, heads, n, l, true).total;
+}
+
+int bsa_attn_bwd_one_pass(const void *q, const void *k, const void *v, const void *out,
+                          const void *dout, const float *lse, int32_t batch, int32_t heads,
+                          int32_t n, int32_t head_dim, float softmax_scale,
+                          const bsa_block_lists *l, void *dq, void *dk, void *dv, void *workspace,
+                          size_t workspace_bytes, bsa_stream_t stream) {
+  return attn_bwd_contiguous(q, k, v, out, dout, lse, batch, heads, n, head_dim, softmax_scale, l,
+                             dq, dk, dv, workspace, workspace_bytes, stream, true);
 }
 
 int bsa_attn_dense_masked_ref(const void *q, const void *k, const void *v, int32_t batch,

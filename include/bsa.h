@@ -562,7 +562,8 @@ int bsa_attn_dense_masked_ref(const void *q, const void *k, const void *v,
  * at least bsa_attn_bwd_workspace_bytes() bytes, 16-byte aligned, owned by the
  * caller. Supported: block 64 or 128, head_dim 64 or 128 (block-64 lists
  * run as 128-row tiles with a mask of the listed 64 x 64 quarters).
- * Deterministic: every output row is written by one
+ * Two kernels: dK/dV per key block, then dQ per query block (which
+ * recomputes S and dP). Deterministic: every output row is written by one
  * CTA, no atomics. Asynchronous on `stream`; device timeouts are reported
  * through bsa_get_device_status(). Returns BSA_OK or an argument / CUDA error.
  */
@@ -654,6 +655,41 @@ int bsa_attn_bwd_varlen(const void *q, const bsa_layout *q_layout,
  */
 size_t bsa_attn_bwd_workspace_bytes(int32_t batch, int32_t heads, int32_t n,
                                     const bsa_block_lists *lists);
+
+/*
+ * Bytes of device scratch bsa_attn_bwd_one_pass needs: bsa_attn_bwd's, plus
+ * each transposed entry's position in its query row (nnz ints), four dQ part
+ * counters per (batch, head, query block) and an fp32 dQ accumulator row of
+ * 128 floats per padded query row (512 bytes: the largest head_dim). 0 for
+ * invalid arguments or block 64.
+ */
+size_t bsa_attn_bwd_one_pass_workspace_bytes(int32_t batch, int32_t heads, int32_t n,
+                                             const bsa_block_lists *lists);
+
+/*
+ * bsa_attn_bwd's gradients from ONE kernel (block 128): per (batch*head, key
+ * block) it computes S, dP, dV, dK and this key block's part of dQ for each
+ * listed query block once (five block products per listed pair instead of
+ * seven), and the dQ parts of a query block are added in the order of its
+ * row's key blocks: a counter per (query block, 32 rows) admits them one by
+ * one into an fp32 accumulator row in the workspace, the last part writes
+ * dq. Deterministic (the same sum in the same order on every call); dk, dv
+ * are bit-identical to bsa_attn_bwd, dq equal up to rounding order. On a B200
+ * it is slower than bsa_attn_bwd on the radial workloads: the ordered dQ
+ * parts are 64 KB of fp32 per listed block pair through L2 (measured on Wan:
+ * 84.8 ms against 32.5 ms; 50.1 ms with unordered atomic adds, 27.7 ms
+ * without any dQ accumulation). Lists must be well formed
+ * (bsa_validate_lists): with a duplicated or out-of-range entry a row's
+ * counter may never reach a part's turn and the call ends with
+ * BSA_ERR_DEVICE_TIMEOUT after the wait limit. Arguments as bsa_attn_bwd,
+ * workspace bsa_attn_bwd_one_pass_workspace_bytes(); BSA_ERR_UNSUPPORTED for
+ * block 64. Asynchronous.
+ */
+int bsa_attn_bwd_one_pass(const void *q, const void *k, const void *v, const void *out,
+                          const void *dout, const float *lse, int32_t batch, int32_t heads,
+                          int32_t n, int32_t head_dim, float softmax_scale,
+                          const bsa_block_lists *lists, void *dq, void *dk, void *dv,
+                          void *workspace, size_t workspace_bytes, bsa_stream_t stream);
 
 /*
  * Bytes of device workspace bsa_attn_bwd_host needs: device copies of q, k,

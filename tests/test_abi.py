@@ -130,13 +130,19 @@ def test_backward_workspace_and_host_checks(lib):
     ls = BlockListsC(1, 256, 256, 128, 1000, 0, 0)
     # lse2 + delta: 2 x 40 x 256 x 128 floats; 256 bytes of work counters;
     # offsets 257 ints; 1000 entries
-    expect = 2 * 40 * 256 * 128 * 4 + 256 + 1280 + 4096
+    common = 2 * 40 * 256 * 128 * 4 + 256 + 1280 + 4096
+    expect = common
     assert lib.bsa_attn_bwd_workspace_bytes(1, 40, 32760, ctypes.byref(ls)) == expect
+    # the one-pass kernel: plus the entries' row positions, 4 dQ part
+    # counters per query block, fp32 dQ rows of 128 per padded query row
+    one = common + 4096 + 40 * 256 * 4 * 4 + 40 * 256 * 128 * 128 * 4
+    assert lib.bsa_attn_bwd_one_pass_workspace_bytes(1, 40, 32760, ctypes.byref(ls)) == one
     assert lib.bsa_attn_bwd_workspace_bytes(1, 40, 32769, ctypes.byref(ls)) == 0  # nqb mismatch
-    # block 64: the same plus masks of the transposed entries and the 128-row tile lists
+    # block 64: masks of the transposed entries and the 128-row tile lists
     ls64 = BlockListsC(1, 512, 512, 64, 1000, 0, 0)
-    expect64 = expect + 1024 + 1280 + 4096 + 1024
+    expect64 = common + 1024 + 1280 + 4096 + 1024
     assert lib.bsa_attn_bwd_workspace_bytes(1, 40, 32760, ctypes.byref(ls64)) == expect64
+    assert lib.bsa_attn_bwd_one_pass_workspace_bytes(1, 40, 32760, ctypes.byref(ls64)) == 0
     assert lib.bsa_attn_bwd_workspace_bytes(1, 40, 32769, ctypes.byref(ls64)) == 0  # nqb mismatch
     # bad arguments are rejected on the host, before any CUDA call
     p = ctypes.c_void_p(4096)
