@@ -726,6 +726,26 @@ __global__ void __launch_bounds__(384, 1)
           // a row without a reference maximum has every column at -inf here
           // (its block maximum is -inf): any finite bias gives P = 0, sum 0
           const float bias = MODE == kModeQuarters && m_ref == -INFINITY ? 0.f : -m_ref;
+          if (MODE == kModeQuarters) {
+            // the exponentials of a key half this warp's query half does not
+            // list are not computed (P = 0 there); both halves listed: the
+            // same operations in the same order as a whole row
+            float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                             make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            if (qbits & 1u) {
+              exp2_pack_pairs<BN, 0, 0, BN / 4>(s, sl2, bias, pk, acc);
+            } else {
+#pragma unroll
+              for (int c = 0; c < BN / 4; ++c) pk[c] = 0u;
+            }
+            if (qbits & 2u) {
+              exp2_pack_pairs<BN, 0, BN / 4, BN / 2>(s, sl2, bias, pk, acc);
+            } else {
+#pragma unroll
+              for (int c = BN / 4; c < BN / 2; ++c) pk[c] = 0u;
+            }
+            return exp2_row_sum(acc);
+          }
           return valid < BN ? exp2_pack_row<BN, 0>(s, sl2, bias, pk)
                             : exp2_pack_row<BN, kEmuPairsPer8>(s, sl2, bias, pk);
         };

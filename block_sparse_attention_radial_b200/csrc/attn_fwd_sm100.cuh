@@ -269,15 +269,15 @@ constexpr int kEmuPairsPer8 = BSA_EMU_PAIRS;
 
 // p = 2^(s * sl2 + neg) for one row of BN scores: returns the fp32 row sum and
 // the values packed as bf16 pairs. EMU of every 8 pairs use the polynomial.
-template <int BN, int EMU>
-__device__ __forceinline__ float exp2_pack_row(const float (&s)[BN], float sl2, float neg,
-                                               uint32_t (&pk)[BN / 2]) {
+// Column pairs [C0, C1) of the row into the four partial sums acc (pair c
+// into acc[c % 4]); a whole row is [0, BN / 2) and then exp2_row_sum.
+template <int BN, int EMU, int C0, int C1>
+__device__ __forceinline__ void exp2_pack_pairs(const float (&s)[BN], float sl2, float neg,
+                                                uint32_t (&pk)[BN / 2], float2 (&acc)[4]) {
   const float2 neg2 = make_float2(neg, neg);
   const float2 sl2v = make_float2(sl2, sl2);
-  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                   make_float2(0.f, 0.f)};
 #pragma unroll
-  for (int c = 0; c < BN / 2; ++c) {
+  for (int c = C0; c < C1; ++c) {
     const float2 x = ffma2(make_float2(s[2 * c], s[2 * c + 1]), sl2v, neg2);
     float2 pp;
     if ((c & 7) < EMU) {
@@ -288,8 +288,20 @@ __device__ __forceinline__ float exp2_pack_row(const float (&s)[BN], float sl2, 
     acc[c & 3] = fadd2(acc[c & 3], pp);
     pk[c] = pack_bf16x2(pp.x, pp.y);
   }
+}
+
+__device__ __forceinline__ float exp2_row_sum(const float2 (&acc)[4]) {
   const float2 a = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
   return a.x + a.y;
+}
+
+template <int BN, int EMU>
+__device__ __forceinline__ float exp2_pack_row(const float (&s)[BN], float sl2, float neg,
+                                               uint32_t (&pk)[BN / 2]) {
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};
+  exp2_pack_pairs<BN, EMU, 0, BN / 2>(s, sl2, neg, pk, acc);
+  return exp2_row_sum(acc);
 }
 
 template <int D, int BN>
