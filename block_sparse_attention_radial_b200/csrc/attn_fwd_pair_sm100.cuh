@@ -182,6 +182,33 @@ struct UnionWalker {
   }
 };
 
+// Key blocks of one query-block pair from the two rows' bitmaps in shared
+// memory, walked as their union (rows generated ahead by the item fetcher).
+struct BitmapWalker {
+  const volatile uint32_t *a, *b;
+  int w, nw;
+  uint32_t cur;
+  __device__ __forceinline__ void reset(const uint32_t *ba, const uint32_t *bb, int nwords) {
+    a = ba;
+    b = bb;
+    nw = nwords;
+    w = 0;
+    cur = nwords > 0 ? (a[0] | b[0]) : 0u;
+  }
+  __device__ __forceinline__ bool next(int &kb, bool &inA, bool &inB) {
+    while (cur == 0u) {
+      if (++w >= nw) return false;
+      cur = a[w] | b[w];
+    }
+    const int bit = __ffs(cur) - 1;
+    cur &= cur - 1u;
+    kb = w * 32 + bit;
+    inA = ((a[w] >> bit) & 1u) != 0u;
+    inB = ((b[w] >> bit) & 1u) != 0u;
+    return true;
+  }
+};
+
 constexpr int kItemN = 4;  // work items in flight between the producer and the consumers
 
 struct PairItem {
@@ -328,6 +355,15 @@ __global__ void __launch_bounds__(384, 1)
   // from tile patterns only)
   __shared__ bsa_tile_pattern prod_pat;
   __shared__ __align__(8) uint64_t bar_item_full[kItemN], bar_item_empty[kItemN];
+  // Rows generated in the kernel: warp 10 takes the work items instead of
+  // the producer and generates each item's two rows into bitmaps here
+  // (rows of up to kGenRowWords * 32 key blocks; longer rows are generated
+  // by the producer as it walks them), a few items ahead of the walk.
+  constexpr bool kGen = MODE == kModePatterns || MODE == kModeRadial;
+  constexpr int kGenRowWords = 32;
+  __shared__ uint32_t row_bits[kGen ? kItemN : 1][2][kGen ? kGenRowWords : 1];
+  __shared__ int row_len[kGen ? kItemN : 1][2];
+  const bool bitmaps = kGen && p.nkb <= kGenRowWords * 32;
 
   const uint32_t raw = smem_addr(dsmem);
   uint8_t *base = dsmem + (((raw + 1023u) & ~1023u) - raw);
@@ -355,7 +391,9 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int i = 0; i < kItemN; ++i) {
       mbar_init(&bar_item_full[i], 1);
-      mbar_init(&bar_item_empty[i], 9);  // the MMA lane and one lane per softmax warp
+      // the MMA lane and one lane per softmax warp (and, for generated rows,
+      // the producer once it has walked the item's bitmaps)
+      mbar_init(&bar_item_empty[i], kGen ? 10 : 9);
     }
     abort_flag = 0;
     fence_barrier_init();
@@ -393,15 +431,28 @@ __global__ void __launch_bounds__(384, 1)
         bool ok = true;
         for (int k = 0; ok; ++k) {
           const int slot = k % kItemN;
-          if (!(ok = lane_wait(&bar_item_empty[slot], ((k / kItemN) & 1) ^ 1, wc, kBarItem, k)))
-            break;
-          int idx = atomicAdd(p.item_counter, 1);
-          if (idx >= p.total_items) idx = -1;
-          item_ring[slot] = idx;
-          mbar_arrive(&bar_item_full[slot]);
+          int idx;
+          if (kGen) {  // warp 10 takes the items
+            if (!(ok = lane_wait(&bar_item_full[slot], (k / kItemN) & 1, wc, kBarItem, k))) break;
+            idx = *static_cast<volatile int *>(&item_ring[slot]);
+          } else {
+            if (!(ok = lane_wait(&bar_item_empty[slot], ((k / kItemN) & 1) ^ 1, wc, kBarItem, k)))
+              break;
+            idx = atomicAdd(p.item_counter, 1);
+            if (idx >= p.total_items) idx = -1;
+            item_ring[slot] = idx;
+            mbar_arrive(&bar_item_full[slot]);
+          }
           if (idx < 0) break;
-          const PairItem it = decode_pair<MODE>(idx, p, npairs, vt);
-          if (it.lenA == 0 && it.lenB == 0) continue;
+          PairItem it = decode_pair<MODE>(idx, p, npairs, vt);
+          if (bitmaps) {
+            it.lenA = *static_cast<volatile int *>(&row_len[slot][0]);
+            it.lenB = *static_cast<volatile int *>(&row_len[slot][1]);
+          }
+          if (it.lenA == 0 && it.lenB == 0) {
+            if (kGen) mbar_arrive(&bar_item_empty[slot]);
+            continue;
+          }
           if (!(ok = lane_wait(&bar_q_empty, (qcount & 1u) ^ 1u, wc, kBarQEmpty, qcount))) break;
           mbar_arrive_expect_tx(&bar_q_full, 2 * C::Q_BYTES);
           const int ib = it.bh / p.heads, ih = it.bh - ib * p.heads;
@@ -412,15 +463,20 @@ __global__ void __launch_bounds__(384, 1)
           // Same walk and same first-use order as the MMA issuer: at step j it
           // needs V(j-1) first when tile A listed j-1 or A skips j, and K(j)
           // first otherwise.
-          if (MODE == kModePatterns) prod_pat = p.patterns[it.list];
           UnionWalker<MODE> uw;
-          uw.reset(p, it.list, it.qa, it.a0, it.lenA, it.b0, it.lenB, it.nkb, &prod_pat);
+          BitmapWalker bw;
+          if (bitmaps) {
+            bw.reset(row_bits[slot][0], row_bits[slot][1], (it.nkb + 31) >> 5);
+          } else {
+            if (MODE == kModePatterns) prod_pat = p.patterns[it.list];
+            uw.reset(p, it.list, it.qa, it.a0, it.lenA, it.b0, it.lenB, it.nkb, &prod_pat);
+          }
           bool pa = false, pb = false;
           int prev_kb = 0;
           while (ok) {
             int kb = 0;
             bool a = false, b = false;
-            const bool more = uw.next(kb, a, b);
+            const bool more = bitmaps ? bw.next(kb, a, b) : uw.next(kb, a, b);
             const bool need_v = pa || pb;
             if (!more && !need_v) break;
             const bool v_first = pa || !a;
@@ -459,6 +515,8 @@ __global__ void __launch_bounds__(384, 1)
             prev_kb = kb;
             if (!more) break;
           }
+          // the item's rows are walked: its slot may take the next item
+          if (kGen && ok) mbar_arrive(&bar_item_empty[slot]);
         }
         WaitCtx drain{&abort_flag, p.wait_limit_ns, kRoleProducer};
         int zero = 0;
@@ -498,9 +556,18 @@ __global__ void __launch_bounds__(384, 1)
           const int slot = k % kItemN;
           if (!(ok = lane_wait(&bar_item_full[slot], (k / kItemN) & 1, wc, kBarItem, k))) break;
           const int idx = *static_cast<volatile int *>(&item_ring[slot]);
+          int glen[2] = {0, 0};
+          if (bitmaps && idx >= 0) {  // read before the slot is released
+            glen[0] = *static_cast<volatile int *>(&row_len[slot][0]);
+            glen[1] = *static_cast<volatile int *>(&row_len[slot][1]);
+          }
           mbar_arrive(&bar_item_empty[slot]);
           if (idx < 0) break;
-          const PairItem it = decode_pair<MODE>(idx, p, npairs, vt);
+          PairItem it = decode_pair<MODE>(idx, p, npairs, vt);
+          if (bitmaps) {
+            it.lenA = glen[0];
+            it.lenB = glen[1];
+          }
           if (it.lenA == 0 && it.lenB == 0) continue;
           if (!(ok = lane_wait(&bar_q_full, qcount & 1u, wc, kBarQFull, qcount))) break;
           tc_fence_after();
@@ -608,8 +675,55 @@ __global__ void __launch_bounds__(384, 1)
         wait_bounded(&bar_final, 0, drain, kBarFinal, qcount);
       }
       __syncwarp();
+    } else if (kGen && warp == 10) {
+      // ------------------------------------------------- item fetcher (rows
+      // generated in the kernel): takes the work items from the counter and,
+      // a few items ahead of the producer's walk, generates each item's two
+      // rows into bitmaps (lane r generates row r; every lane clears a word)
+      wc.role = kRoleProducer;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int slot = k % kItemN;
+        if (!(ok = warp_wait(&bar_item_empty[slot], ((k / kItemN) & 1) ^ 1, wc, kBarItem, k)))
+          break;
+        int idx = 0;
+        if (lane == 0) {
+          idx = atomicAdd(p.item_counter, 1);
+          if (idx >= p.total_items) idx = -1;
+        }
+        idx = __shfl_sync(0xffffffffu, idx, 0);
+        if (idx >= 0 && bitmaps) {
+          const PairItem it = decode_pair<MODE>(idx, p, npairs, vt);
+          row_bits[slot][0][lane] = 0u;
+          row_bits[slot][1][lane] = 0u;
+          __syncwarp();
+          if (lane < 2) {
+            const int qb = it.qa + lane;
+            int cnt = 0;
+            if (qb < it.nqb) {
+              RowSource<MODE> rs;
+              rs.reset(p, it.list, qb, lane == 0 ? it.a0 : it.b0, lane == 0 ? it.lenA : it.lenB,
+                       it.nkb, MODE == kModePatterns ? p.patterns + it.list : nullptr);
+              for (int kb = rs.next(); kb != INT_MAX; kb = rs.next()) {
+                if (kb < 0 || kb >= it.nkb) continue;
+                row_bits[slot][lane][kb >> 5] |= 1u << (kb & 31);
+                ++cnt;
+              }
+            }
+            row_len[slot][lane] = cnt;
+          }
+          __syncwarp();
+        }
+        if (lane == 0) {
+          item_ring[slot] = idx;
+          mbar_arrive(&bar_item_full[slot]);
+        }
+        __syncwarp();
+        if (idx < 0) break;
+      }
     }
-    // warps 10 and 11 have no role: they wait at the final barrier
+    // warp 11 (and warp 10 when rows come from lists) has no role: it waits
+    // at the final barrier
   } else {
     // ------------------------------------------------------------ softmax
     // Warpgroup t (warps 4t..4t+3) serves tile t; thread = row = TMEM lane.
@@ -628,13 +742,14 @@ __global__ void __launch_bounds__(384, 1)
       const int slot = k % kItemN;
       if (!(ok = warp_wait(&bar_item_full[slot], (k / kItemN) & 1, wc, kBarItem, k))) break;
       const int idx = *static_cast<volatile int *>(&item_ring[slot]);
+      const int glen = bitmaps && idx >= 0 ? *static_cast<volatile int *>(&row_len[slot][t]) : 0;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_item_empty[slot]);
       if (idx < 0) break;
       const PairItem it = decode_pair<MODE>(idx, p, npairs, vt);
       const int qb = it.qa + t;
       if (qb >= it.nqb) continue;
-      const int len = t == 0 ? it.lenA : it.lenB;
+      const int len = bitmaps ? glen : (t == 0 ? it.lenA : it.lenB);
       const int a0 = t == 0 ? it.a0 : it.b0;
       const int row = qb * BN + row_in_tile;
       const bool store = row < it.n;
