@@ -693,24 +693,29 @@ __global__ void __launch_bounds__(384, 1)
         }
         idx = __shfl_sync(0xffffffffu, idx, 0);
         if (idx >= 0 && bitmaps) {
+          // the list builders' own row marking, spread over the warp's lanes
           const PairItem it = decode_pair<MODE>(idx, p, npairs, vt);
-          row_bits[slot][0][lane] = 0u;
-          row_bits[slot][1][lane] = 0u;
-          __syncwarp();
-          if (lane < 2) {
-            const int qb = it.qa + lane;
-            int cnt = 0;
+          const int words = (it.nkb + 31) >> 5;
+#pragma unroll 1
+          for (int r = 0; r < 2; ++r) {
+            uint32_t *bits = row_bits[slot][r];
+            const int qb = it.qa + r;
+            bits[lane] = 0u;
+            __syncwarp();
             if (qb < it.nqb) {
-              RowSource<MODE> rs;
-              rs.reset(p, it.list, qb, lane == 0 ? it.a0 : it.b0, lane == 0 ? it.lenA : it.lenB,
-                       it.nkb, MODE == kModePatterns ? p.patterns + it.list : nullptr);
-              for (int kb = rs.next(); kb != INT_MAX; kb = rs.next()) {
-                if (kb < 0 || kb >= it.nkb) continue;
-                row_bits[slot][lane][kb >> 5] |= 1u << (kb & 31);
-                ++cnt;
+              if (MODE == kModeRadial) {
+                radial_mark_row(p.radial, qb, bits, lane, 32);
+              } else {
+                const bsa_tile_pattern &pat = p.patterns[it.list];
+                const bool pok = pattern_ok(pat, p.num_pattern_columns);
+                pattern_row_words(pat, pok, qb, it.nkb, bits, words, lane, 32);
+                __syncwarp();
+                if (pok) pattern_row_columns(pat, p.pattern_columns, it.nkb, bits, lane, 32, false);
               }
             }
-            row_len[slot][lane] = cnt;
+            __syncwarp();
+            const int cnt = __reduce_add_sync(0xffffffffu, __popc(bits[lane]));
+            if (lane == 0) row_len[slot][r] = cnt;
           }
           __syncwarp();
         }

@@ -62,18 +62,20 @@ __device__ __forceinline__ int band_of(int d) { return 31 - __clz(d < 1 ? 1 : d)
 // Text tokens (after the video tokens) are global: a query block holding a
 // text token lists every key block, and every query block lists the key
 // blocks that hold text tokens.
-__device__ void radial_mark_row(const RadialGeom g, int qb, uint32_t *bits) {
+// Threads tid of nthr share the work (a CTA, or one warp of the attention
+// kernel that generates rows ahead of its producer).
+__device__ void radial_mark_row(const RadialGeom g, int qb, uint32_t *bits, int tid, int nthr) {
   const int t0 = qb * g.block;
   const int t1 = min(g.n, t0 + g.block);  // query tokens [t0, t1)
   if (t1 > g.nv) {
-    for (int b = threadIdx.x; b < g.nb; b += blockDim.x) atomicOr(&bits[b >> 5], 1u << (b & 31));
+    for (int b = tid; b < g.nb; b += nthr) atomicOr(&bits[b >> 5], 1u << (b & 31));
     return;
   }
-  for (int b = g.nv / g.block + threadIdx.x; g.nv < g.n && b < g.nb; b += blockDim.x)
+  for (int b = g.nv / g.block + tid; g.nv < g.n && b < g.nb; b += nthr)
     atomicOr(&bits[b >> 5], 1u << (b & 31));
   const int fa = t0 / g.tpf, fb = (t1 - 1) / g.tpf;
   const int pairs = (fb - fa + 1) * g.frames;
-  for (int p = threadIdx.x; p < pairs; p += blockDim.x) {
+  for (int p = tid; p < pairs; p += nthr) {
     const int fi = fa + p / g.frames, fj = p % g.frames;
     const int d = abs(fi - fj);
     const int r = band_of(d);
@@ -92,7 +94,7 @@ __device__ void radial_mark_row(const RadialGeom g, int qb, uint32_t *bits) {
 __device__ void radial_row_bitmap(const RadialGeom g, int qb, uint32_t *bits, int words) {
   for (int i = threadIdx.x; i < words; i += blockDim.x) bits[i] = 0u;
   __syncthreads();
-  radial_mark_row(g, qb, bits);
+  radial_mark_row(g, qb, bits, threadIdx.x, blockDim.x);
   __syncthreads();
 }
 

@@ -29,12 +29,11 @@ __device__ __forceinline__ bool pattern_ok(const bsa_tile_pattern &p, long long 
          p.columns_end <= num_columns;
 }
 
-// Row qb of pattern p as a bitmap over the nkb key blocks. Each thread builds
-// whole words from the band and axial terms; the stripe columns are then OR-ed
-// in. Ends with the CTA synchronised.
-__device__ void pattern_row_bitmap(const bsa_tile_pattern &p, bool ok, const int32_t *columns,
-                                   int qb, int nkb, uint32_t *bits, int words) {
-  for (int wd = threadIdx.x; wd < words; wd += blockDim.x) {
+// The words [tid, tid + nthr, ...) of a row's bitmap from its bands and
+// axial term (no stripe columns yet); key blocks >= nkb stay clear.
+__device__ void pattern_row_words(const bsa_tile_pattern &p, bool ok, int qb, int nkb,
+                                  uint32_t *bits, int words, int tid, int nthr) {
+  for (int wd = tid; wd < words; wd += nthr) {
     uint32_t m = 0u;
     if (ok) {
       for (int t = 0; t < p.num_bands; ++t)
@@ -57,14 +56,28 @@ __device__ void pattern_row_bitmap(const bsa_tile_pattern &p, bool ok, const int
     if (left < 32) m &= left <= 0 ? 0u : ((1u << left) - 1u);
     bits[wd] = m;
   }
+}
+
+// The stripe columns OR-ed into the row's bitmap (after its words are
+// written); a column outside [0, nkb) is an argument error when `report`.
+__device__ void pattern_row_columns(const bsa_tile_pattern &p, const int32_t *columns, int nkb,
+                                    uint32_t *bits, int tid, int nthr, bool report) {
+  for (long long e = static_cast<long long>(p.columns_begin) + tid; e < p.columns_end; e += nthr) {
+    const int c = columns[e];
+    if (c >= 0 && c < nkb) atomicOr(&bits[c >> 5], 1u << (c & 31));
+    else if (report) record_status(1u /* BSA_ERR_INVALID_ARG */);
+  }
+}
+
+// Row qb of pattern p as a bitmap over the nkb key blocks. Each thread builds
+// whole words from the band and axial terms; the stripe columns are then OR-ed
+// in. Ends with the CTA synchronised.
+__device__ void pattern_row_bitmap(const bsa_tile_pattern &p, bool ok, const int32_t *columns,
+                                   int qb, int nkb, uint32_t *bits, int words) {
+  pattern_row_words(p, ok, qb, nkb, bits, words, threadIdx.x, blockDim.x);
   __syncthreads();
   if (ok) {
-    for (long long e = static_cast<long long>(p.columns_begin) + threadIdx.x; e < p.columns_end;
-         e += blockDim.x) {
-      const int c = columns[e];
-      if (c >= 0 && c < nkb) atomicOr(&bits[c >> 5], 1u << (c & 31));
-      else record_status(1u /* BSA_ERR_INVALID_ARG */);
-    }
+    pattern_row_columns(p, columns, nkb, bits, threadIdx.x, blockDim.x, true);
   } else if (threadIdx.x == 0) {
     record_status(1u /* BSA_ERR_INVALID_ARG */);
   }

@@ -240,8 +240,8 @@ __global__ void radial_pair_union_kernel(RadialGeom g, int32_t *cost) {
   const int pr = blockIdx.x, words = (g.nb + 31) >> 5;
   for (int i = threadIdx.x; i < words; i += blockDim.x) bits[i] = 0u;
   __syncthreads();
-  radial_mark_row(g, 2 * pr, bits);
-  if (2 * pr + 1 < g.nb) radial_mark_row(g, 2 * pr + 1, bits);
+  radial_mark_row(g, 2 * pr, bits, threadIdx.x, blockDim.x);
+  if (2 * pr + 1 < g.nb) radial_mark_row(g, 2 * pr + 1, bits, threadIdx.x, blockDim.x);
   __syncthreads();
   int c = 0;
   for (int i = threadIdx.x; i < words; i += blockDim.x) c += __popc(bits[i]);
