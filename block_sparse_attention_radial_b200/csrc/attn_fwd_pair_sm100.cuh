@@ -62,7 +62,6 @@ struct PairCfg {
   static constexpr int NS_FIT = (kSmemLimit - 1024 - 512 - 2 * Q_BYTES) / TILE_BYTES;
   static constexpr int NS = NS_FIT > 8 ? 8 : NS_FIT;
   static constexpr int DSMEM_USED = 1024 + 2 * Q_BYTES + NS * TILE_BYTES;
-  static_assert(kSmemLimit - DSMEM_USED >= 1664, "static shared memory of the pair kernel");
   static constexpr int DSMEM = DSMEM_USED > 122880 ? DSMEM_USED : 122880;
   static constexpr uint32_t S_COL = 0;           // S of tile t at S_COL + 128 t
   static constexpr uint32_t O_COL = 256;         // O of tile t at O_COL + D t
