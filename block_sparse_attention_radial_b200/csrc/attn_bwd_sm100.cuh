@@ -218,10 +218,12 @@ __device__ int merge_tile_row(const int32_t *col_idx, int a0, int a1, int b0, in
 }
 
 // rows = num_lists * nt tile rows; nqb, nkb count 64-blocks.
+// (first: also write tile_ptr[0] = 0; later segments of a concatenation
+// leave the entry before them alone)
 __global__ void tile_count_kernel(const int32_t *row_ptr, const int32_t *col_idx, int nqb, int nkb,
-                                  int nnz, int nt, int rows, int32_t *tile_ptr) {
+                                  int nnz, int nt, int rows, int32_t *tile_ptr, int first) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i == 0) tile_ptr[0] = 0;
+  if (first && i == 0) tile_ptr[0] = 0;
   if (i >= rows) return;
   const int list = i / nt, t = i - list * nt;
   const int32_t *rp = row_ptr + static_cast<long long>(list) * nqb;

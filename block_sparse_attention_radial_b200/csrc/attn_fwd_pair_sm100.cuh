@@ -100,8 +100,16 @@ struct RowReader {
 // kModeQuarters: block-64 lists merged into 128-row tile lists, each entry
 // with the mask of its listed 64 x 64 quarters (the softmax masks the rest).
 enum : int {
-  kModeLists = 0, kModeVarlen = 1, kModePatterns = 2, kModeRadial = 3, kModeQuarters = 4
+  kModeLists = 0, kModeVarlen = 1, kModePatterns = 2, kModeRadial = 3, kModeQuarters = 4,
+  kModeVarlenQuarters = 5  // a variable-length batch of block-64 lists as quarter tiles
 };
+
+__host__ __device__ constexpr bool mode_varlen(int m) {
+  return m == kModeVarlen || m == kModeVarlenQuarters;
+}
+__host__ __device__ constexpr bool mode_quarters(int m) {
+  return m == kModeQuarters || m == kModeVarlenQuarters;
+}
 
 // One row's key blocks in ascending order, by mode; next() returns INT_MAX
 // past the end.
@@ -127,6 +135,9 @@ struct RowSource<kModeVarlen> : RowSource<kModeLists> {};
 
 template <>
 struct RowSource<kModeQuarters> : RowSource<kModeLists> {};
+
+template <>
+struct RowSource<kModeVarlenQuarters> : RowSource<kModeLists> {};
 
 template <>
 struct RowSource<kModePatterns> {
@@ -242,7 +253,7 @@ template <int MODE>
 __device__ __forceinline__ PairItem decode_pair(int idx, const FwdParams &p, int npairs,
                                                 const VarlenTable &vt) {
   PairItem it;
-  if (MODE != kModeVarlen) {
+  if (!mode_varlen(MODE)) {
     it.n = p.n;
     it.nqb = p.nqb;
     it.nkb = p.nkb;
@@ -778,7 +789,7 @@ __global__ void __launch_bounds__(384, 1)
       // Lists are sorted, so only the row's last block can be the ragged
       // final key block; its valid column count is taken once per item.
       int last_valid;
-      if (MODE == kModeLists || MODE == kModeVarlen || MODE == kModeQuarters) {
+      if (MODE == kModeLists || mode_varlen(MODE) || mode_quarters(MODE)) {
         const int last_kb = min(max(__ldg(p.col_idx + a0 + len - 1), 0), it.nkb - 1);
         last_valid = min(it.n - last_kb * BN, BN);
       } else {
@@ -798,12 +809,12 @@ __global__ void __launch_bounds__(384, 1)
       }
       // With quarter masks a row half may have nothing listed in its first
       // blocks: it then carries no reference maximum (-inf) until it does.
-      float m_ref = MODE == kModeQuarters ? -INFINITY : 0.f, l = 0.f;
+      float m_ref = mode_quarters(MODE) ? -INFINITY : 0.f, l = 0.f;
       const int qhalf = wq >> 1;  // the 64-row half of the tile this warp's rows are in
       for (int j = 0; j < len; ++j) {
         // this block's listed key halves for the warp's query half
         const uint32_t qbits =
-            MODE == kModeQuarters ? (__ldg(p.tile_mask + a0 + j) >> (2 * qhalf)) & 3u : 3u;
+            mode_quarters(MODE) ? (__ldg(p.tile_mask + a0 + j) >> (2 * qhalf)) & 3u : 3u;
         if (!(ok = warp_wait(&bar_s_full[t], scnt & 1u, wc, kBarSFull, scnt))) break;
         ++scnt;
         tc_fence_after();
@@ -826,7 +837,7 @@ __global__ void __launch_bounds__(384, 1)
           for (int c = 0; c < BN; ++c)
             if (c >= valid) s[c] = -INFINITY;
         }
-        if (MODE == kModeQuarters && qbits != 3u) {  // an unlisted key half
+        if (mode_quarters(MODE) && qbits != 3u) {  // an unlisted key half
 #pragma unroll
           for (int c = 0; c < BN; ++c)
             if (!((qbits >> (c >> 6)) & 1u)) s[c] = -INFINITY;
@@ -849,8 +860,8 @@ __global__ void __launch_bounds__(384, 1)
         auto exp_row = [&]() {
           // a row without a reference maximum has every column at -inf here
           // (its block maximum is -inf): any finite bias gives P = 0, sum 0
-          const float bias = MODE == kModeQuarters && m_ref == -INFINITY ? 0.f : -m_ref;
-          if (MODE == kModeQuarters) {
+          const float bias = mode_quarters(MODE) && m_ref == -INFINITY ? 0.f : -m_ref;
+          if (mode_quarters(MODE)) {
             // the exponentials of a key half this warp's query half does not
             // list are not computed (P = 0 there); both halves listed: the
             // same operations in the same order as a whole row
@@ -876,7 +887,7 @@ __global__ void __launch_bounds__(384, 1)
         float alpha = 1.f;
         bool rescale = false;
         float sum;
-        if (MODE == kModeQuarters) {
+        if (mode_quarters(MODE)) {
           // rows without a reference yet take this block's maximum (still
           // -inf when none of the row's columns here is listed); the vote
           // keeps the branch warp-uniform

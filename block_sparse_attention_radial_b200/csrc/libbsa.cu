@@ -54,10 +54,10 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   bool probed = false;
   int cc_major = 0, cc_minor = 0, sms = 0;
-  bool attrs_set[16] = {};
+  bool attrs_set[18] = {};
   bool ref_attrs_set[4] = {false, false, false, false};
   bool gemm_attrs_set[4] = {false, false, false, false};
-  bool pair_attrs_set[10] = {};
+  bool pair_attrs_set[12] = {};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -394,6 +394,8 @@ int launch_pair(const QkvViews &x, int32_t n, const FwdParams &p, DeviceInfo *de
     case kModePatterns: return launch_pair_mode<D, kModePatterns>(tq, tk, tv, p, dev, t, stream);
     case kModeRadial: return launch_pair_mode<D, kModeRadial>(tq, tk, tv, p, dev, t, stream);
     case kModeQuarters: return launch_pair_mode<D, kModeQuarters>(tq, tk, tv, p, dev, t, stream);
+    case kModeVarlenQuarters:
+      return launch_pair_mode<D, kModeVarlenQuarters>(tq, tk, tv, p, dev, t, stream);
     default: return launch_pair_mode<D, kModeLists>(tq, tk, tv, p, dev, t, stream);
   }
 }
@@ -425,7 +427,7 @@ int run_fwd(const QkvViews &x, int32_t n, int32_t head_dim, float softmax_scale,
     const int rows_t = l->num_lists * nt;
     const long long cap = l->nnz > 0 ? l->nnz : 1;
     tile_count_kernel<<<(rows_t + 127) / 128, 128, 0, stream>>>(
-        l->row_ptr, l->col_idx, nqb, l->num_k_blocks, l->nnz, nt, rows_t, tile_ptr);
+        l->row_ptr, l->col_idx, nqb, l->num_k_blocks, l->nnz, nt, rows_t, tile_ptr, 1);
     BSA_CUDA(cudaGetLastError());
     scan_rows_kernel<<<1, 1024, 0, stream>>>(tile_ptr, rows_t);
     BSA_CUDA(cudaGetLastError());
@@ -550,6 +552,27 @@ int varlen_table(int32_t num_items, const int32_t *cu, int32_t heads, int block,
 size_t varlen_order_bytes(const VarlenTable &vt, int num_lists) {
   return ((static_cast<size_t>(num_lists) * vt.pair0[vt.num_items] * sizeof(int32_t) + 255) &
           ~size_t(255)) + 256;
+}
+
+// Scratch of a variable-length forward: the work order and counter over the
+// 128-row tables' pairs (vt128), then, for block-64 lists, the items' tile
+// lists (offsets of num_lists * sum_b nt_b rows, entries and quarter masks,
+// at most one tile entry per 64-block entry).
+struct VarlenFwdLayout {
+  size_t tile_ptr, tile_col, tile_mask, total;
+};
+VarlenFwdLayout varlen_fwd_layout(const VarlenTable &vt128, const bsa_block_lists *l) {
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  VarlenFwdLayout w;
+  w.tile_ptr = w.tile_col = w.tile_mask = w.total = varlen_order_bytes(vt128, l->num_lists);
+  if (l->block == 64) {
+    const size_t cap = l->nnz > 0 ? static_cast<size_t>(l->nnz) : 1;
+    w.tile_col = w.tile_ptr + up((static_cast<size_t>(l->num_lists) * vt128.row0[vt128.num_items] + 1) *
+                                 sizeof(int32_t));
+    w.tile_mask = w.tile_col + up(cap * sizeof(int32_t));
+    w.total = w.tile_mask + up(cap);
+  }
+  return w;
 }
 
 // ------------------------------------------------ rows generated in-kernel
@@ -697,13 +720,16 @@ int launch_bwd_kernels(const BwdViews &x, int32_t n_map, BwdParams &p, bool mask
   const bool varlen = vt != nullptr;
   using DkdvFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, BwdParams,
                           VarlenTable);
-  DkdvFn dkdv = varlen   ? attn_bwd_dkdv_kernel<D, false, true>
+  DkdvFn dkdv = varlen   ? (masked ? attn_bwd_dkdv_kernel<D, true, true>
+                                   : attn_bwd_dkdv_kernel<D, false, true>)
                 : masked ? attn_bwd_dkdv_kernel<D, true, false>
                          : attn_bwd_dkdv_kernel<D, false, false>;
-  DkdvFn dq = varlen   ? attn_bwd_dq_kernel<D, false, true>
+  DkdvFn dq = varlen   ? (masked ? attn_bwd_dq_kernel<D, true, true>
+                                 : attn_bwd_dq_kernel<D, false, true>)
               : masked ? attn_bwd_dq_kernel<D, true, false>
                        : attn_bwd_dq_kernel<D, false, false>;
-  const int slot = 8 + (D == 128 ? 3 : 0) + (varlen ? 2 : masked ? 1 : 0);
+  const int slot = varlen && masked ? 16 + (D == 128 ? 1 : 0)
+                                    : 8 + (D == 128 ? 3 : 0) + (varlen ? 2 : masked ? 1 : 0);
   {
     std::lock_guard<std::mutex> lk(g_dev_mu);
     if (!dev->attrs_set[slot]) {
@@ -831,7 +857,7 @@ int launch_bwd(const BwdViews &x, const float *lse, int32_t n, float softmax_sca
     const long long cap = l_in->nnz > 0 ? l_in->nnz : 1;
     tile_count_kernel<<<(rows_t + 127) / 128, 128, 0, stream>>>(
         l_in->row_ptr, l_in->col_idx, l_in->num_q_blocks, l_in->num_k_blocks, l_in->nnz, nt,
-        rows_t, tile_ptr);
+        rows_t, tile_ptr, 1);
     BSA_CUDA(cudaGetLastError());
     scan_rows_kernel<<<1, 1024, 0, stream>>>(tile_ptr, rows_t);
     BSA_CUDA(cudaGetLastError());
@@ -900,8 +926,10 @@ int launch_bwd(const BwdViews &x, const float *lse, int32_t n, float softmax_sca
 // dK/dV and one dQ launch over every item's work.
 template <int D>
 int launch_bwd_varlen(const BwdViews &x, const float *lse, int32_t total, float softmax_scale,
-                      const bsa_block_lists *l, const VarlenTable &vt, uint8_t *ws,
-                      DeviceInfo *dev, cudaStream_t stream) {
+                      const bsa_block_lists *l, const VarlenTable &vt_l, const VarlenTable &vt,
+                      uint8_t *ws, DeviceInfo *dev, cudaStream_t stream) {
+  // vt_l: the items in blocks of the lists; vt: in 128-row tiles (the
+  // kernels' blocks; the same table at block 128)
   const int R = vt.row0[vt.num_items];
   const BwdLayout w = bwd_layout(1, x.heads, R * kBwdBlock, l);
   float *lse2 = reinterpret_cast<float *>(ws + w.lse2);
@@ -910,48 +938,89 @@ int launch_bwd_varlen(const BwdViews &x, const float *lse, int32_t total, float 
   int32_t *row_idx = reinterpret_cast<int32_t *>(ws + w.row_idx);
   int32_t *counters = reinterpret_cast<int32_t *>(ws + w.counters);
   const int L = l->num_lists;
+  const long long cap = l->nnz > 0 ? l->nnz : 1;
+  // block-64 lists: the items' tile lists with the quarter masks, as in the
+  // forward (counts per item, one scan, fills per item)
+  const int32_t *rows = l->row_ptr, *cols = l->col_idx;
+  const uint8_t *rmask = nullptr;
+  uint8_t *cmask = nullptr;
+  if (l->block != kBwdBlock) {
+    int32_t *tile_ptr = reinterpret_cast<int32_t *>(ws + w.tile_ptr);
+    int32_t *tile_col = reinterpret_cast<int32_t *>(ws + w.tile_col);
+    uint8_t *tile_mask = ws + w.tile_mask;
+    bool first_seg = true;
+    for (int b = 0; b < vt.num_items; ++b) {
+      const int nq = vt_l.row0[b + 1] - vt_l.row0[b], nt = vt.row0[b + 1] - vt.row0[b];
+      if (nt == 0) continue;
+      const int rows_t = L * nt;
+      tile_count_kernel<<<(rows_t + 127) / 128, 128, 0, stream>>>(
+          l->row_ptr + static_cast<long long>(L) * vt_l.row0[b], l->col_idx, nq, nq, l->nnz, nt,
+          rows_t, tile_ptr + static_cast<long long>(L) * vt.row0[b], first_seg ? 1 : 0);
+      BSA_CUDA(cudaGetLastError());
+      first_seg = false;
+    }
+    scan_rows_kernel<<<1, 1024, 0, stream>>>(tile_ptr, L * R);
+    BSA_CUDA(cudaGetLastError());
+    for (int b = 0; b < vt.num_items; ++b) {
+      const int nq = vt_l.row0[b + 1] - vt_l.row0[b], nt = vt.row0[b + 1] - vt.row0[b];
+      if (nt == 0) continue;
+      const int rows_t = L * nt;
+      tile_fill_kernel<<<(rows_t + 127) / 128, 128, 0, stream>>>(
+          l->row_ptr + static_cast<long long>(L) * vt_l.row0[b], l->col_idx, nq, nq, l->nnz, nt,
+          rows_t, tile_ptr + static_cast<long long>(L) * vt.row0[b], tile_col, tile_mask, cap);
+      BSA_CUDA(cudaGetLastError());
+    }
+    rows = tile_ptr;
+    cols = tile_col;
+    rmask = tile_mask;
+    cmask = ws + w.cmask;
+  }
+  const int nnz = static_cast<int>(l->block != kBwdBlock ? cap : l->nnz);
   bool first = true;
   for (int b = 0; b < vt.num_items; ++b) {
     const int nq = vt.row0[b + 1] - vt.row0[b];
     if (nq == 0) continue;
     const int32_t t0 = vt.tok0[b], n_b = vt.tok0[b + 1] - t0;
     const long long base = static_cast<long long>(x.heads) * vt.row0[b] * kBwdBlock;
-    const long long rows = static_cast<long long>(x.heads) * nq * kBwdBlock;
-    bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 255) / 256), 256, 0, stream>>>(
+    const long long prow = static_cast<long long>(x.heads) * nq * kBwdBlock;
+    bwd_prep_kernel<D><<<static_cast<unsigned>((prow + 255) / 256), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(x.out) + static_cast<long long>(t0) * x.lo.token_stride,
         static_cast<const __nv_bfloat16 *>(x.dout) + static_cast<long long>(t0) * x.ldo.token_stride,
         lse + t0, lse2 + base, delta + base, n_b, nq, x.heads, 0, x.lo.head_stride,
-        x.lo.token_stride, 0, x.ldo.head_stride, x.ldo.token_stride, 0, total, rows, counters);
+        x.lo.token_stride, 0, x.ldo.head_stride, x.ldo.token_stride, 0, total, prow, counters);
     BSA_CUDA(cudaGetLastError());
     const long long lr = static_cast<long long>(L) * vt.row0[b];
-    csc_count_kernel<<<L * nq, 256, 0, stream>>>(l->row_ptr + lr, l->col_idx, nq, nq, l->nnz,
-                                                 col_ptr + lr, first ? 1 : 0);
+    csc_count_kernel<<<L * nq, 256, 0, stream>>>(rows + lr, cols, nq, nq, nnz, col_ptr + lr,
+                                                 first ? 1 : 0);
     BSA_CUDA(cudaGetLastError());
     first = false;
   }
-  const int cols = L * R;
-  scan_rows_kernel<<<1, 1024, 0, stream>>>(col_ptr, cols);
+  scan_rows_kernel<<<1, 1024, 0, stream>>>(col_ptr, L * R);
   BSA_CUDA(cudaGetLastError());
   for (int b = 0; b < vt.num_items; ++b) {
     const int nq = vt.row0[b + 1] - vt.row0[b];
     if (nq == 0) continue;
     const long long lr = static_cast<long long>(L) * vt.row0[b];
-    csc_fill_kernel<<<L * nq, 256, 0, stream>>>(l->row_ptr + lr, l->col_idx, nq, nq, l->nnz,
-                                                col_ptr + lr, row_idx, l->nnz > 0 ? l->nnz : 1,
-                                                nullptr, nullptr, nullptr);
+    csc_fill_kernel<<<L * nq, 256, 0, stream>>>(rows + lr, cols, nq, nq, nnz, col_ptr + lr,
+                                                row_idx, nnz > 0 ? nnz : 1, rmask, cmask,
+                                                nullptr);
     BSA_CUDA(cudaGetLastError());
   }
   BwdParams p = bwd_params<D>(x, l, softmax_scale);
+  p.row_ptr = rows;
+  p.col_idx = cols;
+  p.nnz = nnz;
   p.col_ptr = col_ptr;
   p.row_idx = row_idx;
-  p.rmask = p.cmask = nullptr;
+  p.rmask = rmask;
+  p.cmask = cmask;
   p.lse2 = lse2;
   p.delta = delta;
   p.n = total;
   p.nqb = p.nkb = 0;  // per item, from the table
   p.item_counter = counters;
   const long long items = static_cast<long long>(x.heads) * R;
-  return launch_bwd_kernels<D>(x, total, p, false, &vt, items, items, dev, stream);
+  return launch_bwd_kernels<D>(x, total, p, rmask != nullptr, &vt, items, items, dev, stream);
 }
 
 // Self-test of the two exp2 paths of the attention softmax against exp2f.
@@ -1304,10 +1373,11 @@ int bsa_attn_fwd_strided(const void *q, const bsa_layout *q_layout, const void *
 size_t bsa_attn_fwd_varlen_workspace_bytes(int32_t num_items, const int32_t *cu_seqlens,
                                            int32_t heads, const bsa_block_lists *l) {
   if (!l || heads < 1 || (l->num_lists != 1 && l->num_lists != heads)) return 0;
+  if (l->block != 64 && l->block != 128) return 0;
   VarlenTable vt;
   int32_t mx = 0;
   if (varlen_table(num_items, cu_seqlens, heads, 128, &vt, &mx) != BSA_OK) return 0;
-  return varlen_order_bytes(vt, l->num_lists);
+  return varlen_fwd_layout(vt, l).total;
 }
 
 int bsa_attn_fwd_varlen(const void *q, const bsa_layout *q_layout, const void *k,
@@ -1322,13 +1392,17 @@ int bsa_attn_fwd_varlen(const void *q, const bsa_layout *q_layout, const void *k
     return BSA_ERR_INVALID_ARG;
   if (heads < 1) return BSA_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
-  if (l->block != 128) return BSA_ERR_UNSUPPORTED;
+  if (l->block != 64 && l->block != 128) return BSA_ERR_UNSUPPORTED;
   if (l->num_lists != 1 && l->num_lists != heads) return BSA_ERR_INVALID_ARG;
   if (l->nnz < 0) return BSA_ERR_INVALID_ARG;
-  VarlenTable vt;
-  int32_t max_nqb = 0;
+  // vt: the items in blocks of the lists; vt128: in 128-row tiles (the
+  // kernel's pairs and work items; the same table at block 128)
+  VarlenTable vt, vt128;
+  int32_t max_nqb = 0, max_nt = 0;
   int st;
   if ((st = varlen_table(num_items, cu_seqlens, heads, l->block, &vt, &max_nqb)) != BSA_OK)
+    return st;
+  if ((st = varlen_table(num_items, cu_seqlens, heads, 128, &vt128, &max_nt)) != BSA_OK)
     return st;
   const int32_t total = cu_seqlens[num_items];
   if (l->num_q_blocks != vt.row0[num_items] || l->num_k_blocks != max_nqb)
@@ -1347,8 +1421,8 @@ int bsa_attn_fwd_varlen(const void *q, const bsa_layout *q_layout, const void *k
       overlaps(out, so, k, layout_span_bytes(*k_layout, 1, heads, total, head_dim)) ||
       overlaps(out, so, v, layout_span_bytes(*v_layout, 1, heads, total, head_dim)))
     return BSA_ERR_INVALID_ARG;
-  if (!workspace || !aligned16(workspace) ||
-      workspace_bytes < varlen_order_bytes(vt, l->num_lists))
+  const VarlenFwdLayout wl = varlen_fwd_layout(vt128, l);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < wl.total)
     return BSA_ERR_INVALID_ARG;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return BSA_ERR_INVALID_ARG;
   DeviceInfo *dev = nullptr;
@@ -1361,26 +1435,68 @@ int bsa_attn_fwd_varlen(const void *q, const bsa_layout *q_layout, const void *k
     g_fault_flags = 0;
   }
   const int L = l->num_lists;
-  int32_t *order = static_cast<int32_t *>(workspace);
-  int32_t *counter = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) +
-                                                 varlen_order_bytes(vt, L) - 256);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  int32_t *order = reinterpret_cast<int32_t *>(ws);
+  int32_t *counter = reinterpret_cast<int32_t *>(ws + varlen_order_bytes(vt128, L) - 256);
+  // The kernel walks 128-row tiles: block-128 lists as they are; block-64
+  // lists merged item by item into tile lists with the quarter masks
+  // (counts per item, one scan over every item's tile rows, fills per item)
+  const int32_t *rows = l->row_ptr;
+  const int32_t *cols = l->col_idx;
+  const uint8_t *masks = nullptr;
+  int32_t nnz = l->nnz;
+  if (l->block == 64) {
+    int32_t *tile_ptr = reinterpret_cast<int32_t *>(ws + wl.tile_ptr);
+    int32_t *tile_col = reinterpret_cast<int32_t *>(ws + wl.tile_col);
+    uint8_t *tile_mask = ws + wl.tile_mask;
+    const long long cap = l->nnz > 0 ? l->nnz : 1;
+    bool first_seg = true;
+    for (int b = 0; b < num_items; ++b) {
+      const int nq = vt.row0[b + 1] - vt.row0[b], nt = vt128.row0[b + 1] - vt128.row0[b];
+      if (nt == 0) continue;
+      const int rows_t = L * nt;
+      tile_count_kernel<<<(rows_t + 127) / 128, 128, 0, stream>>>(
+          l->row_ptr + static_cast<long long>(L) * vt.row0[b], l->col_idx, nq, nq, l->nnz, nt,
+          rows_t, tile_ptr + static_cast<long long>(L) * vt128.row0[b], first_seg ? 1 : 0);
+      BSA_CUDA(cudaGetLastError());
+      first_seg = false;
+    }
+    const int all_rows = L * vt128.row0[num_items];
+    scan_rows_kernel<<<1, 1024, 0, stream>>>(tile_ptr, all_rows);
+    BSA_CUDA(cudaGetLastError());
+    for (int b = 0; b < num_items; ++b) {
+      const int nq = vt.row0[b + 1] - vt.row0[b], nt = vt128.row0[b + 1] - vt128.row0[b];
+      if (nt == 0) continue;
+      const int rows_t = L * nt;
+      tile_fill_kernel<<<(rows_t + 127) / 128, 128, 0, stream>>>(
+          l->row_ptr + static_cast<long long>(L) * vt.row0[b], l->col_idx, nq, nq, l->nnz, nt,
+          rows_t, tile_ptr + static_cast<long long>(L) * vt128.row0[b], tile_col, tile_mask, cap);
+      BSA_CUDA(cudaGetLastError());
+    }
+    rows = tile_ptr;
+    cols = tile_col;
+    masks = tile_mask;
+    nnz = static_cast<int32_t>(cap);
+  }
   // work order per item: each item's pairs longest union first, per list;
   // the first launch also zeroes the work counter
   bool first = true;
   for (int b = 0; b < num_items; ++b) {
-    const int nqb = vt.row0[b + 1] - vt.row0[b];
+    const int nqb = vt128.row0[b + 1] - vt128.row0[b];
     if (nqb == 0) continue;
     const int npairs = (nqb + 1) / 2;
     const size_t smem = static_cast<size_t>(npairs <= kLptMaxRows ? npairs : 0) * sizeof(int);
     pair_order_kernel<<<L, 1024, smem, stream>>>(
-        l->row_ptr + static_cast<long long>(L) * vt.row0[b], l->col_idx, nqb, l->nnz,
-        order + static_cast<long long>(L) * vt.pair0[b], kLptMaxRows, first ? counter : nullptr);
+        rows + static_cast<long long>(L) * vt128.row0[b], cols, nqb, nnz,
+        order + static_cast<long long>(L) * vt128.pair0[b], kLptMaxRows,
+        first ? counter : nullptr);
     BSA_CUDA(cudaGetLastError());
     first = false;
   }
   FwdParams p;
-  p.row_ptr = l->row_ptr;
-  p.col_idx = l->col_idx;
+  p.row_ptr = rows;
+  p.col_idx = cols;
+  p.tile_mask = masks;
   p.order = order;
   p.item_counter = counter;
   p.out = static_cast<__nv_bfloat16 *>(out);
@@ -1390,11 +1506,11 @@ int bsa_attn_fwd_varlen(const void *q, const bsa_layout *q_layout, const void *k
   p.lse = lse;
   p.heads = heads;
   p.n = total;
-  p.nqb = l->num_q_blocks;
-  p.nkb = l->num_k_blocks;
+  p.nqb = vt128.row0[num_items];
+  p.nkb = max_nt;
   p.num_lists = L;
-  p.nnz = l->nnz;
-  p.total_items = vt.work0[num_items];
+  p.nnz = nnz;
+  p.total_items = vt128.work0[num_items];
   const float scale =
       softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -1412,8 +1528,9 @@ int bsa_attn_fwd_varlen(const void *q, const bsa_layout *q_layout, const void *k
   x.lv = *v_layout;
   x.batch = 1;
   x.heads = heads;
-  if (head_dim == 128) return launch_pair<128>(x, total, p, dev, kModeVarlen, &vt, stream);
-  return launch_pair<64>(x, total, p, dev, kModeVarlen, &vt, stream);
+  const int mode = l->block == 64 ? kModeVarlenQuarters : kModeVarlen;
+  if (head_dim == 128) return launch_pair<128>(x, total, p, dev, mode, &vt128, stream);
+  return launch_pair<64>(x, total, p, dev, mode, &vt128, stream);
 }
 
 size_t bsa_attn_fwd_patterns_workspace_bytes(int32_t num_patterns, int32_t num_q_blocks) {
@@ -1664,7 +1781,8 @@ int bsa_attn_bwd_strided(const void *q, const bsa_layout *q_layout, const void *
 
 size_t bsa_attn_bwd_varlen_workspace_bytes(int32_t num_items, const int32_t *cu_seqlens,
                                            int32_t heads, const bsa_block_lists *l) {
-  if (!l || heads < 1 || l->block != 128 || (l->num_lists != 1 && l->num_lists != heads))
+  if (!l || heads < 1 || (l->block != 64 && l->block != 128) ||
+      (l->num_lists != 1 && l->num_lists != heads))
     return 0;
   VarlenTable vt;
   int32_t mx = 0;
@@ -1691,20 +1809,23 @@ int bsa_attn_bwd_varlen(const void *q, const bsa_layout *q_layout, const void *k
   if (!lse || !l || !l->row_ptr || (l->nnz > 0 && !l->col_idx)) return BSA_ERR_INVALID_ARG;
   if (heads < 1) return BSA_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
-  if (l->block != 128) return BSA_ERR_UNSUPPORTED;
+  if (l->block != 64 && l->block != 128) return BSA_ERR_UNSUPPORTED;
   if (l->num_lists != 1 && l->num_lists != heads) return BSA_ERR_INVALID_ARG;
   if (l->nnz < 0) return BSA_ERR_INVALID_ARG;
-  VarlenTable vt;
-  int32_t max_nqb = 0;
+  // vt_l: the items in blocks of the lists; vt: in 128-row tiles
+  VarlenTable vt_l, vt;
+  int32_t max_nqb = 0, max_nt = 0;
   int st;
-  if ((st = varlen_table(num_items, cu_seqlens, heads, l->block, &vt, &max_nqb)) != BSA_OK)
+  if ((st = varlen_table(num_items, cu_seqlens, heads, l->block, &vt_l, &max_nqb)) != BSA_OK)
+    return st;
+  if ((st = varlen_table(num_items, cu_seqlens, heads, kBwdBlock, &vt, &max_nt)) != BSA_OK)
     return st;
   const int32_t total = cu_seqlens[num_items];
-  if (l->num_q_blocks != vt.row0[num_items] || l->num_k_blocks != max_nqb)
+  if (l->num_q_blocks != vt_l.row0[num_items] || l->num_k_blocks != max_nqb)
     return BSA_ERR_INVALID_ARG;
   if (static_cast<long long>(heads) * total > 0x7fffffffLL ||
       static_cast<long long>(l->num_lists) * l->num_q_blocks > 0x7fffffffLL ||
-      static_cast<long long>(heads) * l->num_q_blocks * kBwdBlock > 0x7fffffffLL)
+      static_cast<long long>(heads) * vt.row0[num_items] * kBwdBlock > 0x7fffffffLL)
     return BSA_ERR_UNSUPPORTED;
   // the packed sequence is a batch of one: [1, heads, total, head_dim] views
   const size_t lbytes = static_cast<size_t>(heads) * total * sizeof(float);
@@ -1718,8 +1839,8 @@ int bsa_attn_bwd_varlen(const void *q, const bsa_layout *q_layout, const void *k
   const BwdViews x = bwd_views(ptrs, lays, 1, heads);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   if (head_dim == 128)
-    return launch_bwd_varlen<128>(x, lse, total, softmax_scale, l, vt, ws, dev, stream);
-  return launch_bwd_varlen<64>(x, lse, total, softmax_scale, l, vt, ws, dev, stream);
+    return launch_bwd_varlen<128>(x, lse, total, softmax_scale, l, vt_l, vt, ws, dev, stream);
+  return launch_bwd_varlen<64>(x, lse, total, softmax_scale, l, vt_l, vt, ws, dev, stream);
 }
 
 size_t bsa_attn_bwd_workspace_bytes(int32_t batch, int32_t heads, int32_t n,

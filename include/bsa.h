@@ -378,7 +378,8 @@ int bsa_attn_fwd_radial(const void *q, const void *k, const void *v,
 
 /*
  * Bytes of device scratch bsa_attn_fwd_varlen needs (the per-item work order
- * and the work counter); 0 for invalid arguments.
+ * and the work counter; for block-64 lists also the items' 128-row tile
+ * lists: offsets, entries and quarter masks); 0 for invalid arguments.
  */
 size_t bsa_attn_fwd_varlen_workspace_bytes(int32_t num_items, const int32_t *cu_seqlens,
                                            int32_t heads, const bsa_block_lists *lists);
@@ -400,17 +401,19 @@ size_t bsa_attn_fwd_varlen_workspace_bytes(int32_t num_items, const int32_t *cu_
  *        num_items + 1 token offsets: cu_seqlens[0] = 0, non-decreasing, total
  *        >= 1 (empty items are allowed).
  * lists  the items' lists concatenated as bsa_joint_mask_build_varlen writes
- *        them: block 128; num_q_blocks = sum_b ceil(n_b / 128); num_k_blocks
- *        = max_b ceil(n_b / 128); num_lists 1 (each item's list shared by its
- *        heads) or heads (item b's rows hold its lists for heads 0..heads-1,
- *        one after another, nqb_b rows each); column indices count key blocks
- *        inside the item.
+ *        them: block 64 or 128; num_q_blocks = sum_b ceil(n_b / block);
+ *        num_k_blocks = max_b ceil(n_b / block); num_lists 1 (each item's list
+ *        shared by its heads) or heads (item b's rows hold its lists for heads
+ *        0..heads-1, one after another, nqb_b rows each); column indices count
+ *        key blocks inside the item. Block-64 lists run, item by item, as
+ *        128-row tiles with a mask of their listed 64 x 64 quarters (built in
+ *        the workspace), like bsa_attn_fwd's.
  * lse    device fp32 [heads, total] (natural log, -inf for a row without
  *        keys), or NULL.
  * workspace  bsa_attn_fwd_varlen_workspace_bytes() bytes of device scratch.
  * Results for each item equal bsa_attn_fwd on that item alone, bit for bit.
- * Returns BSA_ERR_UNSUPPORTED for block 64 or head_dim other than 64 / 128;
- * other errors as bsa_attn_fwd. Asynchronous.
+ * Returns BSA_ERR_UNSUPPORTED for a block other than 64 / 128 or head_dim
+ * other than 64 / 128; other errors as bsa_attn_fwd. Asynchronous.
  */
 int bsa_attn_fwd_varlen(const void *q, const bsa_layout *q_layout,
                         const void *k, const bsa_layout *k_layout,
@@ -602,8 +605,10 @@ int bsa_attn_bwd_strided(const void *q, const bsa_layout *q_layout,
 /*
  * Bytes of device scratch bsa_attn_bwd_varlen needs: lse * log2(e) and delta
  * for every item's query rows padded to whole 128-row blocks, per head (2 x 4
- * bytes each), the transposed lists of all items (num_lists * sum_b nqb_b + 1
- * offsets, nnz entries) and two work counters. 0 for invalid arguments.
+ * bytes each), the transposed lists of all items (num_lists * sum_b nt_b + 1
+ * offsets, nnz entries; nt_b = ceil(n_b / 128)) and two work counters; for
+ * block-64 lists also the items' tile lists and one mask byte per tile and
+ * per transposed entry. 0 for invalid arguments.
  */
 size_t bsa_attn_bwd_varlen_workspace_bytes(int32_t num_items, const int32_t *cu_seqlens,
                                            int32_t heads, const bsa_block_lists *lists);
@@ -619,7 +624,9 @@ size_t bsa_attn_bwd_varlen_workspace_bytes(int32_t num_items, const int32_t *cu_
  *        rules as bsa_attn_bwd_strided with batch 1 and n = total.
  * lse    the forward's fp32 [heads, total] log-sum-exp (required), as
  *        bsa_attn_fwd_varlen writes it.
- * num_items, cu_seqlens, lists  as for bsa_attn_fwd_varlen (block 128).
+ * num_items, cu_seqlens, lists  as for bsa_attn_fwd_varlen (block 64 or 128;
+ *        block-64 lists run as 128-row tiles with quarter masks, like
+ *        bsa_attn_bwd's).
  * workspace  bsa_attn_bwd_varlen_workspace_bytes() bytes of device scratch,
  *        16-byte aligned, overlapping no view and not lse.
  * Per item a prep launch (delta, lse * log2(e)) and the item's columns of
@@ -629,9 +636,9 @@ size_t bsa_attn_bwd_varlen_workspace_bytes(int32_t num_items, const int32_t *cu_
  * are not touched. Each item's gradients are bit-identical to bsa_attn_bwd
  * on that item alone. Every element of the views must be finite (an item's
  * last blocks read the next item's tokens, which enter with weight 0).
- * Deterministic. Returns
- * BSA_ERR_UNSUPPORTED for block 64 or head_dim other than 64 / 128; other
- * errors as bsa_attn_bwd_strided. Asynchronous.
+ * Deterministic. Returns BSA_ERR_UNSUPPORTED for a block other than 64 /
+ * 128 or head_dim other than 64 / 128; other errors as bsa_attn_bwd_strided.
+ * Asynchronous.
  */
 int bsa_attn_bwd_varlen(const void *q, const bsa_layout *q_layout,
                         const void *k, const bsa_layout *k_layout,

@@ -424,13 +424,17 @@ def test_varlen_host_checks(lib):
                                        0.0, ref(ls), out, ref(lay), None, w, wsb, None)
 
     assert lib.bsa_attn_fwd_varlen_workspace_bytes(3, cu_ok, H, ref(lists())) == 256 + 256
+    # block 64: plus the items' tile lists (7 + 1 offsets, 10 entries, 10 masks)
+    assert lib.bsa_attn_fwd_varlen_workspace_bytes(3, cu_ok, H, ref(lists(block=64))) == \
+        256 + 256 + 256 + 256 + 256
     assert call(items=0) == 1 and call(items=65) == 1
     assert call(cu=(ctypes.c_int32 * 4)(1, 300, 300, 700)) == 1      # cu[0] != 0
     assert call(cu=(ctypes.c_int32 * 4)(0, 300, 200, 700)) == 1      # decreasing
     assert call(cu=(ctypes.c_int32 * 2)(0, 0), items=1) == 1          # no tokens at all
     assert call(ls=lists(nq=6)) == 1                                  # row count mismatch
     assert call(ls=lists(nk=7)) == 1                                  # widest item is 4
-    assert call(ls=lists(block=64, nq=14, nk=7)) == 2                 # block 64 unsupported
+    assert call(ls=lists(block=64, nq=14, nk=7)) == 1                 # 12 blocks of 64, not 14
+    assert call(ls=lists(block=32, nq=24, nk=13)) == 2                # block 32 unsupported
     assert call(ls=lists(L=3)) == 1                                   # num_lists not 1 or H
     assert call(hd=96) == 2
     assert call(wsb=256) == 1                                         # workspace too small
@@ -475,13 +479,18 @@ def test_varlen_backward_host_checks(lib):
     # 1792 rows each, counters, 7 + 1 column pointers, 10 entries, each part
     # 256-byte aligned
     assert ws == 7168 + 7168 + 256 + 256 + 256
-    assert lib.bsa_attn_bwd_varlen_workspace_bytes(3, cu_ok, H, ref(lists(block=64))) == 0
+    assert lib.bsa_attn_bwd_varlen_workspace_bytes(3, cu_ok, H, ref(lists(block=32))) == 0
+    # block 64: plus the tile lists (7 + 1 offsets, 10 entries, 10 mask
+    # bytes) and one mask byte per transposed entry
+    assert lib.bsa_attn_bwd_varlen_workspace_bytes(3, cu_ok, H, ref(lists(block=64))) == \
+        ws + 256 + 256 + 256 + 256
     assert call(items=0) == 1 and call(items=65) == 1
     assert call(cu=(ctypes.c_int32 * 4)(1, 300, 300, 700)) == 1      # cu[0] != 0
     assert call(cu=(ctypes.c_int32 * 4)(0, 300, 200, 700)) == 1      # decreasing
     assert call(ls=lists(nq=6)) == 1                                  # row count mismatch
     assert call(ls=lists(nk=5)) == 1                                  # widest item is 4
-    assert call(ls=lists(block=64, nq=14, nk=7)) == 2                 # block 64 unsupported
+    assert call(ls=lists(block=64, nq=14, nk=7)) == 1                 # 12 blocks of 64, not 14
+    assert call(ls=lists(block=32, nq=24, nk=13)) == 2                # block 32 unsupported
     assert call(ls=lists(L=3)) == 1                                   # num_lists not 1 or H
     assert call(hd=96) == 2
     assert call(lse_=None) == 1                                       # lse required

@@ -6,7 +6,7 @@ on each item alone.
 
 Items differ in frame count, tokens per frame and text length, so their token
 counts, query-block counts and lists all differ; one forward launch serves
-them all. Backward bars as the regular backward's (relative RMS 5e-3, max-abs
+them all, at block 128 and at block 64 (quarter tiles). Backward bars as the regular backward's (relative RMS 5e-3, max-abs
 2e-2 of the oracle's largest entry, per item and tensor).
 """
 
@@ -237,3 +237,45 @@ def test_varlen_backward_medium_batch_matches_single_items(bsa):
         gi = bsa.attention_backward(*views, lse[:, t0:t1].contiguous().unsqueeze(0), one)
         for got, g1, name in zip((dq, dk, dv), gi, ("dq", "dk", "dv")):
             assert torch.equal(g1[0].permute(1, 0, 2), got[t0:t1]), f"item {b} {name} differs"
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_varlen_block64_forward_and_backward(bsa, D):
+    """Block-64 lists of a variable-length batch (items merged into 128-row
+    tiles with quarter masks, item by item): forward and backward against the
+    float64 oracle per item and bit-identical to the regular block-64 entries
+    on each item alone."""
+    H = 2
+    items = ITEMS + [(1, 50, 0)]                  # the last item: one block of 64
+    lengths = [f * s + t for f, s, t in items]
+    cu = _cu(lengths)
+    total = int(cu[-1])
+    q, k, v = _packed(total, H, D, seed=30 + D)
+    do = torch.randn((total, H, D), generator=torch.Generator().manual_seed(D + 1)).to(torch.bfloat16)
+    lists = bsa.radial_block_lists_varlen(items, 64)
+    qd, kd, vd, dod = (x.cuda() for x in (q, k, v, do))
+    out, lse = bsa.attention_varlen(qd, kd, vd, cu, lists)
+    dq, dk, dv = bsa.attention_varlen_backward(qd, kd, vd, out, dod, lse, cu, lists)
+    assert bsa.bsa_get_device_status() == 0
+    rp, ci = oracle.varlen_block_lists(items, 64)
+    item_lists = oracle.split_item_lists(rp, ci, [-(-n // 64) for n in lengths])
+    qf, kf, vf, df = (x.float().numpy() for x in (q, k, v, do))
+    ref_o, ref_l = oracle.varlen_masked_attention_fp64(qf, kf, vf, cu, item_lists, 1, 64)
+    refs = oracle.varlen_masked_attention_backward_fp64(qf, kf, vf, df, cu, item_lists, 1, 64)
+    o, l_ = out.cpu(), lse.cpu()
+    got = [g.cpu() for g in (dq, dk, dv)]
+    for b, (f, s_, t) in enumerate(items):
+        t0, t1 = int(cu[b]), int(cu[b + 1])
+        assert_close(o[t0:t1].float().numpy(), ref_o[t0:t1], l_[:, t0:t1].numpy(),
+                     ref_l[:, t0:t1], f"block-64 varlen item {b}")
+        for g, r, name in zip(got, refs, ("dq", "dk", "dv")):
+            _grad_close(g[t0:t1].float().numpy(), r[t0:t1], f"block-64 varlen item {b} {name}")
+        one = bsa.radial_block_lists(f, s_, 64, text_tokens=t)
+        views = [_item_view(x, t0, t1) for x in (qd, kd, vd)]
+        oi, li = bsa.attention(*views, one)
+        assert torch.equal(oi[0].permute(1, 0, 2).cpu(), o[t0:t1]), f"item {b} output differs"
+        assert torch.equal(li[0].cpu(), l_[:, t0:t1]), f"item {b} lse differs"
+        gi = bsa.attention_backward(*views, _item_view(out, t0, t1), _item_view(dod, t0, t1),
+                                    lse[:, t0:t1].contiguous().unsqueeze(0), one)
+        for g, g1, name in zip(got, gi, ("dq", "dk", "dv")):
+            assert torch.equal(g1[0].permute(1, 0, 2).cpu(), g[t0:t1]), f"item {b} {name} differs"
