@@ -279,3 +279,40 @@ def test_varlen_block64_forward_and_backward(bsa, D):
                                     lse[:, t0:t1].contiguous().unsqueeze(0), one)
         for g, g1, name in zip(got, gi, ("dq", "dk", "dv")):
             assert torch.equal(g1[0].permute(1, 0, 2).cpu(), g[t0:t1]), f"item {b} {name} differs"
+
+
+def test_varlen_block64_per_head_lists_and_edge_items(bsa):
+    # per-head random block-64 lists; an empty item, a one-token item and an
+    # item of an odd number of 64-blocks; forward and backward against the oracle
+    H, D, blk = 2, 64, 64
+    lengths = [300, 0, 1, 192, 700]
+    cu = _cu(lengths)
+    total = int(cu[-1])
+    q, k, v = _packed(total, H, D, seed=51)
+    do = torch.randn((total, H, D), generator=torch.Generator().manual_seed(52)).to(torch.bfloat16)
+    nqbs = [-(-n // blk) for n in lengths]
+    rps, cis, item_lists, off = [], [], [], 0
+    for b, nqb in enumerate(nqbs):
+        if nqb == 0:
+            item_lists.append((np.zeros(1, dtype=np.int64), np.zeros(0, dtype=np.int64)))
+            continue
+        rp, ci = random_block_lists(H * nqb, nqb, 0.5, seed=60 + b)
+        item_lists.append((rp, ci))
+        rps.append(np.asarray(rp[:-1]) + off)
+        cis.append(np.asarray(ci))
+        off += int(rp[-1])
+    row_ptr = np.concatenate(rps + [np.array([off])])
+    col_idx = np.concatenate(cis)
+    lists = bsa.block_lists_from_csr(row_ptr, col_idx, H, sum(nqbs), blk)
+    lists.k_blocks = max(nqbs)
+    qd, kd, vd, dod = (x.cuda() for x in (q, k, v, do))
+    out, lse = bsa.attention_varlen(qd, kd, vd, cu, lists)
+    dq, dk, dv = bsa.attention_varlen_backward(qd, kd, vd, out, dod, lse, cu, lists)
+    assert bsa.bsa_get_device_status() == 0
+    qf, kf, vf, df = (x.float().numpy() for x in (q, k, v, do))
+    ref_o, ref_l = oracle.varlen_masked_attention_fp64(qf, kf, vf, cu, item_lists, H, blk)
+    assert_close(out.cpu().float().numpy(), ref_o, lse.cpu().numpy(), ref_l,
+                 "per-head block-64 varlen")
+    refs = oracle.varlen_masked_attention_backward_fp64(qf, kf, vf, df, cu, item_lists, H, blk)
+    for g, r, name in zip((dq, dk, dv), refs, ("dq", "dk", "dv")):
+        _grad_close(g.cpu().float().numpy(), r, f"per-head block-64 varlen {name}")
